@@ -1,0 +1,169 @@
+"""CPU oracle of the routed MoE layer forward -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+may import this package.  The CUDA library never loads it and shares no code
+with it; both are handed the same seeded input buffers.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, fp64; the router logit is the
+fp32 fused-multiply-add chain both sides agree on).  This module only compiles
+it with gcc and marshals numpy arrays through ctypes.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(brute force, closed forms, invariants, library routines) -- none is unpinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(_HERE, "moe_oracle.c")
+LIB = os.path.join(_HERE, "libmoe_oracle.so")
+
+
+def build(src: str = SRC, out: str = LIB, force: bool = False) -> str:
+    """Compile the oracle with gcc (no fp contraction, so only the explicit fmaf
+    calls fuse)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+               "-shared", "-o", tmp, src, "-lm", "-lpthread"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+    return out
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bf16_bits(t) -> np.ndarray:
+    """bf16 tensor (torch) or uint16 array -> contiguous uint16 numpy array of its bits."""
+    if isinstance(t, np.ndarray):
+        assert t.dtype == np.uint16
+        return np.ascontiguousarray(t)
+    import torch
+    assert t.dtype == torch.bfloat16
+    return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def _f32(t):
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return np.ascontiguousarray(t, dtype=np.float32)
+    return np.ascontiguousarray(t.detach().cpu().float().numpy())
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+class Oracle:
+    """ctypes view of one build of the oracle library."""
+
+    def __init__(self, lib_path: str | None = None):
+        lib = ctypes.CDLL(lib_path or build())
+        P = ctypes.c_void_p
+        i = ctypes.c_int
+        lib.oracle_route.argtypes = [i, i, i, i, P, P, P, P, P, P, P, i]
+        lib.oracle_route.restype = i
+        lib.oracle_permute.argtypes = [i, i, P, P, P, P, i, P, P]
+        lib.oracle_permute.restype = i
+        lib.oracle_combine_ffn.argtypes = [i, i, i, P, P, P, P, P, P, i, P, P, i]
+        lib.oracle_combine_ffn.restype = i
+        self.lib = lib
+
+    def route(self, x, router_w, bias, top_k: int, want_logits: bool = False,
+              nthreads: int | None = None):
+        """Router + softmax over the top-k.  Returns (idx int32 [T,k], gate fp64 [T,k])
+        and, with ``want_logits``, also (logits fp32 [T,E], logits fp64 [T,E])."""
+        xb, wb, bb = _bf16_bits(x), _bf16_bits(router_w), _f32(bias)
+        T, H = xb.shape
+        H2, E = wb.shape
+        assert H == H2
+        idx = np.zeros((T, top_k), np.int32)
+        gate = np.zeros((T, top_k), np.float64)
+        l32 = np.zeros((T, E), np.float32) if want_logits else None
+        l64 = np.zeros((T, E), np.float64) if want_logits else None
+        rc = self.lib.oracle_route(T, H, E, top_k, _ptr(xb), _ptr(wb), _ptr(bb), _ptr(idx),
+                                   _ptr(gate), _ptr(l32), _ptr(l64), nthreads or default_threads())
+        if rc:
+            raise ValueError(f"oracle_route rejected its arguments (code {rc})")
+        return (idx, gate, l32, l64) if want_logits else (idx, gate)
+
+    def permute(self, idx, E: int, bm: int = 128):
+        """Stable counting sort of the flat assignments by expert.  Returns a dict with
+        offsets [E+1], sorted_to_flat [A], flat_to_sorted [A], tile_list [n,3], num_tiles."""
+        fl = np.ascontiguousarray(np.asarray(idx, dtype=np.int32).reshape(-1))
+        A = fl.size
+        off = np.zeros(E + 1, np.int32)
+        s2f = np.zeros(max(A, 1), np.int32)
+        f2s = np.zeros(max(A, 1), np.int32)
+        nt = np.zeros(1, np.int32)
+        rc = self.lib.oracle_permute(A, E, _ptr(fl), _ptr(off), _ptr(s2f), _ptr(f2s), bm, None,
+                                     _ptr(nt))
+        if rc:
+            raise ValueError(f"oracle_permute rejected its arguments (code {rc})")
+        tl = np.zeros((max(int(nt[0]), 1), 3), np.int32)
+        self.lib.oracle_permute(A, E, _ptr(fl), _ptr(off), _ptr(s2f), _ptr(f2s), bm, _ptr(tl),
+                                _ptr(nt))
+        return {"offsets": off, "sorted_to_flat": s2f[:A], "flat_to_sorted": f2s[:A],
+                "tile_list": tl[: int(nt[0])], "num_tiles": int(nt[0])}
+
+    def combine_ffn(self, x, idx, gate, w_gate, w_up, w_down, tokens=None,
+                    nthreads: int | None = None):
+        """Gate-weighted sum of the selected experts' SwiGLU FFN outputs, fp64 [n,H]."""
+        xb = _bf16_bits(x)
+        T, H = xb.shape
+        wg, wu, wd = _bf16_bits(w_gate), _bf16_bits(w_up), _bf16_bits(w_down)
+        E, I, H2 = wg.shape
+        assert H2 == H and wd.shape == (E, H, I) and wu.shape == wg.shape
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        k = idx.shape[1]
+        tok = None if tokens is None else np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+        n = T if tok is None else tok.size
+        out = np.zeros((n, H), np.float64)
+        rc = self.lib.oracle_combine_ffn(H, I, k, _ptr(xb), _ptr(idx), _ptr(gate), _ptr(wg),
+                                         _ptr(wu), _ptr(wd), n, _ptr(tok), _ptr(out),
+                                         nthreads or default_threads())
+        if rc:
+            raise ValueError(f"oracle_combine_ffn rejected its arguments (code {rc})")
+        return out
+
+    def forward(self, x, router_w, bias, w_gate, w_up, w_down, top_k: int, tokens=None,
+                nthreads: int | None = None):
+        """The whole layer for the given tokens (all when None): (out fp64, idx, gate)."""
+        idx, gate = self.route(x, router_w, bias, top_k, nthreads=nthreads)
+        out = self.combine_ffn(x, idx, gate, w_gate, w_up, w_down, tokens, nthreads)
+        return out, idx, gate
+
+
+_default: Oracle | None = None
+
+
+def get() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def route(*a, **kw):
+    return get().route(*a, **kw)
+
+
+def permute(*a, **kw):
+    return get().permute(*a, **kw)
+
+
+def combine_ffn(*a, **kw):
+    return get().combine_ffn(*a, **kw)
+
+
+def forward(*a, **kw):
+    return get().forward(*a, **kw)

@@ -1,0 +1,286 @@
+/*
+ * moe_oracle.c -- plain CPU oracle of the routed MoE layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this library.  It shares no code, header,
+ * table or helper with the CUDA path; both sides are handed the same seeded
+ * input buffers and nothing else.
+ *
+ * What it computes (vLLM fused-MoE page, section 02 "what the fused MoE kernel
+ * computes": a router picks the top-k of E experts for every token, each chosen
+ * expert is a gate/up/down FFN with SwiGLU, and the top-k outputs are summed
+ * with the gating weights; Weave review section 1.2 and the stepwise-vs-fused
+ * comparison page section 2 give the same route -> dispatch -> expert FFN ->
+ * combine data path):
+ *
+ *   l[t,e]  = sum_h x[t,h] * Wr[h,e]  (+ bias[e])           router logits
+ *   S_t     = the k experts with the largest l[t,.], listed by descending
+ *             logit, equal logits ordered by ascending expert index
+ *   g[t,j]  = exp(l[t,S_j]) / sum_{i<k} exp(l[t,S_i])        softmax over the top-k
+ *   out[t]  = sum_j g[t,j] * Wd_e ( silu(Wg_e x_t) * (Wu_e x_t) ),  e = S_j
+ *   silu(a) = a / (1 + exp(-a))
+ *
+ * Readings taken where the pages are silent (each is listed in the design notes):
+ *  - the router logit is an fp32 value with a fixed evaluation order: a chain of
+ *    fused multiply-adds over h ascending starting from 0, the bias added last
+ *    in fp32.  Routing is an integer decision made on that fp32 value, so both
+ *    sides take it in the same precision.
+ *  - ties in the top-k go to the lower expert index.
+ *  - gates and the expert FFN are evaluated in fp64 from the bf16 inputs; no
+ *    intermediate is rounded.
+ *  - the permutation into expert groups is a stable counting sort of the flat
+ *    assignment list (flat = t*k + j) by expert; group offsets carry no padding.
+ *
+ * Deliberately slow and direct: no blocking, no fusion, no reordering.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------- scalars */
+
+static float bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static double bf16_to_f64(uint16_t b) { return (double)bf16_to_f32(b); }
+
+static double silu(double a) { return a / (1.0 + exp(-a)); }
+
+/* ------------------------------------------------------------ the router */
+
+/* Router logits for one token: fp32 fused multiply-add chain over h ascending,
+ * then + bias[e] in fp32.  Also returns the fp64 value of the same sum (for the
+ * routing-margin diagnostics and the pins), when logit64 is not NULL. */
+static void router_logits_token(int H, int E, const uint16_t *xt, const uint16_t *wr,
+                                const float *bias, float *logit32, double *logit64)
+{
+    for (int e = 0; e < E; ++e) {
+        float acc = 0.0f;
+        double acc64 = 0.0;
+        for (int h = 0; h < H; ++h) {
+            float a = bf16_to_f32(xt[h]);
+            float w = bf16_to_f32(wr[(size_t)h * E + e]);
+            acc = fmaf(a, w, acc);
+            acc64 += (double)a * (double)w;
+        }
+        if (bias) {
+            acc = acc + bias[e];
+            acc64 += (double)bias[e];
+        }
+        logit32[e] = acc;
+        if (logit64) logit64[e] = acc64;
+    }
+}
+
+/* Top-k by repeated arg-max: strictly larger wins, so among equal logits the
+ * lower expert index is taken first. */
+static void topk_token(int E, int k, const float *l, int32_t *idx, unsigned char *taken)
+{
+    memset(taken, 0, (size_t)E);
+    for (int j = 0; j < k; ++j) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+            if (taken[e]) continue;
+            if (best < 0 || l[e] > l[best]) best = e;
+        }
+        taken[best] = 1;
+        idx[j] = best;
+    }
+}
+
+/* Softmax over the k selected logits, in fp64. */
+static void gates_token(int k, const float *l, const int32_t *idx, double *g)
+{
+    double m = (double)l[idx[0]];
+    for (int j = 1; j < k; ++j)
+        if ((double)l[idx[j]] > m) m = (double)l[idx[j]];
+    double s = 0.0;
+    for (int j = 0; j < k; ++j) s += exp((double)l[idx[j]] - m);
+    for (int j = 0; j < k; ++j) g[j] = exp((double)l[idx[j]] - m) / s;
+}
+
+typedef struct {
+    int T, H, E, k;
+    const uint16_t *x, *wr;
+    const float *bias;
+    int32_t *idx;
+    double *gate;
+    float *logits32;
+    double *logits64;
+    int t0, t1;
+} route_job;
+
+static void *route_worker(void *p)
+{
+    route_job *j = (route_job *)p;
+    float *l = (float *)malloc(sizeof(float) * (size_t)j->E);
+    unsigned char *taken = (unsigned char *)malloc((size_t)j->E);
+    for (int t = j->t0; t < j->t1; ++t) {
+        double *l64 = j->logits64 ? j->logits64 + (size_t)t * j->E : NULL;
+        router_logits_token(j->H, j->E, j->x + (size_t)t * j->H, j->wr, j->bias, l, l64);
+        if (j->logits32) memcpy(j->logits32 + (size_t)t * j->E, l, sizeof(float) * (size_t)j->E);
+        topk_token(j->E, j->k, l, j->idx + (size_t)t * j->k, taken);
+        gates_token(j->k, l, j->idx + (size_t)t * j->k, j->gate + (size_t)t * j->k);
+    }
+    free(l);
+    free(taken);
+    return NULL;
+}
+
+/* Router + softmax top-k for all T tokens.
+ *   x [T,H] bf16, wr [H,E] bf16, bias [E] fp32 or NULL
+ *   -> idx [T,k] int32, gate [T,k] fp64, optional logits32 / logits64 [T,E]. */
+int oracle_route(int T, int H, int E, int k, const uint16_t *x, const uint16_t *wr,
+                 const float *bias, int32_t *idx, double *gate, float *logits32,
+                 double *logits64, int nthreads)
+{
+    if (T < 0 || H <= 0 || E <= 0 || k < 1 || k > E) return 1;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > T) nthreads = T > 0 ? T : 1;
+    pthread_t th[256];
+    route_job jobs[256];
+    if (nthreads > 256) nthreads = 256;
+    for (int i = 0; i < nthreads; ++i) {
+        route_job j = {T, H, E, k, x, wr, bias, idx, gate, logits32, logits64,
+                       (int)((long)T * i / nthreads), (int)((long)T * (i + 1) / nthreads)};
+        jobs[i] = j;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, route_worker, &jobs[i]);
+    route_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    return 0;
+}
+
+/* --------------------------------------------------------------- permute */
+
+/* Stable counting sort of the flat assignment list by expert.
+ *   idx [A] (A = T*k, flat = t*k + j)
+ *   -> offsets [E+1], sorted_to_flat [A], flat_to_sorted [A]
+ *   -> tile_list [3*n] of {expert, row_start, rows}: for e ascending, the
+ *      row blocks of bm rows covering each group, and *num_tiles = n.
+ * tile_list may be NULL (then only *num_tiles is produced). */
+int oracle_permute(int A, int E, const int32_t *idx, int32_t *offsets, int32_t *sorted_to_flat,
+                   int32_t *flat_to_sorted, int bm, int32_t *tile_list, int32_t *num_tiles)
+{
+    if (A < 0 || E <= 0 || bm <= 0) return 1;
+    for (int f = 0; f < A; ++f)
+        if (idx[f] < 0 || idx[f] >= E) return 2;
+    int pos = 0;
+    for (int e = 0; e < E; ++e) {
+        offsets[e] = pos;
+        for (int f = 0; f < A; ++f) {
+            if (idx[f] == e) {
+                sorted_to_flat[pos] = f;
+                flat_to_sorted[f] = pos;
+                ++pos;
+            }
+        }
+    }
+    offsets[E] = pos;
+    int n = 0;
+    for (int e = 0; e < E; ++e) {
+        int c = offsets[e + 1] - offsets[e];
+        for (int r = 0; r < c; r += bm) {
+            if (tile_list) {
+                tile_list[3 * n + 0] = e;
+                tile_list[3 * n + 1] = offsets[e] + r;
+                tile_list[3 * n + 2] = (c - r) < bm ? (c - r) : bm;
+            }
+            ++n;
+        }
+    }
+    *num_tiles = n;
+    return 0;
+}
+
+/* ----------------------------------------------------------- expert FFN */
+
+/* One expert applied to one token, in fp64:
+ *   y = Wd_e ( silu(Wg_e x) * (Wu_e x) )
+ * wg, wu: [E,I,H] bf16; wd: [E,H,I] bf16; a: scratch [I]. */
+static void expert_ffn(int H, int I, int e, const double *x, const uint16_t *wg,
+                       const uint16_t *wu, const uint16_t *wd, double *a, double *y)
+{
+    const uint16_t *g = wg + (size_t)e * I * H;
+    const uint16_t *u = wu + (size_t)e * I * H;
+    const uint16_t *d = wd + (size_t)e * H * I;
+    for (int i = 0; i < I; ++i) {
+        double sg = 0.0, su = 0.0;
+        for (int h = 0; h < H; ++h) {
+            sg += bf16_to_f64(g[(size_t)i * H + h]) * x[h];
+            su += bf16_to_f64(u[(size_t)i * H + h]) * x[h];
+        }
+        a[i] = silu(sg) * su;
+    }
+    for (int o = 0; o < H; ++o) {
+        double s = 0.0;
+        for (int i = 0; i < I; ++i) s += bf16_to_f64(d[(size_t)o * I + i]) * a[i];
+        y[o] = s;
+    }
+}
+
+typedef struct {
+    int H, I, k;
+    const uint16_t *x, *wg, *wu, *wd;
+    const int32_t *idx;
+    const double *gate;
+    const int32_t *tokens;
+    double *out;
+    int n0, n1;
+} ffn_job;
+
+static void *ffn_worker(void *p)
+{
+    ffn_job *j = (ffn_job *)p;
+    double *xt = (double *)malloc(sizeof(double) * (size_t)j->H);
+    double *a = (double *)malloc(sizeof(double) * (size_t)j->I);
+    double *y = (double *)malloc(sizeof(double) * (size_t)j->H);
+    for (int n = j->n0; n < j->n1; ++n) {
+        int t = j->tokens ? j->tokens[n] : n;
+        for (int h = 0; h < j->H; ++h) xt[h] = bf16_to_f64(j->x[(size_t)t * j->H + h]);
+        double *o = j->out + (size_t)n * j->H;
+        for (int h = 0; h < j->H; ++h) o[h] = 0.0;
+        for (int q = 0; q < j->k; ++q) {
+            int e = j->idx[(size_t)t * j->k + q];
+            double g = j->gate[(size_t)t * j->k + q];
+            expert_ffn(j->H, j->I, e, xt, j->wg, j->wu, j->wd, a, y);
+            for (int h = 0; h < j->H; ++h) o[h] += g * y[h];
+        }
+    }
+    free(xt);
+    free(a);
+    free(y);
+    return NULL;
+}
+
+/* Gate-weighted sum of the selected experts' FFN outputs, per token, in fp64.
+ *   idx/gate: [T,k] routing (from oracle_route); tokens: the n token ids to
+ *   evaluate (NULL = tokens 0..n-1)  ->  out [n,H] fp64. */
+int oracle_combine_ffn(int H, int I, int k, const uint16_t *x, const int32_t *idx,
+                       const double *gate, const uint16_t *wg, const uint16_t *wu,
+                       const uint16_t *wd, int n, const int32_t *tokens, double *out,
+                       int nthreads)
+{
+    if (H <= 0 || I <= 0 || k < 1 || n < 0) return 1;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > n) nthreads = n > 0 ? n : 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    ffn_job jobs[256];
+    for (int i = 0; i < nthreads; ++i) {
+        ffn_job j = {H, I, k, x, wg, wu, wd, idx, gate, tokens, out,
+                     (int)((long)n * i / nthreads), (int)((long)n * (i + 1) / nthreads)};
+        jobs[i] = j;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, ffn_worker, &jobs[i]);
+    ffn_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    return 0;
+}

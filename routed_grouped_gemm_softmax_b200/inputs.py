@@ -1,0 +1,174 @@
+"""Seeded synthetic inputs for the MoE layer workloads.
+
+This module is shared by the CUDA path's tests/benchmark and by the CPU oracle's
+tests.  It holds none of the layer's arithmetic: it only draws numbers.
+
+Generator (counter based, identical on CPU and CUDA up to last-ulp differences of
+the fp64 ``log``/``cos`` between host libm and the device):
+
+* splitmix64 (S. Vigna's published mixer): output ``i`` of the stream with key
+  ``K`` is ``mix(K + (i + 1) * 0x9E3779B97F4A7C15)`` with
+  ``mix(z) = z3`` where ``z1 = (z ^ z>>30) * 0xBF58476D1CE4E5B9``,
+  ``z2 = (z1 ^ z1>>27) * 0x94D049BB133111EB``, ``z3 = z2 ^ z2>>31`` (mod 2**64,
+  logical shifts).
+* uniforms from the top 53 bits; Box-Muller from two consecutive draws
+  ``n = sqrt(-2 ln u1) cos(2 pi u2)`` with ``u1`` in (0, 1] and ``u2`` in [0, 1).
+* scaled by the tensor's standard deviation in fp64, rounded to fp32, then
+  round-to-nearest-even to bf16.
+
+Every tensor has its own stream key ``mix(seed * 0x9E3779B97F4A7C15 + tensor_id)``;
+tensors are drawn as x (0), router_w (1), bias (2), w_gate (3), w_up (4),
+w_down (5).
+
+The five workloads are the configurations of the layer the pages describe
+(vLLM fused-MoE page, section 02: a router picks top-k of E experts, each a
+gate/up/down SwiGLU FFN; shapes and distributions as listed in ``CONFIGS``).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+_GOLDEN = 0x9E3779B97F4A7C15
+_M1 = 0xBF58476D1CE4E5B9
+_M2 = 0x94D049BB133111EB
+_MASK64 = (1 << 64) - 1
+
+TENSOR_IDS = {"x": 0, "router_w": 1, "bias": 2, "w_gate": 3, "w_up": 4, "w_down": 5}
+
+
+def _s64(v: int) -> int:
+    v &= _MASK64
+    return v - (1 << 64) if v >= (1 << 63) else v
+
+
+def _lsr(z: torch.Tensor, s: int) -> torch.Tensor:
+    # logical right shift of an int64 tensor holding a uint64 bit pattern
+    return (z >> s) & ((1 << (64 - s)) - 1)
+
+
+def _mix_t(z: torch.Tensor) -> torch.Tensor:
+    z = (z ^ _lsr(z, 30)) * _s64(_M1)
+    z = (z ^ _lsr(z, 27)) * _s64(_M2)
+    return z ^ _lsr(z, 31)
+
+
+def _mix_int(z: int) -> int:
+    z &= _MASK64
+    z = ((z ^ (z >> 30)) * _M1) & _MASK64
+    z = ((z ^ (z >> 27)) * _M2) & _MASK64
+    return z ^ (z >> 31)
+
+
+def stream_key(seed: int, tensor_id: int) -> int:
+    return _mix_int(seed * _GOLDEN + tensor_id)
+
+
+def splitmix64(key: int, start: int, count: int, device="cpu") -> torch.Tensor:
+    """Raw 64-bit outputs ``start .. start+count-1`` of the stream (int64 bit patterns)."""
+    i = torch.arange(start + 1, start + 1 + count, dtype=torch.int64, device=device)
+    z = i * _s64(_GOLDEN) + _s64(key)
+    return _mix_t(z)
+
+
+def normal(key: int, start: int, count: int, device="cpu") -> torch.Tensor:
+    """Standard normals ``start .. start+count-1`` of a stream, in fp64."""
+    z = splitmix64(key, 2 * start, 2 * count, device).view(count, 2)
+    two53 = 2.0 ** -53
+    u1 = (_lsr(z[:, 0], 11).to(torch.float64) + 1.0) * two53
+    u2 = _lsr(z[:, 1], 11).to(torch.float64) * two53
+    return torch.sqrt(-2.0 * torch.log(u1)) * torch.cos((2.0 * math.pi) * u2)
+
+
+def gaussian_tensor(seed: int, name: str, shape, std: float, device="cpu",
+                    out_dtype=torch.bfloat16, chunk: int = 1 << 24) -> torch.Tensor:
+    """``std * N(0,1)`` drawn from the tensor's stream, fp64 -> fp32 -> ``out_dtype``."""
+    key = stream_key(seed, TENSOR_IDS[name])
+    n = 1
+    for s in shape:
+        n *= int(s)
+    out = torch.empty(n, dtype=out_dtype, device=device)
+    for s0 in range(0, n, chunk):
+        c = min(chunk, n - s0)
+        v = normal(key, s0, c, device) * std
+        out[s0:s0 + c] = v.to(torch.float32).to(out_dtype)
+    return out.view(*shape)
+
+
+@dataclass(frozen=True)
+class MoEConfig:
+    name: str
+    T: int
+    H: int
+    E: int
+    top_k: int
+    I: int
+    seed: int
+    dtype: str = "bf16"          # "bf16" or "fp8"
+    zipf_s: float | None = None  # per-expert router bias making popularity ~ Zipf(s)
+    router_std: float = 0.02
+
+    @property
+    def A(self) -> int:
+        return self.T * self.top_k
+
+    def replace(self, **kw) -> "MoEConfig":
+        d = dict(self.__dict__)
+        d.update(kw)
+        return MoEConfig(**d)
+
+
+CONFIGS = {
+    "tiny": MoEConfig("tiny", T=64, H=256, E=8, top_k=2, I=512, seed=0),
+    "decode": MoEConfig("decode", T=16, H=2048, E=256, top_k=8, I=512, seed=1),
+    "prefill": MoEConfig("prefill", T=4096, H=2048, E=256, top_k=8, I=512, seed=2),
+    "skewed": MoEConfig("skewed", T=8192, H=4096, E=64, top_k=6, I=1408, seed=3, zipf_s=1.2),
+    "fp8": MoEConfig("fp8", T=1024, H=7168, E=256, top_k=8, I=2048, seed=4, dtype="fp8"),
+}
+
+
+def zipf_bias(E: int, s: float) -> torch.Tensor:
+    """Per-expert router bias ``ln p_e`` with ``p_e ~ (e+1)^-s`` normalised (expert 0 hottest).
+
+    Under Gumbel-like logit noise of unit scale, top-1 choice frequencies then follow
+    the Zipf law; this is an input recipe, not part of the layer.
+    """
+    r = torch.arange(1, E + 1, dtype=torch.float64)
+    p = r.pow(-s)
+    p = p / p.sum()
+    return torch.log(p).to(torch.float32)
+
+
+@dataclass
+class MoEInputs:
+    cfg: MoEConfig
+    x: torch.Tensor            # [T, H] bf16
+    router_w: torch.Tensor     # [H, E] bf16
+    bias: torch.Tensor | None  # [E] fp32 or None
+    w_gate: torch.Tensor       # [E, I, H] bf16 (fp32 master values for the fp8 config)
+    w_up: torch.Tensor         # [E, I, H]
+    w_down: torch.Tensor       # [E, H, I]
+    extra: dict = field(default_factory=dict)
+
+
+def make_inputs(cfg: MoEConfig, device="cpu", weights: bool = True) -> MoEInputs:
+    """Draw the workload's tensors in the fixed order x, router_w, [bias], w_gate, w_up, w_down.
+
+    Expert weights ~ N(0, 1/sqrt(fan_in)) (fan_in = H for gate/up, I for down);
+    x ~ N(0, 1); router_w ~ N(0, 0.02).  For the fp8 workload the expert weights
+    are returned as fp32 underlying values (each side quantises them itself).
+    """
+    T, H, E, I = cfg.T, cfg.H, cfg.E, cfg.I
+    x = gaussian_tensor(cfg.seed, "x", (T, H), 1.0, device)
+    rw = gaussian_tensor(cfg.seed, "router_w", (H, E), cfg.router_std, device)
+    bias = zipf_bias(E, cfg.zipf_s).to(device) if cfg.zipf_s is not None else None
+    wdt = torch.float32 if cfg.dtype == "fp8" else torch.bfloat16
+    if weights:
+        wg = gaussian_tensor(cfg.seed, "w_gate", (E, I, H), 1.0 / math.sqrt(H), device, wdt)
+        wu = gaussian_tensor(cfg.seed, "w_up", (E, I, H), 1.0 / math.sqrt(H), device, wdt)
+        wd = gaussian_tensor(cfg.seed, "w_down", (E, H, I), 1.0 / math.sqrt(I), device, wdt)
+    else:
+        wg = wu = wd = None
+    return MoEInputs(cfg, x, rw, bias, wg, wu, wd)

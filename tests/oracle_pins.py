@@ -1,0 +1,271 @@
+"""Pins of the CPU oracle to facts outside itself.
+
+Each ``pin_*`` takes an ``oracle.Oracle`` and raises ``AssertionError`` when the
+oracle disagrees with brute force, a closed form, an invariant or a library
+routine.  ``test_oracle_pins.py`` runs them on the real oracle;
+``test_oracle_mutants.py`` runs them on copies of the oracle with a planted
+mistake and requires every mistake to be caught by at least one pin.
+
+Definition pinned (vLLM fused-MoE page, section 02): top-k routing by router
+logits, softmax-normalised gating over the chosen k, a gate/up/down SwiGLU FFN
+per expert, and the gate-weighted sum of the k expert outputs.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_inputs
+
+
+def _bf16(a) -> torch.Tensor:
+    return torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def _f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().double().numpy()
+
+
+def tiny_inputs(**kw):
+    cfg = CONFIGS["tiny"].replace(**kw)
+    return make_inputs(cfg)
+
+
+# ------------------------------------------------------------------ router
+
+def pin_logits_vs_fp64_matmul(orc):
+    """fp32 FMA-chain logits agree with an fp64 numpy matmul within the chain's
+    forward error bound (n*u*sum|x*w|), and the oracle's own fp64 logits agree with
+    numpy's to 1e-12 relative.  A transposed/dropped/shifted term breaks this."""
+    for bias_on in (False, True):
+        inp = tiny_inputs(zipf_s=1.2 if bias_on else None)
+        idx, gate, l32, l64 = orc.route(inp.x, inp.router_w, inp.bias, 2, want_logits=True)
+        X, W = _f64(inp.x), _f64(inp.router_w)
+        ref = X @ W
+        if inp.bias is not None:
+            ref = ref + inp.bias.double().numpy()[None, :]
+        mag = np.abs(X) @ np.abs(W)
+        H = X.shape[1]
+        bound = (H + 2) * 2.0 ** -24 * (mag + (np.abs(inp.bias.double().numpy())[None, :]
+                                               if inp.bias is not None else 0.0)) + 1e-30
+        assert np.all(np.abs(l32.astype(np.float64) - ref) <= bound), "fp32 logits off the bound"
+        assert np.allclose(l64, ref, rtol=1e-12, atol=1e-12), "fp64 logits differ from matmul"
+
+
+def pin_logit_chain_order(orc):
+    """Closed form of the fixed evaluation order: with x = [1, 2^-12, 2^-12] and
+    w = [1, 2^-12, 2^-12] the chain fma over h ascending gives 1 + 2^-24 -> 1
+    (tie to even) twice, i.e. exactly 1.0f; summing the small terms first would
+    give 1 + 2^-23.  Integer-valued inputs give the exact integer dot product."""
+    s = 2.0 ** -12
+    x = _bf16([[1.0, s, s]])
+    w = _bf16([[1.0, 0.0], [s, 0.0], [s, 0.0]])
+    _, _, l32, _ = orc.route(x, w, None, 1, want_logits=True)
+    assert l32[0, 0] == np.float32(1.0), l32[0, 0]
+    x = _bf16([[3, -2, 5, 7]])
+    w = _bf16([[1, 2], [4, -3], [-1, 2], [2, 1]])
+    _, _, l32, _ = orc.route(x, w, None, 2, want_logits=True)
+    assert l32[0, 0] == 3 - 8 - 5 + 14 and l32[0, 1] == 6 + 6 + 10 + 7, l32
+
+
+def pin_topk_brute_force(orc):
+    """Tiny: the selected k equal the first k of a library sort by (-logit, e), and no
+    other k-subset has a larger logit sum (brute-force enumeration of all subsets)."""
+    inp = tiny_inputs()
+    for k in (1, 2, 3, 8):
+        idx, _, l32, _ = orc.route(inp.x, inp.router_w, None, k, want_logits=True)
+        E = l32.shape[1]
+        for t in range(l32.shape[0]):
+            order = sorted(range(E), key=lambda e: (-float(l32[t, e]), e))
+            assert list(idx[t]) == order[:k], (t, idx[t], order[:k])
+            best = max(sum(float(l32[t, e]) for e in c) for c in itertools.combinations(range(E), k))
+            assert sum(float(l32[t, e]) for e in idx[t]) == best
+
+
+def pin_ties_lower_index(orc):
+    """Equal logits go to the lower expert index: router_w = 0 gives experts 0..k-1
+    with gates 1/k; a bias with exact ties [0,1,0,1,1] picks [1,3,4,0,2]."""
+    inp = tiny_inputs()
+    z = torch.zeros_like(inp.router_w)
+    for k in (1, 3, 8):
+        idx, gate = orc.route(inp.x, z, None, k)
+        assert np.all(idx == np.arange(k)[None, :])
+        assert np.all(gate == 1.0 / k) if k in (1, 8) else np.allclose(gate, 1.0 / k, rtol=0, atol=1e-15)
+    x = _bf16(np.ones((2, 4)))
+    w = _bf16(np.zeros((4, 5)))
+    bias = torch.tensor([0.0, 1.0, 0.0, 1.0, 1.0])
+    idx, _ = orc.route(x, w, bias, 5)
+    assert np.all(idx == np.array([1, 3, 4, 0, 2])[None, :]), idx
+
+
+def pin_gates(orc):
+    """Gates sum to 1; k=1 gives exactly 1; k=2 matches the closed form
+    1/(1+exp(l1-l0)); and softmax over all E renormalised over the chosen k
+    (scipy) equals the softmax over the chosen k."""
+    from scipy.special import softmax
+    inp = tiny_inputs()
+    idx, gate = orc.route(inp.x, inp.router_w, None, 1)
+    assert np.all(gate == 1.0)
+    idx, gate, l32, _ = orc.route(inp.x, inp.router_w, None, 2, want_logits=True)
+    l = l32.astype(np.float64)
+    for t in range(l.shape[0]):
+        d = l[t, idx[t, 1]] - l[t, idx[t, 0]]
+        assert abs(gate[t, 0] - 1.0 / (1.0 + math.exp(d))) <= 1e-15
+    for k in (3, 5):
+        idx, gate, l32, _ = orc.route(inp.x, inp.router_w, None, k, want_logits=True)
+        assert np.all(np.abs(gate.sum(1) - 1.0) <= 1e-12)
+        p = softmax(l32.astype(np.float64), axis=1)
+        sel = np.take_along_axis(p, idx.astype(np.int64), 1)
+        assert np.allclose(gate, sel / sel.sum(1, keepdims=True), rtol=1e-12, atol=0)
+
+
+def pin_bias_enters_logits(orc):
+    """A per-expert bias shifts every token's logit by exactly bias[e] (up to the one
+    fp32 rounding of the final add): with a huge bias on expert 5 every token picks 5 first."""
+    inp = tiny_inputs()
+    b = torch.zeros(8)
+    b[5] = 1000.0
+    idx, _, l32, _ = orc.route(inp.x, inp.router_w, b, 2, want_logits=True)
+    _, _, l0, _ = orc.route(inp.x, inp.router_w, None, 2, want_logits=True)
+    assert np.all(idx[:, 0] == 5)
+    assert np.all(l32[:, 5] == (l0[:, 5] + np.float32(1000.0)))
+    assert np.all(np.delete(l32, 5, 1) == np.delete(l0, 5, 1))
+
+
+# ----------------------------------------------------------------- permute
+
+def _check_permute(idx, E, p, bm=128):
+    fl = np.asarray(idx).reshape(-1)
+    A = fl.size
+    s2f, f2s, off = p["sorted_to_flat"], p["flat_to_sorted"], p["offsets"]
+    assert off[0] == 0 and off[E] == A and np.all(np.diff(off) >= 0)
+    assert np.array_equal(np.diff(off), np.bincount(fl, minlength=E))
+    assert np.array_equal(np.sort(s2f), np.arange(A)), "not a bijection"
+    assert np.array_equal(s2f[f2s], np.arange(A)) and np.array_equal(f2s[s2f], np.arange(A))
+    assert np.array_equal(s2f, np.argsort(fl, kind="stable")), "not the stable sort"
+    tiles = [(e, off[e] + r, min(bm, off[e + 1] - off[e] - r))
+             for e in range(E) for r in range(0, off[e + 1] - off[e], bm)]
+    assert p["num_tiles"] == len(tiles)
+    assert [tuple(int(v) for v in row) for row in p["tile_list"]] == tiles
+
+
+def pin_permute(orc):
+    """Bijection + inverse, offsets = cumulative bincount, order = numpy's stable
+    argsort, tile list = closed form; on skewed, empty and single-expert routings."""
+    rng = np.random.default_rng(7)
+    cases = [(rng.integers(0, 8, size=(64, 2)), 8),
+             (rng.integers(0, 256, size=(512, 8)), 256),
+             (np.zeros((300, 1), np.int64), 4),                   # one expert holds all
+             (np.minimum(rng.zipf(1.5, size=(1000, 3)) - 1, 15), 16),
+             (np.zeros((0, 2), np.int64), 8)]                     # empty
+    for bm in (128, 7):
+        for idx, E in cases:
+            p = orc.permute(idx, E, bm=bm)
+            _check_permute(idx, E, p, bm)
+
+
+# ------------------------------------------------------------- expert FFN
+
+def _dense_reference(inp, idx, gate):
+    """Brute force: every expert on every token (numpy fp64 matmuls), masked by a
+    dense [T,E] gate matrix that is zero for experts a token did not pick."""
+    X = _f64(inp.x)
+    Wg, Wu, Wd = _f64(inp.w_gate), _f64(inp.w_up), _f64(inp.w_down)
+    T, E = X.shape[0], Wg.shape[0]
+    G = np.zeros((T, E))
+    for t in range(T):
+        for j in range(idx.shape[1]):
+            G[t, idx[t, j]] += gate[t, j]
+    out = np.zeros_like(X)
+    for e in range(E):
+        g = X @ Wg[e].T
+        u = X @ Wu[e].T
+        a = (g / (1.0 + np.exp(-g))) * u
+        out += G[:, e:e + 1] * (a @ Wd[e].T)
+    return out
+
+
+def pin_ffn_dense_brute_force(orc):
+    """Tiny: the per-token sparse evaluation equals the dense all-experts evaluation."""
+    for k in (1, 2, 5):
+        inp = tiny_inputs(T=24)
+        idx, gate = orc.route(inp.x, inp.router_w, None, k)
+        out = orc.combine_ffn(inp.x, idx, gate, inp.w_gate, inp.w_up, inp.w_down)
+        ref = _dense_reference(inp, idx, gate)
+        assert np.allclose(out, ref, rtol=1e-11, atol=1e-12), np.abs(out - ref).max()
+
+
+def pin_topk_all_uniform_is_mean(orc):
+    """top_k = E with router_w = 0 (uniform gates 1/E): out = mean_e FFN_e(x) (torch fp64)."""
+    inp = tiny_inputs(T=16)
+    z = torch.zeros_like(inp.router_w)
+    out, idx, gate = orc.forward(inp.x, z, None, inp.w_gate, inp.w_up, inp.w_down, top_k=8)
+    x = inp.x.double()
+    ys = []
+    for e in range(8):
+        a = F.silu(x @ inp.w_gate[e].double().T) * (x @ inp.w_up[e].double().T)
+        ys.append(a @ inp.w_down[e].double().T)
+    ref = torch.stack(ys).mean(0).numpy()
+    assert np.allclose(out, ref, rtol=1e-11, atol=1e-12), np.abs(out - ref).max()
+
+
+def pin_identical_experts(orc):
+    """All experts identical: out = FFN(x) whatever the routing (gates sum to 1)."""
+    inp = tiny_inputs(T=16)
+    wg = inp.w_gate[:1].expand_as(inp.w_gate).contiguous()
+    wu = inp.w_up[:1].expand_as(inp.w_up).contiguous()
+    wd = inp.w_down[:1].expand_as(inp.w_down).contiguous()
+    out, _, _ = orc.forward(inp.x, inp.router_w, None, wg, wu, wd, top_k=3)
+    x = inp.x.double()
+    ref = ((F.silu(x @ wg[0].double().T) * (x @ wu[0].double().T)) @ wd[0].double().T).numpy()
+    assert np.allclose(out, ref, rtol=1e-11, atol=1e-12)
+
+
+def pin_single_expert_is_swiglu_mlp(orc):
+    """E = 1, k = 1: the layer is a textbook SwiGLU MLP (torch fp64 silu and matmuls)."""
+    inp = tiny_inputs(T=12, E=1)
+    out, idx, gate = orc.forward(inp.x, inp.router_w, None, inp.w_gate, inp.w_up, inp.w_down, top_k=1)
+    assert np.all(idx == 0) and np.all(gate == 1.0)
+    x = inp.x.double()
+    ref = ((F.silu(x @ inp.w_gate[0].double().T) * (x @ inp.w_up[0].double().T))
+           @ inp.w_down[0].double().T).numpy()
+    assert np.allclose(out, ref, rtol=1e-11, atol=1e-12)
+
+
+def pin_linear_in_down_proj(orc):
+    """Doubling W_down (exact in bf16) doubles the output exactly."""
+    inp = tiny_inputs(T=8)
+    idx, gate = orc.route(inp.x, inp.router_w, None, 2)
+    a = orc.combine_ffn(inp.x, idx, gate, inp.w_gate, inp.w_up, inp.w_down)
+    b = orc.combine_ffn(inp.x, idx, gate, inp.w_gate, inp.w_up, inp.w_down * 2)
+    assert np.array_equal(b, 2 * a)
+
+
+def pin_worked_example(orc):
+    """Hand-derived example: x = [1, 2]; router columns give logits (1, 2, 1.5) so the
+    top-2 is (1, 2) with gates (1/(1+e^-0.5), 1/(1+e^0.5)); with I = 1,
+      expert 1: g = 1, u = 2, a = 2 silu(1), y = a * (1, -1)
+      expert 2: g = 2, u = 3, a = 3 silu(2), y = a * (0.5, 2)."""
+    x = _bf16([[1.0, 2.0]])
+    rw = _bf16([[1.0, 0.0, 0.5], [0.0, 1.0, 0.5]])
+    wg = _bf16([[[0.0, 0.0]], [[1.0, 0.0]], [[0.0, 1.0]]])
+    wu = _bf16([[[0.0, 0.0]], [[0.0, 1.0]], [[1.0, 1.0]]])
+    wd = _bf16([[[0.0], [0.0]], [[1.0], [-1.0]], [[0.5], [2.0]]])
+    out, idx, gate = orc.forward(x, rw, None, wg, wu, wd, top_k=2)
+    assert list(idx[0]) == [1, 2]
+    g0, g1 = 1.0 / (1.0 + math.exp(-0.5)), 1.0 / (1.0 + math.exp(0.5))
+    assert abs(gate[0, 0] - g0) < 1e-15 and abs(gate[0, 1] - g1) < 1e-15
+    silu = lambda v: v / (1.0 + math.exp(-v))
+    a1, a2 = 2.0 * silu(1.0), 3.0 * silu(2.0)
+    ref = [g0 * a1 + g1 * 0.5 * a2, -g0 * a1 + g1 * 2.0 * a2]
+    assert np.allclose(out[0], ref, rtol=1e-14, atol=0), (out[0], ref)
+
+
+ALL_PINS = [pin_logits_vs_fp64_matmul, pin_logit_chain_order, pin_topk_brute_force,
+            pin_ties_lower_index, pin_gates, pin_bias_enters_logits, pin_permute,
+            pin_ffn_dense_brute_force, pin_topk_all_uniform_is_mean, pin_identical_experts,
+            pin_single_expert_is_swiglu_mlp, pin_linear_in_down_proj, pin_worked_example]
