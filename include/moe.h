@@ -1,0 +1,154 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed MoE layer forward.
+ *
+ * The layer (vLLM fused-MoE page, section 02 "what the fused MoE kernel
+ * computes"; the same route -> dispatch -> expert FFN -> combine path as the
+ * Weave review, section 1.2, and the stepwise-vs-fused comparison page,
+ * section 2):
+ *
+ *   logit[t,e] = sum_h x[t,h] * router_w[h,e]  (+ router_bias[e])
+ *   S_t        = top_k experts by logit, descending; equal logits -> lower index
+ *   gate[t,j]  = softmax of the logits of S_t (over the k chosen experts)
+ *   out[t]     = sum_j gate[t,j] * W_down[e] ( silu(W_gate[e] x_t) * (W_up[e] x_t) ),
+ *                e = S_t[j],  silu(a) = a / (1 + exp(-a))
+ *
+ * The router logit is an fp32 value with a fixed evaluation order -- a chain of
+ * fused multiply-adds over h ascending starting from 0, then + bias[e] in fp32 --
+ * so the routing decision is reproducible bit for bit by any implementation
+ * that follows the same order.
+ *
+ * Conventions shared by every call
+ *  - Pointers are DEVICE pointers unless stated otherwise; the caller owns all
+ *    memory, including the workspace.  The library never allocates or frees
+ *    device memory and never synchronises, except moe_get_device_status().
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    All work is enqueued asynchronously on it; calls on one workspace must not
+ *    overlap on the GPU.
+ *  - Layouts (row-major, element type in brackets):
+ *      x          [T, H]     bf16
+ *      router_w   [H, E]     bf16
+ *      router_bias[E]        fp32, may be NULL
+ *      w_gate     [E, I, H]  bf16 (each expert's rows are K-major, nn.Linear style)
+ *      w_up       [E, I, H]  bf16
+ *      w_down     [E, H, I]  bf16
+ *      out        [T, H]     bf16
+ *      topk_idx   [T, top_k] int32,  topk_w [T, top_k] fp32
+ *    The flat assignment index of (t, j) is f = t*top_k + j.
+ *  - Host-detectable errors return at once and enqueue nothing:
+ *      MOE_ERR_INVALID_ARG  NULL dims or required pointer, T < 0, H/I/E <= 0,
+ *                           top_k < 1 or > E, H or I not a multiple of 64
+ *      MOE_ERR_UNSUPPORTED  E > 1024
+ *      MOE_ERR_WORKSPACE    ws NULL/misaligned (256 B) or ws_bytes too small
+ *      MOE_ERR_CUDA         a launch failed (cudaGetLastError)
+ *    T == 0 is a no-op that returns MOE_OK.
+ *  - Errors found on the device (an expert index outside [0,E) handed to
+ *    moe_permute, a pipeline wait that exceeded its time limit) are recorded in
+ *    a status word inside the workspace; moe_permute and moe_forward clear it
+ *    when they start, and moe_get_device_status() reads it.
+ *  - Results do not depend on the number of GEMM CTAs or on the order in which
+ *    they claim work: every sum is taken in an order fixed by the data alone.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_WORKSPACE = 3,
+    MOE_ERR_CUDA = 4,
+    MOE_ERR_TIMEOUT = 5,     /* device: a pipeline wait ran past its limit */
+    MOE_ERR_BAD_INDEX = 6    /* device: an expert index outside [0, E) */
+} moe_status_t;
+
+typedef struct {
+    int32_t T;      /* tokens */
+    int32_t H;      /* hidden size */
+    int32_t I;      /* expert intermediate size */
+    int32_t E;      /* experts */
+    int32_t top_k;  /* experts per token */
+} moe_dims_t;
+
+enum { MOE_DTYPE_BF16 = 0 };
+
+/* Rows of the GEMM tiles; tile_list entries cover at most this many rows. */
+#define MOE_TILE_ROWS 128
+
+/* Bytes of workspace every call below needs for these dims (256-byte aligned
+ * base required).  Returns 0 for invalid dims.  The workspace holds the router
+ * logits, the permutation scratch, the expert-sorted activations and the
+ * intermediate h and per-assignment outputs. */
+size_t moe_workspace_size(const moe_dims_t *d, int dtype);
+
+/* Upper bound of the number of tile_list entries moe_permute can produce:
+ * ceil(T*top_k / 128) + min(E, T*top_k). */
+int32_t moe_max_tiles(const moe_dims_t *d);
+
+/* Router logits, top-k selection and softmax gating (vLLM fused-MoE page,
+ * section 02: each token's router picks the top-k experts; the k outputs are
+ * later summed with these gating weights).
+ *   x, router_w, router_bias (nullable)  ->  topk_idx [T,k] int32 (descending
+ *   logit, ties to the lower index), topk_w [T,k] fp32 (sums to 1 per token). */
+moe_status_t moe_route(const moe_dims_t *d, const void *x, const void *router_w,
+                       const float *router_bias, int32_t *topk_idx, float *topk_w,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/* Permute: group the flat assignments by expert (vLLM fused-MoE page, section
+ * 02: tokens are sorted and grouped by expert before the grouped GEMM).  A
+ * stable counting sort by expert of f = 0..T*k-1:
+ *   expert_offsets [E+1]  group e occupies sorted rows [off[e], off[e+1]), no padding
+ *   sorted_to_flat [T*k]  flat index of each sorted row (ascending within a group)
+ *   flat_to_sorted [T*k]  inverse permutation
+ *   tile_list [3*moe_max_tiles]  {expert, row_start, rows} for e ascending and
+ *                         each 128-row block of group e (rows <= 128)
+ *   num_tiles [1]         number of tile_list entries (device int32)
+ * topk_idx entries outside [0,E) are skipped and flagged MOE_ERR_BAD_INDEX. */
+moe_status_t moe_permute(const moe_dims_t *d, const int32_t *topk_idx, int32_t *expert_offsets,
+                         int32_t *sorted_to_flat, int32_t *flat_to_sorted, int32_t *tile_list,
+                         int32_t *num_tiles, void *ws, size_t ws_bytes, void *stream);
+
+/* The whole layer: route, permute, grouped gate/up GEMM with SwiGLU, grouped
+ * down GEMM, gate-weighted combine (stepwise-vs-fused comparison page, section
+ * 2: two linear layers with SwiGLU per expert between dispatch and combine).
+ * Expert GEMMs run on the tensor cores with fp32 accumulation; the SwiGLU
+ * output h and the per-assignment expert outputs are rounded to bf16; the
+ * combine sums the k contributions in fp32 in ascending j and rounds to bf16. */
+moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_w,
+                         const float *router_bias, const void *w_gate, const void *w_up,
+                         const void *w_down, void *out, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, returns the device status word of the workspace
+ * (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_BAD_INDEX; MOE_ERR_CUDA if the stream
+ * reports an error) and clears it. */
+moe_status_t moe_get_device_status(void *ws, void *stream);
+
+/* Number of persistent CTAs each grouped GEMM launches (0 = one per SM, the
+ * default).  Results are bitwise independent of it; it exists so that tests can
+ * check that.  Process-wide setting. */
+void moe_set_gemm_ctas(int32_t ctas);
+
+/* Order in which the GEMM CTAs claim work items: 0 = ascending (default),
+ * 1 = descending.  Results are bitwise independent of it.  Process-wide. */
+void moe_set_claim_order(int32_t reverse);
+
+/* Stage timing hook for benchmarks.  With `events` pointing at MOE_STAGE_EVENTS
+ * caller-created cudaEvent_t handles (passed as void*), every later moe_forward
+ * records them on its stream at the stage boundaries: [0] start, [1] routed,
+ * [2] permuted (groups, tile list, sorted activations), [3] gate/up GEMM done,
+ * [4] down GEMM done, [5] combined.  The handles must stay valid while set;
+ * NULL (or n != MOE_STAGE_EVENTS) turns recording off.  Process-wide. */
+#define MOE_STAGE_EVENTS 6
+void moe_set_stage_events(void *const *events, int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,197 @@
+"""Thin Python binding of the C ABI in ``include/moe.h`` (argument marshalling only).
+
+Every step of the layer runs in the CUDA library ``libmoe_b200.so``; PyTorch only
+provides device memory and the current stream.  If the library is missing the
+calls raise -- there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+                3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT",
+                6: "MOE_ERR_BAD_INDEX"}
+EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "moe_forward",
+           "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order",
+           "moe_set_stage_events"]
+STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
+TILE_ROWS = 128
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)}")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("top_k", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} (run __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        D = ctypes.POINTER(Dims)
+        L.moe_workspace_size.argtypes = [D, ctypes.c_int]
+        L.moe_workspace_size.restype = SZ
+        L.moe_max_tiles.argtypes = [D]
+        L.moe_max_tiles.restype = I32
+        L.moe_route.argtypes = [D, P, P, P, P, P, P, SZ, P]
+        L.moe_route.restype = ctypes.c_int
+        L.moe_permute.argtypes = [D, P, P, P, P, P, P, P, SZ, P]
+        L.moe_permute.restype = ctypes.c_int
+        L.moe_forward.argtypes = [D, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_forward.restype = ctypes.c_int
+        L.moe_get_device_status.argtypes = [P, P]
+        L.moe_get_device_status.restype = ctypes.c_int
+        L.moe_set_gemm_ctas.argtypes = [I32]
+        L.moe_set_gemm_ctas.restype = None
+        L.moe_set_claim_order.argtypes = [I32]
+        L.moe_set_claim_order.restype = None
+        L.moe_set_stage_events.argtypes = [P, I32]
+        L.moe_set_stage_events.restype = None
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != MOE_OK:
+        raise MoEError(code, where)
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def dims(T, H, I, E, top_k) -> Dims:
+    return Dims(int(T), int(H), int(I), int(E), int(top_k))
+
+
+def moe_workspace_size(T, H, I, E, top_k) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(dims(T, H, I, E, top_k)), 0))
+
+
+def moe_max_tiles(T, H, I, E, top_k) -> int:
+    return int(lib().moe_max_tiles(ctypes.byref(dims(T, H, I, E, top_k))))
+
+
+def workspace(T, H, I, E, top_k, device) -> torch.Tensor:
+    n = moe_workspace_size(T, H, I, E, top_k)
+    if n == 0:
+        raise MoEError(1, "moe_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def moe_route(x, router_w, bias, top_k: int, topk_idx=None, topk_w=None, ws=None, stream=None,
+              I: int = 64):
+    """Router + softmax top-k; returns (topk_idx int32 [T,k], topk_w fp32 [T,k])."""
+    T, H = x.shape
+    E = router_w.shape[1]
+    dev = x.device
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(router_w, torch.bfloat16, (H, E), "router_w")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "router_bias")
+    topk_idx = torch.empty((T, top_k), dtype=torch.int32, device=dev) if topk_idx is None else topk_idx
+    topk_w = torch.empty((T, top_k), dtype=torch.float32, device=dev) if topk_w is None else topk_w
+    ws = workspace(T, H, I, E, top_k, dev) if ws is None else ws
+    d = dims(T, H, I, E, top_k)
+    _check(lib().moe_route(ctypes.byref(d), _p(x), _p(router_w), _p(bias), _p(topk_idx), _p(topk_w),
+                           _p(ws), ws.numel(), _stream(stream, dev)), "moe_route")
+    return topk_idx, topk_w
+
+
+def moe_permute(topk_idx, E: int, ws=None, stream=None, H: int = 64, I: int = 64):
+    """Stable grouping of the flat assignments by expert; returns a dict of device tensors
+    (offsets, sorted_to_flat, flat_to_sorted, tile_list [max_tiles,3], num_tiles [1])."""
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    _need(topk_idx, torch.int32, (T, k), "topk_idx")
+    A = T * k
+    nt_max = max(moe_max_tiles(T, H, I, E, k), 1)
+    res = {"offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+           "sorted_to_flat": torch.empty(max(A, 1), dtype=torch.int32, device=dev),
+           "flat_to_sorted": torch.empty(max(A, 1), dtype=torch.int32, device=dev),
+           "tile_list": torch.empty((nt_max, 3), dtype=torch.int32, device=dev),
+           "num_tiles": torch.zeros(1, dtype=torch.int32, device=dev)}
+    ws = workspace(T, H, I, E, k, dev) if ws is None else ws
+    d = dims(T, H, I, E, k)
+    _check(lib().moe_permute(ctypes.byref(d), _p(topk_idx), _p(res["offsets"]), _p(res["sorted_to_flat"]),
+                             _p(res["flat_to_sorted"]), _p(res["tile_list"]), _p(res["num_tiles"]),
+                             _p(ws), ws.numel(), _stream(stream, dev)), "moe_permute")
+    return res
+
+
+def moe_forward(x, router_w, bias, w_gate, w_up, w_down, top_k: int, out=None, ws=None, stream=None):
+    """The MoE layer forward; returns out bf16 [T,H]."""
+    T, H = x.shape
+    E, I, _ = w_gate.shape
+    dev = x.device
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(router_w, torch.bfloat16, (H, E), "router_w")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "router_bias")
+    _need(w_gate, torch.bfloat16, (E, I, H), "w_gate")
+    _need(w_up, torch.bfloat16, (E, I, H), "w_up")
+    _need(w_down, torch.bfloat16, (E, H, I), "w_down")
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    _need(out, torch.bfloat16, (T, H), "out")
+    ws = workspace(T, H, I, E, top_k, dev) if ws is None else ws
+    d = dims(T, H, I, E, top_k)
+    _check(lib().moe_forward(ctypes.byref(d), _p(x), _p(router_w), _p(bias), _p(w_gate), _p(w_up),
+                             _p(w_down), _p(out), _p(ws), ws.numel(), _stream(stream, dev)),
+           "moe_forward")
+    return out
+
+
+def moe_get_device_status(ws, stream=None) -> int:
+    """Synchronise the stream and return (and clear) the workspace's device status word."""
+    return int(lib().moe_get_device_status(_p(ws), _stream(stream, ws.device)))
+
+
+def set_gemm_ctas(n: int):
+    lib().moe_set_gemm_ctas(int(n))
+
+
+def set_claim_order(reverse: bool):
+    lib().moe_set_claim_order(1 if reverse else 0)
+
+
+def set_stage_events(events):
+    """Record these 6 torch.cuda.Events at the stage boundaries of every later
+    moe_forward (None turns it off).  Each event must have been recorded once so
+    that its CUDA handle exists."""
+    if events is None:
+        lib().moe_set_stage_events(None, 0)
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    set_stage_events._keep = arr
+    lib().moe_set_stage_events(arr, len(events))

@@ -1,0 +1,305 @@
+// grouped_gemm.cu -- persistent grouped GEMMs of the expert FFN on the 5th-gen
+// tensor cores (tcgen05 + TMEM + TMA), sm_100a.
+//
+// Work decomposition.  The expert FFN is a batch of small GEMMs, one per expert
+// group (GC-MoE page: "grouped GEMM batches the experts' small matrix products
+// into one kernel"; vLLM fused-MoE page, section 02).  A work item is one
+// (m-tile, n-tile) pair, where the m-tiles are the 128-row blocks of the expert
+// groups listed by the permutation (FlashMoE, section 3: 128x128-class tile
+// tasks).  CTAs are persistent -- one per SM -- and claim the next item from a
+// global atomic counter whenever they are free (the Weave review, section 2.2:
+// a task queue plus an atomic counter from which idle SMs grab the next task),
+// so a hot expert's many tiles spread over every SM instead of queueing on a
+// fixed subset.  Items are numbered m-tile-major, so the n-tiles of one m-tile
+// and the m-tiles of one expert are claimed close together and share the A rows
+// and the expert's weight tiles in L2 (the GROUP_SIZE_M idea of the vLLM page,
+// section 03).
+//
+// CTA roles (192 threads):
+//   warp 0, lane 0: claims items, feeds a ring of item ids to the other roles,
+//                   and streams A and B tiles into a 4-stage shared-memory ring
+//                   with TMA (128-byte swizzle), one mbarrier pair per stage;
+//   warp 1        : allocates 512 TMEM columns; lane 0 issues tcgen05.mma
+//                   (M=128, N=256, K=16, bf16 in, fp32 accumulate) into one of
+//                   two TMEM accumulators, releasing each stage with
+//                   tcgen05.commit;
+//   warps 2-5     : epilogue -- tcgen05.ld of the accumulator (each warp reads
+//                   its 32-lane quarter), then
+//                   mode 0 (gate/up): h = silu(gate) * up, rounded to bf16,
+//                   mode 1 (down)   : y row of the assignment, rounded to bf16,
+//                   rows past the group's end masked.
+// Every accumulation order is fixed by the tile and the K loop, never by which
+// CTA ran the item, so results are bitwise independent of the schedule.
+// Every wait is bounded; a wait that runs out records MOE_ERR_TIMEOUT in the
+// workspace status word and the CTA unwinds (waiting, again bounded, for its
+// own TMA copies and MMAs) before freeing TMEM.
+#include "moe_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = kTileRows;  // 128 rows per tile
+constexpr int BK = 64;         // 64 bf16 = one 128-byte swizzle row
+constexpr int BN = 256;        // MMA N
+constexpr int STAGES = 4;
+constexpr int RING = 4;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;   // two 128 x 256 fp32 accumulators
+
+struct Ctrl {
+    uint64_t full[STAGES];   // TMA bytes landed in stage s
+    uint64_t empty[STAGES];  // MMAs reading stage s finished
+    uint64_t accf[2];        // accumulator a holds a finished tile
+    uint64_t acce[2];        // epilogue drained accumulator a
+    uint64_t itf[RING];      // ring slot r holds the next item id
+    uint64_t ite[RING];      // every role has read ring slot r
+    uint64_t fin;            // all MMAs of this CTA are done
+    int32_t ring[RING];
+    uint32_t tmem_base;
+};
+
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + sizeof(Ctrl);
+
+__device__ __forceinline__ void record_status(int32_t *status, int code) { atomicCAS(status, 0, code); }
+
+__device__ __forceinline__ float silu(float a) { return a / (1.0f + __expf(-a)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1, const GemmArgs g)
+{
+    // output columns per tile: mode 0 packs 128 gate + 128 up columns into N=256
+    constexpr int BNO = MODE == 0 ? BN / 2 : BN;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    uint8_t *sA = smem_raw + pad;
+    uint8_t *sB = sA + STAGES * A_BYTES;
+    Ctrl *S = reinterpret_cast<Ctrl *>(sB + STAGES * B_BYTES);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int n_tiles = (g.N + BNO - 1) / BNO;
+    const int num_kb = g.K / BK;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&S->full[s], 1);
+            mbar_init(&S->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&S->accf[a], 1);
+            mbar_init(&S->acce[a], 4);
+        }
+        for (int r = 0; r < RING; ++r) {
+            mbar_init(&S->itf[r], 1);
+            mbar_init(&S->ite[r], 5);  // the MMA thread + 4 epilogue warps
+        }
+        mbar_init(&S->fin, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB0);
+        if (MODE == 0) tma_prefetch_desc(&tmB1);
+    }
+    if (warp == 1) tmem_alloc(&S->tmem_base, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------ scheduler + TMA producer
+        if (lane == 0) {
+            const int total = *g.ntiles * n_tiles;
+            int stage = 0, rs = 0;
+            uint32_t phase = 0, rphase = 0;
+            uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
+            bool ok = true;
+            for (;;) {
+                int item = atomicAdd(g.counter, 1);
+                if (item >= total)
+                    item = -1;
+                else if (g.reverse)
+                    item = total - 1 - item;
+                if (!mbar_wait(&S->ite[rs], rphase ^ 1)) { ok = false; break; }
+                S->ring[rs] = item;
+                mbar_arrive(&S->itf[rs]);
+                if (++rs == RING) { rs = 0; rphase ^= 1; }
+                if (item < 0) break;
+                const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
+                const int expert = g.tiles[3 * mt], row0 = g.tiles[3 * mt + 1];
+                const int n0 = nt * BNO;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&S->empty[stage], phase ^ 1)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&S->full[stage], A_BYTES + B_BYTES);
+                    armed |= 1u << stage;
+                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                    uint8_t *a_dst = sA + stage * A_BYTES;
+                    uint8_t *b_dst = sB + stage * B_BYTES;
+                    tma_load_2d(a_dst, &tmA, &S->full[stage], kb * BK, row0);
+                    tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
+                    if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (!ok) {
+                record_status(g.status, MOE_ERR_TIMEOUT);
+                if (mbar_wait(&S->ite[rs], rphase ^ 1)) {
+                    S->ring[rs] = -1;
+                    mbar_arrive(&S->itf[rs]);
+                }
+            }
+            // never leave with TMA copies still landing in shared memory
+            for (int s = 0; s < STAGES; ++s)
+                if ((armed >> s) & 1u)
+                    if (!mbar_wait(&S->full[s], (armed_par >> s) & 1u)) record_status(g.status, MOE_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+            int stage = 0, rs = 0, acc = 0;
+            uint32_t phase = 0, rphase = 0, aphase = 0;
+            bool ok = true;
+            for (;;) {
+                if (!mbar_wait(&S->itf[rs], rphase)) { ok = false; break; }
+                const int item = S->ring[rs];
+                mbar_arrive(&S->ite[rs]);
+                if (++rs == RING) { rs = 0; rphase ^= 1; }
+                if (item < 0) break;
+                if (!mbar_wait(&S->acce[acc], aphase ^ 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&S->full[stage], phase)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+                    const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_bf16(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), IDESC,
+                                 (kb | k) != 0);
+                    mma_commit(&S->empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&S->accf[acc]);
+                if (++acc == 2) { acc = 0; aphase ^= 1; }
+            }
+            if (!ok) record_status(g.status, MOE_ERR_TIMEOUT);
+            // TMEM may only be released once every MMA issued here has completed
+            mma_commit(&S->fin);
+            if (!mbar_wait(&S->fin, 0)) record_status(g.status, MOE_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may read
+        const int row = q * 32 + lane;
+        int rs = 0, acc = 0;
+        uint32_t rphase = 0, aphase = 0;
+        for (;;) {
+            if (!mbar_wait(&S->itf[rs], rphase)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
+            const int item = S->ring[rs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S->ite[rs]);
+            if (++rs == RING) { rs = 0; rphase ^= 1; }
+            if (item < 0) break;
+            const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
+            const int row0 = g.tiles[3 * mt + 1], rows = g.tiles[3 * mt + 2];
+            const bool row_ok = row < rows;
+            if (!mbar_wait(&S->accf[acc], aphase)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
+            tc_fence_after();
+            const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+            if (MODE == 0) {
+                __nv_bfloat16 *orow = g.out + (size_t)(row0 + row) * g.N;
+#pragma unroll 1
+                for (int c = 0; c < BNO / 32; ++c) {
+                    uint32_t gr[32], ur[32];
+                    tmem_ld32_sync(tb + c * 32, gr);
+                    tmem_ld32_sync(tb + BNO + c * 32, ur);
+                    const int col = nt * BNO + c * 32;
+                    if (row_ok && col < g.N) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float h0 = silu(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
+                            const float h1 = silu(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
+                            pk[i] = pack_bf16(h0, h1);
+                        }
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            } else {
+                const int flat = row_ok ? g.row_map[row0 + row] : 0;
+                __nv_bfloat16 *orow = g.out + (size_t)flat * g.N;
+#pragma unroll 1
+                for (int c = 0; c < BNO / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32_sync(tb + c * 32, r);
+                    const int col = nt * BNO + c * 32;
+                    if (row_ok && col < g.N) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S->acce[acc]);
+            if (++acc == 2) { acc = 0; aphase ^= 1; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
+                                const CUtensorMap &tmB1, cudaStream_t st)
+{
+    const int grid = g.ctas > 0 ? g.ctas : num_sms();
+    cudaError_t e;
+    if (g.mode == 0) {
+        e = cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        grouped_gemm_kernel<0><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
+    } else {
+        e = cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        grouped_gemm_kernel<1><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,248 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument checks, workspace
+// carving, TMA descriptor encoding and the launch sequence of the layer.
+//
+// moe_forward enqueues, on the caller's stream:
+//   route_logits -> route_topk          (router, softmax over the top-k)
+//   perm_count -> perm_scan -> perm_scatter   (group assignments by expert)
+//   gather_rows                         (activations in expert-sorted order)
+//   grouped GEMM mode 0                 (gate/up + SwiGLU -> h)
+//   grouped GEMM mode 1                 (down -> one row per assignment)
+//   combine                             (gate-weighted sum back to token order)
+// following the route -> dispatch -> expert FFN -> combine stages of the
+// stepwise-vs-fused comparison page (section 6, stepwise pseudo-code), on one GPU.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "moe_internal.h"
+
+namespace {
+
+std::atomic<int> g_gemm_ctas{0};
+std::atomic<int> g_claim_reverse{0};
+std::mutex g_ev_mu;
+cudaEvent_t g_stage_ev[MOE_STAGE_EVENTS];
+bool g_stage_on = false;
+
+struct StageMarks {
+    cudaEvent_t ev[MOE_STAGE_EVENTS];
+    bool on = false;
+    StageMarks()
+    {
+        std::lock_guard<std::mutex> lk(g_ev_mu);
+        on = g_stage_on;
+        for (int i = 0; i < MOE_STAGE_EVENTS; ++i) ev[i] = g_stage_ev[i];
+    }
+    cudaError_t mark(int i, cudaStream_t st) const { return on ? cudaEventRecord(ev[i], st) : cudaSuccess; }
+};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 matrix [rows, cols] (row-major), tiles of box_rows x 64 with the 128-byte swizzle.
+bool encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 weights [E, rows, cols], tiles of box_rows x 64 of one expert.
+bool encode_3d(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {cols, rows, E};
+    const cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+    const cuuint32_t box[3] = {64, box_rows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+moe_status_t check_dims(const moe_dims_t *d)
+{
+    if (!d) return MOE_ERR_INVALID_ARG;
+    if (d->T < 0 || d->H <= 0 || d->I <= 0 || d->E <= 0) return MOE_ERR_INVALID_ARG;
+    if (d->top_k < 1 || d->top_k > d->E) return MOE_ERR_INVALID_ARG;
+    if (d->H % 64 != 0 || d->I % 64 != 0) return MOE_ERR_INVALID_ARG;
+    if (d->E > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    if ((int64_t)d->T * d->top_k > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status_t check_ws(const moe_dims_t *d, const void *ws, size_t ws_bytes)
+{
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < moe::ws_layout(*d).total) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+template <class T>
+T *at(void *ws, size_t off)
+{
+    return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_dims_t *d, int dtype)
+{
+    if (check_dims(d) != MOE_OK || dtype != MOE_DTYPE_BF16) return 0;
+    return moe::ws_layout(*d).total;
+}
+
+int32_t moe_max_tiles(const moe_dims_t *d)
+{
+    if (check_dims(d) != MOE_OK) return 0;
+    const int64_t A = (int64_t)d->T * d->top_k;
+    return (int32_t)((A + moe::kTileRows - 1) / moe::kTileRows + (A < d->E ? A : d->E));
+}
+
+void moe_set_gemm_ctas(int32_t ctas) { g_gemm_ctas.store(ctas > 0 ? ctas : 0); }
+
+void moe_set_claim_order(int32_t reverse) { g_claim_reverse.store(reverse ? 1 : 0); }
+
+void moe_set_stage_events(void *const *events, int32_t n)
+{
+    std::lock_guard<std::mutex> lk(g_ev_mu);
+    g_stage_on = events != nullptr && n == MOE_STAGE_EVENTS;
+    for (int i = 0; i < MOE_STAGE_EVENTS; ++i)
+        g_stage_ev[i] = g_stage_on ? static_cast<cudaEvent_t>(events[i]) : nullptr;
+}
+
+moe_status_t moe_route(const moe_dims_t *d, const void *x, const void *router_w, const float *router_bias,
+                       int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status_t s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (d->T == 0) return MOE_OK;
+    if (!x || !router_w || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if ((s = check_ws(d, ws, ws_bytes)) != MOE_OK) return s;
+    const moe::WsLayout L = moe::ws_layout(*d);
+    return cuda_status(moe::launch_route(*d, static_cast<const __nv_bfloat16 *>(x),
+                                         static_cast<const __nv_bfloat16 *>(router_w), router_bias,
+                                         at<float>(ws, L.logits), topk_idx, topk_w,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_permute(const moe_dims_t *d, const int32_t *topk_idx, int32_t *expert_offsets,
+                         int32_t *sorted_to_flat, int32_t *flat_to_sorted, int32_t *tile_list,
+                         int32_t *num_tiles, void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status_t s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (d->T == 0) return MOE_OK;
+    if (!topk_idx || !expert_offsets || !sorted_to_flat || !flat_to_sorted || !tile_list || !num_tiles)
+        return MOE_ERR_INVALID_ARG;
+    if ((s = check_ws(d, ws, ws_bytes)) != MOE_OK) return s;
+    const moe::WsLayout L = moe::ws_layout(*d);
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(moe::launch_permute(*d, L, topk_idx, at<int32_t>(ws, L.blk_cnt),
+                                           at<int32_t>(ws, L.blk_base), expert_offsets, sorted_to_flat,
+                                           flat_to_sorted, tile_list, num_tiles, at<moe::WsHeader>(ws, 0),
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_w, const float *router_bias,
+                         const void *w_gate, const void *w_up, const void *w_down, void *out, void *ws,
+                         size_t ws_bytes, void *stream)
+{
+    moe_status_t s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (d->T == 0) return MOE_OK;
+    if (!x || !router_w || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+    if ((s = check_ws(d, ws, ws_bytes)) != MOE_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const moe::WsLayout L = moe::ws_layout(*d);
+    const int A = d->T * d->top_k;
+    auto *hdr = at<moe::WsHeader>(ws, 0);
+    auto *xs = at<__nv_bfloat16>(ws, L.xs);
+    auto *h = at<__nv_bfloat16>(ws, L.h);
+    auto *y = at<__nv_bfloat16>(ws, L.y);
+    auto *idx = at<int32_t>(ws, L.idx);
+    auto *gate = at<float>(ws, L.gate);
+    auto *s2f = at<int32_t>(ws, L.s2f);
+    auto *tiles = at<int32_t>(ws, L.tiles);
+    auto *ntiles = at<int32_t>(ws, L.ntiles);
+
+    CUtensorMap tm_xs, tm_wg, tm_wu, tm_h, tm_wd;
+    if (!encode_2d(&tm_xs, xs, A, d->H, moe::kTileRows) ||
+        !encode_3d(&tm_wg, w_gate, d->E, d->I, d->H, 128) ||
+        !encode_3d(&tm_wu, w_up, d->E, d->I, d->H, 128) ||
+        !encode_2d(&tm_h, h, A, d->I, moe::kTileRows) ||
+        !encode_3d(&tm_wd, w_down, d->E, d->H, d->I, 256))
+        return MOE_ERR_CUDA;
+
+    const StageMarks marks;
+    cudaError_t e = marks.mark(0, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(moe::WsHeader), st);
+    if (e == cudaSuccess)
+        e = moe::launch_route(*d, static_cast<const __nv_bfloat16 *>(x),
+                              static_cast<const __nv_bfloat16 *>(router_w), router_bias, at<float>(ws, L.logits),
+                              idx, gate, st);
+    if (e == cudaSuccess) e = marks.mark(1, st);
+    if (e == cudaSuccess)
+        e = moe::launch_permute(*d, L, idx, at<int32_t>(ws, L.blk_cnt), at<int32_t>(ws, L.blk_base),
+                                at<int32_t>(ws, L.offsets), s2f, at<int32_t>(ws, L.f2s), tiles, ntiles, hdr, st);
+    if (e == cudaSuccess)
+        e = moe::launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), s2f, A, d->H, d->top_k, xs, st);
+    if (e == cudaSuccess) e = marks.mark(2, st);
+    const int ctas = g_gemm_ctas.load(), rev = g_claim_reverse.load();
+    if (e == cudaSuccess) {
+        moe::GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, h, nullptr, ctas, rev};
+        e = moe::launch_grouped_gemm(g1, tm_xs, tm_wg, tm_wu, st);
+    }
+    if (e == cudaSuccess) e = marks.mark(3, st);
+    if (e == cudaSuccess) {
+        moe::GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, y, s2f, ctas, rev};
+        e = moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st);
+    }
+    if (e == cudaSuccess) e = marks.mark(4, st);
+    if (e == cudaSuccess)
+        e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st);
+    if (e == cudaSuccess) e = marks.mark(5, st);
+    return cuda_status(e);
+}
+
+moe_status_t moe_get_device_status(void *ws, void *stream)
+{
+    if (!ws) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    int32_t v = 0;
+    if (cudaMemcpy(&v, ws, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    const int32_t zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    return static_cast<moe_status_t>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// moe_internal.h -- workspace layout and kernel launchers shared by the library's
+// translation units (not part of the public ABI).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kTileRows = MOE_TILE_ROWS;  // BM of the grouped GEMMs
+constexpr int kMaxExperts = 1024;
+
+// Header at the start of every workspace.
+struct WsHeader {
+    int32_t status;       // device status word (moe_status_t), sticky until read
+    int32_t counter[7];   // work-claim counters of the persistent GEMMs
+};
+
+// Byte offsets of every region of the workspace (256-byte aligned each).
+struct WsLayout {
+    size_t logits, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xs, h, y, total;
+    int nb;      // permutation chunks
+    int chunk;   // flat entries per chunk
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Entries of the flat assignment list handled by one permutation chunk: the
+// scatter kernel keeps a [warps x E] table of per-warp counts in shared memory,
+// so wide expert counts use fewer warps.
+inline int perm_warps(int E)
+{
+    int w = 8192 / (E > 0 ? E : 1);
+    if (w > 32) w = 32;
+    if (w < 1) w = 1;
+    return w;
+}
+
+inline WsLayout ws_layout(const moe_dims_t &d)
+{
+    WsLayout L{};
+    const size_t A = static_cast<size_t>(d.T) * d.top_k;
+    const int warps = perm_warps(d.E);
+    L.chunk = 32 * warps;
+    L.nb = static_cast<int>((A + L.chunk - 1) / L.chunk);
+    const size_t max_tiles = (A + kTileRows - 1) / kTileRows + (A < (size_t)d.E ? A : (size_t)d.E);
+    size_t o = align_up(sizeof(WsHeader), 256);
+    auto take = [&](size_t bytes) {
+        size_t at = o;
+        o = align_up(o + bytes, 1024);
+        return at;
+    };
+    L.logits = take(static_cast<size_t>(d.T) * d.E * 4);
+    L.blk_cnt = take(static_cast<size_t>(L.nb > 0 ? L.nb : 1) * d.E * 4);
+    L.blk_base = take(static_cast<size_t>(L.nb > 0 ? L.nb : 1) * d.E * 4);
+    L.idx = take(A * 4);
+    L.gate = take(A * 4);
+    L.offsets = take(static_cast<size_t>(d.E + 1) * 4);
+    L.s2f = take(A * 4);
+    L.f2s = take(A * 4);
+    L.tiles = take(max_tiles * 3 * 4);
+    L.ntiles = take(4);
+    L.xs = take(A * d.H * 2);
+    L.h = take(A * d.I * 2);
+    L.y = take(A * d.H * 2);
+    L.total = o;
+    return L;
+}
+
+// ------------------------------------------------------------ launchers
+// Each returns cudaGetLastError() of its launch(es).
+
+cudaError_t launch_route(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
+                         const float *bias, float *logits, int32_t *idx, float *gate,
+                         cudaStream_t st);
+
+cudaError_t launch_permute(const moe_dims_t &d, const WsLayout &L, const int32_t *idx,
+                           int32_t *blk_cnt, int32_t *blk_base, int32_t *offsets, int32_t *s2f,
+                           int32_t *f2s, int32_t *tiles, int32_t *ntiles, WsHeader *hdr,
+                           cudaStream_t st);
+
+cudaError_t launch_gather_rows(const __nv_bfloat16 *x, const int32_t *s2f, int A, int H, int top_k,
+                               __nv_bfloat16 *xs, cudaStream_t st);
+
+cudaError_t launch_combine(const __nv_bfloat16 *y, const float *gate, int T, int H, int top_k,
+                           __nv_bfloat16 *out, cudaStream_t st);
+
+// Grouped GEMMs over the tile list.  mode 0: h = silu(A Wg^T) * (A Wu^T) (A = the
+// expert-sorted activations, B = gate/up weights); mode 1: y[s2f[row]] = A Wd^T
+// (A = h).  The tensor maps are encoded by the caller.
+struct GemmArgs {
+    int mode;
+    int K, N;
+    const int32_t *tiles;
+    const int32_t *ntiles;
+    int32_t *counter;
+    int32_t *status;
+    __nv_bfloat16 *out;
+    const int32_t *row_map;
+    int ctas;
+    int reverse;
+};
+cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
+                                const CUtensorMap &tmB1, cudaStream_t st);
+
+int num_sms();
+
+}  // namespace moe

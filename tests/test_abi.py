@@ -1,0 +1,70 @@
+"""The C-ABI library loads and exports every symbol include/moe.h declares; the host-side
+argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from routed_grouped_gemm_softmax_b200 import api, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return api.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 8, names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in moe.h but not exported"
+    assert sorted(names) == sorted(api.EXPORTS)
+
+
+def test_workspace_size_and_tiles(L):
+    for (T, H, I, E, k) in [(64, 256, 512, 8, 2), (16, 2048, 512, 256, 8), (4096, 2048, 512, 256, 8),
+                            (8192, 4096, 1408, 64, 6)]:
+        n = api.moe_workspace_size(T, H, I, E, k)
+        A = T * k
+        # at least the three activation-sized buffers plus the logits
+        assert n >= A * H * 2 * 2 + A * I * 2 + T * E * 4
+        assert n % 1024 == 0
+        assert api.moe_max_tiles(T, H, I, E, k) == (A + 127) // 128 + min(A, E)
+    assert api.moe_workspace_size(64, 100, 512, 8, 2) == 0   # H not a multiple of 64
+    assert api.moe_workspace_size(64, 256, 512, 8, 9) == 0   # top_k > E
+    assert api.moe_workspace_size(64, 256, 512, 2000, 2) == 0  # too many experts
+
+
+def test_host_argument_errors(L):
+    null = None
+    d = api.dims(4, 256, 512, 8, 2)
+    # missing inputs are rejected before any device work
+    assert L.moe_route(ctypes.byref(d), null, null, null, null, null, null, 0, null) == 1
+    assert L.moe_forward(ctypes.byref(d), null, null, null, null, null, null, null, null, 0, null) == 1
+    assert L.moe_permute(ctypes.byref(d), null, null, null, null, null, null, null, 0, null) == 1
+    bad = api.dims(4, 256, 512, 8, 0)
+    assert L.moe_route(ctypes.byref(bad), null, null, null, null, null, null, 0, null) == 1
+    wide = api.dims(4, 256, 512, 4096, 2)
+    assert L.moe_route(ctypes.byref(wide), null, null, null, null, null, null, 0, null) == 2
+    assert L.moe_route(None, null, null, null, null, null, null, 0, null) == 1
+    # T == 0 is a no-op
+    zero = api.dims(0, 256, 512, 8, 2)
+    assert L.moe_forward(ctypes.byref(zero), null, null, null, null, null, null, null, null, 0, null) == 0
+    # a workspace that is too small or misaligned
+    buf = ctypes.create_string_buffer(4096)
+    addr = (ctypes.addressof(buf) + 255) // 256 * 256
+    fake = ctypes.c_void_p(addr)
+    assert L.moe_route(ctypes.byref(d), fake, fake, null, fake, fake, fake, 16, null) == 3
+    assert L.moe_route(ctypes.byref(d), fake, fake, null, fake, fake, ctypes.c_void_p(addr + 8),
+                       1 << 30, null) == 3
+    assert L.moe_get_device_status(null, null) == 1

@@ -1,0 +1,206 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Routing (expert indices), the permutation, the group offsets and the tile list
+must match bit for bit; gates to a relative 1e-5; the layer output (bf16) to
+max-abs <= 2e-2 and relative L2 <= 5e-3 against the fp64 oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import (compare_out, compare_permute, compare_routing, device_inputs,
+                         sample_tokens)
+from routed_grouped_gemm_softmax_b200 import api
+from routed_grouped_gemm_softmax_b200.inputs import CONFIGS
+
+pytestmark = pytest.mark.gpu
+
+# Small-to-mid shapes that the oracle finishes in seconds, spanning several tiles
+# and ragged tails in rows (groups not a multiple of 128) and columns (I = 64 mod 128).
+SMALL = {
+    "tiny": CONFIGS["tiny"],
+    "ragged": CONFIGS["tiny"].replace(name="ragged", T=300, H=512, E=16, top_k=4, I=192, seed=11),
+    "ragged_bias": CONFIGS["tiny"].replace(name="ragged_bias", T=517, H=320, E=12, top_k=3, I=320,
+                                           seed=12, zipf_s=1.2),
+    "one_token": CONFIGS["tiny"].replace(name="one_token", T=1, H=256, E=8, top_k=2, seed=13),
+    "top1": CONFIGS["tiny"].replace(name="top1", T=200, top_k=1, seed=14),
+    "topk_all": CONFIGS["tiny"].replace(name="topk_all", T=96, top_k=8, seed=15),
+    "wide_e": CONFIGS["tiny"].replace(name="wide_e", T=40, H=256, E=300, top_k=5, I=128, seed=16),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib_and_defaults():
+    api.lib()
+    api.set_gemm_ctas(0)
+    api.set_claim_order(False)
+    yield
+    api.set_gemm_ctas(0)
+    api.set_claim_order(False)
+
+
+def _full_layer_check(cfg, zero_router=False):
+    g, c = device_inputs(cfg, zero_router)
+    k = cfg.top_k
+    idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], k)
+    idx, w = api.moe_route(g["x"], g["router_w"], g["bias"], k)
+    compare_routing(idx, w, idx_ref, gate_ref, cfg.name)
+    perm_ref = oracle.permute(idx_ref, cfg.E)
+    compare_permute(api.moe_permute(idx, cfg.E), perm_ref, cfg.name)
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, "cuda")
+    out = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k, ws=ws)
+    assert api.moe_get_device_status(ws) == api.MOE_OK
+    ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"])
+    return compare_out(out, ref, cfg.name)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_small(name):
+    _full_layer_check(SMALL[name])
+
+
+def test_uniform_router_all_to_first_experts():
+    # router_w = 0: every logit ties, so every token picks experts 0..k-1 (lower index
+    # wins) with gates 1/k -- k groups of T rows (several tiles each), the rest empty.
+    cfg = CONFIGS["tiny"].replace(name="ties", T=300, top_k=3, seed=21)
+    _full_layer_check(cfg, zero_router=True)
+
+
+def test_one_hot_expert_takes_everything():
+    # A huge bias on one expert routes every token's first choice there (one group of
+    # T rows = many m-tiles on one expert; the claim queue spreads them over all SMs).
+    cfg = CONFIGS["tiny"].replace(name="hot", T=700, top_k=2, seed=22)
+    g, c = device_inputs(cfg)
+    bias = torch.zeros(cfg.E, dtype=torch.float32)
+    bias[3] = 1000.0
+    g["bias"], c["bias"] = bias.cuda(), bias
+    idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], bias, 2)
+    assert np.all(idx_ref[:, 0] == 3)
+    out = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], 2)
+    ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"])
+    compare_out(out, ref, "hot")
+
+
+def test_group_sizes_at_tile_edges():
+    # Groups of exactly 128 rows (one full tile), 129 rows (a full tile plus one row)
+    # and 5 rows.  Router rows 0 and 1 give logit(e) = x0*e - x1*e^2, which with
+    # x1 = 1 peaks exactly at e = x0/2, so x0 chooses each token's expert.
+    cfg = CONFIGS["tiny"].replace(name="edges", T=128 + 129 + 5, top_k=1, seed=23)
+    g, c = device_inputs(cfg)
+    x = c["x"].clone()
+    rw = torch.zeros_like(c["router_w"])
+    e = torch.arange(8, dtype=torch.float32)
+    rw[0, :] = e.to(torch.bfloat16)
+    rw[1, :] = (-e * e).to(torch.bfloat16)
+    x[:, 1] = 1.0
+    x[:128, 0] = 0.0      # expert 0
+    x[128:257, 0] = 14.0  # expert 7
+    x[257:, 0] = 6.0      # expert 3
+    g["x"], c["x"] = x.cuda(), x
+    g["router_w"], c["router_w"] = rw.cuda(), rw
+    idx_ref, gate_ref = oracle.route(x, rw, None, 1)
+    counts = np.bincount(idx_ref[:, 0], minlength=8)
+    assert counts[0] == 128 and counts[7] == 129 and counts[3] == 5
+    perm_ref = oracle.permute(idx_ref, 8)
+    idx, w = api.moe_route(g["x"], g["router_w"], None, 1)
+    compare_routing(idx, w, idx_ref, gate_ref, "edges")
+    compare_permute(api.moe_permute(idx, 8), perm_ref, "edges")
+    out = api.moe_forward(g["x"], g["router_w"], None, g["w_gate"], g["w_up"], g["w_down"], 1)
+    ref = oracle.combine_ffn(x, idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"])
+    compare_out(out, ref, "edges")
+
+
+def test_schedule_independence():
+    # The result is bitwise the same whatever the number of persistent CTAs and the
+    # order in which they claim items: sums are ordered by the tile, not the schedule.
+    cfg = CONFIGS["tiny"].replace(name="sched", T=640, H=512, E=16, top_k=4, I=384, seed=24)
+    g, _ = device_inputs(cfg)
+    outs = []
+    try:
+        for ctas, rev in [(0, False), (1, False), (7, True), (148, False), (0, True), (3, True)]:
+            api.set_gemm_ctas(ctas)
+            api.set_claim_order(rev)
+            outs.append(api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"],
+                                        g["w_down"], cfg.top_k).clone())
+    finally:
+        api.set_gemm_ctas(0)
+        api.set_claim_order(False)
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
+def test_repeat_calls_same_workspace():
+    # Counters and status are reset by the calls themselves: back-to-back calls on one
+    # workspace give identical results (graph-replay style reuse).
+    cfg = SMALL["ragged"]
+    g, _ = device_inputs(cfg)
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k, "cuda")
+    a = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k, ws=ws).clone()
+    b = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k, ws=ws)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert api.moe_get_device_status(ws) == api.MOE_OK
+
+
+def test_cuda_graph_replay():
+    cfg = SMALL["ragged"]
+    g, c = device_inputs(cfg)
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k, "cuda")
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k,
+                        out=out, ws=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k,
+                        out=out, ws=ws)
+    out.zero_()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], cfg.top_k)
+    ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"])
+    compare_out(out, ref, "graph")
+    del graph
+
+
+def test_bad_expert_index_flagged():
+    idx = torch.tensor([[0, 1], [5, 9]], dtype=torch.int32, device="cuda")  # 9 >= E=8
+    ws = api.workspace(2, 256, 64, 8, 2, "cuda")
+    api.moe_permute(idx, 8, ws=ws)
+    assert api.moe_get_device_status(ws) == 6  # MOE_ERR_BAD_INDEX
+    assert api.moe_get_device_status(ws) == api.MOE_OK  # cleared by the read
+
+
+def test_empty_batch_is_noop():
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    rw = torch.zeros(256, 8, dtype=torch.bfloat16, device="cuda")
+    wg = torch.zeros(8, 64, 256, dtype=torch.bfloat16, device="cuda")
+    wd = torch.zeros(8, 256, 64, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    out = api.moe_forward(x, rw, None, wg, wg, wd, 2, ws=ws)
+    assert out.shape == (0, 256)
+
+
+# ------------------------------------------------------------- full-size configs
+
+@pytest.mark.parametrize("name", ["decode", "prefill", "skewed"])
+def test_full_size(name):
+    """Full-size workloads: routing, permutation and offsets bit-exact for every token;
+    the layer output checked on a sample of tokens the oracle evaluates one by one."""
+    cfg = CONFIGS[name]
+    g, c = device_inputs(cfg)
+    k = cfg.top_k
+    idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], k)
+    idx, w = api.moe_route(g["x"], g["router_w"], g["bias"], k)
+    compare_routing(idx, w, idx_ref, gate_ref, name)
+    compare_permute(api.moe_permute(idx, cfg.E), oracle.permute(idx_ref, cfg.E), name)
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, "cuda")
+    out = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k, ws=ws)
+    assert api.moe_get_device_status(ws) == api.MOE_OK
+    tok = sample_tokens(cfg.T, 24, seed=cfg.seed)
+    ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"], tokens=tok)
+    compare_out(out[torch.as_tensor(tok, device="cuda").long()], ref, name)
