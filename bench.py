@@ -1,0 +1,445 @@
+"""Benchmark of the MoE layer forward on B200: tokens/s of whole layer steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|tiny]
+                    [--impl ours|reference]
+
+One step = one pass of the whole layer (router softmax top-k, permute, grouped
+gate/up GEMM + SwiGLU, grouped down GEMM, combine) over one batch of seeded
+synthetic inputs already resident in HBM.  L2 is flushed (a 512 MiB write)
+before every step, outside that step's CUDA-event pair.  Prints one JSON line.
+
+Multi-GPU: the layer does not shard on one node in this design, so N GPUs run N
+independent replicas (one process per GPU, launched by torchrun); the time is the
+max over ranks and ``value`` counts the tokens of all ranks.
+
+``--impl reference`` times the CPU oracle (the only reference there is) on the
+host cores, rank 0 only, each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime as _dt
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at 1 B200; % of BF16/FP8 TC peak or % of HBM BW"
+KERNELS_PER_FORWARD = 9   # logits, top-k, count, scan, scatter, gather, GEMM x2, combine
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 512 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="decode", choices=sorted(CONFIGS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sources_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "routed_grouped_gemm_softmax_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, stage: str):
+    """DRAM bytes per launch of `stage` from the committed ncu capture summary, or None
+    when there is none or the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    rec = d.get(workload, {}).get(stage)
+    if not rec or rec.get("sources") != kernel_sources_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms in the background."""
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.lines = []
+        try:
+            p = torch.cuda.get_device_properties(device)
+            target = ["-i", f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"]
+        except Exception:
+            target = []
+        self.cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                    "-lms", "50", *target]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self, t0: float, t1: float):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                ts = _dt.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            if not (t0 - 0.05 <= ts <= t1 + 0.05):
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------- per-stage bytes
+
+def stage_work(cfg, counts):
+    """Algorithmic bytes and FLOPs of each stage for the realised routing (counts[e] =
+    rows of expert e).  Intermediates a fused design would not write are excluded only
+    where the stage's own definition does not need them."""
+    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k
+    A = T * k
+    D = int(sum(1 for c in counts if c > 0))
+    return {
+        "route": {"bytes": T * H * 2 + H * E * 2 + A * 8, "flops": 2.0 * T * H * E, "alu": True},
+        "gemm_gate_up": {"bytes": D * 2 * I * H * 2 + A * H * 2 + A * I * 2, "flops": 2.0 * A * H * 2 * I},
+        "gemm_down": {"bytes": D * H * I * 2 + A * I * 2 + A * H * 2, "flops": 2.0 * A * I * H},
+        "combine": {"bytes": A * H * 2 + A * 4 + T * H * 2, "flops": 2.0 * A * H},
+        "_D": D,
+    }
+
+
+def roofline_for(stage, work, ms, peaks, peaks_kind, sustained, workload):
+    w = work[stage]
+    t = ms * 1e-3
+    bw_time = w["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    pk_tf = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    tc_time = w["flops"] / (pk_tf * 1e12)
+    if w.get("alu") or bw_time >= tc_time:
+        achieved = w["bytes"] / t / 1e9
+        r = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = w["flops"] / t / 1e12
+        r = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk_tf, "unit": "TFLOP/s"}
+    r["frac"] = round(achieved / r["peak"], 4)
+    r["traffic"] = recorded_traffic(workload, stage)
+    r["kernel"] = stage
+    r["algorithmic_bytes"] = w["bytes"]
+    r["algorithmic_flops"] = w["flops"]
+    r["peak_source"] = f"{peaks_kind}" + ("" if r["bound"] == "hbm" else (" sustained" if sustained else " burst"))
+    r["ms"] = round(ms, 4)
+    return r
+
+
+# ------------------------------------------------------------- CPU oracle leg
+
+def host_inputs(cfg, inp=None):
+    """The workload's tensors as host numpy arrays (bf16 bit patterns), drawn on the GPU
+    when one is present (data preparation only; nothing of the layer runs there)."""
+    import types
+
+    import numpy as np
+    if inp is None:
+        inp = make_inputs(cfg, device="cuda" if torch.cuda.is_available() else "cpu")
+
+    def bits(t):
+        return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    return types.SimpleNamespace(
+        x=bits(inp.x), router_w=bits(inp.router_w),
+        bias=None if inp.bias is None else inp.bias.detach().cpu().float().numpy(),
+        w_gate=bits(inp.w_gate), w_up=bits(inp.w_up), w_down=bits(inp.w_down))
+
+
+def oracle_step_timer(cfg, h):
+    """Returns f(n) -> (route seconds, FFN seconds) for one oracle pass: the routing of
+    all T tokens plus the expert FFN/combine of n sampled tokens; and the threads used."""
+    import numpy as np
+
+    import oracle
+    threads = oracle.default_threads()
+    rng = np.random.default_rng(cfg.seed)
+
+    def run(n):
+        t0 = time.perf_counter()
+        idx, gate = oracle.route(h.x, h.router_w, h.bias, cfg.top_k, nthreads=threads)
+        t1 = time.perf_counter()
+        tok = np.sort(rng.choice(cfg.T, size=n, replace=False)).astype(np.int32)
+        oracle.combine_ffn(h.x, idx, gate, h.w_gate, h.w_up, h.w_down, tokens=tok, nthreads=threads)
+        t2 = time.perf_counter()
+        return t1 - t0, t2 - t1
+    return run, threads
+
+
+def cpu_baseline(cfg, h, budget_s=20.0):
+    run, threads = oracle_step_timer(cfg, h)
+    n = min(cfg.T, max(threads, 1))
+    tr, tf = run(n)
+    per_tok = tf / n
+    # layer tokens/s estimate: routing all T tokens + FFN of all T at the measured per-token rate
+    n_tot, t_route, t_ffn, reps = 0, 0.0, 0.0, 0
+    t_start = time.perf_counter()
+    while time.perf_counter() - t_start < budget_s:
+        m = min(cfg.T, max(n, int(max(1.0, budget_s / 4) / max(per_tok, 1e-9))))
+        a, b = run(m)
+        t_route += a
+        t_ffn += b
+        n_tot += m
+        reps += 1
+    est = cfg.T / (t_route / reps + (t_ffn / n_tot) * cfg.T)
+    return {"value": round(est, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{reps} passes of: router+top-k over all {cfg.T} tokens, expert FFN + "
+                      f"combine of {n_tot // reps} sampled tokens (fp64 CPU oracle); "
+                      f"tokens/s = T / (route time + per-token FFN time * T)"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    cfg = CONFIGS[args.workload]
+    run, threads = oracle_step_timer(cfg, host_inputs(cfg))
+    tr, tf = run(min(cfg.T, threads))
+    per_tok = tf / min(cfg.T, threads)
+    budget = 150.0 / max(args.steps + args.warmup, 1)
+    n = int(min(cfg.T, max(1, (budget - tr) / max(per_tok, 1e-9))))
+    for _ in range(args.warmup):
+        run(n)
+    tot_r = tot_f = 0.0
+    for _ in range(args.steps):
+        a, b = run(n)
+        tot_r += a
+        tot_f += b
+    step_s = tot_r / args.steps + tot_f / args.steps * cfg.T / n
+    value = cfg.T / step_s
+    sample = (f"each step: router+top-k over all {cfg.T} tokens + expert FFN/combine of {n} sampled "
+              f"tokens, scaled to the full batch (fp64 CPU oracle, {threads} threads)")
+    line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": config_block(cfg, world),
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_block(cfg, world):
+    return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.top_k,
+            "seed": cfg.seed, "router_bias": "zipf(1.2)" if cfg.zipf_s else None,
+            "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
+            "l2": "flushed before every step (512 MiB write, outside the step's events)",
+            "launch": "one moe_forward call per step on one stream"}
+
+
+# ---------------------------------------------------------------- our arm
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        barrier(world)
+        return
+    from routed_grouped_gemm_softmax_b200 import api
+
+    cfg = CONFIGS[args.workload]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    inp = make_inputs(cfg, device=dev)
+    x, rw, bias = inp.x, inp.router_w, inp.bias
+    wg, wu, wd = inp.w_gate, inp.w_up, inp.w_down
+    k = cfg.top_k
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, dev)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        api.moe_forward(x, rw, bias, wg, wu, wd, k, out=out, ws=ws, stream=stream)
+
+    # events: one set of 6 stage marks per timed step (the first and last bracket the step)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for s in ev:
+        for e in s:
+            e.record(stream)
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    status = api.moe_get_device_status(ws)
+    if status != api.MOE_OK:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.2)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(1)
+        api.set_stage_events(ev[i])
+        step()
+    api.set_stage_events(None)
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall1 = time.time()
+    time.sleep(0.1)
+    sampler.stop()
+    status = api.moe_get_device_status(ws)
+    if status != api.MOE_OK:
+        raise RuntimeError(f"device status {status} after the timed steps")
+
+    step_ms = [ev[i][0].elapsed_time(ev[i][5]) for i in range(args.steps)]
+    stage_ms = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
+                for j, name in enumerate(api.STAGES)}
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    value = cfg.T * world * args.steps / (total_ms * 1e-3)
+
+    # routing of this workload (for the touched-expert weight bytes)
+    idx, _ = api.moe_route(x, rw, bias, k)
+    counts = torch.bincount(idx.view(-1).long(), minlength=cfg.E).tolist()
+    work = stage_work(cfg, counts)
+    peaks, peaks_kind = load_peaks()
+    dominant = max(("route", "gemm_gate_up", "gemm_down", "combine"), key=lambda s: stage_ms[s])
+    sustained = total_ms > 1000.0
+    roof = roofline_for(dominant, work, stage_ms[dominant], peaks, peaks_kind, sustained, cfg.name)
+    stages = {s: {"ms": round(stage_ms[s], 4)} for s in api.STAGES}
+    for s in ("route", "gemm_gate_up", "gemm_down", "combine"):
+        r = roofline_for(s, work, stage_ms[s], peaks, peaks_kind, sustained, cfg.name)
+        stages[s].update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_host = x.cpu().pin_memory()
+        out_host = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty_like(x)
+        n_e2e = max(1, min(args.steps, 200))
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(n_e2e)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for a, b in pairs:
+            flush.fill_(1)
+            a.record(stream)
+            x_dev.copy_(x_host, non_blocking=True)
+            api.moe_forward(x_dev, rw, bias, wg, wu, wd, k, out=out, ws=ws, stream=stream)
+            out_host.copy_(out, non_blocking=True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in pairs), world) / n_e2e
+        e2e = {"value": round(cfg.T * world / (e2e_ms * 1e-3), 3), "unit": "tokens/s",
+               "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
+               "ms_per_step": round(e2e_ms, 4)}
+
+    clocks = sampler.summary(t_wall0, t_wall1)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, host_inputs(cfg, inp))
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": config_block(cfg, world),
+                "roofline": roof, "stages": stages, "experts_touched": work["_D"],
+                "e2e": e2e, "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+                "clocks": clocks, "cpu_baseline": cpu,
+                "p99_ms_per_step": round(sorted(step_ms)[min(len(step_ms) - 1, math.ceil(0.99 * len(step_ms)) - 1)], 5)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
