@@ -65,7 +65,8 @@ typedef enum {
     MOE_ERR_WORKSPACE = 3,
     MOE_ERR_CUDA = 4,
     MOE_ERR_TIMEOUT = 5,     /* device: a pipeline wait ran past its limit */
-    MOE_ERR_BAD_INDEX = 6    /* device: an expert index outside [0, E) */
+    MOE_ERR_BAD_INDEX = 6,   /* device: an expert index outside [0, E) */
+    MOE_ERR_TOO_LARGE = 7    /* moe_forward_noalloc: dims need more than its fixed scratch */
 } moe_status_t;
 
 typedef struct {
@@ -146,6 +147,28 @@ void moe_set_claim_order(int32_t reverse);
  * NULL (or n != MOE_STAGE_EVENTS) turns recording off.  Process-wide. */
 #define MOE_STAGE_EVENTS 6
 void moe_set_stage_events(void *const *events, int32_t n);
+
+/* The layer forward for callers that cannot allocate device memory (the pages
+ * have no counterpart; this is a deployment convenience of this library).
+ * Same arguments and result as moe_forward minus the workspace: the scratch is
+ * a fixed array of MOE_NOALLOC_SCRATCH_BYTES inside the library's device image,
+ * present on every GPU that loads the library until the process exits.  It
+ * suits callers whose device memory belongs to an allocator they cannot reach,
+ * or that must never allocate on their serving path.
+ *  - Dims whose moe_workspace_size exceeds the array are rejected with
+ *    MOE_ERR_TOO_LARGE (with H=2048, I=512, E=256, top_k=8 that is above
+ *    about 220 tokens); invalid dims give the same errors as moe_forward.
+ *  - The first call made with a device current looks up the array's device
+ *    address on that device; make that first call before any stream capture.
+ *  - Nothing is allocated, freed or synchronised.  Every call shares the one
+ *    array and leaves its contents behind; the parts that must start at zero
+ *    are cleared by each call.  Calls whose GPU work overlaps (other streams,
+ *    unordered host threads) race on the array: serialise them.
+ *  - Device-side status (timeouts) is kept in the array and not reported. */
+#define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
+moe_status_t moe_forward_noalloc(const moe_dims_t *d, const void *x, const void *router_w,
+                                 const float *router_bias, const void *w_gate, const void *w_up,
+                                 const void *w_down, void *out, void *stream);
 
 #ifdef __cplusplus
 }

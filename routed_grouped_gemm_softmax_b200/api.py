@@ -17,10 +17,11 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT",
-                6: "MOE_ERR_BAD_INDEX"}
+                6: "MOE_ERR_BAD_INDEX", 7: "MOE_ERR_TOO_LARGE"}
 EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "moe_forward",
            "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order",
-           "moe_set_stage_events"]
+           "moe_set_stage_events", "moe_forward_noalloc"]
+NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
 TILE_ROWS = 128
 
@@ -66,6 +67,8 @@ def lib():
         L.moe_set_claim_order.restype = None
         L.moe_set_stage_events.argtypes = [P, I32]
         L.moe_set_stage_events.restype = None
+        L.moe_forward_noalloc.argtypes = [D, P, P, P, P, P, P, P, P]
+        L.moe_forward_noalloc.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -169,6 +172,31 @@ def moe_forward(x, router_w, bias, w_gate, w_up, w_down, top_k: int, out=None, w
     _check(lib().moe_forward(ctypes.byref(d), _p(x), _p(router_w), _p(bias), _p(w_gate), _p(w_up),
                              _p(w_down), _p(out), _p(ws), ws.numel(), _stream(stream, dev)),
            "moe_forward")
+    return out
+
+
+def moe_forward_noalloc(x, router_w, bias, w_gate, w_up, w_down, top_k: int, out=None, stream=None):
+    """The layer forward without a workspace argument, for callers that cannot allocate
+    device memory: the library's fixed internal scratch is used instead (dims that need
+    more than NOALLOC_SCRATCH_BYTES raise MOE_ERR_TOO_LARGE).  Calls that overlap on
+    the GPU share that scratch and race; ``out`` is the only buffer this binding may
+    allocate, and only when the caller passes none."""
+    T, H = x.shape
+    E, I, _ = w_gate.shape
+    dev = x.device
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(router_w, torch.bfloat16, (H, E), "router_w")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "router_bias")
+    _need(w_gate, torch.bfloat16, (E, I, H), "w_gate")
+    _need(w_up, torch.bfloat16, (E, I, H), "w_up")
+    _need(w_down, torch.bfloat16, (E, H, I), "w_down")
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    _need(out, torch.bfloat16, (T, H), "out")
+    d = dims(T, H, I, E, top_k)
+    _check(lib().moe_forward_noalloc(ctypes.byref(d), _p(x), _p(router_w), _p(bias), _p(w_gate),
+                                     _p(w_up), _p(w_down), _p(out), _stream(stream, dev)),
+           "moe_forward_noalloc")
     return out
 
 

@@ -1,0 +1,64 @@
+"""The forward entry point for callers that cannot allocate device memory.
+
+moe_forward_noalloc runs the layer with the library's fixed internal scratch
+instead of a caller-provided workspace -- for code that has no access to an
+allocator on its serving path.  Its results must match the regular
+moe_forward (which takes a workspace) on the same inputs, call after call.
+This file is named so that pytest collects it last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import compare_out, device_inputs
+from routed_grouped_gemm_softmax_b200 import api
+from routed_grouped_gemm_softmax_b200.inputs import CONFIGS
+
+pytestmark = pytest.mark.gpu
+
+
+def _call_noalloc(g, k, out):
+    """Straight through the C ABI, with the device pointers only."""
+    T, H = g["x"].shape
+    E, I, _ = g["w_gate"].shape
+    d = api.dims(T, H, I, E, k)
+    p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return api.lib().moe_forward_noalloc(ctypes.byref(d), p(g["x"]), p(g["router_w"]), p(g["bias"]),
+                                         p(g["w_gate"]), p(g["w_up"]), p(g["w_down"]), p(out), st)
+
+
+@pytest.mark.parametrize("name", ["decode", "tiny"])
+def test_noalloc_matches_workspace_forward_twice(name):
+    cfg = CONFIGS[name]
+    g, c = device_inputs(cfg)
+    k = cfg.top_k
+    ref = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k)
+    torch.cuda.synchronize()
+    ref_f64 = ref.float().cpu().double().numpy()
+    for call in range(2):
+        out = torch.full_like(ref, float("nan"))
+        assert _call_noalloc(g, k, out) == api.MOE_OK
+        torch.cuda.synchronize()
+        compare_out(out, ref_f64, f"{name} no-alloc call {call} vs moe_forward")
+    # and both against the oracle on a few tokens
+    idx, gate = oracle.route(c["x"], c["router_w"], c["bias"], k)
+    tok = [0, cfg.T // 2, cfg.T - 1]
+    o = oracle.combine_ffn(c["x"], idx, gate, c["w_gate"], c["w_up"], c["w_down"], tokens=tok)
+    compare_out(out[tok], o, f"{name} no-alloc vs oracle")
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    # with H=2048, I=512, E=256, k=8 the fixed scratch holds up to 223 tokens
+    T, H, I, E, k = 224, 2048, 512, 256, 8
+    assert api.moe_workspace_size(T, H, I, E, k) > api.NOALLOC_SCRATCH_BYTES
+    assert api.moe_workspace_size(T - 1, H, I, E, k) <= api.NOALLOC_SCRATCH_BYTES
+    d = api.dims(T, H, I, E, k)
+    dummy = torch.empty(16, dtype=torch.bfloat16, device="cuda")
+    p = ctypes.c_void_p(dummy.data_ptr())
+    rc = api.lib().moe_forward_noalloc(ctypes.byref(d), p, p, None, p, p, p, p, None)
+    assert rc == 7  # MOE_ERR_TOO_LARGE, before any device work
+    bad = api.dims(16, 2048, 512, 256, 0)
+    assert api.lib().moe_forward_noalloc(ctypes.byref(bad), p, p, None, p, p, p, p, None) == 1
