@@ -51,7 +51,20 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--shape", default="",
+                   help="override config fields, e.g. T=1024,E=64 (reduced cases for profiler captures)")
     return p.parse_args()
+
+
+def workload_config(args):
+    cfg = CONFIGS[args.workload]
+    if args.shape:
+        kw = {}
+        for item in args.shape.split(","):
+            key, val = item.split("=")
+            kw[key.strip()] = int(val)
+        cfg = cfg.replace(name=f"{cfg.name}[{args.shape}]", **kw)
+    return cfg
 
 
 # ------------------------------------------------------------------ helpers
@@ -66,10 +79,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_sources_hash() -> str:
+STAGE_SOURCES = {
+    "route": ["route.cu"],
+    "gemm_gate_up": ["grouped_gemm.cu", "sm100_ptx.cuh", "moe_internal.h"],
+    "gemm_down": ["grouped_gemm.cu", "sm100_ptx.cuh", "moe_internal.h"],
+    "combine": ["combine.cu"],
+}
+
+
+def kernel_sources_hash(stage: str) -> str:
+    """Hash of the CUDA sources a stage's kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "routed_grouped_gemm_softmax_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in STAGE_SOURCES.get(stage, sorted(os.listdir(csrc))):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -85,7 +107,7 @@ def recorded_traffic(workload: str, stage: str):
     except (OSError, ValueError):
         return None
     rec = d.get(workload, {}).get(stage)
-    if not rec or rec.get("sources") != kernel_sources_hash():
+    if not rec or rec.get("sources") != kernel_sources_hash(stage):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -281,7 +303,7 @@ def cpu_baseline(cfg, h, budget_s=20.0):
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    cfg = CONFIGS[args.workload]
+    cfg = workload_config(args)
     run, threads = oracle_step_timer(cfg, host_inputs(cfg))
     tr, tf = run(min(cfg.T, threads))
     per_tok = tf / min(cfg.T, threads)
@@ -329,7 +351,7 @@ def main():
         return
     from routed_grouped_gemm_softmax_b200 import api
 
-    cfg = CONFIGS[args.workload]
+    cfg = workload_config(args)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     inp = make_inputs(cfg, device=dev)

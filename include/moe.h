@@ -36,7 +36,8 @@
  *    The flat assignment index of (t, j) is f = t*top_k + j.
  *  - Host-detectable errors return at once and enqueue nothing:
  *      MOE_ERR_INVALID_ARG  NULL dims or required pointer, T < 0, H/I/E <= 0,
- *                           top_k < 1 or > E, H or I not a multiple of 64
+ *                           top_k < 1 or > E, H or I not a multiple of 64,
+ *                           x, router_w, the expert weights or out not 16-byte aligned
  *      MOE_ERR_UNSUPPORTED  E > 1024
  *      MOE_ERR_WORKSPACE    ws NULL/misaligned (256 B) or ws_bytes too small
  *      MOE_ERR_CUDA         a launch failed (cudaGetLastError)
@@ -138,6 +139,16 @@ void moe_set_gemm_ctas(int32_t ctas);
 /* Order in which the GEMM CTAs claim work items: 0 = ascending (default),
  * 1 = descending.  Results are bitwise independent of it.  Process-wide. */
 void moe_set_claim_order(int32_t reverse);
+
+/* Failure-detection test hook.  Every wait inside the grouped GEMM pipelines
+ * is bounded; `us` sets that bound in microseconds (<= 0: the default, 2 s).
+ * With `stall_test` nonzero, the MMA thread of every GEMM CTA first waits on a
+ * barrier that nothing ever signals, so its wait -- and then the waits of the
+ * other roles -- run out.  A wait that runs out makes the kernel record
+ * MOE_ERR_TIMEOUT in the workspace status word and unwind (its own TMA copies
+ * and MMAs are drained under the default bound before TMEM is freed), so the
+ * context stays usable.  Process-wide; for tests only. */
+void moe_set_wait_limit_us(int32_t us, int32_t stall_test);
 
 /* Stage timing hook for benchmarks.  With `events` pointing at MOE_STAGE_EVENTS
  * caller-created cudaEvent_t handles (passed as void*), every later moe_forward

@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 6: "MOE_ERR_BAD_INDEX", 7: "MOE_ERR_TOO_LARGE"}
 EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "moe_forward",
            "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order",
-           "moe_set_stage_events", "moe_forward_noalloc"]
+           "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us"]
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
 TILE_ROWS = 128
@@ -67,6 +67,8 @@ def lib():
         L.moe_set_claim_order.restype = None
         L.moe_set_stage_events.argtypes = [P, I32]
         L.moe_set_stage_events.restype = None
+        L.moe_set_wait_limit_us.argtypes = [I32, I32]
+        L.moe_set_wait_limit_us.restype = None
         L.moe_forward_noalloc.argtypes = [D, P, P, P, P, P, P, P, P]
         L.moe_forward_noalloc.restype = ctypes.c_int
         _lib = L
@@ -207,6 +209,12 @@ def moe_get_device_status(ws, stream=None) -> int:
 
 def set_gemm_ctas(n: int):
     lib().moe_set_gemm_ctas(int(n))
+
+
+def set_wait_limit_us(us: int, stall_test: bool = False):
+    """Limit of each GEMM pipeline wait in microseconds (<= 0 restores the 2 s default);
+    ``stall_test`` makes every GEMM CTA wait on a barrier nothing signals (tests only)."""
+    lib().moe_set_wait_limit_us(int(us), 1 if stall_test else 0)
 
 
 def set_claim_order(reverse: bool):

@@ -30,9 +30,10 @@
 //                   rows past the group's end masked.
 // Every accumulation order is fixed by the tile and the K loop, never by which
 // CTA ran the item, so results are bitwise independent of the schedule.
-// Every wait is bounded; a wait that runs out records MOE_ERR_TIMEOUT in the
-// workspace status word and the CTA unwinds (waiting, again bounded, for its
-// own TMA copies and MMAs) before freeing TMEM.
+// Every wait is bounded (GemmArgs::wait_ns); a wait that runs out records
+// MOE_ERR_TIMEOUT in the workspace status word and the CTA unwinds -- waiting,
+// with the fixed default bound, for its own TMA copies and MMAs -- before
+// freeing TMEM.
 #include "moe_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -57,6 +58,7 @@ struct Ctrl {
     uint64_t itf[RING];      // ring slot r holds the next item id
     uint64_t ite[RING];      // every role has read ring slot r
     uint64_t fin;            // all MMAs of this CTA are done
+    uint64_t never;          // nothing ever arrives here (timeout test)
     int32_t ring[RING];
     uint32_t tmem_base;
 };
@@ -104,6 +106,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             mbar_init(&S->ite[r], 5);  // the MMA thread + 4 epilogue warps
         }
         mbar_init(&S->fin, 1);
+        mbar_init(&S->never, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB0);
@@ -129,7 +132,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     item = -1;
                 else if (g.reverse)
                     item = total - 1 - item;
-                if (!mbar_wait(&S->ite[rs], rphase ^ 1)) { ok = false; break; }
+                if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
                 S->ring[rs] = item;
                 mbar_arrive(&S->itf[rs]);
                 if (++rs == RING) { rs = 0; rphase ^= 1; }
@@ -138,7 +141,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const int expert = g.tiles[3 * mt], row0 = g.tiles[3 * mt + 1];
                 const int n0 = nt * BNO;
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(&S->empty[stage], phase ^ 1)) { ok = false; break; }
+                    if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
                     mbar_arrive_expect_tx(&S->full[stage], A_BYTES + B_BYTES);
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -170,18 +173,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
             int stage = 0, rs = 0, acc = 0;
             uint32_t phase = 0, rphase = 0, aphase = 0;
-            bool ok = true;
-            for (;;) {
-                if (!mbar_wait(&S->itf[rs], rphase)) { ok = false; break; }
+            // timeout test: wait (bounded) on a barrier nothing signals, then unwind
+            bool ok = !(g.stall_test && !mbar_wait(&S->never, 0, g.wait_ns));
+            while (ok) {
+                if (!mbar_wait(&S->itf[rs], rphase, g.wait_ns)) { ok = false; break; }
                 const int item = S->ring[rs];
                 mbar_arrive(&S->ite[rs]);
                 if (++rs == RING) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
-                if (!mbar_wait(&S->acce[acc], aphase ^ 1)) { ok = false; break; }
+                if (!mbar_wait(&S->acce[acc], aphase ^ 1, g.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(&S->full[stage], phase)) { ok = false; break; }
+                    if (!mbar_wait(&S->full[stage], phase, g.wait_ns)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
                     const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
@@ -209,7 +213,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         int rs = 0, acc = 0;
         uint32_t rphase = 0, aphase = 0;
         for (;;) {
-            if (!mbar_wait(&S->itf[rs], rphase)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
+            if (!mbar_wait(&S->itf[rs], rphase, g.wait_ns)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
             const int item = S->ring[rs];
             __syncwarp();
             if (lane == 0) mbar_arrive(&S->ite[rs]);
@@ -218,7 +222,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
             const int row0 = g.tiles[3 * mt + 1], rows = g.tiles[3 * mt + 2];
             const bool row_ok = row < rows;
-            if (!mbar_wait(&S->accf[acc], aphase)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
+            if (!mbar_wait(&S->accf[acc], aphase, g.wait_ns)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
             tc_fence_after();
             const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
             if (MODE == 0) {

@@ -20,6 +20,8 @@ namespace {
 
 std::atomic<int> g_gemm_ctas{0};
 std::atomic<int> g_claim_reverse{0};
+std::atomic<unsigned long long> g_wait_ns{0};
+std::atomic<int> g_stall_test{0};
 std::mutex g_ev_mu;
 cudaEvent_t g_stage_ev[MOE_STAGE_EVENTS];
 bool g_stage_on = false;
@@ -109,6 +111,10 @@ T *at(void *ws, size_t off)
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// Activations, weights and outputs are read and written in 16-byte vectors (and the
+// weights by TMA, which needs 16-byte aligned bases).
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 }  // namespace
 
 extern "C" {
@@ -130,6 +136,12 @@ void moe_set_gemm_ctas(int32_t ctas) { g_gemm_ctas.store(ctas > 0 ? ctas : 0); }
 
 void moe_set_claim_order(int32_t reverse) { g_claim_reverse.store(reverse ? 1 : 0); }
 
+void moe_set_wait_limit_us(int32_t us, int32_t stall_test)
+{
+    g_wait_ns.store(us > 0 ? static_cast<unsigned long long>(us) * 1000ull : 0ull);
+    g_stall_test.store(stall_test ? 1 : 0);
+}
+
 void moe_set_stage_events(void *const *events, int32_t n)
 {
     std::lock_guard<std::mutex> lk(g_ev_mu);
@@ -145,6 +157,7 @@ moe_status_t moe_route(const moe_dims_t *d, const void *x, const void *router_w,
     if (s != MOE_OK) return s;
     if (d->T == 0) return MOE_OK;
     if (!x || !router_w || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(router_w)) return MOE_ERR_INVALID_ARG;
     if ((s = check_ws(d, ws, ws_bytes)) != MOE_OK) return s;
     const moe::WsLayout L = moe::ws_layout(*d);
     return cuda_status(moe::launch_route(*d, static_cast<const __nv_bfloat16 *>(x),
@@ -180,6 +193,9 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
     if (s != MOE_OK) return s;
     if (d->T == 0) return MOE_OK;
     if (!x || !router_w || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+        !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
     if ((s = check_ws(d, ws, ws_bytes)) != MOE_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const moe::WsLayout L = moe::ws_layout(*d);
@@ -217,13 +233,16 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
         e = moe::launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), s2f, A, d->H, d->top_k, xs, st);
     if (e == cudaSuccess) e = marks.mark(2, st);
     const int ctas = g_gemm_ctas.load(), rev = g_claim_reverse.load();
+    const unsigned long long wl = g_wait_ns.load();
+    const uint64_t wait_ns = wl ? wl : 2000000000ull;
+    const int stall = g_stall_test.load();
     if (e == cudaSuccess) {
-        moe::GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, h, nullptr, ctas, rev};
+        moe::GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, h, nullptr, ctas, rev, wait_ns, stall};
         e = moe::launch_grouped_gemm(g1, tm_xs, tm_wg, tm_wu, st);
     }
     if (e == cudaSuccess) e = marks.mark(3, st);
     if (e == cudaSuccess) {
-        moe::GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, y, s2f, ctas, rev};
+        moe::GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, y, s2f, ctas, rev, wait_ns, stall};
         e = moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st);
     }
     if (e == cudaSuccess) e = marks.mark(4, st);

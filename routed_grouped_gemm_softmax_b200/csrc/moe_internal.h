@@ -103,6 +103,8 @@ struct GemmArgs {
     const int32_t *row_map;
     int ctas;
     int reverse;
+    uint64_t wait_ns;  // limit of each pipeline wait
+    int stall_test;    // MMA thread first waits on a barrier nothing signals
 };
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
                                 const CUtensorMap &tmB1, cudaStream_t st);

@@ -11,8 +11,9 @@
 // are reproducible bit for bit.
 //
 // Kernel 1 (route_logits): a CUDA-core tile of TT tokens x TE experts per CTA,
-//   operands staged in shared memory as fp32 (bf16 -> fp32 is exact), each
-//   thread owning RT x RE independent chains.
+//   operands staged in double-buffered shared memory as fp32 (bf16 -> fp32 is
+//   exact), the next chunk prefetched into registers, each thread owning RT x RE
+//   independent chains.
 // Kernel 2 (route_topk): one warp per token; k rounds of a warp arg-max with the
 //   (larger logit, then lower index) order, then the softmax over the k chosen
 //   logits with the maximum subtracted.
@@ -24,21 +25,105 @@
 namespace moe {
 namespace {
 
-constexpr int HC = 32;  // h values staged per step
+// Logits tile kernel.  A CTA owns TT tokens x TE experts, a thread RT x RE of them.
+// The h axis is walked in chunks of HC: the chunk after the current one is fetched
+// from global memory into registers (bf16) while the current one -- already in
+// shared memory as fp32, x transposed to [h][token] so a thread's tokens are
+// contiguous -- feeds the FMA chains; one barrier per chunk.
+template <int TT, int TE, int RT, int RE, int HC>
+struct LogitsTile {
+    static constexpr int NX = TE / RE;             // threads along experts
+    static constexpr int NT = (TT / RT) * NX;      // threads per CTA
+    static constexpr int XV = TT * HC / 8;         // 16-byte vectors of an x chunk
+    static constexpr int WV = HC * TE / 8;         // 16-byte vectors of a router_w chunk
+    static constexpr int XPT = (XV + NT - 1) / NT; // x vectors per thread
+    static constexpr int WPT = (WV + NT - 1) / NT; // w vectors per thread
+    static constexpr int SMEM_FLOATS = 2 * HC * (TT + TE);
+};
 
-template <int TT, int TE, int RT, int RE>
-__global__ void __launch_bounds__((TT / RT) * (TE / RE))
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8])
+{
+    const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 t = __bfloat1622float2(p[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+template <int TT, int TE, int RT, int RE, int HC>
+__global__ void __launch_bounds__(LogitsTile<TT, TE, RT, RE, HC>::NT)
 route_logits_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ wr,
                     const float *__restrict__ bias, int T, int H, int E, float *__restrict__ logits)
 {
-    constexpr int NX = TE / RE;           // threads along experts
-    constexpr int NT = (TT / RT) * NX;    // threads per CTA
-    __shared__ float xs[TT * (HC + 1)];   // [token][h], padded row
-    __shared__ __align__(16) float wsm[HC * TE];  // [h][expert]
+    using L = LogitsTile<TT, TE, RT, RE, HC>;
+    extern __shared__ __align__(16) float lsm[];
+    // two buffers of x chunks, [h][token], then two of router_w chunks, [h][expert]
+    auto xs = [&](int buf) { return lsm + buf * (HC * TT); };
+    auto ws = [&](int buf) { return lsm + 2 * HC * TT + buf * (HC * TE); };
 
     const int tid = threadIdx.x;
-    const int tx = tid % NX, ty = tid / NX;
+    const int tx = tid % L::NX, ty = tid / L::NX;
     const int t0 = blockIdx.x * TT, e0 = blockIdx.y * TE;
+    const bool wvec = (E % 8) == 0;  // router_w rows are 16-byte aligned
+
+    uint4 xr[L::XPT], wrg[L::WPT];
+    auto fetch = [&](int h0) {
+#pragma unroll
+        for (int i = 0; i < L::XPT; ++i) {
+            const int v = tid + i * L::NT;
+            xr[i] = make_uint4(0, 0, 0, 0);
+            if (v < L::XV) {
+                const int tt = v % TT, h = h0 + (v / TT) * 8;
+                if (t0 + tt < T) xr[i] = *reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * H + h);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < L::WPT; ++i) {
+            const int v = tid + i * L::NT;
+            wrg[i] = make_uint4(0, 0, 0, 0);
+            if (v < L::WV) {
+                const int hh = v / (TE / 8), e = e0 + (v % (TE / 8)) * 8;
+                const __nv_bfloat16 *src = wr + (size_t)(h0 + hh) * E + e;
+                if (wvec && e + 8 <= E) {
+                    wrg[i] = *reinterpret_cast<const uint4 *>(src);
+                } else {
+                    const unsigned short *s16 = reinterpret_cast<const unsigned short *>(src);
+                    uint32_t u[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        if (e + q < E) u[q / 2] |= static_cast<uint32_t>(s16[q]) << (16 * (q & 1));
+                    wrg[i] = make_uint4(u[0], u[1], u[2], u[3]);
+                }
+            }
+        }
+    };
+    auto stash = [&](int buf) {
+#pragma unroll
+        for (int i = 0; i < L::XPT; ++i) {
+            const int v = tid + i * L::NT;
+            if (v < L::XV) {
+                const int tt = v % TT, hq = (v / TT) * 8;
+                float f[8];
+                bf16x8_to_f32(xr[i], f);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) xs(buf)[(hq + q) * TT + tt] = f[q];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < L::WPT; ++i) {
+            const int v = tid + i * L::NT;
+            if (v < L::WV) {
+                const int hh = v / (TE / 8), e8 = (v % (TE / 8)) * 8;
+                float f[8];
+                bf16x8_to_f32(wrg[i], f);
+                float4 *dst = reinterpret_cast<float4 *>(ws(buf) + hh * TE + e8);
+                dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+                dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+            }
+        }
+    };
 
     float acc[RT][RE];
 #pragma unroll
@@ -46,38 +131,46 @@ route_logits_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__
 #pragma unroll
         for (int c = 0; c < RE; ++c) acc[r][c] = 0.0f;
 
-    for (int h0 = 0; h0 < H; h0 += HC) {
-        __syncthreads();
-        for (int i = tid; i < TT * HC; i += NT) {
-            const int tt = i / HC, hh = i % HC;
-            const int t = t0 + tt, h = h0 + hh;
-            xs[tt * (HC + 1) + hh] = (t < T && h < H) ? __bfloat162float(x[(size_t)t * H + h]) : 0.0f;
-        }
-        for (int i = tid; i < HC * TE; i += NT) {
-            const int hh = i / TE, ee = i % TE;
-            const int h = h0 + hh, e = e0 + ee;
-            wsm[i] = (h < H && e < E) ? __bfloat162float(wr[(size_t)h * E + e]) : 0.0f;
-        }
-        __syncthreads();
-        const int hn = (H - h0) < HC ? (H - h0) : HC;
-        // Chains stop at h = H-1: padding columns would add 0*0 terms, which leave
-        // the chain unchanged, but the loop bound keeps the chain length exactly H.
-        for (int hh = 0; hh < hn; ++hh) {
+    const int nchunks = H / HC;
+    fetch(0);
+    stash(0);
+    __syncthreads();
+    for (int ch = 0; ch < nchunks; ++ch) {
+        const int buf = ch & 1;
+        if (ch + 1 < nchunks) fetch((ch + 1) * HC);
+        const float *xb = xs(buf);
+        const float *wb = ws(buf);
+        // h ascending inside the chunk, chunks ascending: each chain runs h = 0..H-1 in order
+#pragma unroll 4
+        for (int hh = 0; hh < HC; ++hh) {
             float a[RT], b[RE];
+            if constexpr (RT % 4 == 0) {
 #pragma unroll
-            for (int r = 0; r < RT; ++r) a[r] = xs[(ty * RT + r) * (HC + 1) + hh];
-            if constexpr (RE == 4) {
-                const float4 v = *reinterpret_cast<const float4 *>(&wsm[hh * TE + tx * 4]);
-                b[0] = v.x; b[1] = v.y; b[2] = v.z; b[3] = v.w;
+                for (int r = 0; r < RT; r += 4) {
+                    const float4 v = *reinterpret_cast<const float4 *>(xb + hh * TT + ty * RT + r);
+                    a[r] = v.x; a[r + 1] = v.y; a[r + 2] = v.z; a[r + 3] = v.w;
+                }
             } else {
 #pragma unroll
-                for (int c = 0; c < RE; ++c) b[c] = wsm[hh * TE + tx * RE + c];
+                for (int r = 0; r < RT; ++r) a[r] = xb[hh * TT + ty * RT + r];
+            }
+            if constexpr (RE % 4 == 0) {
+#pragma unroll
+                for (int c = 0; c < RE; c += 4) {
+                    const float4 v = *reinterpret_cast<const float4 *>(wb + hh * TE + tx * RE + c);
+                    b[c] = v.x; b[c + 1] = v.y; b[c + 2] = v.z; b[c + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < RE; ++c) b[c] = wb[hh * TE + tx * RE + c];
             }
 #pragma unroll
             for (int r = 0; r < RT; ++r)
 #pragma unroll
                 for (int c = 0; c < RE; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
         }
+        if (ch + 1 < nchunks) stash(buf ^ 1);
+        __syncthreads();
     }
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
@@ -92,6 +185,112 @@ route_logits_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__
             }
         }
     }
+}
+
+// Small batches (T <= 32): one chain per thread, TP tokens x TE experts per CTA.
+// The chain is latency-bound (H dependent FMAs), so the kernel only has to keep
+// its operands arriving: chunks of HC h-values stream into an S-stage shared
+// memory ring with cp.async (bf16, converted at use), S-1 chunks in flight --
+// with 16 stages of 128 values the whole H = 2048 slice is requested at once.
+template <int TP, int TE, int HC, int S>
+struct SmallTile {
+    static constexpr int NT = TP * TE;
+    static constexpr int XROW = HC * 2 + 16;            // bytes per token row (padded)
+    static constexpr int XBYTES = TP * XROW;
+    static constexpr int WBYTES = HC * TE * 2;
+    static constexpr int STAGE = XBYTES + WBYTES;
+    static constexpr int SMEM = S * STAGE;
+};
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int TP, int TE, int HC, int S>
+__global__ void __launch_bounds__(TP * TE)
+route_logits_small_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ wr,
+                          const float *__restrict__ bias, int T, int H, int E, float *__restrict__ logits)
+{
+    using L = SmallTile<TP, TE, HC, S>;
+    extern __shared__ __align__(16) uint8_t ssm[];
+    const int tid = threadIdx.x;
+    const int tt = tid / TE, ee = tid % TE;
+    const int e0 = blockIdx.x * TE;
+    const int nchunks = H / HC;
+
+    auto issue = [&](int ch) {
+        if (ch < nchunks) {
+            uint8_t *st = ssm + (ch % S) * L::STAGE;
+            const int h0 = ch * HC;
+            for (int v = tid; v < TP * (HC / 8); v += L::NT) {  // x: TP rows of HC values
+                const int r = v / (HC / 8), c8 = (v % (HC / 8)) * 8;
+                if (r < T) cp_async16(st + r * L::XROW + c8 * 2, x + (size_t)r * H + h0 + c8);
+            }
+            for (int v = tid; v < HC * (TE / 8); v += L::NT) {  // router_w: HC rows of TE experts
+                const int hh = v / (TE / 8), c8 = (v % (TE / 8)) * 8;
+                if (e0 + c8 < E) cp_async16(st + L::XBYTES + (hh * TE + c8) * 2, wr + (size_t)(h0 + hh) * E + e0 + c8);
+            }
+        }
+        cp_async_commit();  // one group per chunk slot, empty past the end
+    };
+
+    float acc = 0.0f;
+#pragma unroll
+    for (int s = 0; s < S - 1; ++s) issue(s);
+    for (int ch = 0; ch < nchunks; ++ch) {
+        cp_async_wait<S - 2>();
+        __syncthreads();             // chunk ch visible to all; stage (ch-1)%S free
+        issue(ch + S - 1);
+        const uint8_t *st = ssm + (ch % S) * L::STAGE;
+        const __nv_bfloat16 *xr = reinterpret_cast<const __nv_bfloat16 *>(st + tt * L::XROW);
+        const __nv_bfloat16 *wc = reinterpret_cast<const __nv_bfloat16 *>(st + L::XBYTES) + ee;
+#pragma unroll 8
+        for (int hh = 0; hh < HC; ++hh)
+            acc = fmaf(__bfloat162float(xr[hh]), __bfloat162float(wc[hh * TE]), acc);
+    }
+    cp_async_wait<0>();
+    const int e = e0 + ee;
+    if (tt < T && e < E) {
+        float v = acc;
+        if (bias) v = __fadd_rn(v, bias[e]);
+        logits[(size_t)tt * E + e] = v;
+    }
+}
+
+template <int TP, int TE, int HC, int S>
+cudaError_t launch_logits_small(const __nv_bfloat16 *x, const __nv_bfloat16 *wr, const float *bias, int T, int H,
+                                int E, float *logits, cudaStream_t st)
+{
+    using L = SmallTile<TP, TE, HC, S>;
+    auto kern = route_logits_small_kernel<TP, TE, HC, S>;
+    if (L::SMEM > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<(E + TE - 1) / TE, L::NT, L::SMEM, st>>>(x, wr, bias, T, H, E, logits);
+    return cudaGetLastError();
+}
+
+template <int TT, int TE, int RT, int RE, int HC>
+cudaError_t launch_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wr, const float *bias, int T, int H,
+                          int E, float *logits, cudaStream_t st)
+{
+    using L = LogitsTile<TT, TE, RT, RE, HC>;
+    const size_t smem = (size_t)L::SMEM_FLOATS * sizeof(float);
+    auto kern = route_logits_kernel<TT, TE, RT, RE, HC>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    dim3 grid((T + TT - 1) / TT, (E + TE - 1) / TE);
+    kern<<<grid, L::NT, smem, st>>>(x, wr, bias, T, H, E, logits);
+    return cudaGetLastError();
 }
 
 // (v1, e1) ranks before (v2, e2): larger logit first, equal logits -> lower index.
@@ -177,14 +376,20 @@ cudaError_t launch_route(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv
                          cudaStream_t st)
 {
     const int T = d.T, H = d.H, E = d.E, k = d.top_k;
-    if (T <= 32) {
-        dim3 grid((T + 15) / 16, (E + 15) / 16);
-        route_logits_kernel<16, 16, 1, 1><<<grid, 256, 0, st>>>(x, wr, bias, T, H, E, logits);
-    } else {
-        dim3 grid((T + 63) / 64, (E + 63) / 64);
-        route_logits_kernel<64, 64, 4, 4><<<grid, 256, 0, st>>>(x, wr, bias, T, H, E, logits);
-    }
-    cudaError_t e = cudaGetLastError();
+    // Pick the tile so that enough warps exist to cover the SMs: small batches get
+    // one chain per thread, large ones register-blocked 8x4 or 4x4 chains.
+    cudaError_t e;
+    const long tiles64 = (long)((T + 63) / 64) * ((E + 63) / 64);
+    if (T <= 16 && E % 8 == 0 && H % 128 == 0)
+        e = launch_logits_small<16, 8, 128, 16>(x, wr, bias, T, H, E, logits, st);
+    else if (T <= 32 && E % 8 == 0 && H % 128 == 0)
+        e = launch_logits_small<32, 8, 128, 16>(x, wr, bias, T, H, E, logits, st);
+    else if (T <= 32)
+        e = launch_logits<16, 16, 1, 1, 64>(x, wr, bias, T, H, E, logits, st);
+    else if (tiles64 * 4 >= 4 * num_sms())
+        e = launch_logits<64, 64, 8, 4, 32>(x, wr, bias, T, H, E, logits, st);
+    else
+        e = launch_logits<32, 64, 4, 4, 32>(x, wr, bias, T, H, E, logits, st);
     if (e != cudaSuccess) return e;
     const int vpl = (E + 31) / 32;
     if (vpl <= 1) return launch_topk<1>(logits, T, E, k, idx, gate, st);

@@ -167,6 +167,26 @@ def test_cuda_graph_replay():
     del graph
 
 
+def test_pipeline_wait_timeout_is_reported_and_recoverable():
+    # Test hook: every GEMM CTA's MMA thread first waits on a barrier that nothing
+    # signals, with a 2 ms bound.  The wait runs out, the kernels record
+    # MOE_ERR_TIMEOUT, drain their own copies and return; the next call with the
+    # default settings must be correct on the same workspace.
+    cfg = SMALL["ragged"]
+    g, c = device_inputs(cfg)
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k, "cuda")
+    try:
+        api.set_wait_limit_us(2000, stall_test=True)
+        api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k, ws=ws)
+        assert api.moe_get_device_status(ws) == 5  # MOE_ERR_TIMEOUT
+    finally:
+        api.set_wait_limit_us(0, stall_test=False)
+    out = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k, ws=ws)
+    assert api.moe_get_device_status(ws) == api.MOE_OK
+    idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], cfg.top_k)
+    compare_out(out, oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"]), "after timeout")
+
+
 def test_bad_expert_index_flagged():
     idx = torch.tensor([[0, 1], [5, 9]], dtype=torch.int32, device="cuda")  # 9 >= E=8
     ws = api.workspace(2, 256, 64, 8, 2, "cuda")
