@@ -75,6 +75,14 @@ class Oracle:
         lib.oracle_permute.restype = i
         lib.oracle_combine_ffn.argtypes = [i, i, i, P, P, P, P, P, P, i, P, P, i]
         lib.oracle_combine_ffn.restype = i
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_encode_array.argtypes = [i, P, P]
+        lib.oracle_e4m3_encode_array.restype = None
+        lib.oracle_quantize_rows.argtypes = [i, i, P, P, P]
+        lib.oracle_quantize_rows.restype = i
+        lib.oracle_combine_ffn_fp8.argtypes = [i, i, i, P, P, P, P, P, P, P, P, P, i, P, P, i]
+        lib.oracle_combine_ffn_fp8.restype = i
         self.lib = lib
 
     def route(self, x, router_w, bias, top_k: int, want_logits: bool = False,
@@ -135,6 +143,55 @@ class Oracle:
             raise ValueError(f"oracle_combine_ffn rejected its arguments (code {rc})")
         return out
 
+    # ------------------------------------------------------------ FP8 variant
+
+    def e4m3_decode(self, codes) -> np.ndarray:
+        c = np.asarray(codes, dtype=np.uint8).reshape(-1)
+        return np.array([self.lib.oracle_e4m3_decode(int(v)) for v in c]).reshape(np.shape(codes))
+
+    def e4m3_encode(self, values) -> np.ndarray:
+        v = np.ascontiguousarray(np.asarray(values, dtype=np.float32).reshape(-1))
+        q = np.zeros(v.size, np.uint8)
+        self.lib.oracle_e4m3_encode_array(v.size, _ptr(v), _ptr(q))
+        return q.reshape(np.shape(values))
+
+    def quantize_rows(self, a):
+        """Per-row, per-128-column e4m3 quantisation of a bf16 [R,K] matrix:
+        returns (codes uint8 [R,K], scales fp32 [R,K/128])."""
+        ab = _bf16_bits(a)
+        R, K = ab.shape
+        q = np.zeros((R, K), np.uint8)
+        s = np.zeros((R, K // 128), np.float32)
+        rc = self.lib.oracle_quantize_rows(R, K, _ptr(ab), _ptr(q), _ptr(s))
+        if rc:
+            raise ValueError(f"oracle_quantize_rows rejected its arguments (code {rc})")
+        return q, s
+
+    def combine_ffn_fp8(self, x, idx, gate, wg_q, wg_s, wu_q, wu_s, wd_q, wd_s, tokens=None,
+                        nthreads: int | None = None):
+        """FP8 block-scaled expert FFN + gate-weighted combine, fp64 [n,H]."""
+        xb = _bf16_bits(x)
+        T, H = xb.shape
+        def u8(t):
+            return np.ascontiguousarray(t.cpu().view(__import__("torch").uint8).numpy()
+                                        if hasattr(t, "cpu") else np.asarray(t, dtype=np.uint8))
+        wg, wu, wd = u8(wg_q), u8(wu_q), u8(wd_q)
+        sg, su, sd = _f32(wg_s), _f32(wu_s), _f32(wd_s)
+        E, I, H2 = wg.shape
+        assert H2 == H and wd.shape == (E, H, I)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        k = idx.shape[1]
+        tok = None if tokens is None else np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+        n = T if tok is None else tok.size
+        out = np.zeros((n, H), np.float64)
+        rc = self.lib.oracle_combine_ffn_fp8(H, I, k, _ptr(xb), _ptr(idx), _ptr(gate), _ptr(wg), _ptr(sg),
+                                             _ptr(wu), _ptr(su), _ptr(wd), _ptr(sd), n, _ptr(tok),
+                                             _ptr(out), nthreads or default_threads())
+        if rc:
+            raise ValueError(f"oracle_combine_ffn_fp8 rejected its arguments (code {rc})")
+        return out
+
     def forward(self, x, router_w, bias, w_gate, w_up, w_down, top_k: int, tokens=None,
                 nthreads: int | None = None):
         """The whole layer for the given tokens (all when None): (out fp64, idx, gate)."""
@@ -167,3 +224,11 @@ def combine_ffn(*a, **kw):
 
 def forward(*a, **kw):
     return get().forward(*a, **kw)
+
+
+def quantize_rows(*a, **kw):
+    return get().quantize_rows(*a, **kw)
+
+
+def combine_ffn_fp8(*a, **kw):
+    return get().combine_ffn_fp8(*a, **kw)

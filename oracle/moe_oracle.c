@@ -31,6 +31,15 @@
  *  - the permutation into expert groups is a stable counting sort of the flat
  *    assignment list (flat = t*k + j) by expert; group offsets carry no padding.
  *
+ * FP8 block-scaled variant (GC-MoE page: block-scaled FP8/FP4 MMA with SwiGLU
+ * and requantisation fused; vLLM fused-MoE page, section 03: fp8 weights with
+ * [128,128] blocks): weights come as e4m3 codes with one fp32 scale per
+ * 128x128 block; activations (x, and h after SwiGLU) are quantised per row per
+ * 128-column group with s = amax/448 (fp32) and q = e4m3 round-to-nearest-even
+ * of clamp(v/s, -448, 448) (fp32 division); amax = 0 gives s = 1, q = 0.  Each
+ * GEMM is sum over 128-wide K blocks of sa[row,kb] * sb[nblk,kb] * (qa . qb)_kb,
+ * evaluated in fp64 from the exact decoded codes.
+ *
  * Deliberately slow and direct: no blocking, no fusion, no reordering.
  */
 #include <math.h>
@@ -281,6 +290,185 @@ int oracle_combine_ffn(int H, int I, int k, const uint16_t *x, const int32_t *id
     }
     for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, ffn_worker, &jobs[i]);
     ffn_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    return 0;
+}
+
+/* -------------------------------------------------------------- FP8 e4m3 */
+
+/* Value of an e4m3 (OCP "fn" variant) code: 1 sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent 0 is subnormal (m/8 * 2^-6); 0x7F/0xFF are
+ * NaN (returned as NaN here); there is no infinity; the largest finite value
+ * is 448. */
+double oracle_e4m3_decode(uint8_t c)
+{
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = (double)m / 8.0 * ldexp(1.0, -6);
+    else
+        v = (1.0 + (double)m / 8.0) * ldexp(1.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* All 256 decoded codes, built once from oracle_e4m3_decode (a speed-up of the
+ * GEMM loops only; the definition is the function above). */
+static double g_e4m3[256];
+static pthread_once_t g_e4m3_once = PTHREAD_ONCE_INIT;
+static void build_e4m3_table(void)
+{
+    for (int c = 0; c < 256; ++c) g_e4m3[c] = oracle_e4m3_decode((uint8_t)c);
+}
+static double e4m3(uint8_t c) { return g_e4m3[c]; }
+
+/* Round-to-nearest-even e4m3 code of a value already inside [-448, 448]:
+ * the nearest finite code by brute force over all 127 magnitudes; on a tie the
+ * code whose last mantissa bit is 0. */
+uint8_t oracle_e4m3_encode(float v)
+{
+    double a = fabs((double)v);
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c < 127; ++c) {
+        double d = fabs(oracle_e4m3_decode((uint8_t)c) - a);
+        if (d < bd || (d == bd && (c & 1) == 0 && (best & 1) == 1)) {
+            bd = d;
+            best = c;
+        }
+    }
+    if (best != 0 && v < 0) best |= 0x80;
+    if (best == 0 && signbit(v)) best = 0x80;
+    return (uint8_t)best;
+}
+
+/* Codes of n values already inside [-448, 448]. */
+void oracle_e4m3_encode_array(int n, const float *v, uint8_t *q)
+{
+    for (int i = 0; i < n; ++i) q[i] = oracle_e4m3_encode(v[i]);
+}
+
+/* Quantise one group of n fp32 values: s = amax/448, q = e4m3(clamp(v/s)). */
+static float quantize_group(const float *v, int n, uint8_t *q)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i)
+        if (fabsf(v[i]) > amax) amax = fabsf(v[i]);
+    if (amax == 0.0f) {
+        for (int i = 0; i < n; ++i) q[i] = 0;
+        return 1.0f;
+    }
+    float s = amax / 448.0f;
+    for (int i = 0; i < n; ++i) {
+        float r = v[i] / s;
+        if (r > 448.0f) r = 448.0f;
+        if (r < -448.0f) r = -448.0f;
+        q[i] = oracle_e4m3_encode(r);
+    }
+    return s;
+}
+
+/* Per-row, per-128-column-group quantisation of a bf16 matrix [R, K]
+ * (K a multiple of 128): q [R, K] e4m3 codes, s [R, K/128] fp32 scales. */
+int oracle_quantize_rows(int R, int K, const uint16_t *a, uint8_t *q, float *s)
+{
+    if (R < 0 || K <= 0 || K % 128) return 1;
+    float buf[128];
+    for (int r = 0; r < R; ++r)
+        for (int g = 0; g < K / 128; ++g) {
+            for (int i = 0; i < 128; ++i) buf[i] = bf16_to_f32(a[(size_t)r * K + g * 128 + i]);
+            s[(size_t)r * (K / 128) + g] = quantize_group(buf, 128, q + (size_t)r * K + g * 128);
+        }
+    return 0;
+}
+
+/* One row of a block-scaled GEMM: out[n] = sum_kb sa[kb] * sb[n/128, kb] *
+ * sum_{k in kb} qa[k] * qb[n, k], for n in [0, N); qb [N, K] codes, sb [N/128,
+ * K/128] scales, qa [K] codes, sa [K/128] scales. */
+static void fp8_row_gemm(int N, int K, const uint8_t *qa, const float *sa, const uint8_t *qb,
+                         const float *sb, double *out)
+{
+    const int KB = K / 128;
+    for (int n = 0; n < N; ++n) {
+        double acc = 0.0;
+        for (int kb = 0; kb < KB; ++kb) {
+            double part = 0.0;
+            for (int k = kb * 128; k < kb * 128 + 128; ++k)
+                part += e4m3(qa[k]) * e4m3(qb[(size_t)n * K + k]);
+            acc += (double)sa[kb] * (double)sb[(size_t)(n / 128) * KB + kb] * part;
+        }
+        out[n] = acc;
+    }
+}
+
+typedef struct {
+    int H, I, k;
+    const uint16_t *x;
+    const int32_t *idx;
+    const double *gate;
+    const uint8_t *wg, *wu, *wd;
+    const float *sg, *su, *sd;
+    const int32_t *tokens;
+    double *out;
+    int n0, n1;
+} ffn8_job;
+
+static void *ffn8_worker(void *p)
+{
+    ffn8_job *j = (ffn8_job *)p;
+    const int H = j->H, I = j->I;
+    uint8_t *qx = (uint8_t *)malloc((size_t)H);
+    float *sx = (float *)malloc(sizeof(float) * (size_t)(H / 128));
+    double *g = (double *)malloc(sizeof(double) * (size_t)I);
+    double *u = (double *)malloc(sizeof(double) * (size_t)I);
+    float *h = (float *)malloc(sizeof(float) * (size_t)I);
+    uint8_t *qh = (uint8_t *)malloc((size_t)I);
+    float *sh = (float *)malloc(sizeof(float) * (size_t)(I / 128));
+    double *y = (double *)malloc(sizeof(double) * (size_t)H);
+    for (int n = j->n0; n < j->n1; ++n) {
+        int t = j->tokens ? j->tokens[n] : n;
+        oracle_quantize_rows(1, H, j->x + (size_t)t * H, qx, sx);
+        double *o = j->out + (size_t)n * H;
+        for (int c = 0; c < H; ++c) o[c] = 0.0;
+        for (int q = 0; q < j->k; ++q) {
+            int e = j->idx[(size_t)t * j->k + q];
+            double gt = j->gate[(size_t)t * j->k + q];
+            fp8_row_gemm(I, H, qx, sx, j->wg + (size_t)e * I * H, j->sg + (size_t)e * (I / 128) * (H / 128), g);
+            fp8_row_gemm(I, H, qx, sx, j->wu + (size_t)e * I * H, j->su + (size_t)e * (I / 128) * (H / 128), u);
+            for (int i = 0; i < I; ++i) h[i] = (float)(silu(g[i]) * u[i]);
+            for (int b = 0; b < I / 128; ++b) sh[b] = quantize_group(h + b * 128, 128, qh + b * 128);
+            fp8_row_gemm(H, I, qh, sh, j->wd + (size_t)e * H * I, j->sd + (size_t)e * (H / 128) * (I / 128), y);
+            for (int c = 0; c < H; ++c) o[c] += gt * y[c];
+        }
+    }
+    free(qx); free(sx); free(g); free(u); free(h); free(qh); free(sh); free(y);
+    return NULL;
+}
+
+/* FP8 variant of oracle_combine_ffn: x [T,H] bf16 is quantised per token per
+ * 128 columns, each chosen expert's gate/up GEMMs are block-scaled sums, the
+ * SwiGLU output h (rounded to fp32) is requantised per 128 columns, the down
+ * GEMM is block-scaled, and the k results are summed with the gates in fp64.
+ *   wg/wu [E,I,H] codes with sg/su [E,I/128,H/128]; wd [E,H,I] with sd [E,H/128,I/128]. */
+int oracle_combine_ffn_fp8(int H, int I, int k, const uint16_t *x, const int32_t *idx,
+                           const double *gate, const uint8_t *wg, const float *sg, const uint8_t *wu,
+                           const float *su, const uint8_t *wd, const float *sd, int n,
+                           const int32_t *tokens, double *out, int nthreads)
+{
+    if (H <= 0 || I <= 0 || H % 128 || I % 128 || k < 1 || n < 0) return 1;
+    pthread_once(&g_e4m3_once, build_e4m3_table);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > n) nthreads = n > 0 ? n : 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    ffn8_job jobs[256];
+    for (int i = 0; i < nthreads; ++i) {
+        ffn8_job jb = {H, I, k, x, idx, gate, wg, wu, wd, sg, su, sd, tokens, out,
+                       (int)((long)n * i / nthreads), (int)((long)n * (i + 1) / nthreads)};
+        jobs[i] = jb;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, ffn8_worker, &jobs[i]);
+    ffn8_worker(&jobs[0]);
     for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
     return 0;
 }

@@ -34,6 +34,8 @@
 // MOE_ERR_TIMEOUT in the workspace status word and the CTA unwinds -- waiting,
 // with the fixed default bound, for its own TMA copies and MMAs -- before
 // freeing TMEM.
+#include <mutex>
+
 #include "moe_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -283,26 +285,41 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
 int num_sms()
 {
+    static int cached[64] = {};
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
     return n;
+}
+
+// The kernels need more than the default 48 KB of dynamic shared memory; the
+// attribute is set once per device (and per kernel) rather than on every launch.
+static bool smem_attr_ready(int mode)
+{
+    static std::mutex mu;
+    static uint64_t done[2] = {0, 0};  // bit per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    if (done[mode] >> dev & 1ull) return true;
+    cudaError_t e = mode == 0 ? cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)
+                              : cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return false;
+    done[mode] |= 1ull << dev;
+    return true;
 }
 
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
                                 const CUtensorMap &tmB1, cudaStream_t st)
 {
     const int grid = g.ctas > 0 ? g.ctas : num_sms();
-    cudaError_t e;
-    if (g.mode == 0) {
-        e = cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
+    if (!smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
+    if (g.mode == 0)
         grouped_gemm_kernel<0><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
-    } else {
-        e = cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
+    else
         grouped_gemm_kernel<1><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
-    }
     return cudaGetLastError();
 }
 

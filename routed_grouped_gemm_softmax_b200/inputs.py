@@ -153,12 +153,54 @@ class MoEInputs:
     extra: dict = field(default_factory=dict)
 
 
+def quantize_blocks_e4m3(w: torch.Tensor):
+    """Input recipe of the fp8 workload's weights (given to the layer pre-quantised):
+    one fp32 scale per 128x128 block of each expert matrix [E, N, K],
+    s = amax/448 (s = 1 for an all-zero block), codes = e4m3(clamp(w/s, +-448))
+    via torch's float8_e4m3fn cast.  Returns (codes uint8 [E,N,K], scales fp32
+    [E, N/128, K/128])."""
+    E, N, K = w.shape
+    b = w.view(E, N // 128, 128, K // 128, 128).float()
+    amax = b.abs().amax(dim=(2, 4))
+    s = torch.where(amax == 0, torch.ones_like(amax), amax / 448.0)
+    q = (b / s[:, :, None, :, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    return q.view(torch.uint8).reshape(E, N, K).contiguous(), s.contiguous()
+
+
+def make_fp8_weights(cfg: MoEConfig, device="cpu", experts_per_chunk: int = 8):
+    """The fp8 workload's expert weights: drawn like the bf16 ones (fp32 master values
+    ~ N(0, 1/sqrt(fan_in)), same streams) and block-quantised, a few experts at a
+    time so the fp32 values never exist in full.  Returns a dict of codes/scales."""
+    E, I, H = cfg.E, cfg.I, cfg.H
+    out = {}
+    for name, (N, K) in (("w_gate", (I, H)), ("w_up", (I, H)), ("w_down", (H, I))):
+        key = stream_key(cfg.seed, TENSOR_IDS[name])
+        std = 1.0 / math.sqrt(K)
+        q = torch.empty((E, N, K), dtype=torch.uint8, device=device)
+        sc = torch.empty((E, N // 128, K // 128), dtype=torch.float32, device=device)
+        per = N * K
+        for e0 in range(0, E, experts_per_chunk):
+            e1 = min(E, e0 + experts_per_chunk)
+            v = torch.empty((e1 - e0) * per, dtype=torch.float32, device=device)
+            step = 1 << 24
+            for s0 in range(0, v.numel(), step):
+                c = min(step, v.numel() - s0)
+                v[s0:s0 + c] = (normal(key, e0 * per + s0, c, device) * std).to(torch.float32)
+            qq, ss = quantize_blocks_e4m3(v.view(e1 - e0, N, K))
+            q[e0:e1] = qq
+            sc[e0:e1] = ss
+        out[name + "_q"] = q
+        out[name + "_s"] = sc
+    return out
+
+
 def make_inputs(cfg: MoEConfig, device="cpu", weights: bool = True) -> MoEInputs:
     """Draw the workload's tensors in the fixed order x, router_w, [bias], w_gate, w_up, w_down.
 
     Expert weights ~ N(0, 1/sqrt(fan_in)) (fan_in = H for gate/up, I for down);
     x ~ N(0, 1); router_w ~ N(0, 0.02).  For the fp8 workload the expert weights
-    are returned as fp32 underlying values (each side quantises them itself).
+    are returned as fp32 underlying values; ``make_fp8_weights`` gives the quantised
+    codes and block scales both sides consume.
     """
     T, H, E, I = cfg.T, cfg.H, cfg.E, cfg.I
     x = gaussian_tensor(cfg.seed, "x", (T, H), 1.0, device)

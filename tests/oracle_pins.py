@@ -269,3 +269,113 @@ ALL_PINS = [pin_logits_vs_fp64_matmul, pin_logit_chain_order, pin_topk_brute_for
             pin_ties_lower_index, pin_gates, pin_bias_enters_logits, pin_permute,
             pin_ffn_dense_brute_force, pin_topk_all_uniform_is_mean, pin_identical_experts,
             pin_single_expert_is_swiglu_mlp, pin_linear_in_down_proj, pin_worked_example]
+
+
+# ------------------------------------------------------------- FP8 variant
+
+def _e4m3_torch(v):
+    """Library rounding: torch's float8_e4m3fn cast (values already in +-448)."""
+    return torch.as_tensor(np.asarray(v, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def pin_e4m3_codes_vs_torch(orc):
+    """Decoding every finite code matches torch's float8_e4m3fn -> float; encoding matches
+    torch's cast on random values, on every exact midpoint between neighbouring codes
+    (ties to even) and on the subnormal range."""
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    dec = orc.e4m3_decode(codes)
+    ref = torch.as_tensor(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(dec, ref)
+    pos = np.sort(np.unique(np.abs(dec)))
+    mids = (pos[:-1] + pos[1:]) / 2
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([mids, -mids, pos, -pos, rng.uniform(-448, 448, 5000),
+                           rng.uniform(-0.02, 0.02, 2000), [0.0, -0.0, 448.0, -448.0]]).astype(np.float32)
+    assert np.array_equal(orc.e4m3_encode(vals), _e4m3_torch(vals))
+
+
+def pin_quantize_rows(orc):
+    """Row/128-group quantiser: scale = amax/448 in fp32, codes = e4m3(clamp(v/s)) (torch
+    cast as the rounding routine), round-trip error within half an e4m3 step, a zero
+    group gives scale 1 and zero codes."""
+    rng = np.random.default_rng(5)
+    a = torch.as_tensor(rng.standard_normal((6, 384)).astype(np.float32)).to(torch.bfloat16)
+    a[2, 128:256] = 0.0
+    a[4, :] *= 1e-3
+    q, s = orc.quantize_rows(a)
+    f = a.float().view(6, 3, 128)
+    amax = f.abs().amax(-1)
+    s_ref = torch.where(amax == 0, torch.ones_like(amax), amax / 448.0)
+    assert np.array_equal(s, s_ref.numpy())
+    r = (f / s_ref[..., None]).clamp(-448, 448)
+    assert np.array_equal(q, _e4m3_torch(r.reshape(6, 384).numpy()))
+    assert np.all(q[2, 128:256] == 0) and s[2, 1] == 1.0
+    deq = torch.as_tensor(q).view(torch.float8_e4m3fn).double().view(6, 3, 128) * torch.as_tensor(s).double()[..., None]
+    err = (deq - f.double()).abs()
+    assert torch.all(err <= (f.double().abs() * 2.0 ** -4 + torch.as_tensor(s).double()[..., None] * 2.0 ** -10))
+
+
+def _fp8_case(E=3, H=256, I=256, T=10, k=2, seed=9):
+    from routed_grouped_gemm_softmax_b200.inputs import make_fp8_weights
+    cfg = CONFIGS["fp8"].replace(E=E, H=H, I=I, T=T, top_k=k, seed=seed)
+    inp = make_inputs(cfg, weights=False)
+    return cfg, inp, make_fp8_weights(cfg)
+
+
+def _fp8_dense_reference(inp, w, idx, gate):
+    """Brute force: dequantise every weight to fp64 (torch float8 -> float), quantise x and
+    h with torch casts, run dense fp64 matmuls for every expert, mask by the gates."""
+    def deq(q, s):
+        E, N, K = q.shape
+        v = q.view(torch.float8_e4m3fn).double().view(E, N // 128, 128, K // 128, 128)
+        return (v * s.double()[:, :, None, :, None]).view(E, N, K)
+
+    def quant_rows(m32):  # m32: fp32 [R, K] -> dequantised fp64 [R, K]
+        R, K = m32.shape
+        g = m32.view(R, K // 128, 128)
+        amax = g.abs().amax(-1)
+        s = torch.where(amax == 0, torch.ones_like(amax), amax / 448.0)
+        qq = (g / s[..., None]).clamp(-448, 448).to(torch.float8_e4m3fn)
+        return (qq.double() * s.double()[..., None]).view(R, K)
+
+    Wg, Wu, Wd = deq(w["w_gate_q"], w["w_gate_s"]), deq(w["w_up_q"], w["w_up_s"]), deq(w["w_down_q"], w["w_down_s"])
+    X = quant_rows(inp.x.float())
+    T, E = X.shape[0], Wg.shape[0]
+    G = torch.zeros(T, E, dtype=torch.float64)
+    for t in range(T):
+        for j in range(idx.shape[1]):
+            G[t, int(idx[t, j])] += float(gate[t, j])
+    out = torch.zeros(T, X.shape[1], dtype=torch.float64)
+    for e in range(E):
+        h = (F.silu(X @ Wg[e].T) * (X @ Wu[e].T)).float()
+        out += G[:, e:e + 1] * (quant_rows(h) @ Wd[e].T)
+    return out.numpy()
+
+
+def pin_fp8_ffn_dense_brute_force(orc):
+    """FP8 layer: the oracle's blockwise sums equal the dense dequantise-then-matmul
+    evaluation (torch casts for every quantisation decision) on a small case."""
+    cfg, inp, w = _fp8_case()
+    idx, gate = orc.route(inp.x, inp.router_w, None, cfg.top_k)
+    out = orc.combine_ffn_fp8(inp.x, idx, gate, w["w_gate_q"], w["w_gate_s"], w["w_up_q"], w["w_up_s"],
+                              w["w_down_q"], w["w_down_s"])
+    ref = _fp8_dense_reference(inp, w, idx, gate)
+    assert np.allclose(out, ref, rtol=1e-9, atol=1e-12), np.abs(out - ref).max()
+
+
+def pin_fp8_close_to_unquantised(orc):
+    """The fp8 layer approximates the unquantised layer on the same master weights
+    (bf16 copies): relative L2 error of a few percent, far below 1."""
+    cfg, inp, w = _fp8_case(T=16)
+    full = make_inputs(cfg)
+    idx, gate = orc.route(inp.x, inp.router_w, None, cfg.top_k)
+    a = orc.combine_ffn_fp8(inp.x, idx, gate, w["w_gate_q"], w["w_gate_s"], w["w_up_q"], w["w_up_s"],
+                            w["w_down_q"], w["w_down_s"])
+    b = orc.combine_ffn(inp.x, idx, gate, full.w_gate.to(torch.bfloat16), full.w_up.to(torch.bfloat16),
+                        full.w_down.to(torch.bfloat16))
+    rel = np.linalg.norm(a - b) / np.linalg.norm(b)
+    assert 1e-3 < rel < 0.08, rel
+
+
+ALL_PINS += [pin_e4m3_codes_vs_torch, pin_quantize_rows, pin_fp8_ffn_dense_brute_force,
+             pin_fp8_close_to_unquantised]

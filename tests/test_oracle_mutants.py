@@ -28,6 +28,11 @@ MUTANTS = {
                               "        for (int h = H - 1; h >= 0; --h) {\n            float a"),
     "tile_rows_not_clipped": ("(c - r) < bm ? (c - r) : bm", "bm"),
     "permute_offsets_shifted": ("offsets[e] = pos;", "offsets[e] = pos + (e > 0);"),
+    "e4m3_tie_away": ("(d == bd && (c & 1) == 0 && (best & 1) == 1)", "(d == bd && c > best)"),
+    "fp8_scale_transposed": ("sb[(size_t)(n / 128) * KB + kb]", "sb[(size_t)kb * (N / 128) + n / 128]"),
+    "fp8_act_scale_dropped": ("acc += (double)sa[kb] * (double)sb", "acc += (double)sb"),
+    "fp8_amax_448_off": ("float s = amax / 448.0f;", "float s = amax / 440.0f;"),
+    "fp8_h_not_requantised": ("fp8_row_gemm(H, I, qh, sh,", "fp8_row_gemm(H, I, qh, sx,"),
 }
 
 
