@@ -34,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_fp8_weights, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at 1 B200; % of BF16/FP8 TC peak or % of HBM BW"
 KERNELS_PER_FORWARD = 9   # logits, top-k, count, scan, scatter, gather, GEMM x2, combine
@@ -203,25 +203,32 @@ def max_over_ranks(v: float, world: int) -> float:
 
 def stage_work(cfg, counts):
     """Algorithmic bytes and FLOPs of each stage for the realised routing (counts[e] =
-    rows of expert e).  Intermediates a fused design would not write are excluded only
-    where the stage's own definition does not need them."""
+    rows of expert e).  Weight bytes count only the touched experts; fp8 weights and
+    activations take one byte per element plus one fp32 scale per 128x128 weight
+    block or per 128 activation values."""
     T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k
     A = T * k
     D = int(sum(1 for c in counts if c > 0))
+    fp8 = cfg.dtype == "fp8"
+    wb = 1 if fp8 else 2
+    wsc = (lambda n, kk: (n // 128) * (kk // 128) * 4) if fp8 else (lambda n, kk: 0)
+    ab = (lambda n: n + n // 128 * 4) if fp8 else (lambda n: 2 * n)   # activation bytes of n values
     return {
         "route": {"bytes": T * H * 2 + H * E * 2 + A * 8, "flops": 2.0 * T * H * E, "alu": True},
-        "gemm_gate_up": {"bytes": D * 2 * I * H * 2 + A * H * 2 + A * I * 2, "flops": 2.0 * A * H * 2 * I},
-        "gemm_down": {"bytes": D * H * I * 2 + A * I * 2 + A * H * 2, "flops": 2.0 * A * I * H},
+        "gemm_gate_up": {"bytes": D * (2 * I * H * wb + 2 * wsc(I, H)) + ab(A * H) + ab(A * I),
+                         "flops": 2.0 * A * H * 2 * I},
+        "gemm_down": {"bytes": D * (H * I * wb + wsc(H, I)) + ab(A * I) + A * H * 2, "flops": 2.0 * A * I * H},
         "combine": {"bytes": A * H * 2 + A * 4 + T * H * 2, "flops": 2.0 * A * H},
         "_D": D,
     }
 
 
-def roofline_for(stage, work, ms, peaks, peaks_kind, sustained, workload):
+def roofline_for(stage, work, ms, peaks, peaks_kind, sustained, workload, fp8=False):
     w = work[stage]
     t = ms * 1e-3
     bw_time = w["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    pk_tf = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    # fp8 tensor peak = measured bf16 peak x the nominal fp8/bf16 ratio (4.5 / 2.25 PF)
+    pk_tf = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * (2.0 if fp8 else 1.0)
     tc_time = w["flops"] / (pk_tf * 1e12)
     if w.get("alu") or bw_time >= tc_time:
         achieved = w["bytes"] / t / 1e9
@@ -234,14 +241,15 @@ def roofline_for(stage, work, ms, peaks, peaks_kind, sustained, workload):
     r["kernel"] = stage
     r["algorithmic_bytes"] = w["bytes"]
     r["algorithmic_flops"] = w["flops"]
-    r["peak_source"] = f"{peaks_kind}" + ("" if r["bound"] == "hbm" else (" sustained" if sustained else " burst"))
+    r["peak_source"] = f"{peaks_kind}" + ("" if r["bound"] == "hbm" else (" sustained" if sustained else " burst")
+                                          + (" bf16 x 2 (nominal fp8/bf16 ratio)" if fp8 else ""))
     r["ms"] = round(ms, 4)
     return r
 
 
 # ------------------------------------------------------------- CPU oracle leg
 
-def host_inputs(cfg, inp=None):
+def host_inputs(cfg, inp=None, w8=None):
     """The workload's tensors as host numpy arrays (bf16 bit patterns), drawn on the GPU
     when one is present (data preparation only; nothing of the layer runs there)."""
     import types
@@ -252,10 +260,16 @@ def host_inputs(cfg, inp=None):
 
     def bits(t):
         return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-    return types.SimpleNamespace(
+    ns = types.SimpleNamespace(
         x=bits(inp.x), router_w=bits(inp.router_w),
-        bias=None if inp.bias is None else inp.bias.detach().cpu().float().numpy(),
-        w_gate=bits(inp.w_gate), w_up=bits(inp.w_up), w_down=bits(inp.w_down))
+        bias=None if inp.bias is None else inp.bias.detach().cpu().float().numpy(), fp8=None)
+    if cfg.dtype == "fp8":
+        if w8 is None:
+            w8 = make_fp8_weights(cfg, device=inp.x.device)
+        ns.fp8 = {k: v.detach().cpu().numpy() for k, v in w8.items()}
+    else:
+        ns.w_gate, ns.w_up, ns.w_down = bits(inp.w_gate), bits(inp.w_up), bits(inp.w_down)
+    return ns
 
 
 def oracle_step_timer(cfg, h):
@@ -272,7 +286,12 @@ def oracle_step_timer(cfg, h):
         idx, gate = oracle.route(h.x, h.router_w, h.bias, cfg.top_k, nthreads=threads)
         t1 = time.perf_counter()
         tok = np.sort(rng.choice(cfg.T, size=n, replace=False)).astype(np.int32)
-        oracle.combine_ffn(h.x, idx, gate, h.w_gate, h.w_up, h.w_down, tokens=tok, nthreads=threads)
+        if h.fp8 is not None:
+            f = h.fp8
+            oracle.combine_ffn_fp8(h.x, idx, gate, f["w_gate_q"], f["w_gate_s"], f["w_up_q"], f["w_up_s"],
+                                   f["w_down_q"], f["w_down_s"], tokens=tok, nthreads=threads)
+        else:
+            oracle.combine_ffn(h.x, idx, gate, h.w_gate, h.w_up, h.w_down, tokens=tok, nthreads=threads)
         t2 = time.perf_counter()
         return t1 - t0, t2 - t1
     return run, threads
@@ -334,6 +353,7 @@ def run_reference(args, world, rank):
 
 def config_block(cfg, world):
     return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.top_k,
+            "weights": "e4m3 + fp32 128x128 block scales" if cfg.dtype == "fp8" else "bf16",
             "seed": cfg.seed, "router_bias": "zipf(1.2)" if cfg.zipf_s else None,
             "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
             "l2": "flushed before every step (512 MiB write, outside the step's events)",
@@ -354,17 +374,24 @@ def main():
     cfg = workload_config(args)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    inp = make_inputs(cfg, device=dev)
+    fp8 = cfg.dtype == "fp8"
+    inp = make_inputs(cfg, device=dev, weights=not fp8)
     x, rw, bias = inp.x, inp.router_w, inp.bias
-    wg, wu, wd = inp.w_gate, inp.w_up, inp.w_down
     k = cfg.top_k
-    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, dev)
+    if fp8:
+        w8 = make_fp8_weights(cfg, device=dev)
+        wq = (w8["w_gate_q"], w8["w_gate_s"], w8["w_up_q"], w8["w_up_s"], w8["w_down_q"], w8["w_down_s"])
+        forward = lambda xx, st: api.moe_forward_fp8(xx, rw, bias, *wq, k, out=out, ws=ws, stream=st)
+    else:
+        wg, wu, wd = inp.w_gate, inp.w_up, inp.w_down
+        forward = lambda xx, st: api.moe_forward(xx, rw, bias, wg, wu, wd, k, out=out, ws=ws, stream=st)
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, dev, api.DTYPE_FP8 if fp8 else api.DTYPE_BF16)
     out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        api.moe_forward(x, rw, bias, wg, wu, wd, k, out=out, ws=ws, stream=stream)
+        forward(x, stream)
 
     # events: one set of 6 stage marks per timed step (the first and last bracket the step)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
@@ -389,7 +416,7 @@ def main():
             for i in range(args.steps):
                 flush.fill_(1)
                 api.set_stage_events(ev[i])
-                api.moe_forward(x, rw, bias, wg, wu, wd, k, out=out, ws=ws, stream=cap)
+                forward(x, cap)
     api.set_stage_events(None)
     stream.wait_stream(cap)
     graph.replay()  # one untimed replay so the timed one starts warm
@@ -426,10 +453,10 @@ def main():
     peaks, peaks_kind = load_peaks()
     dominant = max(("route", "gemm_gate_up", "gemm_down", "combine"), key=lambda s: stage_ms[s])
     sustained = total_ms > 1000.0
-    roof = roofline_for(dominant, work, stage_ms[dominant], peaks, peaks_kind, sustained, cfg.name)
+    roof = roofline_for(dominant, work, stage_ms[dominant], peaks, peaks_kind, sustained, cfg.name, fp8)
     stages = {s: {"ms": round(stage_ms[s], 4)} for s in api.STAGES}
     for s in ("route", "gemm_gate_up", "gemm_down", "combine"):
-        r = roofline_for(s, work, stage_ms[s], peaks, peaks_kind, sustained, cfg.name)
+        r = roofline_for(s, work, stage_ms[s], peaks, peaks_kind, sustained, cfg.name, fp8)
         stages[s].update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
 
     # end to end through the public API with host buffers
@@ -447,7 +474,7 @@ def main():
             flush.fill_(1)
             a.record(stream)
             x_dev.copy_(x_host, non_blocking=True)
-            api.moe_forward(x_dev, rw, bias, wg, wu, wd, k, out=out, ws=ws, stream=stream)
+            forward(x_dev, stream)
             out_host.copy_(out, non_blocking=True)
             b.record(stream)
         torch.cuda.synchronize()
@@ -459,12 +486,13 @@ def main():
     clocks = sampler.summary(t_wall0, t_wall1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(cfg, host_inputs(cfg, inp))
+        cpu = cpu_baseline(cfg, host_inputs(cfg, inp, w8 if fp8 else None))
 
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 5),
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "e4m3" if fp8 else "bf16",
                 "data": "synthetic", "config": config_block(cfg, world),
                 "roofline": roof, "stages": stages, "experts_touched": work["_D"],
                 "e2e": e2e, "gpu_launches": KERNELS_PER_FORWARD * args.steps,

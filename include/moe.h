@@ -78,7 +78,7 @@ typedef struct {
     int32_t top_k;  /* experts per token */
 } moe_dims_t;
 
-enum { MOE_DTYPE_BF16 = 0 };
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8 = 1 };
 
 /* Rows of the GEMM tiles; tile_list entries cover at most this many rows. */
 #define MOE_TILE_ROWS 128
@@ -125,6 +125,30 @@ moe_status_t moe_permute(const moe_dims_t *d, const int32_t *topk_idx, int32_t *
 moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_w,
                          const float *router_bias, const void *w_gate, const void *w_up,
                          const void *w_down, void *out, void *ws, size_t ws_bytes, void *stream);
+
+/* FP8 block-scaled layer (GC-MoE page: block-scaled FP8 MMA on Blackwell with
+ * SwiGLU and requantisation fused; vLLM fused-MoE page, section 03: fp8 weights
+ * in [128,128] blocks).  Routing is the bf16 router of moe_route.  Weights are
+ * e4m3 codes (uint8, OCP "fn" encoding) with one fp32 scale per 128x128 block:
+ *   w_gate_q / w_up_q [E, I, H] with w_gate_s / w_up_s [E, I/128, H/128],
+ *   w_down_q [E, H, I] with w_down_s [E, H/128, I/128].
+ * x (bf16) is quantised per token per 128 columns: s = amax/448 (s = 1 for an
+ * all-zero group), q = e4m3 round-to-nearest-even of clamp(v/s, -448, 448);
+ * each GEMM is sum over 128-wide K blocks of s_x * s_w * (codes . codes) in fp32
+ * on the tensor cores (kind::f8f6f4) with the scaling applied per K block; h =
+ * silu(gate) * up is requantised the same way; the down GEMM's per-assignment
+ * rows are rounded to bf16 and combined as in moe_forward; out is bf16.
+ * Needs H and I multiples of 128 and ws_bytes >= moe_workspace_size(d,
+ * MOE_DTYPE_FP8); other rules as moe_forward. */
+moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *router_w,
+                             const float *router_bias, const uint8_t *w_gate_q, const float *w_gate_s,
+                             const uint8_t *w_up_q, const float *w_up_s, const uint8_t *w_down_q,
+                             const float *w_down_s, void *out, void *ws, size_t ws_bytes, void *stream);
+
+/* The activation quantiser of moe_forward_fp8 on its own: a [R, K] bf16 (K a
+ * multiple of 128, 16-byte aligned) -> q [R, K] e4m3 codes and s [R, K/128]
+ * fp32 scales, per row per 128 columns as described above.  Needs no workspace. */
+moe_status_t moe_quantize_rows_fp8(int32_t R, int32_t K, const void *a, uint8_t *q, float *s, void *stream);
 
 /* Synchronises `stream`, returns the device status word of the workspace
  * (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_BAD_INDEX; MOE_ERR_CUDA if the stream

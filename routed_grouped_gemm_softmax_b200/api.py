@@ -20,7 +20,9 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 6: "MOE_ERR_BAD_INDEX", 7: "MOE_ERR_TOO_LARGE"}
 EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "moe_forward",
            "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order",
-           "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us"]
+           "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",
+           "moe_forward_fp8", "moe_quantize_rows_fp8"]
+DTYPE_BF16, DTYPE_FP8 = 0, 1
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
 TILE_ROWS = 128
@@ -67,6 +69,10 @@ def lib():
         L.moe_set_claim_order.restype = None
         L.moe_set_stage_events.argtypes = [P, I32]
         L.moe_set_stage_events.restype = None
+        L.moe_forward_fp8.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_forward_fp8.restype = ctypes.c_int
+        L.moe_quantize_rows_fp8.argtypes = [I32, I32, P, P, P, P]
+        L.moe_quantize_rows_fp8.restype = ctypes.c_int
         L.moe_set_wait_limit_us.argtypes = [I32, I32]
         L.moe_set_wait_limit_us.restype = None
         L.moe_forward_noalloc.argtypes = [D, P, P, P, P, P, P, P, P]
@@ -100,16 +106,16 @@ def dims(T, H, I, E, top_k) -> Dims:
     return Dims(int(T), int(H), int(I), int(E), int(top_k))
 
 
-def moe_workspace_size(T, H, I, E, top_k) -> int:
-    return int(lib().moe_workspace_size(ctypes.byref(dims(T, H, I, E, top_k)), 0))
+def moe_workspace_size(T, H, I, E, top_k, dtype: int = DTYPE_BF16) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(dims(T, H, I, E, top_k)), int(dtype)))
 
 
 def moe_max_tiles(T, H, I, E, top_k) -> int:
     return int(lib().moe_max_tiles(ctypes.byref(dims(T, H, I, E, top_k))))
 
 
-def workspace(T, H, I, E, top_k, device) -> torch.Tensor:
-    n = moe_workspace_size(T, H, I, E, top_k)
+def workspace(T, H, I, E, top_k, device, dtype: int = DTYPE_BF16) -> torch.Tensor:
+    n = moe_workspace_size(T, H, I, E, top_k, dtype)
     if n == 0:
         raise MoEError(1, "moe_workspace_size")
     return torch.empty(n, dtype=torch.uint8, device=device)
@@ -175,6 +181,45 @@ def moe_forward(x, router_w, bias, w_gate, w_up, w_down, top_k: int, out=None, w
                              _p(w_down), _p(out), _p(ws), ws.numel(), _stream(stream, dev)),
            "moe_forward")
     return out
+
+
+def moe_forward_fp8(x, router_w, bias, w_gate_q, w_gate_s, w_up_q, w_up_s, w_down_q, w_down_s,
+                    top_k: int, out=None, ws=None, stream=None):
+    """The FP8 block-scaled layer; weights are uint8 e4m3 codes with fp32 128x128 block
+    scales; returns out bf16 [T,H]."""
+    T, H = x.shape
+    E, I, _ = w_gate_q.shape
+    dev = x.device
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(router_w, torch.bfloat16, (H, E), "router_w")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "router_bias")
+    for t, shp, nm in ((w_gate_q, (E, I, H), "w_gate_q"), (w_up_q, (E, I, H), "w_up_q"),
+                       (w_down_q, (E, H, I), "w_down_q")):
+        _need(t, torch.uint8, shp, nm)
+    for t, shp, nm in ((w_gate_s, (E, I // 128, H // 128), "w_gate_s"), (w_up_s, (E, I // 128, H // 128), "w_up_s"),
+                       (w_down_s, (E, H // 128, I // 128), "w_down_s")):
+        _need(t, torch.float32, shp, nm)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    _need(out, torch.bfloat16, (T, H), "out")
+    ws = workspace(T, H, I, E, top_k, dev, DTYPE_FP8) if ws is None else ws
+    d = dims(T, H, I, E, top_k)
+    _check(lib().moe_forward_fp8(ctypes.byref(d), _p(x), _p(router_w), _p(bias), _p(w_gate_q), _p(w_gate_s),
+                                 _p(w_up_q), _p(w_up_s), _p(w_down_q), _p(w_down_s), _p(out), _p(ws),
+                                 ws.numel(), _stream(stream, dev)), "moe_forward_fp8")
+    return out
+
+
+def moe_quantize_rows_fp8(a, q=None, s=None, stream=None):
+    """Per-row, per-128-column e4m3 quantisation of a bf16 [R,K] matrix on the GPU:
+    returns (codes uint8 [R,K], scales fp32 [R,K/128])."""
+    R, K = a.shape
+    _need(a, torch.bfloat16, (R, K), "a")
+    q = torch.empty((R, K), dtype=torch.uint8, device=a.device) if q is None else q
+    s = torch.empty((R, K // 128), dtype=torch.float32, device=a.device) if s is None else s
+    _check(lib().moe_quantize_rows_fp8(int(R), int(K), _p(a), _p(q), _p(s), _stream(stream, a.device)),
+           "moe_quantize_rows_fp8")
+    return q, s
 
 
 def moe_forward_noalloc(x, router_w, bias, w_gate, w_up, w_down, top_k: int, out=None, stream=None):

@@ -1,0 +1,398 @@
+// fp8.cu -- the FP8 block-scaled variant of the layer on sm_100a.
+//
+// Weights arrive as e4m3 codes with one fp32 scale per 128x128 block;
+// activations are quantised per row per 128 columns (x before the gate/up GEMM,
+// h after SwiGLU) with s = amax/448 and q = e4m3_rn(clamp(v/s, +-448)).  The
+// GC-MoE page describes this family of kernels on Blackwell: block-scaled tcgen05
+// MMA with SwiGLU and requantisation fused into the GEMM; the vLLM page
+// (section 03) lists fp8 configs with [128,128] weight blocks.
+//
+// Hardware block scaling (kind::mxf8f6f4) takes one power-of-two scale per 32
+// elements, which cannot hold these fp32 per-128 scales.  So each 128-wide K
+// block is one MMA group of kind::f8f6f4 (4 x K=32) into a fresh TMEM buffer,
+// and the epilogue warps promote it: acc += (s_a[row,kb] * s_b[nblk,kb]) * P_kb,
+// in fp32 registers, while the tensor cores fill the other TMEM buffer.
+//
+// CTA roles (320 threads): warp 0 claims work items and streams 128x128-byte A
+// tiles and 256x128-byte B tiles with TMA (one stage = one K block); warp 1 owns
+// TMEM and issues the MMAs; warps 2-9 are the epilogue, two warps per TMEM lane
+// quarter, each owning 128 of the 256 accumulator columns of its rows.
+// Mode 0 (gate/up): columns 0-127 are gate, 128-255 up, of the same 128 rows of
+// I; a thread owns 64 gate + 64 up columns, forms h = silu(g) * u, and the two
+// warps sharing a row exchange their partial amax through shared memory to
+// quantise the 128-column group.  Mode 1 (down): y rows in bf16.
+// Every wait is bounded, as in the bf16 kernel.
+#include <cuda_fp8.h>
+
+#include <mutex>
+
+#include "moe_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = kTileRows;
+constexpr int BKB = 128;                // bytes (= e4m3 elements) of K per stage
+constexpr int BN = 256;
+constexpr int STAGES = 4;
+constexpr int RING = 4;
+constexpr int A_BYTES = BM * BKB;       // 16 KB
+constexpr int B_BYTES = BN * BKB;       // 32 KB
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct Ctrl8 {
+    uint64_t full[STAGES], empty[STAGES];
+    uint64_t accf[2], acce[2];
+    uint64_t itf[RING], ite[RING];
+    uint64_t xbar[4];  // per lane quarter: the two epilogue warps of those rows
+    uint64_t fin, never;
+    int32_t ring[RING];
+    uint32_t tmem_base;
+    float xam[2][2][BM];  // [item parity][half][row]: partial amax of h
+};
+
+constexpr size_t SMEM8 = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + sizeof(Ctrl8);
+
+__device__ __forceinline__ void record(int32_t *status, int code) { atomicCAS(status, 0, code); }
+
+__device__ __forceinline__ float silu(float a) { return a / (1.0f + __expf(-a)); }
+
+// e4m3 code of v / s, round to nearest even, clamped to +-448.
+__device__ __forceinline__ uint32_t e4m3_pair(float a, float b)
+{
+    const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+    return static_cast<uint32_t>(p);
+}
+
+__device__ __forceinline__ float qdiv(float v, float s)
+{
+    return fminf(fmaxf(__fdiv_rn(v, s), -448.0f), 448.0f);
+}
+
+// kind::f8f6f4 instruction descriptor: e4m3 A and B (K-major), fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
+{
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+
+// ------------------------------------------------------------ quantiser
+
+// Rows of a bf16 matrix quantised per 128-column group.  Row r reads source row
+// map ? map[r] / k : r, so the same kernel gathers x into expert order.  One warp
+// per row; lane l holds elements 4l..4l+3 of the current group.
+__global__ void quantize_rows_kernel(const __nv_bfloat16 *__restrict__ src, const int32_t *__restrict__ map,
+                                     int k, int R, int K, uint8_t *__restrict__ q, float *__restrict__ s)
+{
+    const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= R) return;
+    const int sr = map ? map[row] / k : row;
+    const __nv_bfloat16 *a = src + (size_t)sr * K;
+    for (int g = 0; g < K / 128; ++g) {
+        const uint2 raw = *reinterpret_cast<const uint2 *>(a + g * 128 + lane * 4);
+        const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+        const float2 v01 = __bfloat1622float2(p[0]), v23 = __bfloat1622float2(p[1]);
+        float m = fmaxf(fmaxf(fabsf(v01.x), fabsf(v01.y)), fmaxf(fabsf(v23.x), fabsf(v23.y)));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        uint32_t packed = 0;
+        float sc = 1.0f;
+        if (m != 0.0f) {
+            sc = __fdiv_rn(m, 448.0f);
+            packed = e4m3_pair(qdiv(v01.x, sc), qdiv(v01.y, sc)) | (e4m3_pair(qdiv(v23.x, sc), qdiv(v23.y, sc)) << 16);
+        }
+        *reinterpret_cast<uint32_t *>(q + (size_t)row * K + g * 128 + lane * 4) = packed;
+        if (lane == 0) s[(size_t)row * (K / 128) + g] = sc;
+    }
+}
+
+// ----------------------------------------------------------- grouped GEMM
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const Fp8GemmArgs g)
+{
+    constexpr int BNO = MODE == 0 ? BN / 2 : BN;  // output columns per tile
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    uint8_t *sA = smem_raw + pad;
+    uint8_t *sB = sA + STAGES * A_BYTES;
+    Ctrl8 *S = reinterpret_cast<Ctrl8 *>(sB + STAGES * B_BYTES);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int n_tiles = (g.N + BNO - 1) / BNO;
+    const int KB = g.K / BKB;
+    const int NB = g.N / 128;  // 128-row weight blocks along N
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&S->full[s], 1);
+            mbar_init(&S->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&S->accf[a], 1);
+            mbar_init(&S->acce[a], EPI_WARPS);
+        }
+        for (int r = 0; r < RING; ++r) {
+            mbar_init(&S->itf[r], 1);
+            mbar_init(&S->ite[r], 1 + EPI_WARPS);
+        }
+        for (int q = 0; q < 4; ++q) mbar_init(&S->xbar[q], 2);
+        mbar_init(&S->fin, 1);
+        mbar_init(&S->never, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB0);
+        if (MODE == 0) tma_prefetch_desc(&tmB1);
+    }
+    if (warp == 1) tmem_alloc(&S->tmem_base, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------ scheduler + TMA producer
+        if (lane == 0) {
+            const int total = *g.ntiles * n_tiles;
+            int stage = 0, rs = 0;
+            uint32_t phase = 0, rphase = 0, armed = 0, armed_par = 0;
+            bool ok = true;
+            for (;;) {
+                int item = atomicAdd(g.counter, 1);
+                if (item >= total)
+                    item = -1;
+                else if (g.reverse)
+                    item = total - 1 - item;
+                if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
+                S->ring[rs] = item;
+                mbar_arrive(&S->itf[rs]);
+                if (++rs == RING) { rs = 0; rphase ^= 1; }
+                if (item < 0) break;
+                const int mt = item / n_tiles, nt = item - mt * n_tiles;
+                const int expert = g.tiles[3 * mt], row0 = g.tiles[3 * mt + 1];
+                const int n0 = nt * BNO;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&S->full[stage], A_BYTES + B_BYTES);
+                    armed |= 1u << stage;
+                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                    uint8_t *b_dst = sB + stage * B_BYTES;
+                    tma_load_2d(sA + stage * A_BYTES, &tmA, &S->full[stage], kb * BKB, row0);
+                    tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BKB, n0, expert);
+                    if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BKB, n0, expert);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (!ok) {
+                record(g.status, MOE_ERR_TIMEOUT);
+                if (mbar_wait(&S->ite[rs], rphase ^ 1)) {
+                    S->ring[rs] = -1;
+                    mbar_arrive(&S->itf[rs]);
+                }
+            }
+            for (int s = 0; s < STAGES; ++s)
+                if ((armed >> s) & 1u)
+                    if (!mbar_wait(&S->full[s], (armed_par >> s) & 1u)) record(g.status, MOE_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
+            int stage = 0, rs = 0, acc = 0;
+            uint32_t phase = 0, rphase = 0, aphase = 0;
+            bool ok = !(g.stall_test && !mbar_wait(&S->never, 0, g.wait_ns));
+            while (ok) {
+                if (!mbar_wait(&S->itf[rs], rphase, g.wait_ns)) { ok = false; break; }
+                const int item = S->ring[rs];
+                mbar_arrive(&S->ite[rs]);
+                if (++rs == RING) { rs = 0; rphase ^= 1; }
+                if (item < 0) break;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&S->acce[acc], aphase ^ 1, g.wait_ns)) { ok = false; break; }
+                    tc_fence_after();
+                    if (!mbar_wait(&S->full[stage], phase, g.wait_ns)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
+                    const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+                    const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BKB / 32; ++k)
+                        mma_e4m3(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), IDESC, k != 0);
+                    mma_commit(&S->empty[stage]);
+                    mma_commit(&S->accf[acc]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (++acc == 2) { acc = 0; aphase ^= 1; }
+                }
+            }
+            if (!ok) record(g.status, MOE_ERR_TIMEOUT);
+            mma_commit(&S->fin);
+            if (!mbar_wait(&S->fin, 0)) record(g.status, MOE_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;             // TMEM lane quarter
+        const int half = (warp - 2) / 4;    // which 128 accumulator columns
+        const int row = q * 32 + lane;
+        int rs = 0, acc = 0;
+        uint32_t rphase = 0, aphase = 0, xphase = 0;
+        int parity = 0;
+        for (;;) {
+            if (!mbar_wait(&S->itf[rs], rphase, g.wait_ns)) { record(g.status, MOE_ERR_TIMEOUT); break; }
+            const int item = S->ring[rs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S->ite[rs]);
+            if (++rs == RING) { rs = 0; rphase ^= 1; }
+            if (item < 0) break;
+            const int mt = item / n_tiles, nt = item - mt * n_tiles;
+            const int expert = g.tiles[3 * mt], row0 = g.tiles[3 * mt + 1], rows = g.tiles[3 * mt + 2];
+            const bool row_ok = row < rows;
+            const int n0 = nt * BNO;
+            const float *sa = g.sa + (size_t)(row0 + (row_ok ? row : 0)) * KB;
+            // weight-scale rows of the 128-row blocks this thread's columns fall in
+            const int nb0 = MODE == 0 ? n0 / 128 : n0 / 128 + half;
+            const bool nb_ok = nb0 < NB;
+            const float *sb0 = g.sb0 + ((size_t)expert * NB + (nb_ok ? nb0 : 0)) * KB;
+            const float *sb1 = MODE == 0 ? g.sb1 + ((size_t)expert * NB + nb0) * KB : sb0;
+
+            float accr[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) accr[i] = 0.0f;
+            bool ok = true;
+            for (int kb = 0; kb < KB; ++kb) {
+                const float a_s = row_ok ? sa[kb] : 0.0f;
+                const float c0 = nb_ok ? a_s * sb0[kb] : 0.0f;
+                const float c1 = MODE == 0 ? a_s * sb1[kb] : c0;
+                if (!mbar_wait(&S->accf[acc], aphase, g.wait_ns)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    // mode 0: chunks 0-3 = gate columns, 4-7 = up columns of this half
+                    const int col = MODE == 0 ? (c < 4 ? half * 64 + c * 16 : 128 + half * 64 + (c - 4) * 16)
+                                              : half * 128 + c * 16;
+                    const float cs = (MODE == 0 && c >= 4) ? c1 : c0;
+                    uint32_t r[16];
+                    tmem_ld16_sync(tb + col, r);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) accr[c * 16 + i] = fmaf(cs, __uint_as_float(r[i]), accr[c * 16 + i]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S->acce[acc]);
+                if (++acc == 2) { acc = 0; aphase ^= 1; }
+            }
+            if (!ok) { record(g.status, MOE_ERR_TIMEOUT); break; }
+
+            if (MODE == 0) {
+                // h = silu(gate) * up for this thread's 64 columns, then the 128-column
+                // group's amax from both halves, then e4m3 codes and the group scale.
+                float m = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    accr[i] = silu(accr[i]) * accr[64 + i];
+                    m = fmaxf(m, fabsf(accr[i]));
+                }
+                S->xam[parity][half][row] = m;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S->xbar[q]);
+                if (!mbar_wait(&S->xbar[q], xphase, g.wait_ns)) { record(g.status, MOE_ERR_TIMEOUT); break; }
+                xphase ^= 1;
+                const float amax = fmaxf(S->xam[parity][0][row], S->xam[parity][1][row]);
+                parity ^= 1;
+                const float sc = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+                const int col = n0 + half * 64;
+                if (row_ok && col < g.N) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = amax == 0.0f ? 0u
+                                             : e4m3_pair(qdiv(accr[4 * i], sc), qdiv(accr[4 * i + 1], sc)) |
+                                                   (e4m3_pair(qdiv(accr[4 * i + 2], sc), qdiv(accr[4 * i + 3], sc)) << 16);
+                    uint4 *dst = reinterpret_cast<uint4 *>(g.out_q + (size_t)(row0 + row) * g.N + col);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    if (half == 0) g.out_s[(size_t)(row0 + row) * NB + n0 / 128] = sc;
+                }
+            } else {
+                const int col = n0 + half * 128;
+                if (row_ok && col < g.N) {
+                    const int flat = g.row_map[row0 + row];
+                    uint4 *dst = reinterpret_cast<uint4 *>(g.out + (size_t)flat * g.N + col);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 v[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) v[j] = __floats2bfloat162_rn(accr[8 * i + 2 * j], accr[8 * i + 2 * j + 1]);
+                        dst[i] = *reinterpret_cast<uint4 *>(v);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+bool fp8_smem_attr_ready(int mode)
+{
+    static std::mutex mu;
+    static uint64_t done[2] = {0, 0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    if (done[mode] >> dev & 1ull) return true;
+    cudaError_t e = mode == 0 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM8)
+                              : cudaFuncSetAttribute(grouped_gemm_fp8_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM8);
+    if (e != cudaSuccess) return false;
+    done[mode] |= 1ull << dev;
+    return true;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_rows(const __nv_bfloat16 *src, const int32_t *map, int k, int R, int K, uint8_t *q,
+                                 float *s, cudaStream_t st)
+{
+    const int rows_per_block = 8;
+    quantize_rows_kernel<<<(R + rows_per_block - 1) / rows_per_block, rows_per_block * 32, 0, st>>>(src, map, k, R,
+                                                                                                   K, q, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
+                                    const CUtensorMap &tmB1, cudaStream_t st)
+{
+    const int grid = g.ctas > 0 ? g.ctas : num_sms();
+    if (!fp8_smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
+    if (g.mode == 0)
+        grouped_gemm_fp8_kernel<0><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
+    else
+        grouped_gemm_fp8_kernel<1><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -35,7 +35,12 @@ struct StageMarks {
         on = g_stage_on;
         for (int i = 0; i < MOE_STAGE_EVENTS; ++i) ev[i] = g_stage_ev[i];
     }
-    cudaError_t mark(int i, cudaStream_t st) const { return on ? cudaEventRecord(ev[i], st) : cudaSuccess; }
+    // External records become event-record nodes when the stream is being captured
+    // into a CUDA graph, so a replayed graph still timestamps every stage.
+    cudaError_t mark(int i, cudaStream_t st) const
+    {
+        return on ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal) : cudaSuccess;
+    }
 };
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -72,6 +77,34 @@ bool encode_2d(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, u
 }
 
 // bf16 weights [E, rows, cols], tiles of box_rows x 64 of one expert.
+// e4m3 matrix [rows, cols] bytes, tiles of box_rows x 128 bytes with the 128-byte swizzle.
+bool encode_2d_u8(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {128, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// e4m3 weights [E, rows, cols] bytes, tiles of box_rows x 128 bytes of one expert.
+bool encode_3d_u8(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {cols, rows, E};
+    const cuuint64_t strides[2] = {cols, rows * cols};
+    const cuuint32_t box[3] = {128, box_rows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_3d(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows)
 {
     EncodeTiledFn f = encode_fn();
@@ -121,7 +154,12 @@ extern "C" {
 
 size_t moe_workspace_size(const moe_dims_t *d, int dtype)
 {
-    if (check_dims(d) != MOE_OK || dtype != MOE_DTYPE_BF16) return 0;
+    if (check_dims(d) != MOE_OK) return 0;
+    if (dtype == MOE_DTYPE_FP8) {
+        if (d->H % 128 || d->I % 128) return 0;
+        return moe::ws_layout(*d, MOE_DTYPE_FP8).total;
+    }
+    if (dtype != MOE_DTYPE_BF16) return 0;
     return moe::ws_layout(*d).total;
 }
 
@@ -244,6 +282,88 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
     if (e == cudaSuccess) {
         moe::GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, y, s2f, ctas, rev, wait_ns, stall};
         e = moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st);
+    }
+    if (e == cudaSuccess) e = marks.mark(4, st);
+    if (e == cudaSuccess)
+        e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st);
+    if (e == cudaSuccess) e = marks.mark(5, st);
+    return cuda_status(e);
+}
+
+moe_status_t moe_quantize_rows_fp8(int32_t R, int32_t K, const void *a, uint8_t *q, float *s, void *stream)
+{
+    if (R < 0 || K <= 0 || K % 128) return MOE_ERR_INVALID_ARG;
+    if (R == 0) return MOE_OK;
+    if (!a || !q || !s || !aligned16(a) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_quantize_rows(static_cast<const __nv_bfloat16 *>(a), nullptr, 1, R, K, q, s,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *router_w, const float *router_bias,
+                             const uint8_t *w_gate_q, const float *w_gate_s, const uint8_t *w_up_q,
+                             const float *w_up_s, const uint8_t *w_down_q, const float *w_down_s, void *out,
+                             void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status_t s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (d->H % 128 || d->I % 128) return MOE_ERR_INVALID_ARG;
+    if (d->T == 0) return MOE_OK;
+    if (!x || !router_w || !w_gate_q || !w_gate_s || !w_up_q || !w_up_s || !w_down_q || !w_down_s || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(w_gate_q) || !aligned16(w_up_q) ||
+        !aligned16(w_down_q) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    const moe::WsLayout L = moe::ws_layout(*d, MOE_DTYPE_FP8);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int A = d->T * d->top_k;
+    auto *hdr = at<moe::WsHeader>(ws, 0);
+    auto *xs = at<uint8_t>(ws, L.xs);
+    auto *xs_s = at<float>(ws, L.xs_s);
+    auto *h = at<uint8_t>(ws, L.h);
+    auto *h_s = at<float>(ws, L.h_s);
+    auto *y = at<__nv_bfloat16>(ws, L.y);
+    auto *idx = at<int32_t>(ws, L.idx);
+    auto *gate = at<float>(ws, L.gate);
+    auto *s2f = at<int32_t>(ws, L.s2f);
+    auto *tiles = at<int32_t>(ws, L.tiles);
+    auto *ntiles = at<int32_t>(ws, L.ntiles);
+
+    CUtensorMap tm_xs, tm_wg, tm_wu, tm_h, tm_wd;
+    if (!encode_2d_u8(&tm_xs, xs, A, d->H, moe::kTileRows) || !encode_3d_u8(&tm_wg, w_gate_q, d->E, d->I, d->H, 128) ||
+        !encode_3d_u8(&tm_wu, w_up_q, d->E, d->I, d->H, 128) || !encode_2d_u8(&tm_h, h, A, d->I, moe::kTileRows) ||
+        !encode_3d_u8(&tm_wd, w_down_q, d->E, d->H, d->I, 256))
+        return MOE_ERR_CUDA;
+
+    const StageMarks marks;
+    cudaError_t e = marks.mark(0, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(moe::WsHeader), st);
+    if (e == cudaSuccess)
+        e = moe::launch_route(*d, static_cast<const __nv_bfloat16 *>(x),
+                              static_cast<const __nv_bfloat16 *>(router_w), router_bias, at<float>(ws, L.logits),
+                              idx, gate, st);
+    if (e == cudaSuccess) e = marks.mark(1, st);
+    if (e == cudaSuccess)
+        e = moe::launch_permute(*d, L, idx, at<int32_t>(ws, L.blk_cnt), at<int32_t>(ws, L.blk_base),
+                                at<int32_t>(ws, L.offsets), s2f, at<int32_t>(ws, L.f2s), tiles, ntiles, hdr, st);
+    if (e == cudaSuccess)
+        e = moe::launch_quantize_rows(static_cast<const __nv_bfloat16 *>(x), s2f, d->top_k, A, d->H, xs, xs_s, st);
+    if (e == cudaSuccess) e = marks.mark(2, st);
+    const int ctas = g_gemm_ctas.load(), rev = g_claim_reverse.load();
+    const unsigned long long wl = g_wait_ns.load();
+    const uint64_t wait_ns = wl ? wl : 2000000000ull;
+    const int stall = g_stall_test.load();
+    if (e == cudaSuccess) {
+        moe::Fp8GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, xs_s, w_gate_s, w_up_s,
+                            h, h_s, nullptr, nullptr, ctas, rev, wait_ns, stall};
+        e = moe::launch_grouped_gemm_fp8(g1, tm_xs, tm_wg, tm_wu, st);
+    }
+    if (e == cudaSuccess) e = marks.mark(3, st);
+    if (e == cudaSuccess) {
+        moe::Fp8GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, h_s, w_down_s, w_down_s,
+                            nullptr, nullptr, y, s2f, ctas, rev, wait_ns, stall};
+        e = moe::launch_grouped_gemm_fp8(g2, tm_h, tm_wd, tm_wd, st);
     }
     if (e == cudaSuccess) e = marks.mark(4, st);
     if (e == cudaSuccess)

@@ -22,7 +22,7 @@ struct WsHeader {
 
 // Byte offsets of every region of the workspace (256-byte aligned each).
 struct WsLayout {
-    size_t logits, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xs, h, y, total;
+    size_t logits, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xs, xs_s, h, h_s, y, total;
     int nb;      // permutation chunks
     int chunk;   // flat entries per chunk
 };
@@ -40,8 +40,11 @@ inline int perm_warps(int E)
     return w;
 }
 
-inline WsLayout ws_layout(const moe_dims_t &d)
+// Workspace regions; with fp8 the sorted activations and h are e4m3 codes plus
+// one fp32 scale per 128 columns.
+inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
 {
+    const bool fp8 = dtype == MOE_DTYPE_FP8;
     WsLayout L{};
     const size_t A = static_cast<size_t>(d.T) * d.top_k;
     const int warps = perm_warps(d.E);
@@ -64,8 +67,10 @@ inline WsLayout ws_layout(const moe_dims_t &d)
     L.f2s = take(A * 4);
     L.tiles = take(max_tiles * 3 * 4);
     L.ntiles = take(4);
-    L.xs = take(A * d.H * 2);
-    L.h = take(A * d.I * 2);
+    L.xs = take(A * d.H * (fp8 ? 1 : 2));
+    L.xs_s = take(fp8 ? A * (d.H / 128) * 4 : 0);
+    L.h = take(A * d.I * (fp8 ? 1 : 2));
+    L.h_s = take(fp8 ? A * (d.I / 128) * 4 : 0);
     L.y = take(A * d.H * 2);
     L.total = o;
     return L;
@@ -108,6 +113,32 @@ struct GemmArgs {
 };
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
                                 const CUtensorMap &tmB1, cudaStream_t st);
+
+// FP8 block-scaled grouped GEMMs (fp8.cu).  mode 0: h codes/scales from
+// silu(A Wg^T) * (A Wu^T); mode 1: y[row_map[row]] = A Wd^T in bf16.
+struct Fp8GemmArgs {
+    int mode;
+    int K, N;
+    const int32_t *tiles;
+    const int32_t *ntiles;
+    int32_t *counter;
+    int32_t *status;
+    const float *sa;   // activation scales [rows, K/128]
+    const float *sb0;  // weight scales [E, N/128, K/128] (gate or down)
+    const float *sb1;  // up scales (mode 0)
+    uint8_t *out_q;    // mode 0: h codes [rows, N]
+    float *out_s;      // mode 0: h scales [rows, N/128]
+    __nv_bfloat16 *out;      // mode 1: y [T*k, N]
+    const int32_t *row_map;  // mode 1: sorted row -> flat row
+    int ctas;
+    int reverse;
+    uint64_t wait_ns;
+    int stall_test;
+};
+cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
+                                    const CUtensorMap &tmB1, cudaStream_t st);
+cudaError_t launch_quantize_rows(const __nv_bfloat16 *src, const int32_t *map, int k, int R, int K, uint8_t *q,
+                                 float *s, cudaStream_t st);
 
 int num_sms();
 

@@ -1,0 +1,113 @@
+"""FP8 block-scaled layer: CUDA path vs the CPU oracle through the C ABI.
+
+The activation quantiser's codes and scales must match the oracle bit for bit (same
+bf16 inputs, same fp32 decisions).  The layer output is compared with the fp8
+oracle at relative L2 <= 3e-2; routing is the bf16 router and stays bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import compare_routing, sample_tokens
+from routed_grouped_gemm_softmax_b200 import api
+from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_fp8_weights, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+FP8_REL_L2 = 3e-2
+
+
+def rel_l2(out_gpu, ref):
+    o = out_gpu.float().cpu().double().numpy()
+    return float(np.linalg.norm(o - ref) / np.linalg.norm(ref))
+
+
+def test_quantizer_bit_exact():
+    rng = np.random.default_rng(1)
+    a = torch.as_tensor(rng.standard_normal((37, 1024)).astype(np.float32) * 3).to(torch.bfloat16)
+    a[3, 128:256] = 0.0                    # all-zero group -> scale 1, codes 0
+    a[5, :] *= 1e-30                       # tiny values (subnormal e4m3 codes)
+    a[7, 0] = 1e4                          # one huge value per group
+    q, s = api.moe_quantize_rows_fp8(a.cuda())
+    qr, sr = oracle.quantize_rows(a)
+    assert np.array_equal(s.cpu().numpy(), sr)
+    assert np.array_equal(q.cpu().numpy(), qr)
+
+
+def _fp8_case(cfg, device="cuda"):
+    inp = make_inputs(cfg, device=device, weights=False)
+    w = make_fp8_weights(cfg, device=device)
+    return inp, w
+
+
+def _run_fp8(cfg, inp, w):
+    g = {k: v.cuda() for k, v in w.items()}
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k, "cuda", api.DTYPE_FP8)
+    bias = None if inp.bias is None else inp.bias.cuda()
+    out = api.moe_forward_fp8(inp.x.cuda(), inp.router_w.cuda(), bias, g["w_gate_q"], g["w_gate_s"],
+                              g["w_up_q"], g["w_up_s"], g["w_down_q"], g["w_down_s"], cfg.top_k, ws=ws)
+    assert api.moe_get_device_status(ws) == api.MOE_OK
+    return out
+
+
+def _oracle_fp8(cfg, inp, w, tokens=None):
+    x, rw = inp.x.cpu(), inp.router_w.cpu()
+    bias = None if inp.bias is None else inp.bias.cpu()
+    idx, gate = oracle.route(x, rw, bias, cfg.top_k)
+    if tokens is None:
+        wc = {k: v.cpu() for k, v in w.items()}
+        return oracle.combine_ffn_fp8(x, idx, gate, wc["w_gate_q"], wc["w_gate_s"], wc["w_up_q"],
+                                      wc["w_up_s"], wc["w_down_q"], wc["w_down_s"]), idx, gate
+    # only the experts the sampled tokens use, re-indexed
+    used = np.unique(idx[tokens].reshape(-1))
+    remap = np.full(cfg.E, -1, np.int32)
+    remap[used] = np.arange(used.size, dtype=np.int32)
+    sel = torch.as_tensor(used, device=w["w_gate_q"].device).long()
+    wc = {k: v.index_select(0, sel).cpu() for k, v in w.items()}
+    idx_c = np.where(np.isin(np.arange(cfg.T)[:, None], tokens), remap[idx], 0).astype(np.int32)
+    out = oracle.combine_ffn_fp8(x, idx_c, gate, wc["w_gate_q"], wc["w_gate_s"], wc["w_up_q"], wc["w_up_s"],
+                                 wc["w_down_q"], wc["w_down_s"], tokens=tokens)
+    return out, idx, gate
+
+
+SMALL = {
+    "fp8_small": CONFIGS["fp8"].replace(name="fp8_small", T=64, H=256, E=8, top_k=2, I=256),
+    "fp8_ragged": CONFIGS["fp8"].replace(name="fp8_ragged", T=150, H=384, E=12, top_k=3, I=384, seed=7),
+    "fp8_bias": CONFIGS["fp8"].replace(name="fp8_bias", T=130, H=512, E=16, top_k=4, I=256, seed=8,
+                                       zipf_s=1.2),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_fp8_layer_small(name):
+    cfg = SMALL[name]
+    inp, w = _fp8_case(cfg)
+    out = _run_fp8(cfg, inp, w)
+    ref, idx, gate = _oracle_fp8(cfg, inp, w)
+    bias = None if inp.bias is None else inp.bias.cuda()
+    i_g, w_g = api.moe_route(inp.x.cuda(), inp.router_w.cuda(), bias, cfg.top_k)
+    compare_routing(i_g, w_g, idx, gate, name)
+    r = rel_l2(out, ref)
+    assert r <= FP8_REL_L2, f"{name}: rel_l2={r:.3e}"
+
+
+def test_fp8_zero_router_all_tokens_to_first_experts():
+    cfg = SMALL["fp8_small"].replace(name="fp8_ties", T=300, top_k=3, seed=9)
+    inp, w = _fp8_case(cfg)
+    inp.router_w = torch.zeros_like(inp.router_w)
+    out = _run_fp8(cfg, inp, w)
+    ref, _, _ = _oracle_fp8(cfg, inp, w)
+    assert rel_l2(out, ref) <= FP8_REL_L2
+
+
+def test_fp8_full_size_sampled():
+    cfg = CONFIGS["fp8"]
+    inp, w = _fp8_case(cfg)
+    out = _run_fp8(cfg, inp, w)
+    tok = sample_tokens(cfg.T, 6, seed=cfg.seed)
+    ref, idx, gate = _oracle_fp8(cfg, inp, w, tokens=tok)
+    i_g, w_g = api.moe_route(inp.x, inp.router_w, None, cfg.top_k)
+    compare_routing(i_g, w_g, idx, gate, "fp8")
+    r = rel_l2(out[torch.as_tensor(tok, device="cuda").long()], ref)
+    assert r <= FP8_REL_L2, f"fp8 full size: rel_l2={r:.3e}"
