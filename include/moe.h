@@ -150,6 +150,15 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
  * fp32 scales, per row per 128 columns as described above.  Needs no workspace. */
 moe_status_t moe_quantize_rows_fp8(int32_t R, int32_t K, const void *a, uint8_t *q, float *s, void *stream);
 
+/* Where the last moe_forward / moe_forward_fp8 left its routing inside the
+ * workspace, for inspection: out[i] receives the byte offset of
+ *   0 topk_idx [T,k] int32    1 topk_w [T,k] fp32      2 expert_offsets [E+1]
+ *   3 sorted_to_flat [T*k]    4 flat_to_sorted [T*k]    5 tile_list [3*max_tiles]
+ *   6 num_tiles [1]
+ * (same meaning as the outputs of moe_route and moe_permute).  Writes
+ * min(n, 7) entries; returns MOE_ERR_INVALID_ARG for invalid dims or dtype. */
+moe_status_t moe_workspace_offsets(const moe_dims_t *d, int dtype, size_t *out, int32_t n);
+
 /* Synchronises `stream`, returns the device status word of the workspace
  * (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_BAD_INDEX; MOE_ERR_CUDA if the stream
  * reports an error) and clears it. */

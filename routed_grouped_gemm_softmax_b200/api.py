@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "moe_forward",
            "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order",
            "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",
-           "moe_forward_fp8", "moe_quantize_rows_fp8"]
+           "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets"]
 DTYPE_BF16, DTYPE_FP8 = 0, 1
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
@@ -73,6 +73,8 @@ def lib():
         L.moe_forward_fp8.restype = ctypes.c_int
         L.moe_quantize_rows_fp8.argtypes = [I32, I32, P, P, P, P]
         L.moe_quantize_rows_fp8.restype = ctypes.c_int
+        L.moe_workspace_offsets.argtypes = [D, ctypes.c_int, P, I32]
+        L.moe_workspace_offsets.restype = ctypes.c_int
         L.moe_set_wait_limit_us.argtypes = [I32, I32]
         L.moe_set_wait_limit_us.restype = None
         L.moe_forward_noalloc.argtypes = [D, P, P, P, P, P, P, P, P]
@@ -245,6 +247,24 @@ def moe_forward_noalloc(x, router_w, bias, w_gate, w_up, w_down, top_k: int, out
                                      _p(w_up), _p(w_down), _p(out), _stream(stream, dev)),
            "moe_forward_noalloc")
     return out
+
+
+def forward_routing(ws, T, H, I, E, top_k, dtype: int = DTYPE_BF16) -> dict:
+    """Views into the workspace of the routing the last forward on it computed
+    (topk_idx, topk_w, offsets, sorted_to_flat, flat_to_sorted, tile_list, num_tiles)."""
+    offs = (ctypes.c_size_t * 7)()
+    _check(lib().moe_workspace_offsets(ctypes.byref(dims(T, H, I, E, top_k)), int(dtype), offs, 7),
+           "moe_workspace_offsets")
+    A = T * top_k
+    nt = moe_max_tiles(T, H, I, E, top_k)
+
+    def view(i, n, dt):
+        nbytes = n * torch.tensor([], dtype=dt).element_size()
+        return ws[offs[i]:offs[i] + nbytes].view(dt)
+    return {"topk_idx": view(0, A, torch.int32).view(T, top_k), "topk_w": view(1, A, torch.float32).view(T, top_k),
+            "offsets": view(2, E + 1, torch.int32), "sorted_to_flat": view(3, A, torch.int32),
+            "flat_to_sorted": view(4, A, torch.int32), "tile_list": view(5, 3 * nt, torch.int32).view(nt, 3),
+            "num_tiles": view(6, 1, torch.int32)}
 
 
 def moe_get_device_status(ws, stream=None) -> int:

@@ -148,6 +148,34 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
 // weights by TMA, which needs 16-byte aligned bases).
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Router and permute: one fused launch for small batches, otherwise the logits,
+// top-k and three permute kernels.  Stage mark 1 (routed) is recorded between the
+// two in the multi-kernel form and together with the fused launch otherwise.
+cudaError_t route_and_permute(const moe_dims_t &d, const moe::WsLayout &L, const void *x, const void *router_w,
+                              const float *router_bias, void *ws, moe::WsHeader *hdr, const StageMarks &marks,
+                              cudaStream_t st)
+{
+    auto *idx = at<int32_t>(ws, L.idx);
+    auto *gate = at<float>(ws, L.gate);
+    auto *s2f = at<int32_t>(ws, L.s2f);
+    auto *tiles = at<int32_t>(ws, L.tiles);
+    auto *ntiles = at<int32_t>(ws, L.ntiles);
+    const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+    const auto *wb = static_cast<const __nv_bfloat16 *>(router_w);
+    if (moe::small_route_permute_ok(d)) {
+        cudaError_t e = moe::launch_route_permute_small(d, xb, wb, router_bias, at<float>(ws, L.logits), idx, gate,
+                                                        at<int32_t>(ws, L.offsets), s2f, at<int32_t>(ws, L.f2s),
+                                                        tiles, ntiles, hdr, st);
+        return e == cudaSuccess ? marks.mark(1, st) : e;
+    }
+    cudaError_t e = moe::launch_route(d, xb, wb, router_bias, at<float>(ws, L.logits), idx, gate, st);
+    if (e == cudaSuccess) e = marks.mark(1, st);
+    if (e == cudaSuccess)
+        e = moe::launch_permute(d, L, idx, at<int32_t>(ws, L.blk_cnt), at<int32_t>(ws, L.blk_base),
+                                at<int32_t>(ws, L.offsets), s2f, at<int32_t>(ws, L.f2s), tiles, ntiles, hdr, st);
+    return e;
+}
+
 }  // namespace
 
 extern "C" {
@@ -259,14 +287,7 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
     const StageMarks marks;
     cudaError_t e = marks.mark(0, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(moe::WsHeader), st);
-    if (e == cudaSuccess)
-        e = moe::launch_route(*d, static_cast<const __nv_bfloat16 *>(x),
-                              static_cast<const __nv_bfloat16 *>(router_w), router_bias, at<float>(ws, L.logits),
-                              idx, gate, st);
-    if (e == cudaSuccess) e = marks.mark(1, st);
-    if (e == cudaSuccess)
-        e = moe::launch_permute(*d, L, idx, at<int32_t>(ws, L.blk_cnt), at<int32_t>(ws, L.blk_base),
-                                at<int32_t>(ws, L.offsets), s2f, at<int32_t>(ws, L.f2s), tiles, ntiles, hdr, st);
+    if (e == cudaSuccess) e = route_and_permute(*d, L, x, router_w, router_bias, ws, hdr, marks, st);
     if (e == cudaSuccess)
         e = moe::launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), s2f, A, d->H, d->top_k, xs, st);
     if (e == cudaSuccess) e = marks.mark(2, st);
@@ -339,14 +360,7 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
     const StageMarks marks;
     cudaError_t e = marks.mark(0, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(moe::WsHeader), st);
-    if (e == cudaSuccess)
-        e = moe::launch_route(*d, static_cast<const __nv_bfloat16 *>(x),
-                              static_cast<const __nv_bfloat16 *>(router_w), router_bias, at<float>(ws, L.logits),
-                              idx, gate, st);
-    if (e == cudaSuccess) e = marks.mark(1, st);
-    if (e == cudaSuccess)
-        e = moe::launch_permute(*d, L, idx, at<int32_t>(ws, L.blk_cnt), at<int32_t>(ws, L.blk_base),
-                                at<int32_t>(ws, L.offsets), s2f, at<int32_t>(ws, L.f2s), tiles, ntiles, hdr, st);
+    if (e == cudaSuccess) e = route_and_permute(*d, L, x, router_w, router_bias, ws, hdr, marks, st);
     if (e == cudaSuccess)
         e = moe::launch_quantize_rows(static_cast<const __nv_bfloat16 *>(x), s2f, d->top_k, A, d->H, xs, xs_s, st);
     if (e == cudaSuccess) e = marks.mark(2, st);
@@ -370,6 +384,15 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
         e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st);
     if (e == cudaSuccess) e = marks.mark(5, st);
     return cuda_status(e);
+}
+
+moe_status_t moe_workspace_offsets(const moe_dims_t *d, int dtype, size_t *out, int32_t n)
+{
+    if (!out || n < 0 || moe_workspace_size(d, dtype) == 0) return MOE_ERR_INVALID_ARG;
+    const moe::WsLayout L = moe::ws_layout(*d, dtype);
+    const size_t v[7] = {L.idx, L.gate, L.offsets, L.s2f, L.f2s, L.tiles, L.ntiles};
+    for (int i = 0; i < n && i < 7; ++i) out[i] = v[i];
+    return MOE_OK;
 }
 
 moe_status_t moe_get_device_status(void *ws, void *stream)

@@ -18,6 +18,7 @@ constexpr int kMaxExperts = 1024;
 struct WsHeader {
     int32_t status;       // device status word (moe_status_t), sticky until read
     int32_t counter[7];   // work-claim counters of the persistent GEMMs
+    int32_t pad[8];
 };
 
 // Byte offsets of every region of the workspace (256-byte aligned each).
@@ -82,6 +83,14 @@ inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
 cudaError_t launch_route(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
                          const float *bias, float *logits, int32_t *idx, float *gate,
                          cudaStream_t st);
+
+// Router + permute in two launches for small batches (T <= 32, E % 8 == 0,
+// H % 128 == 0, T*k <= 4096).
+bool small_route_permute_ok(const moe_dims_t &d);
+cudaError_t launch_route_permute_small(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
+                                       const float *bias, float *logits, int32_t *idx, float *gate,
+                                       int32_t *offsets, int32_t *s2f, int32_t *f2s, int32_t *tiles,
+                                       int32_t *ntiles, WsHeader *hdr, cudaStream_t st);
 
 cudaError_t launch_permute(const moe_dims_t &d, const WsLayout &L, const int32_t *idx,
                            int32_t *blk_cnt, int32_t *blk_base, int32_t *offsets, int32_t *s2f,

@@ -301,21 +301,19 @@ __device__ __forceinline__ bool ranks_before(float v1, int e1, float v2, int e2)
     return v1 > v2 || (v1 == v2 && e1 < e2);
 }
 
+// One warp: top-k of one token's E logits (larger logit first, equal logits ->
+// lower index) and the softmax over the chosen k.  `sv` is k floats of scratch.
 template <int MAXV>
-__global__ void route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
-                                  int32_t *__restrict__ idx, float *__restrict__ gate)
+__device__ __forceinline__ void topk_softmax_warp(const float *__restrict__ lrow, int E, int k,
+                                                  int32_t *__restrict__ idx_out, float *__restrict__ gate_out,
+                                                  float *sv)
 {
-    extern __shared__ float sel[];  // [warps][k] chosen logits
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int t = blockIdx.x * (blockDim.x / 32) + warp;
-    if (t >= T) return;
-    float *sv = sel + (size_t)warp * k;
-
+    const int lane = threadIdx.x % 32;
     float v[MAXV];
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
         const int e = lane + 32 * i;
-        v[i] = e < E ? logits[(size_t)t * E + e] : 0.0f;
+        v[i] = e < E ? lrow[e] : 0.0f;
     }
     uint32_t taken = 0;
     for (int j = 0; j < k; ++j) {
@@ -340,7 +338,7 @@ __global__ void route_topk_kernel(const float *__restrict__ logits, int T, int E
         }
         if ((be & 31) == lane) taken |= 1u << (be >> 5);
         if (lane == 0) {
-            idx[(size_t)t * k + j] = be;
+            idx_out[j] = be;
             sv[j] = bv;
         }
     }
@@ -350,7 +348,20 @@ __global__ void route_topk_kernel(const float *__restrict__ logits, int T, int E
     for (int j = lane; j < k; j += 32) s += expf(sv[j] - m);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    for (int j = lane; j < k; j += 32) gate[(size_t)t * k + j] = expf(sv[j] - m) / s;
+    for (int j = lane; j < k; j += 32) gate_out[j] = expf(sv[j] - m) / s;
+    __syncwarp();
+}
+
+template <int MAXV>
+__global__ void route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
+                                  int32_t *__restrict__ idx, float *__restrict__ gate)
+{
+    extern __shared__ float sel[];  // [warps][k] chosen logits
+    const int warp = threadIdx.x / 32;
+    const int t = blockIdx.x * (blockDim.x / 32) + warp;
+    if (t >= T) return;
+    topk_softmax_warp<MAXV>(logits + (size_t)t * E, E, k, idx + (size_t)t * k, gate + (size_t)t * k,
+                            sel + (size_t)warp * k);
 }
 
 template <int MAXV>
@@ -369,7 +380,255 @@ cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *idx, 
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------
+// Small batches, router + permute in two launches.  route_logits_pipe_kernel is
+// route_logits_small_kernel with the chain fed from registers: eight x values
+// arrive in one 16-byte shared load and the next eight (and their weights) are
+// loaded while the current eight feed the FMA chain.  topk_permute_small_kernel
+// then runs one CTA: top-k and softmax per token (a warp each) and the stable
+// grouping by expert of the T*k assignments -- the same results as
+// route_topk_kernel and the three permute kernels.
+struct SmallRouteOut {
+    float *logits;
+    int32_t *idx;
+    float *gate;
+    int32_t *offsets, *s2f, *f2s, *tiles, *ntiles;
+    int32_t *counters;
+    int ncounters;
+    int32_t *status;
+};
+
+// Exclusive scan of one value per thread over the CTA (blockDim <= 1024).
+__device__ int cta_exclusive_scan(int v, int *wtot, int &total)
+{
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+    int inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += o;
+    }
+    if (lane == 31) wtot[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const int w = lane < nw ? wtot[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += o;
+        }
+        if (lane < nw) wtot[lane] = wi - w;
+        if (lane == 31) wtot[32] = wi;
+    }
+    __syncthreads();
+    const int res = wtot[warp] + inc - v;
+    total = wtot[32];
+    __syncthreads();
+    return res;
+}
+
+// Stable counting sort of A flat assignments by expert inside one CTA (A small).
+__device__ void permute_in_cta(const int32_t *__restrict__ idx, int A, int E, const SmallRouteOut &o, int *sm)
+{
+    const int NT = blockDim.x, tid = threadIdx.x, lane = tid % 32, warp = tid / 32, nw = NT / 32;
+    int *cursor = sm;             // [E]
+    int *wtot = sm + E;           // [33]
+    for (int e = tid; e < E; e += NT) cursor[e] = 0;
+    __syncthreads();
+    for (int f = tid; f < A; f += NT) {
+        const int e = idx[f];
+        if (e >= 0 && e < E)
+            atomicAdd(&cursor[e], 1);
+        else
+            atomicCAS(o.status, 0, MOE_ERR_BAD_INDEX);
+    }
+    __syncthreads();
+    // each thread owns a contiguous run of experts for the two scans
+    const int per = (E + NT - 1) / NT;
+    const int e_lo = min(E, tid * per), e_hi = min(E, e_lo + per);
+    int rows = 0, tls = 0;
+    for (int e = e_lo; e < e_hi; ++e) {
+        rows += cursor[e];
+        tls += (cursor[e] + kTileRows - 1) / kTileRows;
+    }
+    int total_rows = 0, total_tiles = 0;
+    int off = cta_exclusive_scan(rows, wtot, total_rows);
+    int toff = cta_exclusive_scan(tls, wtot, total_tiles);
+    for (int e = e_lo; e < e_hi; ++e) {
+        const int c = cursor[e];
+        o.offsets[e] = off;
+        for (int m = 0; m * kTileRows < c; ++m) {
+            int32_t *tl = o.tiles + 3 * (size_t)(toff + m);
+            tl[0] = e;
+            tl[1] = off + m * kTileRows;
+            tl[2] = min(kTileRows, c - m * kTileRows);
+        }
+        toff += (c + kTileRows - 1) / kTileRows;
+        cursor[e] = off;  // becomes the next free sorted row of expert e
+        off += c;
+    }
+    if (tid == 0) {
+        o.offsets[E] = total_rows;
+        *o.ntiles = total_tiles;
+    }
+    __syncthreads();
+    // chunks in order; inside a chunk, warps in order; inside a warp, lanes by rank
+    for (int c0 = 0; c0 < A; c0 += NT) {
+        const int f = c0 + tid;
+        const int e = f < A ? idx[f] : -1;
+        const bool valid = e >= 0 && e < E;
+        const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        for (int w = 0; w < nw; ++w) {
+            if (warp == w && valid) {
+                const int pos = cursor[e] + rank;
+                o.s2f[pos] = f;
+                o.f2s[f] = pos;
+            }
+            __syncwarp();
+            if (warp == w && valid && rank == 0) cursor[e] += __popc(peers);
+            __syncthreads();
+        }
+    }
+    if (tid < o.ncounters) o.counters[tid] = 0;
+}
+
+template <int TP, int TE, int HC, int S>
+__global__ void __launch_bounds__(TP * TE)
+route_logits_pipe_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ wr,
+                         const float *__restrict__ bias, int T, int H, int E, float *__restrict__ logits)
+{
+    using L = SmallTile<TP, TE, HC, S>;
+    extern __shared__ __align__(16) uint8_t ssm[];
+    const int tid = threadIdx.x;
+    const int tt = tid / TE, ee = tid % TE;
+    const int e0 = blockIdx.x * TE;
+    const int nchunks = H / HC;
+
+    auto issue = [&](int ch) {
+        if (ch < nchunks) {
+            uint8_t *st = ssm + (ch % S) * L::STAGE;
+            const int h0 = ch * HC;
+            for (int v = tid; v < TP * (HC / 8); v += L::NT) {
+                const int r = v / (HC / 8), c8 = (v % (HC / 8)) * 8;
+                if (r < T) cp_async16(st + r * L::XROW + c8 * 2, x + (size_t)r * H + h0 + c8);
+            }
+            for (int v = tid; v < HC * (TE / 8); v += L::NT) {
+                const int hh = v / (TE / 8), c8 = (v % (TE / 8)) * 8;
+                if (e0 + c8 < E) cp_async16(st + L::XBYTES + (hh * TE + c8) * 2, wr + (size_t)(h0 + hh) * E + e0 + c8);
+            }
+        }
+        cp_async_commit();
+    };
+
+    float acc = 0.0f;
+#pragma unroll
+    for (int s = 0; s < S - 1; ++s) issue(s);
+    for (int ch = 0; ch < nchunks; ++ch) {
+        cp_async_wait<S - 2>();
+        __syncthreads();
+        issue(ch + S - 1);
+        const uint8_t *st = ssm + (ch % S) * L::STAGE;
+        const uint4 *xv = reinterpret_cast<const uint4 *>(st + tt * L::XROW);
+        const unsigned short *wc = reinterpret_cast<const unsigned short *>(st + L::XBYTES) + ee;
+        uint4 xq = xv[0];
+        unsigned short w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = wc[j * TE];
+#pragma unroll
+        for (int h8 = 0; h8 < HC / 8; ++h8) {
+            uint4 xn = xq;
+            unsigned short wn[8];
+            if (h8 + 1 < HC / 8) {
+                xn = xv[h8 + 1];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) wn[j] = wc[((h8 + 1) * 8 + j) * TE];
+            }
+            const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float a = __uint_as_float((j & 1) ? (xw[j / 2] & 0xFFFF0000u) : (xw[j / 2] << 16));
+                const float b = __uint_as_float(static_cast<uint32_t>(w[j]) << 16);
+                acc = fmaf(a, b, acc);
+            }
+            xq = xn;
+            if (h8 + 1 < HC / 8) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[j] = wn[j];
+            }
+        }
+    }
+    cp_async_wait<0>();
+    const int e = e0 + ee;
+    if (tt < T && e < E) {
+        float v = acc;
+        if (bias) v = __fadd_rn(v, bias[e]);
+        logits[(size_t)tt * E + e] = v;
+    }
+}
+
+// Top-k + softmax for every token (one warp per token) and the stable grouping by
+// expert of the T*k assignments, in one CTA: small batches only (T <= 32).
+template <int MAXV>
+__global__ void __launch_bounds__(1024) topk_permute_small_kernel(int T, int E, int k, SmallRouteOut o)
+{
+    extern __shared__ __align__(16) uint8_t tsm[];
+    const int warp = threadIdx.x / 32, nw = blockDim.x / 32;
+    float *sv = reinterpret_cast<float *>(tsm);  // [nw][k]
+    for (int t = warp; t < T; t += nw)
+        topk_softmax_warp<MAXV>(o.logits + (size_t)t * E, E, k, o.idx + (size_t)t * k, o.gate + (size_t)t * k,
+                                sv + (size_t)warp * k);
+    __syncthreads();
+    permute_in_cta(o.idx, T * k, E, o, reinterpret_cast<int *>(tsm) + nw * k);
+}
+
 }  // namespace
+
+bool small_route_permute_ok(const moe_dims_t &d)
+{
+    return d.T <= 32 && d.E % 8 == 0 && d.H % 128 == 0 && (long)d.T * d.top_k <= 4096;
+}
+
+cudaError_t launch_route_permute_small(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
+                                       const float *bias, float *logits, int32_t *idx, float *gate,
+                                       int32_t *offsets, int32_t *s2f, int32_t *f2s, int32_t *tiles,
+                                       int32_t *ntiles, WsHeader *hdr, cudaStream_t st)
+{
+    SmallRouteOut o{logits, idx, gate, offsets, s2f, f2s, tiles, ntiles, hdr->counter, 7, &hdr->status};
+    cudaError_t e;
+    if (d.T <= 16) {
+        using L = SmallTile<16, 8, 128, 16>;
+        auto kern = route_logits_pipe_kernel<16, 8, 128, 16>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+        if (e != cudaSuccess) return e;
+        kern<<<(d.E + 7) / 8, L::NT, L::SMEM, st>>>(x, wr, bias, d.T, d.H, d.E, logits);
+    } else {
+        using L = SmallTile<32, 8, 128, 16>;
+        auto kern = route_logits_pipe_kernel<32, 8, 128, 16>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+        if (e != cudaSuccess) return e;
+        kern<<<(d.E + 7) / 8, L::NT, L::SMEM, st>>>(x, wr, bias, d.T, d.H, d.E, logits);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int warps = d.T < 4 ? 4 : d.T;
+    const size_t smem = ((size_t)warps * d.top_k + d.E + 64) * 4;
+    const int vpl = (d.E + 31) / 32;
+    auto launch = [&](auto kern) {
+        if (smem > 48 * 1024) {
+            cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (r != cudaSuccess) return r;
+        }
+        kern<<<1, warps * 32, smem, st>>>(d.T, d.E, d.top_k, o);
+        return cudaGetLastError();
+    };
+    if (vpl <= 1) return launch(topk_permute_small_kernel<1>);
+    if (vpl <= 2) return launch(topk_permute_small_kernel<2>);
+    if (vpl <= 4) return launch(topk_permute_small_kernel<4>);
+    if (vpl <= 8) return launch(topk_permute_small_kernel<8>);
+    if (vpl <= 16) return launch(topk_permute_small_kernel<16>);
+    return launch(topk_permute_small_kernel<32>);
+}
 
 cudaError_t launch_route(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
                          const float *bias, float *logits, int32_t *idx, float *gate,

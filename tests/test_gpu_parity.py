@@ -142,6 +142,24 @@ def test_repeat_calls_same_workspace():
     assert api.moe_get_device_status(ws) == api.MOE_OK
 
 
+@pytest.mark.parametrize("name", ["decode", "one_token", "small32"])
+def test_forward_routing_matches_oracle(name):
+    # The forward's own routing and permutation (read back from its workspace) must be
+    # bit-exact too -- for small batches they come from the fused router+permute kernel.
+    cfg = {"decode": CONFIGS["decode"], "one_token": SMALL["one_token"],
+           "small32": CONFIGS["decode"].replace(name="small32", T=29, E=64, top_k=6, seed=31)}[name]
+    g, c = device_inputs(cfg)
+    k = cfg.top_k
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, "cuda")
+    for _ in range(2):  # the second call checks the self-reset of the router's ticket
+        api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k, ws=ws)
+        assert api.moe_get_device_status(ws) == api.MOE_OK
+        r = api.forward_routing(ws, cfg.T, cfg.H, cfg.I, cfg.E, k)
+        idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], k)
+        compare_routing(r["topk_idx"], r["topk_w"], idx_ref, gate_ref, name)
+        compare_permute(r, oracle.permute(idx_ref, cfg.E), name)
+
+
 def test_cuda_graph_replay():
     cfg = SMALL["ragged"]
     g, c = device_inputs(cfg)
