@@ -44,8 +44,8 @@
  *    T == 0 is a no-op that returns MOE_OK.
  *  - Errors found on the device (an expert index outside [0,E) handed to
  *    moe_permute, a pipeline wait that exceeded its time limit) are recorded in
- *    a status word inside the workspace; moe_permute and moe_forward clear it
- *    when they start, and moe_get_device_status() reads it.
+ *    a status word inside the workspace; moe_route, moe_permute and the
+ *    forwards clear it when they start, and moe_get_device_status() reads it.
  *  - Results do not depend on the number of GEMM CTAs or on the order in which
  *    they claim work: every sum is taken in an order fixed by the data alone.
  */
@@ -67,7 +67,8 @@ typedef enum {
     MOE_ERR_CUDA = 4,
     MOE_ERR_TIMEOUT = 5,     /* device: a pipeline wait ran past its limit */
     MOE_ERR_BAD_INDEX = 6,   /* device: an expert index outside [0, E) */
-    MOE_ERR_TOO_LARGE = 7    /* moe_forward_noalloc: dims need more than its fixed scratch */
+    MOE_ERR_TOO_LARGE = 7,   /* moe_forward_noalloc: dims need more than its fixed scratch */
+    MOE_ERR_ROUTER_BOUND = 8 /* device: a tensor-core router logit fell outside its error bound */
 } moe_status_t;
 
 typedef struct {
@@ -97,7 +98,11 @@ int32_t moe_max_tiles(const moe_dims_t *d);
  * section 02: each token's router picks the top-k experts; the k outputs are
  * later summed with these gating weights).
  *   x, router_w, router_bias (nullable)  ->  topk_idx [T,k] int32 (descending
- *   logit, ties to the lower index), topk_w [T,k] fp32 (sums to 1 per token). */
+ *   logit, ties to the lower index), topk_w [T,k] fp32 (sums to 1 per token).
+ * For T > 32 the logits are first computed on the tensor cores and the fp32
+ * chain is evaluated only for the experts within a rounding-error bound of the
+ * k-th choice; the result is that of the chain definition.  A chain value found
+ * outside its bound records MOE_ERR_ROUTER_BOUND in the status word. */
 moe_status_t moe_route(const moe_dims_t *d, const void *x, const void *router_w,
                        const float *router_bias, int32_t *topk_idx, float *topk_w,
                        void *ws, size_t ws_bytes, void *stream);
@@ -201,7 +206,7 @@ void moe_set_stage_events(void *const *events, int32_t n);
  * or that must never allocate on their serving path.
  *  - Dims whose moe_workspace_size exceeds the array are rejected with
  *    MOE_ERR_TOO_LARGE (with H=2048, I=512, E=256, top_k=8 that is above
- *    about 220 tokens); invalid dims give the same errors as moe_forward.
+ *    209 tokens); invalid dims give the same errors as moe_forward.
  *  - The first call made with a device current looks up the array's device
  *    address on that device; make that first call before any stream capture.
  *  - Nothing is allocated, freed or synchronised.  Every call shares the one

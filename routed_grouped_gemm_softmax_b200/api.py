@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT",
-                6: "MOE_ERR_BAD_INDEX", 7: "MOE_ERR_TOO_LARGE"}
+                6: "MOE_ERR_BAD_INDEX", 7: "MOE_ERR_TOO_LARGE",
+                8: "MOE_ERR_ROUTER_BOUND"}
 EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "moe_forward",
            "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order",
            "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",

@@ -20,7 +20,10 @@
 // Mode 0 (gate/up): columns 0-127 are gate, 128-255 up, of the same 128 rows of
 // I; a thread owns 64 gate + 64 up columns, forms h = silu(g) * u, and the two
 // warps sharing a row exchange their partial amax through shared memory to
-// quantise the 128-column group.  Mode 1 (down): y rows in bf16.
+// quantise the 128-column group.  Mode 1 (down): y rows in bf16.  Mode 2 (bf16
+// operands, no scales, plain 128-row blocks, K optionally split over items):
+// the router's tensor-core logits, each 64-wide K block summed out of TMEM in
+// fp32 so the accumulation error does not grow with H.
 // Every wait is bounded, as in the bf16 kernel.
 #include <cuda_fp8.h>
 
@@ -122,12 +125,15 @@ __global__ void quantize_rows_kernel(const __nv_bfloat16 *__restrict__ src, cons
 
 // ----------------------------------------------------------- grouped GEMM
 
-template <int MODE>
+template <int MODE, bool BF16>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const Fp8GemmArgs g)
 {
     constexpr int BNO = MODE == 0 ? BN / 2 : BN;  // output columns per tile
+    constexpr int KEL = BF16 ? 64 : 128;          // elements of K per stage (128 bytes)
+    const bool dense = g.tiles == nullptr;        // mode 2: plain 128-row blocks of A
+    const int ksplit = g.ksplit > 0 ? g.ksplit : 1;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *sA = smem_raw + pad;
@@ -136,7 +142,8 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int n_tiles = (g.N + BNO - 1) / BNO;
-    const int KB = g.K / BKB;
+    const int KB = g.K / KEL;
+    const int KBS = (KB + ksplit - 1) / ksplit;  // K blocks per item
     const int NB = g.N / 128;  // 128-row weight blocks along N
 
     if (warp == 0 && lane == 0) {
@@ -169,7 +176,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     if (warp == 0) {
         // ------------------------------------------------ scheduler + TMA producer
         if (lane == 0) {
-            const int total = *g.ntiles * n_tiles;
+            const int total = (dense ? (g.M + BM - 1) / BM : *g.ntiles) * n_tiles * ksplit;
             int stage = 0, rs = 0;
             uint32_t phase = 0, rphase = 0, armed = 0, armed_par = 0;
             bool ok = true;
@@ -184,18 +191,20 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 mbar_arrive(&S->itf[rs]);
                 if (++rs == RING) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
-                const int mt = item / n_tiles, nt = item - mt * n_tiles;
-                const int expert = g.tiles[3 * mt], row0 = g.tiles[3 * mt + 1];
+                const int ks = item % ksplit, mn = item / ksplit;
+                const int mt = mn / n_tiles, nt = mn - mt * n_tiles;
+                const int expert = dense ? 0 : g.tiles[3 * mt], row0 = dense ? mt * BM : g.tiles[3 * mt + 1];
                 const int n0 = nt * BNO;
-                for (int kb = 0; kb < KB; ++kb) {
+                const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
                     mbar_arrive_expect_tx(&S->full[stage], A_BYTES + B_BYTES);
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     uint8_t *b_dst = sB + stage * B_BYTES;
-                    tma_load_2d(sA + stage * A_BYTES, &tmA, &S->full[stage], kb * BKB, row0);
-                    tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BKB, n0, expert);
-                    if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BKB, n0, expert);
+                    tma_load_2d(sA + stage * A_BYTES, &tmA, &S->full[stage], kb * KEL, row0);
+                    tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * KEL, n0, expert);
+                    if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * KEL, n0, expert);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
@@ -215,7 +224,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
+            constexpr uint32_t IDESC = BF16 ? idesc_bf16_f32(BM, BN) : idesc_e4m3_f32(BM, BN);
             int stage = 0, rs = 0, acc = 0;
             uint32_t phase = 0, rphase = 0, aphase = 0;
             bool ok = !(g.stall_test && !mbar_wait(&S->never, 0, g.wait_ns));
@@ -225,7 +234,8 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 mbar_arrive(&S->ite[rs]);
                 if (++rs == RING) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
-                for (int kb = 0; kb < KB; ++kb) {
+                const int kb0 = (item % ksplit) * KBS, kbn = min(KB, kb0 + KBS) - kb0;
+                for (int kb = 0; kb < kbn; ++kb) {
                     if (!mbar_wait(&S->acce[acc], aphase ^ 1, g.wait_ns)) { ok = false; break; }
                     tc_fence_after();
                     if (!mbar_wait(&S->full[stage], phase, g.wait_ns)) { ok = false; break; }
@@ -234,8 +244,12 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                     const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
                     const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
-                    for (int k = 0; k < BKB / 32; ++k)
-                        mma_e4m3(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), IDESC, k != 0);
+                    for (int k = 0; k < 4; ++k) {  // 4 x 32 bytes of K: K=32 e4m3 or K=16 bf16 each
+                        if (BF16)
+                            mma_bf16(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), IDESC, k != 0);
+                        else
+                            mma_e4m3(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), IDESC, k != 0);
+                    }
                     mma_commit(&S->empty[stage]);
                     mma_commit(&S->accf[acc]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -262,25 +276,32 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             if (lane == 0) mbar_arrive(&S->ite[rs]);
             if (++rs == RING) { rs = 0; rphase ^= 1; }
             if (item < 0) break;
-            const int mt = item / n_tiles, nt = item - mt * n_tiles;
-            const int expert = g.tiles[3 * mt], row0 = g.tiles[3 * mt + 1], rows = g.tiles[3 * mt + 2];
+            const int ks = item % ksplit, mn = item / ksplit;
+            const int mt = mn / n_tiles, nt = mn - mt * n_tiles;
+            const int expert = dense ? 0 : g.tiles[3 * mt];
+            const int row0 = dense ? mt * BM : g.tiles[3 * mt + 1];
+            const int rows = dense ? min(BM, g.M - row0) : g.tiles[3 * mt + 2];
             const bool row_ok = row < rows;
             const int n0 = nt * BNO;
-            const float *sa = g.sa + (size_t)(row0 + (row_ok ? row : 0)) * KB;
-            // weight-scale rows of the 128-row blocks this thread's columns fall in
+            const int kb0 = ks * KBS, kbn = min(KB, kb0 + KBS) - kb0;
+            // scales: activation row, and the 128-row weight blocks of this thread's columns
             const int nb0 = MODE == 0 ? n0 / 128 : n0 / 128 + half;
             const bool nb_ok = nb0 < NB;
-            const float *sb0 = g.sb0 + ((size_t)expert * NB + (nb_ok ? nb0 : 0)) * KB;
-            const float *sb1 = MODE == 0 ? g.sb1 + ((size_t)expert * NB + nb0) * KB : sb0;
+            const float *sa = MODE == 2 ? nullptr : g.sa + (size_t)(row0 + (row_ok ? row : 0)) * KB + kb0;
+            const float *sb0 = MODE == 2 ? nullptr : g.sb0 + ((size_t)expert * NB + (nb_ok ? nb0 : 0)) * KB + kb0;
+            const float *sb1 = MODE == 0 ? g.sb1 + ((size_t)expert * NB + nb0) * KB + kb0 : sb0;
 
             float accr[128];
 #pragma unroll
             for (int i = 0; i < 128; ++i) accr[i] = 0.0f;
             bool ok = true;
-            for (int kb = 0; kb < KB; ++kb) {
-                const float a_s = row_ok ? sa[kb] : 0.0f;
-                const float c0 = nb_ok ? a_s * sb0[kb] : 0.0f;
-                const float c1 = MODE == 0 ? a_s * sb1[kb] : c0;
+            for (int kb = 0; kb < kbn; ++kb) {
+                float c0 = 1.0f, c1 = 1.0f;  // mode 2: plain sum of the K-block partials
+                if (MODE != 2) {
+                    const float a_s = row_ok ? sa[kb] : 0.0f;
+                    c0 = nb_ok ? a_s * sb0[kb] : 0.0f;
+                    c1 = MODE == 0 ? a_s * sb1[kb] : c0;
+                }
                 if (!mbar_wait(&S->accf[acc], aphase, g.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
@@ -290,6 +311,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                     const int col = MODE == 0 ? (c < 4 ? half * 64 + c * 16 : 128 + half * 64 + (c - 4) * 16)
                                               : half * 128 + c * 16;
                     const float cs = (MODE == 0 && c >= 4) ? c1 : c0;
+                    if (MODE == 2 && n0 + col >= g.N) continue;  // warp-uniform: columns past E
                     uint32_t r[16];
                     tmem_ld16_sync(tb + col, r);
 #pragma unroll
@@ -332,6 +354,22 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                     for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                     if (half == 0) g.out_s[(size_t)(row0 + row) * NB + n0 / 128] = sc;
                 }
+            } else if (MODE == 2) {
+                // partial logits of K split ks: [ksplit][M][N] fp32
+                const int col = n0 + half * 128;
+                if (row_ok && col < g.N) {
+                    float *dst = g.out_f32 + ((size_t)ks * g.M + row0 + row) * g.N + col;
+                    if (col + 128 <= g.N && (g.N & 3) == 0) {  // rows 16-byte aligned
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            reinterpret_cast<float4 *>(dst)[i] =
+                                make_float4(accr[4 * i], accr[4 * i + 1], accr[4 * i + 2], accr[4 * i + 3]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 128; ++i)
+                            if (col + i < g.N) dst[i] = accr[i];
+                    }
+                }
             } else {
                 const int col = n0 + half * 128;
                 if (row_ok && col < g.N) {
@@ -360,13 +398,15 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 bool fp8_smem_attr_ready(int mode)
 {
     static std::mutex mu;
-    static uint64_t done[2] = {0, 0};
+    static uint64_t done[3] = {0, 0, 0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::lock_guard<std::mutex> lk(mu);
     if (done[mode] >> dev & 1ull) return true;
-    cudaError_t e = mode == 0 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM8)
-                              : cudaFuncSetAttribute(grouped_gemm_fp8_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM8);
+    const int a = (int)SMEM8;
+    cudaError_t e = mode == 0 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                  : mode == 1 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                              : cudaFuncSetAttribute(grouped_gemm_fp8_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, a);
     if (e != cudaSuccess) return false;
     done[mode] |= 1ull << dev;
     return true;
@@ -389,9 +429,11 @@ cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const CUtensorMap &tmA
     const int grid = g.ctas > 0 ? g.ctas : num_sms();
     if (!fp8_smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
     if (g.mode == 0)
-        grouped_gemm_fp8_kernel<0><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
+        grouped_gemm_fp8_kernel<0, false><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
+    else if (g.mode == 1)
+        grouped_gemm_fp8_kernel<1, false><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
     else
-        grouped_gemm_fp8_kernel<1><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
+        grouped_gemm_fp8_kernel<2, true><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
     return cudaGetLastError();
 }
 

@@ -27,6 +27,7 @@
 //                   its 32-lane quarter), then
 //                   mode 0 (gate/up): h = silu(gate) * up, rounded to bf16,
 //                   mode 1 (down)   : y row of the assignment, rounded to bf16,
+//                   mode 2 (dense)  : fp32 rows (the router's tensor-core logits),
 //                   rows past the group's end masked.
 // Every accumulation order is fixed by the tile and the K loop, never by which
 // CTA ran the item, so results are bitwise independent of the schedule.
@@ -84,6 +85,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 {
     // output columns per tile: mode 0 packs 128 gate + 128 up columns into N=256
     constexpr int BNO = MODE == 0 ? BN / 2 : BN;
+    const bool dense = g.tiles == nullptr;  // mode 2: m-tiles are plain 128-row blocks of A
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *sA = smem_raw + pad;
@@ -123,7 +125,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (warp == 0) {
         // ------------------------------------------------ scheduler + TMA producer
         if (lane == 0) {
-            const int total = *g.ntiles * n_tiles;
+            const int total = (dense ? (g.M + BM - 1) / BM : *g.ntiles) * n_tiles;
             int stage = 0, rs = 0;
             uint32_t phase = 0, rphase = 0;
             uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
@@ -140,7 +142,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (++rs == RING) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
                 const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
-                const int expert = g.tiles[3 * mt], row0 = g.tiles[3 * mt + 1];
+                const int expert = dense ? 0 : g.tiles[3 * mt], row0 = dense ? mt * BM : g.tiles[3 * mt + 1];
                 const int n0 = nt * BNO;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
@@ -222,7 +224,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (++rs == RING) { rs = 0; rphase ^= 1; }
             if (item < 0) break;
             const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
-            const int row0 = g.tiles[3 * mt + 1], rows = g.tiles[3 * mt + 2];
+            const int row0 = dense ? mt * BM : g.tiles[3 * mt + 1];
+            const int rows = dense ? min(BM, g.M - row0) : g.tiles[3 * mt + 2];
             const bool row_ok = row < rows;
             if (!mbar_wait(&S->accf[acc], aphase, g.wait_ns)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
             tc_fence_after();
@@ -246,6 +249,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            } else if (MODE == 2) {
+                float *orow = g.out_f32 + (size_t)(row0 + row) * g.N;
+#pragma unroll 1
+                for (int c = 0; c < BNO / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32_sync(tb + c * 32, r);
+                    const int col = nt * BNO + c * 32;
+                    if (row_ok && col + 32 <= g.N && (g.N & 3) == 0) {  // rows 16-byte aligned
+                        float4 *dst = reinterpret_cast<float4 *>(orow + col);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                 __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                    } else if (row_ok && col < g.N) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (col + i < g.N) orow[col + i] = __uint_as_float(r[i]);
                     }
                 }
             } else {
@@ -299,13 +321,14 @@ int num_sms()
 static bool smem_attr_ready(int mode)
 {
     static std::mutex mu;
-    static uint64_t done[2] = {0, 0};  // bit per device
+    static uint64_t done[3] = {0, 0, 0};  // bit per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::lock_guard<std::mutex> lk(mu);
     if (done[mode] >> dev & 1ull) return true;
     cudaError_t e = mode == 0 ? cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)
-                              : cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+                  : mode == 1 ? cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)
+                              : cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return false;
     done[mode] |= 1ull << dev;
     return true;
@@ -318,8 +341,10 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const
     if (!smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
     if (g.mode == 0)
         grouped_gemm_kernel<0><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
-    else
+    else if (g.mode == 1)
         grouped_gemm_kernel<1><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
+    else
+        grouped_gemm_kernel<2><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
     return cudaGetLastError();
 }
 

@@ -144,6 +144,12 @@ T *at(void *ws, size_t off)
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+moe::RouterScratch router_scratch(void *ws, const moe::WsLayout &L)
+{
+    return moe::RouterScratch{at<__nv_bfloat16>(ws, L.wrt), at<float>(ws, L.wsq), at<int32_t>(ws, L.rncand),
+                              at<int32_t>(ws, L.rcand), at<moe::RouterCand>(ws, L.rlist)};
+}
+
 // Activations, weights and outputs are read and written in 16-byte vectors (and the
 // weights by TMA, which needs 16-byte aligned bases).
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -168,7 +174,8 @@ cudaError_t route_and_permute(const moe_dims_t &d, const moe::WsLayout &L, const
                                                         tiles, ntiles, hdr, st);
         return e == cudaSuccess ? marks.mark(1, st) : e;
     }
-    cudaError_t e = moe::launch_route(d, xb, wb, router_bias, at<float>(ws, L.logits), idx, gate, st);
+    cudaError_t e =
+        moe::launch_route(d, xb, wb, router_bias, at<float>(ws, L.logits), idx, gate, router_scratch(ws, L), hdr, st);
     if (e == cudaSuccess) e = marks.mark(1, st);
     if (e == cudaSuccess)
         e = moe::launch_permute(d, L, idx, at<int32_t>(ws, L.blk_cnt), at<int32_t>(ws, L.blk_base),
@@ -177,6 +184,28 @@ cudaError_t route_and_permute(const moe_dims_t &d, const moe::WsLayout &L, const
 }
 
 }  // namespace
+
+namespace moe {
+// The router's tensor-core logits: the block-promoting GEMM (fp8.cu, mode 2, bf16
+// operands) over plain 128-row blocks of x against the transposed router matrix,
+// K split over enough items to occupy the GPU.  Uses work counter 2.
+cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, int T, int H, int E, float *logits,
+                             WsHeader *hdr, int *ksplit_out, cudaStream_t st)
+{
+    CUtensorMap tm_x, tm_w;
+    if (!encode_2d(&tm_x, x, T, H, kTileRows) || !encode_3d(&tm_w, wrt, 1, E, H, 256)) return cudaErrorInvalidValue;
+    const int items = ((T + kTileRows - 1) / kTileRows) * ((E + 255) / 256);
+    int ks = (120 + items - 1) / items;
+    ks = ks < 1 ? 1 : ks > kRouterKSplitMax ? kRouterKSplitMax : ks;
+    if (ks > H / 64) ks = H / 64;
+    *ksplit_out = ks;
+    cudaError_t e = cudaMemsetAsync(&hdr->counter[2], 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return e;
+    Fp8GemmArgs g{2, H, E, nullptr, nullptr, &hdr->counter[2], &hdr->status, nullptr, nullptr, nullptr, nullptr,
+                  nullptr, nullptr, nullptr, 0, 0, 2000000000ull, 0, T, ks, logits};
+    return launch_grouped_gemm_fp8(g, tm_x, tm_w, tm_w, st);
+}
+}  // namespace moe
 
 extern "C" {
 
@@ -226,10 +255,13 @@ moe_status_t moe_route(const moe_dims_t *d, const void *x, const void *router_w,
     if (!aligned16(x) || !aligned16(router_w)) return MOE_ERR_INVALID_ARG;
     if ((s = check_ws(d, ws, ws_bytes)) != MOE_OK) return s;
     const moe::WsLayout L = moe::ws_layout(*d);
-    return cuda_status(moe::launch_route(*d, static_cast<const __nv_bfloat16 *>(x),
-                                         static_cast<const __nv_bfloat16 *>(router_w), router_bias,
-                                         at<float>(ws, L.logits), topk_idx, topk_w,
-                                         static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
+    if (e == cudaSuccess)
+        e = moe::launch_route(*d, static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(router_w),
+                              router_bias, at<float>(ws, L.logits), topk_idx, topk_w, router_scratch(ws, L),
+                              at<moe::WsHeader>(ws, 0), st);
+    return cuda_status(e);
 }
 
 moe_status_t moe_permute(const moe_dims_t *d, const int32_t *topk_idx, int32_t *expert_offsets,

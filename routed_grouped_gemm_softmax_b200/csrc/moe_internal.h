@@ -13,6 +13,7 @@ namespace moe {
 
 constexpr int kTileRows = MOE_TILE_ROWS;  // BM of the grouped GEMMs
 constexpr int kMaxExperts = 1024;
+constexpr int kRouterKSplitMax = 8;  // K slices of the router's tensor-core logits
 
 // Header at the start of every workspace.
 struct WsHeader {
@@ -23,7 +24,8 @@ struct WsHeader {
 
 // Byte offsets of every region of the workspace (256-byte aligned each).
 struct WsLayout {
-    size_t logits, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xs, xs_s, h, h_s, y, total;
+    size_t logits, wrt, wsq, rncand, rcand, rlist, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xs, xs_s, h, h_s, y,
+        total;
     int nb;      // permutation chunks
     int chunk;   // flat entries per chunk
 };
@@ -58,7 +60,13 @@ inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
         o = align_up(o + bytes, 1024);
         return at;
     };
-    L.logits = take(static_cast<size_t>(d.T) * d.E * 4);
+    L.logits = take(static_cast<size_t>(d.T) * d.E * 4 * kRouterKSplitMax);
+    L.wrt = take(static_cast<size_t>(d.E) * d.H * 2);
+    L.wsq = take(static_cast<size_t>(d.E) * 4);
+    const bool tc_router = d.T > 32;  // the certified router's candidate lists
+    L.rncand = take(tc_router ? static_cast<size_t>(d.T) * 4 : 0);
+    L.rcand = take(tc_router ? static_cast<size_t>(d.T) * d.E * 4 : 0);
+    L.rlist = take(tc_router ? static_cast<size_t>(d.T) * d.E * 16 : 0);
     L.blk_cnt = take(static_cast<size_t>(L.nb > 0 ? L.nb : 1) * d.E * 4);
     L.blk_base = take(static_cast<size_t>(L.nb > 0 ? L.nb : 1) * d.E * 4);
     L.idx = take(A * 4);
@@ -80,9 +88,26 @@ inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
 // ------------------------------------------------------------ launchers
 // Each returns cudaGetLastError() of its launch(es).
 
+// Candidate of the certified router: token, expert, tensor-core logit (+bias), bound.
+struct RouterCand {
+    int t, e;
+    float v, d;
+};
+
+// Scratch of the certified router (T > 32).
+struct RouterScratch {
+    __nv_bfloat16 *wrt;  // [E, H] router matrix, transposed
+    float *wsq;          // [E] squared column norms
+    int32_t *ncand;      // [T]
+    int32_t *cand;       // [T, E]
+    RouterCand *list;    // [T*E]
+};
+
+// Router: for T <= 32 the CUDA-core fp32 chains; above, tensor-core logits
+// certified against the chains.  Uses work counters 2 and 3 and the status word.
 cudaError_t launch_route(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
                          const float *bias, float *logits, int32_t *idx, float *gate,
-                         cudaStream_t st);
+                         const RouterScratch &rs, WsHeader *hdr, cudaStream_t st);
 
 // Router + permute in two launches for small batches (T <= 32, E % 8 == 0,
 // H % 128 == 0, T*k <= 4096).
@@ -119,12 +144,16 @@ struct GemmArgs {
     int reverse;
     uint64_t wait_ns;  // limit of each pipeline wait
     int stall_test;    // MMA thread first waits on a barrier nothing signals
+    int M;             // mode 2 (no tile list): rows of A
+    float *out_f32;    // mode 2: fp32 output [M, N]
 };
+// mode 2: out_f32 = A B^T over M rows (one "expert"), the router's tensor-core logits.
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
                                 const CUtensorMap &tmB1, cudaStream_t st);
 
 // FP8 block-scaled grouped GEMMs (fp8.cu).  mode 0: h codes/scales from
-// silu(A Wg^T) * (A Wu^T); mode 1: y[row_map[row]] = A Wd^T in bf16.
+// silu(A Wg^T) * (A Wu^T); mode 1: y[row_map[row]] = A Wd^T in bf16; mode 2:
+// bf16 A B^T summed per 64-wide K block into fp32 partials (router logits).
 struct Fp8GemmArgs {
     int mode;
     int K, N;
@@ -143,11 +172,20 @@ struct Fp8GemmArgs {
     int reverse;
     uint64_t wait_ns;
     int stall_test;
+    int M;            // mode 2: rows of A (no tile list)
+    int ksplit;       // mode 2: items per (m-tile, n-tile), each a slice of K
+    float *out_f32;   // mode 2: partial logits [ksplit, M, N]
 };
 cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
                                     const CUtensorMap &tmB1, cudaStream_t st);
 cudaError_t launch_quantize_rows(const __nv_bfloat16 *src, const int32_t *map, int k, int R, int K, uint8_t *q,
                                  float *s, cudaStream_t st);
+
+// Tensor-core router logits: partial sums over ksplit slices of H,
+// logits [ksplit, T, E] with sum_s logits[s] = x [T,H] . wrt [E,H]^T (fp32 per
+// 64-wide K block, then fp32 sums).  Returns ksplit through *ksplit_out.
+cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, int T, int H, int E, float *logits,
+                             WsHeader *hdr, int *ksplit_out, cudaStream_t st);
 
 int num_sms();
 

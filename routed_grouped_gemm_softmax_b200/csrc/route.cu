@@ -583,6 +583,296 @@ __global__ void __launch_bounds__(1024) topk_permute_small_kernel(int T, int E, 
     permute_in_cta(o.idx, T * k, E, o, reinterpret_cast<int *>(tsm) + nw * k);
 }
 
+
+// ------------------------------------------------------------------------
+// Large batches: tensor-core logits certified against the fp32 chain.
+//
+// The router's logit is defined by the fp32 FMA chain; computing all T*E chains
+// costs 2*T*H*E CUDA-core flops.  For T > 32 the chain is instead evaluated only
+// where it can change the answer:
+//  1. Lt = x . Wr on the tensor cores (bf16 in, fp32 accumulate), each 64-wide K
+//     block summed out of TMEM in fp32 and K split over a few slices, against Wr
+//     transposed to [E, H] once per call.
+//  2. Per token, a bound |chain - Lt| <= d_e: the chain's own rounding is at most
+//     H u sum_h |x_h w_he| (u = 2^-24, recursive summation with fma), the
+//     tensor-core value's at most (64 * 4u + (H/64 + slices) u) times the same sum
+//     (each 64-term block accumulated within 4 ulps, then one rounding per block and
+//     slice sum); sum_h |x_h w_he| <= |x_t| |w_e| (Cauchy-Schwarz); 1% margin, plus
+//     a few ulps of the bias add and of the values themselves.
+//  3. tau = the k-th largest lower bound Lt - d.  An expert whose upper bound
+//     Lt + d is below tau has k experts strictly above it, so it cannot be chosen.
+//     The remaining candidates (k of them plus near-ties) go to a compact list
+//     (kernel C1, a warp per token), get the exact chain (C2, a thread per
+//     candidate), and top-k + softmax run on those exact values (C3).
+//  4. Every candidate's exact value is checked against its bound; a miss records
+//     MOE_ERR_ROUTER_BOUND in the status word.
+// The chosen experts and gates are therefore those of the chain definition.
+
+__global__ void router_transpose_kernel(const __nv_bfloat16 *__restrict__ wr, int H, int E,
+                                        __nv_bfloat16 *__restrict__ wrt)
+{
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int h0 = blockIdx.y * 32, e0 = blockIdx.x * 32;
+    const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;  // 32 x 8 threads
+    for (int r = ty; r < 32; r += 8) {
+        const int h = h0 + r, e = e0 + tx;
+        tile[r][tx] = (h < H && e < E) ? wr[(size_t)h * E + e] : __float2bfloat16(0.0f);
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const int e = e0 + r, h = h0 + tx;
+        if (e < E && h < H) wrt[(size_t)e * H + h] = tile[tx][r];
+    }
+}
+
+// Squared norm of each router column (warp per expert, fp32; the bound inflates it).
+__global__ void router_colnorm_kernel(const __nv_bfloat16 *__restrict__ wrt, int H, int E, float *__restrict__ wsq)
+{
+    const int e = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (e >= E) return;
+    float s = 0.0f;
+    for (int h = lane * 8; h < H; h += 256) {
+        float f[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(wrt + (size_t)e * H + h), f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s = fmaf(f[i], f[i], s);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) wsq[e] = s;
+}
+
+// The exact chain of one (token, expert): fma over h ascending from 0, operands
+// streamed from global memory (L1/L2) sixteen 16-byte loads ahead so that the
+// loads' latency hides behind the chain.
+__device__ __forceinline__ float exact_chain(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w,
+                                             int H)
+{
+    constexpr int D = 16;  // loads in flight per operand
+    const uint4 *w4 = reinterpret_cast<const uint4 *>(w);
+    const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
+    const int n8 = H / 8;  // H is a multiple of 64
+    float acc = 0.0f;
+    uint4 wq[D], xq[D];
+#pragma unroll
+    for (int j = 0; j < D; ++j) {
+        wq[j] = j < n8 ? w4[j] : make_uint4(0, 0, 0, 0);
+        xq[j] = j < n8 ? x4[j] : make_uint4(0, 0, 0, 0);
+    }
+    for (int b = 0; b < n8; b += D) {
+#pragma unroll
+        for (int j = 0; j < D; ++j) {
+            if (b + j < n8) {
+                const uint4 wv = wq[j], xv = xq[j];
+                if (b + j + D < n8) {
+                    wq[j] = w4[b + j + D];
+                    xq[j] = x4[b + j + D];
+                }
+                const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w}, xx[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc = fmaf(__uint_as_float(xx[i] << 16), __uint_as_float(ww[i] << 16), acc);
+                    acc = fmaf(__uint_as_float(xx[i] & 0xFFFF0000u), __uint_as_float(ww[i] & 0xFFFF0000u), acc);
+                }
+            }
+        }
+    }
+    return acc;
+}
+
+struct CertifyArgs {
+    const float *lt;        // [ksplit, T, E] partial tensor-core logits; slice 0 later holds exact values
+    int ksplit;
+    const __nv_bfloat16 *x, *wrt;
+    const float *wsq, *bias;
+    int T, H, E, k;
+    float eps;
+    int32_t *ncand;         // [T] candidates per token
+    int32_t *cand;          // [T, E] candidate experts, ascending
+    RouterCand *list;       // compact list of all candidates
+    int32_t *list_len;
+    float *ex;              // [T, E] exact chain values (written for candidates only)
+    int32_t *idx;
+    float *gate;
+    int32_t *status;
+};
+
+// C1: bounds and candidates, one warp per token.
+template <int MAXV>
+__global__ void __launch_bounds__(256) router_candidates_kernel(const CertifyArgs a)
+{
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int t = blockIdx.x * (blockDim.x / 32) + warp;
+    if (t >= a.T) return;
+    const int E = a.E, H = a.H;
+    // tensor-core logits (sum of the K slices) first, so their loads overlap the norm
+    float v[MAXV], d[MAXV];
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) v[i] = 0.0f;
+    for (int q = 0; q < a.ksplit; ++q) {
+        const float *row = a.lt + ((size_t)q * a.T + t) * E;
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) v[i] += row[e];
+        }
+    }
+    float ss = 0.0f;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)t * H);
+#pragma unroll 4
+    for (int h8 = lane; h8 < H / 8; h8 += 32) {
+        float f[8];
+        bf16x8_to_f32(xr[h8], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(f[i], f[i], ss);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float xn = sqrtf(ss) * 1.001f;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            float s = v[i];
+            if (a.bias) s += a.bias[e];
+            v[i] = s;
+            d[i] = a.eps * xn * sqrtf(a.wsq[e]) * 1.001f + fabsf(s) * 4.8e-7f + 1e-30f;
+        } else {
+            v[i] = -INFINITY;
+            d[i] = 0.0f;
+        }
+    }
+    // tau: the k-th largest lower bound v - d
+    uint32_t taken = 0;
+    float tau = -INFINITY;
+    for (int j = 0; j < a.k; ++j) {
+        float bv = -INFINITY;
+        int be = INT_MAX;
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) {
+            const int e = lane + 32 * i;
+            const float lo = v[i] - d[i];
+            if (e < E && !((taken >> i) & 1u) && (be == INT_MAX || lo > bv)) {
+                bv = lo;
+                be = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        tau = bv;
+    }
+    // candidates (upper bound >= tau), ascending expert index, appended contiguously
+    int nc = 0;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const int e = lane + 32 * i;
+        nc += __popc(__ballot_sync(0xffffffffu, e < E && v[i] + d[i] >= tau));
+    }
+    int base = 0;
+    if (lane == 0) base = atomicAdd(a.list_len, nc);
+    base = __shfl_sync(0xffffffffu, base, 0);
+    int pos = 0;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const int e = lane + 32 * i;
+        const bool c = e < E && v[i] + d[i] >= tau;
+        const unsigned m = __ballot_sync(0xffffffffu, c);
+        if (c) {
+            const int p = pos + __popc(m & ((1u << lane) - 1u));
+            a.cand[(size_t)t * E + p] = e;
+            a.list[base + p] = RouterCand{t, e, v[i], d[i]};
+        }
+        pos += __popc(m);
+    }
+    if (lane == 0) a.ncand[t] = nc;
+}
+
+// C2: the exact chain of every candidate, one thread each; checked against its bound.
+__global__ void __launch_bounds__(128) router_chains_kernel(const CertifyArgs a)
+{
+    const int n = *a.list_len;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const RouterCand c = a.list[i];
+        float v = exact_chain(a.x + (size_t)c.t * a.H, a.wrt + (size_t)c.e * a.H, a.H);
+        if (a.bias) v = __fadd_rn(v, a.bias[c.e]);
+        a.ex[(size_t)c.t * a.E + c.e] = v;
+        if (!(fabsf(v - c.v) <= c.d)) atomicCAS(a.status, 0, MOE_ERR_ROUTER_BOUND);
+    }
+}
+
+// C3: top-k (larger exact value first, lower index on ties) and softmax among each
+// token's candidates, one warp per token; the candidates' values are loaded once.
+template <int MAXV>
+__global__ void __launch_bounds__(256) router_select_kernel(const CertifyArgs a)
+{
+    extern __shared__ float rsel[];  // [warps][k]
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int t = blockIdx.x * (blockDim.x / 32) + warp;
+    if (t >= a.T) return;
+    float *sv = rsel + (size_t)warp * a.k;
+    const int nc = a.ncand[t];
+    const int *cand = a.cand + (size_t)t * a.E;
+    const float *ex = a.ex + (size_t)t * a.E;
+    int ce[MAXV];
+    float cv[MAXV];
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const int c = lane + 32 * i;
+        ce[i] = c < nc ? cand[c] : INT_MAX;
+    }
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) cv[i] = ce[i] != INT_MAX ? ex[ce[i]] : 0.0f;
+    for (int j = 0; j < a.k; ++j) {
+        float bv = 0.0f;
+        int be = INT_MAX, bi = -1;
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i)
+            if (ranks_before(cv[i], ce[i], bv, be)) {
+                bv = cv[i];
+                be = ce[i];
+                bi = i;
+            }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (ranks_before(ov, oe, bv, be)) {
+                bv = ov;
+                be = oe;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i)
+            if (i == bi && ce[i] == be) ce[i] = INT_MAX;  // taken
+        if (lane == 0) {
+            a.idx[(size_t)t * a.k + j] = be;
+            sv[j] = bv;
+        }
+    }
+    __syncwarp();
+    const float m = sv[0];
+    float s = 0.0f;
+    for (int j = lane; j < a.k; j += 32) s += expf(sv[j] - m);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    for (int j = lane; j < a.k; j += 32) a.gate[(size_t)t * a.k + j] = expf(sv[j] - m) / s;
+}
+
+template <int MAXV>
+cudaError_t launch_candidates(const CertifyArgs &a, cudaStream_t st)
+{
+    router_candidates_kernel<MAXV><<<(a.T + 7) / 8, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool small_route_permute_ok(const moe_dims_t &d)
@@ -632,12 +922,45 @@ cudaError_t launch_route_permute_small(const moe_dims_t &d, const __nv_bfloat16 
 
 cudaError_t launch_route(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
                          const float *bias, float *logits, int32_t *idx, float *gate,
-                         cudaStream_t st)
+                         const RouterScratch &rs, WsHeader *hdr, cudaStream_t st)
 {
     const int T = d.T, H = d.H, E = d.E, k = d.top_k;
+    int32_t *status = &hdr->status;
+    __nv_bfloat16 *wrt = rs.wrt;
+    float *wsq = rs.wsq;
+    cudaError_t e;
+    const int vpl = (E + 31) / 32;
+    if (T > 32) {
+        dim3 tg((E + 31) / 32, (H + 31) / 32);
+        router_transpose_kernel<<<tg, 256, 0, st>>>(wr, H, E, wrt);
+        router_colnorm_kernel<<<(E + 7) / 8, 256, 0, st>>>(wrt, H, E, wsq);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        int ks = 1;
+        if ((e = tc_router_logits(x, wrt, T, H, E, logits, hdr, &ks, st)) != cudaSuccess) return e;
+        const float u = 5.9604644775390625e-08f;  // 2^-24
+        const float eps = ((float)H * u + 256.0f * u + (float)(H / 64 + ks) * u) * 1.01f;
+        CertifyArgs a{logits, ks, x, wrt, wsq, bias, T, H, E, k, eps, rs.ncand, rs.cand, rs.list, &hdr->counter[3],
+                      logits, idx, gate, status};
+        if ((e = cudaMemsetAsync(&hdr->counter[3], 0, sizeof(int32_t), st)) != cudaSuccess) return e;
+        if (vpl <= 1) e = launch_candidates<1>(a, st);
+        else if (vpl <= 2) e = launch_candidates<2>(a, st);
+        else if (vpl <= 4) e = launch_candidates<4>(a, st);
+        else if (vpl <= 8) e = launch_candidates<8>(a, st);
+        else if (vpl <= 16) e = launch_candidates<16>(a, st);
+        else e = launch_candidates<32>(a, st);
+        if (e != cudaSuccess) return e;
+        router_chains_kernel<<<num_sms() * 8, 128, 0, st>>>(a);
+        const size_t ssm = (size_t)8 * k * sizeof(float);
+        if (vpl <= 1) router_select_kernel<1><<<(T + 7) / 8, 256, ssm, st>>>(a);
+        else if (vpl <= 2) router_select_kernel<2><<<(T + 7) / 8, 256, ssm, st>>>(a);
+        else if (vpl <= 4) router_select_kernel<4><<<(T + 7) / 8, 256, ssm, st>>>(a);
+        else if (vpl <= 8) router_select_kernel<8><<<(T + 7) / 8, 256, ssm, st>>>(a);
+        else if (vpl <= 16) router_select_kernel<16><<<(T + 7) / 8, 256, ssm, st>>>(a);
+        else router_select_kernel<32><<<(T + 7) / 8, 256, ssm, st>>>(a);
+        return cudaGetLastError();
+    }
     // Pick the tile so that enough warps exist to cover the SMs: small batches get
     // one chain per thread, large ones register-blocked 8x4 or 4x4 chains.
-    cudaError_t e;
     const long tiles64 = (long)((T + 63) / 64) * ((E + 63) / 64);
     if (T <= 16 && E % 8 == 0 && H % 128 == 0)
         e = launch_logits_small<16, 8, 128, 16>(x, wr, bias, T, H, E, logits, st);
@@ -650,7 +973,6 @@ cudaError_t launch_route(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv
     else
         e = launch_logits<32, 64, 4, 4, 32>(x, wr, bias, T, H, E, logits, st);
     if (e != cudaSuccess) return e;
-    const int vpl = (E + 31) / 32;
     if (vpl <= 1) return launch_topk<1>(logits, T, E, k, idx, gate, st);
     if (vpl <= 2) return launch_topk<2>(logits, T, E, k, idx, gate, st);
     if (vpl <= 4) return launch_topk<4>(logits, T, E, k, idx, gate, st);
