@@ -155,13 +155,16 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
  * fp32 scales, per row per 128 columns as described above.  Needs no workspace. */
 moe_status_t moe_quantize_rows_fp8(int32_t R, int32_t K, const void *a, uint8_t *q, float *s, void *stream);
 
-/* Where the last moe_forward / moe_forward_fp8 left its routing inside the
- * workspace, for inspection: out[i] receives the byte offset of
+/* Where the last moe_route / moe_forward / moe_forward_fp8 on this workspace
+ * left its routing, for inspection: out[i] receives the byte offset of
  *   0 topk_idx [T,k] int32    1 topk_w [T,k] fp32      2 expert_offsets [E+1]
  *   3 sorted_to_flat [T*k]    4 flat_to_sorted [T*k]    5 tile_list [3*max_tiles]
- *   6 num_tiles [1]
- * (same meaning as the outputs of moe_route and moe_permute).  Writes
- * min(n, 7) entries; returns MOE_ERR_INVALID_ARG for invalid dims or dtype. */
+ *   6 num_tiles [1]           7 logits [T,E] fp32
+ * (0-6 as the outputs of moe_route and moe_permute; 0-1 after moe_route only
+ * when it was given the workspace's own regions).  Entry 7 holds the router's
+ * fp32 chain value (bias included) of every (t,e) when T <= 32, and of at least
+ * each token's chosen experts when T > 32.  Writes min(n, 8) entries; returns
+ * MOE_ERR_INVALID_ARG for invalid dims or dtype. */
 moe_status_t moe_workspace_offsets(const moe_dims_t *d, int dtype, size_t *out, int32_t n);
 
 /* Synchronises `stream`, returns the device status word of the workspace

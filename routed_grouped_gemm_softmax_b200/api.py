@@ -252,9 +252,11 @@ def moe_forward_noalloc(x, router_w, bias, w_gate, w_up, w_down, top_k: int, out
 
 def forward_routing(ws, T, H, I, E, top_k, dtype: int = DTYPE_BF16) -> dict:
     """Views into the workspace of the routing the last forward on it computed
-    (topk_idx, topk_w, offsets, sorted_to_flat, flat_to_sorted, tile_list, num_tiles)."""
-    offs = (ctypes.c_size_t * 7)()
-    _check(lib().moe_workspace_offsets(ctypes.byref(dims(T, H, I, E, top_k)), int(dtype), offs, 7),
+    (topk_idx, topk_w, offsets, sorted_to_flat, flat_to_sorted, tile_list, num_tiles,
+    and the router's fp32 logits [T, E]: every entry for T <= 32, at least the chosen
+    experts' entries above)."""
+    offs = (ctypes.c_size_t * 8)()
+    _check(lib().moe_workspace_offsets(ctypes.byref(dims(T, H, I, E, top_k)), int(dtype), offs, 8),
            "moe_workspace_offsets")
     A = T * top_k
     nt = moe_max_tiles(T, H, I, E, top_k)
@@ -265,7 +267,7 @@ def forward_routing(ws, T, H, I, E, top_k, dtype: int = DTYPE_BF16) -> dict:
     return {"topk_idx": view(0, A, torch.int32).view(T, top_k), "topk_w": view(1, A, torch.float32).view(T, top_k),
             "offsets": view(2, E + 1, torch.int32), "sorted_to_flat": view(3, A, torch.int32),
             "flat_to_sorted": view(4, A, torch.int32), "tile_list": view(5, 3 * nt, torch.int32).view(nt, 3),
-            "num_tiles": view(6, 1, torch.int32)}
+            "num_tiles": view(6, 1, torch.int32), "logits": view(7, T * E, torch.float32).view(T, E)}
 
 
 def moe_get_device_status(ws, stream=None) -> int:

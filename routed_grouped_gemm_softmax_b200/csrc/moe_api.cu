@@ -147,7 +147,7 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
 moe::RouterScratch router_scratch(void *ws, const moe::WsLayout &L)
 {
     return moe::RouterScratch{at<__nv_bfloat16>(ws, L.wrt), at<float>(ws, L.wsq), at<int32_t>(ws, L.rncand),
-                              at<int32_t>(ws, L.rcand), at<moe::RouterCand>(ws, L.rlist)};
+                              at<moe::RouterCand>(ws, L.rlist)};
 }
 
 // Activations, weights and outputs are read and written in 16-byte vectors (and the
@@ -186,6 +186,27 @@ cudaError_t route_and_permute(const moe_dims_t &d, const moe::WsLayout &L, const
 }  // namespace
 
 namespace moe {
+// bf16 matrix [rows, cols] (row-major), tiles of box_rows x box_cols, no swizzle.
+bool encode_plain_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                          uint32_t box_rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 matrix [rows, cols], tiles of box_rows x 64 with the 128-byte swizzle.
+bool encode_sw128_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    return encode_2d(m, base, rows, cols, box_rows);
+}
+
 // The router's tensor-core logits: the block-promoting GEMM (fp8.cu, mode 2, bf16
 // operands) over plain 128-row blocks of x against the transposed router matrix,
 // K split over enough items to occupy the GPU.  Uses work counter 2.
@@ -422,8 +443,8 @@ moe_status_t moe_workspace_offsets(const moe_dims_t *d, int dtype, size_t *out, 
 {
     if (!out || n < 0 || moe_workspace_size(d, dtype) == 0) return MOE_ERR_INVALID_ARG;
     const moe::WsLayout L = moe::ws_layout(*d, dtype);
-    const size_t v[7] = {L.idx, L.gate, L.offsets, L.s2f, L.f2s, L.tiles, L.ntiles};
-    for (int i = 0; i < n && i < 7; ++i) out[i] = v[i];
+    const size_t v[8] = {L.idx, L.gate, L.offsets, L.s2f, L.f2s, L.tiles, L.ntiles, L.logits};
+    for (int i = 0; i < n && i < 8; ++i) out[i] = v[i];
     return MOE_OK;
 }
 

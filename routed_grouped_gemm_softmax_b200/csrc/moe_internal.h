@@ -24,7 +24,7 @@ struct WsHeader {
 
 // Byte offsets of every region of the workspace (256-byte aligned each).
 struct WsLayout {
-    size_t logits, wrt, wsq, rncand, rcand, rlist, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xs, xs_s, h, h_s, y,
+    size_t logits, wrt, wsq, rncand, rlist, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xs, xs_s, h, h_s, y,
         total;
     int nb;      // permutation chunks
     int chunk;   // flat entries per chunk
@@ -62,10 +62,9 @@ inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
     };
     L.logits = take(static_cast<size_t>(d.T) * d.E * 4 * kRouterKSplitMax);
     L.wrt = take(static_cast<size_t>(d.E) * d.H * 2);
-    L.wsq = take(static_cast<size_t>(d.E) * 4);
+    L.wsq = take(static_cast<size_t>(d.E) * 4 * ((d.H + 255) / 256));  // partial squared norms
     const bool tc_router = d.T > 32;  // the certified router's candidate lists
     L.rncand = take(tc_router ? static_cast<size_t>(d.T) * 4 : 0);
-    L.rcand = take(tc_router ? static_cast<size_t>(d.T) * d.E * 4 : 0);
     L.rlist = take(tc_router ? static_cast<size_t>(d.T) * d.E * 16 : 0);
     L.blk_cnt = take(static_cast<size_t>(L.nb > 0 ? L.nb : 1) * d.E * 4);
     L.blk_base = take(static_cast<size_t>(L.nb > 0 ? L.nb : 1) * d.E * 4);
@@ -97,20 +96,23 @@ struct RouterCand {
 // Scratch of the certified router (T > 32).
 struct RouterScratch {
     __nv_bfloat16 *wrt;  // [E, H] router matrix, transposed
-    float *wsq;          // [E] squared column norms
-    int32_t *ncand;      // [T]
-    int32_t *cand;       // [T, E]
-    RouterCand *list;    // [T*E]
+    float *wsq;          // [ceil(H/256), E] partial squared column norms
+    int32_t *ncand;      // [T] candidates per token
+    RouterCand *list;    // [T, E] candidates of each token, ascending expert index
 };
 
-// Router: for T <= 32 the CUDA-core fp32 chains; above, tensor-core logits
-// certified against the chains.  Uses work counters 2 and 3 and the status word.
+// Router: for T <= 32 the CUDA-core fp32 chains (route.cu); above, tensor-core
+// logits certified against the chains (route_certified.cu).  Uses work counter 2
+// and the status word.
 cudaError_t launch_route(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
                          const float *bias, float *logits, int32_t *idx, float *gate,
                          const RouterScratch &rs, WsHeader *hdr, cudaStream_t st);
+cudaError_t launch_route_certified(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
+                                   const float *bias, float *logits, int32_t *idx, float *gate,
+                                   const RouterScratch &rs, WsHeader *hdr, cudaStream_t st);
 
 // Router + permute in two launches for small batches (T <= 32, E % 8 == 0,
-// H % 128 == 0, T*k <= 4096).
+// H % 128 == 0, T*k <= 4096, ceil(T*k/32) * E <= 16384).
 bool small_route_permute_ok(const moe_dims_t &d);
 cudaError_t launch_route_permute_small(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
                                        const float *bias, float *logits, int32_t *idx, float *gate,
@@ -188,5 +190,13 @@ cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, i
                              WsHeader *hdr, int *ksplit_out, cudaStream_t st);
 
 int num_sms();
+
+// Tensor map of a row-major bf16 matrix [rows, cols], box_rows x box_cols tiles,
+// no swizzle (box_cols * 2 a multiple of 16).
+// Tensor map of a row-major bf16 matrix [rows, cols], box_rows x 64 tiles with the
+// 128-byte swizzle (16-byte chunk c of tile row r stored at chunk c ^ (r % 8)).
+bool encode_sw128_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool encode_plain_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                          uint32_t box_rows);
 
 }  // namespace moe

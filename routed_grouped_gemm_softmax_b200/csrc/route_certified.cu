@@ -1,0 +1,447 @@
+// route_certified.cu -- the router for batches of more than 32 tokens: tensor-core
+// logits, certified against the fp32 chain that defines the routing.
+//
+// The router's logit is the fp32 FMA chain over h ascending (route.cu states the
+// contract).  Evaluating all T*E chains costs 2*T*H*E CUDA-core flops, so for large
+// batches the chain is evaluated only where it can change the answer:
+//  1. router_prep_kernel transposes router_w to [E, H] and takes partial squared
+//     column norms (per 256 rows), summed per expert by the certify kernel;
+//  2. Lt = x . Wr on the tensor cores (fp8.cu, mode 2: bf16 in, each 64-wide K
+//     block summed out of TMEM in fp32, K split over a few slices);
+//  3. router_certify_kernel, a CTA per block of tokens:
+//     a. per token (a warp), a bound |chain - Lt| <= d_e: the chain's own rounding
+//        is at most H u sum_h |x_h w_he| (u = 2^-24, recursive summation with fma),
+//        the tensor-core value's at most (64 * 4u + (H/64 + slices) u) times the
+//        same sum (each 64-term block accumulated within 4 ulps, then one rounding
+//        per block and slice sum); sum_h |x_h w_he| <= |x_t| |w_e| (Cauchy-Schwarz);
+//        1% margin, plus a few ulps of the bias add and of the values themselves.
+//        tau = the k-th largest lower bound Lt - d; an expert whose upper bound
+//        Lt + d is below tau has k experts strictly above it and cannot be chosen.
+//        The others -- the k chosen plus near-ties -- are the token's candidates;
+//     b. the exact chain of every candidate of the block: the block's x rows and
+//        all of router_w^T stream through shared memory in chunks of h (tensor-map
+//        tiles, up to three stages on mbarriers), each thread running one or two
+//        chains with the mixed-precision chain step; each exact value is checked
+//        against its bound (a miss records MOE_ERR_ROUTER_BOUND);
+//     c. per token (a warp), top-k and softmax on the candidates' exact values.
+// The chosen experts and gates are therefore those of the chain definition.
+#include <cfloat>
+#include <climits>
+
+#include "moe_internal.h"
+#include "route_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kPrepE = 16;     // experts per CTA of router_prep_kernel
+constexpr int kPrepH = 256;    // h rows per CTA
+
+// Wr [H, E] -> wrt [E, H] (one 256 x 16 tile per CTA), and the partial squared
+// column norms wsq_part[h / 256][e] = sum over the tile's rows of Wr[h, e]^2 (fp32;
+// the bound inflates it).
+__global__ void __launch_bounds__(256) router_prep_kernel(const __nv_bfloat16 *__restrict__ wr, int H, int E,
+                                                          __nv_bfloat16 *__restrict__ wrt,
+                                                          float *__restrict__ wsq_part)
+{
+    __shared__ uint16_t tile[kPrepH][kPrepE + 2];
+    const int tid = threadIdx.x;
+    const int e0 = blockIdx.x * kPrepE, h0 = blockIdx.y * kPrepH;
+    const uint16_t *w16 = reinterpret_cast<const uint16_t *>(wr);
+    uint16_t *o16 = reinterpret_cast<uint16_t *>(wrt);
+    {
+        constexpr int kSteps = kPrepH / (256 / kPrepE);  // 16 threads per row, all loads in flight together
+        uint16_t v[kSteps];
+        const int e = e0 + tid % kPrepE;
+#pragma unroll
+        for (int i = 0; i < kSteps; ++i) {
+            const int h = h0 + tid / kPrepE + i * (256 / kPrepE);
+            v[i] = (h < H && e < E) ? w16[(size_t)h * E + e] : uint16_t(0);
+        }
+#pragma unroll
+        for (int i = 0; i < kSteps; ++i) tile[tid / kPrepE + i * (256 / kPrepE)][tid % kPrepE] = v[i];
+    }
+    __syncthreads();
+    // thread (el, part): rows r = part mod 16 of expert el, then a 16-lane tree
+    const int el = tid / 16, part = tid % 16;
+    float ss = 0.0f;
+    for (int r = part; r < kPrepH; r += 16) {
+        const float f = __uint_as_float(static_cast<uint32_t>(tile[r][el]) << 16);
+        ss = fmaf(f, f, ss);
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (part == 0 && e0 + el < E) wsq_part[(size_t)blockIdx.y * E + e0 + el] = ss;
+    for (int v = tid; v < kPrepE * kPrepH; v += 256) {  // 16 expert rows of 256 values
+        const int ee = v / kPrepH, r = v % kPrepH;
+        const int h = h0 + r, e = e0 + ee;
+        if (h < H && e < E) o16[(size_t)e * H + h] = tile[r][ee];
+    }
+}
+
+constexpr int kCertThreads = 512;
+constexpr int kCertWarps = kCertThreads / 32;
+constexpr int kCertMaxStages = 3;
+constexpr int kCertChains = 2;  // chains per thread per round
+constexpr int kCertMaxTB = 64;  // tokens per CTA
+constexpr int kCertSmem = 227 * 1024;
+
+struct CertifyArgs {
+    const float *lt;        // [ksplit, T, E] partial tensor-core logits
+    float *ex;              // = lt slice 0: receives the exact values of the chosen experts
+    int ksplit;
+    const __nv_bfloat16 *x;
+    const float *wsq_part, *bias;  // wsq_part [nparts, E]
+    int nparts;
+    int T, H, E, k, TB;
+    float eps;
+    int32_t *ncand;         // [T] candidates per token
+    RouterCand *list;       // [T, E] the candidates of token t in slots t*E .. t*E + ncand[t] - 1, ascending e;
+                            // after the chains, .v holds the exact value
+    int32_t *idx;
+    float *gate;
+    int32_t *status;
+    int xrows;              // rows of an x tile (TB rounded up to 8)
+    int erows;              // staged router rows (E rounded up to 8, or to 256 above 256)
+    int ebox;               // rows of one router tile (<= 256)
+    int nbx;                // 64-column tiles per chunk
+    int stages;             // 1..kCertMaxStages
+    int stage_bytes;        // nbx * (xrows + erows) * 128
+};
+
+// Fixed part of the dynamic shared memory: the stage barriers, per-token counts and
+// prefix, squared expert norms, per-warp top-k outputs; the stages follow at a
+// 1024-byte boundary (the 128-byte swizzle repeats every 8 rows of 128 bytes).
+__host__ __device__ inline size_t cert_fixed_bytes(int E, int k)
+{
+    const size_t words = (size_t)kCertMaxTB + (kCertMaxTB + 1) + E + 8 + (size_t)2 * kCertWarps * k;
+    return (kCertMaxStages * 8 + words * 4 + 1023) / 1024 * 1024;
+}
+
+// 16-byte chunk j (0..7) of row r of a 128-byte-swizzled tile.
+__device__ __forceinline__ const uint4 *sw128_chunk(const uint8_t *tile, int r, int j)
+{
+    return reinterpret_cast<const uint4 *>(tile + r * 128 + ((j ^ (r & 7)) << 4));
+}
+
+template <int MAXV>
+__global__ void __launch_bounds__(kCertThreads)
+    router_certify_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                          const CertifyArgs a)
+{
+    extern __shared__ __align__(128) uint8_t csm[];
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    const int E = a.E, H = a.H, k = a.k;
+    const int t0 = blockIdx.x * a.TB;
+    const int tb = min(a.TB, a.T - t0);
+    uint64_t *full = reinterpret_cast<uint64_t *>(csm);        // [kCertMaxStages] staging barriers
+    int *nc = reinterpret_cast<int *>(full + kCertMaxStages);  // [kCertMaxTB]
+    int *cb = nc + kCertMaxTB;                                  // [kCertMaxTB + 1] chain prefix over tokens
+    float *wsq = reinterpret_cast<float *>(cb + kCertMaxTB + 1);  // [E] squared norms of the router columns
+    int *misc = reinterpret_cast<int *>(wsq + E);               // [8]: 1 chains
+    int *wse = misc + 8;                                        // [warps][k]
+    float *wsv = reinterpret_cast<float *>(wse + kCertWarps * k);  // [warps][k]
+    // stages at a 1024-byte boundary of the shared address space (the launch adds 1 KB of slack)
+    const uint32_t fixed_end = smem_u32(csm) + (uint32_t)cert_fixed_bytes(E, k);
+    uint8_t *stage0 = csm + (((fixed_end + 1023u) & ~1023u) - smem_u32(csm));
+
+    if (tid == 0) {
+        for (int s = 0; s < kCertMaxStages; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    for (int e = tid; e < E; e += kCertThreads) {
+        float q = 0.0f;
+        for (int j = 0; j < a.nparts; ++j) q += a.wsq_part[(size_t)j * E + e];
+        wsq[e] = q;
+    }
+    __syncthreads();
+
+    // ---- a. bounds and candidates, a warp per token
+    for (int tl = warp; tl < tb; tl += kCertWarps) {
+        const int t = t0 + tl;
+        float v[MAXV], d[MAXV];
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) v[i] = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kRouterKSplitMax; ++q) {  // slices summed in order; loads issued together
+            if (q < a.ksplit) {
+                const float *row = a.lt + ((size_t)q * a.T + t) * E;
+#pragma unroll
+                for (int i = 0; i < MAXV; ++i) {
+                    const int e = lane + 32 * i;
+                    if (e < E) v[i] += row[e];
+                }
+            }
+        }
+        float ss = 0.0f;
+        const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)t * H);
+#pragma unroll 8
+        for (int h8 = lane; h8 < H / 8; h8 += 32) {
+            const uint4 q = xr[h8];
+            const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float lo = __uint_as_float(w4[i] << 16), hi = __uint_as_float(w4[i] & 0xFFFF0000u);
+                ss = fmaf(lo, lo, ss);
+                ss = fmaf(hi, hi, ss);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float xn = sqrtf(ss) * 1.001f;
+        uint32_t key[MAXV];
+        float lo[MAXV];
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) {
+                float s = v[i];
+                if (a.bias) s += a.bias[e];
+                v[i] = s;
+                d[i] = a.eps * xn * sqrtf(wsq[e]) * 1.001f + fabsf(s) * 4.8e-7f + 1e-30f;
+                lo[i] = v[i] - d[i];
+                key[i] = order_key(lo[i]);
+            } else {
+                v[i] = -INFINITY;
+                d[i] = 0.0f;
+                lo[i] = 0.0f;
+                key[i] = 0u;
+            }
+        }
+        // tau: the k-th largest lower bound
+        warp_topk<MAXV>(key, lo, k, wse + warp * k, wsv + warp * k);
+        const float tau = wsv[warp * k + k - 1];
+        // candidates (upper bound >= tau), ascending expert index
+        RouterCand *out = a.list + (size_t)t * E;
+        int pos = 0;
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) {
+            const int e = lane + 32 * i;
+            const bool c = e < E && v[i] + d[i] >= tau;
+            const unsigned m = __ballot_sync(0xffffffffu, c);
+            if (c) out[pos + __popc(m & ((1u << lane) - 1u))] = RouterCand{t, e, v[i], d[i]};
+            pos += __popc(m);
+        }
+        if (lane == 0) {
+            nc[tl] = pos;
+            a.ncand[t] = pos;
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+
+    // chain prefix over the block's tokens (tb <= 64: two tokens per lane)
+    if (warp == 0) {
+        const int c0 = lane < tb ? nc[lane] : 0, c1 = lane + 32 < tb ? nc[lane + 32] : 0;
+        int i0 = c0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, i0, off);
+            if (lane >= off) i0 += o;
+        }
+        const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
+        int i1 = c1;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, i1, off);
+            if (lane >= off) i1 += o;
+        }
+        cb[lane] = i0 - c0;
+        cb[lane + 32] = tot0 + i1 - c1;
+        if (lane == 31) {
+            cb[64] = tot0 + i1;
+            misc[1] = tot0 + i1;
+        }
+    }
+    __syncthreads();
+    const int nchain = misc[1];
+
+    // ---- b. exact chains of the candidates.  A chunk is nbx 64-column tiles of
+    // h; each tile holds the block's x rows and every router row (router_w^T, all
+    // E experts), loaded by the TMA engine with the 128-byte swizzle so that eight
+    // lanes reading the same 16-byte column of eight rows hit eight bank groups when
+    // the rows differ mod 8.  Chunk g (a running count over rounds) lives in stage
+    // g % stages and completes on full[g % stages]; one CTA barrier per chunk frees
+    // its stage for the refill.
+    const int S = a.stages, hc = a.nbx * 64, nch = (H + hc - 1) / hc;
+    const int tile_rows = a.xrows + a.erows;
+    auto issue = [&](int ch, uint32_t g) {  // thread 0
+        uint8_t *st = stage0 + (size_t)(g % S) * a.stage_bytes;
+        const int nb = min(a.nbx, (H - ch * hc) / 64);
+        mbar_arrive_expect_tx(&full[g % S], (uint32_t)(nb * tile_rows * 128));
+        for (int b = 0; b < nb; ++b) {
+            const int h = ch * hc + b * 64;
+            uint8_t *tile = st + (size_t)b * tile_rows * 128;
+            tma_load_2d(tile, &tm_x, &full[g % S], h, t0);
+            for (int r = 0; r < a.erows; r += a.ebox)
+                tma_load_2d(tile + (size_t)(a.xrows + r) * 128, &tm_w, &full[g % S], h, r);
+        }
+    };
+    uint32_t g0 = 0;
+    bool failed = false;
+    for (int r0 = 0; r0 < nchain; r0 += kCertThreads * kCertChains) {
+        int ctl[kCertChains], cpos[kCertChains];
+        RouterCand cc[kCertChains];
+        float acc[kCertChains];
+        bool on[kCertChains];
+#pragma unroll
+        for (int i = 0; i < kCertChains; ++i) {
+            const int c = r0 + i * kCertThreads + tid;
+            ctl[i] = 0;
+            cpos[i] = 0;
+            acc[i] = 0.0f;
+            on[i] = c < nchain;
+            cc[i] = RouterCand{0, 0, 0.0f, 0.0f};
+            if (on[i]) {
+                int lo = 0, hi = tb;  // largest tl with cb[tl] <= c
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) / 2;
+                    if (cb[mid] <= c) lo = mid;
+                    else hi = mid;
+                }
+                ctl[i] = lo;
+                cpos[i] = c - cb[lo];
+                cc[i] = a.list[(size_t)(t0 + lo) * E + cpos[i]];
+            }
+        }
+        if (tid == 0)
+            for (int ch = 0; ch < min(S, nch); ++ch) issue(ch, g0 + ch);
+        for (int ch = 0; ch < nch; ++ch) {
+            const uint32_t g = g0 + ch;
+            if (!mbar_wait(&full[g % S], (g / S) & 1u, failed ? 1000000ull : kWaitLimitNs)) {
+                failed = true;
+                atomicCAS(a.status, 0, MOE_ERR_TIMEOUT);
+            }
+            const uint8_t *st = stage0 + (size_t)(g % S) * a.stage_bytes;
+            const int nb = min(a.nbx, (H - ch * hc) / 64);
+            for (int b = 0; b < nb; ++b) {
+                const uint8_t *tile = st + (size_t)b * tile_rows * 128;
+                if (on[0] && on[1]) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        acc[0] = chain_step8(*sw128_chunk(tile, ctl[0], j), *sw128_chunk(tile, a.xrows + cc[0].e, j),
+                                             acc[0]);
+                        acc[1] = chain_step8(*sw128_chunk(tile, ctl[1], j), *sw128_chunk(tile, a.xrows + cc[1].e, j),
+                                             acc[1]);
+                    }
+                } else if (on[0]) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        acc[0] = chain_step8(*sw128_chunk(tile, ctl[0], j), *sw128_chunk(tile, a.xrows + cc[0].e, j),
+                                             acc[0]);
+                }
+            }
+            __syncthreads();  // stage g % S consumed by every thread
+            if (tid == 0 && ch + S < nch) issue(ch + S, g + S);
+        }
+        g0 += nch;
+#pragma unroll
+        for (int i = 0; i < kCertChains; ++i)
+            if (on[i]) {
+                float v = acc[i];
+                if (a.bias) v = __fadd_rn(v, a.bias[cc[i].e]);
+                a.list[(size_t)(t0 + ctl[i]) * E + cpos[i]].v = v;
+                if (!(fabsf(v - cc[i].v) <= cc[i].d)) atomicCAS(a.status, 0, MOE_ERR_ROUTER_BOUND);
+            }
+    }
+    __syncthreads();
+
+    // ---- c. top-k (larger exact value first, lower index on ties) and softmax
+    for (int tl = warp; tl < tb; tl += kCertWarps) {
+        const int t = t0 + tl;
+        const int n = nc[tl];
+        const RouterCand *cl = a.list + (size_t)t * E;
+        uint32_t key[MAXV];
+        float val[MAXV];
+        int ce[MAXV];
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i) {
+            const int p = lane + 32 * i;  // candidates are in ascending expert order
+            RouterCand c{0, 0, 0.0f, 0.0f};
+            if (p < n) c = cl[p];
+            ce[i] = c.e;
+            val[i] = c.v;
+            key[i] = p < n ? order_key(c.v) : 0u;
+        }
+        int *se = wse + warp * k;
+        float *sv = wsv + warp * k;
+        warp_topk<MAXV>(key, val, k, se, sv);
+        // slot -> expert: the slot order is the expert order, so the tie rule holds
+        for (int j = 0; j < k; ++j) {
+            const int p = se[j];
+            int mine = 0;
+#pragma unroll
+            for (int i = 0; i < MAXV; ++i)
+                if (i == (p >> 5)) mine = ce[i];
+            const int e = __shfl_sync(0xffffffffu, mine, p & 31);
+            if (lane == 0) {
+                a.idx[(size_t)t * k + j] = e;
+                a.ex[(size_t)t * E + e] = sv[j];
+            }
+        }
+        const float m = sv[0];
+        float s = 0.0f;
+        for (int j = lane; j < k; j += 32) s += expf(sv[j] - m);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        for (int j = lane; j < k; j += 32) a.gate[(size_t)t * k + j] = expf(sv[j] - m) / s;
+        __syncwarp();
+    }
+}
+
+template <int MAXV>
+cudaError_t launch_certify(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const CertifyArgs &a, int grid,
+                           cudaStream_t st)
+{
+    auto kern = router_certify_kernel<MAXV>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kCertSmem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kCertThreads, kCertSmem, st>>>(tm_x, tm_w, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route_certified(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
+                                   const float *bias, float *logits, int32_t *idx, float *gate,
+                                   const RouterScratch &rs, WsHeader *hdr, cudaStream_t st)
+{
+    const int T = d.T, H = d.H, E = d.E, k = d.top_k;
+    const int nparts = (H + kPrepH - 1) / kPrepH;
+    router_prep_kernel<<<dim3((E + kPrepE - 1) / kPrepE, nparts), 256, 0, st>>>(wr, H, E, rs.wrt, rs.wsq);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    int ks = 1;
+    if ((e = tc_router_logits(x, rs.wrt, T, H, E, logits, hdr, &ks, st)) != cudaSuccess) return e;
+    const float u = 5.9604644775390625e-08f;  // 2^-24
+    const float eps = ((float)H * u + 256.0f * u + (float)(H / 64 + ks) * u) * 1.01f;
+    int tb = (T + num_sms() - 1) / num_sms();
+    tb = tb < 1 ? 1 : tb > kCertMaxTB ? kCertMaxTB : tb;
+    const int xrows = (tb + 7) / 8 * 8;
+    const int erows = E <= 256 ? (E + 7) / 8 * 8 : (E + 255) / 256 * 256;
+    const int ebox = erows < 256 ? erows : 256;
+    const size_t room = (size_t)kCertSmem - 1024 - cert_fixed_bytes(E, k);
+    int nbx = 4, stages = 0;
+    for (; nbx >= 1; nbx /= 2) {  // the widest chunk that still leaves two stages
+        stages = (int)(room / ((size_t)nbx * (xrows + erows) * 128));
+        if (stages >= 2 || nbx == 1) break;
+    }
+    if (stages > kCertMaxStages) stages = kCertMaxStages;
+    if (stages < 1) return cudaErrorInvalidValue;
+    CUtensorMap tm_x, tm_w;
+    if (!encode_sw128_2d_bf16(&tm_x, x, T, H, xrows) || !encode_sw128_2d_bf16(&tm_w, rs.wrt, E, H, ebox))
+        return cudaErrorInvalidValue;
+    CertifyArgs a{logits, logits, ks, x, rs.wsq, bias, nparts, T, H, E, k, tb, eps, rs.ncand, rs.list,
+                  idx, gate, &hdr->status, xrows, erows, ebox, nbx, stages, nbx * (xrows + erows) * 128};
+    const int grid = (T + tb - 1) / tb;
+    const int vpl = (E + 31) / 32;
+    if (vpl <= 1) return launch_certify<1>(tm_x, tm_w, a, grid, st);
+    if (vpl <= 2) return launch_certify<2>(tm_x, tm_w, a, grid, st);
+    if (vpl <= 4) return launch_certify<4>(tm_x, tm_w, a, grid, st);
+    if (vpl <= 8) return launch_certify<8>(tm_x, tm_w, a, grid, st);
+    if (vpl <= 16) return launch_certify<16>(tm_x, tm_w, a, grid, st);
+    return launch_certify<32>(tm_x, tm_w, a, grid, st);
+}
+
+}  // namespace moe

@@ -142,22 +142,41 @@ def test_repeat_calls_same_workspace():
     assert api.moe_get_device_status(ws) == api.MOE_OK
 
 
-@pytest.mark.parametrize("name", ["decode", "one_token", "small32"])
+ROUTING_CASES = {
+    "decode": CONFIGS["decode"],
+    "one_token": SMALL["one_token"],
+    "small32": CONFIGS["decode"].replace(name="small32", T=29, E=64, top_k=6, seed=31),
+    "odd_e_small": CONFIGS["tiny"].replace(name="odd_e_small", T=20, H=192, E=12, top_k=3, seed=32),
+    "tiny": CONFIGS["tiny"],
+    "ragged_bias": SMALL["ragged_bias"],
+    "wide_e": SMALL["wide_e"],
+}
+
+
+@pytest.mark.parametrize("name", list(ROUTING_CASES))
 def test_forward_routing_matches_oracle(name):
     # The forward's own routing and permutation (read back from its workspace) must be
-    # bit-exact too -- for small batches they come from the fused router+permute kernel.
-    cfg = {"decode": CONFIGS["decode"], "one_token": SMALL["one_token"],
-           "small32": CONFIGS["decode"].replace(name="small32", T=29, E=64, top_k=6, seed=31)}[name]
+    # bit-exact too -- for small batches they come from the fused router+permute kernel --
+    # and so must the router's fp32 chain values: all of them for T <= 32, the chosen
+    # experts' ones for the certified tensor-core router above.
+    cfg = ROUTING_CASES[name]
     g, c = device_inputs(cfg)
     k = cfg.top_k
     ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, "cuda")
+    idx_ref, gate_ref, l32, _ = oracle.get().route(c["x"], c["router_w"], c["bias"], k, want_logits=True)
     for _ in range(2):  # the second call checks the self-reset of the router's ticket
         api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k, ws=ws)
         assert api.moe_get_device_status(ws) == api.MOE_OK
         r = api.forward_routing(ws, cfg.T, cfg.H, cfg.I, cfg.E, k)
-        idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], k)
         compare_routing(r["topk_idx"], r["topk_w"], idx_ref, gate_ref, name)
         compare_permute(r, oracle.permute(idx_ref, cfg.E), name)
+        lg = r["logits"].cpu().numpy()
+        if cfg.T <= 32:
+            bad = np.argwhere(lg.view(np.uint32) != l32.view(np.uint32))
+        else:
+            rows = np.arange(cfg.T)[:, None]
+            bad = np.argwhere(lg[rows, idx_ref].view(np.uint32) != l32[rows, idx_ref].view(np.uint32))
+        assert bad.size == 0, f"{name}: chain values differ at {bad[:5].tolist()}"
 
 
 def test_cuda_graph_replay():
