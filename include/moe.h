@@ -209,7 +209,7 @@ void moe_set_stage_events(void *const *events, int32_t n);
  * or that must never allocate on their serving path.
  *  - Dims whose moe_workspace_size exceeds the array are rejected with
  *    MOE_ERR_TOO_LARGE (with H=2048, I=512, E=256, top_k=8 that is above
- *    209 tokens); invalid dims give the same errors as moe_forward.
+ *    182 tokens); invalid dims give the same errors as moe_forward.
  *  - The first call made with a device current looks up the array's device
  *    address on that device; make that first call before any stream capture.
  *  - Nothing is allocated, freed or synchronised.  Every call shares the one
