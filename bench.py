@@ -37,7 +37,18 @@ if ROOT not in sys.path:
 from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_fp8_weights, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at 1 B200; % of BF16/FP8 TC peak or % of HBM BW"
-KERNELS_PER_FORWARD = 9   # logits, top-k, count, scan, scatter, gather, GEMM x2, combine
+def kernels_per_forward(cfg) -> int:
+    """Library kernels one forward launches."""
+    A = cfg.T * cfg.top_k
+    if cfg.T > 32:
+        route = 3 + 3      # transpose/norms, tensor-core logits, certify; count, scan, scatter
+    elif cfg.E % 8 == 0 and cfg.H % 128 == 0 and A <= 4096 and (A + 31) // 32 * cfg.E <= 16384:
+        route = 2          # logits, top-k + grouping
+    else:
+        route = 2 + 3      # logits, top-k; count, scan, scatter
+    combine = 0 if cfg.T <= 64 else 1   # small batches combine inside the down GEMM
+    rows = 2 if cfg.dtype == "fp8" else 1   # fp8: quantise per token, then gather; bf16: gather
+    return route + rows + 2 + combine   # + gate/up GEMM, down GEMM
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 512 << 20
 EVICT_FLOATS = 64 << 20   # 256 MiB read after the write, so the flush leaves no dirty lines
@@ -81,10 +92,10 @@ def load_peaks():
 
 
 STAGE_SOURCES = {
-    "route": ["route.cu"],
-    "gemm_gate_up": ["grouped_gemm.cu", "sm100_ptx.cuh", "moe_internal.h"],
-    "gemm_down": ["grouped_gemm.cu", "sm100_ptx.cuh", "moe_internal.h"],
-    "combine": ["combine.cu"],
+    "route": ["route.cu", "route_certified.cu", "route_common.cuh", "fp8.cu", "sm100_ptx.cuh", "moe_internal.h"],
+    "gemm_gate_up": ["grouped_gemm.cu", "fp8.cu", "sm100_ptx.cuh", "moe_internal.h"],
+    "gemm_down": ["grouped_gemm.cu", "fp8.cu", "combine.cuh", "sm100_ptx.cuh", "moe_internal.h"],
+    "combine": ["combine.cu", "combine.cuh"],
 }
 
 
@@ -358,7 +369,8 @@ def config_block(cfg, world):
             "seed": cfg.seed, "router_bias": "zipf(1.2)" if cfg.zipf_s else None,
             "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
             "l2": "flushed before every step: 512 MiB write then 256 MiB read, outside the step's events",
-            "launch": "timed steps: K moe_forward calls captured in one CUDA graph; e2e: direct calls"}
+            "launch": "timed steps: K moe_forward calls captured in one CUDA graph, an event pair per step; "
+                      "stage times from a second graph with events between the stages; e2e: direct calls"}
 
 
 # ---------------------------------------------------------------- our arm
@@ -405,9 +417,12 @@ def main():
     def step():
         forward(x, stream)
 
-    # events: one set of 6 stage marks per timed step (the first and last bracket the step)
+    # events: a start/end pair per timed step, and (in a second, untimed graph) the six
+    # stage marks of every step for the breakdown -- an event between two kernels costs
+    # the step a few microseconds, so the headline time carries only the outer pair
+    ev_step = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    for s in ev:
+    for s in ev + ev_step:
         for e in s:
             e.record(stream)
     for _ in range(max(args.warmup, 3)):
@@ -419,7 +434,7 @@ def main():
         raise RuntimeError(f"device status {status} after warm-up")
 
     # The timed region is one CUDA graph holding the K steps: before each step an L2
-    # flush (outside that step's events), then the step with its own six stage events.
+    # flush (outside that step's events), then the step between its two events.
     cap = torch.cuda.Stream(dev)
     cap.wait_stream(stream)
     graph = torch.cuda.CUDAGraph()
@@ -427,10 +442,20 @@ def main():
         with torch.cuda.graph(graph, stream=cap):
             for i in range(args.steps):
                 flush.fill_(1)
+                api.set_stage_events([ev_step[i][0], None, None, None, None, ev_step[i][1]])
+                forward(x, cap)
+    # the stage breakdown: the same steps with the library's six stage marks
+    graph_stages = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph_stages, stream=cap):
+            for i in range(args.steps):
+                flush.fill_(1)
                 api.set_stage_events(ev[i])
                 forward(x, cap)
     api.set_stage_events(None)
     stream.wait_stream(cap)
+    graph_stages.replay()
+    torch.cuda.synchronize()
     graph.replay()  # one untimed replay so the timed one starts warm
     torch.cuda.synchronize()
 
@@ -449,9 +474,9 @@ def main():
     status = api.moe_get_device_status(ws)
     if status != api.MOE_OK:
         raise RuntimeError(f"device status {status} after the timed steps")
-    del graph
+    del graph, graph_stages
 
-    step_ms = [ev[i][0].elapsed_time(ev[i][5]) for i in range(args.steps)]
+    step_ms = [ev_step[i][0].elapsed_time(ev_step[i][1]) for i in range(args.steps)]
     stage_ms = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
                 for j, name in enumerate(api.STAGES)}
     total_ms = max_over_ranks(sum(step_ms), world)
@@ -507,7 +532,7 @@ def main():
                 "dtype": "e4m3" if fp8 else "bf16",
                 "data": "synthetic", "config": config_block(cfg, world),
                 "roofline": roof, "stages": stages, "experts_touched": work["_D"],
-                "e2e": e2e, "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+                "e2e": e2e, "gpu_launches": kernels_per_forward(cfg) * args.steps,
                 "clocks": clocks, "cpu_baseline": cpu,
                 "p99_ms_per_step": round(sorted(step_ms)[min(len(step_ms) - 1, math.ceil(0.99 * len(step_ms)) - 1)], 5)}
         print(json.dumps(line), flush=True)

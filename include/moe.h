@@ -195,8 +195,10 @@ void moe_set_wait_limit_us(int32_t us, int32_t stall_test);
  * caller-created cudaEvent_t handles (passed as void*), every later moe_forward
  * records them on its stream at the stage boundaries: [0] start, [1] routed,
  * [2] permuted (groups, tile list, sorted activations), [3] gate/up GEMM done,
- * [4] down GEMM done, [5] combined.  The handles must stay valid while set;
- * NULL (or n != MOE_STAGE_EVENTS) turns recording off.  Process-wide. */
+ * [4] down GEMM done, [5] combined.  A NULL entry is skipped (an event between
+ * two kernels costs the step a few microseconds, so whole-step timing passes only
+ * [0] and [5]).  The handles must stay valid while set; events == NULL (or
+ * n != MOE_STAGE_EVENTS) turns recording off.  Process-wide. */
 #define MOE_STAGE_EVENTS 6
 void moe_set_stage_events(void *const *events, int32_t n);
 

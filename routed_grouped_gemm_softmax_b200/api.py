@@ -291,11 +291,12 @@ def set_claim_order(reverse: bool):
 
 def set_stage_events(events):
     """Record these 6 torch.cuda.Events at the stage boundaries of every later
-    moe_forward (None turns it off).  Each event must have been recorded once so
-    that its CUDA handle exists."""
+    moe_forward (None turns it off; a None entry is skipped).  Each event must have
+    been recorded once so that its CUDA handle exists."""
     if events is None:
         lib().moe_set_stage_events(None, 0)
         return
-    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event if e is not None else None)
+                                            for e in events])
     set_stage_events._keep = arr
     lib().moe_set_stage_events(arr, len(events))

@@ -29,7 +29,9 @@
 
 #include <mutex>
 
+#include "combine.cuh"
 #include "moe_internal.h"
+#include "pdl.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {
@@ -94,12 +96,32 @@ __device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64
 
 // ------------------------------------------------------------ quantiser
 
+// The fp8 activations of the forward: x is quantised once per token, then row r of
+// the expert-sorted copy takes token s2f[r] / k's codes and scales (a warp per row).
+__global__ void gather_rows_fp8_kernel(const uint8_t *__restrict__ xq, const float *__restrict__ xq_s,
+                                       const int32_t *__restrict__ s2f, int A, int K, int k, uint8_t *__restrict__ xs,
+                                       float *__restrict__ xs_s)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= A) return;
+    const int t = s2f[row] / k;
+    const uint4 *src = reinterpret_cast<const uint4 *>(xq + (size_t)t * K);
+    uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)row * K);
+    for (int c = lane; c < K / 16; c += 32) dst[c] = src[c];
+    for (int c = lane; c < K / 128; c += 32) xs_s[(size_t)row * (K / 128) + c] = xq_s[(size_t)t * (K / 128) + c];
+}
+
 // Rows of a bf16 matrix quantised per 128-column group.  Row r reads source row
 // map ? map[r] / k : r, so the same kernel gathers x into expert order.  One warp
 // per row; lane l holds elements 4l..4l+3 of the current group.
 __global__ void quantize_rows_kernel(const __nv_bfloat16 *__restrict__ src, const int32_t *__restrict__ map,
                                      int k, int R, int K, uint8_t *__restrict__ q, float *__restrict__ s)
 {
+    pdl_wait();
+    pdl_trigger();
     const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     if (row >= R) return;
@@ -125,7 +147,7 @@ __global__ void quantize_rows_kernel(const __nv_bfloat16 *__restrict__ src, cons
 
 // ----------------------------------------------------------- grouped GEMM
 
-template <int MODE, bool BF16>
+template <int MODE, bool BF16, bool COMB = false>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const Fp8GemmArgs g)
@@ -172,6 +194,8 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
+    pdl_wait();  // the prologue above overlapped the previous kernel
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------ scheduler + TMA producer
@@ -383,6 +407,9 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                         dst[i] = *reinterpret_cast<uint4 *>(v);
                     }
                 }
+                if (COMB)  // both halves of a row arrive (comb_target = 2k), empty ones too
+                    combine_arrive(g.out, g.comb_gate, g.comb_out, g.comb_cnt, g.comb_k, g.comb_target, g.N, n_tiles,
+                                   nt, row_ok, row_ok ? g.row_map[row0 + row] : 0, lane);
             }
         }
     }
@@ -395,20 +422,22 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     }
 }
 
-bool fp8_smem_attr_ready(int mode)
+bool fp8_smem_attr_ready(int v)  // v: 0 gate/up, 1 down, 2 router logits, 3 down with the fused combine
 {
     static std::mutex mu;
-    static uint64_t done[3] = {0, 0, 0};
+    static uint64_t done[4] = {0, 0, 0, 0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::lock_guard<std::mutex> lk(mu);
-    if (done[mode] >> dev & 1ull) return true;
+    if (done[v] >> dev & 1ull) return true;
     const int a = (int)SMEM8;
-    cudaError_t e = mode == 0 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
-                  : mode == 1 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
-                              : cudaFuncSetAttribute(grouped_gemm_fp8_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, a);
+    cudaError_t e = v == 0   ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                  : v == 1 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                  : v == 2 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                           : cudaFuncSetAttribute(grouped_gemm_fp8_kernel<1, false, true>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, a);
     if (e != cudaSuccess) return false;
-    done[mode] |= 1ull << dev;
+    done[v] |= 1ull << dev;
     return true;
 }
 
@@ -418,23 +447,35 @@ cudaError_t launch_quantize_rows(const __nv_bfloat16 *src, const int32_t *map, i
                                  float *s, cudaStream_t st)
 {
     const int rows_per_block = 8;
-    quantize_rows_kernel<<<(R + rows_per_block - 1) / rows_per_block, rows_per_block * 32, 0, st>>>(src, map, k, R,
-                                                                                                   K, q, s);
-    return cudaGetLastError();
+    return launch_pdl(quantize_rows_kernel, dim3((R + rows_per_block - 1) / rows_per_block), dim3(rows_per_block * 32),
+                      0, st, src, map, k, R, K, q, s);
+}
+
+cudaError_t launch_gather_rows_fp8(const uint8_t *xq, const float *xq_s, const int32_t *s2f, int A, int K, int k,
+                                   uint8_t *xs, float *xs_s, cudaStream_t st)
+{
+    const int rows_per_block = 8;
+    return launch_pdl(gather_rows_fp8_kernel, dim3((A + rows_per_block - 1) / rows_per_block),
+                      dim3(rows_per_block * 32), 0, st, xq, xq_s, s2f, A, K, k, xs, xs_s);
 }
 
 cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
                                     const CUtensorMap &tmB1, cudaStream_t st)
 {
     const int grid = g.ctas > 0 ? g.ctas : num_sms();
-    if (!fp8_smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
+    const bool comb = g.mode == 1 && g.comb_cnt != nullptr;
+    if (!fp8_smem_attr_ready(comb ? 3 : g.mode)) return cudaErrorInvalidValue;
+    cudaError_t e;
     if (g.mode == 0)
-        grouped_gemm_fp8_kernel<0, false><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
+        e = launch_pdl(grouped_gemm_fp8_kernel<0, false>, dim3(grid), dim3(THREADS), SMEM8, st, tmA, tmB0, tmB1, g);
+    else if (comb)  // the combine's code is compiled in only here: it costs the epilogue registers
+        e = launch_pdl(grouped_gemm_fp8_kernel<1, false, true>, dim3(grid), dim3(THREADS), SMEM8, st, tmA, tmB0, tmB1,
+                       g);
     else if (g.mode == 1)
-        grouped_gemm_fp8_kernel<1, false><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
+        e = launch_pdl(grouped_gemm_fp8_kernel<1, false>, dim3(grid), dim3(THREADS), SMEM8, st, tmA, tmB0, tmB1, g);
     else
-        grouped_gemm_fp8_kernel<2, true><<<grid, THREADS, SMEM8, st>>>(tmA, tmB0, tmB1, g);
-    return cudaGetLastError();
+        e = launch_pdl(grouped_gemm_fp8_kernel<2, true>, dim3(grid), dim3(THREADS), SMEM8, st, tmA, tmB0, tmB1, g);
+    return e;
 }
 
 }  // namespace moe

@@ -27,6 +27,7 @@
 //                   its 32-lane quarter), then
 //                   mode 0 (gate/up): h = silu(gate) * up, rounded to bf16,
 //                   mode 1 (down)   : y row of the assignment, rounded to bf16,
+//                                     then the fused combine (combine.cuh),
 //                   mode 2 (dense)  : fp32 rows (the router's tensor-core logits),
 //                   rows past the group's end masked.
 // Every accumulation order is fixed by the tile and the K loop, never by which
@@ -37,7 +38,9 @@
 // freeing TMEM.
 #include <mutex>
 
+#include "combine.cuh"
 #include "moe_internal.h"
+#include "pdl.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {
@@ -121,6 +124,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
+    pdl_wait();  // the prologue above overlapped the previous kernel
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------ scheduler + TMA producer
@@ -292,6 +297,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(&S->acce[acc]);
             if (++acc == 2) { acc = 0; aphase ^= 1; }
+            if (MODE == 1 && g.comb_cnt)  // the accumulator is already released
+                combine_arrive(g.out, g.comb_gate, g.comb_out, g.comb_cnt, g.comb_k, g.comb_target, g.N, n_tiles,
+                               nt, row_ok, row_ok ? g.row_map[row0 + row] : 0, lane);
         }
     }
 
@@ -339,13 +347,14 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const
 {
     const int grid = g.ctas > 0 ? g.ctas : num_sms();
     if (!smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
+    cudaError_t e;
     if (g.mode == 0)
-        grouped_gemm_kernel<0><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
+        e = launch_pdl(grouped_gemm_kernel<0>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g);
     else if (g.mode == 1)
-        grouped_gemm_kernel<1><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
+        e = launch_pdl(grouped_gemm_kernel<1>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g);
     else
-        grouped_gemm_kernel<2><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB0, tmB1, g);
-    return cudaGetLastError();
+        e = launch_pdl(grouped_gemm_kernel<2>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g);
+    return e;
 }
 
 }  // namespace moe

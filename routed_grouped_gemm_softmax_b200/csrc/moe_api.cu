@@ -39,7 +39,7 @@ struct StageMarks {
     // into a CUDA graph, so a replayed graph still timestamps every stage.
     cudaError_t mark(int i, cudaStream_t st) const
     {
-        return on ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal) : cudaSuccess;
+        return on && ev[i] ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal) : cudaSuccess;
     }
 };
 
@@ -338,8 +338,9 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
         return MOE_ERR_CUDA;
 
     const StageMarks marks;
+    const bool fused = d->T <= moe::kFusedCombineMaxT;  // combine inside the down GEMM
     cudaError_t e = marks.mark(0, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(moe::WsHeader), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);  // header + combine counts
     if (e == cudaSuccess) e = route_and_permute(*d, L, x, router_w, router_bias, ws, hdr, marks, st);
     if (e == cudaSuccess)
         e = moe::launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), s2f, A, d->H, d->top_k, xs, st);
@@ -354,11 +355,13 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
     }
     if (e == cudaSuccess) e = marks.mark(3, st);
     if (e == cudaSuccess) {
-        moe::GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, y, s2f, ctas, rev, wait_ns, stall};
+        moe::GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, y, s2f, ctas, rev, wait_ns,
+                         stall, 0, nullptr, gate, fused ? at<int32_t>(ws, L.ccnt) : nullptr,
+                         static_cast<__nv_bfloat16 *>(out), d->top_k, d->top_k};
         e = moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st);
     }
     if (e == cudaSuccess) e = marks.mark(4, st);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && !fused)
         e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st);
     if (e == cudaSuccess) e = marks.mark(5, st);
     return cuda_status(e);
@@ -411,11 +414,17 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
         return MOE_ERR_CUDA;
 
     const StageMarks marks;
+    const bool fused = d->T <= moe::kFusedCombineMaxT;  // combine inside the down GEMM
     cudaError_t e = marks.mark(0, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(moe::WsHeader), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);  // header + combine counts
     if (e == cudaSuccess) e = route_and_permute(*d, L, x, router_w, router_bias, ws, hdr, marks, st);
+    // x quantised once per token, then its codes gathered into expert order
     if (e == cudaSuccess)
-        e = moe::launch_quantize_rows(static_cast<const __nv_bfloat16 *>(x), s2f, d->top_k, A, d->H, xs, xs_s, st);
+        e = moe::launch_quantize_rows(static_cast<const __nv_bfloat16 *>(x), nullptr, 1, d->T, d->H,
+                                      at<uint8_t>(ws, L.xq), at<float>(ws, L.xq_s), st);
+    if (e == cudaSuccess)
+        e = moe::launch_gather_rows_fp8(at<uint8_t>(ws, L.xq), at<float>(ws, L.xq_s), s2f, A, d->H, d->top_k, xs,
+                                        xs_s, st);
     if (e == cudaSuccess) e = marks.mark(2, st);
     const int ctas = g_gemm_ctas.load(), rev = g_claim_reverse.load();
     const unsigned long long wl = g_wait_ns.load();
@@ -429,11 +438,13 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
     if (e == cudaSuccess) e = marks.mark(3, st);
     if (e == cudaSuccess) {
         moe::Fp8GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, h_s, w_down_s, w_down_s,
-                            nullptr, nullptr, y, s2f, ctas, rev, wait_ns, stall};
+                            nullptr, nullptr, y, s2f, ctas, rev, wait_ns, stall, 0, 1, nullptr, gate,
+                            fused ? at<int32_t>(ws, L.ccnt) : nullptr, static_cast<__nv_bfloat16 *>(out), d->top_k,
+                            2 * d->top_k};
         e = moe::launch_grouped_gemm_fp8(g2, tm_h, tm_wd, tm_wd, st);
     }
     if (e == cudaSuccess) e = marks.mark(4, st);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && !fused)
         e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st);
     if (e == cudaSuccess) e = marks.mark(5, st);
     return cuda_status(e);

@@ -24,7 +24,7 @@ struct WsHeader {
 
 // Byte offsets of every region of the workspace (256-byte aligned each).
 struct WsLayout {
-    size_t logits, wrt, wsq, rncand, rlist, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xs, xs_s, h, h_s, y,
+    size_t ccnt, clear_bytes, logits, wrt, wsq, rncand, rlist, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xq, xq_s, xs, xs_s, h, h_s, y,
         total;
     int nb;      // permutation chunks
     int chunk;   // flat entries per chunk
@@ -44,7 +44,7 @@ inline int perm_warps(int E)
 }
 
 // Workspace regions; with fp8 the sorted activations and h are e4m3 codes plus
-// one fp32 scale per 128 columns.
+// one fp32 scale per 128 columns, and x is quantised per token before the gather.
 inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
 {
     const bool fp8 = dtype == MOE_DTYPE_FP8;
@@ -55,6 +55,10 @@ inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
     L.nb = static_cast<int>((A + L.chunk - 1) / L.chunk);
     const size_t max_tiles = (A + kTileRows - 1) / kTileRows + (A < (size_t)d.E ? A : (size_t)d.E);
     size_t o = align_up(sizeof(WsHeader), 256);
+    // the fused combine's arrival counts follow the header, so one memset clears both
+    L.ccnt = o;
+    o = align_up(o + static_cast<size_t>(d.T) * ((d.H + 255) / 256) * 4, 1024);
+    L.clear_bytes = L.ccnt + static_cast<size_t>(d.T) * ((d.H + 255) / 256) * 4;
     auto take = [&](size_t bytes) {
         size_t at = o;
         o = align_up(o + bytes, 1024);
@@ -75,6 +79,8 @@ inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
     L.f2s = take(A * 4);
     L.tiles = take(max_tiles * 3 * 4);
     L.ntiles = take(4);
+    L.xq = take(fp8 ? static_cast<size_t>(d.T) * d.H : 0);  // fp8: x quantised once per token
+    L.xq_s = take(fp8 ? static_cast<size_t>(d.T) * (d.H / 128) * 4 : 0);
     L.xs = take(A * d.H * (fp8 ? 1 : 2));
     L.xs_s = take(fp8 ? A * (d.H / 128) * 4 : 0);
     L.h = take(A * d.I * (fp8 ? 1 : 2));
@@ -127,8 +133,6 @@ cudaError_t launch_permute(const moe_dims_t &d, const WsLayout &L, const int32_t
 cudaError_t launch_gather_rows(const __nv_bfloat16 *x, const int32_t *s2f, int A, int H, int top_k,
                                __nv_bfloat16 *xs, cudaStream_t st);
 
-cudaError_t launch_combine(const __nv_bfloat16 *y, const float *gate, int T, int H, int top_k,
-                           __nv_bfloat16 *out, cudaStream_t st);
 
 // Grouped GEMMs over the tile list.  mode 0: h = silu(A Wg^T) * (A Wu^T) (A = the
 // expert-sorted activations, B = gate/up weights); mode 1: y[s2f[row]] = A Wd^T
@@ -148,6 +152,14 @@ struct GemmArgs {
     int stall_test;    // MMA thread first waits on a barrier nothing signals
     int M;             // mode 2 (no tile list): rows of A
     float *out_f32;    // mode 2: fp32 output [M, N]
+    // mode 1, fused combine (comb_cnt non-null): after its y rows of an n-tile are
+    // written, the last of the comb_target arrivals for (token, n-tile) sums the
+    // token's k rows of that n-tile into comb_out.
+    const float *comb_gate;
+    int32_t *comb_cnt;            // [T, ceil(N / 256)], zero before the launch
+    __nv_bfloat16 *comb_out;      // [T, N]
+    int comb_k;
+    int comb_target;
 };
 // mode 2: out_f32 = A B^T over M rows (one "expert"), the router's tensor-core logits.
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
@@ -177,17 +189,31 @@ struct Fp8GemmArgs {
     int M;            // mode 2: rows of A (no tile list)
     int ksplit;       // mode 2: items per (m-tile, n-tile), each a slice of K
     float *out_f32;   // mode 2: partial logits [ksplit, M, N]
+    const float *comb_gate;  // mode 1 fused combine, as in GemmArgs
+    int32_t *comb_cnt;
+    __nv_bfloat16 *comb_out;
+    int comb_k;
+    int comb_target;
 };
 cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
                                     const CUtensorMap &tmB1, cudaStream_t st);
 cudaError_t launch_quantize_rows(const __nv_bfloat16 *src, const int32_t *map, int k, int R, int K, uint8_t *q,
                                  float *s, cudaStream_t st);
+// fp8 rows into expert order: xs[r] = xq[s2f[r] / k] (K codes) and xs_s[r] = xq_s[...] (K/128 scales).
+cudaError_t launch_gather_rows_fp8(const uint8_t *xq, const float *xq_s, const int32_t *s2f, int A, int K, int k,
+                                   uint8_t *xs, float *xs_s, cudaStream_t st);
 
 // Tensor-core router logits: partial sums over ksplit slices of H,
 // logits [ksplit, T, E] with sum_s logits[s] = x [T,H] . wrt [E,H]^T (fp32 per
 // 64-wide K block, then fp32 sums).  Returns ksplit through *ksplit_out.
 cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, int T, int H, int E, float *logits,
                              WsHeader *hdr, int *ksplit_out, cudaStream_t st);
+
+// Gate-weighted combine of the k per-assignment rows of every token (combine.cu).
+cudaError_t launch_combine(const __nv_bfloat16 *y, const float *gate, int T, int H, int top_k,
+                           __nv_bfloat16 *out, cudaStream_t st);
+// Batches up to this many tokens combine inside the down GEMM's epilogue.
+constexpr int kFusedCombineMaxT = 64;
 
 int num_sms();
 

@@ -16,6 +16,7 @@
 //   scatter each entry's rank among equal experts earlier in its chunk (warp
 //           match + per-warp counts) -> sorted_to_flat / flat_to_sorted
 #include "moe_internal.h"
+#include "pdl.cuh"
 
 namespace moe {
 namespace {
@@ -28,6 +29,8 @@ __device__ __forceinline__ void record_status(int32_t *status, int code)
 __global__ void perm_count_kernel(const int32_t *__restrict__ idx, int A, int E, int chunk,
                                   int32_t *__restrict__ blk_cnt, int32_t *status)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ int hist[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
@@ -79,6 +82,8 @@ perm_scan_kernel(int E, int nb, const int32_t *__restrict__ blk_cnt, int32_t *__
                  int32_t *__restrict__ offsets, int32_t *__restrict__ tiles,
                  int32_t *__restrict__ ntiles, int32_t *counters, int ncounters)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int warp_tot[33];
     const int e = threadIdx.x;
     int cnt = 0;
@@ -114,6 +119,8 @@ __global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int A, int 
                                     const int32_t *__restrict__ blk_base, int32_t *__restrict__ s2f,
                                     int32_t *__restrict__ f2s)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ int wcnt[];  // [warps][E]: entries of each expert in each warp
     const int nw = blockDim.x / 32;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -139,6 +146,8 @@ __global__ void gather_rows_kernel(const __nv_bfloat16 *__restrict__ x,
                                    const int32_t *__restrict__ s2f, int A, int H, int k,
                                    __nv_bfloat16 *__restrict__ xs)
 {
+    pdl_wait();
+    pdl_trigger();
     const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     if (row >= A) return;
@@ -156,22 +165,23 @@ cudaError_t launch_permute(const moe_dims_t &d, const WsLayout &L, const int32_t
                            cudaStream_t st)
 {
     const int A = d.T * d.top_k, E = d.E;
-    perm_count_kernel<<<L.nb, 256, E * sizeof(int), st>>>(idx, A, E, L.chunk, blk_cnt,
-                                                          hdr ? &hdr->status : nullptr);
-    perm_scan_kernel<<<1, 1024, 0, st>>>(E, L.nb, blk_cnt, blk_base, offsets, tiles, ntiles,
-                                         hdr ? hdr->counter : nullptr, hdr ? 7 : 0);
-    perm_scatter_kernel<<<L.nb, L.chunk, (size_t)(L.chunk / 32) * E * sizeof(int), st>>>(
-        idx, A, E, blk_base, s2f, f2s);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(perm_count_kernel, dim3(L.nb), dim3(256), E * sizeof(int), st, idx, A, E, L.chunk,
+                               blk_cnt, hdr ? &hdr->status : nullptr);
+    if (e == cudaSuccess)
+        e = launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, st, E, L.nb, blk_cnt, blk_base, offsets, tiles,
+                       ntiles, hdr ? hdr->counter : nullptr, hdr ? 7 : 0);
+    if (e == cudaSuccess)
+        e = launch_pdl(perm_scatter_kernel, dim3(L.nb), dim3(L.chunk), (size_t)(L.chunk / 32) * E * sizeof(int), st,
+                       idx, A, E, blk_base, s2f, f2s);
+    return e;
 }
 
 cudaError_t launch_gather_rows(const __nv_bfloat16 *x, const int32_t *s2f, int A, int H, int top_k,
                                __nv_bfloat16 *xs, cudaStream_t st)
 {
     const int rows_per_block = 8;
-    gather_rows_kernel<<<(A + rows_per_block - 1) / rows_per_block, rows_per_block * 32, 0, st>>>(
-        x, s2f, A, H, top_k, xs);
-    return cudaGetLastError();
+    return launch_pdl(gather_rows_kernel, dim3((A + rows_per_block - 1) / rows_per_block), dim3(rows_per_block * 32),
+                      0, st, x, s2f, A, H, top_k, xs);
 }
 
 }  // namespace moe

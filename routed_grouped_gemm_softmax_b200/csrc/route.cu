@@ -20,6 +20,7 @@
 #include <climits>
 
 #include "moe_internal.h"
+#include "pdl.cuh"
 #include "route_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -58,6 +59,8 @@ __global__ void __launch_bounds__(LogitsTile<TT, TE, RT, RE, HC>::NT)
 route_logits_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ wr,
                     const float *__restrict__ bias, int T, int H, int E, float *__restrict__ logits)
 {
+    pdl_wait();
+    pdl_trigger();
     using L = LogitsTile<TT, TE, RT, RE, HC>;
     extern __shared__ __align__(16) float lsm[];
     // two buffers of x chunks, [h][token], then two of router_w chunks, [h][expert]
@@ -200,8 +203,7 @@ cudaError_t launch_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wr, const
         if (e != cudaSuccess) return e;
     }
     dim3 grid((T + TT - 1) / TT, (E + TE - 1) / TE);
-    kern<<<grid, L::NT, smem, st>>>(x, wr, bias, T, H, E, logits);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(L::NT), smem, st, x, wr, bias, T, H, E, logits);
 }
 
 // Small batches (T <= 32): one chain per thread, TP tokens x TE experts per CTA.
@@ -227,6 +229,8 @@ __global__ void __launch_bounds__(TP * TE)
 route_logits_small_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ wr,
                           const float *__restrict__ bias, int T, int H, int E, float *__restrict__ logits)
 {
+    pdl_wait();
+    pdl_trigger();
     using L = SmallTile<TP, TE, HC, S>;
     extern __shared__ __align__(16) uint8_t ssm[];
     const int tid = threadIdx.x;
@@ -291,8 +295,7 @@ cudaError_t launch_logits_small(const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
         if (e != cudaSuccess) return e;
     }
-    kern<<<(E + TE - 1) / TE, L::NT, L::SMEM, st>>>(x, wr, bias, T, H, E, logits);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((E + TE - 1) / TE), dim3(L::NT), L::SMEM, st, x, wr, bias, T, H, E, logits);
 }
 
 // Small batches, whole rows resident: the same chains as route_logits_small_kernel
@@ -331,6 +334,8 @@ __global__ void __launch_bounds__(TP * 8) route_logits_tma_kernel(const __grid_c
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_wait();
+    pdl_trigger();
     if (tid < 32) {
         if (tid == 0) {
             mbar_arrive_expect_tx(&bars[0], (uint32_t)(rows * H * 2));
@@ -394,8 +399,7 @@ bool try_launch_logits_tma(const __nv_bfloat16 *x, const __nv_bfloat16 *wr, cons
     auto kern = route_logits_tma_kernel<TP>;
     *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (*err != cudaSuccess) return true;
-    kern<<<E / 8, TP * 8, smem, st>>>(tm, x, bias, T, H, E, logits, status);
-    *err = cudaGetLastError();
+    *err = launch_pdl(kern, dim3(E / 8), dim3(TP * 8), smem, st, tm, x, bias, T, H, E, logits, status);
     return true;
 }
 
@@ -443,6 +447,8 @@ template <int MAXV>
 __global__ void route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
                                   int32_t *__restrict__ idx, float *__restrict__ gate)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(16) uint8_t tksm[];  // [warps][k] experts, then [warps][k] values
     const int warp = threadIdx.x / 32, nw = blockDim.x / 32, lane = threadIdx.x % 32;
     const int t = blockIdx.x * nw + warp;
@@ -468,8 +474,8 @@ cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *idx, 
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    route_topk_kernel<MAXV><<<(T + warps - 1) / warps, warps * 32, smem, st>>>(logits, T, E, k, idx, gate);
-    return cudaGetLastError();
+    return launch_pdl(route_topk_kernel<MAXV>, dim3((T + warps - 1) / warps), dim3(warps * 32), smem, st, logits, T,
+                      E, k, idx, gate);
 }
 
 // ------------------------------------------------------------------------
@@ -508,6 +514,8 @@ __host__ __device__ inline size_t small_topk_permute_smem(int T, int E, int k, i
 template <int MAXV>
 __global__ void __launch_bounds__(1024) topk_permute_small_kernel(int T, int E, int k, SmallRouteOut o)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(16) uint8_t tsm[];
     const int tid = threadIdx.x, NT = blockDim.x, lane = tid % 32, warp = tid / 32, nw = NT / 32;
     const int A = T * k, nch = (A + 31) / 32;
@@ -632,8 +640,7 @@ cudaError_t launch_route_permute_small(const moe_dims_t &d, const __nv_bfloat16 
             cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (r != cudaSuccess) return r;
         }
-        kern<<<1, warps * 32, smem, st>>>(d.T, d.E, d.top_k, o);
-        return cudaGetLastError();
+        return launch_pdl(kern, dim3(1), dim3(warps * 32), smem, st, d.T, d.E, d.top_k, o);
     };
     if (vpl <= 1) return launch(topk_permute_small_kernel<1>);
     if (vpl <= 2) return launch(topk_permute_small_kernel<2>);

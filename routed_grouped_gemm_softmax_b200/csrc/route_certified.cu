@@ -29,6 +29,7 @@
 #include <climits>
 
 #include "moe_internal.h"
+#include "pdl.cuh"
 #include "route_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -45,6 +46,8 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const __nv_bfloat16 *_
                                                           __nv_bfloat16 *__restrict__ wrt,
                                                           float *__restrict__ wsq_part)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ uint16_t tile[kPrepH][kPrepE + 2];
     const int tid = threadIdx.x;
     const int e0 = blockIdx.x * kPrepE, h0 = blockIdx.y * kPrepH;
@@ -150,6 +153,8 @@ __global__ void __launch_bounds__(kCertThreads)
         for (int s = 0; s < kCertMaxStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
+    pdl_wait();
+    pdl_trigger();
     for (int e = tid; e < E; e += kCertThreads) {
         float q = 0.0f;
         for (int j = 0; j < a.nparts; ++j) q += a.wsq_part[(size_t)j * E + e];
@@ -397,8 +402,7 @@ cudaError_t launch_certify(const CUtensorMap &tm_x, const CUtensorMap &tm_w, con
     auto kern = router_certify_kernel<MAXV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kCertSmem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kCertThreads, kCertSmem, st>>>(tm_x, tm_w, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(kCertThreads), kCertSmem, st, tm_x, tm_w, a);
 }
 
 }  // namespace
@@ -409,8 +413,8 @@ cudaError_t launch_route_certified(const moe_dims_t &d, const __nv_bfloat16 *x, 
 {
     const int T = d.T, H = d.H, E = d.E, k = d.top_k;
     const int nparts = (H + kPrepH - 1) / kPrepH;
-    router_prep_kernel<<<dim3((E + kPrepE - 1) / kPrepE, nparts), 256, 0, st>>>(wr, H, E, rs.wrt, rs.wsq);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(router_prep_kernel, dim3((E + kPrepE - 1) / kPrepE, nparts), dim3(256), 0, st, wr, H,
+                               E, rs.wrt, rs.wsq);
     if (e != cudaSuccess) return e;
     int ks = 1;
     if ((e = tc_router_logits(x, rs.wrt, T, H, E, logits, hdr, &ks, st)) != cudaSuccess) return e;
