@@ -115,34 +115,56 @@ __global__ void gather_rows_fp8_kernel(const uint8_t *__restrict__ xq, const flo
 }
 
 // Rows of a bf16 matrix quantised per 128-column group.  Row r reads source row
-// map ? map[r] / k : r, so the same kernel gathers x into expert order.  One warp
-// per row; lane l holds elements 4l..4l+3 of the current group.
+// map ? map[r] / k : r.  A warp takes eight groups (1024 columns) of one row: four
+// lanes per group, 32 values each in four 16-byte loads, the group's amax over the
+// four lanes, then 32 codes in two 16-byte stores.
 __global__ void quantize_rows_kernel(const __nv_bfloat16 *__restrict__ src, const int32_t *__restrict__ map,
                                      int k, int R, int K, uint8_t *__restrict__ q, float *__restrict__ s)
 {
     pdl_wait();
     pdl_trigger();
-    const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int warps_per_row = (K / 128 + 7) / 8;
+    const long wid = (long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    if (row >= R) return;
+    if (wid >= (long)R * warps_per_row) return;
+    const int row = (int)(wid / warps_per_row);
+    const int g = (int)(wid % warps_per_row) * 8 + lane / 4;  // this lane's group
+    const int sub = lane % 4;
+    const bool has = g < K / 128;                              // warp-uniform per group of 4 lanes
     const int sr = map ? map[row] / k : row;
-    const __nv_bfloat16 *a = src + (size_t)sr * K;
-    for (int g = 0; g < K / 128; ++g) {
-        const uint2 raw = *reinterpret_cast<const uint2 *>(a + g * 128 + lane * 4);
-        const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-        const float2 v01 = __bfloat1622float2(p[0]), v23 = __bfloat1622float2(p[1]);
-        float m = fmaxf(fmaxf(fabsf(v01.x), fabsf(v01.y)), fmaxf(fabsf(v23.x), fabsf(v23.y)));
+    float v[32];
+    float m = 0.0f;
+    if (has) {
+        const uint4 *a = reinterpret_cast<const uint4 *>(src + (size_t)sr * K + g * 128 + sub * 32);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        uint32_t packed = 0;
-        float sc = 1.0f;
-        if (m != 0.0f) {
-            sc = __fdiv_rn(m, 448.0f);
-            packed = e4m3_pair(qdiv(v01.x, sc), qdiv(v01.y, sc)) | (e4m3_pair(qdiv(v23.x, sc), qdiv(v23.y, sc)) << 16);
+        for (int i = 0; i < 4; ++i) {
+            const uint4 raw = a[i];
+            const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(p[j]);
+                v[8 * i + 2 * j] = f.x;
+                v[8 * i + 2 * j + 1] = f.y;
+                m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
         }
-        *reinterpret_cast<uint32_t *>(q + (size_t)row * K + g * 128 + lane * 4) = packed;
-        if (lane == 0) s[(size_t)row * (K / 128) + g] = sc;
     }
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    if (!has) return;
+    float sc = 1.0f;
+    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (m != 0.0f) {
+        sc = __fdiv_rn(m, 448.0f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            w[i] = e4m3_pair(qdiv(v[4 * i], sc), qdiv(v[4 * i + 1], sc)) |
+                   (e4m3_pair(qdiv(v[4 * i + 2], sc), qdiv(v[4 * i + 3], sc)) << 16);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(q + (size_t)row * K + g * 128 + sub * 32);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    if (sub == 0) s[(size_t)row * (K / 128) + g] = sc;
 }
 
 // ----------------------------------------------------------- grouped GEMM
@@ -319,27 +341,54 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 #pragma unroll
             for (int i = 0; i < 128; ++i) accr[i] = 0.0f;
             bool ok = true;
+            // the scales of K block kb + 1 are loaded while block kb is promoted
+            float na = 0.0f, nb0v = 0.0f, nb1v = 0.0f;
+            if (MODE != 2 && kbn > 0) {
+                na = row_ok ? sa[0] : 0.0f;
+                nb0v = nb_ok ? sb0[0] : 0.0f;
+                nb1v = MODE == 0 ? sb1[0] : 0.0f;
+            }
             for (int kb = 0; kb < kbn; ++kb) {
                 float c0 = 1.0f, c1 = 1.0f;  // mode 2: plain sum of the K-block partials
                 if (MODE != 2) {
-                    const float a_s = row_ok ? sa[kb] : 0.0f;
-                    c0 = nb_ok ? a_s * sb0[kb] : 0.0f;
-                    c1 = MODE == 0 ? a_s * sb1[kb] : c0;
+                    const float a_s = na;
+                    c0 = nb_ok ? a_s * nb0v : 0.0f;
+                    c1 = MODE == 0 ? a_s * nb1v : c0;
+                    if (kb + 1 < kbn) {
+                        na = row_ok ? sa[kb + 1] : 0.0f;
+                        nb0v = nb_ok ? sb0[kb + 1] : 0.0f;
+                        nb1v = MODE == 0 ? sb1[kb + 1] : 0.0f;
+                    }
                 }
                 if (!mbar_wait(&S->accf[acc], aphase, g.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+                // mode 0: chunks 0-3 = gate columns, 4-7 = up columns of this half
+                auto chunk_col = [&](int c) {
+                    return MODE == 0 ? (c < 4 ? half * 64 + c * 16 : 128 + half * 64 + (c - 4) * 16) : half * 128 + c * 16;
+                };
+                if (MODE != 2) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    // mode 0: chunks 0-3 = gate columns, 4-7 = up columns of this half
-                    const int col = MODE == 0 ? (c < 4 ? half * 64 + c * 16 : 128 + half * 64 + (c - 4) * 16)
-                                              : half * 128 + c * 16;
-                    const float cs = (MODE == 0 && c >= 4) ? c1 : c0;
-                    if (MODE == 2 && n0 + col >= g.N) continue;  // warp-uniform: columns past E
-                    uint32_t r[16];
-                    tmem_ld16_sync(tb + col, r);
+                    for (int c = 0; c < 8; c += 2) {  // two loads per TMEM wait
+                        uint32_t ra[16], rb[16];
+                        tmem_ld16x2_sync(tb + chunk_col(c), tb + chunk_col(c + 1), ra, rb);
+                        const float cs = (MODE == 0 && c >= 4) ? c1 : c0;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) accr[c * 16 + i] = fmaf(cs, __uint_as_float(r[i]), accr[c * 16 + i]);
+                        for (int i = 0; i < 16; ++i) {
+                            accr[c * 16 + i] = fmaf(cs, __uint_as_float(ra[i]), accr[c * 16 + i]);
+                            accr[(c + 1) * 16 + i] = fmaf(cs, __uint_as_float(rb[i]), accr[(c + 1) * 16 + i]);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const int col = chunk_col(c);
+                        if (n0 + col >= g.N) continue;  // warp-uniform: columns past E
+                        uint32_t r[16];
+                        tmem_ld16_sync(tb + col, r);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) accr[c * 16 + i] = fmaf(c0, __uint_as_float(r[i]), accr[c * 16 + i]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -446,9 +495,9 @@ bool fp8_smem_attr_ready(int v)  // v: 0 gate/up, 1 down, 2 router logits, 3 dow
 cudaError_t launch_quantize_rows(const __nv_bfloat16 *src, const int32_t *map, int k, int R, int K, uint8_t *q,
                                  float *s, cudaStream_t st)
 {
-    const int rows_per_block = 8;
-    return launch_pdl(quantize_rows_kernel, dim3((R + rows_per_block - 1) / rows_per_block), dim3(rows_per_block * 32),
-                      0, st, src, map, k, R, K, q, s);
+    const long warps = (long)R * ((K / 128 + 7) / 8);
+    return launch_pdl(quantize_rows_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, st, src, map, k, R, K, q,
+                      s);
 }
 
 cudaError_t launch_gather_rows_fp8(const uint8_t *xq, const float *xq_s, const int32_t *s2f, int A, int K, int k,
