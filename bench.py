@@ -37,6 +37,27 @@ if ROOT not in sys.path:
 from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_fp8_weights, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at 1 B200; % of BF16/FP8 TC peak or % of HBM BW"
+GEMM_TRACE_CTAS = 1024
+
+
+def schedule_stats(trace, mode):
+    """Per GEMM: the span from the first CTA start to the last CTA end, and how busy the
+    CTAs were over it (busy = that CTA's own start-to-end time)."""
+    out = {"mode": mode}
+    for k, name in enumerate(("gemm_gate_up", "gemm_down")):
+        spans = [(trace[2 * (k * GEMM_TRACE_CTAS + c)], trace[2 * (k * GEMM_TRACE_CTAS + c) + 1])
+                 for c in range(GEMM_TRACE_CTAS)]
+        spans = [(a, b) for a, b in spans if b > a > 0]
+        if not spans:
+            continue
+        t0, t1 = min(a for a, _ in spans), max(b for _, b in spans)
+        busy = sorted((b - a) / (t1 - t0) for a, b in spans)
+        out[name] = {"ctas": len(spans), "span_us": round((t1 - t0) / 1e3, 1),
+                     "busy_mean": round(sum(busy) / len(busy), 3), "busy_min": round(busy[0], 3),
+                     "busy_median": round(busy[len(busy) // 2], 3)}
+    return out
+
+
 def kernels_per_forward(cfg) -> int:
     """Library kernels one forward launches."""
     A = cfg.T * cfg.top_k
@@ -63,6 +84,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--schedule", default="queue", choices=["queue", "static_items", "static_experts"],
+                   help="how the GEMM CTAs get work items: the atomic queue (the design), or a static "
+                        "split of the items or of the experts (ablations)")
     p.add_argument("--shape", default="",
                    help="override config fields, e.g. T=1024,E=64 (reduced cases for profiler captures)")
     return p.parse_args()
@@ -425,6 +449,7 @@ def main():
     for s in ev + ev_step:
         for e in s:
             e.record(stream)
+    api.set_claim_order(False if args.schedule == "queue" else args.schedule)
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
         step()
@@ -444,18 +469,23 @@ def main():
                 flush.fill_(1)
                 api.set_stage_events([ev_step[i][0], None, None, None, None, ev_step[i][1]])
                 forward(x, cap)
-    # the stage breakdown: the same steps with the library's six stage marks
+    # the stage breakdown: the same steps with the library's six stage marks, and the
+    # GEMM CTAs' busy spans (the last step's remain in the trace buffer)
+    trace = torch.zeros(4 * GEMM_TRACE_CTAS, dtype=torch.int64, device=dev)
     graph_stages = torch.cuda.CUDAGraph()
     with torch.cuda.stream(cap):
         with torch.cuda.graph(graph_stages, stream=cap):
             for i in range(args.steps):
                 flush.fill_(1)
                 api.set_stage_events(ev[i])
+                api.set_gemm_trace(trace)
                 forward(x, cap)
     api.set_stage_events(None)
+    api.set_gemm_trace(None)
     stream.wait_stream(cap)
     graph_stages.replay()
     torch.cuda.synchronize()
+    sched = schedule_stats(trace.cpu().tolist(), args.schedule)
     graph.replay()  # one untimed replay so the timed one starts warm
     torch.cuda.synchronize()
 
@@ -532,7 +562,7 @@ def main():
                 "dtype": "e4m3" if fp8 else "bf16",
                 "data": "synthetic", "config": config_block(cfg, world),
                 "roofline": roof, "stages": stages, "experts_touched": work["_D"],
-                "e2e": e2e, "gpu_launches": kernels_per_forward(cfg) * args.steps,
+                "e2e": e2e, "gpu_launches": kernels_per_forward(cfg) * args.steps, "schedule": sched,
                 "clocks": clocks, "cpu_baseline": cpu,
                 "p99_ms_per_step": round(sorted(step_ms)[min(len(step_ms) - 1, math.ceil(0.99 * len(step_ms)) - 1)], 5)}
         print(json.dumps(line), flush=True)

@@ -177,9 +177,22 @@ moe_status_t moe_get_device_status(void *ws, void *stream);
  * check that.  Process-wide setting. */
 void moe_set_gemm_ctas(int32_t ctas);
 
-/* Order in which the GEMM CTAs claim work items: 0 = ascending (default),
- * 1 = descending.  Results are bitwise independent of it.  Process-wide. */
-void moe_set_claim_order(int32_t reverse);
+/* How the GEMM CTAs get their work items (the (m-tile, n-tile) pairs of the
+ * expert groups): 0 = the shared atomic queue in ascending order (default);
+ * 1 = the queue in descending order; 2 = a static split, CTA c taking items
+ * c, c + grid, ...; 3 = a static expert binding, CTA c taking every item of
+ * the experts e with e % grid == c (the fixed expert-to-SM assignment that the
+ * Weave review, section 2.2, contrasts with dynamic SM scheduling).  Results
+ * are bitwise independent of it; modes 2 and 3 exist to measure what the queue
+ * buys.  Process-wide. */
+void moe_set_claim_order(int32_t mode);
+
+/* Scheduling trace for benchmarks.  With `trace` a device buffer of 4 * ctas
+ * uint64 values (ctas >= the GEMM grid, 148 by default), every later forward
+ * records per GEMM CTA the %globaltimer (ns) when it started work and when it
+ * finished: [2c], [2c + 1] for the gate/up GEMM, [2 ctas + 2c], [2 ctas + 2c + 1]
+ * for the down GEMM.  NULL turns it off.  Process-wide. */
+void moe_set_gemm_trace(unsigned long long *trace, int32_t ctas);
 
 /* Failure-detection test hook.  Every wait inside the grouped GEMM pipelines
  * is bounded; `us` sets that bound in microseconds (<= 0: the default, 2 s).

@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 6: "MOE_ERR_BAD_INDEX", 7: "MOE_ERR_TOO_LARGE",
                 8: "MOE_ERR_ROUTER_BOUND"}
 EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "moe_forward",
-           "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order",
+           "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order", "moe_set_gemm_trace",
            "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",
            "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets"]
 DTYPE_BF16, DTYPE_FP8 = 0, 1
@@ -285,8 +285,23 @@ def set_wait_limit_us(us: int, stall_test: bool = False):
     lib().moe_set_wait_limit_us(int(us), 1 if stall_test else 0)
 
 
-def set_claim_order(reverse: bool):
-    lib().moe_set_claim_order(1 if reverse else 0)
+CLAIM_MODES = {"queue": 0, "queue_desc": 1, "static_items": 2, "static_experts": 3}
+
+
+def set_claim_order(reverse):
+    """False/True: the GEMMs' atomic work queue ascending/descending; or one of the
+    CLAIM_MODES names ("static_items", "static_experts" replace the queue)."""
+    mode = CLAIM_MODES[reverse] if isinstance(reverse, str) else (1 if reverse else 0)
+    lib().moe_set_claim_order(mode)
+
+
+def set_gemm_trace(buf):
+    """Record per GEMM CTA its start/end %globaltimer into `buf` (a CUDA int64 tensor of
+    4 * ctas entries, see moe_set_gemm_trace), or turn the trace off with None."""
+    if buf is None:
+        lib().moe_set_gemm_trace(None, 0)
+    else:
+        lib().moe_set_gemm_trace(ctypes.c_void_p(buf.data_ptr()), buf.numel() // 4)
 
 
 def set_stage_events(events):

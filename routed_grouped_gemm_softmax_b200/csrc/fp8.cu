@@ -171,7 +171,7 @@ __global__ void quantize_rows_kernel(const __nv_bfloat16 *__restrict__ src, cons
 
 template <int MODE, bool BF16, bool COMB = false>
 __global__ void __launch_bounds__(THREADS, 1)
-grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const Fp8GemmArgs g)
 {
     constexpr int BNO = MODE == 0 ? BN / 2 : BN;  // output columns per tile
@@ -207,7 +207,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         mbar_init(&S->fin, 1);
         mbar_init(&S->never, 1);
         fence_mbar_init();
-        tma_prefetch_desc(&tmA);
+        for (int b = 0; b < kABoxes; ++b) tma_prefetch_desc(&tmA.m[b]);
         tma_prefetch_desc(&tmB0);
         if (MODE == 0) tma_prefetch_desc(&tmB1);
     }
@@ -218,6 +218,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     const uint32_t tmem = S->tmem_base;
     pdl_wait();  // the prologue above overlapped the previous kernel
     pdl_trigger();
+    if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
     if (warp == 0) {
         // ------------------------------------------------ scheduler + TMA producer
@@ -226,12 +227,9 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             int stage = 0, rs = 0;
             uint32_t phase = 0, rphase = 0, armed = 0, armed_par = 0;
             bool ok = true;
+            int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
             for (;;) {
-                int item = atomicAdd(g.counter, 1);
-                if (item >= total)
-                    item = -1;
-                else if (g.reverse)
-                    item = total - 1 - item;
+                const int item = claim_item(g.reverse, g.counter, total, n_tiles * ksplit, dense ? nullptr : g.tiles, cursor);
                 if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
                 S->ring[rs] = item;
                 mbar_arrive(&S->itf[rs]);
@@ -240,15 +238,17 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 const int ks = item % ksplit, mn = item / ksplit;
                 const int mt = mn / n_tiles, nt = mn - mt * n_tiles;
                 const int expert = dense ? 0 : g.tiles[3 * mt], row0 = dense ? mt * BM : g.tiles[3 * mt + 1];
+                const int rows = dense ? min(BM, g.M - row0) : g.tiles[3 * mt + 2];
+                const int ab = a_box(rows);  // the A box that covers the tile's rows
                 const int n0 = nt * BNO;
                 const int kb0 = ks * KBS, kb1 = min(KB, kb0 + KBS);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&S->full[stage], A_BYTES + B_BYTES);
+                    mbar_arrive_expect_tx(&S->full[stage], a_box_rows(ab) * 128 + B_BYTES);
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     uint8_t *b_dst = sB + stage * B_BYTES;
-                    tma_load_2d(sA + stage * A_BYTES, &tmA, &S->full[stage], kb * KEL, row0);
+                    tma_load_2d(sA + stage * A_BYTES, &tmA.m[ab], &S->full[stage], kb * KEL, row0);
                     tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * KEL, n0, expert);
                     if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * KEL, n0, expert);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -465,6 +465,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 
     tc_fence_before();
     __syncthreads();
+    if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x + 1] = globaltimer_ns();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
@@ -508,7 +509,7 @@ cudaError_t launch_gather_rows_fp8(const uint8_t *xq, const float *xq_s, const i
                       dim3(rows_per_block * 32), 0, st, xq, xq_s, s2f, A, K, k, xs, xs_s);
 }
 
-cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
+cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                     const CUtensorMap &tmB1, cudaStream_t st)
 {
     const int grid = g.ctas > 0 ? g.ctas : num_sms();

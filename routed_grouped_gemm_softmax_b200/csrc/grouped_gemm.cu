@@ -83,7 +83,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const GemmArgs g)
 {
     // output columns per tile: mode 0 packs 128 gate + 128 up columns into N=256
@@ -115,7 +115,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         mbar_init(&S->fin, 1);
         mbar_init(&S->never, 1);
         fence_mbar_init();
-        tma_prefetch_desc(&tmA);
+        for (int b = 0; b < kABoxes; ++b) tma_prefetch_desc(&tmA.m[b]);
         tma_prefetch_desc(&tmB0);
         if (MODE == 0) tma_prefetch_desc(&tmB1);
     }
@@ -126,6 +126,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const uint32_t tmem = S->tmem_base;
     pdl_wait();  // the prologue above overlapped the previous kernel
     pdl_trigger();
+    if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
     if (warp == 0) {
         // ------------------------------------------------ scheduler + TMA producer
@@ -135,12 +136,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             uint32_t phase = 0, rphase = 0;
             uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
             bool ok = true;
+            int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
             for (;;) {
-                int item = atomicAdd(g.counter, 1);
-                if (item >= total)
-                    item = -1;
-                else if (g.reverse)
-                    item = total - 1 - item;
+                const int item = claim_item(g.reverse, g.counter, total, n_tiles, dense ? nullptr : g.tiles, cursor);
                 if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
                 S->ring[rs] = item;
                 mbar_arrive(&S->itf[rs]);
@@ -148,15 +146,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (item < 0) break;
                 const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
                 const int expert = dense ? 0 : g.tiles[3 * mt], row0 = dense ? mt * BM : g.tiles[3 * mt + 1];
+                const int rows = dense ? min(BM, g.M - row0) : g.tiles[3 * mt + 2];
+                const int ab = a_box(rows);  // the A box that covers the tile's rows
                 const int n0 = nt * BNO;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&S->full[stage], A_BYTES + B_BYTES);
+                    mbar_arrive_expect_tx(&S->full[stage], a_box_rows(ab) * BK * 2 + B_BYTES);
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     uint8_t *a_dst = sA + stage * A_BYTES;
                     uint8_t *b_dst = sB + stage * B_BYTES;
-                    tma_load_2d(a_dst, &tmA, &S->full[stage], kb * BK, row0);
+                    tma_load_2d(a_dst, &tmA.m[ab], &S->full[stage], kb * BK, row0);
                     tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
                     if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -305,6 +305,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
+    if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x + 1] = globaltimer_ns();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
@@ -342,7 +343,7 @@ static bool smem_attr_ready(int mode)
     return true;
 }
 
-cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
+cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                 const CUtensorMap &tmB1, cudaStream_t st)
 {
     const int grid = g.ctas > 0 ? g.ctas : num_sms();

@@ -20,6 +20,8 @@ namespace {
 
 std::atomic<int> g_gemm_ctas{0};
 std::atomic<int> g_claim_reverse{0};
+std::atomic<unsigned long long *> g_trace{nullptr};
+std::atomic<int> g_trace_ctas{0};
 std::atomic<unsigned long long> g_wait_ns{0};
 std::atomic<int> g_stall_test{0};
 std::mutex g_ev_mu;
@@ -207,14 +209,27 @@ bool encode_sw128_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint6
     return encode_2d(m, base, rows, cols, box_rows);
 }
 
+// A-operand tensor maps with boxes of 16/32/64/128 rows (bf16 64 columns, or 128
+// e4m3 bytes), 128-byte swizzle.
+bool encode_a_maps(AMaps *m, const void *base, uint64_t rows, uint64_t cols, bool u8)
+{
+    for (int b = 0; b < kABoxes; ++b) {
+        const uint32_t br = (uint32_t)a_box_rows(b);
+        if (!(u8 ? encode_2d_u8(&m->m[b], base, rows, cols, br) : encode_2d(&m->m[b], base, rows, cols, br)))
+            return false;
+    }
+    return true;
+}
+
 // The router's tensor-core logits: the block-promoting GEMM (fp8.cu, mode 2, bf16
 // operands) over plain 128-row blocks of x against the transposed router matrix,
 // K split over enough items to occupy the GPU.  Uses work counter 2.
 cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, int T, int H, int E, float *logits,
                              WsHeader *hdr, int *ksplit_out, cudaStream_t st)
 {
-    CUtensorMap tm_x, tm_w;
-    if (!encode_2d(&tm_x, x, T, H, kTileRows) || !encode_3d(&tm_w, wrt, 1, E, H, 256)) return cudaErrorInvalidValue;
+    AMaps tm_x;
+    CUtensorMap tm_w;
+    if (!encode_a_maps(&tm_x, x, T, H, false) || !encode_3d(&tm_w, wrt, 1, E, H, 256)) return cudaErrorInvalidValue;
     const int items = ((T + kTileRows - 1) / kTileRows) * ((E + 255) / 256);
     int ks = (120 + items - 1) / items;
     ks = ks < 1 ? 1 : ks > kRouterKSplitMax ? kRouterKSplitMax : ks;
@@ -250,7 +265,13 @@ int32_t moe_max_tiles(const moe_dims_t *d)
 
 void moe_set_gemm_ctas(int32_t ctas) { g_gemm_ctas.store(ctas > 0 ? ctas : 0); }
 
-void moe_set_claim_order(int32_t reverse) { g_claim_reverse.store(reverse ? 1 : 0); }
+void moe_set_claim_order(int32_t mode) { g_claim_reverse.store(mode < 0 ? 0 : mode > 3 ? 3 : mode); }
+
+void moe_set_gemm_trace(unsigned long long *trace, int32_t ctas)
+{
+    g_trace.store(trace && ctas > 0 ? trace : nullptr);
+    g_trace_ctas.store(ctas > 0 ? ctas : 0);
+}
 
 void moe_set_wait_limit_us(int32_t us, int32_t stall_test)
 {
@@ -329,11 +350,12 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
     auto *tiles = at<int32_t>(ws, L.tiles);
     auto *ntiles = at<int32_t>(ws, L.ntiles);
 
-    CUtensorMap tm_xs, tm_wg, tm_wu, tm_h, tm_wd;
-    if (!encode_2d(&tm_xs, xs, A, d->H, moe::kTileRows) ||
+    moe::AMaps tm_xs, tm_h;
+    CUtensorMap tm_wg, tm_wu, tm_wd;
+    if (!moe::encode_a_maps(&tm_xs, xs, A, d->H, false) ||
         !encode_3d(&tm_wg, w_gate, d->E, d->I, d->H, 128) ||
         !encode_3d(&tm_wu, w_up, d->E, d->I, d->H, 128) ||
-        !encode_2d(&tm_h, h, A, d->I, moe::kTileRows) ||
+        !moe::encode_a_maps(&tm_h, h, A, d->I, false) ||
         !encode_3d(&tm_wd, w_down, d->E, d->H, d->I, 256))
         return MOE_ERR_CUDA;
 
@@ -346,11 +368,13 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
         e = moe::launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), s2f, A, d->H, d->top_k, xs, st);
     if (e == cudaSuccess) e = marks.mark(2, st);
     const int ctas = g_gemm_ctas.load(), rev = g_claim_reverse.load();
+    unsigned long long *trace1 = g_trace.load(), *trace2 = trace1 ? trace1 + 2 * g_trace_ctas.load() : nullptr;
     const unsigned long long wl = g_wait_ns.load();
     const uint64_t wait_ns = wl ? wl : 2000000000ull;
     const int stall = g_stall_test.load();
     if (e == cudaSuccess) {
         moe::GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, h, nullptr, ctas, rev, wait_ns, stall};
+        g1.trace = trace1;
         e = moe::launch_grouped_gemm(g1, tm_xs, tm_wg, tm_wu, st);
     }
     if (e == cudaSuccess) e = marks.mark(3, st);
@@ -358,6 +382,7 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
         moe::GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, y, s2f, ctas, rev, wait_ns,
                          stall, 0, nullptr, gate, fused ? at<int32_t>(ws, L.ccnt) : nullptr,
                          static_cast<__nv_bfloat16 *>(out), d->top_k, d->top_k};
+        g2.trace = trace2;
         e = moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st);
     }
     if (e == cudaSuccess) e = marks.mark(4, st);
@@ -407,9 +432,10 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
     auto *tiles = at<int32_t>(ws, L.tiles);
     auto *ntiles = at<int32_t>(ws, L.ntiles);
 
-    CUtensorMap tm_xs, tm_wg, tm_wu, tm_h, tm_wd;
-    if (!encode_2d_u8(&tm_xs, xs, A, d->H, moe::kTileRows) || !encode_3d_u8(&tm_wg, w_gate_q, d->E, d->I, d->H, 128) ||
-        !encode_3d_u8(&tm_wu, w_up_q, d->E, d->I, d->H, 128) || !encode_2d_u8(&tm_h, h, A, d->I, moe::kTileRows) ||
+    moe::AMaps tm_xs, tm_h;
+    CUtensorMap tm_wg, tm_wu, tm_wd;
+    if (!moe::encode_a_maps(&tm_xs, xs, A, d->H, true) || !encode_3d_u8(&tm_wg, w_gate_q, d->E, d->I, d->H, 128) ||
+        !encode_3d_u8(&tm_wu, w_up_q, d->E, d->I, d->H, 128) || !moe::encode_a_maps(&tm_h, h, A, d->I, true) ||
         !encode_3d_u8(&tm_wd, w_down_q, d->E, d->H, d->I, 256))
         return MOE_ERR_CUDA;
 
@@ -427,12 +453,14 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
                                         xs_s, st);
     if (e == cudaSuccess) e = marks.mark(2, st);
     const int ctas = g_gemm_ctas.load(), rev = g_claim_reverse.load();
+    unsigned long long *trace1 = g_trace.load(), *trace2 = trace1 ? trace1 + 2 * g_trace_ctas.load() : nullptr;
     const unsigned long long wl = g_wait_ns.load();
     const uint64_t wait_ns = wl ? wl : 2000000000ull;
     const int stall = g_stall_test.load();
     if (e == cudaSuccess) {
         moe::Fp8GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, xs_s, w_gate_s, w_up_s,
                             h, h_s, nullptr, nullptr, ctas, rev, wait_ns, stall};
+        g1.trace = trace1;
         e = moe::launch_grouped_gemm_fp8(g1, tm_xs, tm_wg, tm_wu, st);
     }
     if (e == cudaSuccess) e = marks.mark(3, st);
@@ -441,6 +469,7 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
                             nullptr, nullptr, y, s2f, ctas, rev, wait_ns, stall, 0, 1, nullptr, gate,
                             fused ? at<int32_t>(ws, L.ccnt) : nullptr, static_cast<__nv_bfloat16 *>(out), d->top_k,
                             2 * d->top_k};
+        g2.trace = trace2;
         e = moe::launch_grouped_gemm_fp8(g2, tm_h, tm_wd, tm_wd, st);
     }
     if (e == cudaSuccess) e = marks.mark(4, st);

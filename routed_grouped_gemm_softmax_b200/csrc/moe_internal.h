@@ -137,6 +137,16 @@ cudaError_t launch_gather_rows(const __nv_bfloat16 *x, const int32_t *s2f, int A
 // Grouped GEMMs over the tile list.  mode 0: h = silu(A Wg^T) * (A Wu^T) (A = the
 // expert-sorted activations, B = gate/up weights); mode 1: y[s2f[row]] = A Wd^T
 // (A = h).  The tensor maps are encoded by the caller.
+// Tensor maps of one A operand with boxes of 16, 32, 64 and 128 rows: a tile loads
+// only the smallest box that covers its rows (the rest of its shared-memory tile is
+// left as it is; those output rows are masked).
+constexpr int kABoxes = 4;
+struct AMaps {
+    CUtensorMap m[kABoxes];
+};
+__host__ __device__ inline int a_box(int rows) { return rows <= 16 ? 0 : rows <= 32 ? 1 : rows <= 64 ? 2 : 3; }
+__host__ __device__ inline int a_box_rows(int b) { return 16 << b; }
+
 struct GemmArgs {
     int mode;
     int K, N;
@@ -147,7 +157,7 @@ struct GemmArgs {
     __nv_bfloat16 *out;
     const int32_t *row_map;
     int ctas;
-    int reverse;
+    int reverse;       // claim mode: 0/1 queue ascending/descending, 2 static items, 3 static experts
     uint64_t wait_ns;  // limit of each pipeline wait
     int stall_test;    // MMA thread first waits on a barrier nothing signals
     int M;             // mode 2 (no tile list): rows of A
@@ -160,9 +170,10 @@ struct GemmArgs {
     __nv_bfloat16 *comb_out;      // [T, N]
     int comb_k;
     int comb_target;
+    unsigned long long *trace;  // per CTA {start, end} globaltimer (ns), or null
 };
 // mode 2: out_f32 = A B^T over M rows (one "expert"), the router's tensor-core logits.
-cudaError_t launch_grouped_gemm(const GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
+cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                 const CUtensorMap &tmB1, cudaStream_t st);
 
 // FP8 block-scaled grouped GEMMs (fp8.cu).  mode 0: h codes/scales from
@@ -183,7 +194,7 @@ struct Fp8GemmArgs {
     __nv_bfloat16 *out;      // mode 1: y [T*k, N]
     const int32_t *row_map;  // mode 1: sorted row -> flat row
     int ctas;
-    int reverse;
+    int reverse;  // claim mode, as in GemmArgs
     uint64_t wait_ns;
     int stall_test;
     int M;            // mode 2: rows of A (no tile list)
@@ -194,8 +205,9 @@ struct Fp8GemmArgs {
     __nv_bfloat16 *comb_out;
     int comb_k;
     int comb_target;
+    unsigned long long *trace;  // per CTA {start, end} globaltimer (ns), or null
 };
-cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const CUtensorMap &tmA, const CUtensorMap &tmB0,
+cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                     const CUtensorMap &tmB1, cudaStream_t st);
 cudaError_t launch_quantize_rows(const __nv_bfloat16 *src, const int32_t *map, int k, int R, int K, uint8_t *q,
                                  float *s, cudaStream_t st);

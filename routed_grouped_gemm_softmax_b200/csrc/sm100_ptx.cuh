@@ -20,6 +20,32 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// The next work item of this CTA (-1: none left).  Mode 0/1: the shared atomic
+// queue, ascending or descending; mode 2: a static split, CTA c taking items c,
+// c + grid, ...; mode 3: a static expert binding, CTA c taking (in order) every
+// item of the experts e with e % grid == c.  Modes 2 and 3 exist to measure what
+// the queue buys on skewed routing.  items_per_mtile maps an item to its m-tile.
+__device__ __forceinline__ int claim_item(int mode, int32_t *counter, int total, int items_per_mtile,
+                                          const int32_t *tiles, int &cursor)
+{
+    if (mode <= 1) {
+        const int item = atomicAdd(counter, 1);
+        if (item >= total) return -1;
+        return mode == 1 ? total - 1 - item : item;
+    }
+    if (mode == 2) {
+        const int item = cursor;
+        cursor += gridDim.x;
+        return item < total ? item : -1;
+    }
+    while (cursor < total) {
+        const int item = cursor++;
+        const int e = tiles ? tiles[3 * (item / items_per_mtile)] : 0;
+        if (e % (int)gridDim.x == (int)blockIdx.x) return item;
+    }
+    return -1;
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)

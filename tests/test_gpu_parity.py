@@ -121,7 +121,8 @@ def test_schedule_independence(T):
     g, _ = device_inputs(cfg)
     outs = []
     try:
-        for ctas, rev in [(0, False), (1, False), (7, True), (148, False), (0, True), (3, True)]:
+        for ctas, rev in [(0, False), (1, False), (7, True), (148, False), (0, True), (3, True),
+                          (0, "static_items"), (0, "static_experts"), (5, "static_experts")]:
             api.set_gemm_ctas(ctas)
             api.set_claim_order(rev)
             outs.append(api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"],
