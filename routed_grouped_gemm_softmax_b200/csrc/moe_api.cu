@@ -173,7 +173,8 @@ cudaError_t route_and_permute(const moe_dims_t &d, const moe::WsLayout &L, const
     if (moe::small_route_permute_ok(d)) {
         cudaError_t e = moe::launch_route_permute_small(d, xb, wb, router_bias, at<float>(ws, L.logits), idx, gate,
                                                         at<int32_t>(ws, L.offsets), s2f, at<int32_t>(ws, L.f2s),
-                                                        tiles, ntiles, hdr, st);
+                                                        tiles, ntiles, hdr, at<int32_t>(ws, L.ccnt),
+                                                        (int)((L.clear_bytes - L.ccnt) / 4), st);
         return e == cudaSuccess ? marks.mark(1, st) : e;
     }
     cudaError_t e =
@@ -362,7 +363,8 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
     const StageMarks marks;
     const bool fused = d->T <= moe::kFusedCombineMaxT;  // combine inside the down GEMM
     cudaError_t e = marks.mark(0, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);  // header + combine counts
+    if (e == cudaSuccess && !moe::small_route_permute_ok(*d))  // else the router's kernels clear them
+        e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);          // header + combine counts
     if (e == cudaSuccess) e = route_and_permute(*d, L, x, router_w, router_bias, ws, hdr, marks, st);
     if (e == cudaSuccess)
         e = moe::launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), s2f, A, d->H, d->top_k, xs, st);
@@ -442,7 +444,8 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
     const StageMarks marks;
     const bool fused = d->T <= moe::kFusedCombineMaxT;  // combine inside the down GEMM
     cudaError_t e = marks.mark(0, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);  // header + combine counts
+    if (e == cudaSuccess && !moe::small_route_permute_ok(*d))  // else the router's kernels clear them
+        e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);          // header + combine counts
     if (e == cudaSuccess) e = route_and_permute(*d, L, x, router_w, router_bias, ws, hdr, marks, st);
     // x quantised once per token, then its codes gathered into expert order
     if (e == cudaSuccess)

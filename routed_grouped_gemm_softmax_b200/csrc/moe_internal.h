@@ -118,12 +118,14 @@ cudaError_t launch_route_certified(const moe_dims_t &d, const __nv_bfloat16 *x, 
                                    const RouterScratch &rs, WsHeader *hdr, cudaStream_t st);
 
 // Router + permute in two launches for small batches (T <= 32, E % 8 == 0,
-// H % 128 == 0, T*k <= 4096, ceil(T*k/32) * E <= 16384).
+// H % 128 == 0, T*k <= 4096, ceil(T*k/32) * E <= 16384).  They also clear the
+// workspace header (status word, work counters) and the nccnt combine counts,
+// so a forward on this path needs no memset.
 bool small_route_permute_ok(const moe_dims_t &d);
 cudaError_t launch_route_permute_small(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
                                        const float *bias, float *logits, int32_t *idx, float *gate,
                                        int32_t *offsets, int32_t *s2f, int32_t *f2s, int32_t *tiles,
-                                       int32_t *ntiles, WsHeader *hdr, cudaStream_t st);
+                                       int32_t *ntiles, WsHeader *hdr, int32_t *ccnt, int nccnt, cudaStream_t st);
 
 cudaError_t launch_permute(const moe_dims_t &d, const WsLayout &L, const int32_t *idx,
                            int32_t *blk_cnt, int32_t *blk_base, int32_t *offsets, int32_t *s2f,

@@ -303,8 +303,10 @@ cudaError_t launch_logits_small(const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
 // TP rows arrive as untiled bulk copies (one per row, on one barrier); router_w's
 // 8-expert column slice arrives as 256 x 8 tiles of a tensor map (one barrier per
 // 256 values of h), so the chains start as soon as the first tile lands and no
-// thread spends issue slots on staging.  Needs E % 8 == 0, H % 256 == 0 and
-// TP * (2H + 16) + 16H bytes of shared memory.
+// thread spends issue slots on staging.  A CTA takes TP = 8 tokens (blockIdx.y) of
+// the 8 experts: every step reads a weight and an eighth of an x vector from
+// shared memory, so few warps per SM keep the loads under the fma latency.  Needs
+// E % 8 == 0, H % 256 == 0 and TP * (2H + 16) + 16H bytes of shared memory.
 constexpr int kLogitsChunk = 256;
 
 __host__ __device__ inline size_t logits_tma_smem(int TP, int H)
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(TP * 8) route_logits_tma_kernel(const __grid_c
                                                                   const __nv_bfloat16 *__restrict__ x,
                                                                   const float *__restrict__ bias, int T, int H,
                                                                   int E, float *__restrict__ logits,
-                                                                  int32_t *__restrict__ status)
+                                                                  int32_t *__restrict__ status, int clear_status)
 {
     extern __shared__ __align__(128) uint8_t tsm_l[];
     constexpr int TE = 8;
@@ -328,7 +330,8 @@ __global__ void __launch_bounds__(TP * 8) route_logits_tma_kernel(const __grid_c
     uint8_t *wsm = tsm_l + (256 + (size_t)TP * pitch + 127) / 128 * 128;
     const int tid = threadIdx.x, tt = tid / TE, ee = tid % TE;
     const int e0 = blockIdx.x * TE;
-    const int rows = min(TP, T);
+    const int t0 = blockIdx.y * TP;
+    const int rows = min(TP, T - t0);
     if (tid == 0) {
         for (int i = 0; i <= nch; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
@@ -336,6 +339,7 @@ __global__ void __launch_bounds__(TP * 8) route_logits_tma_kernel(const __grid_c
     __syncthreads();
     pdl_wait();
     pdl_trigger();
+    if (clear_status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *status = 0;  // first kernel of a forward
     if (tid < 32) {
         if (tid == 0) {
             mbar_arrive_expect_tx(&bars[0], (uint32_t)(rows * H * 2));
@@ -345,7 +349,8 @@ __global__ void __launch_bounds__(TP * 8) route_logits_tma_kernel(const __grid_c
             }
         }
         __syncwarp();
-        for (int r = tid; r < rows; r += 32) bulk_load(xs + (size_t)r * pitch, x + (size_t)r * H, H * 2, &bars[0]);
+        for (int r = tid; r < rows; r += 32)
+            bulk_load(xs + (size_t)r * pitch, x + (size_t)(t0 + r) * H, H * 2, &bars[0]);
     }
     bool ok = mbar_wait(&bars[0], 0);
     float acc = 0.0f;
@@ -380,17 +385,17 @@ __global__ void __launch_bounds__(TP * 8) route_logits_tma_kernel(const __grid_c
         return;
     }
     const int e = e0 + ee;
-    if (tt < T && e < E) {
+    if (tt < rows && e < E) {
         float v = acc;
         if (bias) v = __fadd_rn(v, bias[e]);
-        logits[(size_t)tt * E + e] = v;
+        logits[(size_t)(t0 + tt) * E + e] = v;
     }
 }
 
 // Launches the TMA-fed kernel when the shape allows it (returns false otherwise).
 template <int TP>
 bool try_launch_logits_tma(const __nv_bfloat16 *x, const __nv_bfloat16 *wr, const float *bias, int T, int H, int E,
-                           float *logits, int32_t *status, cudaStream_t st, cudaError_t *err)
+                           float *logits, int32_t *status, int clear_status, cudaStream_t st, cudaError_t *err)
 {
     const size_t smem = logits_tma_smem(TP, H);
     if (E % 8 || H % kLogitsChunk || H / kLogitsChunk > 31 || smem > 227 * 1024) return false;
@@ -399,19 +404,21 @@ bool try_launch_logits_tma(const __nv_bfloat16 *x, const __nv_bfloat16 *wr, cons
     auto kern = route_logits_tma_kernel<TP>;
     *err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (*err != cudaSuccess) return true;
-    *err = launch_pdl(kern, dim3(E / 8), dim3(TP * 8), smem, st, tm, x, bias, T, H, E, logits, status);
+    *err = launch_pdl(kern, dim3(E / 8, (T + TP - 1) / TP), dim3(TP * 8), smem, st, tm, x, bias, T, H, E, logits,
+                      status, clear_status);
     return true;
 }
 
 // The small-batch logits: TMA-fed when the rows fit in shared memory, else the
-// cp.async ring.
+// cp.async ring.  With clear_status the status word is zeroed first (by the TMA
+// kernel, or by a memset ahead of the cp.async one).
 cudaError_t launch_logits_small_any(const __nv_bfloat16 *x, const __nv_bfloat16 *wr, const float *bias, int T,
-                                    int H, int E, float *logits, int32_t *status, cudaStream_t st)
+                                    int H, int E, float *logits, int32_t *status, cudaStream_t st,
+                                    bool clear_status = false)
 {
     cudaError_t err = cudaSuccess;
-    if (T <= 16 ? try_launch_logits_tma<16>(x, wr, bias, T, H, E, logits, status, st, &err)
-                : try_launch_logits_tma<32>(x, wr, bias, T, H, E, logits, status, st, &err))
-        return err;
+    if (try_launch_logits_tma<8>(x, wr, bias, T, H, E, logits, status, clear_status, st, &err)) return err;
+    if (clear_status && (err = cudaMemsetAsync(status, 0, sizeof(int32_t), st)) != cudaSuccess) return err;
     return T <= 16 ? launch_logits_small<16, 8, 128, 16>(x, wr, bias, T, H, E, logits, st)
                    : launch_logits_small<32, 8, 128, 16>(x, wr, bias, T, H, E, logits, st);
 }
@@ -500,6 +507,8 @@ struct SmallRouteOut {
     int32_t *offsets, *s2f, *f2s, *tiles, *ntiles;
     int32_t *counters;
     int ncounters;
+    int32_t *ccnt;   // the fused combine's arrival counts, zeroed here
+    int nccnt;
     int32_t *status;
 };
 
@@ -614,6 +623,7 @@ __global__ void __launch_bounds__(1024) topk_permute_small_kernel(int T, int E, 
         }
     }
     if (tid < o.ncounters) o.counters[tid] = 0;
+    for (int i = tid; i < o.nccnt; i += NT) o.ccnt[i] = 0;
 }
 
 }  // namespace
@@ -627,10 +637,10 @@ bool small_route_permute_ok(const moe_dims_t &d)
 cudaError_t launch_route_permute_small(const moe_dims_t &d, const __nv_bfloat16 *x, const __nv_bfloat16 *wr,
                                        const float *bias, float *logits, int32_t *idx, float *gate,
                                        int32_t *offsets, int32_t *s2f, int32_t *f2s, int32_t *tiles,
-                                       int32_t *ntiles, WsHeader *hdr, cudaStream_t st)
+                                       int32_t *ntiles, WsHeader *hdr, int32_t *ccnt, int nccnt, cudaStream_t st)
 {
-    SmallRouteOut o{logits, idx, gate, offsets, s2f, f2s, tiles, ntiles, hdr->counter, 7, &hdr->status};
-    cudaError_t e = launch_logits_small_any(x, wr, bias, d.T, d.H, d.E, logits, &hdr->status, st);
+    SmallRouteOut o{logits, idx, gate, offsets, s2f, f2s, tiles, ntiles, hdr->counter, 7, ccnt, nccnt, &hdr->status};
+    cudaError_t e = launch_logits_small_any(x, wr, bias, d.T, d.H, d.E, logits, &hdr->status, st, true);
     if (e != cudaSuccess) return e;
     const int warps = d.T < 4 ? 4 : d.T;
     const size_t smem = small_topk_permute_smem(d.T, d.E, d.top_k, warps);
