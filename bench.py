@@ -87,6 +87,8 @@ def parse():
     p.add_argument("--schedule", default="queue", choices=["queue", "static_items", "static_experts"],
                    help="how the GEMM CTAs get work items: the atomic queue (the design), or a static "
                         "split of the items or of the experts (ablations)")
+    p.add_argument("--pair", default="auto", choices=["auto", "always", "never"],
+                   help="the bf16 GEMMs on CTA pairs (tcgen05 cta_group::2): automatic choice or forced")
     p.add_argument("--shape", default="",
                    help="override config fields, e.g. T=1024,E=64 (reduced cases for profiler captures)")
     return p.parse_args()
@@ -450,6 +452,7 @@ def main():
         for e in s:
             e.record(stream)
     api.set_claim_order(False if args.schedule == "queue" else args.schedule)
+    api.set_pair_mma(args.pair)
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
         step()

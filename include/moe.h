@@ -187,6 +187,13 @@ void moe_set_gemm_ctas(int32_t ctas);
  * buys.  Process-wide. */
 void moe_set_claim_order(int32_t mode);
 
+/* Pair-of-CTA GEMMs (tcgen05 cta_group::2: a 256 x 256 tile per 2-CTA cluster,
+ * each CTA loading half the operands).  0 = automatic (the bf16 forward uses
+ * them when the batch is not a small one and averages at least 512 rows per
+ * expert), 1 = whenever the forward can (tests), 2 = never.  Results are bitwise
+ * independent of it.  Process-wide. */
+void moe_set_pair_mma(int32_t mode);
+
 /* Scheduling trace for benchmarks.  With `trace` a device buffer of 4 * ctas
  * uint64 values (ctas >= the GEMM grid, 148 by default), every later forward
  * records per GEMM CTA the %globaltimer (ns) when it started work and when it

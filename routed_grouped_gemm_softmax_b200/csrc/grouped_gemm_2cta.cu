@@ -1,0 +1,434 @@
+// grouped_gemm_2cta.cu -- the bf16 grouped GEMMs with pair-of-CTA MMAs
+// (tcgen05 cta_group::2), for expert groups large enough to be compute-bound.
+//
+// A work item is one (pair tile, n-tile): a pair tile is up to 256 rows of one
+// expert group, split 128 + 128 over the two CTAs of a cluster.  One MMA of
+// M = 256, N = 256, K = 16 reads the A rows from both CTAs' shared memory and B
+// from both too -- each CTA holds only half of the 256 B rows (the gate rows on
+// CTA 0 and the up rows on CTA 1 in the gate/up GEMM; the first and second 128
+// output columns in the down GEMM) -- so per CTA a 64-wide K block moves 32 KB
+// instead of the 48 KB of the one-CTA kernel for the same tensor-core work.  Each
+// CTA's TMEM accumulator holds its own 128 rows x 256 columns, so the epilogue is
+// the one-CTA kernel's.
+//
+// Roles: CTA 0 (the leader) claims items from the atomic queue and hands each one
+// to CTA 1 through its shared memory; in both CTAs warp 0 streams that CTA's A and
+// B halves with TMA, completing on the leader's stage barrier; the leader's warp 1
+// issues the MMAs and commits each stage, the accumulators and the end to both
+// CTAs' barriers at once (tcgen05.commit with a CTA mask); warps 2-5 of both CTAs
+// drain their accumulator halves.  No TMA load is multicast.  Every wait is
+// bounded, and a CTA leaves only after the other has finished touching it.
+#include <mutex>
+
+#include "moe_internal.h"
+#include "pdl.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int HALF = kTileRows;        // rows per CTA of a pair tile
+constexpr int BK2 = 64;
+constexpr int BN2 = 256;               // MMA N (128 B rows per CTA)
+constexpr int ST2 = 6;
+constexpr int RING2 = 4;
+constexpr int A2_BYTES = HALF * BK2 * 2;   // 16 KB
+constexpr int B2_BYTES = 128 * BK2 * 2;    // 16 KB
+constexpr int THREADS2 = 192;
+constexpr uint32_t TMEM_COLS2 = 512;
+
+struct Ctrl2 {
+    uint64_t full[ST2];    // leader: both CTAs' TMA bytes of stage s landed (2 arrivals + tx)
+    uint64_t empty[ST2];   // each: the pair's MMAs reading stage s finished
+    uint64_t accf[2];      // each: accumulator a holds a finished tile
+    uint64_t acce[2];      // leader: all 8 epilogue warps drained accumulator a
+    uint64_t itf[RING2];   // each: ring slot r holds the next item
+    uint64_t ite[RING2];   // leader: the 10 consumers of both CTAs read slot r
+    uint64_t fin;          // each: every MMA of the pair completed
+    uint64_t bye;          // each: the other CTA is done touching this one
+    int32_t ring[RING2];
+    uint32_t tmem_base;
+};
+
+constexpr size_t SMEM2 = 1024 + (size_t)ST2 * (A2_BYTES + B2_BYTES) + sizeof(Ctrl2);
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(const void *p, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void arrive_remote(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// The stage arrival of the peer's producer: relaxed, since it publishes no data of
+// its own (its TMA bytes complete on the barrier themselves); a release at cluster
+// scope would wait for every earlier memory operation of the thread.
+__device__ __forceinline__ void arrive_expect_tx_remote(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void st_remote(uint32_t addr, int32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// TMA tile loads into this CTA's shared memory that complete on a barrier of either CTA.
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *tm, uint32_t bar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *tm, uint32_t bar, int x, int y, int z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
+        "r"(0u), "r"(0u)
+        : "memory");
+}
+// Arrive (once the MMAs issued so far complete) on `bar` in both CTAs of the pair.
+__device__ __forceinline__ void mma_commit_pair(uint64_t *bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+
+// Bounded wait with cluster-scope acquire: these barriers are also arrived on from
+// the other CTA (remote arrives, TMA completions, multicast commits).
+__device__ __forceinline__ bool try_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool wait2(uint64_t *bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs)
+{
+    if (try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 256; ++i)
+            if (try_wait_cluster(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+__device__ __forceinline__ void record2(int32_t *status, int code) { atomicCAS(status, 0, code); }
+__device__ __forceinline__ float silu2(float a) { return a / (1.0f + __expf(-a)); }
+__device__ __forceinline__ uint32_t pack_bf16_2(float a, float b)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// MODE 0: h = silu(x Wg^T) * (x Wu^T) -> bf16 rows of h; MODE 1: y rows of x Wd^T.
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
+    grouped_gemm_2cta_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB0,
+                             const __grid_constant__ CUtensorMap tmB1, const GemmArgs g, const int32_t *tiles2,
+                             const int32_t *ntiles2)
+{
+    constexpr int BNO = MODE == 0 ? BN2 / 2 : BN2;  // output columns per item
+    extern __shared__ uint8_t smem2[];
+    const uint32_t pad = (1024u - (smem_u32(smem2) & 1023u)) & 1023u;
+    uint8_t *sA = smem2 + pad;
+    uint8_t *sB = sA + ST2 * A2_BYTES;
+    Ctrl2 *S = reinterpret_cast<Ctrl2 *>(sB + ST2 * B2_BYTES);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_rank();
+    const int n_tiles = (g.N + BNO - 1) / BNO;
+    const int num_kb = g.K / BK2;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < ST2; ++s) {
+            mbar_init(&S->full[s], 2);
+            mbar_init(&S->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&S->accf[a], 1);
+            mbar_init(&S->acce[a], 8);
+        }
+        for (int r = 0; r < RING2; ++r) {
+            mbar_init(&S->itf[r], 1);
+            mbar_init(&S->ite[r], 10);
+        }
+        mbar_init(&S->fin, 1);
+        mbar_init(&S->bye, 1);
+        fence_mbar_init();
+        for (int b = 0; b < kABoxes; ++b) tma_prefetch_desc(&tmA.m[b]);
+        tma_prefetch_desc(&tmB0);
+        if (MODE == 0) tma_prefetch_desc(&tmB1);
+    }
+    if (warp == 1) tmem_alloc_pair(&S->tmem_base, TMEM_COLS2);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem = S->tmem_base;
+    pdl_wait();
+    pdl_trigger();
+    if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
+
+    if (warp == 0) {
+        // -------------------------------- item hand-off (leader) + TMA producer (both)
+        if (lane == 0) {
+            const int total = *ntiles2 * n_tiles;
+            int stage = 0, rs = 0, cursor = 0;
+            uint32_t phase = 0, rphase = 0;
+            bool ok = true;
+            for (;;) {
+                int item;
+                if (rank == 0) {
+                    item = claim_item(g.reverse, g.counter, total, n_tiles, tiles2, cursor);
+                    if (!wait2(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
+                    S->ring[rs] = item;
+                    st_remote(peer_addr(&S->ring[rs], 1), item);
+                    mbar_arrive(&S->itf[rs]);
+                    arrive_remote(peer_addr(&S->itf[rs], 1));
+                } else {
+                    if (!wait2(&S->itf[rs], rphase, g.wait_ns)) { ok = false; break; }
+                    item = S->ring[rs];
+                    arrive_remote(peer_addr(&S->ite[rs], 0));
+                }
+                if (++rs == RING2) { rs = 0; rphase ^= 1; }
+                if (item < 0) break;
+                const int mt = item / n_tiles, nt = item - mt * n_tiles;
+                const int expert = tiles2[3 * mt];
+                const int row0 = tiles2[3 * mt + 1] + (int)rank * HALF;
+                const int rows = min(HALF, max(0, tiles2[3 * mt + 2] - (int)rank * HALF));
+                const int ab = a_box(rows);
+                const uint32_t a_bytes = rows > 0 ? (uint32_t)(a_box_rows(ab) * BK2 * 2) : 0u;
+                // B rows of this CTA: gate (CTA 0) or up (CTA 1) rows nt*128.. ; down: output columns
+                const int nrow = MODE == 0 ? nt * BNO : nt * BNO + (int)rank * 128;
+                const CUtensorMap *bmap = (MODE == 0 && rank == 1) ? &tmB1 : &tmB0;
+                const bool b_in = nrow < g.N;  // a half entirely past N loads nothing (its columns are masked)
+                const uint32_t b_bytes = b_in ? (uint32_t)B2_BYTES : 0u;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait2(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
+                    const uint32_t fb = peer_addr(&S->full[stage], 0);
+                    if (rank == 0)
+                        mbar_arrive_expect_tx(&S->full[stage], a_bytes + b_bytes);
+                    else
+                        arrive_expect_tx_remote(fb, a_bytes + b_bytes);
+                    if (rows > 0) tma_load_2d_pair(sA + stage * A2_BYTES, &tmA.m[ab], fb, kb * BK2, row0);
+                    if (b_in) tma_load_3d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, nrow, expert);
+                    if (++stage == ST2) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (!ok) record2(g.status, MOE_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t IDESC = idesc_bf16_f32(2 * HALF, BN2);
+            int stage = 0, rs = 0, acc = 0;
+            uint32_t phase = 0, rphase = 0, aphase = 0;
+            bool ok = true;
+            for (;;) {
+                if (!wait2(&S->itf[rs], rphase, g.wait_ns)) { ok = false; break; }
+                const int item = S->ring[rs];
+                mbar_arrive(&S->ite[rs]);
+                if (++rs == RING2) { rs = 0; rphase ^= 1; }
+                if (item < 0) break;
+                if (!wait2(&S->acce[acc], aphase ^ 1, g.wait_ns)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>(acc * BN2);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait2(&S->full[stage], phase, g.wait_ns)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * A2_BYTES);
+                    const uint32_t b0 = smem_u32(sB + stage * B2_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK2 / 16; ++k)
+                        mma_bf16_pair(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), IDESC,
+                                      (kb | k) != 0);
+                    mma_commit_pair(&S->empty[stage]);
+                    if (++stage == ST2) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit_pair(&S->accf[acc]);
+                if (++acc == 2) { acc = 0; aphase ^= 1; }
+            }
+            if (!ok) record2(g.status, MOE_ERR_TIMEOUT);
+            mma_commit_pair(&S->fin);  // once every MMA issued here has completed
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        int rs = 0, acc = 0;
+        uint32_t rphase = 0, aphase = 0;
+        for (;;) {
+            if (!wait2(&S->itf[rs], rphase, g.wait_ns)) { record2(g.status, MOE_ERR_TIMEOUT); break; }
+            const int item = S->ring[rs];
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(&S->ite[rs]);
+                else arrive_remote(peer_addr(&S->ite[rs], 0));
+            }
+            if (++rs == RING2) { rs = 0; rphase ^= 1; }
+            if (item < 0) break;
+            const int mt = item / n_tiles, nt = item - mt * n_tiles;
+            const int row0 = tiles2[3 * mt + 1] + (int)rank * HALF;
+            const int rows = min(HALF, max(0, tiles2[3 * mt + 2] - (int)rank * HALF));
+            const bool row_ok = row < rows;
+            if (!wait2(&S->accf[acc], aphase, g.wait_ns)) { record2(g.status, MOE_ERR_TIMEOUT); break; }
+            tc_fence_after();
+            const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN2);
+            if (MODE == 0) {
+                __nv_bfloat16 *orow = g.out + (size_t)(row0 + row) * g.N;
+#pragma unroll 1
+                for (int c = 0; c < BNO / 32; ++c) {
+                    uint32_t gr[32], ur[32];
+                    tmem_ld32_sync(tb + c * 32, gr);
+                    tmem_ld32_sync(tb + BNO + c * 32, ur);
+                    const int col = nt * BNO + c * 32;
+                    if (row_ok && col < g.N) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float h0 = silu2(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
+                            const float h1 = silu2(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
+                            pk[i] = pack_bf16_2(h0, h1);
+                        }
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            } else {
+                const int flat = row_ok ? g.row_map[row0 + row] : 0;
+                __nv_bfloat16 *orow = g.out + (size_t)flat * g.N;
+#pragma unroll 1
+                for (int c = 0; c < BNO / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32_sync(tb + c * 32, r);
+                    const int col = nt * BNO + c * 32;
+                    if (row_ok && col < g.N) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk[i] = pack_bf16_2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(&S->acce[acc]);
+                else arrive_remote(peer_addr(&S->acce[acc], 0));
+            }
+            if (++acc == 2) { acc = 0; aphase ^= 1; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x + 1] = globaltimer_ns();
+    if (warp == 1) {
+        // every MMA of the pair (which reads this CTA's shared memory and writes its
+        // TMEM) has completed before TMEM is freed and the CTA may leave
+        if (lane == 0 && !wait2(&S->fin, 0)) record2(g.status, MOE_ERR_TIMEOUT);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, TMEM_COLS2);
+    }
+    __syncthreads();
+    // leave only after the other CTA is done with this one (remote arrives, stores)
+    if (threadIdx.x == 0) {
+        arrive_remote(peer_addr(&S->bye, rank ^ 1u));
+        if (!wait2(&S->bye, 0)) record2(g.status, MOE_ERR_TIMEOUT);
+    }
+    __syncthreads();
+}
+
+bool smem2_ready(int mode)
+{
+    static std::mutex mu;
+    static uint64_t done[2] = {0, 0};  // per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lk(mu);
+    if (done[mode] >> dev & 1ull) return true;
+    cudaError_t e = mode == 0 ? cudaFuncSetAttribute(grouped_gemm_2cta_kernel<0>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2)
+                              : cudaFuncSetAttribute(grouped_gemm_2cta_kernel<1>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2);
+    if (e != cudaSuccess) return false;
+    done[mode] |= 1ull << dev;
+    return true;
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm_2cta(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
+                                     const CUtensorMap &tmB1, const int32_t *tiles2, const int32_t *ntiles2,
+                                     cudaStream_t st)
+{
+    int grid = (g.ctas > 0 ? g.ctas : num_sms()) / 2 * 2;
+    if (grid < 2) grid = 2;
+    if (!smem2_ready(g.mode)) return cudaErrorInvalidValue;
+    if (g.mode == 0)
+        return launch_pdl(grouped_gemm_2cta_kernel<0>, dim3(grid), dim3(THREADS2), SMEM2, st, tmA, tmB0, tmB1, g,
+                          tiles2, ntiles2);
+    return launch_pdl(grouped_gemm_2cta_kernel<1>, dim3(grid), dim3(THREADS2), SMEM2, st, tmA, tmB0, tmB1, g, tiles2,
+                      ntiles2);
+}
+
+}  // namespace moe

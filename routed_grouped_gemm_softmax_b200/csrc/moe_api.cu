@@ -21,6 +21,7 @@ namespace {
 std::atomic<int> g_gemm_ctas{0};
 std::atomic<int> g_claim_reverse{0};
 std::atomic<unsigned long long *> g_trace{nullptr};
+std::atomic<int> g_pair_mode{0};  // 0 auto, 1 pair GEMMs whenever possible, 2 never
 std::atomic<int> g_trace_ctas{0};
 std::atomic<unsigned long long> g_wait_ns{0};
 std::atomic<int> g_stall_test{0};
@@ -182,7 +183,8 @@ cudaError_t route_and_permute(const moe_dims_t &d, const moe::WsLayout &L, const
     if (e == cudaSuccess) e = marks.mark(1, st);
     if (e == cudaSuccess)
         e = moe::launch_permute(d, L, idx, at<int32_t>(ws, L.blk_cnt), at<int32_t>(ws, L.blk_base),
-                                at<int32_t>(ws, L.offsets), s2f, at<int32_t>(ws, L.f2s), tiles, ntiles, hdr, st);
+                                at<int32_t>(ws, L.offsets), s2f, at<int32_t>(ws, L.f2s), tiles, ntiles, hdr, st,
+                                at<int32_t>(ws, L.tiles2), at<int32_t>(ws, L.ntiles2));
     return e;
 }
 
@@ -267,6 +269,8 @@ int32_t moe_max_tiles(const moe_dims_t *d)
 void moe_set_gemm_ctas(int32_t ctas) { g_gemm_ctas.store(ctas > 0 ? ctas : 0); }
 
 void moe_set_claim_order(int32_t mode) { g_claim_reverse.store(mode < 0 ? 0 : mode > 3 ? 3 : mode); }
+
+void moe_set_pair_mma(int32_t mode) { g_pair_mode.store(mode < 0 || mode > 2 ? 0 : mode); }
 
 void moe_set_gemm_trace(unsigned long long *trace, int32_t ctas)
 {
@@ -353,11 +357,16 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
 
     moe::AMaps tm_xs, tm_h;
     CUtensorMap tm_wg, tm_wu, tm_wd;
+    // pair-of-CTA GEMMs for groups large enough to be compute-bound (on average at
+    // least 512 rows per expert), on the queue's claim modes
+    const int pair_mode = g_pair_mode.load();
+    const bool pairs = pair_mode != 2 && g_claim_reverse.load() <= 1 && !moe::small_route_permute_ok(*d) &&
+                       (pair_mode == 1 || (long)A >= 512L * d->E);
     if (!moe::encode_a_maps(&tm_xs, xs, A, d->H, false) ||
         !encode_3d(&tm_wg, w_gate, d->E, d->I, d->H, 128) ||
         !encode_3d(&tm_wu, w_up, d->E, d->I, d->H, 128) ||
         !moe::encode_a_maps(&tm_h, h, A, d->I, false) ||
-        !encode_3d(&tm_wd, w_down, d->E, d->H, d->I, 256))
+        !encode_3d(&tm_wd, w_down, d->E, d->H, d->I, pairs ? 128 : 256))
         return MOE_ERR_CUDA;
 
     const StageMarks marks;
@@ -377,7 +386,9 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
     if (e == cudaSuccess) {
         moe::GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, h, nullptr, ctas, rev, wait_ns, stall};
         g1.trace = trace1;
-        e = moe::launch_grouped_gemm(g1, tm_xs, tm_wg, tm_wu, st);
+        e = pairs ? moe::launch_grouped_gemm_2cta(g1, tm_xs, tm_wg, tm_wu, at<int32_t>(ws, L.tiles2),
+                                                  at<int32_t>(ws, L.ntiles2), st)
+                  : moe::launch_grouped_gemm(g1, tm_xs, tm_wg, tm_wu, st);
     }
     if (e == cudaSuccess) e = marks.mark(3, st);
     if (e == cudaSuccess) {
@@ -385,7 +396,9 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
                          stall, 0, nullptr, gate, fused ? at<int32_t>(ws, L.ccnt) : nullptr,
                          static_cast<__nv_bfloat16 *>(out), d->top_k, d->top_k};
         g2.trace = trace2;
-        e = moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st);
+        e = pairs ? moe::launch_grouped_gemm_2cta(g2, tm_h, tm_wd, tm_wd, at<int32_t>(ws, L.tiles2),
+                                                  at<int32_t>(ws, L.ntiles2), st)
+                  : moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st);
     }
     if (e == cudaSuccess) e = marks.mark(4, st);
     if (e == cudaSuccess && !fused)

@@ -24,7 +24,7 @@ struct WsHeader {
 
 // Byte offsets of every region of the workspace (256-byte aligned each).
 struct WsLayout {
-    size_t ccnt, clear_bytes, logits, wrt, wsq, rncand, rlist, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, xq, xq_s, xs, xs_s, h, h_s, y,
+    size_t ccnt, clear_bytes, logits, wrt, wsq, rncand, rlist, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, tiles2, ntiles2, xq, xq_s, xs, xs_s, h, h_s, y,
         total;
     int nb;      // permutation chunks
     int chunk;   // flat entries per chunk
@@ -79,6 +79,8 @@ inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
     L.f2s = take(A * 4);
     L.tiles = take(max_tiles * 3 * 4);
     L.ntiles = take(4);
+    L.tiles2 = take(((A + 2 * kTileRows - 1) / (2 * kTileRows) + (A < (size_t)d.E ? A : (size_t)d.E)) * 3 * 4);
+    L.ntiles2 = take(4);
     L.xq = take(fp8 ? static_cast<size_t>(d.T) * d.H : 0);  // fp8: x quantised once per token
     L.xq_s = take(fp8 ? static_cast<size_t>(d.T) * (d.H / 128) * 4 : 0);
     L.xs = take(A * d.H * (fp8 ? 1 : 2));
@@ -127,10 +129,11 @@ cudaError_t launch_route_permute_small(const moe_dims_t &d, const __nv_bfloat16 
                                        int32_t *offsets, int32_t *s2f, int32_t *f2s, int32_t *tiles,
                                        int32_t *ntiles, WsHeader *hdr, int32_t *ccnt, int nccnt, cudaStream_t st);
 
+// Also writes the 2 x 128-row pair tiles when tiles2 is non-null.
 cudaError_t launch_permute(const moe_dims_t &d, const WsLayout &L, const int32_t *idx,
                            int32_t *blk_cnt, int32_t *blk_base, int32_t *offsets, int32_t *s2f,
                            int32_t *f2s, int32_t *tiles, int32_t *ntiles, WsHeader *hdr,
-                           cudaStream_t st);
+                           cudaStream_t st, int32_t *tiles2 = nullptr, int32_t *ntiles2 = nullptr);
 
 cudaError_t launch_gather_rows(const __nv_bfloat16 *x, const int32_t *s2f, int A, int H, int top_k,
                                __nv_bfloat16 *xs, cudaStream_t st);
@@ -177,6 +180,12 @@ struct GemmArgs {
 // mode 2: out_f32 = A B^T over M rows (one "expert"), the router's tensor-core logits.
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                 const CUtensorMap &tmB1, cudaStream_t st);
+
+// The bf16 grouped GEMMs (modes 0 and 1) on CTA pairs, cta_group::2 MMAs over the
+// 2 x 128-row pair tiles tiles2 (grouped_gemm_2cta.cu); queue claim modes only.
+cudaError_t launch_grouped_gemm_2cta(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
+                                     const CUtensorMap &tmB1, const int32_t *tiles2, const int32_t *ntiles2,
+                                     cudaStream_t st);
 
 // FP8 block-scaled grouped GEMMs (fp8.cu).  mode 0: h codes/scales from
 // silu(A Wg^T) * (A Wu^T); mode 1: y[row_map[row]] = A Wd^T in bf16; mode 2:

@@ -80,7 +80,8 @@ __device__ int block_exclusive_scan(int v, int *warp_tot, int &total)
 __global__ void __launch_bounds__(1024)
 perm_scan_kernel(int E, int nb, const int32_t *__restrict__ blk_cnt, int32_t *__restrict__ blk_base,
                  int32_t *__restrict__ offsets, int32_t *__restrict__ tiles,
-                 int32_t *__restrict__ ntiles, int32_t *counters, int ncounters)
+                 int32_t *__restrict__ ntiles, int32_t *counters, int ncounters, int32_t *__restrict__ tiles2,
+                 int32_t *__restrict__ ntiles2)
 {
     pdl_wait();
     pdl_trigger();
@@ -98,6 +99,17 @@ perm_scan_kernel(int E, int nb, const int32_t *__restrict__ blk_cnt, int32_t *__
     const int off = block_exclusive_scan(cnt, warp_tot, total_rows);
     const int nt = (cnt + kTileRows - 1) / kTileRows;
     const int tstart = block_exclusive_scan(nt, warp_tot, total_tiles);
+    // pair tiles of 2 x 128 rows for the 2-CTA GEMMs (optional)
+    int total_pairs = 0;
+    const int np = (cnt + 2 * kTileRows - 1) / (2 * kTileRows);
+    const int pstart = tiles2 ? block_exclusive_scan(np, warp_tot, total_pairs) : 0;
+    if (tiles2 && e < E)
+        for (int m = 0; m < np; ++m) {
+            int32_t *tl = tiles2 + 3 * (size_t)(pstart + m);
+            tl[0] = e;
+            tl[1] = off + m * 2 * kTileRows;
+            tl[2] = min(2 * kTileRows, cnt - m * 2 * kTileRows);
+        }
     if (e < E) {
         offsets[e] = off;
         for (int b = 0; b < nb; ++b) blk_base[(size_t)b * E + e] += off;
@@ -111,6 +123,7 @@ perm_scan_kernel(int E, int nb, const int32_t *__restrict__ blk_cnt, int32_t *__
     if (threadIdx.x == 0) {
         offsets[E] = total_rows;
         *ntiles = total_tiles;
+        if (ntiles2) *ntiles2 = total_pairs;
     }
     if (counters && threadIdx.x < ncounters) counters[threadIdx.x] = 0;
 }
@@ -162,14 +175,14 @@ __global__ void gather_rows_kernel(const __nv_bfloat16 *__restrict__ x,
 cudaError_t launch_permute(const moe_dims_t &d, const WsLayout &L, const int32_t *idx,
                            int32_t *blk_cnt, int32_t *blk_base, int32_t *offsets, int32_t *s2f,
                            int32_t *f2s, int32_t *tiles, int32_t *ntiles, WsHeader *hdr,
-                           cudaStream_t st)
+                           cudaStream_t st, int32_t *tiles2, int32_t *ntiles2)
 {
     const int A = d.T * d.top_k, E = d.E;
     cudaError_t e = launch_pdl(perm_count_kernel, dim3(L.nb), dim3(256), E * sizeof(int), st, idx, A, E, L.chunk,
                                blk_cnt, hdr ? &hdr->status : nullptr);
     if (e == cudaSuccess)
         e = launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, st, E, L.nb, blk_cnt, blk_base, offsets, tiles,
-                       ntiles, hdr ? hdr->counter : nullptr, hdr ? 7 : 0);
+                       ntiles, hdr ? hdr->counter : nullptr, hdr ? 7 : 0, tiles2, ntiles2);
     if (e == cudaSuccess)
         e = launch_pdl(perm_scatter_kernel, dim3(L.nb), dim3(L.chunk), (size_t)(L.chunk / 32) * E * sizeof(int), st,
                        idx, A, E, blk_base, s2f, f2s);

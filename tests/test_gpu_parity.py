@@ -134,6 +134,41 @@ def test_schedule_independence(T):
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
 
 
+PAIR_CASES = {
+    "ragged": SMALL["ragged"],            # ~75 rows per expert: pair tiles with an empty second half
+    "ragged_bias": SMALL["ragged_bias"],  # H = 320: a down n-tile whose second half lies past H
+    "deep": CONFIGS["tiny"].replace(name="deep", T=2048, H=256, E=4, top_k=2, I=256, seed=25),  # full pairs
+}
+
+
+@pytest.mark.parametrize("name", list(PAIR_CASES))
+def test_pair_cta_gemms(name):
+    # The pair-of-CTA GEMMs (cta_group::2) against the oracle, and bitwise stable
+    # across grid sizes and claim orders.
+    cfg = PAIR_CASES[name]
+    g, c = device_inputs(cfg)
+    k = cfg.top_k
+    outs = []
+    try:
+        api.set_pair_mma("always")
+        for ctas, rev in [(0, False), (2, False), (0, True), (10, True)]:
+            api.set_gemm_ctas(ctas)
+            api.set_claim_order(rev)
+            ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, "cuda")
+            outs.append(api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k,
+                                        ws=ws).clone())
+            assert api.moe_get_device_status(ws) == api.MOE_OK
+    finally:
+        api.set_pair_mma("auto")
+        api.set_gemm_ctas(0)
+        api.set_claim_order(False)
+    idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], k)
+    ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"])
+    compare_out(outs[0], ref, f"{name} pair GEMMs")
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
 def test_repeat_calls_same_workspace():
     # Counters and status are reset by the calls themselves: back-to-back calls on one
     # workspace give identical results (graph-replay style reuse).
