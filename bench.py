@@ -119,8 +119,9 @@ def load_peaks():
 
 STAGE_SOURCES = {
     "route": ["route.cu", "route_certified.cu", "route_common.cuh", "fp8.cu", "sm100_ptx.cuh", "moe_internal.h"],
-    "gemm_gate_up": ["grouped_gemm.cu", "fp8.cu", "sm100_ptx.cuh", "moe_internal.h"],
-    "gemm_down": ["grouped_gemm.cu", "fp8.cu", "combine.cuh", "sm100_ptx.cuh", "moe_internal.h"],
+    "gemm_gate_up": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "sm100_ptx.cuh", "moe_internal.h"],
+    "gemm_down": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "combine.cuh", "sm100_ptx.cuh",
+                  "moe_internal.h"],
     "combine": ["combine.cu", "combine.cuh"],
 }
 
