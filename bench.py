@@ -89,6 +89,8 @@ def parse():
                         "split of the items or of the experts (ablations)")
     p.add_argument("--pair", default="auto", choices=["auto", "always", "never"],
                    help="the bf16 GEMMs on CTA pairs (tcgen05 cta_group::2): automatic choice or forced")
+    p.add_argument("--swap-ab", default="auto", choices=["auto", "always", "never"],
+                   help="the fp8 gate/up GEMM with swapped MMA operands: automatic choice or forced")
     p.add_argument("--shape", default="",
                    help="override config fields, e.g. T=1024,E=64 (reduced cases for profiler captures)")
     return p.parse_args()
@@ -118,10 +120,12 @@ def load_peaks():
 
 
 STAGE_SOURCES = {
-    "route": ["route.cu", "route_certified.cu", "route_common.cuh", "fp8.cu", "sm100_ptx.cuh", "moe_internal.h"],
-    "gemm_gate_up": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "sm100_ptx.cuh", "moe_internal.h"],
-    "gemm_down": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "combine.cuh", "sm100_ptx.cuh",
-                  "moe_internal.h"],
+    "route": ["route.cu", "route_certified.cu", "route_common.cuh", "fp8.cu", "fp8_common.cuh", "sm100_ptx.cuh",
+              "moe_internal.h"],
+    "gemm_gate_up": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "fp8_swapab.cu", "fp8_common.cuh",
+                     "sm100_ptx.cuh", "moe_internal.h"],
+    "gemm_down": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "fp8_common.cuh", "combine.cuh",
+                  "sm100_ptx.cuh", "moe_internal.h"],
     "combine": ["combine.cu", "combine.cuh"],
 }
 
@@ -454,6 +458,7 @@ def main():
             e.record(stream)
     api.set_claim_order(False if args.schedule == "queue" else args.schedule)
     api.set_pair_mma(args.pair)
+    api.set_fp8_swap_ab(args.swap_ab)
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
         step()

@@ -194,6 +194,15 @@ void moe_set_claim_order(int32_t mode);
  * independent of it.  Process-wide. */
 void moe_set_pair_mma(int32_t mode);
 
+/* The fp8 forward's gate/up GEMM with the MMA operands' roles swapped: 128 weight
+ * rows on the MMA's M side and the expert group's token rows, rounded up to 16,
+ * on its N side, so the tensor work and the per-K-block promotion follow the
+ * group's size instead of a 128-row tile.  0 = automatic (used when the batch
+ * averages at most 64 rows per expert), 1 = always (tests), 2 = never.  Both
+ * forms compute the same blockwise-scaled sums; the output stays within the fp8
+ * layer's tolerance either way.  Process-wide. */
+void moe_set_fp8_swap_ab(int32_t mode);
+
 /* Scheduling trace for benchmarks.  With `trace` a device buffer of 4 * ctas
  * uint64 values (ctas >= the GEMM grid, 148 by default), every later forward
  * records per GEMM CTA the %globaltimer (ns) when it started work and when it

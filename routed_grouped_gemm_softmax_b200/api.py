@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 8: "MOE_ERR_ROUTER_BOUND"}
 EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "moe_forward",
            "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order", "moe_set_gemm_trace",
-           "moe_set_pair_mma",
+           "moe_set_pair_mma", "moe_set_fp8_swap_ab",
            "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",
            "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets"]
 DTYPE_BF16, DTYPE_FP8 = 0, 1
@@ -73,6 +73,8 @@ def lib():
         L.moe_set_gemm_trace.restype = None
         L.moe_set_pair_mma.argtypes = [I32]
         L.moe_set_pair_mma.restype = None
+        L.moe_set_fp8_swap_ab.argtypes = [I32]
+        L.moe_set_fp8_swap_ab.restype = None
         L.moe_set_stage_events.argtypes = [P, I32]
         L.moe_set_stage_events.restype = None
         L.moe_forward_fp8.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -303,6 +305,11 @@ def set_claim_order(reverse):
 def set_pair_mma(mode: str):
     """"auto" (default), "always" or "never": the bf16 forward's pair-of-CTA GEMMs."""
     lib().moe_set_pair_mma({"auto": 0, "always": 1, "never": 2}[mode])
+
+
+def set_fp8_swap_ab(mode: str):
+    """"auto" (default), "always" or "never": the fp8 gate/up GEMM with swapped MMA operands."""
+    lib().moe_set_fp8_swap_ab({"auto": 0, "always": 1, "never": 2}[mode])
 
 
 def set_gemm_trace(buf):

@@ -22,6 +22,7 @@ std::atomic<int> g_gemm_ctas{0};
 std::atomic<int> g_claim_reverse{0};
 std::atomic<unsigned long long *> g_trace{nullptr};
 std::atomic<int> g_pair_mode{0};  // 0 auto, 1 pair GEMMs whenever possible, 2 never
+std::atomic<int> g_fp8_swap{0};   // 0 auto, 1 swapped fp8 gate/up GEMM always, 2 never
 std::atomic<int> g_trace_ctas{0};
 std::atomic<unsigned long long> g_wait_ns{0};
 std::atomic<int> g_stall_test{0};
@@ -271,6 +272,7 @@ void moe_set_gemm_ctas(int32_t ctas) { g_gemm_ctas.store(ctas > 0 ? ctas : 0); }
 void moe_set_claim_order(int32_t mode) { g_claim_reverse.store(mode < 0 ? 0 : mode > 3 ? 3 : mode); }
 
 void moe_set_pair_mma(int32_t mode) { g_pair_mode.store(mode < 0 || mode > 2 ? 0 : mode); }
+void moe_set_fp8_swap_ab(int32_t mode) { g_fp8_swap.store(mode < 0 || mode > 2 ? 0 : mode); }
 
 void moe_set_gemm_trace(unsigned long long *trace, int32_t ctas)
 {
@@ -477,7 +479,11 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
         moe::Fp8GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, xs_s, w_gate_s, w_up_s,
                             h, h_s, nullptr, nullptr, ctas, rev, wait_ns, stall};
         g1.trace = trace1;
-        e = moe::launch_grouped_gemm_fp8(g1, tm_xs, tm_wg, tm_wu, st);
+        // operands swapped when the groups average at most 64 rows per expert
+        const int sw = g_fp8_swap.load();
+        const bool swap = sw == 1 || (sw == 0 && (long)A <= 64L * d->E);
+        e = swap ? moe::launch_grouped_gemm_fp8_swapab(g1, tm_xs, tm_wg, tm_wu, st)
+                 : moe::launch_grouped_gemm_fp8(g1, tm_xs, tm_wg, tm_wu, st);
     }
     if (e == cudaSuccess) e = marks.mark(3, st);
     if (e == cudaSuccess) {

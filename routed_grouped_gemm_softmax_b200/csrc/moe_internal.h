@@ -220,6 +220,11 @@ struct Fp8GemmArgs {
 };
 cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                     const CUtensorMap &tmB1, cudaStream_t st);
+// The fp8 gate/up GEMM (mode 0 only) with the MMA operands swapped: 128 weight rows
+// on the M side, the tile's token rows (rounded up to 16) on the N side
+// (fp8_swapab.cu); for expert groups much shorter than a 128-row tile.
+cudaError_t launch_grouped_gemm_fp8_swapab(const Fp8GemmArgs &g, const AMaps &tmX, const CUtensorMap &tmWg,
+                                           const CUtensorMap &tmWu, cudaStream_t st);
 cudaError_t launch_quantize_rows(const __nv_bfloat16 *src, const int32_t *map, int k, int R, int K, uint8_t *q,
                                  float *s, cudaStream_t st);
 // fp8 rows into expert order: xs[r] = xq[s2f[r] / k] (K codes) and xs_s[r] = xq_s[...] (K/128 scales).

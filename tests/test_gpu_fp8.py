@@ -111,3 +111,42 @@ def test_fp8_full_size_sampled():
     compare_routing(i_g, w_g, idx, gate, "fp8")
     r = rel_l2(out[torch.as_tensor(tok, device="cuda").long()], ref)
     assert r <= FP8_REL_L2, f"fp8 full size: rel_l2={r:.3e}"
+
+
+SWAP_CASES = {
+    "ragged": SMALL["fp8_ragged"],   # ~38 rows per expert: 48-row MMAs, partial chunks
+    "bias": SMALL["fp8_bias"],       # skewed groups: 16- to 128-row tiles in one launch
+    "full_tiles": SMALL["fp8_small"].replace(name="fp8_full_tiles", T=300, top_k=3, seed=9),  # zero router below
+    "k_chunks": CONFIGS["fp8"].replace(name="fp8_k_chunks", T=96, H=2304, E=8, top_k=2, I=256, seed=11),  # 18 K blocks
+}
+
+
+@pytest.mark.parametrize("name", list(SWAP_CASES))
+def test_fp8_swapped_gate_up_gemm(name):
+    # The gate/up GEMM with swapped MMA operands (weights on M, token rows on N)
+    # against the oracle and against the one-CTA fp8 kernel, and bitwise stable
+    # across grid sizes and claim orders.
+    cfg = SWAP_CASES[name]
+    inp, w = _fp8_case(cfg)
+    if name == "full_tiles":
+        inp.router_w = torch.zeros_like(inp.router_w)   # 300 rows on each of experts 0-2
+    outs = []
+    try:
+        api.set_fp8_swap_ab("never")
+        base = _run_fp8(cfg, inp, w).clone()
+        api.set_fp8_swap_ab("always")
+        for ctas, mode in [(0, False), (3, True), (0, "static_items"), (7, "static_experts")]:
+            api.set_gemm_ctas(ctas)
+            api.set_claim_order(mode)
+            outs.append(_run_fp8(cfg, inp, w).clone())
+    finally:
+        api.set_fp8_swap_ab("auto")
+        api.set_gemm_ctas(0)
+        api.set_claim_order(False)
+    ref, _, _ = _oracle_fp8(cfg, inp, w)
+    assert rel_l2(outs[0], ref) <= FP8_REL_L2, f"{name} swapped: rel_l2={rel_l2(outs[0], ref):.3e}"
+    assert rel_l2(base, ref) <= FP8_REL_L2, f"{name} one-CTA: rel_l2={rel_l2(base, ref):.3e}"
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    # same blockwise products and the same fp32 promotion, SwiGLU and quantiser
+    assert torch.equal(outs[0].view(torch.int16), base.view(torch.int16))
