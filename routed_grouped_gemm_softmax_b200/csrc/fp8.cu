@@ -184,7 +184,11 @@ grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    pdl_wait();  // the prologue above overlapped the previous kernel
+    // The prologue above overlapped the previous kernel.  Modes 0 and 1: warp 0 waits
+    // for it inside the producer, after the first stages' weight loads (mode 2's B
+    // operand is the previous kernel's output).
+    constexpr bool kEarlyB = MODE != 2;
+    if (!(kEarlyB && warp == 0)) pdl_wait();
     pdl_trigger();
     if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
@@ -196,6 +200,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant
             uint32_t phase = 0, rphase = 0, armed = 0, armed_par = 0;
             bool ok = true;
             int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
+            bool held = kEarlyB;  // A loads of the first item's first stages wait for the previous kernel
             for (;;) {
                 const int item = claim_item(g.reverse, g.counter, total, n_tiles * ksplit, dense ? nullptr : g.tiles, cursor);
                 if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
@@ -216,10 +221,16 @@ grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     uint8_t *b_dst = sB + stage * B_BYTES;
-                    tma_load_2d(sA + stage * A_BYTES, &tmA.m[ab], &S->full[stage], kb * KEL, row0);
+                    if (!held) tma_load_2d(sA + stage * A_BYTES, &tmA.m[ab], &S->full[stage], kb * KEL, row0);
                     tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * KEL, n0, expert);
                     if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * KEL, n0, expert);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (held && kb + 1 - kb0 == min(STAGES, kb1 - kb0)) {  // first item: stage j holds its K block kb0 + j
+                        pdl_wait();
+                        held = false;
+                        for (int j = 0; j <= kb - kb0; ++j)
+                            tma_load_2d(sA + j * A_BYTES, &tmA.m[ab], &S->full[j], (kb0 + j) * KEL, row0);
+                    }
                 }
                 if (!ok) break;
             }

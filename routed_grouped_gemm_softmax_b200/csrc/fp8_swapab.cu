@@ -132,7 +132,10 @@ grouped_gemm_fp8_swapab_kernel(const __grid_constant__ AMaps tmX, const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    pdl_wait();  // the prologue above overlapped the previous kernel
+    // The prologue above overlapped the previous kernel; warp 0 waits for it inside the
+    // producer, after the first stages' weight loads (only the activation rows are the
+    // previous kernel's output).
+    if (warp != 0) pdl_wait();
     pdl_trigger();
     if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
@@ -144,6 +147,7 @@ grouped_gemm_fp8_swapab_kernel(const __grid_constant__ AMaps tmX, const __grid_c
             uint32_t phase = 0, rphase = 0, armed = 0, armed_par = 0;
             bool ok = true;
             int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
+            bool held = true;  // activation loads of the first item's first stages wait for the previous kernel
             for (;;) {
                 const int item = claim_item(g.reverse, g.counter, total, 2 * n_tiles, g.tiles, cursor);
                 if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
@@ -161,10 +165,16 @@ grouped_gemm_fp8_swapab_kernel(const __grid_constant__ AMaps tmX, const __grid_c
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     uint8_t *w_dst = sW + stage * W_BYTES;
-                    tma_load_2d(sX + stage * X_BYTES, &tmX.m[xb], &S->full[stage], kb * KBYTES, it.row0);
+                    if (!held) tma_load_2d(sX + stage * X_BYTES, &tmX.m[xb], &S->full[stage], kb * KBYTES, it.row0);
                     tma_load_3d(w_dst, &tmWg, &S->full[stage], kb * KBYTES, n0, it.expert);
                     tma_load_3d(w_dst + W_BYTES / 2, &tmWu, &S->full[stage], kb * KBYTES, n0, it.expert);
                     if (++stage == SST) { stage = 0; phase ^= 1; }
+                    if (held && kb + 1 == min(SST, KB)) {  // first item: stage j holds K block j
+                        pdl_wait();
+                        held = false;
+                        for (int j = 0; j <= kb; ++j)
+                            tma_load_2d(sX + j * X_BYTES, &tmX.m[xb], &S->full[j], j * KBYTES, it.row0);
+                    }
                 }
                 if (!ok) break;
             }

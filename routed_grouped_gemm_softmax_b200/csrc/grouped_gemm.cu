@@ -124,7 +124,11 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    pdl_wait();  // the prologue above overlapped the previous kernel
+    // The prologue above overlapped the previous kernel.  Modes 0 and 1: warp 0 waits
+    // for it inside the producer, after the first stages' weight loads (the weights
+    // are the layer's inputs; only the A rows are the previous kernel's output).
+    constexpr bool kEarlyB = MODE != 2;
+    if (!(kEarlyB && warp == 0)) pdl_wait();
     pdl_trigger();
     if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
@@ -137,6 +141,7 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
             uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
             bool ok = true;
             int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
+            bool held = kEarlyB;  // A loads of the first item's first stages wait for the previous kernel
             for (;;) {
                 const int item = claim_item(g.reverse, g.counter, total, n_tiles, dense ? nullptr : g.tiles, cursor);
                 if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
@@ -154,12 +159,17 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                     mbar_arrive_expect_tx(&S->full[stage], a_box_rows(ab) * BK * 2 + B_BYTES);
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-                    uint8_t *a_dst = sA + stage * A_BYTES;
                     uint8_t *b_dst = sB + stage * B_BYTES;
-                    tma_load_2d(a_dst, &tmA.m[ab], &S->full[stage], kb * BK, row0);
+                    if (!held) tma_load_2d(sA + stage * A_BYTES, &tmA.m[ab], &S->full[stage], kb * BK, row0);
                     tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
                     if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (held && kb + 1 == min(STAGES, num_kb)) {  // first item: stage j holds K block j
+                        pdl_wait();
+                        held = false;
+                        for (int j = 0; j <= kb; ++j)
+                            tma_load_2d(sA + j * A_BYTES, &tmA.m[ab], &S->full[j], j * BK, row0);
+                    }
                 }
                 if (!ok) break;
             }

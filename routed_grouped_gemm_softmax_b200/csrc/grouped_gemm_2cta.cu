@@ -213,7 +213,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
     cluster_sync();  // both CTAs' barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    pdl_wait();
+    // The prologue above overlapped the previous kernel; warp 0 waits for it inside the
+    // producer, after the first stages' weight loads (only the A rows are the previous
+    // kernel's output).
+    if (warp != 0) pdl_wait();
     pdl_trigger();
     if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
@@ -224,6 +227,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
             int stage = 0, rs = 0, cursor = 0;
             uint32_t phase = 0, rphase = 0;
             bool ok = true;
+            bool held = true;  // A loads of the first item's first stages wait for the previous kernel
             for (;;) {
                 int item;
                 if (rank == 0) {
@@ -258,9 +262,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                         mbar_arrive_expect_tx(&S->full[stage], a_bytes + b_bytes);
                     else
                         arrive_expect_tx_remote(fb, a_bytes + b_bytes);
-                    if (rows > 0) tma_load_2d_pair(sA + stage * A2_BYTES, &tmA.m[ab], fb, kb * BK2, row0);
+                    if (rows > 0 && !held) tma_load_2d_pair(sA + stage * A2_BYTES, &tmA.m[ab], fb, kb * BK2, row0);
                     if (b_in) tma_load_3d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, nrow, expert);
                     if (++stage == ST2) { stage = 0; phase ^= 1; }
+                    if (held && kb + 1 == min(ST2, num_kb)) {  // first item: stage j holds K block j
+                        pdl_wait();
+                        held = false;
+                        if (rows > 0)
+                            for (int j = 0; j <= kb; ++j)
+                                tma_load_2d_pair(sA + j * A2_BYTES, &tmA.m[ab], peer_addr(&S->full[j], 0), j * BK2,
+                                                 row0);
+                    }
                 }
                 if (!ok) break;
             }
