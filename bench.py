@@ -215,16 +215,31 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+def rank_env():
+    """(world size, rank, local rank) from the launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU: the process group the replicas use for their barrier and
+    the max over ranks (NCCL on the GPUs; gloo for the CPU tests of this logic)."""
+    world, rank, local = rank_env()
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=_dt.timedelta(seconds=60))
     return world, rank, local
+
+
+def dist_teardown(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 def barrier(world):
@@ -237,9 +252,14 @@ def max_over_ranks(v: float, world: int) -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def throughput(tokens_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job tokens/s: the tokens every replica processed over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (total_ms * 1e-3)
 
 
 # ----------------------------------------------------------- per-stage bytes
@@ -408,11 +428,13 @@ def config_block(cfg, world):
 
 def main():
     args = parse()
-    world, rank, local = dist_setup(args)
     if args.impl == "reference":
+        # rank 0 alone times the oracle on the host cores; the other ranks have no work
+        # and open no process group
+        world, rank, _ = rank_env()
         run_reference(args, world, rank)
-        barrier(world)
         return
+    world, rank, local = dist_setup()
     from routed_grouped_gemm_softmax_b200 import api
 
     cfg = workload_config(args)
@@ -520,7 +542,7 @@ def main():
                 for j, name in enumerate(api.STAGES)}
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
-    value = cfg.T * world * args.steps / (total_ms * 1e-3)
+    value = throughput(cfg.T, world, args.steps, total_ms)
 
     # routing of this workload (for the touched-expert weight bytes)
     idx, _ = api.moe_route(x, rw, bias, k)
@@ -555,7 +577,7 @@ def main():
             b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in pairs), world) / n_e2e
-        e2e = {"value": round(cfg.T * world / (e2e_ms * 1e-3), 3), "unit": "tokens/s",
+        e2e = {"value": round(throughput(cfg.T, world, 1, e2e_ms), 3), "unit": "tokens/s",
                "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
                "ms_per_step": round(e2e_ms, 4)}
 
@@ -575,9 +597,7 @@ def main():
                 "clocks": clocks, "cpu_baseline": cpu,
                 "p99_ms_per_step": round(sorted(step_ms)[min(len(step_ms) - 1, math.ceil(0.99 * len(step_ms)) - 1)], 5)}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    dist_teardown(world)
 
 
 if __name__ == "__main__":
