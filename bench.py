@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import torch
@@ -156,23 +157,56 @@ def recorded_traffic(workload: str, stage: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 50 ms in the background."""
+    """SM clock and clock-event (throttle) reasons of this GPU while the timed region
+    runs: NVML polled every 2 ms from a background thread (the timed region can be a
+    few milliseconds long), or nvidia-smi every 50 ms where NVML is missing.  Reads
+    only; changes no setting."""
     Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device: int):
         self.proc = None
         self.lines = []
+        self.samples = []  # NVML: (unix time, SM MHz, reason bitmask)
+        self.nv = self.handle = self.thread = None
+        self.max_mhz = None
+        self.stop_flag = threading.Event()
         try:
             p = torch.cuda.get_device_properties(device)
-            target = ["-i", f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"]
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
         except Exception:
-            target = []
+            bus = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.handle = (pynvml.nvmlDeviceGetHandleByPciBusId(bus) if bus else
+                           pynvml.nvmlDeviceGetHandleByIndex(device))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self.nv = pynvml
+            self.bits = (pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                         pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap)
+        except Exception:
+            self.nv = self.handle = None
         self.cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                    "-lms", "50", *target]
+                    "-lms", "50", *(["-i", bus] if bus else [])]
+
+    def _poll(self):
+        nv, h = self.nv, self.handle
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append((time.time(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                     int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def start(self):
+        if self.nv is not None:
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
@@ -180,6 +214,10 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            return
         if self.proc is None:
             return
         self.proc.terminate()
@@ -191,8 +229,14 @@ class ClockSampler:
         self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
     def summary(self, t0: float, t1: float):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], self.max_mhz, set()
+        if self.thread is not None:
+            for ts, mhz, bits in self.samples:
+                if t0 <= ts <= t1:
+                    sm.append(mhz)
+                    reasons.update(n for n, b in zip(self.NAMES, self.bits) if bits & b)
+            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                    "reasons": sorted(reasons), "samples": len(sm), "source": "nvml, 2 ms"}
         for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
@@ -208,11 +252,11 @@ class ClockSampler:
                 mx = float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(self.NAMES, f[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 50 ms"}
 
 
 def rank_env():
