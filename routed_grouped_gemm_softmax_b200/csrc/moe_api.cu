@@ -378,7 +378,8 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
         e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);          // header + combine counts
     if (e == cudaSuccess) e = route_and_permute(*d, L, x, router_w, router_bias, ws, hdr, marks, st);
     if (e == cudaSuccess)
-        e = moe::launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), s2f, A, d->H, d->top_k, xs, st);
+        e = moe::launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), at<int32_t>(ws, L.f2s), d->T, d->H,
+                                    d->top_k, xs, st);
     if (e == cudaSuccess) e = marks.mark(2, st);
     const int ctas = g_gemm_ctas.load(), rev = g_claim_reverse.load();
     unsigned long long *trace1 = g_trace.load(), *trace2 = trace1 ? trace1 + 2 * g_trace_ctas.load() : nullptr;

@@ -135,7 +135,8 @@ cudaError_t launch_permute(const moe_dims_t &d, const WsLayout &L, const int32_t
                            int32_t *f2s, int32_t *tiles, int32_t *ntiles, WsHeader *hdr,
                            cudaStream_t st, int32_t *tiles2 = nullptr, int32_t *ntiles2 = nullptr);
 
-cudaError_t launch_gather_rows(const __nv_bfloat16 *x, const int32_t *s2f, int A, int H, int top_k,
+// xs[f2s[f]] = x[f / k] for every assignment f = t*k + j (a warp per assignment, flat order).
+cudaError_t launch_gather_rows(const __nv_bfloat16 *x, const int32_t *f2s, int T, int H, int top_k,
                                __nv_bfloat16 *xs, cudaStream_t st);
 
 

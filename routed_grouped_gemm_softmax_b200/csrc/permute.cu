@@ -155,18 +155,24 @@ __global__ void perm_scatter_kernel(const int32_t *__restrict__ idx, int A, int 
     f2s[f] = pos;
 }
 
+// x rows into expert-sorted order, a warp per assignment in flat order: warp f
+// copies x[f / k] to xs[f2s[f]].  The k copies of a token are made by neighbouring
+// warps, close in time, so x is read from DRAM about once; walking the sorted rows
+// instead reads each x row k times far apart, and the copy's own write stream evicts
+// x from L2 in between.
 __global__ void gather_rows_kernel(const __nv_bfloat16 *__restrict__ x,
-                                   const int32_t *__restrict__ s2f, int A, int H, int k,
+                                   const int32_t *__restrict__ f2s, int A, int H, int k,
                                    __nv_bfloat16 *__restrict__ xs)
 {
     pdl_wait();
     pdl_trigger();
-    const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int f = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    if (row >= A) return;
-    const int t = s2f[row] / k;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
-    uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)row * H);
+    if (f >= A) return;
+    const int pos = f2s[f];
+    if ((unsigned)pos >= (unsigned)A) return;  // never outside xs
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(f / k) * H);
+    uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)pos * H);
     for (int c = lane; c < H / 8; c += 32) dst[c] = src[c];
 }
 
@@ -189,12 +195,12 @@ cudaError_t launch_permute(const moe_dims_t &d, const WsLayout &L, const int32_t
     return e;
 }
 
-cudaError_t launch_gather_rows(const __nv_bfloat16 *x, const int32_t *s2f, int A, int H, int top_k,
+cudaError_t launch_gather_rows(const __nv_bfloat16 *x, const int32_t *f2s, int T, int H, int top_k,
                                __nv_bfloat16 *xs, cudaStream_t st)
 {
-    const int rows_per_block = 8;
+    const int A = T * top_k, rows_per_block = 8;
     return launch_pdl(gather_rows_kernel, dim3((A + rows_per_block - 1) / rows_per_block), dim3(rows_per_block * 32),
-                      0, st, x, s2f, A, H, top_k, xs);
+                      0, st, x, f2s, A, H, top_k, xs);
 }
 
 }  // namespace moe
