@@ -1,0 +1,118 @@
+"""Host-side arithmetic of bench.py, on the CPU: launch counts, algorithmic bytes and
+FLOPs, the roofline's bound and fraction, the traffic record's source check, and the
+clock summary.  The expected values are worked out by hand from the layer's shapes
+(the per-stage formulas of the design notes) or taken from the ncu launch lists."""
+import json
+import os
+
+import pytest
+
+import bench
+from routed_grouped_gemm_softmax_b200.inputs import CONFIGS
+
+PEAKS = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1200.0}
+
+
+def test_kernels_per_forward_match_the_launch_lists():
+    # one forward's kernels, as listed by ncu on the GPU:
+    # decode: logits, top-k + grouping, gather, gate/up GEMM, down GEMM (combine inside)
+    assert bench.kernels_per_forward(CONFIGS["decode"]) == 5
+    # prefill/skewed: prep, tensor-core logits, certify, count, scan, scatter, gather,
+    # two GEMMs, combine
+    assert bench.kernels_per_forward(CONFIGS["prefill"]) == 10
+    assert bench.kernels_per_forward(CONFIGS["skewed"]) == 10
+    # fp8: as prefill, with the per-token quantiser before the (fp8) gather
+    assert bench.kernels_per_forward(CONFIGS["fp8"]) == 11
+    # tiny (T = 64): the large-batch router, the combine inside the down GEMM
+    assert bench.kernels_per_forward(CONFIGS["tiny"]) == 9
+
+
+def test_stage_work_bf16_by_hand():
+    cfg = CONFIGS["tiny"].replace(name="w", T=4, H=256, I=128, E=4, top_k=2)
+    w = bench.stage_work(cfg, [3, 0, 5, 0])  # two experts touched, A = 8 rows
+    assert w["_D"] == 2
+    # gate/up: 2 experts x (gate + up) x I x H bf16 + 8 rows of x in + 8 rows of h out
+    assert w["gemm_gate_up"]["bytes"] == 2 * 2 * 128 * 256 * 2 + 8 * 256 * 2 + 8 * 128 * 2 == 268288
+    assert w["gemm_gate_up"]["flops"] == 2 * 8 * 256 * 256
+    # down: 2 experts x H x I bf16 + 8 rows of h in + 8 rows of y out
+    assert w["gemm_down"]["bytes"] == 2 * 256 * 128 * 2 + 8 * 128 * 2 + 8 * 256 * 2 == 137216
+    assert w["gemm_down"]["flops"] == 2 * 8 * 128 * 256
+    # combine: y in, gates in, out
+    assert w["combine"]["bytes"] == 8 * 256 * 2 + 8 * 4 + 4 * 256 * 2
+    # router: x, router_w, indices + gates
+    assert w["route"]["bytes"] == 4 * 256 * 2 + 256 * 4 * 2 + 8 * 8
+
+
+def test_stage_work_fp8_by_hand():
+    cfg = CONFIGS["fp8"].replace(name="w8", T=4, H=256, I=256, E=4, top_k=2)
+    w = bench.stage_work(cfg, [8, 0, 0, 0])  # one expert, A = 8
+    # e4m3 gate + up (1 byte) + a 2 x 2 grid of fp32 block scales each; x and h rows
+    # as codes + one fp32 scale per 128 values
+    weights = 2 * 256 * 256 + 2 * (2 * 2 * 4)
+    rows = 8 * 256 + 8 * 2 * 4
+    assert w["gemm_gate_up"]["bytes"] == weights + rows + rows == 135328
+    assert w["gemm_down"]["bytes"] == (256 * 256 + 2 * 2 * 4) + rows + 8 * 256 * 2
+
+
+def test_roofline_picks_the_binding_resource():
+    work = {"g": {"bytes": 6e9, "flops": 1e12}, "t": {"bytes": 1e9, "flops": 3e12}}
+    r = bench.roofline_for("g", work, 2.0, PEAKS, "measured", False, "none")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(3000.0) and r["frac"] == pytest.approx(0.5)
+    r = bench.roofline_for("t", work, 4.0, PEAKS, "measured", False, "none")
+    assert r["bound"] == "tensor" and r["peak"] == 1500.0
+    assert r["achieved"] == pytest.approx(750.0) and r["frac"] == pytest.approx(0.5)
+    # a kernel timed inside a long run takes the sustained peak; fp8 doubles it
+    assert bench.roofline_for("t", work, 4.0, PEAKS, "measured", True, "none")["peak"] == 1200.0
+    assert bench.roofline_for("t", work, 4.0, PEAKS, "measured", False, "none", fp8=True)["peak"] == 3000.0
+
+
+def test_recorded_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
+    (tmp_path / "profiles").mkdir()
+    rec = {"decode": {"gemm_gate_up": {"dram_bytes_per_launch": 123, "sources": "aaaa"}}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_sources_hash", lambda stage: "aaaa")
+    assert bench.recorded_traffic("decode", "gemm_gate_up") == 123
+    assert bench.recorded_traffic("decode", "gemm_down") is None
+    monkeypatch.setattr(bench, "kernel_sources_hash", lambda stage: "bbbb")  # the kernel changed
+    assert bench.recorded_traffic("decode", "gemm_gate_up") is None
+
+
+def test_kernel_sources_hash_covers_the_stage_files():
+    for stage, files in bench.STAGE_SOURCES.items():
+        csrc = os.path.join(bench.ROOT, "routed_grouped_gemm_softmax_b200", "csrc")
+        assert all(os.path.exists(os.path.join(csrc, f)) for f in files), stage
+        assert len(bench.kernel_sources_hash(stage)) == 16
+
+
+def _sampler():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.lines, s.samples, s.thread, s.max_mhz = [], [], None, None
+    return s
+
+
+def test_clock_summary_from_nvidia_smi_lines():
+    s = _sampler()
+    s.lines = [
+        "2026/12/02 10:00:00.000, 1100, 1965, 300.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/02 10:00:01.000, 1900, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/02 10:00:01.050, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/02 10:00:01.100, 1700, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "garbage",
+    ]
+    import datetime as dt
+    t0 = dt.datetime(2026, 12, 2, 10, 0, 1).timestamp()
+    c = s.summary(t0, t0 + 0.1)
+    assert c["samples"] == 3 and c["sm_mhz"] == 1800.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_summary_from_nvml_samples():
+    s = _sampler()
+    s.thread, s.max_mhz = object(), 1965.0
+    s.bits = (0x8, 0x40, 0x20, 0x4)  # hw slowdown, hw thermal, sw thermal, sw power cap
+    s.samples = [(0.5, 1000.0, 0x0), (1.0, 1965.0, 0x0), (1.001, 1900.0, 0x4), (1.002, 1500.0, 0x40), (2.0, 1.0, 0x8)]
+    c = s.summary(1.0, 1.5)
+    assert c["samples"] == 3 and c["sm_mhz"] == 1900.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
