@@ -330,6 +330,42 @@ def stage_work(cfg, counts):
     }
 
 
+def layer_work(cfg, counts):
+    """The whole layer's algorithmic bytes and FLOPs: the touched experts' weights (with
+    their block scales for fp8), x, out, router_w and the chosen indices and gates; the
+    router and expert FLOPs.  The expert-ordered copy of x, h and y are the
+    implementation's own traffic, counted apart in `implementation_bytes` (each written
+    once and read once)."""
+    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k
+    A = T * k
+    D = int(sum(1 for c in counts if c > 0))
+    if cfg.dtype == "fp8":
+        per_expert = 3 * I * H + 3 * (I // 128) * (H // 128) * 4
+        inter = 2 * (A * H + A * H // 128 * 4) + 2 * (A * I + A * I // 128 * 4) + 2 * A * H * 2
+    else:
+        per_expert = 3 * I * H * 2
+        inter = 2 * (A * H * 2) + 2 * (A * I * 2) + 2 * (A * H * 2)
+    return {"bytes": D * per_expert + 2 * T * H * 2 + H * E * 2 + A * 8,
+            "flops": 2.0 * A * H * 2 * I + 2.0 * A * I * H + 2.0 * T * H * E,
+            "implementation_bytes": inter}
+
+
+def layer_roofline(cfg, counts, ms, peaks, peaks_kind, sustained):
+    """The layer per step against its binding roofline: HBM when its algorithmic bytes
+    take longer at the measured bandwidth than its FLOPs at the measured tensor peak."""
+    w = layer_work(cfg, counts)
+    fp8 = cfg.dtype == "fp8"
+    pk_tf = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * (2.0 if fp8 else 1.0)
+    t = ms * 1e-3
+    if w["bytes"] / (peaks["hbm_gbs"] * 1e9) >= w["flops"] / (pk_tf * 1e12):
+        achieved, peak, unit, bound = w["bytes"] / t / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+    else:
+        achieved, peak, unit, bound = w["flops"] / t / 1e12, pk_tf, "TFLOP/s", "tensor"
+    return {"bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "algorithmic_bytes": w["bytes"], "algorithmic_flops": w["flops"],
+            "implementation_bytes": w["implementation_bytes"], "peak_source": peaks_kind, "ms": round(ms, 5)}
+
+
 def roofline_for(stage, work, ms, peaks, peaks_kind, sustained, workload, fp8=False):
     w = work[stage]
     t = ms * 1e-3
@@ -596,6 +632,10 @@ def main():
     dominant = max(("route", "gemm_gate_up", "gemm_down", "combine"), key=lambda s: stage_ms[s])
     sustained = total_ms > 1000.0
     roof = roofline_for(dominant, work, stage_ms[dominant], peaks, peaks_kind, sustained, cfg.name, fp8)
+    try:  # an extra view of the same step; never allowed to cost the bench line
+        layer_roof = layer_roofline(cfg, counts, ms_per_step, peaks, peaks_kind, sustained)
+    except Exception as exc:
+        layer_roof = {"error": repr(exc)}
     stages = {s: {"ms": round(stage_ms[s], 4)} for s in api.STAGES}
     for s in ("route", "gemm_gate_up", "gemm_down", "combine"):
         r = roofline_for(s, work, stage_ms[s], peaks, peaks_kind, sustained, cfg.name, fp8)
@@ -636,7 +676,7 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "e4m3" if fp8 else "bf16",
                 "data": "synthetic", "config": config_block(cfg, world),
-                "roofline": roof, "stages": stages, "experts_touched": work["_D"],
+                "roofline": roof, "layer_roofline": layer_roof, "stages": stages, "experts_touched": work["_D"],
                 "e2e": e2e, "gpu_launches": kernels_per_forward(cfg) * args.steps, "schedule": sched,
                 "clocks": clocks, "cpu_baseline": cpu,
                 "p99_ms_per_step": round(sorted(step_ms)[min(len(step_ms) - 1, math.ceil(0.99 * len(step_ms)) - 1)], 5)}

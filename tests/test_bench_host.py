@@ -116,3 +116,36 @@ def test_clock_summary_from_nvml_samples():
     c = s.summary(1.0, 1.5)
     assert c["samples"] == 3 and c["sm_mhz"] == 1900.0 and c["sm_max_mhz"] == 1965.0
     assert c["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+
+
+def test_layer_work_matches_the_config_table():
+    # whole-layer bytes and FLOPs of the four workloads, as tabulated from their shapes:
+    # Decode D x 6.29 MB + 1.2 MB, 0.82 GFLOP; Prefill 1.61 GB + 35 MB (all 256 experts),
+    # 206.2 + 4.3 GFLOP; Skewed 2.21 GB + 135 MB, 1700.8 + 4.3 GFLOP; FP8 11.28 GB of
+    # e4m3 weights and scales + 33 MB, 721.6 + 3.8 GFLOP
+    dec = bench.layer_work(CONFIGS["decode"], [1] * 103 + [0] * 153)
+    assert dec["bytes"] == 103 * 6291456 + 1180672
+    assert dec["flops"] / 1e9 == pytest.approx(0.822, abs=1e-3)
+    pre = bench.layer_work(CONFIGS["prefill"], [1] * 256)
+    assert pre["bytes"] / 1e9 == pytest.approx(1.61 + 0.035, abs=0.01)
+    assert pre["flops"] / 1e9 == pytest.approx(206.2 + 4.3, abs=0.1)
+    skw = bench.layer_work(CONFIGS["skewed"], [1] * 64)
+    assert skw["bytes"] / 1e9 == pytest.approx(2.21 + 0.135, abs=0.01)
+    assert skw["flops"] / 1e9 == pytest.approx(1700.8 + 4.3, abs=0.1)
+    f8 = bench.layer_work(CONFIGS["fp8"], [1] * 256)
+    assert f8["bytes"] / 1e9 == pytest.approx(11.28 + 0.033, abs=0.01)
+    assert f8["flops"] / 1e9 == pytest.approx(721.6 + 3.8, abs=0.1)
+    # the expert-ordered copy of x, h and y: written once, read once
+    assert dec["implementation_bytes"] == 2 * (128 * 2048 * 2) + 2 * (128 * 512 * 2) + 2 * (128 * 2048 * 2)
+
+
+def test_layer_roofline_bound_and_fraction():
+    cfg = CONFIGS["decode"]
+    counts = [1] * 103 + [0] * 153
+    r = bench.layer_roofline(cfg, counts, 0.1, PEAKS, "measured", False)
+    b = bench.layer_work(cfg, counts)["bytes"]
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(b / 1e-4 / 1e9, abs=0.1)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6000.0, abs=1e-4)
+    r = bench.layer_roofline(CONFIGS["skewed"], [1] * 64, 2.0, PEAKS, "measured", False)
+    assert r["bound"] == "tensor" and r["peak"] == 1500.0
