@@ -168,7 +168,8 @@ moe_status_t moe_quantize_rows_fp8(int32_t R, int32_t K, const void *a, uint8_t 
 moe_status_t moe_workspace_offsets(const moe_dims_t *d, int dtype, size_t *out, int32_t n);
 
 /* Synchronises `stream`, returns the device status word of the workspace
- * (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_BAD_INDEX; MOE_ERR_CUDA if the stream
+ * (MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX or MOE_ERR_ROUTER_BOUND -- the first
+ * error recorded since the word was last cleared; MOE_ERR_CUDA if the stream
  * reports an error) and clears it. */
 moe_status_t moe_get_device_status(void *ws, void *stream);
 
