@@ -72,6 +72,12 @@ def kernels_per_forward(cfg) -> int:
     rows = 2 if cfg.dtype == "fp8" else 1   # fp8: quantise per token, then gather; bf16: gather
     return route + rows + 2 + combine   # + gate/up GEMM, down GEMM
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+B200_SMS, FP32_LANES_PER_SM = 148, 128   # CUDA-core fp32 FMA lanes of one B200
+
+
+def alu_peak_tflops(sm_max_mhz: float) -> float:
+    """CUDA-core fp32 peak: every lane retiring one FMA (2 FLOPs) per cycle at the max SM clock."""
+    return B200_SMS * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12
 FLUSH_BYTES = 512 << 20
 EVICT_FLOATS = 64 << 20   # 256 MiB read after the write, so the flush leaves no dirty lines
 
@@ -115,9 +121,11 @@ def load_peaks():
     try:
         with open(path) as f:
             d = json.load(f)
-        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+        p = {k: float(d[k]) for k in FALLBACK_PEAKS}
+        p["sm_max_mhz"] = float(d.get("sm_max_mhz", 1965.0))
+        return p, "measured"
     except (OSError, KeyError, ValueError):
-        return dict(FALLBACK_PEAKS), "fallback"
+        return dict(FALLBACK_PEAKS, sm_max_mhz=1965.0), "fallback"
 
 
 STAGE_SOURCES = {
@@ -321,7 +329,9 @@ def stage_work(cfg, counts):
     wsc = (lambda n, kk: (n // 128) * (kk // 128) * 4) if fp8 else (lambda n, kk: 0)
     ab = (lambda n: n + n // 128 * 4) if fp8 else (lambda n: 2 * n)   # activation bytes of n values
     return {
-        "route": {"bytes": T * H * 2 + H * E * 2 + A * 8, "flops": 2.0 * T * H * E, "alu": True},
+        # T <= 32: every logit is an fp32 FMA chain on the CUDA cores; above, the logits run
+        # on the tensor cores and only the candidates' chains on the CUDA cores
+        "route": {"bytes": T * H * 2 + H * E * 2 + A * 8, "flops": 2.0 * T * H * E, "alu": T <= 32},
         "gemm_gate_up": {"bytes": D * (2 * I * H * wb + 2 * wsc(I, H)) + ab(A * H) + ab(A * I),
                          "flops": 2.0 * A * H * 2 * I},
         "gemm_down": {"bytes": D * (H * I * wb + wsc(H, I)) + ab(A * I) + A * H * 2, "flops": 2.0 * A * I * H},
@@ -373,7 +383,11 @@ def roofline_for(stage, work, ms, peaks, peaks_kind, sustained, workload, fp8=Fa
     # fp8 tensor peak = measured bf16 peak x the nominal fp8/bf16 ratio (4.5 / 2.25 PF)
     pk_tf = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * (2.0 if fp8 else 1.0)
     tc_time = w["flops"] / (pk_tf * 1e12)
-    if w.get("alu") or bw_time >= tc_time:
+    if w.get("alu"):
+        achieved = w["flops"] / t / 1e12
+        r = {"bound": "alu", "achieved": round(achieved, 3),
+             "peak": round(alu_peak_tflops(peaks.get("sm_max_mhz", 1965.0)), 1), "unit": "TFLOP/s"}
+    elif bw_time >= tc_time:
         achieved = w["bytes"] / t / 1e9
         r = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     else:
@@ -384,8 +398,11 @@ def roofline_for(stage, work, ms, peaks, peaks_kind, sustained, workload, fp8=Fa
     r["kernel"] = stage
     r["algorithmic_bytes"] = w["bytes"]
     r["algorithmic_flops"] = w["flops"]
-    r["peak_source"] = f"{peaks_kind}" + ("" if r["bound"] == "hbm" else (" sustained" if sustained else " burst")
-                                          + (" bf16 x 2 (nominal fp8/bf16 ratio)" if fp8 else ""))
+    if r["bound"] == "alu":
+        r["peak_source"] = "148 SMs x 128 fp32 lanes x 2 FLOPs x the max SM clock"
+    else:
+        r["peak_source"] = f"{peaks_kind}" + ("" if r["bound"] == "hbm" else (" sustained" if sustained else " burst")
+                                              + (" bf16 x 2 (nominal fp8/bf16 ratio)" if fp8 else ""))
     r["ms"] = round(ms, 4)
     return r
 

@@ -149,3 +149,21 @@ def test_layer_roofline_bound_and_fraction():
     assert r["frac"] == pytest.approx(r["achieved"] / 6000.0, abs=1e-4)
     r = bench.layer_roofline(CONFIGS["skewed"], [1] * 64, 2.0, PEAKS, "measured", False)
     assert r["bound"] == "tensor" and r["peak"] == 1500.0
+
+
+def test_alu_bound_router_stage():
+    # the small-batch router is fp32 FMA chains on the CUDA cores: reported against
+    # 148 SMs x 128 lanes x 2 FLOPs x 1965 MHz = 74.4 TFLOP/s
+    assert bench.alu_peak_tflops(1965.0) == pytest.approx(74.45, abs=0.01)
+    w = bench.stage_work(CONFIGS["decode"], [1] * 103 + [0] * 153)
+    assert w["route"]["alu"] and not bench.stage_work(CONFIGS["prefill"], [1] * 256)["route"]["alu"]
+    peaks = dict(PEAKS, sm_max_mhz=1965.0)
+    r = bench.roofline_for("route", w, 0.02, peaks, "measured", False, "none")
+    assert r["bound"] == "alu" and r["unit"] == "TFLOP/s" and r["peak"] == pytest.approx(74.4, abs=0.1)
+    assert r["achieved"] == pytest.approx(2.0 * 16 * 2048 * 256 / 2e-5 / 1e12, abs=1e-3)
+
+
+def test_load_peaks_carries_the_sm_clock():
+    p, kind = bench.load_peaks()
+    assert kind in ("measured", "fallback") and p["sm_max_mhz"] > 0
+    assert all(k in p for k in bench.FALLBACK_PEAKS)
