@@ -1,7 +1,7 @@
 """Benchmark of the MoE layer forward on B200: tokens/s of whole layer steps.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|tiny]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|fp8|tiny]
+                    [--impl ours|reference] [--schedule ...] [--pair ...] [--swap-ab ...] [--shape K=V,...]
 
 One step = one pass of the whole layer (router softmax top-k, permute, grouped
 gate/up GEMM + SwiGLU, grouped down GEMM, combine) over one batch of seeded
