@@ -1,6 +1,9 @@
 // fp8_swapab.cu -- the fp8 gate/up GEMM with the MMA operands' roles swapped, for
 // expert groups much shorter than a 128-row tile.
 //
+// The GC-MoE page (its compute-partition section) runs the expert GEMMs on
+// Blackwell as operand-swapped tcgen05 block-scaled MMAs with SwiGLU and
+// requantisation fused; this kernel is that idea for this layer's fp32 block scales.
 // The one-CTA fp8 kernel (fp8.cu) puts a tile's token rows on the MMA's M side, so
 // a group of 32 tokens still costs a 128-row MMA and a 128-row promotion of every K
 // block.  Here the M side is 128 weight rows (output features of I) and the N side
