@@ -75,6 +75,8 @@ class Oracle:
         lib.oracle_permute.restype = i
         lib.oracle_combine_ffn.argtypes = [i, i, i, P, P, P, P, P, P, i, P, P, i]
         lib.oracle_combine_ffn.restype = i
+        lib.oracle_shared_ffn.argtypes = [i, i, P, P, P, P, i, P, P, i]
+        lib.oracle_shared_ffn.restype = i
         lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         lib.oracle_e4m3_decode.restype = ctypes.c_double
         lib.oracle_e4m3_encode_array.argtypes = [i, P, P]
@@ -141,6 +143,24 @@ class Oracle:
                                          nthreads or default_threads())
         if rc:
             raise ValueError(f"oracle_combine_ffn rejected its arguments (code {rc})")
+        return out
+
+    def shared_ffn(self, x, w_gate, w_up, w_down, tokens=None, nthreads: int | None = None):
+        """A shared expert's SwiGLU FFN output for every token (weight 1), fp64 [n,H]:
+        w_gate, w_up [I,H], w_down [H,I] bf16.  The layer with a shared expert is
+        combine_ffn(...) + shared_ffn(...)."""
+        xb = _bf16_bits(x)
+        T, H = xb.shape
+        wg, wu, wd = _bf16_bits(w_gate), _bf16_bits(w_up), _bf16_bits(w_down)
+        I, H2 = wg.shape
+        assert H2 == H and wu.shape == wg.shape and wd.shape == (H, I)
+        tok = None if tokens is None else np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+        n = T if tok is None else tok.size
+        out = np.zeros((n, H), np.float64)
+        rc = self.lib.oracle_shared_ffn(H, I, _ptr(xb), _ptr(wg), _ptr(wu), _ptr(wd), n, _ptr(tok),
+                                        _ptr(out), nthreads or default_threads())
+        if rc:
+            raise ValueError(f"oracle_shared_ffn rejected its arguments (code {rc})")
         return out
 
     # ------------------------------------------------------------ FP8 variant
@@ -228,6 +248,10 @@ def forward(*a, **kw):
 
 def quantize_rows(*a, **kw):
     return get().quantize_rows(*a, **kw)
+
+
+def shared_ffn(*a, **kw):
+    return get().shared_ffn(*a, **kw)
 
 
 def combine_ffn_fp8(*a, **kw):

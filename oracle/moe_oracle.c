@@ -40,6 +40,10 @@
  * GEMM is sum over 128-wide K blocks of sa[row,kb] * sb[nblk,kb] * (qa . qb)_kb,
  * evaluated in fp64 from the exact decoded codes.
  *
+ * Shared expert (GC-MoE page: "optional shared experts" fused into the expert
+ * kernel, not defined there): one more SwiGLU FFN that every token passes through
+ * with weight 1, added to the routed sum (oracle_shared_ffn; the caller adds).
+ *
  * Deliberately slow and direct: no blocking, no fusion, no reordering.
  */
 #include <math.h>
@@ -290,6 +294,58 @@ int oracle_combine_ffn(int H, int I, int k, const uint16_t *x, const int32_t *id
     }
     for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, ffn_worker, &jobs[i]);
     ffn_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    return 0;
+}
+
+/* ---------------------------------------------------------- shared expert */
+
+typedef struct {
+    int H, I;
+    const uint16_t *x, *wg, *wu, *wd;
+    const int32_t *tokens;
+    double *out;
+    int n0, n1;
+} shared_job;
+
+static void *shared_worker(void *p)
+{
+    shared_job *j = (shared_job *)p;
+    double *xt = (double *)malloc(sizeof(double) * (size_t)j->H);
+    double *a = (double *)malloc(sizeof(double) * (size_t)j->I);
+    for (int n = j->n0; n < j->n1; ++n) {
+        int t = j->tokens ? j->tokens[n] : n;
+        for (int h = 0; h < j->H; ++h) xt[h] = bf16_to_f64(j->x[(size_t)t * j->H + h]);
+        expert_ffn(j->H, j->I, 0, xt, j->wg, j->wu, j->wd, a, j->out + (size_t)n * j->H);
+    }
+    free(xt);
+    free(a);
+    return NULL;
+}
+
+/* A shared expert: one gate/up/down SwiGLU FFN that every token passes through with
+ * weight 1, its output added to the gate-weighted sum of the routed experts (the
+ * GC-MoE page fuses "optional shared experts" into its expert kernel without
+ * defining them; this is the plainest reading).  The caller adds the two:
+ *   out[n] = oracle_combine_ffn(...)[n] + this[n].
+ *   wg, wu: [I,H] bf16; wd: [H,I] bf16; tokens as in oracle_combine_ffn
+ *   ->  out [n,H] fp64 (overwritten). */
+int oracle_shared_ffn(int H, int I, const uint16_t *x, const uint16_t *wg, const uint16_t *wu,
+                      const uint16_t *wd, int n, const int32_t *tokens, double *out, int nthreads)
+{
+    if (H <= 0 || I <= 0 || n < 0) return 1;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > n) nthreads = n > 0 ? n : 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    shared_job jobs[256];
+    for (int i = 0; i < nthreads; ++i) {
+        shared_job j = {H, I, x, wg, wu, wd, tokens, out,
+                        (int)((long)n * i / nthreads), (int)((long)n * (i + 1) / nthreads)};
+        jobs[i] = j;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, shared_worker, &jobs[i]);
+    shared_worker(&jobs[0]);
     for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
     return 0;
 }

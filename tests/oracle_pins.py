@@ -379,3 +379,33 @@ def pin_fp8_close_to_unquantised(orc):
 
 ALL_PINS += [pin_e4m3_codes_vs_torch, pin_quantize_rows, pin_fp8_ffn_dense_brute_force,
              pin_fp8_close_to_unquantised]
+
+
+# ------------------------------------------------------------- shared expert
+
+def pin_shared_expert_is_swiglu_mlp(orc):
+    """A shared expert (every token, weight 1) is a textbook SwiGLU MLP: torch fp64
+    silu(x Wg^T) * (x Wu^T), then Wd, on all tokens and on a subset in any order.
+    Its intermediate size differs from the routed experts' so that a mixed-up
+    shape or transposed operand cannot pass.  With the weights of routed expert e
+    it equals the layer restricted to expert e with gate 1."""
+    inp = tiny_inputs(T=12)
+    H, I_s = inp.x.shape[1], 192
+    g = torch.Generator().manual_seed(7)
+    wg = (torch.randn(I_s, H, generator=g, dtype=torch.float64) / H ** 0.5).to(torch.bfloat16)
+    wu = (torch.randn(I_s, H, generator=g, dtype=torch.float64) / H ** 0.5).to(torch.bfloat16)
+    wd = (torch.randn(H, I_s, generator=g, dtype=torch.float64) / I_s ** 0.5).to(torch.bfloat16)
+    out = orc.shared_ffn(inp.x, wg, wu, wd)
+    X = inp.x.double()
+    ref = (F.silu(X @ wg.double().T) * (X @ wu.double().T)) @ wd.double().T
+    assert np.allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+    sub = orc.shared_ffn(inp.x, wg, wu, wd, tokens=[5, 2, 11])
+    assert np.array_equal(sub, out[[5, 2, 11]])
+    e = 3
+    T = inp.x.shape[0]
+    one = orc.combine_ffn(inp.x, np.full((T, 1), e, np.int32), np.ones((T, 1)), inp.w_gate, inp.w_up, inp.w_down)
+    same = orc.shared_ffn(inp.x, inp.w_gate[e], inp.w_up[e], inp.w_down[e])
+    assert np.allclose(same, one, rtol=1e-13, atol=1e-13)
+
+
+ALL_PINS += [pin_shared_expert_is_swiglu_mlp]

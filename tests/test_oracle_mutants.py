@@ -33,6 +33,8 @@ MUTANTS = {
     "fp8_act_scale_dropped": ("acc += (double)sa[kb] * (double)sb", "acc += (double)sb"),
     "fp8_amax_448_off": ("float s = amax / 448.0f;", "float s = amax / 440.0f;"),
     "fp8_h_not_requantised": ("fp8_row_gemm(H, I, qh, sh,", "fp8_row_gemm(H, I, qh, sx,"),
+    "shared_gate_up_swapped": ("expert_ffn(j->H, j->I, 0, xt, j->wg, j->wu, j->wd,",
+                               "expert_ffn(j->H, j->I, 0, xt, j->wu, j->wg, j->wd,"),
 }
 
 
