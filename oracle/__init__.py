@@ -85,6 +85,14 @@ class Oracle:
         lib.oracle_quantize_rows.restype = i
         lib.oracle_combine_ffn_fp8.argtypes = [i, i, i, P, P, P, P, P, P, P, P, P, i, P, P, i]
         lib.oracle_combine_ffn_fp8.restype = i
+        lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e2m1_decode.restype = ctypes.c_double
+        lib.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e2m1_encode.restype = ctypes.c_uint8
+        lib.oracle_mx_quantize_rows.argtypes = [i, i, P, i, P, P]
+        lib.oracle_mx_quantize_rows.restype = i
+        lib.oracle_combine_ffn_mx.argtypes = [i, i, i, P, P, P, P, P, P, P, P, P, i, P, P, i]
+        lib.oracle_combine_ffn_mx.restype = i
         self.lib = lib
 
     def route(self, x, router_w, bias, top_k: int, want_logits: bool = False,
@@ -210,6 +218,51 @@ class Oracle:
                                              _ptr(out), nthreads or default_threads())
         if rc:
             raise ValueError(f"oracle_combine_ffn_fp8 rejected its arguments (code {rc})")
+        return out
+
+    # ---------------------------------------------- MX (FP4 weights, FP8 activations)
+
+    MX_E4M3, MX_E2M1 = 0, 1
+
+    def e2m1_decode(self, codes) -> np.ndarray:
+        c = np.asarray(codes, dtype=np.uint8).reshape(-1)
+        return np.array([self.lib.oracle_e2m1_decode(int(v)) for v in c]).reshape(np.shape(codes))
+
+    def e2m1_encode(self, values) -> np.ndarray:
+        v = np.asarray(values, dtype=np.float32).reshape(-1)
+        return np.array([self.lib.oracle_e2m1_encode(float(a)) for a in v], np.uint8).reshape(np.shape(values))
+
+    def mx_quantize_rows(self, a, fmt: int):
+        """OCP MX quantisation of an fp32 matrix [R,K] (K % 32 == 0) per row and per 32
+        columns: (codes uint8 [R,K], e8m0 scale codes uint8 [R,K/32])."""
+        af = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+        R, K = af.shape
+        q = np.zeros((R, K), np.uint8)
+        x = np.zeros((R, K // 32), np.uint8)
+        rc = self.lib.oracle_mx_quantize_rows(R, K, _ptr(af), int(fmt), _ptr(q), _ptr(x))
+        if rc:
+            raise ValueError(f"oracle_mx_quantize_rows rejected its arguments (code {rc})")
+        return q, x
+
+    def combine_ffn_mx(self, x, idx, gate, wg_q, wg_x, wu_q, wu_x, wd_q, wd_x, tokens=None,
+                       nthreads: int | None = None):
+        """The MX variant of combine_ffn: e2m1 weight codes [E,N,K] with e8m0 scale codes
+        [E,N,K/32]; x and h quantised to MX e4m3 per 32 values.  fp64 [n,H]."""
+        xb = _bf16_bits(x)
+        T, H = xb.shape
+        arrs = [np.ascontiguousarray(np.asarray(a, dtype=np.uint8)) for a in (wg_q, wg_x, wu_q, wu_x, wd_q, wd_x)]
+        E, I, H2 = arrs[0].shape
+        assert H2 == H and arrs[1].shape == (E, I, H // 32) and arrs[4].shape == (E, H, I)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        tok = None if tokens is None else np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+        n = T if tok is None else tok.size
+        out = np.zeros((n, H), np.float64)
+        rc = self.lib.oracle_combine_ffn_mx(H, I, idx.shape[1], _ptr(xb), _ptr(idx), _ptr(gate),
+                                            *[_ptr(a) for a in arrs], n, _ptr(tok), _ptr(out),
+                                            nthreads or default_threads())
+        if rc:
+            raise ValueError(f"oracle_combine_ffn_mx rejected its arguments (code {rc})")
         return out
 
     def forward(self, x, router_w, bias, w_gate, w_up, w_down, top_k: int, tokens=None,

@@ -40,6 +40,12 @@
  * GEMM is sum over 128-wide K blocks of sa[row,kb] * sb[nblk,kb] * (qa . qb)_kb,
  * evaluated in fp64 from the exact decoded codes.
  *
+ * MX variant (GC-MoE page: FP8/FP4 block-scaled MMA on Blackwell; the element
+ * and scale formats are those of the OCP Microscaling Formats spec v1.0): weights
+ * as e2m1 codes and activations (x, and h after SwiGLU) as e4m3 codes, each with
+ * one power-of-two e8m0 scale per 32 values along K; every GEMM is a sum over
+ * 32-wide K blocks of 2^(Xa + Xb) * (codes . codes) in fp64 (oracle_combine_ffn_mx).
+ *
  * Shared expert (GC-MoE page: "optional shared experts" fused into the expert
  * kernel, not defined there): one more SwiGLU FFN that every token passes through
  * with weight 1, added to the routed sum (oracle_shared_ffn; the caller adds).
@@ -525,6 +531,181 @@ int oracle_combine_ffn_fp8(int H, int I, int k, const uint16_t *x, const int32_t
     }
     for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, ffn8_worker, &jobs[i]);
     ffn8_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    return 0;
+}
+
+/* ------------------------------------------------- MX (OCP microscaling) */
+
+/* Value of an e2m1 (FP4) code, bits s eem: 1 sign bit, 2 exponent bits with bias
+ * 1, 1 mantissa bit; exponent 0 is subnormal (m * 0.5).  The magnitudes are 0,
+ * 0.5, 1, 1.5, 2, 3, 4, 6; there is no infinity or NaN. */
+double oracle_e2m1_decode(uint8_t c)
+{
+    int sgn = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+    double v = e == 0 ? 0.5 * m : (1.0 + 0.5 * m) * ldexp(1.0, e - 1);
+    return sgn ? -v : v;
+}
+
+/* Round-to-nearest-even code of a value inside the format's range: the nearest of
+ * the nmag magnitudes (codes 0..nmag-1 in increasing order) by brute force; on a
+ * tie the code whose last (mantissa) bit is 0.  sign_bit is the code's sign bit. */
+static uint8_t encode_rne(double v, double (*decode)(uint8_t), int nmag, int sign_bit)
+{
+    double a = fabs(v);
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c < nmag; ++c) {
+        double d = fabs(decode((uint8_t)c) - a);
+        if (d < bd || (d == bd && !(c & 1) && (best & 1))) {  /* a tie goes to the even code */
+            bd = d;
+            best = c;
+        }
+    }
+    if (best != 0 && v < 0) best |= 1 << sign_bit;
+    return (uint8_t)best;
+}
+
+uint8_t oracle_e2m1_encode(float v) { return encode_rne((double)v, oracle_e2m1_decode, 8, 3); }
+
+/* The two MX element formats used here: e4m3 (largest exponent emax = 8, largest
+ * value 448) and e2m1 (emax = 2, largest value 6). */
+enum { MX_E4M3 = 0, MX_E2M1 = 1 };
+#define MX_BLOCK 32
+
+/* One MX block of 32 fp32 values (OCP Microscaling Formats, v1.0, the conversion
+ * of a block: the shared scale is 2^X with X = floor(log2(max |v|)) - emax of the
+ * element format, stored as an e8m0 code X + 127; each element is v / 2^X rounded
+ * to nearest-even in the element format, values past its largest magnitude
+ * clamped to it).  Readings: X is clamped to [-127, 127]; an all-zero block gets
+ * X = 0 and zero codes.  Returns the e8m0 code; q receives the element codes. */
+static uint8_t mx_quantize_block(const float *v, int fmt, uint8_t *q)
+{
+    const int emax = fmt == MX_E4M3 ? 8 : 2;
+    const double vmax = fmt == MX_E4M3 ? 448.0 : 6.0;
+    double amax = 0.0;
+    for (int i = 0; i < MX_BLOCK; ++i)
+        if (fabs((double)v[i]) > amax) amax = fabs((double)v[i]);
+    if (amax == 0.0) {
+        for (int i = 0; i < MX_BLOCK; ++i) q[i] = 0;
+        return 127;
+    }
+    int ex;
+    frexp(amax, &ex);  /* amax = f * 2^ex, f in [0.5, 1): floor(log2(amax)) = ex - 1 */
+    int X = ex - 1 - emax;
+    if (X < -127) X = -127;
+    if (X > 127) X = 127;
+    for (int i = 0; i < MX_BLOCK; ++i) {
+        double r = ldexp((double)v[i], -X);
+        if (r > vmax) r = vmax;
+        if (r < -vmax) r = -vmax;
+        q[i] = fmt == MX_E4M3 ? encode_rne(r, oracle_e4m3_decode, 127, 7) : encode_rne(r, oracle_e2m1_decode, 8, 3);
+    }
+    return (uint8_t)(X + 127);
+}
+
+/* Per-row MX quantisation of an fp32 matrix [R, K] (K a multiple of 32):
+ * q [R, K] element codes (one per byte), x [R, K/32] e8m0 scale codes. */
+int oracle_mx_quantize_rows(int R, int K, const float *a, int fmt, uint8_t *q, uint8_t *x)
+{
+    if (R < 0 || K <= 0 || K % MX_BLOCK || (fmt != MX_E4M3 && fmt != MX_E2M1)) return 1;
+    for (int r = 0; r < R; ++r)
+        for (int b = 0; b < K / MX_BLOCK; ++b)
+            x[(size_t)r * (K / MX_BLOCK) + b] =
+                mx_quantize_block(a + (size_t)r * K + b * MX_BLOCK, fmt, q + (size_t)r * K + b * MX_BLOCK);
+    return 0;
+}
+
+/* One row of an MX GEMM, activations e4m3 and weights e2m1:
+ *   out[n] = sum_kb 2^(xa[kb] - 127) * 2^(xb[n,kb] - 127) * sum_{k in kb} a_k * b_{n,k}
+ * over blocks kb of 32 along K; qb [N, K] e2m1 codes, xb [N, K/32]. */
+static void mx_row_gemm(int N, int K, const uint8_t *qa, const uint8_t *xa, const uint8_t *qb,
+                        const uint8_t *xb, double *out)
+{
+    const int KB = K / MX_BLOCK;
+    for (int n = 0; n < N; ++n) {
+        double acc = 0.0;
+        for (int kb = 0; kb < KB; ++kb) {
+            double part = 0.0;
+            for (int k = kb * MX_BLOCK; k < kb * MX_BLOCK + MX_BLOCK; ++k)
+                part += e4m3(qa[k]) * oracle_e2m1_decode(qb[(size_t)n * K + k]);
+            acc += ldexp(1.0, (int)xa[kb] - 127) * ldexp(1.0, (int)xb[(size_t)n * KB + kb] - 127) * part;
+        }
+        out[n] = acc;
+    }
+}
+
+typedef struct {
+    int H, I, k;
+    const uint16_t *x;
+    const int32_t *idx;
+    const double *gate;
+    const uint8_t *wg, *wu, *wd, *xg, *xu, *xd;
+    const int32_t *tokens;
+    double *out;
+    int n0, n1;
+} ffnmx_job;
+
+static void *ffnmx_worker(void *p)
+{
+    ffnmx_job *j = (ffnmx_job *)p;
+    const int H = j->H, I = j->I;
+    float *xf = (float *)malloc(sizeof(float) * (size_t)H);
+    uint8_t *qx = (uint8_t *)malloc((size_t)H);
+    uint8_t *sx = (uint8_t *)malloc((size_t)(H / MX_BLOCK));
+    double *g = (double *)malloc(sizeof(double) * (size_t)I);
+    double *u = (double *)malloc(sizeof(double) * (size_t)I);
+    float *h = (float *)malloc(sizeof(float) * (size_t)I);
+    uint8_t *qh = (uint8_t *)malloc((size_t)I);
+    uint8_t *sh = (uint8_t *)malloc((size_t)(I / MX_BLOCK));
+    double *y = (double *)malloc(sizeof(double) * (size_t)H);
+    for (int n = j->n0; n < j->n1; ++n) {
+        int t = j->tokens ? j->tokens[n] : n;
+        for (int c = 0; c < H; ++c) xf[c] = bf16_to_f32(j->x[(size_t)t * H + c]);
+        oracle_mx_quantize_rows(1, H, xf, MX_E4M3, qx, sx);
+        double *o = j->out + (size_t)n * H;
+        for (int c = 0; c < H; ++c) o[c] = 0.0;
+        for (int q = 0; q < j->k; ++q) {
+            int e = j->idx[(size_t)t * j->k + q];
+            double gt = j->gate[(size_t)t * j->k + q];
+            mx_row_gemm(I, H, qx, sx, j->wg + (size_t)e * I * H, j->xg + (size_t)e * I * (H / MX_BLOCK), g);
+            mx_row_gemm(I, H, qx, sx, j->wu + (size_t)e * I * H, j->xu + (size_t)e * I * (H / MX_BLOCK), u);
+            for (int i = 0; i < I; ++i) h[i] = (float)(silu(g[i]) * u[i]);
+            oracle_mx_quantize_rows(1, I, h, MX_E4M3, qh, sh);
+            mx_row_gemm(H, I, qh, sh, j->wd + (size_t)e * H * I, j->xd + (size_t)e * H * (I / MX_BLOCK), y);
+            for (int c = 0; c < H; ++c) o[c] += gt * y[c];
+        }
+    }
+    free(xf); free(qx); free(sx); free(g); free(u); free(h); free(qh); free(sh); free(y);
+    return NULL;
+}
+
+/* MX variant of oracle_combine_ffn (FP4 weights, FP8 activations, each with one
+ * power-of-two scale per 32 values along K): x [T,H] bf16 is quantised per token
+ * to MX e4m3, each chosen expert's gate/up GEMMs are MX block sums against e2m1
+ * weights, the SwiGLU output h (rounded to fp32) is requantised to MX e4m3, the
+ * down GEMM is an MX block sum, and the k results are summed with the gates in fp64.
+ *   wg/wu [E,I,H] e2m1 codes with xg/xu [E,I,H/32] e8m0 codes; wd [E,H,I] with
+ *   xd [E,H,I/32]. */
+int oracle_combine_ffn_mx(int H, int I, int k, const uint16_t *x, const int32_t *idx,
+                          const double *gate, const uint8_t *wg, const uint8_t *xg, const uint8_t *wu,
+                          const uint8_t *xu, const uint8_t *wd, const uint8_t *xd, int n,
+                          const int32_t *tokens, double *out, int nthreads)
+{
+    if (H <= 0 || I <= 0 || H % MX_BLOCK || I % MX_BLOCK || k < 1 || n < 0) return 1;
+    pthread_once(&g_e4m3_once, build_e4m3_table);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > n) nthreads = n > 0 ? n : 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    ffnmx_job jobs[256];
+    for (int i = 0; i < nthreads; ++i) {
+        ffnmx_job jb = {H, I, k, x, idx, gate, wg, wu, wd, xg, xu, xd, tokens, out,
+                        (int)((long)n * i / nthreads), (int)((long)n * (i + 1) / nthreads)};
+        jobs[i] = jb;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, ffnmx_worker, &jobs[i]);
+    ffnmx_worker(&jobs[0]);
     for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
     return 0;
 }

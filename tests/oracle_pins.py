@@ -409,3 +409,136 @@ def pin_shared_expert_is_swiglu_mlp(orc):
 
 
 ALL_PINS += [pin_shared_expert_is_swiglu_mlp]
+
+
+# --------------------------------------------- MX variant (FP4 weights, FP8 acts)
+
+E2M1_MAGS = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]   # the e2m1 magnitudes, OCP MX v1.0 table
+
+
+def _e4m3_mags():
+    """The 127 finite non-negative e4m3 magnitudes, decoded by torch's float8_e4m3fn."""
+    return torch.arange(127, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+
+
+def _rne_code(v, mags, sign_bit):
+    """Nearest magnitude by brute force; a tie goes to the even code."""
+    a = abs(float(v))
+    d = np.abs(np.asarray(mags) - a)
+    near = np.flatnonzero(d == d.min())
+    c = int(near[0]) if near.size == 1 else int([n for n in near if n % 2 == 0][0])
+    return c | ((1 << sign_bit) if (v < 0 and c != 0) else 0)
+
+
+def _mx_quant_ref(row, fmt):
+    """Reference MX quantisation of one row (numpy): per 32 values, X = floor(log2 amax)
+    - emax (np.frexp), elements round-to-nearest-even of v / 2^X, clamped."""
+    mags, sb, emax, vmax = (_e4m3_mags(), 7, 8, 448.0) if fmt == 0 else (E2M1_MAGS, 3, 2, 6.0)
+    row = np.asarray(row, dtype=np.float32).astype(np.float64)
+    q = np.zeros(row.size, np.uint8)
+    xs = np.zeros(row.size // 32, np.uint8)
+    for b in range(row.size // 32):
+        blk = row[b * 32:(b + 1) * 32]
+        amax = np.abs(blk).max()
+        if amax == 0.0:
+            xs[b] = 127
+            continue
+        X = int(np.clip(np.frexp(amax)[1] - 1 - emax, -127, 127))
+        xs[b] = X + 127
+        r = np.clip(np.ldexp(blk, -X), -vmax, vmax)
+        q[b * 32:(b + 1) * 32] = [_rne_code(v, mags, sb) for v in r]
+    return q, xs
+
+
+def _mx_dequant(q, xs, fmt):
+    mags = _e4m3_mags() if fmt == 0 else np.asarray(E2M1_MAGS)
+    sb = 7 if fmt == 0 else 3
+    q = np.asarray(q, dtype=np.int64)
+    mag = mags[q & ((1 << sb) - 1)] * np.where(q >> sb, -1.0, 1.0)
+    sc = np.ldexp(1.0, np.repeat(np.asarray(xs, dtype=np.int64) - 127, 32, axis=-1))
+    return mag * sc
+
+
+def pin_e2m1_codes(orc):
+    """e2m1 decoding is the OCP table; encoding is the nearest code with ties to the even
+    code, on random values, every midpoint between neighbours, and past the largest."""
+    codes = np.arange(16, dtype=np.uint8)
+    ref = np.array(E2M1_MAGS + [-m for m in E2M1_MAGS])
+    assert np.array_equal(orc.e2m1_decode(codes), ref)
+    vals = list(np.random.default_rng(3).uniform(-6.5, 6.5, 500).astype(np.float32))
+    vals += [(a + b) / 2 for a, b in zip(E2M1_MAGS, E2M1_MAGS[1:])] + [-0.75, -2.5, 6.0, 7.0, -9.0]
+    got = orc.e2m1_encode(np.asarray(vals, np.float32))
+    assert [int(c) for c in got] == [_rne_code(v, E2M1_MAGS, 3) for v in vals]
+
+
+def pin_mx_quantize_rows(orc):
+    """MX quantisation of both element formats equals the reference on random rows of
+    many magnitudes, an all-zero block, a block with one huge value and exact powers of two."""
+    rng = np.random.default_rng(4)
+    rows = [rng.standard_normal(64) * 10.0 ** rng.uniform(-3, 3) for _ in range(6)]
+    special = np.zeros(64)
+    special[32:] = rng.standard_normal(32)
+    special[40] = 3.0e4
+    rows += [special, np.ldexp(1.0, np.arange(-20, 44))]
+    a = np.asarray(rows, dtype=np.float32)
+    for fmt in (0, 1):
+        q, xs = orc.mx_quantize_rows(a, fmt)
+        for r in range(a.shape[0]):
+            qr, xr = _mx_quant_ref(a[r], fmt)
+            assert np.array_equal(xs[r], xr), (fmt, r)
+            assert np.array_equal(q[r], qr), (fmt, r)
+        assert list(xs[6][:1]) == [127] and not q[6][:32].any()   # the all-zero block
+
+
+def _mx_case():
+    rng = np.random.default_rng(5)
+    T, H, I, E, k = 6, 64, 96, 3, 2
+    x = torch.as_tensor(rng.standard_normal((T, H)).astype(np.float32)).to(torch.bfloat16)
+    master = {n: rng.standard_normal((E,) + s).astype(np.float32) / np.sqrt(s[1])
+              for n, s in (("w_gate", (I, H)), ("w_up", (I, H)), ("w_down", (H, I)))}
+    w = {}
+    for n, m in master.items():
+        E_, N, K = m.shape
+        qs = [_mx_quant_ref(m[e, r], 1) for e in range(E_) for r in range(N)]
+        w[n + "_q"] = np.stack([a for a, _ in qs]).reshape(E_, N, K)
+        w[n + "_x"] = np.stack([b for _, b in qs]).reshape(E_, N, K // 32)
+    idx = np.array([[0, 1], [2, 0], [1, 2], [0, 2], [2, 1], [1, 0]], np.int32)
+    gate = rng.uniform(0.1, 1.0, (T, k))
+    gate /= gate.sum(1, keepdims=True)
+    return x, master, w, idx, gate
+
+
+def pin_mx_ffn_dense_brute_force(orc):
+    """The MX layer equals a dense evaluation: every quantisation by the reference, the
+    codes dequantised, then fp64 matmuls, SwiGLU (torch silu), h rounded to fp32."""
+    x, _, w, idx, gate = _mx_case()
+    out = orc.combine_ffn_mx(x, idx, gate, w["w_gate_q"], w["w_gate_x"], w["w_up_q"], w["w_up_x"],
+                             w["w_down_q"], w["w_down_x"])
+    deq = {n: _mx_dequant(w[n + "_q"], w[n + "_x"], 1) for n in ("w_gate", "w_up", "w_down")}
+    X = x.float().numpy()
+    ref = np.zeros(out.shape)
+    for t in range(X.shape[0]):
+        qx, sx = _mx_quant_ref(X[t], 0)
+        xd = _mx_dequant(qx, sx, 0)
+        for j in range(idx.shape[1]):
+            e = idx[t, j]
+            g, u = deq["w_gate"][e] @ xd, deq["w_up"][e] @ xd
+            h = (F.silu(torch.as_tensor(g)) * torch.as_tensor(u)).numpy().astype(np.float32)
+            qh, sh = _mx_quant_ref(h, 0)
+            ref[t] += gate[t, j] * (deq["w_down"][e] @ _mx_dequant(qh, sh, 0))
+    assert np.allclose(out, ref, rtol=1e-10, atol=1e-12), np.abs(out - ref).max()
+
+
+def pin_mx_close_to_unquantised(orc):
+    """With FP4 weights and FP8 activations the layer stays near the unquantised layer
+    on the same master weights (rel-L2 well below 1: no dropped scale or factor 2^k)."""
+    x, master, w, idx, gate = _mx_case()
+    out = orc.combine_ffn_mx(x, idx, gate, w["w_gate_q"], w["w_gate_x"], w["w_up_q"], w["w_up_x"],
+                             w["w_down_q"], w["w_down_x"])
+    ref = orc.combine_ffn(x, idx, gate, *[torch.as_tensor(master[n]).to(torch.bfloat16)
+                                          for n in ("w_gate", "w_up", "w_down")])
+    r = np.linalg.norm(out - ref) / np.linalg.norm(ref)
+    assert r < 0.3, r
+
+
+ALL_PINS += [pin_e2m1_codes, pin_mx_quantize_rows, pin_mx_ffn_dense_brute_force, pin_mx_close_to_unquantised]

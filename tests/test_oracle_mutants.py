@@ -35,6 +35,11 @@ MUTANTS = {
     "fp8_h_not_requantised": ("fp8_row_gemm(H, I, qh, sh,", "fp8_row_gemm(H, I, qh, sx,"),
     "shared_gate_up_swapped": ("expert_ffn(j->H, j->I, 0, xt, j->wg, j->wu, j->wd,",
                                "expert_ffn(j->H, j->I, 0, xt, j->wu, j->wg, j->wd,"),
+    "mx_tie_away": ("(d == bd && !(c & 1) && (best & 1))", "(d == bd && c > best)"),
+    "mx_scale_exponent_off": ("int X = ex - 1 - emax;", "int X = ex - emax;"),
+    "mx_act_scale_dropped": ("acc += ldexp(1.0, (int)xa[kb] - 127) * ldexp", "acc += ldexp"),
+    "mx_h_wrong_format": ("oracle_mx_quantize_rows(1, I, h, MX_E4M3, qh, sh);",
+                          "oracle_mx_quantize_rows(1, I, h, MX_E2M1, qh, sh);"),
 }
 
 
