@@ -194,6 +194,52 @@ def make_fp8_weights(cfg: MoEConfig, device="cpu", experts_per_chunk: int = 8):
     return out
 
 
+E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)  # codes 0..7 (OCP MX v1.0)
+
+
+def quantize_blocks_mx_e2m1(w: torch.Tensor):
+    """Input recipe of MX (FP4) expert weights: per row, per 32 values along K, a
+    power-of-two scale 2^X with X = floor(log2(amax)) - 2 (clamped to [-127, 127];
+    X = 0 for an all-zero block), stored as the e8m0 code X + 127, and e2m1 codes of
+    w / 2^X clamped to +-6, rounded to the nearest magnitude with ties to the even
+    code.  One code per byte (sign in bit 3).  Returns (codes uint8 [E,N,K], scale
+    codes uint8 [E,N,K/32])."""
+    E, N, K = w.shape
+    b = w.reshape(E, N, K // 32, 32).double()
+    amax = b.abs().amax(-1)
+    X = (torch.frexp(amax).exponent - 3).clamp(-127, 127)
+    X = torch.where(amax == 0, torch.zeros_like(X), X)
+    r = torch.ldexp(b, -X[..., None]).clamp(-6.0, 6.0)
+    mags = torch.tensor(E2M1_MAGNITUDES, dtype=torch.float64, device=w.device)
+    d = (r.abs()[..., None] - mags).abs() + 1e-12 * (torch.arange(8, device=w.device) & 1)  # ties -> even code
+    c = d.argmin(-1).to(torch.uint8)
+    c = torch.where((r < 0) & (c != 0), c | 8, c)
+    return c.reshape(E, N, K).contiguous(), (X + 127).to(torch.uint8).contiguous()
+
+
+def make_mx_weights(cfg: MoEConfig, device="cpu", experts_per_chunk: int = 8):
+    """MX (FP4) expert weights: drawn like the bf16 ones (fp32 master values ~
+    N(0, 1/sqrt(fan_in)), same streams) and quantised by quantize_blocks_mx_e2m1, a
+    few experts at a time.  Returns {name_q: codes [E,N,K], name_x: scale codes [E,N,K/32]}."""
+    E, I, H = cfg.E, cfg.I, cfg.H
+    out = {}
+    for name, (N, K) in (("w_gate", (I, H)), ("w_up", (I, H)), ("w_down", (H, I))):
+        key = stream_key(cfg.seed, TENSOR_IDS[name])
+        std = 1.0 / math.sqrt(K)
+        q = torch.empty((E, N, K), dtype=torch.uint8, device=device)
+        sx = torch.empty((E, N, K // 32), dtype=torch.uint8, device=device)
+        per = N * K
+        for e0 in range(0, E, experts_per_chunk):
+            e1 = min(E, e0 + experts_per_chunk)
+            v = (normal(key, e0 * per, (e1 - e0) * per, device) * std).to(torch.float32)
+            qq, xx = quantize_blocks_mx_e2m1(v.view(e1 - e0, N, K))
+            q[e0:e1] = qq
+            sx[e0:e1] = xx
+        out[name + "_q"] = q
+        out[name + "_x"] = sx
+    return out
+
+
 def make_inputs(cfg: MoEConfig, device="cpu", weights: bool = True) -> MoEInputs:
     """Draw the workload's tensors in the fixed order x, router_w, [bias], w_gate, w_up, w_down.
 
