@@ -68,3 +68,23 @@ def test_host_argument_errors(L):
     assert L.moe_route(ctypes.byref(d), fake, fake, null, fake, fake, ctypes.c_void_p(addr + 8),
                        1 << 30, null) == 3
     assert L.moe_get_device_status(null, null) == 1
+
+
+def test_workspace_regions_do_not_overlap(L):
+    # the routing regions moe_workspace_offsets reports: 1 KiB aligned, inside the
+    # workspace, and each at least as large as moe.h documents before the next begins
+    for dtype in (api.DTYPE_BF16, api.DTYPE_FP8):
+        for (T, H, I, E, k) in [(16, 2048, 512, 256, 8), (4096, 2048, 512, 256, 8), (8192, 4096, 1408, 64, 6),
+                                (150, 384, 384, 12, 3), (1, 256, 256, 300, 4)]:
+            d = api.dims(T, H, I, E, k)
+            size = api.moe_workspace_size(T, H, I, E, k, dtype)
+            off = (ctypes.c_size_t * 8)()
+            assert L.moe_workspace_offsets(ctypes.byref(d), dtype, off, 8) == 0
+            A = T * k
+            need = [A * 4, A * 4, (E + 1) * 4, A * 4, A * 4, 3 * api.moe_max_tiles(T, H, I, E, k) * 4, 4, T * E * 4]
+            regions = sorted(zip(list(off), need))
+            for (o, n), (o2, _) in zip(regions, regions[1:] + [(size, 0)]):
+                assert o % 1024 == 0, (dtype, T, o)
+                assert o + n <= o2, (dtype, T, o, n, o2)
+    bad = api.dims(4, 100, 512, 8, 2)
+    assert L.moe_workspace_offsets(ctypes.byref(bad), 0, (ctypes.c_size_t * 8)(), 8) == 1
