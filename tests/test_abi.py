@@ -88,3 +88,31 @@ def test_workspace_regions_do_not_overlap(L):
                 assert o + n <= o2, (dtype, T, o, n, o2)
     bad = api.dims(4, 100, 512, 8, 2)
     assert L.moe_workspace_offsets(ctypes.byref(bad), 0, (ctypes.c_size_t * 8)(), 8) == 1
+
+
+def test_header_is_plain_c_and_links(L, tmp_path):
+    # a C99 program includes moe.h, links the library and calls its host-only entry
+    # points (workspace sizing; the argument checks), with warnings as errors
+    import subprocess
+
+    lib_dir = os.path.dirname(api.LIB_PATH)
+    src = tmp_path / "use_moe.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "moe.h"
+int main(void) {
+    moe_dims_t d = {16, 2048, 512, 256, 8};
+    size_t ws = moe_workspace_size(&d, MOE_DTYPE_BF16);
+    int32_t tiles = moe_max_tiles(&d);
+    moe_status_t bad = moe_forward(&d, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL);
+    printf("%zu %d %d\n", ws, (int)tiles, (int)bad);
+    return (ws > 0 && tiles == 1 + 128 && bad == MOE_ERR_INVALID_ARG) ? 0 : 1;
+}
+""")
+    exe = tmp_path / "use_moe"
+    inc = os.path.dirname(HEADER)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", inc, str(src), "-o", str(exe),
+                    "-L", lib_dir, "-lmoe_b200", f"-Wl,-rpath,{lib_dir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert int(r.stdout.split()[0]) == api.moe_workspace_size(16, 2048, 512, 256, 8)
