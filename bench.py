@@ -1,12 +1,17 @@
 """Benchmark of the MoE layer forward on B200: tokens/s of whole layer steps.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|skewed|fp8|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|decode|prefill|skewed|fp8|tiny]
                     [--impl ours|reference] [--schedule ...] [--pair ...] [--swap-ab ...] [--shape K=V,...]
 
 One step = one pass of the whole layer (router softmax top-k, permute, grouped
 gate/up GEMM + SwiGLU, grouped down GEMM, combine) over one batch of seeded
 synthetic inputs already resident in HBM.  L2 is flushed (a 512 MiB write, then a 256 MiB read)
 before every step, outside that step's CUDA-event pair.  Prints one JSON line.
+
+With no --workload (``all``) every workload is timed in turn, K steps each, and the
+line printed is the headline workload's -- Skewed (T=8192, H=4096, E=64, top-6,
+I=1408), the largest configuration and the only compute-bound one -- with the
+other four workloads' lines, each complete, under its ``workloads`` key.
 
 Multi-GPU: the layer does not shard on one node in this design, so N GPUs run N
 independent replicas (one process per GPU, launched by torchrun); the time is the
@@ -38,6 +43,8 @@ if ROOT not in sys.path:
 from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_fp8_weights, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at 1 B200; % of BF16/FP8 TC peak or % of HBM BW"
+HEADLINE = "skewed"                                   # the largest configuration
+ALL_ORDER = ["tiny", "decode", "prefill", "fp8", HEADLINE]   # the headline is timed last
 GEMM_TRACE_CTAS = 1024
 
 
@@ -87,10 +94,13 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=400)
     p.add_argument("--warmup", type=int, default=20)
-    p.add_argument("--workload", default="decode", choices=sorted(CONFIGS))
+    p.add_argument("--workload", default="all", choices=["all"] + sorted(CONFIGS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-budget", type=float, default=None,
+                   help="seconds of oracle work behind each cpu_baseline (default 20, or 12 per "
+                        "workload when all workloads run)")
     p.add_argument("--schedule", default="queue", choices=["queue", "static_items", "static_experts"],
                    help="how the GEMM CTAs get work items: the atomic queue (the design), or a static "
                         "split of the items or of the experts (ablations)")
@@ -103,8 +113,9 @@ def parse():
     return p.parse_args()
 
 
-def workload_config(args):
-    cfg = CONFIGS[args.workload]
+def workload_config(args, name=None):
+    name = name or (HEADLINE if args.workload == "all" else args.workload)
+    cfg = CONFIGS[name]
     if args.shape:
         kw = {}
         for item in args.shape.split(","):
@@ -523,18 +534,11 @@ def config_block(cfg, world):
 
 # ---------------------------------------------------------------- our arm
 
-def main():
-    args = parse()
-    if args.impl == "reference":
-        # rank 0 alone times the oracle on the host cores; the other ranks have no work
-        # and open no process group
-        world, rank, _ = rank_env()
-        run_reference(args, world, rank)
-        return
-    world, rank, local = dist_setup()
+def run_one(args, cfg, world, rank, local):
+    """Times `cfg` (K graph-captured steps after W warm-ups) and returns its JSON line
+    (on every rank; rank 0 prints it)."""
     from routed_grouped_gemm_softmax_b200 import api
 
-    cfg = workload_config(args)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     fp8 = cfg.dtype == "fp8"
@@ -685,8 +689,10 @@ def main():
     clocks = sampler.summary(t_wall0, t_wall1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(cfg, host_inputs(cfg, inp, w8 if fp8 else None))
+        budget = args.cpu_budget if args.cpu_budget else (12.0 if args.workload == "all" else 20.0)
+        cpu = cpu_baseline(cfg, host_inputs(cfg, inp, w8 if fp8 else None), budget_s=budget)
 
+    line = None
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 5),
@@ -697,6 +703,42 @@ def main():
                 "e2e": e2e, "gpu_launches": kernels_per_forward(cfg) * args.steps, "schedule": sched,
                 "clocks": clocks, "cpu_baseline": cpu,
                 "p99_ms_per_step": round(sorted(step_ms)[min(len(step_ms) - 1, math.ceil(0.99 * len(step_ms)) - 1)], 5)}
+    torch.cuda.synchronize()
+    return line
+
+
+def run_and_release(args, cfg, world, rank, local):
+    """run_one, then hand this workload's device memory back before the next is drawn."""
+    import gc
+    line = run_one(args, cfg, world, rank, local)
+    gc.collect()
+    torch.cuda.empty_cache()
+    return line
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        # rank 0 alone times the oracle on the host cores; the other ranks have no work
+        # and open no process group
+        world, rank, _ = rank_env()
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(torch.device("cuda", local))
+    if args.workload != "all":
+        line = run_one(args, workload_config(args), world, rank, local)
+    else:
+        # every workload in turn, the headline last; one line: the headline's, with the
+        # others' complete lines under "workloads"
+        lines = {name: run_and_release(args, workload_config(args, name), world, rank, local)
+                 for name in ALL_ORDER}
+        line = lines[HEADLINE]
+        if line is not None:
+            line["workloads"] = {n: lines[n] for n in ALL_ORDER if n != HEADLINE}
+            line["headline"] = (f"{HEADLINE}: the largest configuration (the metric names none); "
+                                f"the other workloads under 'workloads'")
+    if rank == 0:
         print(json.dumps(line), flush=True)
     dist_teardown(world)
 

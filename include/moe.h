@@ -222,6 +222,14 @@ void moe_set_gemm_trace(unsigned long long *trace, int32_t ctas);
  * context stays usable.  Process-wide; for tests only. */
 void moe_set_wait_limit_us(int32_t us, int32_t stall_test);
 
+/* Router audit hook for tests.  With `logits` and `bounds` device buffers of at
+ * least `capacity` fp32 values, every later certified router run (batches of more
+ * than 32 tokens, T*E <= capacity) also writes, for every (t, e), the tensor-core
+ * logit plus bias to logits[t*E + e] and the rounding-error bound it uses for that
+ * logit to bounds[t*E + e], so a test can check |chain - logit| <= bound for every
+ * pair, chosen or not.  NULL (or capacity <= 0) turns it off.  Process-wide. */
+void moe_set_router_audit(float *logits, float *bounds, int64_t capacity);
+
 /* Stage timing hook for benchmarks.  With `events` pointing at MOE_STAGE_EVENTS
  * caller-created cudaEvent_t handles (passed as void*), every later moe_forward
  * records them on its stream at the stage boundaries: [0] start, [1] routed,
@@ -244,7 +252,9 @@ void moe_set_stage_events(void *const *events, int32_t n);
  *    MOE_ERR_TOO_LARGE (with H=2048, I=512, E=256, top_k=8 that is above
  *    182 tokens); invalid dims give the same errors as moe_forward.
  *  - The first call made with a device current looks up the array's device
- *    address on that device; make that first call before any stream capture.
+ *    address on that device and keeps it for the life of the process; make that
+ *    first call before any stream capture, and make no call after a reset of
+ *    that device (cudaDeviceReset), which would leave the kept address stale.
  *  - Nothing is allocated, freed or synchronised.  Every call shares the one
  *    array and leaves its contents behind; the parts that must start at zero
  *    are cleared by each call.  Calls whose GPU work overlaps (other streams,

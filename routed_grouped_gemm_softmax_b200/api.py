@@ -23,7 +23,7 @@ EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "m
            "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order", "moe_set_gemm_trace",
            "moe_set_pair_mma", "moe_set_fp8_swap_ab",
            "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",
-           "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets"]
+           "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets", "moe_set_router_audit"]
 DTYPE_BF16, DTYPE_FP8 = 0, 1
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
@@ -85,6 +85,8 @@ def lib():
         L.moe_workspace_offsets.restype = ctypes.c_int
         L.moe_set_wait_limit_us.argtypes = [I32, I32]
         L.moe_set_wait_limit_us.restype = None
+        L.moe_set_router_audit.argtypes = [P, P, ctypes.c_int64]
+        L.moe_set_router_audit.restype = None
         L.moe_forward_noalloc.argtypes = [D, P, P, P, P, P, P, P, P]
         L.moe_forward_noalloc.restype = ctypes.c_int
         _lib = L
@@ -332,3 +334,15 @@ def set_stage_events(events):
                                             for e in events])
     set_stage_events._keep = arr
     lib().moe_set_stage_events(arr, len(events))
+
+
+def set_router_audit(logits, bounds):
+    """Every later certified router run (T > 32) writes each (t, e)'s tensor-core logit
+    (+bias) into `logits` and its error bound into `bounds` (CUDA fp32 tensors of
+    T*E values or more); None turns it off."""
+    if logits is None:
+        lib().moe_set_router_audit(None, None, 0)
+        return
+    if logits.dtype != torch.float32 or bounds.dtype != torch.float32 or not (logits.is_cuda and bounds.is_cuda):
+        raise ValueError("router audit buffers: CUDA float32 tensors")
+    lib().moe_set_router_audit(_p(logits), _p(bounds), min(logits.numel(), bounds.numel()))

@@ -26,6 +26,9 @@ std::atomic<int> g_fp8_swap{0};   // 0 auto, 1 swapped fp8 gate/up GEMM always, 
 std::atomic<int> g_trace_ctas{0};
 std::atomic<unsigned long long> g_wait_ns{0};
 std::atomic<int> g_stall_test{0};
+std::mutex g_audit_mu;
+float *g_audit_v = nullptr, *g_audit_d = nullptr;  // router audit buffers (test hook)
+int64_t g_audit_cap = 0;
 std::mutex g_ev_mu;
 cudaEvent_t g_stage_ev[MOE_STAGE_EVENTS];
 bool g_stage_on = false;
@@ -148,10 +151,16 @@ T *at(void *ws, size_t off)
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-moe::RouterScratch router_scratch(void *ws, const moe::WsLayout &L)
+moe::RouterScratch router_scratch(void *ws, const moe::WsLayout &L, const moe_dims_t &d)
 {
-    return moe::RouterScratch{at<__nv_bfloat16>(ws, L.wrt), at<float>(ws, L.wsq), at<int32_t>(ws, L.rncand),
-                              at<moe::RouterCand>(ws, L.rlist)};
+    moe::RouterScratch rs{at<__nv_bfloat16>(ws, L.wrt), at<float>(ws, L.wsq), at<int32_t>(ws, L.rncand),
+                          at<moe::RouterCand>(ws, L.rlist), nullptr, nullptr};
+    std::lock_guard<std::mutex> lk(g_audit_mu);
+    if (g_audit_v && (int64_t)d.T * d.E <= g_audit_cap) {
+        rs.audit_v = g_audit_v;
+        rs.audit_d = g_audit_d;
+    }
+    return rs;
 }
 
 // Activations, weights and outputs are read and written in 16-byte vectors (and the
@@ -180,7 +189,7 @@ cudaError_t route_and_permute(const moe_dims_t &d, const moe::WsLayout &L, const
         return e == cudaSuccess ? marks.mark(1, st) : e;
     }
     cudaError_t e =
-        moe::launch_route(d, xb, wb, router_bias, at<float>(ws, L.logits), idx, gate, router_scratch(ws, L), hdr, st);
+        moe::launch_route(d, xb, wb, router_bias, at<float>(ws, L.logits), idx, gate, router_scratch(ws, L, d), hdr, st);
     if (e == cudaSuccess) e = marks.mark(1, st);
     if (e == cudaSuccess)
         e = moe::launch_permute(d, L, idx, at<int32_t>(ws, L.blk_cnt), at<int32_t>(ws, L.blk_base),
@@ -286,6 +295,15 @@ void moe_set_wait_limit_us(int32_t us, int32_t stall_test)
     g_stall_test.store(stall_test ? 1 : 0);
 }
 
+void moe_set_router_audit(float *logits, float *bounds, int64_t capacity)
+{
+    std::lock_guard<std::mutex> lk(g_audit_mu);
+    const bool on = logits && bounds && capacity > 0;
+    g_audit_v = on ? logits : nullptr;
+    g_audit_d = on ? bounds : nullptr;
+    g_audit_cap = on ? capacity : 0;
+}
+
 void moe_set_stage_events(void *const *events, int32_t n)
 {
     std::lock_guard<std::mutex> lk(g_ev_mu);
@@ -308,7 +326,7 @@ moe_status_t moe_route(const moe_dims_t *d, const void *x, const void *router_w,
     cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
     if (e == cudaSuccess)
         e = moe::launch_route(*d, static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(router_w),
-                              router_bias, at<float>(ws, L.logits), topk_idx, topk_w, router_scratch(ws, L),
+                              router_bias, at<float>(ws, L.logits), topk_idx, topk_w, router_scratch(ws, L, *d),
                               at<moe::WsHeader>(ws, 0), st);
     return cuda_status(e);
 }

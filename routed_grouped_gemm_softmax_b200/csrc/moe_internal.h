@@ -107,6 +107,8 @@ struct RouterScratch {
     float *wsq;          // [ceil(H/256), E] partial squared column norms
     int32_t *ncand;      // [T] candidates per token
     RouterCand *list;    // [T, E] candidates of each token, ascending expert index
+    float *audit_v;      // test hook, or null: [T, E] tensor-core logit (+bias) of every (t, e)
+    float *audit_d;      // test hook, or null: [T, E] its rounding-error bound
 };
 
 // Router: for T <= 32 the CUDA-core fp32 chains (route.cu); above, tensor-core

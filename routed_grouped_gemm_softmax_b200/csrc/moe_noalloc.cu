@@ -30,7 +30,9 @@ void *g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address must come from the
-// runtime; it is looked up once per device and cached.
+// runtime; it is looked up once per device and cached for the life of the
+// process (a reset of the device would make the cached address stale, so no call
+// may follow one).
 moe_status_t scratch_on_current_device(void **ptr)
 {
     int dev = 0;

@@ -105,6 +105,7 @@ struct CertifyArgs {
     int32_t *idx;
     float *gate;
     int32_t *status;
+    float *audit_v, *audit_d;  // null, or [T, E]: every tensor-core logit and its bound
     int xrows;              // rows of an x tile (TB rounded up to 8)
     int erows;              // staged router rows (E rounded up to 8, or to 256 above 256)
     int ebox;               // rows of one router tile (<= 256)
@@ -207,6 +208,10 @@ __global__ void __launch_bounds__(kCertThreads)
                 d[i] = a.eps * xn * sqrtf(wsq[e]) * 1.001f + fabsf(s) * 4.8e-7f + 1e-30f;
                 lo[i] = v[i] - d[i];
                 key[i] = order_key(lo[i]);
+                if (a.audit_v) {
+                    a.audit_v[(size_t)t * E + e] = v[i];
+                    a.audit_d[(size_t)t * E + e] = d[i];
+                }
             } else {
                 v[i] = -INFINITY;
                 d[i] = 0.0f;
@@ -437,7 +442,8 @@ cudaError_t launch_route_certified(const moe_dims_t &d, const __nv_bfloat16 *x, 
     if (!encode_sw128_2d_bf16(&tm_x, x, T, H, xrows) || !encode_sw128_2d_bf16(&tm_w, rs.wrt, E, H, ebox))
         return cudaErrorInvalidValue;
     CertifyArgs a{logits, logits, ks, x, rs.wsq, bias, nparts, T, H, E, k, tb, eps, rs.ncand, rs.list,
-                  idx, gate, &hdr->status, xrows, erows, ebox, nbx, stages, nbx * (xrows + erows) * 128};
+                  idx, gate, &hdr->status, rs.audit_v, rs.audit_d, xrows, erows, ebox, nbx, stages,
+                  nbx * (xrows + erows) * 128};
     const int grid = (T + tb - 1) / tb;
     const int vpl = (E + 31) / 32;
     if (vpl <= 1) return launch_certify<1>(tm_x, tm_w, a, grid, st);

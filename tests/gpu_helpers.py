@@ -60,3 +60,12 @@ def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:
     rng = np.random.default_rng(seed)
     s = set([0, T - 1]) | set(rng.choice(T, size=min(n, T), replace=False).tolist())
     return np.array(sorted(s), dtype=np.int32)
+
+
+def hot_expert_tokens(idx_ref: np.ndarray, n: int, seed: int = 0) -> np.ndarray:
+    """A seeded sample of n tokens routed to the most popular expert (its group spans
+    the most m-tiles, and on deep groups the pair-of-CTA tiles)."""
+    hot = int(np.bincount(idx_ref.reshape(-1)).argmax())
+    toks = np.nonzero((idx_ref == hot).any(axis=1))[0]
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(toks, size=min(n, toks.size), replace=False)).astype(np.int32)

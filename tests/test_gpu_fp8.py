@@ -105,11 +105,15 @@ def test_fp8_full_size_sampled():
     cfg = CONFIGS["fp8"]
     inp, w = _fp8_case(cfg)
     out = _run_fp8(cfg, inp, w)
-    tok = sample_tokens(cfg.T, 6, seed=cfg.seed)
+    tok = sample_tokens(cfg.T, 128, seed=cfg.seed)
+    assert tok.size >= 128
     ref, idx, gate = _oracle_fp8(cfg, inp, w, tokens=tok)
     i_g, w_g = api.moe_route(inp.x, inp.router_w, None, cfg.top_k)
     compare_routing(i_g, w_g, idx, gate, "fp8")
-    r = rel_l2(out[torch.as_tensor(tok, device="cuda").long()], ref)
+    o = out[torch.as_tensor(tok, device="cuda").long()]
+    r = rel_l2(o, ref)
+    max_abs = float(np.abs(o.float().cpu().double().numpy() - ref).max())
+    print(f"fp8 full size: {tok.size} tokens, rel_l2={r:.3e} max_abs={max_abs:.3e} (reported)")
     assert r <= FP8_REL_L2, f"fp8 full size: rel_l2={r:.3e}"
 
 

@@ -10,7 +10,7 @@ import torch
 
 import oracle
 from gpu_helpers import (compare_out, compare_permute, compare_routing, device_inputs,
-                         sample_tokens)
+                         hot_expert_tokens, sample_tokens)
 from routed_grouped_gemm_softmax_b200 import api
 from routed_grouped_gemm_softmax_b200.inputs import CONFIGS
 
@@ -132,6 +132,11 @@ def test_schedule_independence(T):
         api.set_claim_order(False)
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    # and the common result against the oracle
+    _, c = device_inputs(cfg)
+    idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], cfg.top_k)
+    compare_out(outs[0], oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"]),
+                f"sched T={T}")
 
 
 PAIR_CASES = {
@@ -286,7 +291,9 @@ def test_empty_batch_is_noop():
 @pytest.mark.parametrize("name", ["decode", "prefill", "skewed"])
 def test_full_size(name):
     """Full-size workloads: routing, permutation and offsets bit-exact for every token;
-    the layer output checked on a sample of tokens the oracle evaluates one by one."""
+    the layer output checked on a sample of tokens the oracle evaluates one by one --
+    at least 256 tokens (every token of Decode), 64 of them routed to the most popular
+    expert, whose group spans the most tiles (on Skewed, pair-of-CTA tiles)."""
     cfg = CONFIGS[name]
     g, c = device_inputs(cfg)
     k = cfg.top_k
@@ -297,6 +304,8 @@ def test_full_size(name):
     ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, "cuda")
     out = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k, ws=ws)
     assert api.moe_get_device_status(ws) == api.MOE_OK
-    tok = sample_tokens(cfg.T, 24, seed=cfg.seed)
+    tok = np.union1d(sample_tokens(cfg.T, 192, seed=cfg.seed), hot_expert_tokens(idx_ref, 64, seed=cfg.seed))
+    assert tok.size >= min(cfg.T, 256)
     ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"], tokens=tok)
-    compare_out(out[torch.as_tensor(tok, device="cuda").long()], ref, name)
+    max_abs, rel = compare_out(out[torch.as_tensor(tok, device="cuda").long()], ref, name)
+    print(f"full size {name}: {tok.size} tokens, max_abs={max_abs:.3e} rel_l2={rel:.3e}")
