@@ -79,7 +79,7 @@ typedef struct {
     int32_t top_k;  /* experts per token */
 } moe_dims_t;
 
-enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8 = 1 };
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8 = 1, MOE_DTYPE_MX = 2 };
 
 /* Rows of the GEMM tiles; tile_list entries cover at most this many rows. */
 #define MOE_TILE_ROWS 128
@@ -131,6 +131,26 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
                          const float *router_bias, const void *w_gate, const void *w_up,
                          const void *w_down, void *out, void *ws, size_t ws_bytes, void *stream);
 
+/* The layer with a shared expert (GC-MoE page, compute-partition section: the
+ * block-scaled expert kernel with "optional shared experts" fused in).  Besides the
+ * k routed experts, every token passes through one shared SwiGLU expert with gate
+ * weight 1:
+ *   out[t] = sum_j gate[t,j] * FFN_{S_t[j]}(x_t)  +  W_sd ( silu(W_sg x_t) * (W_su x_t) )
+ *   shared_gate, shared_up [shared_I, H] bf16, shared_down [H, shared_I] bf16.
+ * shared_I must be a positive multiple of I (0 = no shared expert: moe_forward).  The
+ * shared expert runs inside the same two grouped GEMM launches as the routed ones,
+ * as shared_I / I further "experts" of I columns each that every token is routed to;
+ * its per-slice outputs are rounded to bf16 like the routed experts' and added after
+ * the gate-weighted routed sum (fp32, slices in order), then out is rounded to bf16.
+ * The workspace must hold moe_workspace_size_shared(d, shared_I) bytes; other rules
+ * as moe_forward.  bf16 only. */
+size_t moe_workspace_size_shared(const moe_dims_t *d, int32_t shared_I);
+moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *router_w,
+                                const float *router_bias, const void *w_gate, const void *w_up,
+                                const void *w_down, int32_t shared_I, const void *shared_gate,
+                                const void *shared_up, const void *shared_down, void *out, void *ws,
+                                size_t ws_bytes, void *stream);
+
 /* FP8 block-scaled layer (GC-MoE page: block-scaled FP8 MMA on Blackwell with
  * SwiGLU and requantisation fused; vLLM fused-MoE page, section 03: fp8 weights
  * in [128,128] blocks).  Routing is the bf16 router of moe_route.  Weights are
@@ -149,6 +169,33 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
                              const float *router_bias, const uint8_t *w_gate_q, const float *w_gate_s,
                              const uint8_t *w_up_q, const float *w_up_s, const uint8_t *w_down_q,
                              const float *w_down_s, void *out, void *ws, size_t ws_bytes, void *stream);
+
+/* MX (microscaling) layer with FP4 weights (GC-MoE page, compute-partition
+ * section: block-scaled FP8/FP4 MMAs on Blackwell with the operands swapped and
+ * SwiGLU and requantisation fused).  Formats of the OCP Microscaling spec: weights
+ * are e2m1 codes, two per byte (the code of element 2i in the low nibble of byte i,
+ * of element 2i+1 in the high nibble), with one e8m0 scale code per 32 elements
+ * along K; the scale of a block is 2^(code - 127):
+ *   w_gate_p / w_up_p [E, I, H/2] with w_gate_x / w_up_x [E, I, H/32],
+ *   w_down_p [E, H, I/2] with w_down_x [E, H, I/32]   (uint8).
+ * x (bf16) is quantised per token per 32 columns to MX e4m3: X = floor(log2 amax)
+ * - 8 clamped to [-127, 127] (X = 0 and zero codes for an all-zero block), codes =
+ * e4m3 round-to-nearest-even of clamp(v / 2^X, -448, 448), scale code X + 127.
+ * Each GEMM is the sum over 32-wide K blocks of 2^(Xa + Xw) * (codes . codes),
+ * accumulated in fp32 on the tensor cores (kind::mxf8f6f4 with block scaling); h
+ * = silu(gate) * up (fp32) is requantised to MX e4m3 the same way; the down GEMM's
+ * per-assignment rows are rounded to bf16 and combined as in moe_forward.  Routing
+ * is the bf16 router of moe_route.  Needs H and I multiples of 512 and ws_bytes >=
+ * moe_workspace_size(d, MOE_DTYPE_MX); other rules as moe_forward. */
+moe_status_t moe_forward_mx(const moe_dims_t *d, const void *x, const void *router_w,
+                            const float *router_bias, const uint8_t *w_gate_p, const uint8_t *w_gate_x,
+                            const uint8_t *w_up_p, const uint8_t *w_up_x, const uint8_t *w_down_p,
+                            const uint8_t *w_down_x, void *out, void *ws, size_t ws_bytes, void *stream);
+
+/* The activation quantiser of moe_forward_mx on its own: a [R, K] bf16 (K a
+ * multiple of 32, 16-byte aligned) -> q [R, K] e4m3 codes and x [R, K/32] e8m0 scale
+ * codes, per row per 32 columns as described above.  Needs no workspace. */
+moe_status_t moe_quantize_rows_mx(int32_t R, int32_t K, const void *a, uint8_t *q, uint8_t *x, void *stream);
 
 /* The activation quantiser of moe_forward_fp8 on its own: a [R, K] bf16 (K a
  * multiple of 128, 16-byte aligned) -> q [R, K] e4m3 codes and s [R, K/128]

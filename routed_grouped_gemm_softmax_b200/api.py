@@ -23,7 +23,8 @@ EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "m
            "moe_get_device_status", "moe_set_gemm_ctas", "moe_set_claim_order", "moe_set_gemm_trace",
            "moe_set_pair_mma", "moe_set_fp8_swap_ab",
            "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",
-           "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets", "moe_set_router_audit"]
+           "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets", "moe_set_router_audit",
+           "moe_forward_shared", "moe_workspace_size_shared"]
 DTYPE_BF16, DTYPE_FP8 = 0, 1
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
@@ -85,6 +86,10 @@ def lib():
         L.moe_workspace_offsets.restype = ctypes.c_int
         L.moe_set_wait_limit_us.argtypes = [I32, I32]
         L.moe_set_wait_limit_us.restype = None
+        L.moe_forward_shared.argtypes = [D, P, P, P, P, P, P, I32, P, P, P, P, P, SZ, P]
+        L.moe_forward_shared.restype = ctypes.c_int
+        L.moe_workspace_size_shared.argtypes = [D, I32]
+        L.moe_workspace_size_shared.restype = SZ
         L.moe_set_router_audit.argtypes = [P, P, ctypes.c_int64]
         L.moe_set_router_audit.restype = None
         L.moe_forward_noalloc.argtypes = [D, P, P, P, P, P, P, P, P]
@@ -192,6 +197,43 @@ def moe_forward(x, router_w, bias, w_gate, w_up, w_down, top_k: int, out=None, w
     _check(lib().moe_forward(ctypes.byref(d), _p(x), _p(router_w), _p(bias), _p(w_gate), _p(w_up),
                              _p(w_down), _p(out), _p(ws), ws.numel(), _stream(stream, dev)),
            "moe_forward")
+    return out
+
+
+def moe_workspace_size_shared(T, H, I, E, top_k, shared_I) -> int:
+    return int(lib().moe_workspace_size_shared(ctypes.byref(dims(T, H, I, E, top_k)), int(shared_I)))
+
+
+def moe_forward_shared(x, router_w, bias, w_gate, w_up, w_down, shared_gate, shared_up, shared_down, top_k: int,
+                       out=None, ws=None, stream=None):
+    """The MoE layer forward with a shared expert (shared_gate/up [shared_I, H], shared_down
+    [H, shared_I] bf16, shared_I a multiple of I); returns out bf16 [T,H]."""
+    T, H = x.shape
+    E, I, _ = w_gate.shape
+    SI = shared_gate.shape[0]
+    dev = x.device
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(router_w, torch.bfloat16, (H, E), "router_w")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "router_bias")
+    _need(w_gate, torch.bfloat16, (E, I, H), "w_gate")
+    _need(w_up, torch.bfloat16, (E, I, H), "w_up")
+    _need(w_down, torch.bfloat16, (E, H, I), "w_down")
+    _need(shared_gate, torch.bfloat16, (SI, H), "shared_gate")
+    _need(shared_up, torch.bfloat16, (SI, H), "shared_up")
+    _need(shared_down, torch.bfloat16, (H, SI), "shared_down")
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    _need(out, torch.bfloat16, (T, H), "out")
+    if ws is None:
+        n = moe_workspace_size_shared(T, H, I, E, top_k, SI)
+        if n == 0:
+            raise MoEError(1, "moe_workspace_size_shared")
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    d = dims(T, H, I, E, top_k)
+    _check(lib().moe_forward_shared(ctypes.byref(d), _p(x), _p(router_w), _p(bias), _p(w_gate), _p(w_up),
+                                    _p(w_down), int(SI), _p(shared_gate), _p(shared_up), _p(shared_down), _p(out),
+                                    _p(ws), ws.numel(), _stream(stream, dev)),
+           "moe_forward_shared")
     return out
 
 

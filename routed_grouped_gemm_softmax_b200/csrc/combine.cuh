@@ -19,13 +19,16 @@
 namespace moe {
 
 // out[t, col .. col+7] = bf16(sum_j gate[t,j] * y[t*k + j, col .. col+7]), fp32 fma in
-// ascending j from 0.  Columns at or past N are skipped (N is a multiple of 8).
+// ascending j from 0, then (a shared expert, sh_count > 0) + y[sh_rows0 + s*T + t, ..]
+// for s ascending, each at gate 1.  Columns at or past N are skipped (N is a
+// multiple of 8).
 // FUSED: y was written by other CTAs of the running kernel, so its rows are read
 // from L2 (ld.global.cg), eight rows' loads in flight at once since a lone warp
 // does the work; the standalone kernel relies on its many resident warps instead.
 template <bool FUSED>
 __device__ __forceinline__ void combine_cols(const __nv_bfloat16 *__restrict__ y, const float *__restrict__ gate,
-                                             __nv_bfloat16 *__restrict__ out, int t, int k, int N, int col)
+                                             __nv_bfloat16 *__restrict__ out, int t, int k, int N, int col,
+                                             int sh_count = 0, int T = 0, int sh_rows0 = 0)
 {
     if (col >= N) return;
     float acc[8];
@@ -58,6 +61,10 @@ __device__ __forceinline__ void combine_cols(const __nv_bfloat16 *__restrict__ y
         for (int j = 0; j < k; ++j)
             accumulate(gate[(size_t)t * k + j], *reinterpret_cast<const uint4 *>(y + ((size_t)t * k + j) * N + col));
     }
+    for (int s = 0; s < sh_count; ++s) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(y + ((size_t)sh_rows0 + (size_t)s * T + t) * N + col);
+        accumulate(1.0f, FUSED ? __ldcg(p) : *p);
+    }
     uint4 o;
     __nv_bfloat162 *q = reinterpret_cast<__nv_bfloat162 *>(&o);
 #pragma unroll
@@ -67,14 +74,15 @@ __device__ __forceinline__ void combine_cols(const __nv_bfloat16 *__restrict__ y
 
 // Called by a whole warp after its lanes wrote their y rows of n-tile nt (flat row
 // `flat`, or `has_row` false): counts the arrivals and runs the combines they
-// complete.  cnt is [T, ntiles]; `target` arrivals complete a (token, n-tile).
+// complete.  cnt is [T, ntiles]; `target` arrivals complete a (token, n-tile) --
+// k, plus sh_count for a shared expert, whose rows sh_rows0 + s*T + t follow.
 // Not inlined, so its registers do not add to the epilogue's accumulator pressure.
 static __device__ __noinline__ void combine_arrive(const __nv_bfloat16 *__restrict__ y, const float *__restrict__ gate,
                                                __nv_bfloat16 *__restrict__ out, int32_t *__restrict__ cnt, int k,
                                                int target, int N, int ntiles, int nt, bool has_row, int flat,
-                                               int lane)
+                                               int lane, int sh_count = 0, int T = 0, int sh_rows0 = 0)
 {
-    const int tok = has_row ? flat / k : 0;
+    const int tok = !has_row ? 0 : (sh_count == 0 || flat < sh_rows0) ? flat / k : (flat - sh_rows0) % T;
     bool last = false;
     if (has_row) {
         __threadfence();  // this thread's y row before its arrival
@@ -88,7 +96,7 @@ static __device__ __noinline__ void combine_arrive(const __nv_bfloat16 *__restri
         const int src = __ffs(m) - 1;
         m &= m - 1u;
         const int t = __shfl_sync(0xffffffffu, tok, src);
-        combine_cols<true>(y, gate, out, t, k, N, nt * 256 + lane * 8);  // the n-tile's 256 columns
+        combine_cols<true>(y, gate, out, t, k, N, nt * 256 + lane * 8, sh_count, T, sh_rows0);  // 256 columns
     }
 }
 

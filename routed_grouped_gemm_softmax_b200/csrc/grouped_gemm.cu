@@ -84,7 +84,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB0,
-                    const __grid_constant__ CUtensorMap tmB1, const GemmArgs g)
+                    const __grid_constant__ CUtensorMap tmB1, const GemmArgs g, const __grid_constant__ SharedMaps sm)
 {
     // output columns per tile: mode 0 packs 128 gate + 128 up columns into N=256
     constexpr int BNO = MODE == 0 ? BN / 2 : BN;
@@ -118,6 +118,10 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
         for (int b = 0; b < kABoxes; ++b) tma_prefetch_desc(&tmA.m[b]);
         tma_prefetch_desc(&tmB0);
         if (MODE == 0) tma_prefetch_desc(&tmB1);
+        if (g.sh_count) {
+            tma_prefetch_desc(&sm.b0);
+            if (MODE == 0) tma_prefetch_desc(&sm.b1);
+        }
     }
     if (warp == 1) tmem_alloc(&S->tmem_base, TMEM_COLS);
     tc_fence_before();
@@ -135,7 +139,9 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
     if (warp == 0) {
         // ------------------------------------------------ scheduler + TMA producer
         if (lane == 0) {
-            const int total = (dense ? (g.M + BM - 1) / BM : *g.ntiles) * n_tiles;
+            const int nrouted = dense ? 0 : *g.ntiles;
+            const int sh_tps = g.sh_count ? (g.sh_T + BM - 1) / BM : 1;
+            const int total = (dense ? (g.M + BM - 1) / BM : nrouted + g.sh_count * sh_tps) * n_tiles;
             int stage = 0, rs = 0;
             uint32_t phase = 0, rphase = 0;
             uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
@@ -143,16 +149,22 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
             int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
             bool held = kEarlyB;  // A loads of the first item's first stages wait for the previous kernel
             for (;;) {
-                const int item = claim_item(g.reverse, g.counter, total, n_tiles, dense ? nullptr : g.tiles, cursor);
+                const int item = claim_item(g.reverse, g.counter, total, n_tiles, dense ? nullptr : g.tiles, cursor,
+                                            nrouted, g.sh_e0, sh_tps);
                 if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
                 S->ring[rs] = item;
                 mbar_arrive(&S->itf[rs]);
                 if (++rs == RING) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
                 const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
-                const int expert = dense ? 0 : g.tiles[3 * mt], row0 = dense ? mt * BM : g.tiles[3 * mt + 1];
-                const int rows = dense ? min(BM, g.M - row0) : g.tiles[3 * mt + 2];
-                const int ab = a_box(rows);  // the A box that covers the tile's rows
+                TileRef tr{0, mt * BM, 0, mt * BM, -1};
+                if (dense)
+                    tr.rows = min(BM, g.M - tr.row0);
+                else
+                    tr = tile_ref(g.tiles, nrouted, mt, BM, MODE, g.sh_T, g.sh_rows0, g.sh_e0);
+                const int expert = tr.e, arow0 = tr.arow0;
+                const int ab = a_box(tr.rows);  // the A box that covers the tile's rows
+                const CUtensorMap *amap = (MODE == 0 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
                 const int n0 = nt * BNO;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
@@ -160,15 +172,22 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     uint8_t *b_dst = sB + stage * B_BYTES;
-                    if (!held) tma_load_2d(sA + stage * A_BYTES, &tmA.m[ab], &S->full[stage], kb * BK, row0);
-                    tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
-                    if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
+                    if (!held) tma_load_2d(sA + stage * A_BYTES, amap, &S->full[stage], kb * BK, arow0);
+                    if (tr.s < 0) {
+                        tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
+                        if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
+                    } else if (MODE == 0) {  // shared slice s: rows s*I + n0.. of the shared gate / up
+                        tma_load_2d(b_dst, &sm.b0, &S->full[stage], kb * BK, tr.s * g.N + n0);
+                        tma_load_2d(b_dst + B_BYTES / 2, &sm.b1, &S->full[stage], kb * BK, tr.s * g.N + n0);
+                    } else {  // shared down: columns s*I + kb*BK..
+                        tma_load_2d(b_dst, &sm.b0, &S->full[stage], tr.s * g.K + kb * BK, n0);
+                    }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                     if (held && kb + 1 == min(STAGES, num_kb)) {  // first item: stage j holds K block j
                         pdl_wait();
                         held = false;
                         for (int j = 0; j <= kb; ++j)
-                            tma_load_2d(sA + j * A_BYTES, &tmA.m[ab], &S->full[j], j * BK, row0);
+                            tma_load_2d(sA + j * A_BYTES, amap, &S->full[j], j * BK, arow0);
                     }
                 }
                 if (!ok) break;
@@ -231,6 +250,7 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
         const int row = q * 32 + lane;
         int rs = 0, acc = 0;
         uint32_t rphase = 0, aphase = 0;
+        const int nrouted = dense ? 0 : *g.ntiles;
         for (;;) {
             if (!mbar_wait(&S->itf[rs], rphase, g.wait_ns)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
             const int item = S->ring[rs];
@@ -239,9 +259,17 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
             if (++rs == RING) { rs = 0; rphase ^= 1; }
             if (item < 0) break;
             const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
-            const int row0 = dense ? mt * BM : g.tiles[3 * mt + 1];
-            const int rows = dense ? min(BM, g.M - row0) : g.tiles[3 * mt + 2];
+            int row0 = mt * BM, rows = 0;
+            if (dense) {
+                rows = min(BM, g.M - row0);
+            } else {
+                const TileRef tr = tile_ref(g.tiles, nrouted, mt, BM, MODE, g.sh_T, g.sh_rows0, g.sh_e0);
+                row0 = tr.row0;
+                rows = tr.rows;
+            }
             const bool row_ok = row < rows;
+            // y row of sorted row r: the row map's for the routed rows, r itself for the shared expert's
+            auto flat_of = [&](int r) { return (g.sh_count == 0 || r < g.sh_rows0) ? g.row_map[r] : r; };
             if (!mbar_wait(&S->accf[acc], aphase, g.wait_ns)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
             tc_fence_after();
             const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
@@ -286,7 +314,7 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                     }
                 }
             } else {
-                const int flat = row_ok ? g.row_map[row0 + row] : 0;
+                const int flat = row_ok ? flat_of(row0 + row) : 0;
                 __nv_bfloat16 *orow = g.out + (size_t)flat * g.N;
 #pragma unroll 1
                 for (int c = 0; c < BNO / 32; ++c) {
@@ -309,7 +337,7 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
             if (++acc == 2) { acc = 0; aphase ^= 1; }
             if (MODE == 1 && g.comb_cnt)  // the accumulator is already released
                 combine_arrive(g.out, g.comb_gate, g.comb_out, g.comb_cnt, g.comb_k, g.comb_target, g.N, n_tiles,
-                               nt, row_ok, row_ok ? g.row_map[row0 + row] : 0, lane);
+                               nt, row_ok, row_ok ? flat_of(row0 + row) : 0, lane, g.sh_count, g.sh_T, g.sh_rows0);
         }
     }
 
@@ -354,17 +382,20 @@ static bool smem_attr_ready(int mode)
 }
 
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
-                                const CUtensorMap &tmB1, cudaStream_t st)
+                                const CUtensorMap &tmB1, cudaStream_t st, const SharedMaps *sm)
 {
     const int grid = g.ctas > 0 ? g.ctas : num_sms();
     if (!smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
+    if (g.sh_count && (!sm || g.mode == 2)) return cudaErrorInvalidValue;
+    static const SharedMaps none{};
+    const SharedMaps &s = sm ? *sm : none;
     cudaError_t e;
     if (g.mode == 0)
-        e = launch_pdl(grouped_gemm_kernel<0>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g);
+        e = launch_pdl(grouped_gemm_kernel<0>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s);
     else if (g.mode == 1)
-        e = launch_pdl(grouped_gemm_kernel<1>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g);
+        e = launch_pdl(grouped_gemm_kernel<1>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s);
     else
-        e = launch_pdl(grouped_gemm_kernel<2>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g);
+        e = launch_pdl(grouped_gemm_kernel<2>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s);
     return e;
 }
 

@@ -174,7 +174,7 @@ template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
     grouped_gemm_2cta_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB0,
                              const __grid_constant__ CUtensorMap tmB1, const GemmArgs g, const int32_t *tiles2,
-                             const int32_t *ntiles2)
+                             const int32_t *ntiles2, const __grid_constant__ SharedMaps sm)
 {
     constexpr int BNO = MODE == 0 ? BN2 / 2 : BN2;  // output columns per item
     extern __shared__ uint8_t smem2[];
@@ -206,6 +206,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
         for (int b = 0; b < kABoxes; ++b) tma_prefetch_desc(&tmA.m[b]);
         tma_prefetch_desc(&tmB0);
         if (MODE == 0) tma_prefetch_desc(&tmB1);
+        if (g.sh_count) {
+            tma_prefetch_desc(&sm.b0);
+            if (MODE == 0) tma_prefetch_desc(&sm.b1);
+        }
     }
     if (warp == 1) tmem_alloc_pair(&S->tmem_base, TMEM_COLS2);
     tc_fence_before();
@@ -223,7 +227,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
     if (warp == 0) {
         // -------------------------------- item hand-off (leader) + TMA producer (both)
         if (lane == 0) {
-            const int total = *ntiles2 * n_tiles;
+            const int nrouted = *ntiles2;
+            const int sh_tps = g.sh_count ? (g.sh_T + 2 * HALF - 1) / (2 * HALF) : 1;
+            const int total = (nrouted + g.sh_count * sh_tps) * n_tiles;
             int stage = 0, rs = 0, cursor = 0;
             uint32_t phase = 0, rphase = 0;
             bool ok = true;
@@ -231,7 +237,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
             for (;;) {
                 int item;
                 if (rank == 0) {
-                    item = claim_item(g.reverse, g.counter, total, n_tiles, tiles2, cursor);
+                    item = claim_item(g.reverse, g.counter, total, n_tiles, tiles2, cursor, nrouted, g.sh_e0, sh_tps);
                     if (!wait2(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
                     S->ring[rs] = item;
                     st_remote(peer_addr(&S->ring[rs], 1), item);
@@ -245,14 +251,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                 if (++rs == RING2) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
                 const int mt = item / n_tiles, nt = item - mt * n_tiles;
-                const int expert = tiles2[3 * mt];
-                const int row0 = tiles2[3 * mt + 1] + (int)rank * HALF;
-                const int rows = min(HALF, max(0, tiles2[3 * mt + 2] - (int)rank * HALF));
+                const TileRef tr = tile_ref(tiles2, nrouted, mt, 2 * HALF, MODE, g.sh_T, g.sh_rows0, g.sh_e0);
+                const int expert = tr.e;
+                const int arow0 = tr.arow0 + (int)rank * HALF;  // this CTA's half of the pair tile
+                const int rows = min(HALF, max(0, tr.rows - (int)rank * HALF));
                 const int ab = a_box(rows);
+                const CUtensorMap *amap = (MODE == 0 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
                 const uint32_t a_bytes = rows > 0 ? (uint32_t)(a_box_rows(ab) * BK2 * 2) : 0u;
                 // B rows of this CTA: gate (CTA 0) or up (CTA 1) rows nt*128.. ; down: output columns
                 const int nrow = MODE == 0 ? nt * BNO : nt * BNO + (int)rank * 128;
-                const CUtensorMap *bmap = (MODE == 0 && rank == 1) ? &tmB1 : &tmB0;
+                const CUtensorMap *bmap = (MODE == 0 && rank == 1) ? (tr.s >= 0 ? &sm.b1 : &tmB1)
+                                                                   : (tr.s >= 0 ? &sm.b0 : &tmB0);
                 const bool b_in = nrow < g.N;  // a half entirely past N loads nothing (its columns are masked)
                 const uint32_t b_bytes = b_in ? (uint32_t)B2_BYTES : 0u;
                 for (int kb = 0; kb < num_kb; ++kb) {
@@ -262,16 +271,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                         mbar_arrive_expect_tx(&S->full[stage], a_bytes + b_bytes);
                     else
                         arrive_expect_tx_remote(fb, a_bytes + b_bytes);
-                    if (rows > 0 && !held) tma_load_2d_pair(sA + stage * A2_BYTES, &tmA.m[ab], fb, kb * BK2, row0);
-                    if (b_in) tma_load_3d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, nrow, expert);
+                    if (rows > 0 && !held) tma_load_2d_pair(sA + stage * A2_BYTES, amap, fb, kb * BK2, arow0);
+                    if (b_in) {
+                        if (tr.s < 0)
+                            tma_load_3d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, nrow, expert);
+                        else if (MODE == 0)  // shared slice s: rows s*I + nrow.. of the shared gate / up
+                            tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, tr.s * g.N + nrow);
+                        else  // shared down: columns s*I + kb*BK2..
+                            tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, tr.s * g.K + kb * BK2, nrow);
+                    }
                     if (++stage == ST2) { stage = 0; phase ^= 1; }
                     if (held && kb + 1 == min(ST2, num_kb)) {  // first item: stage j holds K block j
                         pdl_wait();
                         held = false;
                         if (rows > 0)
                             for (int j = 0; j <= kb; ++j)
-                                tma_load_2d_pair(sA + j * A2_BYTES, &tmA.m[ab], peer_addr(&S->full[j], 0), j * BK2,
-                                                 row0);
+                                tma_load_2d_pair(sA + j * A2_BYTES, amap, peer_addr(&S->full[j], 0), j * BK2, arow0);
                     }
                 }
                 if (!ok) break;
@@ -321,6 +336,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
         const int row = q * 32 + lane;
         int rs = 0, acc = 0;
         uint32_t rphase = 0, aphase = 0;
+        const int nrouted = *ntiles2;
+        // y row of sorted row r: the row map's for the routed rows, r itself for the shared expert's
+        auto flat_of = [&](int r) { return (g.sh_count == 0 || r < g.sh_rows0) ? g.row_map[r] : r; };
         for (;;) {
             if (!wait2(&S->itf[rs], rphase, g.wait_ns)) { record2(g.status, MOE_ERR_TIMEOUT); break; }
             const int item = S->ring[rs];
@@ -332,8 +350,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
             if (++rs == RING2) { rs = 0; rphase ^= 1; }
             if (item < 0) break;
             const int mt = item / n_tiles, nt = item - mt * n_tiles;
-            const int row0 = tiles2[3 * mt + 1] + (int)rank * HALF;
-            const int rows = min(HALF, max(0, tiles2[3 * mt + 2] - (int)rank * HALF));
+            const TileRef tr = tile_ref(tiles2, nrouted, mt, 2 * HALF, MODE, g.sh_T, g.sh_rows0, g.sh_e0);
+            const int row0 = tr.row0 + (int)rank * HALF;
+            const int rows = min(HALF, max(0, tr.rows - (int)rank * HALF));
             const bool row_ok = row < rows;
             if (!wait2(&S->accf[acc], aphase, g.wait_ns)) { record2(g.status, MOE_ERR_TIMEOUT); break; }
             tc_fence_after();
@@ -361,7 +380,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                     }
                 }
             } else {
-                const int flat = row_ok ? g.row_map[row0 + row] : 0;
+                const int flat = row_ok ? flat_of(row0 + row) : 0;
                 __nv_bfloat16 *orow = g.out + (size_t)flat * g.N;
 #pragma unroll 1
                 for (int c = 0; c < BNO / 32; ++c) {
@@ -431,16 +450,19 @@ bool smem2_ready(int mode)
 
 cudaError_t launch_grouped_gemm_2cta(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                      const CUtensorMap &tmB1, const int32_t *tiles2, const int32_t *ntiles2,
-                                     cudaStream_t st)
+                                     cudaStream_t st, const SharedMaps *sm)
 {
     int grid = (g.ctas > 0 ? g.ctas : num_sms()) / 2 * 2;
     if (grid < 2) grid = 2;
     if (!smem2_ready(g.mode)) return cudaErrorInvalidValue;
+    if (g.sh_count && !sm) return cudaErrorInvalidValue;
+    static const SharedMaps none{};
+    const SharedMaps &s = sm ? *sm : none;
     if (g.mode == 0)
         return launch_pdl(grouped_gemm_2cta_kernel<0>, dim3(grid), dim3(THREADS2), SMEM2, st, tmA, tmB0, tmB1, g,
-                          tiles2, ntiles2);
+                          tiles2, ntiles2, s);
     return launch_pdl(grouped_gemm_2cta_kernel<1>, dim3(grid), dim3(THREADS2), SMEM2, st, tmA, tmB0, tmB1, g, tiles2,
-                      ntiles2);
+                      ntiles2, s);
 }
 
 }  // namespace moe

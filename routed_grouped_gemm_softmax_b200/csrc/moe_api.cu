@@ -112,6 +112,37 @@ bool encode_3d_u8(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, u
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// e2m1 weights [E, rows, cols] packed two codes per byte, read as 128-code x box_rows
+// tiles that TMA expands to 16 bytes per 16 codes (the MMA's 4-bit operand layout,
+// 128 bytes per tile row), with the 128-byte swizzle.
+bool encode_3d_fp4(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {cols, rows, E};
+    const cuuint64_t strides[2] = {cols / 2, rows * cols / 2};
+    const cuuint32_t box[3] = {128, box_rows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Scale codes (bytes) [E, rows, cols] (E = 1 for a 2-D matrix), boxes of 16 codes x
+// box_rows, no swizzle.
+bool encode_scales_u8(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {cols, rows, E};
+    const cuuint64_t strides[2] = {cols, rows * cols};
+    const cuuint32_t box[3] = {16, box_rows, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, E > 1 ? 3 : 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_3d(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows)
 {
     EncodeTiledFn f = encode_fn();
@@ -265,6 +296,10 @@ size_t moe_workspace_size(const moe_dims_t *d, int dtype)
         if (d->H % 128 || d->I % 128) return 0;
         return moe::ws_layout(*d, MOE_DTYPE_FP8).total;
     }
+    if (dtype == MOE_DTYPE_MX) {
+        if (d->H % 512 || d->I % 512) return 0;
+        return moe::ws_layout(*d, MOE_DTYPE_MX).total;
+    }
     if (dtype != MOE_DTYPE_BF16) return 0;
     return moe::ws_layout(*d).total;
 }
@@ -350,26 +385,48 @@ moe_status_t moe_permute(const moe_dims_t *d, const int32_t *topk_idx, int32_t *
                                            static_cast<cudaStream_t>(stream)));
 }
 
+size_t moe_workspace_size_shared(const moe_dims_t *d, int32_t shared_I)
+{
+    if (check_dims(d) != MOE_OK || shared_I < 0 || shared_I % d->I != 0) return 0;
+    return moe::ws_layout(*d, MOE_DTYPE_BF16, shared_I / d->I).total;
+}
+
 moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_w, const float *router_bias,
                          const void *w_gate, const void *w_up, const void *w_down, void *out, void *ws,
                          size_t ws_bytes, void *stream)
 {
+    return moe_forward_shared(d, x, router_w, router_bias, w_gate, w_up, w_down, 0, nullptr, nullptr, nullptr, out,
+                              ws, ws_bytes, stream);
+}
+
+moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *router_w, const float *router_bias,
+                                const void *w_gate, const void *w_up, const void *w_down, int32_t shared_I,
+                                const void *shared_gate, const void *shared_up, const void *shared_down, void *out,
+                                void *ws, size_t ws_bytes, void *stream)
+{
     moe_status_t s = check_dims(d);
     if (s != MOE_OK) return s;
+    if (shared_I < 0 || shared_I % d->I != 0) return MOE_ERR_INVALID_ARG;
+    const int sh = shared_I / d->I;  // slices of the shared expert, I columns each
     if (d->T == 0) return MOE_OK;
     if (!x || !router_w || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(router_w) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
         !aligned16(out))
         return MOE_ERR_INVALID_ARG;
-    if ((s = check_ws(d, ws, ws_bytes)) != MOE_OK) return s;
+    if (sh && (!shared_gate || !shared_up || !shared_down || !aligned16(shared_gate) || !aligned16(shared_up) ||
+               !aligned16(shared_down)))
+        return MOE_ERR_INVALID_ARG;
+    if ((int64_t)sh * d->T + (int64_t)d->T * d->top_k > (int64_t)INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    const moe::WsLayout L = moe::ws_layout(*d, MOE_DTYPE_BF16, sh);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const moe::WsLayout L = moe::ws_layout(*d);
     const int A = d->T * d->top_k;
+    const int R = A + sh * d->T;  // rows of h and y: the routed assignments, then the shared expert's
     auto *hdr = at<moe::WsHeader>(ws, 0);
     auto *xs = at<__nv_bfloat16>(ws, L.xs);
     auto *h = at<__nv_bfloat16>(ws, L.h);
     auto *y = at<__nv_bfloat16>(ws, L.y);
-    auto *idx = at<int32_t>(ws, L.idx);
     auto *gate = at<float>(ws, L.gate);
     auto *s2f = at<int32_t>(ws, L.s2f);
     auto *tiles = at<int32_t>(ws, L.tiles);
@@ -385,8 +442,16 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
     if (!moe::encode_a_maps(&tm_xs, xs, A, d->H, false) ||
         !encode_3d(&tm_wg, w_gate, d->E, d->I, d->H, 128) ||
         !encode_3d(&tm_wu, w_up, d->E, d->I, d->H, 128) ||
-        !moe::encode_a_maps(&tm_h, h, A, d->I, false) ||
+        !moe::encode_a_maps(&tm_h, h, R, d->I, false) ||
         !encode_3d(&tm_wd, w_down, d->E, d->H, d->I, pairs ? 128 : 256))
+        return MOE_ERR_CUDA;
+    // the shared expert: x itself as its gate/up A operand, its weights as 2-D maps
+    // with the boxes of the routed experts' maps
+    moe::SharedMaps sm1{}, sm2{};
+    if (sh && (!moe::encode_a_maps(&sm1.x, x, d->T, d->H, false) ||
+               !encode_2d(&sm1.b0, shared_gate, shared_I, d->H, 128) ||
+               !encode_2d(&sm1.b1, shared_up, shared_I, d->H, 128) ||
+               !encode_2d(&sm2.b0, shared_down, d->H, shared_I, pairs ? 128 : 256)))
         return MOE_ERR_CUDA;
 
     const StageMarks marks;
@@ -407,23 +472,31 @@ moe_status_t moe_forward(const moe_dims_t *d, const void *x, const void *router_
     if (e == cudaSuccess) {
         moe::GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, h, nullptr, ctas, rev, wait_ns, stall};
         g1.trace = trace1;
+        g1.sh_count = sh;
+        g1.sh_T = d->T;
+        g1.sh_rows0 = A;
+        g1.sh_e0 = d->E;
         e = pairs ? moe::launch_grouped_gemm_2cta(g1, tm_xs, tm_wg, tm_wu, at<int32_t>(ws, L.tiles2),
-                                                  at<int32_t>(ws, L.ntiles2), st)
-                  : moe::launch_grouped_gemm(g1, tm_xs, tm_wg, tm_wu, st);
+                                                  at<int32_t>(ws, L.ntiles2), st, &sm1)
+                  : moe::launch_grouped_gemm(g1, tm_xs, tm_wg, tm_wu, st, &sm1);
     }
     if (e == cudaSuccess) e = marks.mark(3, st);
     if (e == cudaSuccess) {
         moe::GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, y, s2f, ctas, rev, wait_ns,
                          stall, 0, nullptr, gate, fused ? at<int32_t>(ws, L.ccnt) : nullptr,
-                         static_cast<__nv_bfloat16 *>(out), d->top_k, d->top_k};
+                         static_cast<__nv_bfloat16 *>(out), d->top_k, d->top_k + sh};
         g2.trace = trace2;
+        g2.sh_count = sh;
+        g2.sh_T = d->T;
+        g2.sh_rows0 = A;
+        g2.sh_e0 = d->E;
         e = pairs ? moe::launch_grouped_gemm_2cta(g2, tm_h, tm_wd, tm_wd, at<int32_t>(ws, L.tiles2),
-                                                  at<int32_t>(ws, L.ntiles2), st)
-                  : moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st);
+                                                  at<int32_t>(ws, L.ntiles2), st, &sm2)
+                  : moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st, &sm2);
     }
     if (e == cudaSuccess) e = marks.mark(4, st);
     if (e == cudaSuccess && !fused)
-        e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st);
+        e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st, sh, A);
     if (e == cudaSuccess) e = marks.mark(5, st);
     return cuda_status(e);
 }
@@ -516,6 +589,89 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
     if (e == cudaSuccess) e = marks.mark(4, st);
     if (e == cudaSuccess && !fused)
         e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st);
+    if (e == cudaSuccess) e = marks.mark(5, st);
+    return cuda_status(e);
+}
+
+moe_status_t moe_quantize_rows_mx(int32_t R, int32_t K, const void *a, uint8_t *q, uint8_t *x, void *stream)
+{
+    if (R < 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
+    if (R == 0) return MOE_OK;
+    if (!a || !q || !x || !aligned16(a) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_quantize_rows_mx(static_cast<const __nv_bfloat16 *>(a), R, K, q, x,
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward_mx(const moe_dims_t *d, const void *x, const void *router_w, const float *router_bias,
+                            const uint8_t *w_gate_p, const uint8_t *w_gate_x, const uint8_t *w_up_p,
+                            const uint8_t *w_up_x, const uint8_t *w_down_p, const uint8_t *w_down_x, void *out,
+                            void *ws, size_t ws_bytes, void *stream)
+{
+    moe_status_t s = check_dims(d);
+    if (s != MOE_OK) return s;
+    if (d->H % 512 || d->I % 512) return MOE_ERR_INVALID_ARG;
+    if (d->T == 0) return MOE_OK;
+    if (!x || !router_w || !w_gate_p || !w_gate_x || !w_up_p || !w_up_x || !w_down_p || !w_down_x || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(router_w) || !aligned16(w_gate_p) || !aligned16(w_up_p) ||
+        !aligned16(w_down_p) || !aligned16(w_gate_x) || !aligned16(w_up_x) || !aligned16(w_down_x) ||
+        !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_WORKSPACE;
+    const moe::WsLayout L = moe::ws_layout(*d, MOE_DTYPE_MX);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int A = d->T * d->top_k;
+    auto *hdr = at<moe::WsHeader>(ws, 0);
+    auto *xs = at<uint8_t>(ws, L.xs);
+    auto *xs_x = at<uint8_t>(ws, L.xs_s);
+    auto *h = at<uint8_t>(ws, L.h);
+    auto *h_x = at<uint8_t>(ws, L.h_s);
+    auto *y = at<__nv_bfloat16>(ws, L.y);
+    auto *gate = at<float>(ws, L.gate);
+    auto *s2f = at<int32_t>(ws, L.s2f);
+    auto *tiles = at<int32_t>(ws, L.tiles);
+    auto *ntiles = at<int32_t>(ws, L.ntiles);
+
+    const int ctas = g_gemm_ctas.load(), rev = g_claim_reverse.load();
+    unsigned long long *trace1 = g_trace.load(), *trace2 = trace1 ? trace1 + 2 * g_trace_ctas.load() : nullptr;
+    const unsigned long long wl = g_wait_ns.load();
+    const uint64_t wait_ns = wl ? wl : 2000000000ull;
+    const int stall = g_stall_test.load();
+    moe::MxLaunch g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, h, h_x, nullptr, nullptr,
+                     ctas, rev, wait_ns, stall, trace1};
+    moe::MxLaunch g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, nullptr, nullptr, y, s2f,
+                     ctas, rev, wait_ns, stall, trace2};
+    if (!moe::encode_a_maps(&g1.tmX, xs, A, d->H, true) || !encode_3d_fp4(&g1.tmW0, w_gate_p, d->E, d->I, d->H, 128) ||
+        !encode_3d_fp4(&g1.tmW1, w_up_p, d->E, d->I, d->H, 128) ||
+        !encode_scales_u8(&g1.tmSX, xs_x, 1, A, d->H / 32, 64) ||
+        !encode_scales_u8(&g1.tmSW0, w_gate_x, d->E, d->I, d->H / 32, 128) ||
+        !encode_scales_u8(&g1.tmSW1, w_up_x, d->E, d->I, d->H / 32, 128) ||
+        !moe::encode_a_maps(&g2.tmX, h, A, d->I, true) || !encode_3d_fp4(&g2.tmW0, w_down_p, d->E, d->H, d->I, 128) ||
+        !encode_scales_u8(&g2.tmSX, h_x, 1, A, d->I / 32, 64) ||
+        !encode_scales_u8(&g2.tmSW0, w_down_x, d->E, d->H, d->I / 32, 128))
+        return MOE_ERR_CUDA;
+    g2.tmW1 = g2.tmW0;    // the down GEMM's two tiles are rows n0.. and n0+128.. of w_down
+    g2.tmSW1 = g2.tmSW0;
+
+    const StageMarks marks;
+    cudaError_t e = marks.mark(0, st);
+    if (e == cudaSuccess && !moe::small_route_permute_ok(*d))  // else the router's kernels clear them
+        e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);
+    if (e == cudaSuccess) e = route_and_permute(*d, L, x, router_w, router_bias, ws, hdr, marks, st);
+    // x quantised once per token, then its codes and scale codes gathered into expert order
+    if (e == cudaSuccess)
+        e = moe::launch_quantize_rows_mx(static_cast<const __nv_bfloat16 *>(x), d->T, d->H, at<uint8_t>(ws, L.xq),
+                                         at<uint8_t>(ws, L.xq_s), st);
+    if (e == cudaSuccess)
+        e = moe::launch_gather_rows_mx(at<uint8_t>(ws, L.xq), at<uint8_t>(ws, L.xq_s), s2f, A, d->H, d->top_k, xs,
+                                       xs_x, st);
+    if (e == cudaSuccess) e = marks.mark(2, st);
+    if (e == cudaSuccess) e = moe::launch_grouped_gemm_mx(g1, st);
+    if (e == cudaSuccess) e = marks.mark(3, st);
+    if (e == cudaSuccess) e = moe::launch_grouped_gemm_mx(g2, st);
+    if (e == cudaSuccess) e = marks.mark(4, st);
+    if (e == cudaSuccess) e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st);
     if (e == cudaSuccess) e = marks.mark(5, st);
     return cuda_status(e);
 }

@@ -45,9 +45,13 @@ inline int perm_warps(int E)
 
 // Workspace regions; with fp8 the sorted activations and h are e4m3 codes plus
 // one fp32 scale per 128 columns, and x is quantised per token before the gather.
-inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
+inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16, int sh_count = 0)
 {
-    const bool fp8 = dtype == MOE_DTYPE_FP8;
+    const bool fp8 = dtype == MOE_DTYPE_FP8, mx = dtype == MOE_DTYPE_MX;
+    // bytes of the scales of n activation values: fp32 per 128 (fp8), e8m0 per 32 (MX)
+    auto act_scales = [&](size_t n) { return fp8 ? n / 128 * 4 : mx ? n / 32 : 0; };
+    const bool q8 = fp8 || mx;  // one-byte activation codes
+    const size_t SR = static_cast<size_t>(sh_count) * d.T;  // shared expert rows of h and y
     WsLayout L{};
     const size_t A = static_cast<size_t>(d.T) * d.top_k;
     const int warps = perm_warps(d.E);
@@ -81,13 +85,13 @@ inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16)
     L.ntiles = take(4);
     L.tiles2 = take(((A + 2 * kTileRows - 1) / (2 * kTileRows) + (A < (size_t)d.E ? A : (size_t)d.E)) * 3 * 4);
     L.ntiles2 = take(4);
-    L.xq = take(fp8 ? static_cast<size_t>(d.T) * d.H : 0);  // fp8: x quantised once per token
-    L.xq_s = take(fp8 ? static_cast<size_t>(d.T) * (d.H / 128) * 4 : 0);
-    L.xs = take(A * d.H * (fp8 ? 1 : 2));
-    L.xs_s = take(fp8 ? A * (d.H / 128) * 4 : 0);
-    L.h = take(A * d.I * (fp8 ? 1 : 2));
-    L.h_s = take(fp8 ? A * (d.I / 128) * 4 : 0);
-    L.y = take(A * d.H * 2);
+    L.xq = take(q8 ? static_cast<size_t>(d.T) * d.H : 0);  // fp8 / MX: x quantised once per token
+    L.xq_s = take(act_scales(static_cast<size_t>(d.T) * d.H));
+    L.xs = take(A * d.H * (q8 ? 1 : 2));
+    L.xs_s = take(act_scales(A * d.H));
+    L.h = take((A + SR) * d.I * (q8 ? 1 : 2));
+    L.h_s = take(act_scales(A * d.I));
+    L.y = take((A + SR) * d.H * 2);
     L.total = o;
     return L;
 }
@@ -179,16 +183,66 @@ struct GemmArgs {
     int comb_k;
     int comb_target;
     unsigned long long *trace;  // per CTA {start, end} globaltimer (ns), or null
+    // Shared expert (modes 0 and 1; sh_count = 0: none).  Its intermediate width is
+    // sh_count * I, cut into sh_count slices of I: slice s is one more "expert",
+    // number sh_e0 + s, that every token passes through with gate 1.  Its m-tiles
+    // follow the tile list's: block i of slice s covers the h / y rows
+    // sh_rows0 + s * sh_T + [i * BM, min((i + 1) * BM, sh_T)), whose A rows are the
+    // token rows i * BM.. of x in mode 0 (SharedMaps::x) and those h rows in mode 1;
+    // its weights come from SharedMaps::b0 / b1 (2-D maps over the whole shared
+    // matrices, slice s at row s * I (gate/up) or column s * I (down)).  In mode 1
+    // these y rows are written in place (no row map), after the T * k routed rows.
+    int sh_count;
+    int sh_T;
+    int sh_rows0;
+    int sh_e0;
 };
+
+// Tensor maps of the shared expert: x as the gate/up GEMM's A operand (boxes of 16
+// to 128 rows), and the gate/up (b0, b1: [sh_count * I, H]) or down (b0: [H,
+// sh_count * I]) weights as 2-D maps.  Unused (zero) without a shared expert.
+struct SharedMaps {
+    AMaps x;
+    CUtensorMap b0, b1;
+};
+
+// The m-tile `mt` of a grouped GEMM: the tile list's entry for mt < nrouted, else a
+// block of the shared expert (GemmArgs::sh_*), for tiles of `bm` rows.
+struct TileRef {
+    int e, row0, rows;  // expert, first h/y row, rows
+    int arow0;          // first A row (x row of a shared tile in mode 0, else row0)
+    int s;              // shared slice, or -1
+};
+__device__ __forceinline__ TileRef tile_ref(const int32_t *tiles, int nrouted, int mt, int bm, int mode, int sh_T,
+                                            int sh_rows0, int sh_e0)
+{
+    TileRef r;
+    if (mt < nrouted) {
+        r.e = tiles[3 * mt];
+        r.row0 = tiles[3 * mt + 1];
+        r.rows = tiles[3 * mt + 2];
+        r.arow0 = r.row0;
+        r.s = -1;
+        return r;
+    }
+    const int tps = (sh_T + bm - 1) / bm, q = mt - nrouted;
+    const int i = q % tps;
+    r.s = q / tps;
+    r.e = sh_e0 + r.s;
+    r.row0 = sh_rows0 + r.s * sh_T + i * bm;
+    r.rows = min(bm, sh_T - i * bm);
+    r.arow0 = mode == 0 ? i * bm : r.row0;
+    return r;
+}
 // mode 2: out_f32 = A B^T over M rows (one "expert"), the router's tensor-core logits.
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
-                                const CUtensorMap &tmB1, cudaStream_t st);
+                                const CUtensorMap &tmB1, cudaStream_t st, const SharedMaps *sm = nullptr);
 
 // The bf16 grouped GEMMs (modes 0 and 1) on CTA pairs, cta_group::2 MMAs over the
 // 2 x 128-row pair tiles tiles2 (grouped_gemm_2cta.cu); queue claim modes only.
 cudaError_t launch_grouped_gemm_2cta(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                      const CUtensorMap &tmB1, const int32_t *tiles2, const int32_t *ntiles2,
-                                     cudaStream_t st);
+                                     cudaStream_t st, const SharedMaps *sm = nullptr);
 
 // FP8 block-scaled grouped GEMMs (fp8.cu).  mode 0: h codes/scales from
 // silu(A Wg^T) * (A Wu^T); mode 1: y[row_map[row]] = A Wd^T in bf16; mode 2:
@@ -234,15 +288,44 @@ cudaError_t launch_quantize_rows(const __nv_bfloat16 *src, const int32_t *map, i
 cudaError_t launch_gather_rows_fp8(const uint8_t *xq, const float *xq_s, const int32_t *s2f, int A, int K, int k,
                                    uint8_t *xs, float *xs_s, cudaStream_t st);
 
+// MX grouped GEMMs (mx.cu): e2m1 weights x e4m3 activations with e8m0 scales per 32
+// along K, block-scaled on the tensor cores, operands swapped (weight rows on M).
+// mode 0: h codes/scale codes from silu(X Wg^T) * (X Wu^T); mode 1: y[row_map[row]]
+// = X Wd^T in bf16.  K a multiple of 512, N of 128.  Tensor maps: tmX the token
+// rows' codes (16/32/64-row boxes), tmW0/tmW1 the two 128-row weight tiles of an item
+// (16U4_ALIGN16B, 3-D), tmSX the token rows' scale codes (64 x 16 boxes), tmSW0/tmSW1
+// the weight scale codes (3-D, 128 x 16 boxes).
+struct MxLaunch {
+    int mode, K, N;
+    const int32_t *tiles, *ntiles;
+    int32_t *counter, *status;
+    uint8_t *out_q, *out_x;
+    __nv_bfloat16 *out;
+    const int32_t *row_map;
+    int ctas, reverse;
+    uint64_t wait_ns;
+    int stall_test;
+    unsigned long long *trace;
+    AMaps tmX;
+    CUtensorMap tmW0, tmW1, tmSX, tmSW0, tmSW1;
+};
+cudaError_t launch_grouped_gemm_mx(const MxLaunch &l, cudaStream_t st);
+// MX e4m3 codes and e8m0 scale codes (per 32 columns) of bf16 rows [R, K].
+cudaError_t launch_quantize_rows_mx(const __nv_bfloat16 *src, int R, int K, uint8_t *q, uint8_t *x, cudaStream_t st);
+// MX rows into expert order: xs[r] = xq[s2f[r] / k], xs_x[r] = xq_x[s2f[r] / k].
+cudaError_t launch_gather_rows_mx(const uint8_t *xq, const uint8_t *xq_x, const int32_t *s2f, int A, int K, int k,
+                                  uint8_t *xs, uint8_t *xs_x, cudaStream_t st);
+
 // Tensor-core router logits: partial sums over ksplit slices of H,
 // logits [ksplit, T, E] with sum_s logits[s] = x [T,H] . wrt [E,H]^T (fp32 per
 // 64-wide K block, then fp32 sums).  Returns ksplit through *ksplit_out.
 cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, int T, int H, int E, float *logits,
                              WsHeader *hdr, int *ksplit_out, cudaStream_t st);
 
-// Gate-weighted combine of the k per-assignment rows of every token (combine.cu).
+// Gate-weighted combine of the k per-assignment rows of every token (combine.cu),
+// plus, with sh_count > 0, the shared expert's rows y[sh_rows0 + s * T + t] at gate 1.
 cudaError_t launch_combine(const __nv_bfloat16 *y, const float *gate, int T, int H, int top_k,
-                           __nv_bfloat16 *out, cudaStream_t st);
+                           __nv_bfloat16 *out, cudaStream_t st, int sh_count = 0, int sh_rows0 = 0);
 // Batches up to this many tokens combine inside the down GEMM's epilogue.
 constexpr int kFusedCombineMaxT = 64;
 

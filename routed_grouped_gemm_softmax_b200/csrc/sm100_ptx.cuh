@@ -25,8 +25,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
 // c + grid, ...; mode 3: a static expert binding, CTA c taking (in order) every
 // item of the experts e with e % grid == c.  Modes 2 and 3 exist to measure what
 // the queue buys on skewed routing.  items_per_mtile maps an item to its m-tile.
+// m-tiles at or past `nrouted` are a shared expert's (its slices numbered from sh_e0,
+// sh_tps m-tiles each).
 __device__ __forceinline__ int claim_item(int mode, int32_t *counter, int total, int items_per_mtile,
-                                          const int32_t *tiles, int &cursor)
+                                          const int32_t *tiles, int &cursor, int nrouted = 0x7fffffff,
+                                          int sh_e0 = 0, int sh_tps = 1)
 {
     if (mode <= 1) {
         const int item = atomicAdd(counter, 1);
@@ -40,7 +43,8 @@ __device__ __forceinline__ int claim_item(int mode, int32_t *counter, int total,
     }
     while (cursor < total) {
         const int item = cursor++;
-        const int e = tiles ? tiles[3 * (item / items_per_mtile)] : 0;
+        const int mt = item / items_per_mtile;
+        const int e = !tiles ? 0 : mt < nrouted ? tiles[3 * mt] : sh_e0 + (mt - nrouted) / sh_tps;
         if (e % (int)gridDim.x == (int)blockIdx.x) return item;
     }
     return -1;

@@ -36,7 +36,8 @@ _M1 = 0xBF58476D1CE4E5B9
 _M2 = 0x94D049BB133111EB
 _MASK64 = (1 << 64) - 1
 
-TENSOR_IDS = {"x": 0, "router_w": 1, "bias": 2, "w_gate": 3, "w_up": 4, "w_down": 5}
+TENSOR_IDS = {"x": 0, "router_w": 1, "bias": 2, "w_gate": 3, "w_up": 4, "w_down": 5,
+              "shared_gate": 6, "shared_up": 7, "shared_down": 8}
 
 
 def _s64(v: int) -> int:
@@ -238,6 +239,17 @@ def make_mx_weights(cfg: MoEConfig, device="cpu", experts_per_chunk: int = 8):
         out[name + "_q"] = q
         out[name + "_x"] = sx
     return out
+
+
+def make_shared_weights(cfg: MoEConfig, shared_I: int, device="cpu"):
+    """A shared expert's bf16 weights, drawn like the routed experts' (N(0, 1/sqrt(fan_in)),
+    streams 6-8 of the config's seed): (shared_gate [shared_I, H], shared_up [shared_I, H],
+    shared_down [H, shared_I])."""
+    H = cfg.H
+    wg = gaussian_tensor(cfg.seed, "shared_gate", (shared_I, H), 1.0 / math.sqrt(H), device)
+    wu = gaussian_tensor(cfg.seed, "shared_up", (shared_I, H), 1.0 / math.sqrt(H), device)
+    wd = gaussian_tensor(cfg.seed, "shared_down", (H, shared_I), 1.0 / math.sqrt(shared_I), device)
+    return wg, wu, wd
 
 
 def make_inputs(cfg: MoEConfig, device="cpu", weights: bool = True) -> MoEInputs:

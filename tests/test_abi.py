@@ -70,6 +70,27 @@ def test_host_argument_errors(L):
     assert L.moe_get_device_status(null, null) == 1
 
 
+def test_shared_expert_host_checks(L):
+    null = None
+    d = api.dims(64, 256, 512, 8, 2)
+    base = api.moe_workspace_size(64, 256, 512, 8, 2)
+    # no shared expert: the plain layer's workspace; each I-wide slice adds T rows of h and y
+    assert api.moe_workspace_size_shared(64, 256, 512, 8, 2, 0) == base
+    two = api.moe_workspace_size_shared(64, 256, 512, 8, 2, 1024)
+    assert two >= base + 2 * 64 * (512 + 256) * 2
+    assert api.moe_workspace_size_shared(64, 256, 512, 8, 2, 700) == 0   # not a multiple of I
+    assert api.moe_workspace_size_shared(64, 256, 512, 8, 2, -512) == 0
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 15) // 16 * 16)
+    # shared_I not a multiple of I, or missing shared weights: rejected before any device work
+    assert L.moe_forward_shared(ctypes.byref(d), p, p, null, p, p, p, 700, p, p, p, p, null, 0, null) == 1
+    assert L.moe_forward_shared(ctypes.byref(d), p, p, null, p, p, p, 512, null, p, p, p, null, 0, null) == 1
+    # and a workspace sized for the plain layer is too small for a shared expert
+    ws = ctypes.create_string_buffer(base + 512)
+    wsp = ctypes.c_void_p((ctypes.addressof(ws) + 255) // 256 * 256)
+    assert L.moe_forward_shared(ctypes.byref(d), p, p, null, p, p, p, 512, p, p, p, p, wsp, base, null) == 3
+
+
 def test_workspace_regions_do_not_overlap(L):
     # the routing regions moe_workspace_offsets reports: 1 KiB aligned, inside the
     # workspace, and each at least as large as moe.h documents before the next begins

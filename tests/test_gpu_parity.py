@@ -304,8 +304,12 @@ def test_full_size(name):
     ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, "cuda")
     out = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k, ws=ws)
     assert api.moe_get_device_status(ws) == api.MOE_OK
-    tok = np.union1d(sample_tokens(cfg.T, 192, seed=cfg.seed), hot_expert_tokens(idx_ref, 64, seed=cfg.seed))
-    assert tok.size >= min(cfg.T, 256)
+    hot = hot_expert_tokens(idx_ref, 64, seed=cfg.seed)
+    rest = np.setdiff1d(sample_tokens(cfg.T, cfg.T, seed=cfg.seed), hot)  # every other token, shuffled below
+    rng = np.random.default_rng(cfg.seed)
+    extra = rng.permutation(rest)[:max(0, min(cfg.T, 256) - hot.size)]
+    tok = np.union1d(np.union1d(hot, extra), [0, cfg.T - 1]).astype(np.int32)
+    assert tok.size >= min(cfg.T, 256) and np.intersect1d(tok, hot).size == hot.size
     ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"], tokens=tok)
     max_abs, rel = compare_out(out[torch.as_tensor(tok, device="cuda").long()], ref, name)
     print(f"full size {name}: {tok.size} tokens, max_abs={max_abs:.3e} rel_l2={rel:.3e}")
