@@ -1,6 +1,7 @@
 """Benchmark of the MoE layer forward on B200: tokens/s of whole layer steps.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|decode|prefill|skewed|fp8|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload all|decode|prefill|skewed|fp8|tiny|mx|prefill_shared]
                     [--impl ours|reference] [--schedule ...] [--pair ...] [--swap-ab ...] [--shape K=V,...]
 
 One step = one pass of the whole layer (router softmax top-k, permute, grouped
@@ -11,7 +12,10 @@ before every step, outside that step's CUDA-event pair.  Prints one JSON line.
 With no --workload (``all``) every workload is timed in turn, K steps each, and the
 line printed is the headline workload's -- Skewed (T=8192, H=4096, E=64, top-6,
 I=1408), the largest configuration and the only compute-bound one -- with the
-other four workloads' lines, each complete, under its ``workloads`` key.
+other four workloads' lines, each complete, under its ``workloads`` key, together
+with two variants of the layer: ``mx`` (FP4 e2m1 weights and e4m3 activations with
+per-32 power-of-two scales, on the FP8 workload's shapes) and ``prefill_shared`` (the
+Prefill workload with a shared expert of 2 x I columns).
 
 Multi-GPU: the layer does not shard on one node in this design, so N GPUs run N
 independent replicas (one process per GPU, launched by torchrun); the time is the
@@ -40,11 +44,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_fp8_weights, make_inputs  # noqa: E402
+from routed_grouped_gemm_softmax_b200.inputs import (CONFIGS, EXTRA_WORKLOADS, make_fp8_weights,  # noqa: E402
+                                                     make_inputs, make_mx_weights, make_shared_weights, pack_e2m1)
 
 METRIC = "MoE-layer tokens/s at 1 B200; % of BF16/FP8 TC peak or % of HBM BW"
 HEADLINE = "skewed"                                   # the largest configuration
-ALL_ORDER = ["tiny", "decode", "prefill", "fp8", HEADLINE]   # the headline is timed last
+ALL_ORDER = ["tiny", "decode", "prefill", "fp8", "mx", "prefill_shared", HEADLINE]   # the headline is timed last
+WORKLOADS = dict(CONFIGS, **EXTRA_WORKLOADS)
 GEMM_TRACE_CTAS = 1024
 
 
@@ -76,7 +82,9 @@ def kernels_per_forward(cfg) -> int:
     else:
         route = 2 + 3      # logits, top-k; count, scan, scatter
     combine = 0 if cfg.T <= 64 else 1   # small batches combine inside the down GEMM
-    rows = 2 if cfg.dtype == "fp8" else 1   # fp8: quantise per token, then gather; bf16: gather
+    rows = 2 if cfg.dtype in ("fp8", "mx") else 1   # fp8 / MX: quantise per token, then gather; bf16: gather
+    if cfg.dtype == "mx":
+        combine = 1   # the MX down GEMM has no fused combine
     return route + rows + 2 + combine   # + gate/up GEMM, down GEMM
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 B200_SMS, FP32_LANES_PER_SM = 148, 128   # CUDA-core fp32 FMA lanes of one B200
@@ -94,7 +102,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=400)
     p.add_argument("--warmup", type=int, default=20)
-    p.add_argument("--workload", default="all", choices=["all"] + sorted(CONFIGS))
+    p.add_argument("--workload", default="all", choices=["all"] + sorted(WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -108,6 +116,8 @@ def parse():
                    help="the bf16 GEMMs on CTA pairs (tcgen05 cta_group::2): automatic choice or forced")
     p.add_argument("--swap-ab", default="auto", choices=["auto", "always", "never"],
                    help="the fp8 gate/up GEMM with swapped MMA operands: automatic choice or forced")
+    p.add_argument("--fused-combine", default="auto", choices=["auto", "always", "never"],
+                   help="the bf16 combine inside the down GEMM's epilogue: automatic choice or forced")
     p.add_argument("--shape", default="",
                    help="override config fields, e.g. T=1024,E=64 (reduced cases for profiler captures)")
     return p.parse_args()
@@ -115,7 +125,7 @@ def parse():
 
 def workload_config(args, name=None):
     name = name or (HEADLINE if args.workload == "all" else args.workload)
-    cfg = CONFIGS[name]
+    cfg = WORKLOADS[name]
     if args.shape:
         kw = {}
         for item in args.shape.split(","):
@@ -143,8 +153,8 @@ STAGE_SOURCES = {
     "route": ["route.cu", "route_certified.cu", "route_common.cuh", "fp8.cu", "fp8_common.cuh", "sm100_ptx.cuh",
               "moe_internal.h"],
     "gemm_gate_up": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "fp8_swapab.cu", "fp8_common.cuh",
-                     "sm100_ptx.cuh", "moe_internal.h"],
-    "gemm_down": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "fp8_common.cuh", "combine.cuh",
+                     "mx.cu", "sm100_ptx.cuh", "moe_internal.h"],
+    "gemm_down": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "fp8_common.cuh", "mx.cu", "combine.cuh",
                   "sm100_ptx.cuh", "moe_internal.h"],
     "combine": ["combine.cu", "combine.cuh"],
 }
@@ -327,47 +337,65 @@ def throughput(tokens_per_rank: int, world: int, steps: int, total_ms: float) ->
 
 # ----------------------------------------------------------- per-stage bytes
 
+def _weight_bytes(cfg, N, K):
+    """Bytes of one expert's [N, K] weight matrix: bf16; e4m3 + an fp32 scale per 128x128
+    block (fp8); packed e2m1 (half a byte) + an e8m0 scale per 32 along K (MX)."""
+    if cfg.dtype == "fp8":
+        return N * K + (N // 128) * (K // 128) * 4
+    if cfg.dtype == "mx":
+        return N * K // 2 + N * K // 32
+    return N * K * 2
+
+
+def _act_bytes(cfg, n):
+    """Bytes of n activation values as the GEMMs read or write them: bf16; e4m3 + an fp32
+    scale per 128 (fp8); e4m3 + an e8m0 scale per 32 (MX)."""
+    if cfg.dtype == "fp8":
+        return n + n // 128 * 4
+    if cfg.dtype == "mx":
+        return n + n // 32
+    return 2 * n
+
+
 def stage_work(cfg, counts):
     """Algorithmic bytes and FLOPs of each stage for the realised routing (counts[e] =
-    rows of expert e).  Weight bytes count only the touched experts; fp8 weights and
-    activations take one byte per element plus one fp32 scale per 128x128 weight
-    block or per 128 activation values."""
+    rows of expert e).  Weight bytes count only the touched experts, in the workload's
+    storage (_weight_bytes); a shared expert of shared_mult * I columns adds its weights,
+    its T rows of x and h and its FLOPs."""
     T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k
     A = T * k
     D = int(sum(1 for c in counts if c > 0))
-    fp8 = cfg.dtype == "fp8"
-    wb = 1 if fp8 else 2
-    wsc = (lambda n, kk: (n // 128) * (kk // 128) * 4) if fp8 else (lambda n, kk: 0)
-    ab = (lambda n: n + n // 128 * 4) if fp8 else (lambda n: 2 * n)   # activation bytes of n values
+    SI = cfg.shared_mult * I
     return {
         # T <= 32: every logit is an fp32 FMA chain on the CUDA cores; above, the logits run
         # on the tensor cores and only the candidates' chains on the CUDA cores
         "route": {"bytes": T * H * 2 + H * E * 2 + A * 8, "flops": 2.0 * T * H * E, "alu": T <= 32},
-        "gemm_gate_up": {"bytes": D * (2 * I * H * wb + 2 * wsc(I, H)) + ab(A * H) + ab(A * I),
-                         "flops": 2.0 * A * H * 2 * I},
-        "gemm_down": {"bytes": D * (H * I * wb + wsc(H, I)) + ab(A * I) + A * H * 2, "flops": 2.0 * A * I * H},
-        "combine": {"bytes": A * H * 2 + A * 4 + T * H * 2, "flops": 2.0 * A * H},
+        "gemm_gate_up": {"bytes": D * 2 * _weight_bytes(cfg, I, H) + _act_bytes(cfg, A * H) + _act_bytes(cfg, A * I)
+                                  + (2 * SI * H * 2 + T * H * 2 + T * SI * 2 if SI else 0),
+                         "flops": 2.0 * A * H * 2 * I + 2.0 * T * H * 2 * SI},
+        "gemm_down": {"bytes": D * _weight_bytes(cfg, H, I) + _act_bytes(cfg, A * I) + A * H * 2
+                               + (H * SI * 2 + T * SI * 2 + cfg.shared_mult * T * H * 2 if SI else 0),
+                      "flops": 2.0 * A * I * H + 2.0 * T * SI * H},
+        "combine": {"bytes": (A + cfg.shared_mult * T) * H * 2 + A * 4 + T * H * 2, "flops": 2.0 * A * H},
         "_D": D,
     }
 
 
 def layer_work(cfg, counts):
     """The whole layer's algorithmic bytes and FLOPs: the touched experts' weights (with
-    their block scales for fp8), x, out, router_w and the chosen indices and gates; the
-    router and expert FLOPs.  The expert-ordered copy of x, h and y are the
-    implementation's own traffic, counted apart in `implementation_bytes` (each written
-    once and read once)."""
+    their scales where quantised) and a shared expert's, x, out, router_w and the chosen
+    indices and gates; the router and expert FLOPs.  The expert-ordered copy of x, h and
+    y are the implementation's own traffic, counted apart in `implementation_bytes`
+    (each written once and read once)."""
     T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k
     A = T * k
     D = int(sum(1 for c in counts if c > 0))
-    if cfg.dtype == "fp8":
-        per_expert = 3 * I * H + 3 * (I // 128) * (H // 128) * 4
-        inter = 2 * (A * H + A * H // 128 * 4) + 2 * (A * I + A * I // 128 * 4) + 2 * A * H * 2
-    else:
-        per_expert = 3 * I * H * 2
-        inter = 2 * (A * H * 2) + 2 * (A * I * 2) + 2 * (A * H * 2)
-    return {"bytes": D * per_expert + 2 * T * H * 2 + H * E * 2 + A * 8,
-            "flops": 2.0 * A * H * 2 * I + 2.0 * A * I * H + 2.0 * T * H * E,
+    SI, m = cfg.shared_mult * I, cfg.shared_mult
+    per_expert = 2 * _weight_bytes(cfg, I, H) + _weight_bytes(cfg, H, I)
+    inter = 2 * _act_bytes(cfg, A * H) + 2 * _act_bytes(cfg, A * I) + 2 * (A * H * 2)
+    inter += 2 * (m * T * I * 2) + 2 * (m * T * H * 2)  # a shared expert's h and y rows
+    return {"bytes": D * per_expert + 3 * SI * H * 2 + 2 * T * H * 2 + H * E * 2 + A * 8,
+            "flops": 2.0 * A * H * 2 * I + 2.0 * A * I * H + 2.0 * T * H * E + 2.0 * T * H * 3 * SI,
             "implementation_bytes": inter}
 
 
@@ -375,7 +403,7 @@ def layer_roofline(cfg, counts, ms, peaks, peaks_kind, sustained):
     """The layer per step against its binding roofline: HBM when its algorithmic bytes
     take longer at the measured bandwidth than its FLOPs at the measured tensor peak."""
     w = layer_work(cfg, counts)
-    fp8 = cfg.dtype == "fp8"
+    fp8 = cfg.dtype in ("fp8", "mx")  # e4m3 x e4m3 and e2m1 x e4m3 MMAs run at the fp8 rate
     pk_tf = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * (2.0 if fp8 else 1.0)
     t = ms * 1e-3
     if w["bytes"] / (peaks["hbm_gbs"] * 1e9) >= w["flops"] / (pk_tf * 1e12):
@@ -420,26 +448,37 @@ def roofline_for(stage, work, ms, peaks, peaks_kind, sustained, workload, fp8=Fa
 
 # ------------------------------------------------------------- CPU oracle leg
 
-def host_inputs(cfg, inp=None, w8=None):
-    """The workload's tensors as host numpy arrays (bf16 bit patterns), drawn on the GPU
-    when one is present (data preparation only; nothing of the layer runs there)."""
+def host_inputs(cfg, inp=None, wq=None, shared=None):
+    """The workload's tensors as host numpy arrays (bf16 bit patterns; quantised codes
+    and scales for fp8 / MX), drawn on the GPU when one is present (data preparation
+    only; nothing of the layer runs there).  wq: the fp8 or MX weights already drawn."""
     import types
 
     import numpy as np
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
     if inp is None:
-        inp = make_inputs(cfg, device="cuda" if torch.cuda.is_available() else "cpu")
+        inp = make_inputs(cfg, device=dev, weights=cfg.dtype == "bf16")
 
     def bits(t):
         return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
     ns = types.SimpleNamespace(
         x=bits(inp.x), router_w=bits(inp.router_w),
-        bias=None if inp.bias is None else inp.bias.detach().cpu().float().numpy(), fp8=None)
+        bias=None if inp.bias is None else inp.bias.detach().cpu().float().numpy(), fp8=None, mx=None,
+        shared=None)
     if cfg.dtype == "fp8":
-        if w8 is None:
-            w8 = make_fp8_weights(cfg, device=inp.x.device)
-        ns.fp8 = {k: v.detach().cpu().numpy() for k, v in w8.items()}
+        if wq is None:
+            wq = make_fp8_weights(cfg, device=inp.x.device)
+        ns.fp8 = {k: v.detach().cpu().numpy() for k, v in wq.items()}
+    elif cfg.dtype == "mx":
+        if wq is None:
+            wq = make_mx_weights(cfg, device=inp.x.device)
+        ns.mx = {k: v.detach().cpu().numpy() for k, v in wq.items()}
     else:
         ns.w_gate, ns.w_up, ns.w_down = bits(inp.w_gate), bits(inp.w_up), bits(inp.w_down)
+    if cfg.shared_mult:
+        if shared is None:
+            shared = make_shared_weights(cfg, cfg.shared_mult * cfg.I, device=inp.x.device)
+        ns.shared = [bits(t) for t in shared]
     return ns
 
 
@@ -461,8 +500,14 @@ def oracle_step_timer(cfg, h):
             f = h.fp8
             oracle.combine_ffn_fp8(h.x, idx, gate, f["w_gate_q"], f["w_gate_s"], f["w_up_q"], f["w_up_s"],
                                    f["w_down_q"], f["w_down_s"], tokens=tok, nthreads=threads)
+        elif h.mx is not None:
+            f = h.mx
+            oracle.get().combine_ffn_mx(h.x, idx, gate, f["w_gate_q"], f["w_gate_x"], f["w_up_q"], f["w_up_x"],
+                                        f["w_down_q"], f["w_down_x"], tokens=tok, nthreads=threads)
         else:
             oracle.combine_ffn(h.x, idx, gate, h.w_gate, h.w_up, h.w_down, tokens=tok, nthreads=threads)
+        if h.shared is not None:
+            oracle.shared_ffn(h.x, *h.shared, tokens=tok, nthreads=threads)
         t2 = time.perf_counter()
         return t1 - t0, t2 - t1
     return run, threads
@@ -524,7 +569,9 @@ def run_reference(args, world, rank):
 
 def config_block(cfg, world):
     return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.top_k,
-            "weights": "e4m3 + fp32 128x128 block scales" if cfg.dtype == "fp8" else "bf16",
+            "weights": {"fp8": "e4m3 + fp32 128x128 block scales",
+                        "mx": "e2m1 (packed 2 per byte) + e8m0 scale per 32 along K"}.get(cfg.dtype, "bf16"),
+            "shared_expert_I": cfg.shared_mult * cfg.I if cfg.shared_mult else None,
             "seed": cfg.seed, "router_bias": "zipf(1.2)" if cfg.zipf_s else None,
             "global_batch": cfg.T * world, "parallelism": f"replicas{world}",
             "l2": "flushed before every step: 512 MiB write then 256 MiB read, outside the step's events",
@@ -541,18 +588,33 @@ def run_one(args, cfg, world, rank, local):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    fp8 = cfg.dtype == "fp8"
-    inp = make_inputs(cfg, device=dev, weights=not fp8)
+    fp8 = cfg.dtype in ("fp8", "mx")   # quantised: the tensor peak is the fp8 rate
+    inp = make_inputs(cfg, device=dev, weights=cfg.dtype == "bf16")
     x, rw, bias = inp.x, inp.router_w, inp.bias
     k = cfg.top_k
-    if fp8:
+    w8 = shared = None
+    if cfg.dtype == "fp8":
         w8 = make_fp8_weights(cfg, device=dev)
         wq = (w8["w_gate_q"], w8["w_gate_s"], w8["w_up_q"], w8["w_up_s"], w8["w_down_q"], w8["w_down_s"])
         forward = lambda xx, st: api.moe_forward_fp8(xx, rw, bias, *wq, k, out=out, ws=ws, stream=st)
+        ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, dev, api.DTYPE_FP8)
+    elif cfg.dtype == "mx":
+        w8 = make_mx_weights(cfg, device=dev)
+        wq = (pack_e2m1(w8["w_gate_q"]), w8["w_gate_x"], pack_e2m1(w8["w_up_q"]), w8["w_up_x"],
+              pack_e2m1(w8["w_down_q"]), w8["w_down_x"])
+        forward = lambda xx, st: api.moe_forward_mx(xx, rw, bias, *wq, k, out=out, ws=ws, stream=st)
+        ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, dev, api.DTYPE_MX)
+    elif cfg.shared_mult:
+        wg, wu, wd = inp.w_gate, inp.w_up, inp.w_down
+        shared = make_shared_weights(cfg, cfg.shared_mult * cfg.I, device=dev)
+        forward = lambda xx, st: api.moe_forward_shared(xx, rw, bias, wg, wu, wd, *shared, k, out=out, ws=ws,
+                                                        stream=st)
+        ws = torch.empty(api.moe_workspace_size_shared(cfg.T, cfg.H, cfg.I, cfg.E, k, cfg.shared_mult * cfg.I),
+                         dtype=torch.uint8, device=dev)
     else:
         wg, wu, wd = inp.w_gate, inp.w_up, inp.w_down
         forward = lambda xx, st: api.moe_forward(xx, rw, bias, wg, wu, wd, k, out=out, ws=ws, stream=st)
-    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, dev, api.DTYPE_FP8 if fp8 else api.DTYPE_BF16)
+        ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, dev, api.DTYPE_BF16)
     out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     evict_buf = torch.ones(EVICT_FLOATS, dtype=torch.float32, device=dev)
@@ -582,6 +644,7 @@ def run_one(args, cfg, world, rank, local):
     api.set_claim_order(False if args.schedule == "queue" else args.schedule)
     api.set_pair_mma(args.pair)
     api.set_fp8_swap_ab(args.swap_ab)
+    api.set_fused_combine(args.fused_combine)
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
         step()
@@ -690,14 +753,14 @@ def run_one(args, cfg, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         budget = args.cpu_budget if args.cpu_budget else (12.0 if args.workload == "all" else 20.0)
-        cpu = cpu_baseline(cfg, host_inputs(cfg, inp, w8 if fp8 else None), budget_s=budget)
+        cpu = cpu_baseline(cfg, host_inputs(cfg, inp, w8, shared), budget_s=budget)
 
     line = None
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 5),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "e4m3" if fp8 else "bf16",
+                "dtype": {"fp8": "e4m3", "mx": "e2m1 x e4m3 (mx)"}.get(cfg.dtype, "bf16"),
                 "data": "synthetic", "config": config_block(cfg, world),
                 "roofline": roof, "layer_roofline": layer_roof, "stages": stages, "experts_touched": work["_D"],
                 "e2e": e2e, "gpu_launches": kernels_per_forward(cfg) * args.steps, "schedule": sched,

@@ -207,12 +207,28 @@ moe_status_t moe_quantize_rows_fp8(int32_t R, int32_t K, const void *a, uint8_t 
  *   0 topk_idx [T,k] int32    1 topk_w [T,k] fp32      2 expert_offsets [E+1]
  *   3 sorted_to_flat [T*k]    4 flat_to_sorted [T*k]    5 tile_list [3*max_tiles]
  *   6 num_tiles [1]           7 logits [T,E] fp32
+ *   8 xs: the activations in expert-sorted order [T*k, H] (bf16, or 1-byte codes
+ *     for MOE_DTYPE_FP8 / MOE_DTYPE_MX)   9 their scales (fp8: fp32 [T*k, H/128];
+ *     MX: e8m0 codes [T*k, H/32])   10 h [T*k, I] (same types)   11 h's scales
+ *   12 y [T*k, H] bf16, the per-assignment expert outputs in flat order
  * (0-6 as the outputs of moe_route and moe_permute; 0-1 after moe_route only
  * when it was given the workspace's own regions).  Entry 7 holds the router's
  * fp32 chain value (bias included) of every (t,e) when T <= 32, and of at least
- * each token's chosen experts when T > 32.  Writes min(n, 8) entries; returns
+ * each token's chosen experts when T > 32.  Writes min(n, 13) entries; returns
  * MOE_ERR_INVALID_ARG for invalid dims or dtype. */
 moe_status_t moe_workspace_offsets(const moe_dims_t *d, int dtype, size_t *out, int32_t n);
+
+/* The kernels a forward with these dims and dtype launches under the current
+ * process-wide settings, as bits: the two-kernel router + grouping for small batches,
+ * pair-of-CTA GEMM tiles, the combine inside the down GEMM, and both expert GEMMs in
+ * one launch.  -1 for invalid dims or dtype.  Host only; enqueues nothing. */
+enum {
+    MOE_PLAN_SMALL_ROUTER = 1,
+    MOE_PLAN_PAIR_TILES = 2,
+    MOE_PLAN_FUSED_COMBINE = 4,
+    MOE_PLAN_LAYER_GEMM = 8
+};
+int32_t moe_forward_plan(const moe_dims_t *d, int dtype);
 
 /* Synchronises `stream`, returns the device status word of the workspace
  * (MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX or MOE_ERR_ROUTER_BOUND -- the first
@@ -251,6 +267,21 @@ void moe_set_pair_mma(int32_t mode);
  * forms compute the same blockwise-scaled sums; the output stays within the fp8
  * layer's tolerance either way.  Process-wide. */
 void moe_set_fp8_swap_ab(int32_t mode);
+
+/* Where the bf16 forwards sum the k per-assignment rows of a token: 0 = automatic
+ * (inside the down GEMM's epilogue for batches of at most 64 tokens, else a separate
+ * combine kernel), 1 = always inside the down GEMM, 2 = always the separate kernel.
+ * The sum's order is fixed by j either way, so the result is bitwise the same.
+ * Process-wide; for tests and benchmarks. */
+void moe_set_fused_combine(int32_t mode);
+
+/* The bf16 forwards' two expert GEMMs in one persistent launch (the layer kernel:
+ * every gate/up work item is claimed before any down item, and a down item waits --
+ * with a bounded wait -- on a per-m-tile count of the epilogue warps that wrote its
+ * h rows) or in two launches.  0 = automatic (one launch for 128-row tiles, two for
+ * pair-of-CTA tiles), 1 = one launch whenever the tiles are 128-row ones, 2 = two
+ * launches.  Results are bitwise the same.  Process-wide; for tests and benchmarks. */
+void moe_set_layer_gemm(int32_t mode);
 
 /* Scheduling trace for benchmarks.  With `trace` a device buffer of 4 * ctas
  * uint64 values (ctas >= the GEMM grid, 148 by default), every later forward

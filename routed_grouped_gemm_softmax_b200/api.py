@@ -24,8 +24,9 @@ EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "m
            "moe_set_pair_mma", "moe_set_fp8_swap_ab",
            "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",
            "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets", "moe_set_router_audit",
-           "moe_forward_shared", "moe_workspace_size_shared"]
-DTYPE_BF16, DTYPE_FP8 = 0, 1
+           "moe_forward_shared", "moe_workspace_size_shared", "moe_forward_mx", "moe_quantize_rows_mx",
+           "moe_set_fused_combine", "moe_set_layer_gemm", "moe_forward_plan"]
+DTYPE_BF16, DTYPE_FP8, DTYPE_MX = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
 TILE_ROWS = 128
@@ -90,6 +91,16 @@ def lib():
         L.moe_forward_shared.restype = ctypes.c_int
         L.moe_workspace_size_shared.argtypes = [D, I32]
         L.moe_workspace_size_shared.restype = SZ
+        L.moe_forward_plan.argtypes = [D, ctypes.c_int]
+        L.moe_forward_plan.restype = I32
+        L.moe_set_layer_gemm.argtypes = [I32]
+        L.moe_set_layer_gemm.restype = None
+        L.moe_set_fused_combine.argtypes = [I32]
+        L.moe_set_fused_combine.restype = None
+        L.moe_forward_mx.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.moe_forward_mx.restype = ctypes.c_int
+        L.moe_quantize_rows_mx.argtypes = [I32, I32, P, P, P, P]
+        L.moe_quantize_rows_mx.restype = ctypes.c_int
         L.moe_set_router_audit.argtypes = [P, P, ctypes.c_int64]
         L.moe_set_router_audit.restype = None
         L.moe_forward_noalloc.argtypes = [D, P, P, P, P, P, P, P, P]
@@ -237,6 +248,43 @@ def moe_forward_shared(x, router_w, bias, w_gate, w_up, w_down, shared_gate, sha
     return out
 
 
+def moe_forward_mx(x, router_w, bias, w_gate_p, w_gate_x, w_up_p, w_up_x, w_down_p, w_down_x, top_k: int,
+                   out=None, ws=None, stream=None):
+    """The MX layer: e2m1 weights packed two per byte ([E,N,K/2] uint8) with e8m0 scale
+    codes per 32 along K ([E,N,K/32] uint8); returns out bf16 [T,H]."""
+    T, H = x.shape
+    E, I, _ = w_gate_p.shape
+    dev = x.device
+    _need(x, torch.bfloat16, (T, H), "x")
+    _need(router_w, torch.bfloat16, (H, E), "router_w")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "router_bias")
+    for t, shp, nm in ((w_gate_p, (E, I, H // 2), "w_gate_p"), (w_up_p, (E, I, H // 2), "w_up_p"),
+                       (w_down_p, (E, H, I // 2), "w_down_p"), (w_gate_x, (E, I, H // 32), "w_gate_x"),
+                       (w_up_x, (E, I, H // 32), "w_up_x"), (w_down_x, (E, H, I // 32), "w_down_x")):
+        _need(t, torch.uint8, shp, nm)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if out is None else out
+    _need(out, torch.bfloat16, (T, H), "out")
+    ws = workspace(T, H, I, E, top_k, dev, DTYPE_MX) if ws is None else ws
+    d = dims(T, H, I, E, top_k)
+    _check(lib().moe_forward_mx(ctypes.byref(d), _p(x), _p(router_w), _p(bias), _p(w_gate_p), _p(w_gate_x),
+                                _p(w_up_p), _p(w_up_x), _p(w_down_p), _p(w_down_x), _p(out), _p(ws), ws.numel(),
+                                _stream(stream, dev)),
+           "moe_forward_mx")
+    return out
+
+
+def moe_quantize_rows_mx(a, stream=None):
+    """MX e4m3 codes [R,K] and e8m0 scale codes [R,K/32] of a bf16 [R,K] (K % 32 == 0)."""
+    R, K = a.shape
+    _need(a, torch.bfloat16, (R, K), "a")
+    q = torch.empty((R, K), dtype=torch.uint8, device=a.device)
+    x = torch.empty((R, K // 32), dtype=torch.uint8, device=a.device)
+    _check(lib().moe_quantize_rows_mx(int(R), int(K), _p(a), _p(q), _p(x), _stream(stream, a.device)),
+           "moe_quantize_rows_mx")
+    return q, x
+
+
 def moe_forward_fp8(x, router_w, bias, w_gate_q, w_gate_s, w_up_q, w_up_s, w_down_q, w_down_s,
                     top_k: int, out=None, ws=None, stream=None):
     """The FP8 block-scaled layer; weights are uint8 e4m3 codes with fp32 128x128 block
@@ -349,6 +397,24 @@ def set_claim_order(reverse):
 def set_pair_mma(mode: str):
     """"auto" (default), "always" or "never": the bf16 forward's pair-of-CTA GEMMs."""
     lib().moe_set_pair_mma({"auto": 0, "always": 1, "never": 2}[mode])
+
+
+PLAN_SMALL_ROUTER, PLAN_PAIR_TILES, PLAN_FUSED_COMBINE, PLAN_LAYER_GEMM = 1, 2, 4, 8
+
+
+def forward_plan(T, H, I, E, top_k, dtype: int = DTYPE_BF16) -> int:
+    """The kernels a forward would launch now (PLAN_* bits), -1 for invalid dims."""
+    return int(lib().moe_forward_plan(ctypes.byref(dims(T, H, I, E, top_k)), int(dtype)))
+
+
+def set_layer_gemm(mode: str):
+    """"auto" (default), "always" or "never": both bf16 expert GEMMs in one persistent launch."""
+    lib().moe_set_layer_gemm({"auto": 0, "always": 1, "never": 2}[mode])
+
+
+def set_fused_combine(mode: str):
+    """"auto" (default), "always" or "never": the bf16 combine inside the down GEMM."""
+    lib().moe_set_fused_combine({"auto": 0, "always": 1, "never": 2}[mode])
 
 
 def set_fp8_swap_ab(mode: str):

@@ -13,7 +13,8 @@ __device__ __forceinline__ void record(int32_t *status, int code) { atomicCAS(st
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + __expf(-a)); }
 
 // e4m3 codes of a and b (already divided by the scale), round to nearest even,
-// saturated at +-448; a in the low byte.
+// saturated at +-448; a in the low byte.  A negative value that rounds to zero keeps
+// its sign (code 0x80), as an IEEE-style conversion does.
 __device__ __forceinline__ uint32_t e4m3_pair(float a, float b)
 {
     const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);

@@ -81,13 +81,40 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Item `item` of the launch: its phase (1: a down item; in modes 0-2 fixed by the
+// mode, in mode 3 the items past the gate/up ones), m-tile and n-tile.
+struct ItemPos {
+    int p1, mt, nt;
+};
+
+// Waits (at most limit_ns) until *ctr >= target, with acquire ordering at GPU scope.
+__device__ __forceinline__ bool wait_count_at_least(const int32_t *ctr, int target, uint64_t limit_ns)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i) {
+            asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+            if (v >= target) return true;
+        }
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB0,
-                    const __grid_constant__ CUtensorMap tmB1, const GemmArgs g, const __grid_constant__ SharedMaps sm)
+                    const __grid_constant__ CUtensorMap tmB1, const GemmArgs g, const __grid_constant__ SharedMaps sm,
+                    const __grid_constant__ LayerMaps lm)
 {
-    // output columns per tile: mode 0 packs 128 gate + 128 up columns into N=256
-    constexpr int BNO = MODE == 0 ? BN / 2 : BN;
+    // Output columns per tile: the gate/up items pack 128 gate + 128 up columns into
+    // N=256; the down (and dense) items write 256 columns.
+    constexpr int BNO0 = BN / 2, BNO1 = BN;
     const bool dense = g.tiles == nullptr;  // mode 2: m-tiles are plain 128-row blocks of A
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -96,8 +123,10 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
     Ctrl *S = reinterpret_cast<Ctrl *>(sB + STAGES * B_BYTES);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int n_tiles = (g.N + BNO - 1) / BNO;
-    const int num_kb = g.K / BK;
+    // n-tiles and K blocks of the gate/up items (modes 0, 3) and of the down / dense items
+    const int nt0 = (g.N + BNO0 - 1) / BNO0, kb0 = g.K / BK;
+    const int nt1 = MODE == 3 ? (g.N2 + BNO1 - 1) / BNO1 : (g.N + BNO1 - 1) / BNO1;
+    const int kb1 = MODE == 3 ? g.K2 / BK : g.K / BK;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -117,10 +146,11 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
         fence_mbar_init();
         for (int b = 0; b < kABoxes; ++b) tma_prefetch_desc(&tmA.m[b]);
         tma_prefetch_desc(&tmB0);
-        if (MODE == 0) tma_prefetch_desc(&tmB1);
+        if (MODE == 0 || MODE == 3) tma_prefetch_desc(&tmB1);
+        if (MODE == 3) tma_prefetch_desc(&lm.wd);
         if (g.sh_count) {
             tma_prefetch_desc(&sm.b0);
-            if (MODE == 0) tma_prefetch_desc(&sm.b1);
+            if (MODE == 0 || MODE == 3) tma_prefetch_desc(&sm.b1);
         }
     }
     if (warp == 1) tmem_alloc(&S->tmem_base, TMEM_COLS);
@@ -128,20 +158,34 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    // The prologue above overlapped the previous kernel.  Modes 0 and 1: warp 0 waits
-    // for it inside the producer, after the first stages' weight loads (the weights
-    // are the layer's inputs; only the A rows are the previous kernel's output).
+    // The prologue above overlapped the previous kernel.  Modes 0, 1 and 3: warp 0
+    // waits for it inside the producer, after the first stages' weight loads (the
+    // weights are the layer's inputs; only the A rows are the previous kernel's output).
     constexpr bool kEarlyB = MODE != 2;
     if (!(kEarlyB && warp == 0)) pdl_wait();
     pdl_trigger();
     if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
+    // m-tiles: the tile list's, then the shared expert's; the gate/up items of all
+    // m-tiles precede (mode 3) the down items
+    const int nrouted = dense ? 0 : *g.ntiles;
+    const int sh_tps = g.sh_count ? (g.sh_T + BM - 1) / BM : 1;
+    const int mtiles = dense ? (g.M + BM - 1) / BM : nrouted + g.sh_count * sh_tps;
+    const int total0 = MODE == 3 ? mtiles * nt0 : 0;
+    auto pos_of = [&](int item) {
+        ItemPos r;
+        r.p1 = MODE == 1 || MODE == 2 || (MODE == 3 && item >= total0);
+        const int local = MODE == 3 && r.p1 ? item - total0 : item;
+        const int ntl = r.p1 ? nt1 : nt0;
+        r.mt = local / ntl;
+        r.nt = local - r.mt * ntl;
+        return r;
+    };
+
     if (warp == 0) {
         // ------------------------------------------------ scheduler + TMA producer
         if (lane == 0) {
-            const int nrouted = dense ? 0 : *g.ntiles;
-            const int sh_tps = g.sh_count ? (g.sh_T + BM - 1) / BM : 1;
-            const int total = (dense ? (g.M + BM - 1) / BM : nrouted + g.sh_count * sh_tps) * n_tiles;
+            const int total = MODE == 3 ? total0 + mtiles * nt1 : mtiles * (MODE == 0 ? nt0 : nt1);
             int stage = 0, rs = 0;
             uint32_t phase = 0, rphase = 0;
             uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
@@ -149,23 +193,54 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
             int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
             bool held = kEarlyB;  // A loads of the first item's first stages wait for the previous kernel
             for (;;) {
-                const int item = claim_item(g.reverse, g.counter, total, n_tiles, dense ? nullptr : g.tiles, cursor,
-                                            nrouted, g.sh_e0, sh_tps);
+                int item;
+                if (MODE != 3) {
+                    item = claim_item(g.reverse, g.counter, total, MODE == 0 ? nt0 : nt1, dense ? nullptr : g.tiles,
+                                      cursor, nrouted, g.sh_e0, sh_tps);
+                } else if (g.reverse <= 1) {
+                    // the queue; descending within each phase, so that every gate/up item is
+                    // claimed before any down item whatever the order
+                    item = atomicAdd(g.counter, 1);
+                    if (item >= total) item = -1;
+                    else if (g.reverse == 1)
+                        item = item < total0 ? total0 - 1 - item : total0 + (total - 1 - item);
+                } else {
+                    // static: this CTA's items in ascending order, every c-th (mode 2) or those
+                    // of the experts e with e % grid == c (mode 3)
+                    item = -1;
+                    while (cursor < total) {
+                        const int it = cursor;
+                        cursor += g.reverse == 2 ? (int)gridDim.x : 1;
+                        if (g.reverse == 2) { item = it; break; }
+                        const TileRef t = tile_ref(g.tiles, nrouted, pos_of(it).mt, BM, 0, g.sh_T, g.sh_rows0, g.sh_e0);
+                        if (t.e % (int)gridDim.x == (int)blockIdx.x) { item = it; break; }
+                    }
+                }
                 if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
                 S->ring[rs] = item;
                 mbar_arrive(&S->itf[rs]);
                 if (++rs == RING) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
-                const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
-                TileRef tr{0, mt * BM, 0, mt * BM, -1};
+                const ItemPos ip = pos_of(item);
+                const bool p1 = ip.p1;
+                TileRef tr{0, ip.mt * BM, 0, ip.mt * BM, -1};
                 if (dense)
                     tr.rows = min(BM, g.M - tr.row0);
                 else
-                    tr = tile_ref(g.tiles, nrouted, mt, BM, MODE, g.sh_T, g.sh_rows0, g.sh_e0);
+                    tr = tile_ref(g.tiles, nrouted, ip.mt, BM, p1 ? 1 : 0, g.sh_T, g.sh_rows0, g.sh_e0);
                 const int expert = tr.e, arow0 = tr.arow0;
                 const int ab = a_box(tr.rows);  // the A box that covers the tile's rows
-                const CUtensorMap *amap = (MODE == 0 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
-                const int n0 = nt * BNO;
+                const CUtensorMap *amap = MODE == 3 && p1 ? &lm.h.m[ab]
+                                        : (!p1 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
+                const int n0 = ip.nt * (p1 ? BNO1 : BNO0);
+                const int num_kb = p1 ? kb1 : kb0;
+                if (MODE == 3 && p1) {
+                    // the down item reads h rows of m-tile mt: wait until every gate/up item of
+                    // mt has published them, then order those generic-proxy writes before the
+                    // TMA (async-proxy) reads below
+                    if (!wait_count_at_least(g.ready + ip.mt, 4 * nt0, g.wait_ns)) { ok = false; break; }
+                    fence_proxy_async_global();
+                }
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
                     mbar_arrive_expect_tx(&S->full[stage], a_box_rows(ab) * BK * 2 + B_BYTES);
@@ -173,14 +248,21 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     uint8_t *b_dst = sB + stage * B_BYTES;
                     if (!held) tma_load_2d(sA + stage * A_BYTES, amap, &S->full[stage], kb * BK, arow0);
-                    if (tr.s < 0) {
-                        tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
-                        if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
-                    } else if (MODE == 0) {  // shared slice s: rows s*I + n0.. of the shared gate / up
-                        tma_load_2d(b_dst, &sm.b0, &S->full[stage], kb * BK, tr.s * g.N + n0);
-                        tma_load_2d(b_dst + B_BYTES / 2, &sm.b1, &S->full[stage], kb * BK, tr.s * g.N + n0);
-                    } else {  // shared down: columns s*I + kb*BK..
-                        tma_load_2d(b_dst, &sm.b0, &S->full[stage], tr.s * g.K + kb * BK, n0);
+                    if (!p1) {  // gate / up rows n0.. of the expert (or of shared slice s)
+                        if (tr.s < 0) {
+                            tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
+                            tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
+                        } else {
+                            tma_load_2d(b_dst, &sm.b0, &S->full[stage], kb * BK, tr.s * g.N + n0);
+                            tma_load_2d(b_dst + B_BYTES / 2, &sm.b1, &S->full[stage], kb * BK, tr.s * g.N + n0);
+                        }
+                    } else {  // down (or dense) rows n0..: the expert's, or columns s*I.. of the shared down
+                        const CUtensorMap *bm = MODE == 3 ? &lm.wd : &tmB0;
+                        const CUtensorMap *bs = MODE == 3 ? &lm.wd_sh : &sm.b0;
+                        if (tr.s < 0)
+                            tma_load_3d(b_dst, bm, &S->full[stage], kb * BK, n0, expert);
+                        else
+                            tma_load_2d(b_dst, bs, &S->full[stage], tr.s * (MODE == 3 ? g.K2 : g.K) + kb * BK, n0);
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                     if (held && kb + 1 == min(STAGES, num_kb)) {  // first item: stage j holds K block j
@@ -219,6 +301,7 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                 mbar_arrive(&S->ite[rs]);
                 if (++rs == RING) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
+                const int num_kb = pos_of(item).p1 ? kb1 : kb0;
                 if (!mbar_wait(&S->acce[acc], aphase ^ 1, g.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
@@ -250,7 +333,8 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
         const int row = q * 32 + lane;
         int rs = 0, acc = 0;
         uint32_t rphase = 0, aphase = 0;
-        const int nrouted = dense ? 0 : *g.ntiles;
+        // y row of sorted row r: the row map's for the routed rows, r itself for the shared expert's
+        auto flat_of = [&](int r) { return (g.sh_count == 0 || r < g.sh_rows0) ? g.row_map[r] : r; };
         for (;;) {
             if (!mbar_wait(&S->itf[rs], rphase, g.wait_ns)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
             const int item = S->ring[rs];
@@ -258,29 +342,29 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
             if (lane == 0) mbar_arrive(&S->ite[rs]);
             if (++rs == RING) { rs = 0; rphase ^= 1; }
             if (item < 0) break;
-            const int mt = item / n_tiles, nt = item - (item / n_tiles) * n_tiles;
-            int row0 = mt * BM, rows = 0;
+            const ItemPos ip = pos_of(item);
+            const bool p1 = ip.p1;
+            const int nt = ip.nt;
+            int row0 = ip.mt * BM, rows = 0;
             if (dense) {
                 rows = min(BM, g.M - row0);
             } else {
-                const TileRef tr = tile_ref(g.tiles, nrouted, mt, BM, MODE, g.sh_T, g.sh_rows0, g.sh_e0);
+                const TileRef tr = tile_ref(g.tiles, nrouted, ip.mt, BM, p1 ? 1 : 0, g.sh_T, g.sh_rows0, g.sh_e0);
                 row0 = tr.row0;
                 rows = tr.rows;
             }
             const bool row_ok = row < rows;
-            // y row of sorted row r: the row map's for the routed rows, r itself for the shared expert's
-            auto flat_of = [&](int r) { return (g.sh_count == 0 || r < g.sh_rows0) ? g.row_map[r] : r; };
             if (!mbar_wait(&S->accf[acc], aphase, g.wait_ns)) { record_status(g.status, MOE_ERR_TIMEOUT); break; }
             tc_fence_after();
             const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-            if (MODE == 0) {
+            if (!p1) {
                 __nv_bfloat16 *orow = g.out + (size_t)(row0 + row) * g.N;
 #pragma unroll 1
-                for (int c = 0; c < BNO / 32; ++c) {
+                for (int c = 0; c < BNO0 / 32; ++c) {
                     uint32_t gr[32], ur[32];
                     tmem_ld32_sync(tb + c * 32, gr);
-                    tmem_ld32_sync(tb + BNO + c * 32, ur);
-                    const int col = nt * BNO + c * 32;
+                    tmem_ld32_sync(tb + BNO0 + c * 32, ur);
+                    const int col = nt * BNO0 + c * 32;
                     if (row_ok && col < g.N) {
                         uint32_t pk[16];
 #pragma unroll
@@ -297,10 +381,10 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
             } else if (MODE == 2) {
                 float *orow = g.out_f32 + (size_t)(row0 + row) * g.N;
 #pragma unroll 1
-                for (int c = 0; c < BNO / 32; ++c) {
+                for (int c = 0; c < BNO1 / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld32_sync(tb + c * 32, r);
-                    const int col = nt * BNO + c * 32;
+                    const int col = nt * BNO1 + c * 32;
                     if (row_ok && col + 32 <= g.N && (g.N & 3) == 0) {  // rows 16-byte aligned
                         float4 *dst = reinterpret_cast<float4 *>(orow + col);
 #pragma unroll
@@ -314,14 +398,16 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                     }
                 }
             } else {
+                const int N = MODE == 3 ? g.N2 : g.N;
+                __nv_bfloat16 *y = MODE == 3 ? g.out2 : g.out;
                 const int flat = row_ok ? flat_of(row0 + row) : 0;
-                __nv_bfloat16 *orow = g.out + (size_t)flat * g.N;
+                __nv_bfloat16 *orow = y + (size_t)flat * N;
 #pragma unroll 1
-                for (int c = 0; c < BNO / 32; ++c) {
+                for (int c = 0; c < BNO1 / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld32_sync(tb + c * 32, r);
-                    const int col = nt * BNO + c * 32;
-                    if (row_ok && col < g.N) {
+                    const int col = nt * BNO1 + c * 32;
+                    if (row_ok && col < N) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
@@ -335,9 +421,21 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) mbar_arrive(&S->acce[acc]);
             if (++acc == 2) { acc = 0; aphase ^= 1; }
-            if (MODE == 1 && g.comb_cnt)  // the accumulator is already released
-                combine_arrive(g.out, g.comb_gate, g.comb_out, g.comb_cnt, g.comb_k, g.comb_target, g.N, n_tiles,
-                               nt, row_ok, row_ok ? flat_of(row0 + row) : 0, lane, g.sh_count, g.sh_T, g.sh_rows0);
+            if (MODE == 3 && !p1) {
+                // publish this warp's h rows of m-tile mt to the down items: each lane's
+                // stores before the warp's count (release at GPU scope), visible to the TMA
+                // reads that follow the consumer's acquire
+                fence_proxy_async_global();
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();
+                    atomicAdd(g.ready + ip.mt, 1);
+                }
+            }
+            if ((MODE == 1 || (MODE == 3 && p1)) && g.comb_cnt)  // the accumulator is already released
+                combine_arrive(MODE == 3 ? g.out2 : g.out, g.comb_gate, g.comb_out, g.comb_cnt, g.comb_k,
+                               g.comb_target, MODE == 3 ? g.N2 : g.N, nt1, nt, row_ok,
+                               row_ok ? flat_of(row0 + row) : 0, lane, g.sh_count, g.sh_T, g.sh_rows0);
         }
     }
 
@@ -368,35 +466,38 @@ int num_sms()
 static bool smem_attr_ready(int mode)
 {
     static std::mutex mu;
-    static uint64_t done[3] = {0, 0, 0};  // bit per device
+    static uint64_t done[4] = {0, 0, 0, 0};  // bit per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::lock_guard<std::mutex> lk(mu);
     if (done[mode] >> dev & 1ull) return true;
-    cudaError_t e = mode == 0 ? cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)
-                  : mode == 1 ? cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)
-                              : cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    const int a = (int)SMEM_BYTES;
+    cudaError_t e = mode == 0   ? cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                  : mode == 1 ? cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                  : mode == 2 ? cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                              : cudaFuncSetAttribute(grouped_gemm_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, a);
     if (e != cudaSuccess) return false;
     done[mode] |= 1ull << dev;
     return true;
 }
 
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
-                                const CUtensorMap &tmB1, cudaStream_t st, const SharedMaps *sm)
+                                const CUtensorMap &tmB1, cudaStream_t st, const SharedMaps *sm, const LayerMaps *lm)
 {
     const int grid = g.ctas > 0 ? g.ctas : num_sms();
-    if (!smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
+    if (g.mode < 0 || g.mode > 3 || !smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
     if (g.sh_count && (!sm || g.mode == 2)) return cudaErrorInvalidValue;
+    if (g.mode == 3 && (!lm || !g.ready)) return cudaErrorInvalidValue;
     static const SharedMaps none{};
+    static const LayerMaps nolm{};
     const SharedMaps &s = sm ? *sm : none;
-    cudaError_t e;
-    if (g.mode == 0)
-        e = launch_pdl(grouped_gemm_kernel<0>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s);
-    else if (g.mode == 1)
-        e = launch_pdl(grouped_gemm_kernel<1>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s);
-    else
-        e = launch_pdl(grouped_gemm_kernel<2>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s);
-    return e;
+    const LayerMaps &l = lm ? *lm : nolm;
+    switch (g.mode) {
+    case 0: return launch_pdl(grouped_gemm_kernel<0>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s, l);
+    case 1: return launch_pdl(grouped_gemm_kernel<1>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s, l);
+    case 2: return launch_pdl(grouped_gemm_kernel<2>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s, l);
+    default: return launch_pdl(grouped_gemm_kernel<3>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s, l);
+    }
 }
 
 }  // namespace moe

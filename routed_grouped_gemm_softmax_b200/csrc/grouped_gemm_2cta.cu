@@ -20,6 +20,7 @@
 // bounded, and a CTA leaves only after the other has finished touching it.
 #include <mutex>
 
+#include "combine.cuh"
 #include "moe_internal.h"
 #include "pdl.cuh"
 #include "sm100_ptx.cuh"
@@ -406,6 +407,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                 else arrive_remote(peer_addr(&S->acce[acc], 0));
             }
             if (++acc == 2) { acc = 0; aphase ^= 1; }
+            if (MODE == 1 && g.comb_cnt)  // the accumulator is already released
+                combine_arrive(g.out, g.comb_gate, g.comb_out, g.comb_cnt, g.comb_k, g.comb_target, g.N, n_tiles,
+                               nt, row_ok, row_ok ? flat_of(row0 + row) : 0, lane, g.sh_count, g.sh_T, g.sh_rows0);
         }
     }
 
@@ -450,8 +454,9 @@ bool smem2_ready(int mode)
 
 cudaError_t launch_grouped_gemm_2cta(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                      const CUtensorMap &tmB1, const int32_t *tiles2, const int32_t *ntiles2,
-                                     cudaStream_t st, const SharedMaps *sm)
+                                     cudaStream_t st, const SharedMaps *sm, const LayerMaps *lm)
 {
+    if (lm) return cudaErrorInvalidValue;  // the fused layer launch takes 128-row tiles
     int grid = (g.ctas > 0 ? g.ctas : num_sms()) / 2 * 2;
     if (grid < 2) grid = 2;
     if (!smem2_ready(g.mode)) return cudaErrorInvalidValue;

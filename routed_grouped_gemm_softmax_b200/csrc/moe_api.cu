@@ -18,11 +18,16 @@
 
 namespace {
 
+// The fused gate/up + down launch is the default for one-CTA tiles (the layer kernel).
+constexpr bool kLayerGemmAuto = true;
+
 std::atomic<int> g_gemm_ctas{0};
 std::atomic<int> g_claim_reverse{0};
 std::atomic<unsigned long long *> g_trace{nullptr};
 std::atomic<int> g_pair_mode{0};  // 0 auto, 1 pair GEMMs whenever possible, 2 never
 std::atomic<int> g_fp8_swap{0};   // 0 auto, 1 swapped fp8 gate/up GEMM always, 2 never
+std::atomic<int> g_fused_comb{0}; // 0 auto, 1 combine inside the down GEMM always, 2 never
+std::atomic<int> g_layer_gemm{0}; // 0 auto, 1 gate/up and down GEMMs in one launch always, 2 never
 std::atomic<int> g_trace_ctas{0};
 std::atomic<unsigned long long> g_wait_ns{0};
 std::atomic<int> g_stall_test{0};
@@ -128,9 +133,11 @@ bool encode_3d_fp4(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Scale codes (bytes) [E, rows, cols] (E = 1 for a 2-D matrix), boxes of 16 codes x
-// box_rows, no swizzle.
-bool encode_scales_u8(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows)
+// Scale codes (bytes) [E, rows, cols], boxes of 16 codes x box_rows, no swizzle: a
+// 3-D map (rank 3, loaded with 3 coordinates) or, with rank 2, a 2-D one over [rows,
+// cols] (E = 1).
+bool encode_scales_u8(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                      int rank)
 {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
@@ -138,7 +145,8 @@ bool encode_scales_u8(CUtensorMap *m, const void *base, uint64_t E, uint64_t row
     const cuuint64_t strides[2] = {cols, rows * cols};
     const cuuint32_t box[3] = {16, box_rows, 1};
     const cuuint32_t es[3] = {1, 1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, E > 1 ? 3 : 2, const_cast<void *>(base), dims, strides, box, es,
+    if (rank != 3 && !(rank == 2 && E == 1)) return false;
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -192,6 +200,23 @@ moe::RouterScratch router_scratch(void *ws, const moe::WsLayout &L, const moe_di
         rs.audit_d = g_audit_d;
     }
     return rs;
+}
+
+// The bf16 forward's choice of kernels for these dims under the current settings
+// (MOE_PLAN_* bits).
+int bf16_plan(const moe_dims_t &d)
+{
+    const long A = (long)d.T * d.top_k;
+    const bool small = moe::small_route_permute_ok(d);
+    const int pair_mode = g_pair_mode.load();
+    const bool pairs = pair_mode != 2 && g_claim_reverse.load() <= 1 && !small &&
+                       (pair_mode == 1 || A >= 512L * d.E);
+    const int fc = g_fused_comb.load();
+    const bool fused = fc == 1 || (fc == 0 && d.T <= moe::kFusedCombineMaxT);
+    const int lg = g_layer_gemm.load();
+    const bool layer = !pairs && (lg == 1 || (lg == 0 && kLayerGemmAuto));
+    return (small ? MOE_PLAN_SMALL_ROUTER : 0) | (pairs ? MOE_PLAN_PAIR_TILES : 0) |
+           (fused ? MOE_PLAN_FUSED_COMBINE : 0) | (layer ? MOE_PLAN_LAYER_GEMM : 0);
 }
 
 // Activations, weights and outputs are read and written in 16-byte vectors (and the
@@ -317,6 +342,8 @@ void moe_set_claim_order(int32_t mode) { g_claim_reverse.store(mode < 0 ? 0 : mo
 
 void moe_set_pair_mma(int32_t mode) { g_pair_mode.store(mode < 0 || mode > 2 ? 0 : mode); }
 void moe_set_fp8_swap_ab(int32_t mode) { g_fp8_swap.store(mode < 0 || mode > 2 ? 0 : mode); }
+void moe_set_fused_combine(int32_t mode) { g_fused_comb.store(mode < 0 || mode > 2 ? 0 : mode); }
+void moe_set_layer_gemm(int32_t mode) { g_layer_gemm.store(mode < 0 || mode > 2 ? 0 : mode); }
 
 void moe_set_gemm_trace(unsigned long long *trace, int32_t ctas)
 {
@@ -436,9 +463,8 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
     CUtensorMap tm_wg, tm_wu, tm_wd;
     // pair-of-CTA GEMMs for groups large enough to be compute-bound (on average at
     // least 512 rows per expert), on the queue's claim modes
-    const int pair_mode = g_pair_mode.load();
-    const bool pairs = pair_mode != 2 && g_claim_reverse.load() <= 1 && !moe::small_route_permute_ok(*d) &&
-                       (pair_mode == 1 || (long)A >= 512L * d->E);
+    const int plan = bf16_plan(*d);
+    const bool pairs = plan & MOE_PLAN_PAIR_TILES;
     if (!moe::encode_a_maps(&tm_xs, xs, A, d->H, false) ||
         !encode_3d(&tm_wg, w_gate, d->E, d->I, d->H, 128) ||
         !encode_3d(&tm_wu, w_up, d->E, d->I, d->H, 128) ||
@@ -455,7 +481,7 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
         return MOE_ERR_CUDA;
 
     const StageMarks marks;
-    const bool fused = d->T <= moe::kFusedCombineMaxT;  // combine inside the down GEMM
+    const bool fused = plan & MOE_PLAN_FUSED_COMBINE;  // combine inside the down GEMM
     cudaError_t e = marks.mark(0, st);
     if (e == cudaSuccess && !moe::small_route_permute_ok(*d))  // else the router's kernels clear them
         e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);          // header + combine counts
@@ -469,7 +495,31 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
     const unsigned long long wl = g_wait_ns.load();
     const uint64_t wait_ns = wl ? wl : 2000000000ull;
     const int stall = g_stall_test.load();
-    if (e == cudaSuccess) {
+    // the gate/up and the down GEMM in one persistent launch (readiness counters per
+    // m-tile hand h from one to the other)
+    const bool layer = plan & MOE_PLAN_LAYER_GEMM;
+    if (e == cudaSuccess && layer) {
+        moe::GemmArgs gl{3, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, h, s2f, ctas, rev, wait_ns,
+                         stall, 0, nullptr, gate, fused ? at<int32_t>(ws, L.ccnt) : nullptr,
+                         static_cast<__nv_bfloat16 *>(out), d->top_k, d->top_k + sh};
+        gl.trace = trace1;
+        gl.sh_count = sh;
+        gl.sh_T = d->T;
+        gl.sh_rows0 = A;
+        gl.sh_e0 = d->E;
+        gl.K2 = d->I;
+        gl.N2 = d->H;
+        gl.out2 = y;
+        gl.ready = at<int32_t>(ws, L.ready);
+        moe::LayerMaps lm{};
+        lm.h = tm_h;
+        lm.wd = tm_wd;
+        lm.wd_sh = sm2.b0;
+        e = moe::launch_grouped_gemm(gl, tm_xs, tm_wg, tm_wu, st, &sm1, &lm);
+        if (e == cudaSuccess) e = marks.mark(3, st);
+        if (e == cudaSuccess) e = marks.mark(4, st);
+    }
+    if (e == cudaSuccess && !layer) {
         moe::GemmArgs g1{0, d->H, d->I, tiles, ntiles, &hdr->counter[0], &hdr->status, h, nullptr, ctas, rev, wait_ns, stall};
         g1.trace = trace1;
         g1.sh_count = sh;
@@ -479,9 +529,9 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
         e = pairs ? moe::launch_grouped_gemm_2cta(g1, tm_xs, tm_wg, tm_wu, at<int32_t>(ws, L.tiles2),
                                                   at<int32_t>(ws, L.ntiles2), st, &sm1)
                   : moe::launch_grouped_gemm(g1, tm_xs, tm_wg, tm_wu, st, &sm1);
+        if (e == cudaSuccess) e = marks.mark(3, st);
     }
-    if (e == cudaSuccess) e = marks.mark(3, st);
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && !layer) {
         moe::GemmArgs g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, y, s2f, ctas, rev, wait_ns,
                          stall, 0, nullptr, gate, fused ? at<int32_t>(ws, L.ccnt) : nullptr,
                          static_cast<__nv_bfloat16 *>(out), d->top_k, d->top_k + sh};
@@ -493,8 +543,8 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
         e = pairs ? moe::launch_grouped_gemm_2cta(g2, tm_h, tm_wd, tm_wd, at<int32_t>(ws, L.tiles2),
                                                   at<int32_t>(ws, L.ntiles2), st, &sm2)
                   : moe::launch_grouped_gemm(g2, tm_h, tm_wd, tm_wd, st, &sm2);
+        if (e == cudaSuccess) e = marks.mark(4, st);
     }
-    if (e == cudaSuccess) e = marks.mark(4, st);
     if (e == cudaSuccess && !fused)
         e = moe::launch_combine(y, gate, d->T, d->H, d->top_k, static_cast<__nv_bfloat16 *>(out), st, sh, A);
     if (e == cudaSuccess) e = marks.mark(5, st);
@@ -644,12 +694,12 @@ moe_status_t moe_forward_mx(const moe_dims_t *d, const void *x, const void *rout
                      ctas, rev, wait_ns, stall, trace2};
     if (!moe::encode_a_maps(&g1.tmX, xs, A, d->H, true) || !encode_3d_fp4(&g1.tmW0, w_gate_p, d->E, d->I, d->H, 128) ||
         !encode_3d_fp4(&g1.tmW1, w_up_p, d->E, d->I, d->H, 128) ||
-        !encode_scales_u8(&g1.tmSX, xs_x, 1, A, d->H / 32, 64) ||
-        !encode_scales_u8(&g1.tmSW0, w_gate_x, d->E, d->I, d->H / 32, 128) ||
-        !encode_scales_u8(&g1.tmSW1, w_up_x, d->E, d->I, d->H / 32, 128) ||
+        !encode_scales_u8(&g1.tmSX, xs_x, 1, A, d->H / 32, 64, 2) ||
+        !encode_scales_u8(&g1.tmSW0, w_gate_x, d->E, d->I, d->H / 32, 128, 3) ||
+        !encode_scales_u8(&g1.tmSW1, w_up_x, d->E, d->I, d->H / 32, 128, 3) ||
         !moe::encode_a_maps(&g2.tmX, h, A, d->I, true) || !encode_3d_fp4(&g2.tmW0, w_down_p, d->E, d->H, d->I, 128) ||
-        !encode_scales_u8(&g2.tmSX, h_x, 1, A, d->I / 32, 64) ||
-        !encode_scales_u8(&g2.tmSW0, w_down_x, d->E, d->H, d->I / 32, 128))
+        !encode_scales_u8(&g2.tmSX, h_x, 1, A, d->I / 32, 64, 2) ||
+        !encode_scales_u8(&g2.tmSW0, w_down_x, d->E, d->H, d->I / 32, 128, 3))
         return MOE_ERR_CUDA;
     g2.tmW1 = g2.tmW0;    // the down GEMM's two tiles are rows n0.. and n0+128.. of w_down
     g2.tmSW1 = g2.tmSW0;
@@ -676,12 +726,23 @@ moe_status_t moe_forward_mx(const moe_dims_t *d, const void *x, const void *rout
     return cuda_status(e);
 }
 
+int32_t moe_forward_plan(const moe_dims_t *d, int dtype)
+{
+    if (moe_workspace_size(d, dtype) == 0) return -1;
+    if (dtype != MOE_DTYPE_BF16) {  // the fp8 and MX forwards: small router, fused combine for fp8
+        const bool fused = dtype == MOE_DTYPE_FP8 && d->T <= moe::kFusedCombineMaxT;
+        return (moe::small_route_permute_ok(*d) ? MOE_PLAN_SMALL_ROUTER : 0) | (fused ? MOE_PLAN_FUSED_COMBINE : 0);
+    }
+    return bf16_plan(*d);
+}
+
 moe_status_t moe_workspace_offsets(const moe_dims_t *d, int dtype, size_t *out, int32_t n)
 {
     if (!out || n < 0 || moe_workspace_size(d, dtype) == 0) return MOE_ERR_INVALID_ARG;
     const moe::WsLayout L = moe::ws_layout(*d, dtype);
-    const size_t v[8] = {L.idx, L.gate, L.offsets, L.s2f, L.f2s, L.tiles, L.ntiles, L.logits};
-    for (int i = 0; i < n && i < 8; ++i) out[i] = v[i];
+    const size_t v[13] = {L.idx, L.gate, L.offsets, L.s2f, L.f2s, L.tiles, L.ntiles, L.logits,
+                          L.xs, L.xs_s, L.h, L.h_s, L.y};
+    for (int i = 0; i < n && i < 13; ++i) out[i] = v[i];
     return MOE_OK;
 }
 

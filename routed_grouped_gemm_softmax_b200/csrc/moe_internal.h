@@ -24,7 +24,7 @@ struct WsHeader {
 
 // Byte offsets of every region of the workspace (256-byte aligned each).
 struct WsLayout {
-    size_t ccnt, clear_bytes, logits, wrt, wsq, rncand, rlist, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, tiles2, ntiles2, xq, xq_s, xs, xs_s, h, h_s, y,
+    size_t ccnt, ready, clear_bytes, logits, wrt, wsq, rncand, rlist, blk_cnt, blk_base, idx, gate, offsets, s2f, f2s, tiles, ntiles, tiles2, ntiles2, xq, xq_s, xs, xs_s, h, h_s, y,
         total;
     int nb;      // permutation chunks
     int chunk;   // flat entries per chunk
@@ -59,10 +59,14 @@ inline WsLayout ws_layout(const moe_dims_t &d, int dtype = MOE_DTYPE_BF16, int s
     L.nb = static_cast<int>((A + L.chunk - 1) / L.chunk);
     const size_t max_tiles = (A + kTileRows - 1) / kTileRows + (A < (size_t)d.E ? A : (size_t)d.E);
     size_t o = align_up(sizeof(WsHeader), 256);
-    // the fused combine's arrival counts follow the header, so one memset clears both
+    // the fused combine's arrival counts and the fused layer GEMM's per-m-tile
+    // readiness counts follow the header, so one memset clears all three
+    const size_t mtiles = (A + kTileRows - 1) / kTileRows + (A < (size_t)d.E ? A : (size_t)d.E) +
+                          static_cast<size_t>(sh_count) * ((d.T + kTileRows - 1) / kTileRows);
     L.ccnt = o;
-    o = align_up(o + static_cast<size_t>(d.T) * ((d.H + 255) / 256) * 4, 1024);
-    L.clear_bytes = L.ccnt + static_cast<size_t>(d.T) * ((d.H + 255) / 256) * 4;
+    L.ready = L.ccnt + static_cast<size_t>(d.T) * ((d.H + 255) / 256) * 4;
+    L.clear_bytes = L.ready + mtiles * 4;
+    o = align_up(L.clear_bytes, 1024);
     auto take = [&](size_t bytes) {
         size_t at = o;
         o = align_up(o + bytes, 1024);
@@ -196,6 +200,22 @@ struct GemmArgs {
     int sh_T;
     int sh_rows0;
     int sh_e0;
+    // Mode 3, the gate/up and the down GEMM in one persistent launch: the gate/up items
+    // (K, N, out = h) come first in the claim order, then the down items (K2, N2, out2
+    // = y, row_map, fused combine as in mode 1).  A down item of m-tile mt waits (at
+    // most wait_ns) until ready[mt] counts the 4 epilogue warps of every gate/up item
+    // of mt (2 x 4 for pair tiles), then reads those h rows.  ready is zeroed before
+    // the launch.
+    int K2, N2;
+    __nv_bfloat16 *out2;
+    int32_t *ready;
+};
+
+// Tensor maps of the down half of the fused layer GEMM (mode 3): h as its A operand
+// (16 to 128-row boxes), the down weights (3-D) and the shared expert's (2-D).
+struct LayerMaps {
+    AMaps h;
+    CUtensorMap wd, wd_sh;
 };
 
 // Tensor maps of the shared expert: x as the gate/up GEMM's A operand (boxes of 16
@@ -236,13 +256,14 @@ __device__ __forceinline__ TileRef tile_ref(const int32_t *tiles, int nrouted, i
 }
 // mode 2: out_f32 = A B^T over M rows (one "expert"), the router's tensor-core logits.
 cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
-                                const CUtensorMap &tmB1, cudaStream_t st, const SharedMaps *sm = nullptr);
+                                const CUtensorMap &tmB1, cudaStream_t st, const SharedMaps *sm = nullptr,
+                                const LayerMaps *lm = nullptr);
 
 // The bf16 grouped GEMMs (modes 0 and 1) on CTA pairs, cta_group::2 MMAs over the
 // 2 x 128-row pair tiles tiles2 (grouped_gemm_2cta.cu); queue claim modes only.
 cudaError_t launch_grouped_gemm_2cta(const GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                      const CUtensorMap &tmB1, const int32_t *tiles2, const int32_t *ntiles2,
-                                     cudaStream_t st, const SharedMaps *sm = nullptr);
+                                     cudaStream_t st, const SharedMaps *sm = nullptr, const LayerMaps *lm = nullptr);
 
 // FP8 block-scaled grouped GEMMs (fp8.cu).  mode 0: h codes/scales from
 // silu(A Wg^T) * (A Wu^T); mode 1: y[row_map[row]] = A Wd^T in bf16; mode 2:

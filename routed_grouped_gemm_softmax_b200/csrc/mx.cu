@@ -22,11 +22,14 @@
 // rows, which TMA expands on the way in from 16 packed codes in 8 bytes to 16 bytes
 // (the 16U4_ALIGN16B type: the layout the MMA reads for 4-bit operands), both with
 // the 128-byte swizzle.  The scales travel separately: every 4 stages TMA brings a
-// [rows x 16 bytes] block of each operand's e8m0 codes (4 stages x 4 blocks of 32),
-// and four scale warps copy each stage's codes into tensor memory with tcgen05.st
-// in the layout the MMA reads: the scale of M row m in lane m, column m / 32; of N
-// row n in lane n % 32, column n / 32; byte j of the 32-bit cell for the j-th K=32
-// MMA of the stage (its scale-factor id).
+// [rows x 16 bytes] block of each operand's e8m0 codes (4 stages x 4 blocks of 32);
+// four scale warps rearrange each stage's codes in shared memory into 32-row x
+// 16-byte blocks (row r, word w: the codes of operand row 32w + r), and the MMA
+// thread copies those into tensor memory with tcgen05.cp (32x128b, replicated to the
+// four lane quarters), in order with the MMAs that read them.  In tensor memory the
+// MMA finds the scale of M row m in lane m, column m / 32, and of N row n in lane
+// n % 32, column n / 32; byte j of the 32-bit cell for the j-th K=32 MMA of the stage
+// (its scale-factor id).
 //
 // CTA roles (320 threads): warp 0 claims items and streams tiles and scale blocks
 // (TMA); warp 1 owns TMEM and issues the MMAs; warps 2-5 drain the accumulators --
@@ -56,6 +59,7 @@ constexpr int W_TX = FR * KE / 2;       // 8 KB: its transaction bytes (TMA coun
 constexpr int SW_BYTES = FR * 16;       // 2 KB: scale block of one weight tile
 constexpr int SX_BYTES = XR * 16;       // 1 KB: scale block of the token rows
 constexpr int SBUF = 2 * SW_BYTES + SX_BYTES;
+constexpr int CP_BYTES = 3 * 512;       // per stage: the tcgen05.cp sources of weight tiles 0, 1 and the tokens
 constexpr int MTHREADS = 320;
 constexpr uint32_t MTMEM_COLS = 512;
 constexpr uint32_t ACC_COLS = 2 * XR;   // one accumulator buffer: two 64-column accumulators
@@ -72,7 +76,7 @@ struct CtrlM {
     uint32_t tmem_base;
 };
 
-constexpr size_t SMEMM = 1024 + (size_t)MST * (X_BYTES + 2 * W_BYTES) + 2 * SBUF + sizeof(CtrlM);
+constexpr size_t SMEMM = 1024 + (size_t)MST * (X_BYTES + 2 * W_BYTES + CP_BYTES) + 2 * SBUF + sizeof(CtrlM);
 static_assert(SMEMM <= 227 * 1024, "shared memory of the MX GEMM");
 static_assert(SF_COL0 + MST * SF_SLOT <= MTMEM_COLS && 2 * ACC_COLS <= SF_COL0, "TMEM columns of the MX GEMM");
 
@@ -111,15 +115,26 @@ __device__ __forceinline__ void mma_mx(uint32_t d, uint64_t adesc, uint64_t bdes
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v)
+// Shared-memory descriptor of a 32-row x 16-byte block without swizzle (8-row core
+// matrices of 128 contiguous bytes), the source of a 32x128b tcgen05.cp.
+__device__ __forceinline__ uint64_t cp_desc(uint32_t saddr)
 {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(128u >> 4) << 16;  // leading byte offset
+    d |= static_cast<uint64_t>(128u >> 4) << 32;  // stride byte offset: the next 8 rows
+    d |= 1ull << 46;                              // descriptor version
+    return d;
 }
-__device__ __forceinline__ void tmem_st2(uint32_t taddr, uint32_t v0, uint32_t v1)
+
+// Tensor memory columns taddr .. taddr+3 of all 128 lanes <- a 32-row x 16-byte block,
+// row r to lanes r, r+32, r+64 and r+96.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc)
 {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(v0), "r"(v1) : "memory");
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // The MX scale exponent of a block whose largest magnitude is amax: floor(log2 amax)
 // minus the element format's largest exponent (8 for e4m3), within [-127, 127]; 0
@@ -131,10 +146,13 @@ __device__ __forceinline__ int mx_exponent(float amax)
     return x < -127 ? -127 : x > 127 ? 127 : x;
 }
 
-// e4m3 code of v / 2^X, rounded to nearest even and clamped to +-448.
+// e4m3 code of v / 2^X, rounded to nearest even and clamped to +-448; a value that
+// rounds to zero is coded +0 whatever its sign (the MX element conversion here keeps
+// no signed zero).
 __device__ __forceinline__ uint8_t mx_e4m3(float v, int X)
 {
-    return e4m3_one(fminf(fmaxf(ldexpf(v, -X), -448.0f), 448.0f));
+    const uint8_t c = e4m3_one(fminf(fmaxf(ldexpf(v, -X), -448.0f), 448.0f));
+    return (c & 0x7Fu) ? c : 0;
 }
 
 struct MxGemmArgs {
@@ -170,7 +188,8 @@ grouped_gemm_mx_kernel(const __grid_constant__ AMaps tmX, const __grid_constant_
     uint8_t *sX = smem_raw + pad;
     uint8_t *sW = sX + MST * X_BYTES;       // [stage][2][W_BYTES]
     uint8_t *sS = sW + MST * 2 * W_BYTES;   // [2][SBUF]: weight 0, weight 1, token scale blocks
-    CtrlM *S = reinterpret_cast<CtrlM *>(sS + 2 * SBUF);
+    uint8_t *sC = sS + 2 * SBUF;            // [stage][CP_BYTES]: the stage's scales in the tcgen05.cp layout
+    CtrlM *S = reinterpret_cast<CtrlM *>(sC + MST * CP_BYTES);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int mode = g.mode;
@@ -298,6 +317,10 @@ grouped_gemm_mx_kernel(const __grid_constant__ AMaps tmX, const __grid_constant_
                     const uint32_t x0 = smem_u32(sX + stage * X_BYTES);
                     const uint32_t w0 = smem_u32(sW + stage * 2 * W_BYTES), w1 = w0 + W_BYTES;
                     const uint32_t sf = tmem + SF_COL0 + static_cast<uint32_t>(stage) * SF_SLOT;
+                    const uint32_t cp0 = smem_u32(sC + stage * CP_BYTES);
+                    tmem_cp_32x128b_x4(sf, cp_desc(cp0));             // weight tile 0
+                    tmem_cp_32x128b_x4(sf + 4, cp_desc(cp0 + 512));   // weight tile 1
+                    tmem_cp_32x128b_x4(sf + 8, cp_desc(cp0 + 1024));  // token rows
 #pragma unroll
                     for (int k = 0; k < KE / 32; ++k) {
                         const uint64_t xd = sw128_kmajor_desc(x0 + k * 32);
@@ -376,11 +399,10 @@ grouped_gemm_mx_kernel(const __grid_constant__ AMaps tmX, const __grid_constant_
         if (!ok) record(g.status, MOE_ERR_TIMEOUT);
     } else {
         // ---------------------------------------------------------- scale warps
-        // Quarter q writes, for its 32 lanes, the weight rows' scales of each stage
-        // (lane m of the quarter: weight row 32q + m, column q of the slot), and
-        // quarter 0 also the token rows' (lane m: tokens m and m + 32, columns 0, 1).
+        // Per stage, thread (q, lane) moves the codes of weight row 32q + lane of each
+        // tile to word q of row `lane` of that tile's 32 x 16-byte block; the quarter-0
+        // warp also moves tokens lane and lane + 32 to words 0 and 1 of the token block.
         const int q = warp & 3;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
         int rs = 0, stage = 0, gb = 0;
         uint32_t rphase = 0, phase = 0, gphase = 0;
         bool ok = true;
@@ -394,23 +416,25 @@ grouped_gemm_mx_kernel(const __grid_constant__ AMaps tmX, const __grid_constant_
             if (item_rows_m(g.tiles, item, n_tiles).rows <= 0) continue;
             for (int kb = 0; kb < KB && ok; ++kb) {
                 if (kb % SG == 0 && !mbar_wait(&S->sgf[gb], gphase, g.wait_ns)) { ok = false; break; }
+                // the MMAs (and copies) of this stage's previous use are done with its buffer
                 if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
-                tc_fence_after();
                 const uint8_t *sb = sS + gb * SBUF;
+                uint8_t *cp = sC + stage * CP_BYTES;
                 const int u = kb % SG;
                 const int m = q * 32 + lane;
-                const uint32_t v0 = *reinterpret_cast<const uint32_t *>(sb + m * 16 + u * 4);
-                const uint32_t v1 = *reinterpret_cast<const uint32_t *>(sb + SW_BYTES + m * 16 + u * 4);
-                const uint32_t slot = lane_base + SF_COL0 + static_cast<uint32_t>(stage) * SF_SLOT;
-                tmem_st1(slot + q, v0);
-                tmem_st1(slot + 4 + q, v1);
+                *reinterpret_cast<uint32_t *>(cp + lane * 16 + q * 4) =
+                    *reinterpret_cast<const uint32_t *>(sb + m * 16 + u * 4);
+                *reinterpret_cast<uint32_t *>(cp + 512 + lane * 16 + q * 4) =
+                    *reinterpret_cast<const uint32_t *>(sb + SW_BYTES + m * 16 + u * 4);
                 if (q == 0) {
                     const uint8_t *sx = sb + 2 * SW_BYTES;
-                    tmem_st2(slot + 8, *reinterpret_cast<const uint32_t *>(sx + lane * 16 + u * 4),
-                             *reinterpret_cast<const uint32_t *>(sx + (lane + 32) * 16 + u * 4));
+                    uint4 t;
+                    t.x = *reinterpret_cast<const uint32_t *>(sx + lane * 16 + u * 4);
+                    t.y = *reinterpret_cast<const uint32_t *>(sx + (lane + 32) * 16 + u * 4);
+                    t.z = t.w = 0x7F7F7F7Fu;  // unused columns (N <= 64)
+                    *reinterpret_cast<uint4 *>(cp + 1024 + lane * 16) = t;
                 }
-                tmem_st_wait();
-                tc_fence_before();
+                fence_proxy_async_smem();  // the writes above, before the tensor cores' copy reads them
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S->sff[stage]);
                 if (u == SG - 1 || kb == KB - 1) {  // done with this scale block

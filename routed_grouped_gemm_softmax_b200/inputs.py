@@ -107,9 +107,10 @@ class MoEConfig:
     top_k: int
     I: int
     seed: int
-    dtype: str = "bf16"          # "bf16" or "fp8"
+    dtype: str = "bf16"          # "bf16", "fp8" or "mx" (e2m1 weights, e4m3 activations)
     zipf_s: float | None = None  # per-expert router bias making popularity ~ Zipf(s)
     router_std: float = 0.02
+    shared_mult: int = 0         # a shared expert of shared_mult * I columns (0: none)
 
     @property
     def A(self) -> int:
@@ -127,6 +128,14 @@ CONFIGS = {
     "prefill": MoEConfig("prefill", T=4096, H=2048, E=256, top_k=8, I=512, seed=2),
     "skewed": MoEConfig("skewed", T=8192, H=4096, E=64, top_k=6, I=1408, seed=3, zipf_s=1.2),
     "fp8": MoEConfig("fp8", T=1024, H=7168, E=256, top_k=8, I=2048, seed=4, dtype="fp8"),
+}
+
+# Further workloads of the layer's variants (not among the five configurations above):
+# the MX (FP4 weight) layer on the FP8 workload's shapes and inputs, and the Prefill
+# workload with a shared expert of 2 x I columns.
+EXTRA_WORKLOADS = {
+    "mx": CONFIGS["fp8"].replace(name="mx", dtype="mx"),
+    "prefill_shared": CONFIGS["prefill"].replace(name="prefill_shared", shared_mult=2),
 }
 
 
@@ -250,6 +259,14 @@ def make_shared_weights(cfg: MoEConfig, shared_I: int, device="cpu"):
     wu = gaussian_tensor(cfg.seed, "shared_up", (shared_I, H), 1.0 / math.sqrt(H), device)
     wd = gaussian_tensor(cfg.seed, "shared_down", (H, shared_I), 1.0 / math.sqrt(shared_I), device)
     return wg, wu, wd
+
+
+def pack_e2m1(codes: torch.Tensor) -> torch.Tensor:
+    """e2m1 codes one per byte [..., K] -> two per byte [..., K/2]: the code of element
+    2i in the low nibble of byte i, of element 2i+1 in the high nibble (the packed
+    FP4 storage the MX layer reads)."""
+    c = codes.to(torch.uint8)
+    return (c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)
 
 
 def make_inputs(cfg: MoEConfig, device="cpu", weights: bool = True) -> MoEInputs:

@@ -167,3 +167,38 @@ def test_load_peaks_carries_the_sm_clock():
     p, kind = bench.load_peaks()
     assert kind in ("measured", "fallback") and p["sm_max_mhz"] > 0
     assert all(k in p for k in bench.FALLBACK_PEAKS)
+
+
+def test_stage_work_mx_and_shared_by_hand():
+    # MX: e2m1 weights at half a byte plus one e8m0 byte per 32 along K; e4m3 activation
+    # codes plus one byte per 32 values
+    cfg = CONFIGS["fp8"].replace(name="wmx", T=4, H=512, I=512, E=4, top_k=2, dtype="mx")
+    w = bench.stage_work(cfg, [8, 0, 0, 0])  # one expert, A = 8
+    weights = 2 * (512 * 512 // 2 + 512 * 512 // 32)
+    rows = 8 * 512 + 8 * 512 // 32
+    assert w["gemm_gate_up"]["bytes"] == weights + rows + rows == 286976
+    assert w["gemm_down"]["bytes"] == (512 * 256 + 512 * 16) + rows + 8 * 512 * 2
+    # a shared expert of 2 x I columns: its weights, x and h rows, and FLOPs on top
+    sh = CONFIGS["tiny"].replace(name="wsh", T=4, H=256, I=128, E=4, top_k=2, shared_mult=2)
+    base = bench.stage_work(sh.replace(shared_mult=0), [3, 0, 5, 0])
+    ws = bench.stage_work(sh, [3, 0, 5, 0])
+    assert ws["gemm_gate_up"]["bytes"] - base["gemm_gate_up"]["bytes"] == 2 * 256 * 256 * 2 + 4 * 256 * 2 + 4 * 256 * 2
+    assert ws["gemm_gate_up"]["flops"] - base["gemm_gate_up"]["flops"] == 2.0 * 4 * 256 * 2 * 256
+    assert ws["gemm_down"]["flops"] - base["gemm_down"]["flops"] == 2.0 * 4 * 256 * 256
+    assert ws["combine"]["bytes"] - base["combine"]["bytes"] == 2 * 4 * 256 * 2
+
+
+def test_layer_work_mx_is_about_half_of_fp8():
+    f8 = bench.layer_work(CONFIGS["fp8"], [1] * 256)
+    mx = bench.layer_work(CONFIGS["fp8"].replace(name="mx", dtype="mx"), [1] * 256)
+    # 3 matrices of 2048 x 7168 per expert: 0.5 + 1/32 bytes per weight against 1 byte + fp32 per 128x128
+    per_mx = 3 * (2048 * 7168 // 2 + 2048 * 7168 // 32)
+    per_f8 = 3 * 2048 * 7168 + 3 * 16 * 56 * 4
+    assert mx["bytes"] - f8["bytes"] == 256 * (per_mx - per_f8)
+    assert mx["flops"] == f8["flops"]
+
+
+def test_kernels_per_forward_variants():
+    assert bench.kernels_per_forward(bench.WORKLOADS["mx"]) == 11   # as fp8 (T > 64: the standalone combine)
+    assert bench.kernels_per_forward(bench.WORKLOADS["mx"].replace(T=16)) == 2 + 2 + 2 + 1  # no fused combine
+    assert bench.kernels_per_forward(bench.WORKLOADS["prefill_shared"]) == 10   # the shared expert adds none

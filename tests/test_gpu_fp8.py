@@ -29,6 +29,7 @@ def test_quantizer_bit_exact():
     a[3, 128:256] = 0.0                    # all-zero group -> scale 1, codes 0
     a[5, :] *= 1e-30                       # tiny values (subnormal e4m3 codes)
     a[7, 0] = 1e4                          # one huge value per group
+    a[7, 5] = -0.004                       # a negative value that rounds to zero: code -0 (0x80)
     q, s = api.moe_quantize_rows_fp8(a.cuda())
     qr, sr = oracle.quantize_rows(a)
     assert np.array_equal(s.cpu().numpy(), sr)

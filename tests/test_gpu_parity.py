@@ -167,6 +167,18 @@ def test_pair_cta_gemms(name):
         api.set_pair_mma("auto")
         api.set_gemm_ctas(0)
         api.set_claim_order(False)
+    # the combine inside the pair down GEMM's epilogue: the same sum in the same order
+    try:
+        api.set_pair_mma("always")
+        api.set_fused_combine("always")
+        for ctas in (0, 6):
+            api.set_gemm_ctas(ctas)
+            outs.append(api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"],
+                                        k).clone())
+    finally:
+        api.set_pair_mma("auto")
+        api.set_fused_combine("auto")
+        api.set_gemm_ctas(0)
     idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], k)
     ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"])
     compare_out(outs[0], ref, f"{name} pair GEMMs")

@@ -58,17 +58,20 @@ def test_shared_expert_pairs_and_schedules():
     sw = [t.cuda() for t in make_shared_weights(cfg, 2 * cfg.I)]
     outs = []
     try:
-        for pair, ctas, mode in [("always", 0, False), ("always", 6, True), ("never", 0, False),
-                                 ("never", 7, "static_items"), ("never", 5, "static_experts")]:
+        for pair, ctas, mode, fused in [("always", 0, False, "never"), ("always", 6, True, "always"),
+                                        ("never", 0, False, "never"), ("never", 7, "static_items", "always"),
+                                        ("never", 5, "static_experts", "never")]:
             api.set_pair_mma(pair)
             api.set_gemm_ctas(ctas)
             api.set_claim_order(mode)
+            api.set_fused_combine(fused)
             outs.append(api.moe_forward_shared(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"],
                                                g["w_down"], *sw, cfg.top_k).clone())
     finally:
         api.set_pair_mma("auto")
         api.set_gemm_ctas(0)
         api.set_claim_order(False)
+        api.set_fused_combine("auto")
     idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], cfg.top_k)
     compare_out(outs[0], _oracle(c, idx_ref, gate_ref, sw), "sh_deep pairs")
     compare_out(outs[2], _oracle(c, idx_ref, gate_ref, sw), "sh_deep one-CTA")
