@@ -72,8 +72,9 @@ def schedule_stats(trace, mode):
     return out
 
 
-def kernels_per_forward(cfg) -> int:
-    """Library kernels one forward launches."""
+def kernels_per_forward(cfg, plan=None) -> int:
+    """Library kernels one forward launches (plan: the library's MOE_PLAN bits for the
+    run's settings, when known; the layer GEMM is one launch for both expert GEMMs)."""
     A = cfg.T * cfg.top_k
     if cfg.T > 32:
         route = 3 + 3      # transpose/norms, tensor-core logits, certify; count, scan, scatter
@@ -85,7 +86,11 @@ def kernels_per_forward(cfg) -> int:
     rows = 2 if cfg.dtype in ("fp8", "mx") else 1   # fp8 / MX: quantise per token, then gather; bf16: gather
     if cfg.dtype == "mx":
         combine = 1   # the MX down GEMM has no fused combine
-    return route + rows + 2 + combine   # + gate/up GEMM, down GEMM
+    gemms = 2
+    if plan is not None and plan >= 0:
+        combine = 0 if plan & 4 else 1       # MOE_PLAN_FUSED_COMBINE
+        gemms = 1 if plan & 8 else 2         # MOE_PLAN_LAYER_GEMM
+    return route + rows + gemms + combine
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 B200_SMS, FP32_LANES_PER_SM = 148, 128   # CUDA-core fp32 FMA lanes of one B200
 
@@ -116,6 +121,8 @@ def parse():
                    help="the bf16 GEMMs on CTA pairs (tcgen05 cta_group::2): automatic choice or forced")
     p.add_argument("--swap-ab", default="auto", choices=["auto", "always", "never"],
                    help="the fp8 gate/up GEMM with swapped MMA operands: automatic choice or forced")
+    p.add_argument("--layer-gemm", default="auto", choices=["auto", "always", "never"],
+                   help="both bf16 expert GEMMs in one persistent launch: automatic choice or forced")
     p.add_argument("--fused-combine", default="auto", choices=["auto", "always", "never"],
                    help="the bf16 combine inside the down GEMM's epilogue: automatic choice or forced")
     p.add_argument("--shape", default="",
@@ -645,6 +652,7 @@ def run_one(args, cfg, world, rank, local):
     api.set_pair_mma(args.pair)
     api.set_fp8_swap_ab(args.swap_ab)
     api.set_fused_combine(args.fused_combine)
+    api.set_layer_gemm(args.layer_gemm)
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
         step()
@@ -713,15 +721,24 @@ def run_one(args, cfg, world, rank, local):
     counts = torch.bincount(idx.view(-1).long(), minlength=cfg.E).tolist()
     work = stage_work(cfg, counts)
     peaks, peaks_kind = load_peaks()
-    dominant = max(("route", "gemm_gate_up", "gemm_down", "combine"), key=lambda s: stage_ms[s])
+    plan = api.forward_plan(cfg.T, cfg.H, cfg.I, cfg.E, k, {"fp8": api.DTYPE_FP8, "mx": api.DTYPE_MX}.get(
+        cfg.dtype, api.DTYPE_BF16))
+    kernels = ["route", "gemm_gate_up", "gemm_down", "combine"]
+    if plan >= 0 and plan & api.PLAN_LAYER_GEMM:
+        # both expert GEMMs run as one launch (the stage marks around it are 2 and 4)
+        work["gemm_layer"] = {"bytes": work["gemm_gate_up"]["bytes"] + work["gemm_down"]["bytes"],
+                              "flops": work["gemm_gate_up"]["flops"] + work["gemm_down"]["flops"]}
+        stage_ms["gemm_layer"] = stage_ms["gemm_gate_up"] + stage_ms["gemm_down"]
+        kernels = ["route", "gemm_layer", "combine"]
+    dominant = max(kernels, key=lambda s: stage_ms[s])
     sustained = total_ms > 1000.0
     roof = roofline_for(dominant, work, stage_ms[dominant], peaks, peaks_kind, sustained, cfg.name, fp8)
     try:  # an extra view of the same step; never allowed to cost the bench line
         layer_roof = layer_roofline(cfg, counts, ms_per_step, peaks, peaks_kind, sustained)
     except Exception as exc:
         layer_roof = {"error": repr(exc)}
-    stages = {s: {"ms": round(stage_ms[s], 4)} for s in api.STAGES}
-    for s in ("route", "gemm_gate_up", "gemm_down", "combine"):
+    stages = {s: {"ms": round(stage_ms[s], 4)} for s in list(api.STAGES) + kernels}
+    for s in kernels:
         r = roofline_for(s, work, stage_ms[s], peaks, peaks_kind, sustained, cfg.name, fp8)
         stages[s].update({"bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"], "frac": r["frac"]})
 
@@ -763,7 +780,8 @@ def run_one(args, cfg, world, rank, local):
                 "dtype": {"fp8": "e4m3", "mx": "e2m1 x e4m3 (mx)"}.get(cfg.dtype, "bf16"),
                 "data": "synthetic", "config": config_block(cfg, world),
                 "roofline": roof, "layer_roofline": layer_roof, "stages": stages, "experts_touched": work["_D"],
-                "e2e": e2e, "gpu_launches": kernels_per_forward(cfg) * args.steps, "schedule": sched,
+                "e2e": e2e, "gpu_launches": kernels_per_forward(cfg, plan) * args.steps, "schedule": sched,
+                "plan": plan,
                 "clocks": clocks, "cpu_baseline": cpu,
                 "p99_ms_per_step": round(sorted(step_ms)[min(len(step_ms) - 1, math.ceil(0.99 * len(step_ms)) - 1)], 5)}
     torch.cuda.synchronize()

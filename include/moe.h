@@ -278,8 +278,7 @@ void moe_set_fused_combine(int32_t mode);
 /* The bf16 forwards' two expert GEMMs in one persistent launch (the layer kernel:
  * every gate/up work item is claimed before any down item, and a down item waits --
  * with a bounded wait -- on a per-m-tile count of the epilogue warps that wrote its
- * h rows) or in two launches.  0 = automatic (one launch for 128-row tiles, two for
- * pair-of-CTA tiles), 1 = one launch whenever the tiles are 128-row ones, 2 = two
+ * h rows) or in two launches.  0 = automatic (one launch), 1 = one launch, 2 = two
  * launches.  Results are bitwise the same.  Process-wide; for tests and benchmarks. */
 void moe_set_layer_gemm(int32_t mode);
 

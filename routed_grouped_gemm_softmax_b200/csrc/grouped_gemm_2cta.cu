@@ -170,14 +170,33 @@ __device__ __forceinline__ uint32_t pack_bf16_2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// MODE 0: h = silu(x Wg^T) * (x Wu^T) -> bf16 rows of h; MODE 1: y rows of x Wd^T.
+// Waits (at most limit_ns) until *ctr >= target, with acquire ordering at GPU scope.
+__device__ __forceinline__ bool wait_count_at_least2(const int32_t *ctr, int target, uint64_t limit_ns)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i) {
+            asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+            if (v >= target) return true;
+        }
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// MODE 0: h = silu(x Wg^T) * (x Wu^T) -> bf16 rows of h; MODE 1: y rows of x Wd^T;
+// MODE 3: the gate/up items, then the down items, in one launch (GemmArgs, mode 3).
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
     grouped_gemm_2cta_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB0,
                              const __grid_constant__ CUtensorMap tmB1, const GemmArgs g, const int32_t *tiles2,
-                             const int32_t *ntiles2, const __grid_constant__ SharedMaps sm)
+                             const int32_t *ntiles2, const __grid_constant__ SharedMaps sm,
+                             const __grid_constant__ LayerMaps lm)
 {
-    constexpr int BNO = MODE == 0 ? BN2 / 2 : BN2;  // output columns per item
+    constexpr int BNO0 = BN2 / 2, BNO1 = BN2;  // output columns of a gate/up item and of a down item
     extern __shared__ uint8_t smem2[];
     const uint32_t pad = (1024u - (smem_u32(smem2) & 1023u)) & 1023u;
     uint8_t *sA = smem2 + pad;
@@ -185,8 +204,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
     Ctrl2 *S = reinterpret_cast<Ctrl2 *>(sB + ST2 * B2_BYTES);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_rank();
-    const int n_tiles = (g.N + BNO - 1) / BNO;
-    const int num_kb = g.K / BK2;
+    const int NP1 = MODE == 3 ? g.N2 : g.N, KP1 = MODE == 3 ? g.K2 : g.K;  // N and K of the down items
+    const int nt0 = (g.N + BNO0 - 1) / BNO0, kb0 = g.K / BK2;
+    const int nt1 = (NP1 + BNO1 - 1) / BNO1, kb1 = KP1 / BK2;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < ST2; ++s) {
@@ -206,10 +226,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
         fence_mbar_init();
         for (int b = 0; b < kABoxes; ++b) tma_prefetch_desc(&tmA.m[b]);
         tma_prefetch_desc(&tmB0);
-        if (MODE == 0) tma_prefetch_desc(&tmB1);
+        if (MODE != 1) tma_prefetch_desc(&tmB1);
+        if (MODE == 3) tma_prefetch_desc(&lm.wd);
         if (g.sh_count) {
             tma_prefetch_desc(&sm.b0);
-            if (MODE == 0) tma_prefetch_desc(&sm.b1);
+            if (MODE != 1) tma_prefetch_desc(&sm.b1);
         }
     }
     if (warp == 1) tmem_alloc_pair(&S->tmem_base, TMEM_COLS2);
@@ -225,12 +246,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
     pdl_trigger();
     if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
+    // pair tiles: the list's, then the shared expert's; in mode 3 every gate/up item
+    // precedes the down items
+    const int nrouted = *ntiles2;
+    const int sh_tps = g.sh_count ? (g.sh_T + 2 * HALF - 1) / (2 * HALF) : 1;
+    const int mtiles = nrouted + g.sh_count * sh_tps;
+    const int total0 = MODE == 3 ? mtiles * nt0 : 0;
+    auto pos_of = [&](int item, int &mt, int &nt) {  // returns 1 for a down item
+        const int p1 = MODE == 1 || (MODE == 3 && item >= total0);
+        const int local = MODE == 3 && p1 ? item - total0 : item;
+        const int ntl = p1 ? nt1 : nt0;
+        mt = local / ntl;
+        nt = local - mt * ntl;
+        return p1;
+    };
+
     if (warp == 0) {
         // -------------------------------- item hand-off (leader) + TMA producer (both)
         if (lane == 0) {
-            const int nrouted = *ntiles2;
-            const int sh_tps = g.sh_count ? (g.sh_T + 2 * HALF - 1) / (2 * HALF) : 1;
-            const int total = (nrouted + g.sh_count * sh_tps) * n_tiles;
+            const int total = MODE == 3 ? total0 + mtiles * nt1 : mtiles * (MODE == 0 ? nt0 : nt1);
             int stage = 0, rs = 0, cursor = 0;
             uint32_t phase = 0, rphase = 0;
             bool ok = true;
@@ -238,7 +272,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
             for (;;) {
                 int item;
                 if (rank == 0) {
-                    item = claim_item(g.reverse, g.counter, total, n_tiles, tiles2, cursor, nrouted, g.sh_e0, sh_tps);
+                    if (MODE != 3) {
+                        item = claim_item(g.reverse, g.counter, total, MODE == 0 ? nt0 : nt1, tiles2, cursor, nrouted,
+                                          g.sh_e0, sh_tps);
+                    } else {  // the queue; descending within each phase in the reversed order
+                        item = atomicAdd(g.counter, 1);
+                        if (item >= total) item = -1;
+                        else if (g.reverse == 1)
+                            item = item < total0 ? total0 - 1 - item : total0 + (total - 1 - item);
+                    }
                     if (!wait2(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
                     S->ring[rs] = item;
                     st_remote(peer_addr(&S->ring[rs], 1), item);
@@ -251,20 +293,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                 }
                 if (++rs == RING2) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
-                const int mt = item / n_tiles, nt = item - mt * n_tiles;
-                const TileRef tr = tile_ref(tiles2, nrouted, mt, 2 * HALF, MODE, g.sh_T, g.sh_rows0, g.sh_e0);
+                int mt, nt;
+                const bool p1 = pos_of(item, mt, nt);
+                const TileRef tr = tile_ref(tiles2, nrouted, mt, 2 * HALF, p1 ? 1 : 0, g.sh_T, g.sh_rows0, g.sh_e0);
                 const int expert = tr.e;
                 const int arow0 = tr.arow0 + (int)rank * HALF;  // this CTA's half of the pair tile
                 const int rows = min(HALF, max(0, tr.rows - (int)rank * HALF));
                 const int ab = a_box(rows);
-                const CUtensorMap *amap = (MODE == 0 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
+                const CUtensorMap *amap = MODE == 3 && p1 ? &lm.h.m[ab] : (!p1 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
                 const uint32_t a_bytes = rows > 0 ? (uint32_t)(a_box_rows(ab) * BK2 * 2) : 0u;
                 // B rows of this CTA: gate (CTA 0) or up (CTA 1) rows nt*128.. ; down: output columns
-                const int nrow = MODE == 0 ? nt * BNO : nt * BNO + (int)rank * 128;
-                const CUtensorMap *bmap = (MODE == 0 && rank == 1) ? (tr.s >= 0 ? &sm.b1 : &tmB1)
-                                                                   : (tr.s >= 0 ? &sm.b0 : &tmB0);
-                const bool b_in = nrow < g.N;  // a half entirely past N loads nothing (its columns are masked)
+                const int nrow = !p1 ? nt * BNO0 : nt * BNO1 + (int)rank * 128;
+                const CUtensorMap *bmap = !p1 ? (rank == 1 ? (tr.s >= 0 ? &sm.b1 : &tmB1) : (tr.s >= 0 ? &sm.b0 : &tmB0))
+                                        : MODE == 3 ? (tr.s >= 0 ? &lm.wd_sh : &lm.wd)
+                                                    : (tr.s >= 0 ? &sm.b0 : &tmB0);
+                const bool b_in = nrow < (p1 ? NP1 : g.N);  // a half entirely past N loads nothing (masked columns)
                 const uint32_t b_bytes = b_in ? (uint32_t)B2_BYTES : 0u;
+                const int num_kb = p1 ? kb1 : kb0;
+                if (MODE == 3 && p1) {
+                    // the h rows of pair tile mt: wait until every gate/up item of mt published
+                    // them (4 epilogue warps in each of the 2 CTAs), then order those
+                    // generic-proxy writes before this CTA's TMA reads
+                    if (!wait_count_at_least2(g.ready + mt, 8 * nt0, g.wait_ns)) { ok = false; break; }
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                }
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!wait2(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
                     const uint32_t fb = peer_addr(&S->full[stage], 0);
@@ -276,10 +328,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                     if (b_in) {
                         if (tr.s < 0)
                             tma_load_3d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, nrow, expert);
-                        else if (MODE == 0)  // shared slice s: rows s*I + nrow.. of the shared gate / up
+                        else if (!p1)  // shared slice s: rows s*I + nrow.. of the shared gate / up
                             tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, tr.s * g.N + nrow);
                         else  // shared down: columns s*I + kb*BK2..
-                            tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, tr.s * g.K + kb * BK2, nrow);
+                            tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, tr.s * KP1 + kb * BK2, nrow);
                     }
                     if (++stage == ST2) { stage = 0; phase ^= 1; }
                     if (held && kb + 1 == min(ST2, num_kb)) {  // first item: stage j holds K block j
@@ -308,6 +360,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                 mbar_arrive(&S->ite[rs]);
                 if (++rs == RING2) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
+                int mt_, nt_;
+                const int num_kb = pos_of(item, mt_, nt_) ? kb1 : kb0;
                 if (!wait2(&S->acce[acc], aphase ^ 1, g.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + static_cast<uint32_t>(acc * BN2);
@@ -337,7 +391,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
         const int row = q * 32 + lane;
         int rs = 0, acc = 0;
         uint32_t rphase = 0, aphase = 0;
-        const int nrouted = *ntiles2;
         // y row of sorted row r: the row map's for the routed rows, r itself for the shared expert's
         auto flat_of = [&](int r) { return (g.sh_count == 0 || r < g.sh_rows0) ? g.row_map[r] : r; };
         for (;;) {
@@ -350,22 +403,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
             }
             if (++rs == RING2) { rs = 0; rphase ^= 1; }
             if (item < 0) break;
-            const int mt = item / n_tiles, nt = item - mt * n_tiles;
-            const TileRef tr = tile_ref(tiles2, nrouted, mt, 2 * HALF, MODE, g.sh_T, g.sh_rows0, g.sh_e0);
+            int mt, nt;
+            const bool p1 = pos_of(item, mt, nt);
+            const TileRef tr = tile_ref(tiles2, nrouted, mt, 2 * HALF, p1 ? 1 : 0, g.sh_T, g.sh_rows0, g.sh_e0);
             const int row0 = tr.row0 + (int)rank * HALF;
             const int rows = min(HALF, max(0, tr.rows - (int)rank * HALF));
             const bool row_ok = row < rows;
             if (!wait2(&S->accf[acc], aphase, g.wait_ns)) { record2(g.status, MOE_ERR_TIMEOUT); break; }
             tc_fence_after();
             const uint32_t tb = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN2);
-            if (MODE == 0) {
+            if (!p1) {
                 __nv_bfloat16 *orow = g.out + (size_t)(row0 + row) * g.N;
 #pragma unroll 1
-                for (int c = 0; c < BNO / 32; ++c) {
+                for (int c = 0; c < BNO0 / 32; ++c) {
                     uint32_t gr[32], ur[32];
                     tmem_ld32_sync(tb + c * 32, gr);
-                    tmem_ld32_sync(tb + BNO + c * 32, ur);
-                    const int col = nt * BNO + c * 32;
+                    tmem_ld32_sync(tb + BNO0 + c * 32, ur);
+                    const int col = nt * BNO0 + c * 32;
                     if (row_ok && col < g.N) {
                         uint32_t pk[16];
 #pragma unroll
@@ -381,14 +435,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                     }
                 }
             } else {
+                __nv_bfloat16 *y = MODE == 3 ? g.out2 : g.out;
                 const int flat = row_ok ? flat_of(row0 + row) : 0;
-                __nv_bfloat16 *orow = g.out + (size_t)flat * g.N;
+                __nv_bfloat16 *orow = y + (size_t)flat * NP1;
 #pragma unroll 1
-                for (int c = 0; c < BNO / 32; ++c) {
+                for (int c = 0; c < BNO1 / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld32_sync(tb + c * 32, r);
-                    const int col = nt * BNO + c * 32;
-                    if (row_ok && col < g.N) {
+                    const int col = nt * BNO1 + c * 32;
+                    if (row_ok && col < NP1) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
@@ -407,9 +462,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                 else arrive_remote(peer_addr(&S->acce[acc], 0));
             }
             if (++acc == 2) { acc = 0; aphase ^= 1; }
-            if (MODE == 1 && g.comb_cnt)  // the accumulator is already released
-                combine_arrive(g.out, g.comb_gate, g.comb_out, g.comb_cnt, g.comb_k, g.comb_target, g.N, n_tiles,
-                               nt, row_ok, row_ok ? flat_of(row0 + row) : 0, lane, g.sh_count, g.sh_T, g.sh_rows0);
+            if (MODE == 3 && !p1) {
+                // publish this warp's h rows of pair tile mt to the down items (release at
+                // GPU scope after the proxy fence, counted once per warp)
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();
+                    atomicAdd(g.ready + mt, 1);
+                }
+            }
+            if (p1 && g.comb_cnt)  // the accumulator is already released
+                combine_arrive(MODE == 3 ? g.out2 : g.out, g.comb_gate, g.comb_out, g.comb_cnt, g.comb_k,
+                               g.comb_target, NP1, nt1, nt, row_ok, row_ok ? flat_of(row0 + row) : 0, lane,
+                               g.sh_count, g.sh_T, g.sh_rows0);
         }
     }
 
@@ -436,15 +502,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
 bool smem2_ready(int mode)
 {
     static std::mutex mu;
-    static uint64_t done[2] = {0, 0};  // per device
+    static uint64_t done[4] = {0, 0, 0, 0};  // per device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::lock_guard<std::mutex> lk(mu);
     if (done[mode] >> dev & 1ull) return true;
-    cudaError_t e = mode == 0 ? cudaFuncSetAttribute(grouped_gemm_2cta_kernel<0>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2)
-                              : cudaFuncSetAttribute(grouped_gemm_2cta_kernel<1>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2);
+    const int a = (int)SMEM2;
+    cudaError_t e = mode == 0   ? cudaFuncSetAttribute(grouped_gemm_2cta_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                  : mode == 1 ? cudaFuncSetAttribute(grouped_gemm_2cta_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
+                              : cudaFuncSetAttribute(grouped_gemm_2cta_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, a);
     if (e != cudaSuccess) return false;
     done[mode] |= 1ull << dev;
     return true;
@@ -456,18 +522,24 @@ cudaError_t launch_grouped_gemm_2cta(const GemmArgs &g, const AMaps &tmA, const 
                                      const CUtensorMap &tmB1, const int32_t *tiles2, const int32_t *ntiles2,
                                      cudaStream_t st, const SharedMaps *sm, const LayerMaps *lm)
 {
-    if (lm) return cudaErrorInvalidValue;  // the fused layer launch takes 128-row tiles
     int grid = (g.ctas > 0 ? g.ctas : num_sms()) / 2 * 2;
     if (grid < 2) grid = 2;
+    if ((g.mode != 0 && g.mode != 1 && g.mode != 3) || g.reverse > 1) return cudaErrorInvalidValue;
     if (!smem2_ready(g.mode)) return cudaErrorInvalidValue;
     if (g.sh_count && !sm) return cudaErrorInvalidValue;
+    if (g.mode == 3 && (!lm || !g.ready)) return cudaErrorInvalidValue;
     static const SharedMaps none{};
+    static const LayerMaps nolm{};
     const SharedMaps &s = sm ? *sm : none;
+    const LayerMaps &l = lm ? *lm : nolm;
     if (g.mode == 0)
         return launch_pdl(grouped_gemm_2cta_kernel<0>, dim3(grid), dim3(THREADS2), SMEM2, st, tmA, tmB0, tmB1, g,
-                          tiles2, ntiles2, s);
-    return launch_pdl(grouped_gemm_2cta_kernel<1>, dim3(grid), dim3(THREADS2), SMEM2, st, tmA, tmB0, tmB1, g, tiles2,
-                      ntiles2, s);
+                          tiles2, ntiles2, s, l);
+    if (g.mode == 1)
+        return launch_pdl(grouped_gemm_2cta_kernel<1>, dim3(grid), dim3(THREADS2), SMEM2, st, tmA, tmB0, tmB1, g,
+                          tiles2, ntiles2, s, l);
+    return launch_pdl(grouped_gemm_2cta_kernel<3>, dim3(grid), dim3(THREADS2), SMEM2, st, tmA, tmB0, tmB1, g, tiles2,
+                      ntiles2, s, l);
 }
 
 }  // namespace moe

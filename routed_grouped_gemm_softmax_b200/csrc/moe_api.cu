@@ -47,11 +47,16 @@ struct StageMarks {
         on = g_stage_on;
         for (int i = 0; i < MOE_STAGE_EVENTS; ++i) ev[i] = g_stage_ev[i];
     }
-    // External records become event-record nodes when the stream is being captured
-    // into a CUDA graph, so a replayed graph still timestamps every stage.
+    // While the stream is being captured into a CUDA graph, external records become
+    // event-record nodes, so a replayed graph still timestamps every stage; otherwise
+    // the events are recorded directly (the external flag is for captures only).
     cudaError_t mark(int i, cudaStream_t st) const
     {
-        return on && ev[i] ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal) : cudaSuccess;
+        if (!on || !ev[i]) return cudaSuccess;
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return cudaErrorInvalidValue;
+        return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev[i], st, cudaEventRecordExternal)
+                                                   : cudaEventRecord(ev[i], st);
     }
 };
 
@@ -214,7 +219,7 @@ int bf16_plan(const moe_dims_t &d)
     const int fc = g_fused_comb.load();
     const bool fused = fc == 1 || (fc == 0 && d.T <= moe::kFusedCombineMaxT);
     const int lg = g_layer_gemm.load();
-    const bool layer = !pairs && (lg == 1 || (lg == 0 && kLayerGemmAuto));
+    const bool layer = lg == 1 || (lg == 0 && kLayerGemmAuto);
     return (small ? MOE_PLAN_SMALL_ROUTER : 0) | (pairs ? MOE_PLAN_PAIR_TILES : 0) |
            (fused ? MOE_PLAN_FUSED_COMBINE : 0) | (layer ? MOE_PLAN_LAYER_GEMM : 0);
 }
@@ -515,7 +520,9 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
         lm.h = tm_h;
         lm.wd = tm_wd;
         lm.wd_sh = sm2.b0;
-        e = moe::launch_grouped_gemm(gl, tm_xs, tm_wg, tm_wu, st, &sm1, &lm);
+        e = pairs ? moe::launch_grouped_gemm_2cta(gl, tm_xs, tm_wg, tm_wu, at<int32_t>(ws, L.tiles2),
+                                                  at<int32_t>(ws, L.ntiles2), st, &sm1, &lm)
+                  : moe::launch_grouped_gemm(gl, tm_xs, tm_wg, tm_wu, st, &sm1, &lm);
         if (e == cudaSuccess) e = marks.mark(3, st);
         if (e == cudaSuccess) e = marks.mark(4, st);
     }

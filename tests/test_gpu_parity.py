@@ -325,3 +325,48 @@ def test_full_size(name):
     ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"], tokens=tok)
     max_abs, rel = compare_out(out[torch.as_tensor(tok, device="cuda").long()], ref, name)
     print(f"full size {name}: {tok.size} tokens, max_abs={max_abs:.3e} rel_l2={rel:.3e}")
+
+
+LAYER_CASES = {
+    "ragged": (SMALL["ragged"], "auto"),
+    "ragged_bias": (SMALL["ragged_bias"], "auto"),
+    "small_fused_combine": (CONFIGS["tiny"].replace(name="lay48", T=48, H=512, E=16, top_k=4, I=384, seed=26), "auto"),
+    "deep_pairs": (PAIR_CASES["deep"], "always"),
+    "decode": (CONFIGS["decode"], "auto"),
+}
+
+
+@pytest.mark.parametrize("name", list(LAYER_CASES))
+def test_layer_gemm_matches_two_launches(name):
+    # Both expert GEMMs in one persistent launch (down items wait on per-m-tile
+    # readiness counts of the gate/up epilogues) give the two-launch result bit for
+    # bit, over grid sizes (one CTA included: it runs every gate/up item first) and
+    # both queue orders, and the oracle's within tolerance.
+    cfg, pair = LAYER_CASES[name]
+    g, c = device_inputs(cfg)
+    k = cfg.top_k
+    outs = []
+    try:
+        api.set_pair_mma(pair)
+        for lg, ctas, rev in [("never", 0, False), ("always", 0, False), ("always", 2 if pair == "always" else 1, False),
+                              ("always", 6, True), ("always", 148, False)]:
+            api.set_layer_gemm(lg)
+            api.set_gemm_ctas(ctas)
+            api.set_claim_order(rev)
+            ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, "cuda")
+            outs.append(api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k,
+                                        ws=ws).clone())
+            assert api.moe_get_device_status(ws) == api.MOE_OK
+            plan = api.forward_plan(cfg.T, cfg.H, cfg.I, cfg.E, k)
+            assert bool(plan & api.PLAN_LAYER_GEMM) == (lg == "always")
+    finally:
+        api.set_pair_mma("auto")
+        api.set_layer_gemm("auto")
+        api.set_gemm_ctas(0)
+        api.set_claim_order(False)
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], k)
+    tok = sample_tokens(cfg.T, 64, seed=cfg.seed)
+    ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"], tokens=tok)
+    compare_out(outs[1][torch.as_tensor(tok, device="cuda").long()], ref, f"{name} layer GEMM")
