@@ -82,11 +82,12 @@ def kernels_per_forward(cfg, plan=None) -> int:
         route = 2          # logits, top-k + grouping
     else:
         route = 2 + 3      # logits, top-k; count, scan, scatter
-    combine = 0 if cfg.T <= 64 else 1   # small batches combine inside the down GEMM
+    # small batches combine inside the down GEMM (bf16 up to 32 tokens, fp8 up to 64)
+    combine = 0 if cfg.T <= (64 if cfg.dtype == "fp8" else 32) else 1
     rows = 2 if cfg.dtype in ("fp8", "mx") else 1   # fp8 / MX: quantise per token, then gather; bf16: gather
     if cfg.dtype == "mx":
         combine = 1   # the MX down GEMM has no fused combine
-    gemms = 2
+    gemms = 1 if cfg.dtype == "bf16" else 2   # bf16: both expert GEMMs in one launch (the layer kernel)
     if plan is not None and plan >= 0:
         combine = 0 if plan & 4 else 1       # MOE_PLAN_FUSED_COMBINE
         gemms = 1 if plan & 8 else 2         # MOE_PLAN_LAYER_GEMM
@@ -125,6 +126,10 @@ def parse():
                    help="both bf16 expert GEMMs in one persistent launch: automatic choice or forced")
     p.add_argument("--fused-combine", default="auto", choices=["auto", "always", "never"],
                    help="the bf16 combine inside the down GEMM's epilogue: automatic choice or forced")
+    p.add_argument("--tile-sweep", action="store_true",
+                   help="instead of the bench line: time the kernel variants (tile shapes, one or two GEMM "
+                        "launches, combine placement, fp8 operand order) over M buckets of average rows per "
+                        "expert, one JSON line per bucket (the data behind the library's tile table)")
     p.add_argument("--shape", default="",
                    help="override config fields, e.g. T=1024,E=64 (reduced cases for profiler captures)")
     return p.parse_args()
@@ -797,8 +802,86 @@ def run_and_release(args, cfg, world, rank, local):
     return line
 
 
+def tile_sweep(args):
+    """Times the kernel variants the tile table chooses between, per M bucket r (average
+    rows per expert) of H=2048, I=1024, E=64, top-8 with T = r*E/k: CUDA events around
+    the two GEMM stages and the whole step, L2 flushed before every step, median over
+    --steps steps.  bf16: 128-row or pair tiles, one or two GEMM launches, combine
+    inside the down GEMM or not; fp8: plain or swapped gate/up operands."""
+    from routed_grouped_gemm_softmax_b200 import api
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    steps = max(args.steps, 5) if args.steps != 400 else 30
+
+    def time_stages(forward):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+        for s_ in ev:
+            for e in s_:
+                e.record()
+        for _ in range(max(args.warmup, 3)):
+            flush.fill_(1)
+            forward()
+        torch.cuda.synchronize()
+        try:
+            for i in range(steps):
+                flush.fill_(1)
+                api.set_stage_events(ev[i])
+                forward()
+        finally:
+            api.set_stage_events(None)
+        torch.cuda.synchronize()
+        med = lambda a, b: round(statistics.median(ev[i][a].elapsed_time(ev[i][b]) for i in range(steps)) * 1e3, 1)
+        return {"gemm_gate_up_us": med(2, 3), "gemm_down_us": med(3, 4), "step_us": med(0, 5)}
+
+    H, I, E, k = 2048, 1024, 64, 8
+    variants = {"tiles128": ("never", "never", "never"), "tiles128_layer": ("never", "always", "never"),
+                "tiles128_layer_combine_in_down": ("never", "always", "always"), "pairs": ("always", "never", "never"),
+                "pairs_layer": ("always", "always", "never"), "table": ("auto", "auto", "auto")}
+    for r in [1, 2, 4, 8, 16, 32, 64, 96, 128, 192, 256, 384, 512, 768, 1024, 2048, 4096]:
+        T = max(1, r * E // k)
+        cfg = CONFIGS["prefill"].replace(name=f"bucket{r}", T=T, H=H, I=I, E=E, top_k=k, seed=100 + r)
+        inp = make_inputs(cfg, device=dev)
+        ws = api.workspace(T, H, I, E, k, dev)
+        o = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        f = lambda: api.moe_forward(inp.x, inp.router_w, None, inp.w_gate, inp.w_up, inp.w_down, k, out=o, ws=ws)
+        row = {"sweep": "bf16", "rows_per_expert": r, "T": T, "H": H, "I": I, "E": E, "top_k": k}
+        for name, (pm, lg, fc) in variants.items():
+            api.set_pair_mma(pm)
+            api.set_layer_gemm(lg)
+            api.set_fused_combine(fc)
+            row[name] = time_stages(f)
+        api.set_pair_mma("auto")
+        api.set_layer_gemm("auto")
+        api.set_fused_combine("auto")
+        row["table_plan"] = api.forward_plan(T, H, I, E, k)
+        print(json.dumps(row), flush=True)
+        del inp, ws, o, f
+        torch.cuda.empty_cache()
+    for r in [1, 4, 16, 32, 48, 64, 96, 128, 256, 512, 1024]:
+        T = max(1, r * E // k)
+        cfg = CONFIGS["fp8"].replace(name=f"bucket8_{r}", T=T, H=H, I=I, E=E, top_k=k, seed=200 + r)
+        inp = make_inputs(cfg, device=dev, weights=False)
+        w = make_fp8_weights(cfg, device=dev)
+        wq = (w["w_gate_q"], w["w_gate_s"], w["w_up_q"], w["w_up_s"], w["w_down_q"], w["w_down_s"])
+        ws = api.workspace(T, H, I, E, k, dev, api.DTYPE_FP8)
+        o = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        f = lambda: api.moe_forward_fp8(inp.x, inp.router_w, None, *wq, k, out=o, ws=ws)
+        row = {"sweep": "fp8", "rows_per_expert": r, "T": T, "H": H, "I": I, "E": E, "top_k": k}
+        for mode in ("never", "always", "auto"):
+            api.set_fp8_swap_ab(mode)
+            row["swap_" + mode] = time_stages(f)
+        api.set_fp8_swap_ab("auto")
+        print(json.dumps(row), flush=True)
+        del inp, w, wq, ws, o, f
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
+    if args.tile_sweep:
+        tile_sweep(args)
+        return
     if args.impl == "reference":
         # rank 0 alone times the oracle on the host cores; the other ranks have no work
         # and open no process group

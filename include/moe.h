@@ -269,7 +269,7 @@ void moe_set_pair_mma(int32_t mode);
 void moe_set_fp8_swap_ab(int32_t mode);
 
 /* Where the bf16 forwards sum the k per-assignment rows of a token: 0 = automatic
- * (inside the down GEMM's epilogue for batches of at most 64 tokens, else a separate
+ * (inside the down GEMM's epilogue for batches of at most 32 tokens, else a separate
  * combine kernel), 1 = always inside the down GEMM, 2 = always the separate kernel.
  * The sum's order is fixed by j either way, so the result is bitwise the same.
  * Process-wide; for tests and benchmarks. */

@@ -18,9 +18,6 @@
 
 namespace {
 
-// The fused gate/up + down launch is the default for one-CTA tiles (the layer kernel).
-constexpr bool kLayerGemmAuto = true;
-
 std::atomic<int> g_gemm_ctas{0};
 std::atomic<int> g_claim_reverse{0};
 std::atomic<unsigned long long *> g_trace{nullptr};
@@ -211,15 +208,14 @@ moe::RouterScratch router_scratch(void *ws, const moe::WsLayout &L, const moe_di
 // (MOE_PLAN_* bits).
 int bf16_plan(const moe_dims_t &d)
 {
-    const long A = (long)d.T * d.top_k;
+    const moe::TileChoice tc = moe::tile_choice((long long)d.T * d.top_k, d.E);
     const bool small = moe::small_route_permute_ok(d);
     const int pair_mode = g_pair_mode.load();
-    const bool pairs = pair_mode != 2 && g_claim_reverse.load() <= 1 && !small &&
-                       (pair_mode == 1 || A >= 512L * d.E);
+    const bool pairs = pair_mode != 2 && g_claim_reverse.load() <= 1 && !small && (pair_mode == 1 || tc.pair_tiles);
     const int fc = g_fused_comb.load();
     const bool fused = fc == 1 || (fc == 0 && d.T <= moe::kFusedCombineMaxT);
     const int lg = g_layer_gemm.load();
-    const bool layer = lg == 1 || (lg == 0 && kLayerGemmAuto);
+    const bool layer = lg == 1 || (lg == 0 && tc.layer_gemm);
     return (small ? MOE_PLAN_SMALL_ROUTER : 0) | (pairs ? MOE_PLAN_PAIR_TILES : 0) |
            (fused ? MOE_PLAN_FUSED_COMBINE : 0) | (layer ? MOE_PLAN_LAYER_GEMM : 0);
 }
@@ -606,7 +602,7 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
         return MOE_ERR_CUDA;
 
     const StageMarks marks;
-    const bool fused = d->T <= moe::kFusedCombineMaxT;  // combine inside the down GEMM
+    const bool fused = d->T <= moe::kFusedCombineMaxTFp8;  // combine inside the down GEMM
     cudaError_t e = marks.mark(0, st);
     if (e == cudaSuccess && !moe::small_route_permute_ok(*d))  // else the router's kernels clear them
         e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);          // header + combine counts
@@ -630,7 +626,7 @@ moe_status_t moe_forward_fp8(const moe_dims_t *d, const void *x, const void *rou
         g1.trace = trace1;
         // operands swapped when the groups average at most 64 rows per expert
         const int sw = g_fp8_swap.load();
-        const bool swap = sw == 1 || (sw == 0 && (long)A <= 64L * d->E);
+        const bool swap = sw == 1 || (sw == 0 && moe::tile_choice(A, d->E).fp8_swap_ab);
         e = swap ? moe::launch_grouped_gemm_fp8_swapab(g1, tm_xs, tm_wg, tm_wu, st)
                  : moe::launch_grouped_gemm_fp8(g1, tm_xs, tm_wg, tm_wu, st);
     }
@@ -737,7 +733,7 @@ int32_t moe_forward_plan(const moe_dims_t *d, int dtype)
 {
     if (moe_workspace_size(d, dtype) == 0) return -1;
     if (dtype != MOE_DTYPE_BF16) {  // the fp8 and MX forwards: small router, fused combine for fp8
-        const bool fused = dtype == MOE_DTYPE_FP8 && d->T <= moe::kFusedCombineMaxT;
+        const bool fused = dtype == MOE_DTYPE_FP8 && d->T <= moe::kFusedCombineMaxTFp8;
         return (moe::small_route_permute_ok(*d) ? MOE_PLAN_SMALL_ROUTER : 0) | (fused ? MOE_PLAN_FUSED_COMBINE : 0);
     }
     return bf16_plan(*d);

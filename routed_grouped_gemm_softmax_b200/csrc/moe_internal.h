@@ -209,6 +209,11 @@ struct GemmArgs {
     int K2, N2;
     __nv_bfloat16 *out2;
     int32_t *ready;
+    // Gate/up items of routed tiles with a_rows non-null: the A rows are read straight
+    // from x (SharedMaps::xg, one-row boxes) by tile::gather4 loads, row r of a tile
+    // being token a_rows[row0 + r] / a_div (no expert-ordered copy of x is made).
+    const int32_t *a_rows;
+    int a_div;
 };
 
 // Tensor maps of the down half of the fused layer GEMM (mode 3): h as its A operand
@@ -224,6 +229,7 @@ struct LayerMaps {
 struct SharedMaps {
     AMaps x;
     CUtensorMap b0, b1;
+    CUtensorMap xg;  // x with one-row boxes of 64 columns (128-byte swizzle), for tile::gather4 A loads
 };
 
 // The m-tile `mt` of a grouped GEMM: the tile list's entry for mt < nrouted, else a
@@ -347,8 +353,43 @@ cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, i
 // plus, with sh_count > 0, the shared expert's rows y[sh_rows0 + s * T + t] at gate 1.
 cudaError_t launch_combine(const __nv_bfloat16 *y, const float *gate, int T, int H, int top_k,
                            __nv_bfloat16 *out, cudaStream_t st, int sh_count = 0, int sh_rows0 = 0);
-// Batches up to this many tokens combine inside the down GEMM's epilogue.
-constexpr int kFusedCombineMaxT = 64;
+// ----------------------------------------------------------- tile table
+// The kernel variants by M bucket: the batch's average rows per expert r = T*k/E (the
+// vLLM fused-MoE page keys its tuned configs by M the same way, section 03).  Measured
+// on B200 with CUDA events (H=2048, I=1024, E=64, top-8, r = 1 .. 4096, uniform
+// routing; and the Skewed workload, r = 768 with a Zipf-skewed router, at 1x and 2x
+// its tokens):
+//  - pair-of-CTA 256-row tiles lose 3-8% to 128-row tiles below r = 512 and win from
+//    r = 2048 (uniform); on the skewed workload they win at r = 768 (1.68 against
+//    1.72 ms) and r = 1536 (5.6%), its deep hot-expert groups filling the pairs;
+//  - one persistent launch for both GEMMs (the layer kernel) wins 6-14% below r = 512
+//    and on the skewed workload, and is within 1-3% elsewhere;
+//  - the fp8 gate/up GEMM with the operands swapped wins up to r = 64 (up to 40%) and
+//    loses from r = 96 (up to 2x at r = 1024).
+// Each entry covers the buckets up to max_rows.
+struct TileChoice {
+    int max_rows;     // the bucket: average rows per expert <= max_rows
+    bool pair_tiles;  // bf16: 256-row tiles on CTA pairs (tcgen05 cta_group::2)
+    bool layer_gemm;  // bf16: the gate/up and down GEMMs in one launch
+    bool fp8_swap_ab; // fp8: gate/up GEMM with the weight rows on the MMA's M side
+};
+constexpr TileChoice kTileTable[] = {
+    {64, false, true, true},
+    {511, false, true, false},
+    {0x7fffffff, true, true, false},
+};
+inline TileChoice tile_choice(long long A, int E)
+{
+    const long long r = E > 0 ? A / E : A;  // average rows per expert, rounded down
+    for (const TileChoice &t : kTileTable)
+        if (r <= t.max_rows) return t;
+    return kTileTable[sizeof(kTileTable) / sizeof(kTileTable[0]) - 1];
+}
+// Batches up to this many tokens combine inside the down GEMM's epilogue (the sweep:
+// 1% faster at T <= 16, even at 32, 4% slower at 64 and 20-30% slower from 256).
+constexpr int kFusedCombineMaxT = 32;
+// The fp8 down GEMM's fused combine (two epilogue warps per row) keeps its own limit.
+constexpr int kFusedCombineMaxTFp8 = 64;
 
 int num_sms();
 

@@ -137,3 +137,31 @@ int main(void) {
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
     assert int(r.stdout.split()[0]) == api.moe_workspace_size(16, 2048, 512, 256, 8)
+
+
+def test_forward_plan_follows_the_tile_table(L):
+    # The plan query is host-only: the kernels a forward would launch under the
+    # current settings, by the M bucket (average rows per expert) of the batch.
+    plan = lambda T, H, I, E, k, dt=api.DTYPE_BF16: api.forward_plan(T, H, I, E, k, dt)
+    # decode-sized: the two-kernel router, 128-row tiles, one GEMM launch, combine inside
+    assert plan(16, 2048, 512, 256, 8) == api.PLAN_SMALL_ROUTER | api.PLAN_FUSED_COMBINE | api.PLAN_LAYER_GEMM
+    # 128 rows per expert: 128-row tiles, one GEMM launch, the combine kernel
+    assert plan(4096, 2048, 512, 256, 8) == api.PLAN_LAYER_GEMM
+    # 511 rows per expert still 128-row tiles; 512 and up pair tiles
+    assert plan(511 * 64 // 8 + 7, 2048, 1024, 64, 8) & api.PLAN_PAIR_TILES == 0
+    assert plan(512 * 64 // 8, 2048, 1024, 64, 8) & api.PLAN_PAIR_TILES
+    assert plan(8192, 4096, 1408, 64, 6) == api.PLAN_PAIR_TILES | api.PLAN_LAYER_GEMM   # the Skewed workload
+    # the combine inside the down GEMM up to 32 tokens
+    assert plan(32, 512, 512, 64, 8) & api.PLAN_FUSED_COMBINE
+    assert not plan(33, 512, 512, 64, 8) & api.PLAN_FUSED_COMBINE
+    # forced settings
+    try:
+        api.set_pair_mma("never")
+        api.set_layer_gemm("never")
+        assert plan(8192, 4096, 1408, 64, 6) == 0
+    finally:
+        api.set_pair_mma("auto")
+        api.set_layer_gemm("auto")
+    assert plan(64, 100, 512, 8, 2) == -1   # invalid dims
+    assert plan(1024, 7168, 2048, 256, 8, api.DTYPE_FP8) == 0
+    assert plan(16, 7168, 2048, 256, 8, api.DTYPE_FP8) == api.PLAN_SMALL_ROUTER | api.PLAN_FUSED_COMBINE

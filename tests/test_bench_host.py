@@ -15,16 +15,20 @@ PEAKS = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1200
 
 def test_kernels_per_forward_match_the_launch_lists():
     # one forward's kernels, as listed by ncu on the GPU:
-    # decode: logits, top-k + grouping, gather, gate/up GEMM, down GEMM (combine inside)
-    assert bench.kernels_per_forward(CONFIGS["decode"]) == 5
+    # decode: logits, top-k + grouping, gather, the layer GEMM (both expert GEMMs and
+    # the combine in one launch)
+    assert bench.kernels_per_forward(CONFIGS["decode"]) == 4
     # prefill/skewed: prep, tensor-core logits, certify, count, scan, scatter, gather,
-    # two GEMMs, combine
-    assert bench.kernels_per_forward(CONFIGS["prefill"]) == 10
-    assert bench.kernels_per_forward(CONFIGS["skewed"]) == 10
-    # fp8: as prefill, with the per-token quantiser before the (fp8) gather
+    # the layer GEMM, combine
+    assert bench.kernels_per_forward(CONFIGS["prefill"]) == 9
+    assert bench.kernels_per_forward(CONFIGS["skewed"]) == 9
+    # fp8: the large-batch router and grouping, quantiser, gather, two GEMMs, combine
     assert bench.kernels_per_forward(CONFIGS["fp8"]) == 11
-    # tiny (T = 64): the large-batch router, the combine inside the down GEMM
+    # tiny (T = 64): the large-batch router, the layer GEMM, the combine kernel
     assert bench.kernels_per_forward(CONFIGS["tiny"]) == 9
+    # with the library's plan bits: two GEMM launches and the combine inside the second
+    assert bench.kernels_per_forward(CONFIGS["decode"], plan=1 | 4) == 2 + 1 + 2
+    assert bench.kernels_per_forward(CONFIGS["prefill"], plan=2 | 8) == 6 + 1 + 1 + 1
 
 
 def test_stage_work_bf16_by_hand():
@@ -201,4 +205,4 @@ def test_layer_work_mx_is_about_half_of_fp8():
 def test_kernels_per_forward_variants():
     assert bench.kernels_per_forward(bench.WORKLOADS["mx"]) == 11   # as fp8 (T > 64: the standalone combine)
     assert bench.kernels_per_forward(bench.WORKLOADS["mx"].replace(T=16)) == 2 + 2 + 2 + 1  # no fused combine
-    assert bench.kernels_per_forward(bench.WORKLOADS["prefill_shared"]) == 10   # the shared expert adds none
+    assert bench.kernels_per_forward(bench.WORKLOADS["prefill_shared"]) == 9   # the shared expert adds none

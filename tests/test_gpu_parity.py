@@ -120,6 +120,7 @@ def test_schedule_independence(T):
     cfg = CONFIGS["tiny"].replace(name="sched", T=T, H=512, E=16, top_k=4, I=384, seed=24)
     g, _ = device_inputs(cfg)
     outs = []
+    api.set_fused_combine("always" if T <= 64 else "auto")
     try:
         for ctas, rev in [(0, False), (1, False), (7, True), (148, False), (0, True), (3, True),
                           (0, "static_items"), (0, "static_experts"), (5, "static_experts")]:
@@ -130,6 +131,7 @@ def test_schedule_independence(T):
     finally:
         api.set_gemm_ctas(0)
         api.set_claim_order(False)
+        api.set_fused_combine("auto")
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
     # and the common result against the oracle
@@ -370,3 +372,36 @@ def test_layer_gemm_matches_two_launches(name):
     tok = sample_tokens(cfg.T, 64, seed=cfg.seed)
     ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"], tokens=tok)
     compare_out(outs[1][torch.as_tensor(tok, device="cuda").long()], ref, f"{name} layer GEMM")
+
+
+def test_stage_events_outside_and_inside_capture():
+    # The stage marks are recorded on the forward's stream both when the stream is
+    # being captured into a CUDA graph (as graph nodes) and when it is not.
+    cfg = SMALL["ragged"]
+    g, _ = device_inputs(cfg)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(api.STAGES.__len__() + 1)]
+    for e in ev:
+        e.record()
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k, "cuda")
+    try:
+        api.set_stage_events(ev)
+        api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k, ws=ws)
+        torch.cuda.synchronize()
+        direct = [ev[i].elapsed_time(ev[i + 1]) for i in range(len(ev) - 1)]
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(graph, stream=s):
+                api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k,
+                                ws=ws, stream=s)
+    finally:
+        api.set_stage_events(None)
+    torch.cuda.current_stream().wait_stream(s)
+    graph.replay()
+    torch.cuda.synchronize()
+    replayed = [ev[i].elapsed_time(ev[i + 1]) for i in range(len(ev) - 1)]
+    del graph
+    assert all(t >= 0 for t in direct) and sum(direct) > 0
+    assert all(t >= 0 for t in replayed) and sum(replayed) > 0
+    assert api.moe_get_device_status(ws) == api.MOE_OK
