@@ -84,13 +84,17 @@ def kernels_per_forward(cfg, plan=None) -> int:
         route = 2 + 3      # logits, top-k; count, scan, scatter
     # small batches combine inside the down GEMM (bf16 up to 32 tokens, fp8 up to 64)
     combine = 0 if cfg.T <= (64 if cfg.dtype == "fp8" else 32) else 1
-    rows = 2 if cfg.dtype in ("fp8", "mx") else 1   # fp8 / MX: quantise per token, then gather; bf16: gather
+    # fp8 / MX: quantise per token, then gather; bf16: the gather kernel, or (up to 16
+    # rows per expert) the gate/up GEMM gathers x rows itself
+    rows = 2 if cfg.dtype in ("fp8", "mx") else (0 if A <= 16 * cfg.E else 1)
     if cfg.dtype == "mx":
         combine = 1   # the MX down GEMM has no fused combine
     gemms = 1 if cfg.dtype == "bf16" else 2   # bf16: both expert GEMMs in one launch (the layer kernel)
     if plan is not None and plan >= 0:
         combine = 0 if plan & 4 else 1       # MOE_PLAN_FUSED_COMBINE
         gemms = 1 if plan & 8 else 2         # MOE_PLAN_LAYER_GEMM
+        if cfg.dtype == "bf16":
+            rows = 0 if plan & 16 else 1     # MOE_PLAN_DIRECT_A, else the gather kernel
     return route + rows + gemms + combine
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 B200_SMS, FP32_LANES_PER_SM = 148, 128   # CUDA-core fp32 FMA lanes of one B200
@@ -124,6 +128,9 @@ def parse():
                    help="the fp8 gate/up GEMM with swapped MMA operands: automatic choice or forced")
     p.add_argument("--layer-gemm", default="auto", choices=["auto", "always", "never"],
                    help="both bf16 expert GEMMs in one persistent launch: automatic choice or forced")
+    p.add_argument("--direct-a", default="auto", choices=["auto", "always", "never"],
+                   help="bf16 gate/up A rows gathered straight from x by the GEMM, or from a sorted "
+                        "copy of x made by a gather kernel: automatic choice or forced")
     p.add_argument("--fused-combine", default="auto", choices=["auto", "always", "never"],
                    help="the bf16 combine inside the down GEMM's epilogue: automatic choice or forced")
     p.add_argument("--tile-sweep", action="store_true",
@@ -658,6 +665,7 @@ def run_one(args, cfg, world, rank, local):
     api.set_fp8_swap_ab(args.swap_ab)
     api.set_fused_combine(args.fused_combine)
     api.set_layer_gemm(args.layer_gemm)
+    api.set_direct_a(args.direct_a)
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
         step()
@@ -807,7 +815,8 @@ def tile_sweep(args):
     rows per expert) of H=2048, I=1024, E=64, top-8 with T = r*E/k: CUDA events around
     the two GEMM stages and the whole step, L2 flushed before every step, median over
     --steps steps.  bf16: 128-row or pair tiles, one or two GEMM launches, combine
-    inside the down GEMM or not; fp8: plain or swapped gate/up operands."""
+    inside the down GEMM or not, A rows gathered by the GEMM or copied first; fp8:
+    plain or swapped gate/up operands."""
     from routed_grouped_gemm_softmax_b200 import api
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -835,9 +844,11 @@ def tile_sweep(args):
         return {"gemm_gate_up_us": med(2, 3), "gemm_down_us": med(3, 4), "step_us": med(0, 5)}
 
     H, I, E, k = 2048, 1024, 64, 8
-    variants = {"tiles128": ("never", "never", "never"), "tiles128_layer": ("never", "always", "never"),
-                "tiles128_layer_combine_in_down": ("never", "always", "always"), "pairs": ("always", "never", "never"),
-                "pairs_layer": ("always", "always", "never"), "table": ("auto", "auto", "auto")}
+    variants = {"tiles128": ("never", "never", "never", "auto"), "tiles128_layer": ("never", "always", "never", "auto"),
+                "tiles128_layer_combine_in_down": ("never", "always", "always", "auto"),
+                "pairs": ("always", "never", "never", "auto"), "pairs_layer": ("always", "always", "never", "auto"),
+                "table": ("auto", "auto", "auto", "auto"), "table_direct_a": ("auto", "auto", "auto", "always"),
+                "table_sorted_copy": ("auto", "auto", "auto", "never")}
     for r in [1, 2, 4, 8, 16, 32, 64, 96, 128, 192, 256, 384, 512, 768, 1024, 2048, 4096]:
         T = max(1, r * E // k)
         cfg = CONFIGS["prefill"].replace(name=f"bucket{r}", T=T, H=H, I=I, E=E, top_k=k, seed=100 + r)
@@ -846,14 +857,16 @@ def tile_sweep(args):
         o = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         f = lambda: api.moe_forward(inp.x, inp.router_w, None, inp.w_gate, inp.w_up, inp.w_down, k, out=o, ws=ws)
         row = {"sweep": "bf16", "rows_per_expert": r, "T": T, "H": H, "I": I, "E": E, "top_k": k}
-        for name, (pm, lg, fc) in variants.items():
+        for name, (pm, lg, fc, da) in variants.items():
             api.set_pair_mma(pm)
             api.set_layer_gemm(lg)
             api.set_fused_combine(fc)
+            api.set_direct_a(da)
             row[name] = time_stages(f)
         api.set_pair_mma("auto")
         api.set_layer_gemm("auto")
         api.set_fused_combine("auto")
+        api.set_direct_a("auto")
         row["table_plan"] = api.forward_plan(T, H, I, E, k)
         print(json.dumps(row), flush=True)
         del inp, ws, o, f

@@ -208,7 +208,8 @@ moe_status_t moe_quantize_rows_fp8(int32_t R, int32_t K, const void *a, uint8_t 
  *   3 sorted_to_flat [T*k]    4 flat_to_sorted [T*k]    5 tile_list [3*max_tiles]
  *   6 num_tiles [1]           7 logits [T,E] fp32
  *   8 xs: the activations in expert-sorted order [T*k, H] (bf16, or 1-byte codes
- *     for MOE_DTYPE_FP8 / MOE_DTYPE_MX)   9 their scales (fp8: fp32 [T*k, H/128];
+ *     for MOE_DTYPE_FP8 / MOE_DTYPE_MX; a bf16 forward whose plan has
+ *     MOE_PLAN_DIRECT_A does not write it)   9 their scales (fp8: fp32 [T*k, H/128];
  *     MX: e8m0 codes [T*k, H/32])   10 h [T*k, I] (same types)   11 h's scales
  *   12 y [T*k, H] bf16, the per-assignment expert outputs in flat order
  * (0-6 as the outputs of moe_route and moe_permute; 0-1 after moe_route only
@@ -220,13 +221,15 @@ moe_status_t moe_workspace_offsets(const moe_dims_t *d, int dtype, size_t *out, 
 
 /* The kernels a forward with these dims and dtype launches under the current
  * process-wide settings, as bits: the two-kernel router + grouping for small batches,
- * pair-of-CTA GEMM tiles, the combine inside the down GEMM, and both expert GEMMs in
- * one launch.  -1 for invalid dims or dtype.  Host only; enqueues nothing. */
+ * pair-of-CTA GEMM tiles, the combine inside the down GEMM, both expert GEMMs in
+ * one launch, and gate/up A rows gathered straight from x (no sorted copy).  -1 for
+ * invalid dims or dtype.  Host only; enqueues nothing. */
 enum {
     MOE_PLAN_SMALL_ROUTER = 1,
     MOE_PLAN_PAIR_TILES = 2,
     MOE_PLAN_FUSED_COMBINE = 4,
-    MOE_PLAN_LAYER_GEMM = 8
+    MOE_PLAN_LAYER_GEMM = 8,
+    MOE_PLAN_DIRECT_A = 16
 };
 int32_t moe_forward_plan(const moe_dims_t *d, int dtype);
 
@@ -281,6 +284,14 @@ void moe_set_fused_combine(int32_t mode);
  * h rows) or in two launches.  0 = automatic (one launch), 1 = one launch, 2 = two
  * launches.  Results are bitwise the same.  Process-wide; for tests and benchmarks. */
 void moe_set_layer_gemm(int32_t mode);
+
+/* Where the bf16 forwards' gate/up GEMM reads its A rows: straight from x, each
+ * 128-row tile gathering its tokens' rows four at a time (TMA tile::gather4), or
+ * from a copy of x in expert-sorted order made by a gather kernel first (workspace
+ * entry 8).  0 = automatic (straight from x), 1 = straight from x, 2 = the sorted
+ * copy.  The A values are the same bf16 rows either way, so results are bitwise the
+ * same.  Process-wide; for tests and benchmarks. */
+void moe_set_direct_a(int32_t mode);
 
 /* Scheduling trace for benchmarks.  With `trace` a device buffer of 4 * ctas
  * uint64 values (ctas >= the GEMM grid, 148 by default), every later forward

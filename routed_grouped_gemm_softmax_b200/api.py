@@ -25,7 +25,7 @@ EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "m
            "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",
            "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets", "moe_set_router_audit",
            "moe_forward_shared", "moe_workspace_size_shared", "moe_forward_mx", "moe_quantize_rows_mx",
-           "moe_set_fused_combine", "moe_set_layer_gemm", "moe_forward_plan"]
+           "moe_set_fused_combine", "moe_set_layer_gemm", "moe_forward_plan", "moe_set_direct_a"]
 DTYPE_BF16, DTYPE_FP8, DTYPE_MX = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
@@ -95,6 +95,8 @@ def lib():
         L.moe_forward_plan.restype = I32
         L.moe_set_layer_gemm.argtypes = [I32]
         L.moe_set_layer_gemm.restype = None
+        L.moe_set_direct_a.argtypes = [I32]
+        L.moe_set_direct_a.restype = None
         L.moe_set_fused_combine.argtypes = [I32]
         L.moe_set_fused_combine.restype = None
         L.moe_forward_mx.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -399,7 +401,7 @@ def set_pair_mma(mode: str):
     lib().moe_set_pair_mma({"auto": 0, "always": 1, "never": 2}[mode])
 
 
-PLAN_SMALL_ROUTER, PLAN_PAIR_TILES, PLAN_FUSED_COMBINE, PLAN_LAYER_GEMM = 1, 2, 4, 8
+PLAN_SMALL_ROUTER, PLAN_PAIR_TILES, PLAN_FUSED_COMBINE, PLAN_LAYER_GEMM, PLAN_DIRECT_A = 1, 2, 4, 8, 16
 
 
 def forward_plan(T, H, I, E, top_k, dtype: int = DTYPE_BF16) -> int:
@@ -410,6 +412,12 @@ def forward_plan(T, H, I, E, top_k, dtype: int = DTYPE_BF16) -> int:
 def set_layer_gemm(mode: str):
     """"auto" (default), "always" or "never": both bf16 expert GEMMs in one persistent launch."""
     lib().moe_set_layer_gemm({"auto": 0, "always": 1, "never": 2}[mode])
+
+
+def set_direct_a(mode: str):
+    """"auto" (default), "always" or "never": bf16 gate/up A rows gathered straight from x
+    by the GEMM (never: from a sorted copy of x made by a gather kernel first)."""
+    lib().moe_set_direct_a({"auto": 0, "always": 1, "never": 2}[mode])
 
 
 def set_fused_combine(mode: str):

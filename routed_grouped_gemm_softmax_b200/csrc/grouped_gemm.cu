@@ -19,6 +19,9 @@
 //   warp 0, lane 0: claims items, feeds a ring of item ids to the other roles,
 //                   and streams A and B tiles into a 4-stage shared-memory ring
 //                   with TMA (128-byte swizzle), one mbarrier pair per stage;
+//                   with direct A rows, the 32 lanes each gather four x rows of
+//                   a gate/up tile per stage (tile::gather4), so no expert-ordered
+//                   copy of x is written;
 //   warp 1        : allocates 512 TMEM columns; lane 0 issues tcgen05.mma
 //                   (M=128, N=256, K=16, bf16 in, fp32 accumulate) into one of
 //                   two TMEM accumulators, releasing each stage with
@@ -152,6 +155,7 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
             tma_prefetch_desc(&sm.b0);
             if (MODE == 0 || MODE == 3) tma_prefetch_desc(&sm.b1);
         }
+        if ((MODE == 0 || MODE == 3) && g.a_rows) tma_prefetch_desc(&sm.xg);
     }
     if (warp == 1) tmem_alloc(&S->tmem_base, TMEM_COLS);
     tc_fence_before();
@@ -161,8 +165,10 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
     // The prologue above overlapped the previous kernel.  Modes 0, 1 and 3: warp 0
     // waits for it inside the producer, after the first stages' weight loads (the
     // weights are the layer's inputs; only the A rows are the previous kernel's output).
-    constexpr bool kEarlyB = MODE != 2;
-    if (!(kEarlyB && warp == 0)) pdl_wait();
+    // (GemmArgs::tiles_first: the tile list itself is the previous kernel's output, so
+    // warp 0 waits first.)
+    const bool early_b = MODE != 2 && !g.tiles_first;
+    if (!(early_b && warp == 0)) pdl_wait();
     pdl_trigger();
     if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
@@ -184,16 +190,20 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
 
     if (warp == 0) {
         // ------------------------------------------------ scheduler + TMA producer
-        if (lane == 0) {
-            const int total = MODE == 3 ? total0 + mtiles * nt1 : mtiles * (MODE == 0 ? nt0 : nt1);
-            int stage = 0, rs = 0;
-            uint32_t phase = 0, rphase = 0;
-            uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
-            bool ok = true;
-            int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
-            bool held = kEarlyB;  // A loads of the first item's first stages wait for the previous kernel
-            for (;;) {
-                int item;
+        // Lane 0 claims the items, keeps the rings and loads B (and A with row-block
+        // boxes); with direct A rows (GemmArgs::a_rows) each lane gathers four A rows of a
+        // routed gate/up tile per stage, lane l rows 4l..4l+3.
+        const bool gather = (MODE == 0 || MODE == 3) && g.a_rows != nullptr;
+        const int total = MODE == 3 ? total0 + mtiles * nt1 : mtiles * (MODE == 0 ? nt0 : nt1);
+        int stage = 0, rs = 0;
+        uint32_t phase = 0, rphase = 0;
+        uint32_t armed = 0, armed_par = 0;  // stages with a load issued, and its phase
+        bool ok = true;
+        int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
+        bool held = early_b;  // A loads of the first item's first stages wait for the previous kernel
+        for (;;) {
+            int item = -1, okl = 1;
+            if (lane == 0) {
                 if (MODE != 3) {
                     item = claim_item(g.reverse, g.counter, total, MODE == 0 ? nt0 : nt1, dense ? nullptr : g.tiles,
                                       cursor, nrouted, g.sh_e0, sh_tps);
@@ -207,7 +217,6 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                 } else {
                     // static: this CTA's items in ascending order, every c-th (mode 2) or those
                     // of the experts e with e % grid == c (mode 3)
-                    item = -1;
                     while (cursor < total) {
                         const int it = cursor;
                         cursor += g.reverse == 2 ? (int)gridDim.x : 1;
@@ -216,64 +225,102 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                         if (t.e % (int)gridDim.x == (int)blockIdx.x) { item = it; break; }
                     }
                 }
-                if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
-                S->ring[rs] = item;
-                mbar_arrive(&S->itf[rs]);
-                if (++rs == RING) { rs = 0; rphase ^= 1; }
-                if (item < 0) break;
-                const ItemPos ip = pos_of(item);
-                const bool p1 = ip.p1;
-                TileRef tr{0, ip.mt * BM, 0, ip.mt * BM, -1};
-                if (dense)
-                    tr.rows = min(BM, g.M - tr.row0);
-                else
-                    tr = tile_ref(g.tiles, nrouted, ip.mt, BM, p1 ? 1 : 0, g.sh_T, g.sh_rows0, g.sh_e0);
-                const int expert = tr.e, arow0 = tr.arow0;
-                const int ab = a_box(tr.rows);  // the A box that covers the tile's rows
-                const CUtensorMap *amap = MODE == 3 && p1 ? &lm.h.m[ab]
-                                        : (!p1 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
-                const int n0 = ip.nt * (p1 ? BNO1 : BNO0);
-                const int num_kb = p1 ? kb1 : kb0;
-                if (MODE == 3 && p1) {
-                    // the down item reads h rows of m-tile mt: wait until every gate/up item of
-                    // mt has published them, then order those generic-proxy writes before the
-                    // TMA (async-proxy) reads below
-                    if (!wait_count_at_least(g.ready + ip.mt, 4 * nt0, g.wait_ns)) { ok = false; break; }
+                if (mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) {
+                    S->ring[rs] = item;
+                    mbar_arrive(&S->itf[rs]);
+                } else {
+                    okl = 0;
+                }
+            }
+            item = __shfl_sync(0xffffffffu, item, 0);
+            if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+            if (++rs == RING) { rs = 0; rphase ^= 1; }
+            if (item < 0) break;
+            const ItemPos ip = pos_of(item);
+            const bool p1 = ip.p1;
+            TileRef tr{0, ip.mt * BM, 0, ip.mt * BM, -1};
+            if (dense)
+                tr.rows = min(BM, g.M - tr.row0);
+            else
+                tr = tile_ref(g.tiles, nrouted, ip.mt, BM, p1 ? 1 : 0, g.sh_T, g.sh_rows0, g.sh_e0);
+            const int expert = tr.e, arow0 = tr.arow0;
+            const int ab = a_box(tr.rows);  // the A box that covers the tile's rows
+            const CUtensorMap *amap = MODE == 3 && p1 ? &lm.h.m[ab]
+                                    : (!p1 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
+            // direct rows: the x rows (tokens) of this lane's four tile rows, the tail's
+            // missing rows repeating the tile's last one (their products are masked)
+            const bool g4 = gather && !p1 && tr.s < 0;
+            const bool g4_lane = g4 && 4 * lane < tr.rows;
+            int tok[4] = {0, 0, 0, 0};
+            auto load_tokens = [&]() {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int t = g.a_rows[tr.row0 + min(4 * lane + j, tr.rows - 1)] / g.a_div;
+                    tok[j] = (unsigned)t < (unsigned)g.a_tokens ? t : 0;
+                }
+            };
+            if (g4_lane && !held) load_tokens();
+            const uint32_t a_bytes = g4 ? (uint32_t)((tr.rows + 3) / 4) * 512u : (uint32_t)(a_box_rows(ab) * BK * 2);
+            const int n0 = ip.nt * (p1 ? BNO1 : BNO0);
+            const int num_kb = p1 ? kb1 : kb0;
+            if (MODE == 3 && p1) {
+                // the down item reads h rows of m-tile mt: wait until every gate/up item of
+                // mt has published them, then order those generic-proxy writes before the
+                // TMA (async-proxy) reads below
+                if (lane == 0) {
+                    okl = wait_count_at_least(g.ready + ip.mt, 4 * nt0, g.wait_ns);
                     fence_proxy_async_global();
                 }
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&S->full[stage], a_box_rows(ab) * BK * 2 + B_BYTES);
-                    armed |= 1u << stage;
-                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-                    uint8_t *b_dst = sB + stage * B_BYTES;
-                    if (!held) tma_load_2d(sA + stage * A_BYTES, amap, &S->full[stage], kb * BK, arow0);
-                    if (!p1) {  // gate / up rows n0.. of the expert (or of shared slice s)
-                        if (tr.s < 0) {
-                            tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
-                            tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
-                        } else {
-                            tma_load_2d(b_dst, &sm.b0, &S->full[stage], kb * BK, tr.s * g.N + n0);
-                            tma_load_2d(b_dst + B_BYTES / 2, &sm.b1, &S->full[stage], kb * BK, tr.s * g.N + n0);
+                if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+            }
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (lane == 0) {
+                    okl = mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns);
+                    if (okl) {
+                        mbar_arrive_expect_tx(&S->full[stage], a_bytes + B_BYTES);
+                        armed |= 1u << stage;
+                        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                        uint8_t *b_dst = sB + stage * B_BYTES;
+                        if (!held && !g4) tma_load_2d(sA + stage * A_BYTES, amap, &S->full[stage], kb * BK, arow0);
+                        if (!p1) {  // gate / up rows n0.. of the expert (or of shared slice s)
+                            if (tr.s < 0) {
+                                tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
+                                tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
+                            } else {
+                                tma_load_2d(b_dst, &sm.b0, &S->full[stage], kb * BK, tr.s * g.N + n0);
+                                tma_load_2d(b_dst + B_BYTES / 2, &sm.b1, &S->full[stage], kb * BK, tr.s * g.N + n0);
+                            }
+                        } else {  // down (or dense) rows n0..: the expert's, or columns s*I.. of the shared down
+                            const CUtensorMap *bm = MODE == 3 ? &lm.wd : &tmB0;
+                            const CUtensorMap *bs = MODE == 3 ? &lm.wd_sh : &sm.b0;
+                            if (tr.s < 0)
+                                tma_load_3d(b_dst, bm, &S->full[stage], kb * BK, n0, expert);
+                            else
+                                tma_load_2d(b_dst, bs, &S->full[stage], tr.s * (MODE == 3 ? g.K2 : g.K) + kb * BK, n0);
                         }
-                    } else {  // down (or dense) rows n0..: the expert's, or columns s*I.. of the shared down
-                        const CUtensorMap *bm = MODE == 3 ? &lm.wd : &tmB0;
-                        const CUtensorMap *bs = MODE == 3 ? &lm.wd_sh : &sm.b0;
-                        if (tr.s < 0)
-                            tma_load_3d(b_dst, bm, &S->full[stage], kb * BK, n0, expert);
-                        else
-                            tma_load_2d(b_dst, bs, &S->full[stage], tr.s * (MODE == 3 ? g.K2 : g.K) + kb * BK, n0);
                     }
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                    if (held && kb + 1 == min(STAGES, num_kb)) {  // first item: stage j holds K block j
-                        pdl_wait();
-                        held = false;
-                        for (int j = 0; j <= kb; ++j)
+                }
+                if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+                if (g4_lane && !held)
+                    tma_gather4(sA + stage * A_BYTES + lane * 512, &sm.xg, &S->full[stage], kb * BK, tok[0], tok[1],
+                                tok[2], tok[3]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                if (held && kb + 1 == min(STAGES, num_kb)) {  // first item: stage j holds K block j
+                    pdl_wait();
+                    held = false;
+                    if (g4_lane) load_tokens();
+                    for (int j = 0; j <= kb; ++j) {
+                        if (g4_lane)
+                            tma_gather4(sA + j * A_BYTES + lane * 512, &sm.xg, &S->full[j], j * BK, tok[0], tok[1],
+                                        tok[2], tok[3]);
+                        else if (!g4 && lane == 0)
                             tma_load_2d(sA + j * A_BYTES, amap, &S->full[j], j * BK, arow0);
                     }
                 }
-                if (!ok) break;
             }
+            if (!ok) break;
+        }
+        if (lane == 0) {
             if (!ok) {
                 record_status(g.status, MOE_ERR_TIMEOUT);
                 if (mbar_wait(&S->ite[rs], rphase ^ 1)) {
@@ -488,6 +535,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUten
     if (g.mode < 0 || g.mode > 3 || !smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
     if (g.sh_count && (!sm || g.mode == 2)) return cudaErrorInvalidValue;
     if (g.mode == 3 && (!lm || !g.ready)) return cudaErrorInvalidValue;
+    if (g.a_rows && (!sm || g.a_div <= 0 || g.a_tokens <= 0 || (g.mode != 0 && g.mode != 3))) return cudaErrorInvalidValue;
     static const SharedMaps none{};
     static const LayerMaps nolm{};
     const SharedMaps &s = sm ? *sm : none;

@@ -13,7 +13,9 @@
 //
 // Roles: CTA 0 (the leader) claims items from the atomic queue and hands each one
 // to CTA 1 through its shared memory; in both CTAs warp 0 streams that CTA's A and
-// B halves with TMA, completing on the leader's stage barrier; the leader's warp 1
+// B halves with TMA, completing on the leader's stage barrier (with direct A rows the
+// warp's 32 lanes gather a gate/up tile's x rows four at a time, tile::gather4, so
+// no expert-ordered copy of x is written); the leader's warp 1
 // issues the MMAs and commits each stage, the accumulators and the end to both
 // CTAs' barriers at once (tcgen05.commit with a CTA mask); warps 2-5 of both CTAs
 // drain their accumulator halves.  No TMA load is multicast.  Every wait is
@@ -93,6 +95,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *t
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+// Four rows r0..r3 of a one-row-box tensor map to this CTA's dst, signalling the
+// leader CTA's barrier (tile::gather4 of a CTA pair).
+__device__ __forceinline__ void tma_gather4_pair(void *dst, const CUtensorMap *tm, uint32_t bar, int x, int r0, int r1,
+                                                 int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
         : "memory");
 }
 __device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *tm, uint32_t bar, int x, int y, int z)
@@ -232,6 +245,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
             tma_prefetch_desc(&sm.b0);
             if (MODE != 1) tma_prefetch_desc(&sm.b1);
         }
+        if (MODE != 1 && g.a_rows) tma_prefetch_desc(&sm.xg);
     }
     if (warp == 1) tmem_alloc_pair(&S->tmem_base, TMEM_COLS2);
     tc_fence_before();
@@ -242,7 +256,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
     // The prologue above overlapped the previous kernel; warp 0 waits for it inside the
     // producer, after the first stages' weight loads (only the A rows are the previous
     // kernel's output).
-    if (warp != 0) pdl_wait();
+    if (warp != 0 || g.tiles_first) pdl_wait();
     pdl_trigger();
     if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
@@ -263,14 +277,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
 
     if (warp == 0) {
         // -------------------------------- item hand-off (leader) + TMA producer (both)
-        if (lane == 0) {
-            const int total = MODE == 3 ? total0 + mtiles * nt1 : mtiles * (MODE == 0 ? nt0 : nt1);
-            int stage = 0, rs = 0, cursor = 0;
-            uint32_t phase = 0, rphase = 0;
-            bool ok = true;
-            bool held = true;  // A loads of the first item's first stages wait for the previous kernel
-            for (;;) {
-                int item;
+        // Lane 0 hands items over and loads B (and A with row-block boxes); with direct
+        // A rows (GemmArgs::a_rows) each lane gathers four A rows of this CTA's half of
+        // a routed gate/up tile per stage, lane l rows 4l..4l+3.
+        const bool gather = MODE != 1 && g.a_rows != nullptr;
+        const int total = MODE == 3 ? total0 + mtiles * nt1 : mtiles * (MODE == 0 ? nt0 : nt1);
+        int stage = 0, rs = 0, cursor = 0;
+        uint32_t phase = 0, rphase = 0;
+        bool ok = true;
+        bool held = !g.tiles_first;  // A loads of the first item's first stages wait for the previous kernel
+        for (;;) {
+            int item = -1, okl = 1;
+            if (lane == 0) {
                 if (rank == 0) {
                     if (MODE != 3) {
                         item = claim_item(g.reverse, g.counter, total, MODE == 0 ? nt0 : nt1, tiles2, cursor, nrouted,
@@ -281,71 +299,111 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                         else if (g.reverse == 1)
                             item = item < total0 ? total0 - 1 - item : total0 + (total - 1 - item);
                     }
-                    if (!wait2(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
-                    S->ring[rs] = item;
-                    st_remote(peer_addr(&S->ring[rs], 1), item);
-                    mbar_arrive(&S->itf[rs]);
-                    arrive_remote(peer_addr(&S->itf[rs], 1));
+                    if (wait2(&S->ite[rs], rphase ^ 1, g.wait_ns)) {
+                        S->ring[rs] = item;
+                        st_remote(peer_addr(&S->ring[rs], 1), item);
+                        mbar_arrive(&S->itf[rs]);
+                        arrive_remote(peer_addr(&S->itf[rs], 1));
+                    } else {
+                        okl = 0;
+                    }
                 } else {
-                    if (!wait2(&S->itf[rs], rphase, g.wait_ns)) { ok = false; break; }
-                    item = S->ring[rs];
-                    arrive_remote(peer_addr(&S->ite[rs], 0));
+                    if (wait2(&S->itf[rs], rphase, g.wait_ns)) {
+                        item = S->ring[rs];
+                        arrive_remote(peer_addr(&S->ite[rs], 0));
+                    } else {
+                        okl = 0;
+                    }
                 }
-                if (++rs == RING2) { rs = 0; rphase ^= 1; }
-                if (item < 0) break;
-                int mt, nt;
-                const bool p1 = pos_of(item, mt, nt);
-                const TileRef tr = tile_ref(tiles2, nrouted, mt, 2 * HALF, p1 ? 1 : 0, g.sh_T, g.sh_rows0, g.sh_e0);
-                const int expert = tr.e;
-                const int arow0 = tr.arow0 + (int)rank * HALF;  // this CTA's half of the pair tile
-                const int rows = min(HALF, max(0, tr.rows - (int)rank * HALF));
-                const int ab = a_box(rows);
-                const CUtensorMap *amap = MODE == 3 && p1 ? &lm.h.m[ab] : (!p1 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
-                const uint32_t a_bytes = rows > 0 ? (uint32_t)(a_box_rows(ab) * BK2 * 2) : 0u;
-                // B rows of this CTA: gate (CTA 0) or up (CTA 1) rows nt*128.. ; down: output columns
-                const int nrow = !p1 ? nt * BNO0 : nt * BNO1 + (int)rank * 128;
-                const CUtensorMap *bmap = !p1 ? (rank == 1 ? (tr.s >= 0 ? &sm.b1 : &tmB1) : (tr.s >= 0 ? &sm.b0 : &tmB0))
-                                        : MODE == 3 ? (tr.s >= 0 ? &lm.wd_sh : &lm.wd)
-                                                    : (tr.s >= 0 ? &sm.b0 : &tmB0);
-                const bool b_in = nrow < (p1 ? NP1 : g.N);  // a half entirely past N loads nothing (masked columns)
-                const uint32_t b_bytes = b_in ? (uint32_t)B2_BYTES : 0u;
-                const int num_kb = p1 ? kb1 : kb0;
-                if (MODE == 3 && p1) {
-                    // the h rows of pair tile mt: wait until every gate/up item of mt published
-                    // them (4 epilogue warps in each of the 2 CTAs), then order those
-                    // generic-proxy writes before this CTA's TMA reads
-                    if (!wait_count_at_least2(g.ready + mt, 8 * nt0, g.wait_ns)) { ok = false; break; }
+            }
+            item = __shfl_sync(0xffffffffu, item, 0);
+            if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+            if (++rs == RING2) { rs = 0; rphase ^= 1; }
+            if (item < 0) break;
+            int mt, nt;
+            const bool p1 = pos_of(item, mt, nt);
+            const TileRef tr = tile_ref(tiles2, nrouted, mt, 2 * HALF, p1 ? 1 : 0, g.sh_T, g.sh_rows0, g.sh_e0);
+            const int expert = tr.e;
+            const int arow0 = tr.arow0 + (int)rank * HALF;  // this CTA's half of the pair tile
+            const int rows = min(HALF, max(0, tr.rows - (int)rank * HALF));
+            const int ab = a_box(rows);
+            const CUtensorMap *amap = MODE == 3 && p1 ? &lm.h.m[ab] : (!p1 && tr.s >= 0) ? &sm.x.m[ab] : &tmA.m[ab];
+            // direct rows: the x rows (tokens) of this lane's four rows, the tail's missing
+            // rows repeating the half's last one (their products are masked)
+            const bool g4 = gather && !p1 && tr.s < 0;
+            const bool g4_lane = g4 && 4 * lane < rows;
+            int tok[4] = {0, 0, 0, 0};
+            auto load_tokens = [&]() {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int t = g.a_rows[arow0 + min(4 * lane + j, rows - 1)] / g.a_div;
+                    tok[j] = (unsigned)t < (unsigned)g.a_tokens ? t : 0;
+                }
+            };
+            if (g4_lane && !held) load_tokens();
+            const uint32_t a_bytes = rows <= 0 ? 0u
+                                   : g4        ? (uint32_t)((rows + 3) / 4) * 512u
+                                               : (uint32_t)(a_box_rows(ab) * BK2 * 2);
+            // B rows of this CTA: gate (CTA 0) or up (CTA 1) rows nt*128.. ; down: output columns
+            const int nrow = !p1 ? nt * BNO0 : nt * BNO1 + (int)rank * 128;
+            const CUtensorMap *bmap = !p1 ? (rank == 1 ? (tr.s >= 0 ? &sm.b1 : &tmB1) : (tr.s >= 0 ? &sm.b0 : &tmB0))
+                                    : MODE == 3 ? (tr.s >= 0 ? &lm.wd_sh : &lm.wd)
+                                                : (tr.s >= 0 ? &sm.b0 : &tmB0);
+            const bool b_in = nrow < (p1 ? NP1 : g.N);  // a half entirely past N loads nothing (masked columns)
+            const uint32_t b_bytes = b_in ? (uint32_t)B2_BYTES : 0u;
+            const int num_kb = p1 ? kb1 : kb0;
+            if (MODE == 3 && p1) {
+                // the h rows of pair tile mt: wait until every gate/up item of mt published
+                // them (4 epilogue warps in each of the 2 CTAs), then order those
+                // generic-proxy writes before this CTA's TMA reads
+                if (lane == 0) {
+                    okl = wait_count_at_least2(g.ready + mt, 8 * nt0, g.wait_ns);
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                 }
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!wait2(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
-                    const uint32_t fb = peer_addr(&S->full[stage], 0);
-                    if (rank == 0)
-                        mbar_arrive_expect_tx(&S->full[stage], a_bytes + b_bytes);
-                    else
-                        arrive_expect_tx_remote(fb, a_bytes + b_bytes);
-                    if (rows > 0 && !held) tma_load_2d_pair(sA + stage * A2_BYTES, amap, fb, kb * BK2, arow0);
-                    if (b_in) {
-                        if (tr.s < 0)
-                            tma_load_3d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, nrow, expert);
-                        else if (!p1)  // shared slice s: rows s*I + nrow.. of the shared gate / up
-                            tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, tr.s * g.N + nrow);
-                        else  // shared down: columns s*I + kb*BK2..
-                            tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, tr.s * KP1 + kb * BK2, nrow);
-                    }
-                    if (++stage == ST2) { stage = 0; phase ^= 1; }
-                    if (held && kb + 1 == min(ST2, num_kb)) {  // first item: stage j holds K block j
-                        pdl_wait();
-                        held = false;
-                        if (rows > 0)
-                            for (int j = 0; j <= kb; ++j)
-                                tma_load_2d_pair(sA + j * A2_BYTES, amap, peer_addr(&S->full[j], 0), j * BK2, arow0);
+                if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+            }
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const uint32_t fb = peer_addr(&S->full[stage], 0);
+                if (lane == 0) {
+                    okl = wait2(&S->empty[stage], phase ^ 1, g.wait_ns);
+                    if (okl) {
+                        if (rank == 0)
+                            mbar_arrive_expect_tx(&S->full[stage], a_bytes + b_bytes);
+                        else
+                            arrive_expect_tx_remote(fb, a_bytes + b_bytes);
+                        if (rows > 0 && !held && !g4)
+                            tma_load_2d_pair(sA + stage * A2_BYTES, amap, fb, kb * BK2, arow0);
+                        if (b_in) {
+                            if (tr.s < 0)
+                                tma_load_3d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, nrow, expert);
+                            else if (!p1)  // shared slice s: rows s*I + nrow.. of the shared gate / up
+                                tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, tr.s * g.N + nrow);
+                            else  // shared down: columns s*I + kb*BK2..
+                                tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, tr.s * KP1 + kb * BK2, nrow);
+                        }
                     }
                 }
-                if (!ok) break;
+                if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
+                if (g4_lane && !held)
+                    tma_gather4_pair(sA + stage * A2_BYTES + lane * 512, &sm.xg, fb, kb * BK2, tok[0], tok[1], tok[2],
+                                     tok[3]);
+                if (++stage == ST2) { stage = 0; phase ^= 1; }
+                if (held && kb + 1 == min(ST2, num_kb)) {  // first item: stage j holds K block j
+                    pdl_wait();
+                    held = false;
+                    if (g4_lane) load_tokens();
+                    for (int j = 0; j <= kb; ++j) {
+                        if (g4_lane)
+                            tma_gather4_pair(sA + j * A2_BYTES + lane * 512, &sm.xg, peer_addr(&S->full[j], 0),
+                                             j * BK2, tok[0], tok[1], tok[2], tok[3]);
+                        else if (!g4 && lane == 0 && rows > 0)
+                            tma_load_2d_pair(sA + j * A2_BYTES, amap, peer_addr(&S->full[j], 0), j * BK2, arow0);
+                    }
+                }
             }
-            if (!ok) record2(g.status, MOE_ERR_TIMEOUT);
+            if (!ok) break;
         }
+        if (!ok && lane == 0) record2(g.status, MOE_ERR_TIMEOUT);
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader only)
@@ -528,6 +586,7 @@ cudaError_t launch_grouped_gemm_2cta(const GemmArgs &g, const AMaps &tmA, const 
     if (!smem2_ready(g.mode)) return cudaErrorInvalidValue;
     if (g.sh_count && !sm) return cudaErrorInvalidValue;
     if (g.mode == 3 && (!lm || !g.ready)) return cudaErrorInvalidValue;
+    if (g.a_rows && (!sm || g.a_div <= 0 || g.a_tokens <= 0 || g.mode == 1)) return cudaErrorInvalidValue;
     static const SharedMaps none{};
     static const LayerMaps nolm{};
     const SharedMaps &s = sm ? *sm : none;

@@ -25,6 +25,7 @@ std::atomic<int> g_pair_mode{0};  // 0 auto, 1 pair GEMMs whenever possible, 2 n
 std::atomic<int> g_fp8_swap{0};   // 0 auto, 1 swapped fp8 gate/up GEMM always, 2 never
 std::atomic<int> g_fused_comb{0}; // 0 auto, 1 combine inside the down GEMM always, 2 never
 std::atomic<int> g_layer_gemm{0}; // 0 auto, 1 gate/up and down GEMMs in one launch always, 2 never
+std::atomic<int> g_direct_a{0};   // 0 auto, 1 gate/up A rows gathered straight from x always, 2 never
 std::atomic<int> g_trace_ctas{0};
 std::atomic<unsigned long long> g_wait_ns{0};
 std::atomic<int> g_stall_test{0};
@@ -216,8 +217,10 @@ int bf16_plan(const moe_dims_t &d)
     const bool fused = fc == 1 || (fc == 0 && d.T <= moe::kFusedCombineMaxT);
     const int lg = g_layer_gemm.load();
     const bool layer = lg == 1 || (lg == 0 && tc.layer_gemm);
+    const int da = g_direct_a.load();
+    const bool direct = da == 1 || (da == 0 && tc.direct_a);
     return (small ? MOE_PLAN_SMALL_ROUTER : 0) | (pairs ? MOE_PLAN_PAIR_TILES : 0) |
-           (fused ? MOE_PLAN_FUSED_COMBINE : 0) | (layer ? MOE_PLAN_LAYER_GEMM : 0);
+           (fused ? MOE_PLAN_FUSED_COMBINE : 0) | (layer ? MOE_PLAN_LAYER_GEMM : 0) | (direct ? MOE_PLAN_DIRECT_A : 0);
 }
 
 // Activations, weights and outputs are read and written in 16-byte vectors (and the
@@ -345,6 +348,8 @@ void moe_set_pair_mma(int32_t mode) { g_pair_mode.store(mode < 0 || mode > 2 ? 0
 void moe_set_fp8_swap_ab(int32_t mode) { g_fp8_swap.store(mode < 0 || mode > 2 ? 0 : mode); }
 void moe_set_fused_combine(int32_t mode) { g_fused_comb.store(mode < 0 || mode > 2 ? 0 : mode); }
 void moe_set_layer_gemm(int32_t mode) { g_layer_gemm.store(mode < 0 || mode > 2 ? 0 : mode); }
+
+void moe_set_direct_a(int32_t mode) { g_direct_a.store(mode < 0 || mode > 2 ? 0 : mode); }
 
 void moe_set_gemm_trace(unsigned long long *trace, int32_t ctas)
 {
@@ -480,6 +485,13 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
                !encode_2d(&sm1.b1, shared_up, shared_I, d->H, 128) ||
                !encode_2d(&sm2.b0, shared_down, d->H, shared_I, pairs ? 128 : 256)))
         return MOE_ERR_CUDA;
+    // gate/up A rows straight from x: one-row boxes for tile::gather4, the token of
+    // sorted row r being sorted_to_flat[r] / k
+    const bool direct = plan & MOE_PLAN_DIRECT_A;
+    if (direct && !encode_2d(&sm1.xg, x, d->T, d->H, 1)) return MOE_ERR_CUDA;
+    // the tile list is then the output of the kernel just before the gate/up GEMM
+    // when the router and the grouping are one launch
+    const int tiles_first = direct && (plan & MOE_PLAN_SMALL_ROUTER) ? 1 : 0;
 
     const StageMarks marks;
     const bool fused = plan & MOE_PLAN_FUSED_COMBINE;  // combine inside the down GEMM
@@ -487,7 +499,7 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
     if (e == cudaSuccess && !moe::small_route_permute_ok(*d))  // else the router's kernels clear them
         e = cudaMemsetAsync(hdr, 0, L.clear_bytes, st);          // header + combine counts
     if (e == cudaSuccess) e = route_and_permute(*d, L, x, router_w, router_bias, ws, hdr, marks, st);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && !direct)
         e = moe::launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), at<int32_t>(ws, L.f2s), d->T, d->H,
                                     d->top_k, xs, st);
     if (e == cudaSuccess) e = marks.mark(2, st);
@@ -512,6 +524,12 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
         gl.N2 = d->H;
         gl.out2 = y;
         gl.ready = at<int32_t>(ws, L.ready);
+        if (direct) {
+            gl.a_rows = s2f;
+            gl.a_div = d->top_k;
+            gl.a_tokens = d->T;
+            gl.tiles_first = tiles_first;
+        }
         moe::LayerMaps lm{};
         lm.h = tm_h;
         lm.wd = tm_wd;
@@ -529,6 +547,12 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
         g1.sh_T = d->T;
         g1.sh_rows0 = A;
         g1.sh_e0 = d->E;
+        if (direct) {
+            g1.a_rows = s2f;
+            g1.a_div = d->top_k;
+            g1.a_tokens = d->T;
+            g1.tiles_first = tiles_first;
+        }
         e = pairs ? moe::launch_grouped_gemm_2cta(g1, tm_xs, tm_wg, tm_wu, at<int32_t>(ws, L.tiles2),
                                                   at<int32_t>(ws, L.ntiles2), st, &sm1)
                   : moe::launch_grouped_gemm(g1, tm_xs, tm_wg, tm_wu, st, &sm1);

@@ -211,9 +211,13 @@ struct GemmArgs {
     int32_t *ready;
     // Gate/up items of routed tiles with a_rows non-null: the A rows are read straight
     // from x (SharedMaps::xg, one-row boxes) by tile::gather4 loads, row r of a tile
-    // being token a_rows[row0 + r] / a_div (no expert-ordered copy of x is made).
+    // being token a_rows[row0 + r] / a_div (no expert-ordered copy of x is made); a
+    // token outside [0, a_tokens) reads row 0 instead.
     const int32_t *a_rows;
-    int a_div;
+    int a_div, a_tokens;
+    // The tile list is written by the kernel launched just before this one (no other
+    // kernel in between), so it is read only after the programmatic-dependency wait.
+    int tiles_first;
 };
 
 // Tensor maps of the down half of the fused layer GEMM (mode 3): h as its A operand
@@ -372,11 +376,13 @@ struct TileChoice {
     bool pair_tiles;  // bf16: 256-row tiles on CTA pairs (tcgen05 cta_group::2)
     bool layer_gemm;  // bf16: the gate/up and down GEMMs in one launch
     bool fp8_swap_ab; // fp8: gate/up GEMM with the weight rows on the MMA's M side
+    bool direct_a;    // bf16: gate/up A rows gathered straight from x (no sorted copy)
 };
 constexpr TileChoice kTileTable[] = {
-    {64, false, true, true},
-    {511, false, true, false},
-    {0x7fffffff, true, true, false},
+    {16, false, true, true, true},
+    {64, false, true, true, false},
+    {511, false, true, false, false},
+    {0x7fffffff, true, true, false, false},
 };
 inline TileChoice tile_choice(long long A, int E)
 {
@@ -393,11 +399,11 @@ constexpr int kFusedCombineMaxTFp8 = 64;
 
 int num_sms();
 
-// Tensor map of a row-major bf16 matrix [rows, cols], box_rows x box_cols tiles,
-// no swizzle (box_cols * 2 a multiple of 16).
 // Tensor map of a row-major bf16 matrix [rows, cols], box_rows x 64 tiles with the
 // 128-byte swizzle (16-byte chunk c of tile row r stored at chunk c ^ (r % 8)).
 bool encode_sw128_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Tensor map of a row-major bf16 matrix [rows, cols], box_rows x box_cols tiles,
+// no swizzle (box_cols * 2 a multiple of 16).
 bool encode_plain_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                           uint32_t box_rows);
 

@@ -142,7 +142,15 @@ int main(void) {
 def test_forward_plan_follows_the_tile_table(L):
     # The plan query is host-only: the kernels a forward would launch under the
     # current settings, by the M bucket (average rows per expert) of the batch.
-    plan = lambda T, H, I, E, k, dt=api.DTYPE_BF16: api.forward_plan(T, H, I, E, k, dt)
+    bf = lambda T, H, I, E, k: api.forward_plan(T, H, I, E, k, api.DTYPE_BF16)
+    # gate/up A rows straight from x up to 16 rows per expert, the sorted copy above
+    def plan(T, H, I, E, k, dt=api.DTYPE_BF16):
+        p = api.forward_plan(T, H, I, E, k, dt)
+        return p if p < 0 or dt != api.DTYPE_BF16 else p & ~api.PLAN_DIRECT_A
+    for T in (1, 16, 33, 128):
+        assert bf(T, 2048, 1024, 64, 8) & api.PLAN_DIRECT_A
+    for T in (136, 4096, 8192):   # 17 and more rows per expert
+        assert not bf(T, 2048, 1024, 64, 8) & api.PLAN_DIRECT_A
     # decode-sized: the two-kernel router, 128-row tiles, one GEMM launch, combine inside
     assert plan(16, 2048, 512, 256, 8) == api.PLAN_SMALL_ROUTER | api.PLAN_FUSED_COMBINE | api.PLAN_LAYER_GEMM
     # 128 rows per expert: 128-row tiles, one GEMM launch, the combine kernel
@@ -158,10 +166,12 @@ def test_forward_plan_follows_the_tile_table(L):
     try:
         api.set_pair_mma("never")
         api.set_layer_gemm("never")
-        assert plan(8192, 4096, 1408, 64, 6) == 0
+        api.set_direct_a("never")
+        assert bf(8192, 4096, 1408, 64, 6) == 0
     finally:
         api.set_pair_mma("auto")
         api.set_layer_gemm("auto")
+        api.set_direct_a("auto")
     assert plan(64, 100, 512, 8, 2) == -1   # invalid dims
     assert plan(1024, 7168, 2048, 256, 8, api.DTYPE_FP8) == 0
     assert plan(16, 7168, 2048, 256, 8, api.DTYPE_FP8) == api.PLAN_SMALL_ROUTER | api.PLAN_FUSED_COMBINE

@@ -15,20 +15,23 @@ PEAKS = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1200
 
 def test_kernels_per_forward_match_the_launch_lists():
     # one forward's kernels, as listed by ncu on the GPU:
-    # decode: logits, top-k + grouping, gather, the layer GEMM (both expert GEMMs and
-    # the combine in one launch)
-    assert bench.kernels_per_forward(CONFIGS["decode"]) == 4
+    # decode: logits, top-k + grouping, the layer GEMM (x rows gathered by the GEMM,
+    # both expert GEMMs and the combine in one launch)
+    assert bench.kernels_per_forward(CONFIGS["decode"]) == 3
     # prefill/skewed: prep, tensor-core logits, certify, count, scan, scatter, gather,
     # the layer GEMM, combine
     assert bench.kernels_per_forward(CONFIGS["prefill"]) == 9
     assert bench.kernels_per_forward(CONFIGS["skewed"]) == 9
     # fp8: the large-batch router and grouping, quantiser, gather, two GEMMs, combine
     assert bench.kernels_per_forward(CONFIGS["fp8"]) == 11
-    # tiny (T = 64): the large-batch router, the layer GEMM, the combine kernel
-    assert bench.kernels_per_forward(CONFIGS["tiny"]) == 9
-    # with the library's plan bits: two GEMM launches and the combine inside the second
+    # tiny (T = 64, 16 rows per expert): the large-batch router, the layer GEMM
+    # gathering its x rows, the combine kernel
+    assert bench.kernels_per_forward(CONFIGS["tiny"]) == 8
+    # with the library's plan bits: the gather kernel (no direct A rows), two GEMM
+    # launches and the combine inside the second
     assert bench.kernels_per_forward(CONFIGS["decode"], plan=1 | 4) == 2 + 1 + 2
     assert bench.kernels_per_forward(CONFIGS["prefill"], plan=2 | 8) == 6 + 1 + 1 + 1
+    assert bench.kernels_per_forward(CONFIGS["prefill"], plan=2 | 8 | 16) == 6 + 1 + 1
 
 
 def test_stage_work_bf16_by_hand():

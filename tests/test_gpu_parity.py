@@ -12,7 +12,7 @@ import oracle
 from gpu_helpers import (compare_out, compare_permute, compare_routing, device_inputs,
                          hot_expert_tokens, sample_tokens)
 from routed_grouped_gemm_softmax_b200 import api
-from routed_grouped_gemm_softmax_b200.inputs import CONFIGS
+from routed_grouped_gemm_softmax_b200.inputs import CONFIGS, make_shared_weights
 
 pytestmark = pytest.mark.gpu
 
@@ -372,6 +372,68 @@ def test_layer_gemm_matches_two_launches(name):
     tok = sample_tokens(cfg.T, 64, seed=cfg.seed)
     ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"], tokens=tok)
     compare_out(outs[1][torch.as_tensor(tok, device="cuda").long()], ref, f"{name} layer GEMM")
+
+
+DIRECT_A_CASES = {
+    "ragged": (SMALL["ragged"], "auto", 0),            # ragged group tails
+    "one_token": (SMALL["one_token"], "auto", 0),      # one-row tiles
+    "wide_e": (SMALL["wide_e"], "auto", 0),            # 300 experts, mostly one-row groups
+    "ragged_bias": (SMALL["ragged_bias"], "auto", 0),  # H = 320: five 64-column K blocks
+    "decode": (CONFIGS["decode"], "auto", 0),
+    "prefill_rows": (CONFIGS["tiny"].replace(name="da_pf", T=1024, H=512, E=8, top_k=2, I=256, seed=27), "auto", 0),
+    "deep_pairs": (PAIR_CASES["deep"], "always", 0),
+    "ragged_pairs": (PAIR_CASES["ragged"], "always", 0),  # pair tiles with an empty or short second half
+    "ragged_shared": (SMALL["ragged"], "auto", 2),        # the shared expert's tiles read x with row boxes
+    "pairs_shared": (PAIR_CASES["ragged_bias"], "always", 1),
+}
+
+
+@pytest.mark.parametrize("name", list(DIRECT_A_CASES))
+def test_direct_a_rows_match_the_sorted_copy(name):
+    # The gate/up GEMM gathering its A rows straight from x (four rows per TMA
+    # tile::gather4, the tail's missing rows repeating the last) gives the result of
+    # reading the expert-sorted copy of x bit for bit: one or two GEMM launches, one
+    # CTA per SM or a few, both queue orders, with the router's one-launch form (the
+    # tile list written by the kernel just before the GEMM) and its multi-kernel form.
+    cfg, pair, mult = DIRECT_A_CASES[name]
+    g, c = device_inputs(cfg)
+    k = cfg.top_k
+    sw = [t.cuda() for t in make_shared_weights(cfg, mult * cfg.I)] if mult else None
+    outs = []
+    try:
+        api.set_pair_mma(pair)
+        for da, lg, ctas, rev in [("never", "never", 0, False), ("always", "never", 0, False),
+                                  ("always", "always", 0, False), ("never", "always", 0, False),
+                                  ("always", "always", 4, True), ("always", "never", 6, True)]:
+            api.set_direct_a(da)
+            api.set_layer_gemm(lg)
+            api.set_gemm_ctas(ctas)
+            api.set_claim_order(rev)
+            if sw:
+                ws = torch.empty(api.moe_workspace_size_shared(cfg.T, cfg.H, cfg.I, cfg.E, k, mult * cfg.I),
+                                 dtype=torch.uint8, device="cuda")
+                o = api.moe_forward_shared(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"],
+                                           *sw, k, ws=ws)
+            else:
+                ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, k, "cuda")
+                o = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], k, ws=ws)
+            outs.append(o.clone())
+            assert api.moe_get_device_status(ws) == api.MOE_OK
+            plan = api.forward_plan(cfg.T, cfg.H, cfg.I, cfg.E, k)
+            assert bool(plan & api.PLAN_DIRECT_A) == (da == "always")
+    finally:
+        api.set_pair_mma("auto")
+        api.set_direct_a("auto")
+        api.set_layer_gemm("auto")
+        api.set_gemm_ctas(0)
+        api.set_claim_order(False)
+    for i, o in enumerate(outs[1:], 1):
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16)), (name, i)
+    if sw is None:
+        idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], c["bias"], k)
+        tok = sample_tokens(cfg.T, 64, seed=cfg.seed)
+        ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"], tokens=tok)
+        compare_out(outs[1][torch.as_tensor(tok, device="cuda").long()], ref, f"{name} direct A rows")
 
 
 def test_stage_events_outside_and_inside_capture():
