@@ -25,6 +25,7 @@
 //        against its bound (a miss records MOE_ERR_ROUTER_BOUND);
 //     c. per token (a warp), top-k and softmax on the candidates' exact values.
 // The chosen experts and gates are therefore those of the chain definition.
+#include <atomic>
 #include <cfloat>
 #include <climits>
 
@@ -83,11 +84,12 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const __nv_bfloat16 *_
     }
 }
 
-constexpr int kCertThreads = 512;
-constexpr int kCertWarps = kCertThreads / 32;
+// Threads of a certify CTA: 1024 (a chain each, 64 registers) up to 256 experts, 512
+// above (the per-lane arrays of 512 or more experts need the registers).
+constexpr int kCertWarps = 32;  // the most warps a CTA has (sizes the per-warp scratch)
+__host__ __device__ constexpr int cert_threads(int maxv) { return maxv <= 8 ? 1024 : 512; }
 constexpr int kCertMaxStages = 3;
-constexpr int kCertChains = 2;  // chains per thread per round
-constexpr int kCertMaxTB = 64;  // tokens per CTA
+constexpr int kCertMaxTB = 128;  // tokens per block
 constexpr int kCertSmem = 227 * 1024;
 
 struct CertifyArgs {
@@ -97,7 +99,9 @@ struct CertifyArgs {
     const __nv_bfloat16 *x;
     const float *wsq_part, *bias;  // wsq_part [nparts, E]
     int nparts;
-    int T, H, E, k, TB;
+    int T, H, E, k;
+    int TB;                 // tokens of a block: the tokens of one cluster of CTAs
+    int EB;                 // experts of a CTA's slice: CTA r of a cluster runs the chains of experts r*EB ..
     float eps;
     int32_t *ncand;         // [T] candidates per token
     RouterCand *list;       // [T, E] the candidates of token t in slots t*E .. t*E + ncand[t] - 1, ascending e;
@@ -107,20 +111,44 @@ struct CertifyArgs {
     int32_t *status;
     float *audit_v, *audit_d;  // null, or [T, E]: every tensor-core logit and its bound
     int xrows;              // rows of an x tile (TB rounded up to 8)
-    int erows;              // staged router rows (E rounded up to 8, or to 256 above 256)
+    int erows;              // staged router rows (EB rounded up to 8, or to 256 above 256)
     int ebox;               // rows of one router tile (<= 256)
     int nbx;                // 64-column tiles per chunk
     int stages;             // 1..kCertMaxStages
     int stage_bytes;        // nbx * (xrows + erows) * 128
 };
 
-// Fixed part of the dynamic shared memory: the stage barriers, per-token counts and
-// prefix, squared expert norms, per-warp top-k outputs; the stages follow at a
-// 1024-byte boundary (the 128-byte swizzle repeats every 8 rows of 128 bytes).
+// Fixed part of the dynamic shared memory: the stage barriers, per-token counts,
+// first chains and prefix, expert norms, per-warp top-k outputs; the stages follow at
+// a 1024-byte boundary (the 128-byte swizzle repeats every 8 rows of 128 bytes).
 __host__ __device__ inline size_t cert_fixed_bytes(int E, int k)
 {
-    const size_t words = (size_t)kCertMaxTB + (kCertMaxTB + 1) + E + 8 + (size_t)2 * kCertWarps * k;
+    const size_t words = (size_t)3 * kCertMaxTB + (kCertMaxTB + 1) + E + 8 + (size_t)2 * kCertWarps * k;
     return (kCertMaxStages * 8 + words * 4 + 1023) / 1024 * 1024;
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t n;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+    return n;
+}
+// Every thread of every CTA of the cluster arrives; this CTA's threads wait, and the
+// global and shared writes made before the arrival are visible after the wait.  A
+// cluster of one CTA is a plain CTA barrier.
+__device__ __forceinline__ void cluster_barrier(uint32_t csize)
+{
+    if (csize == 1) {
+        __syncthreads();
+        return;
+    }
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // 16-byte chunk j (0..7) of row r of a 128-byte-swizzled tile.
@@ -129,48 +157,86 @@ __device__ __forceinline__ const uint4 *sw128_chunk(const uint8_t *tile, int r, 
     return reinterpret_cast<const uint4 *>(tile + r * 128 + ((j ^ (r & 7)) << 4));
 }
 
-template <int MAXV>
-__global__ void __launch_bounds__(kCertThreads)
+template <int MAXV, int NT = cert_threads(MAXV)>
+__global__ void __launch_bounds__(NT)
     router_certify_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                           const CertifyArgs a)
 {
     extern __shared__ __align__(128) uint8_t csm[];
+    constexpr int NW = NT / 32;
     const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
     const int E = a.E, H = a.H, k = a.k;
-    const int t0 = blockIdx.x * a.TB;
-    const int tb = min(a.TB, a.T - t0);
+    // the cluster's block of tokens; this CTA's slice of the experts, and its share of
+    // the block's tokens in the per-token phases (tokens r, r + C, ...)
+    const uint32_t C = cluster_nctarank(), rank = cluster_ctarank();
+    const int t0 = (int)(blockIdx.x / C) * a.TB;
+    const int tb = max(0, min(a.TB, a.T - t0));
+    const int eb0 = min(E, (int)rank * a.EB), eb1 = min(E, eb0 + a.EB);
     uint64_t *full = reinterpret_cast<uint64_t *>(csm);        // [kCertMaxStages] staging barriers
-    int *nc = reinterpret_cast<int *>(full + kCertMaxStages);  // [kCertMaxTB]
-    int *cb = nc + kCertMaxTB;                                  // [kCertMaxTB + 1] chain prefix over tokens
-    float *wsq = reinterpret_cast<float *>(cb + kCertMaxTB + 1);  // [E] squared norms of the router columns
-    int *misc = reinterpret_cast<int *>(wsq + E);               // [8]: 1 chains
+    int *nc = reinterpret_cast<int *>(full + kCertMaxStages);  // [kCertMaxTB] candidates of the tokens of this CTA
+    int *clo = nc + kCertMaxTB;                                 // [kCertMaxTB] first candidate in the slice
+    int *cnt = clo + kCertMaxTB;                                // [kCertMaxTB] candidates in the slice
+    int *cb = cnt + kCertMaxTB;                                 // [kCertMaxTB + 1] chain prefix over tokens
+    float *wn = reinterpret_cast<float *>(cb + kCertMaxTB + 1);  // [E] norms of the router columns
+    int *misc = reinterpret_cast<int *>(wn + E);                // [8]: 1 chains
     int *wse = misc + 8;                                        // [warps][k]
     float *wsv = reinterpret_cast<float *>(wse + kCertWarps * k);  // [warps][k]
     // stages at a 1024-byte boundary of the shared address space (the launch adds 1 KB of slack)
     const uint32_t fixed_end = smem_u32(csm) + (uint32_t)cert_fixed_bytes(E, k);
     uint8_t *stage0 = csm + (((fixed_end + 1023u) & ~1023u) - smem_u32(csm));
 
+    // A chunk is nbx 64-column tiles of h; each tile holds the block's x rows and the
+    // router rows of the CTA's experts (router_w^T), loaded by the TMA engine with the
+    // 128-byte swizzle so that eight lanes reading the same 16-byte column of eight
+    // rows hit eight bank groups when the rows differ mod 8.  Chunk g (a running count
+    // over rounds) lives in stage g % stages and completes on full[g % stages].
+    const int S = a.stages, hc = a.nbx * 64, nch = (H + hc - 1) / hc;
+    const int tile_rows = a.xrows + a.erows;
+    auto issue = [&](int ch, uint32_t g) {  // thread 0
+        uint8_t *st = stage0 + (size_t)(g % S) * a.stage_bytes;
+        const int nb = min(a.nbx, (H - ch * hc) / 64);
+        mbar_arrive_expect_tx(&full[g % S], (uint32_t)(nb * tile_rows * 128));
+        for (int b = 0; b < nb; ++b) {
+            const int h = ch * hc + b * 64;
+            uint8_t *tile = st + (size_t)b * tile_rows * 128;
+            tma_load_2d(tile, &tm_x, &full[g % S], h, t0);
+            for (int r = 0; r < a.erows; r += a.ebox)
+                tma_load_2d(tile + (size_t)(a.xrows + r) * 128, &tm_w, &full[g % S], h, eb0 + r);
+        }
+    };
+
     if (tid == 0) {
         for (int s = 0; s < kCertMaxStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
+    __syncthreads();
     pdl_wait();
     pdl_trigger();
-    for (int e = tid; e < E; e += kCertThreads) {
+    // The first round's first chunks depend on nothing below: their copies overlap the
+    // bounds.  Every chain round consumes all nch chunks, and a block has at least k
+    // chains, so each of these copies is waited for before the kernel ends.
+    if (tid == 0)
+        for (int ch = 0; ch < min(S, nch); ++ch) issue(ch, ch);
+    for (int e = tid; e < E; e += NT) {
         float q = 0.0f;
         for (int j = 0; j < a.nparts; ++j) q += a.wsq_part[(size_t)j * E + e];
-        wsq[e] = q;
+        wn[e] = sqrtf(q);
     }
     __syncthreads();
 
-    // ---- a. bounds and candidates, a warp per token
-    for (int tl = warp; tl < tb; tl += kCertWarps) {
+    // ---- a. bounds and candidates, a warp per token; the token's loads (bias, the
+    // logit slices, its x row) are all issued before the first is used
+    for (int tl = (int)rank + (int)C * warp; tl < tb; tl += (int)C * NW) {
         const int t = t0 + tl;
-        float v[MAXV], d[MAXV];
+        float bias[MAXV], v[MAXV];
 #pragma unroll
-        for (int i = 0; i < MAXV; ++i) v[i] = 0.0f;
+        for (int i = 0; i < MAXV; ++i) {
+            const int e = lane + 32 * i;
+            bias[i] = (a.bias && e < E) ? a.bias[e] : 0.0f;
+            v[i] = 0.0f;
+        }
 #pragma unroll
-        for (int q = 0; q < kRouterKSplitMax; ++q) {  // slices summed in order; loads issued together
+        for (int q = 0; q < kRouterKSplitMax; ++q) {  // slices summed in order
             if (q < a.ksplit) {
                 const float *row = a.lt + ((size_t)q * a.T + t) * E;
 #pragma unroll
@@ -196,27 +262,21 @@ __global__ void __launch_bounds__(kCertThreads)
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         const float xn = sqrtf(ss) * 1.001f;
+        // the slices' sum, then the bias
         uint32_t key[MAXV];
         float lo[MAXV];
 #pragma unroll
         for (int i = 0; i < MAXV; ++i) {
             const int e = lane + 32 * i;
-            if (e < E) {
-                float s = v[i];
-                if (a.bias) s += a.bias[e];
-                v[i] = s;
-                d[i] = a.eps * xn * sqrtf(wsq[e]) * 1.001f + fabsf(s) * 4.8e-7f + 1e-30f;
-                lo[i] = v[i] - d[i];
-                key[i] = order_key(lo[i]);
-                if (a.audit_v) {
-                    a.audit_v[(size_t)t * E + e] = v[i];
-                    a.audit_d[(size_t)t * E + e] = d[i];
-                }
-            } else {
-                v[i] = -INFINITY;
-                d[i] = 0.0f;
-                lo[i] = 0.0f;
-                key[i] = 0u;
+            float s = v[i];
+            if (a.bias) s += bias[i];
+            v[i] = e < E ? s : -INFINITY;
+            const float d = e < E ? a.eps * xn * wn[e] * 1.001f + fabsf(s) * 4.8e-7f + 1e-30f : 0.0f;
+            lo[i] = e < E ? s - d : 0.0f;
+            key[i] = e < E ? order_key(lo[i]) : 0u;
+            if (a.audit_v && e < E) {
+                a.audit_v[(size_t)t * E + e] = s;
+                a.audit_d[(size_t)t * E + e] = d;
             }
         }
         // tau: the k-th largest lower bound
@@ -228,9 +288,10 @@ __global__ void __launch_bounds__(kCertThreads)
 #pragma unroll
         for (int i = 0; i < MAXV; ++i) {
             const int e = lane + 32 * i;
-            const bool c = e < E && v[i] + d[i] >= tau;
+            const float d = v[i] - lo[i];
+            const bool c = e < E && v[i] + d >= tau;
             const unsigned m = __ballot_sync(0xffffffffu, c);
-            if (c) out[pos + __popc(m & ((1u << lane) - 1u))] = RouterCand{t, e, v[i], d[i]};
+            if (c) out[pos + __popc(m & ((1u << lane) - 1u))] = RouterCand{t, e, v[i], d};
             pos += __popc(m);
         }
         if (lane == 0) {
@@ -239,83 +300,83 @@ __global__ void __launch_bounds__(kCertThreads)
         }
         __syncwarp();
     }
-    __syncthreads();
+    cluster_barrier(C);  // every token's candidates listed
 
-    // chain prefix over the block's tokens (tb <= 64: two tokens per lane)
+    // this CTA's chains: the candidates of the block's tokens in its expert slice (a
+    // contiguous run of each token's list, which ascends by expert)
+    for (int tl = warp; tl < tb; tl += NW) {
+        const int t = t0 + tl;
+        int lo = 0, n = 0;
+        if (C == 1) {
+            n = nc[tl];
+        } else {
+            const int m = a.ncand[t];
+            const RouterCand *cl = a.list + (size_t)t * E;
+            int hi = 0;
+            for (int p = lane; p - lane < m; p += 32) {
+                const int e = p < m ? cl[p].e : INT_MAX;
+                lo += __popc(__ballot_sync(0xffffffffu, e < eb0));
+                hi += __popc(__ballot_sync(0xffffffffu, e < eb1));
+            }
+            n = hi - lo;
+        }
+        if (lane == 0) {
+            clo[tl] = lo;
+            cnt[tl] = n;
+        }
+    }
+    __syncthreads();
+    // chain prefix over the block's tokens (tb <= 128: four tokens per lane)
     if (warp == 0) {
-        const int c0 = lane < tb ? nc[lane] : 0, c1 = lane + 32 < tb ? nc[lane + 32] : 0;
-        int i0 = c0;
+        int c4[4], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int tl = 4 * lane + i;
+            c4[i] = tl < tb ? cnt[tl] : 0;
+            sum += c4[i];
+        }
+        int inc = sum;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, i0, off);
-            if (lane >= off) i0 += o;
+            const int o = __shfl_up_sync(0xffffffffu, inc, off);
+            if (lane >= off) inc += o;
         }
-        const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
-        int i1 = c1;
+        int run = inc - sum;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, i1, off);
-            if (lane >= off) i1 += o;
+        for (int i = 0; i < 4; ++i) {
+            cb[4 * lane + i] = run;
+            run += c4[i];
         }
-        cb[lane] = i0 - c0;
-        cb[lane + 32] = tot0 + i1 - c1;
         if (lane == 31) {
-            cb[64] = tot0 + i1;
-            misc[1] = tot0 + i1;
+            cb[kCertMaxTB] = inc;
+            misc[1] = inc;
         }
     }
     __syncthreads();
     const int nchain = misc[1];
 
-    // ---- b. exact chains of the candidates.  A chunk is nbx 64-column tiles of
-    // h; each tile holds the block's x rows and every router row (router_w^T, all
-    // E experts), loaded by the TMA engine with the 128-byte swizzle so that eight
-    // lanes reading the same 16-byte column of eight rows hit eight bank groups when
-    // the rows differ mod 8.  Chunk g (a running count over rounds) lives in stage
-    // g % stages and completes on full[g % stages]; one CTA barrier per chunk frees
-    // its stage for the refill.
-    const int S = a.stages, hc = a.nbx * 64, nch = (H + hc - 1) / hc;
-    const int tile_rows = a.xrows + a.erows;
-    auto issue = [&](int ch, uint32_t g) {  // thread 0
-        uint8_t *st = stage0 + (size_t)(g % S) * a.stage_bytes;
-        const int nb = min(a.nbx, (H - ch * hc) / 64);
-        mbar_arrive_expect_tx(&full[g % S], (uint32_t)(nb * tile_rows * 128));
-        for (int b = 0; b < nb; ++b) {
-            const int h = ch * hc + b * 64;
-            uint8_t *tile = st + (size_t)b * tile_rows * 128;
-            tma_load_2d(tile, &tm_x, &full[g % S], h, t0);
-            for (int r = 0; r < a.erows; r += a.ebox)
-                tma_load_2d(tile + (size_t)(a.xrows + r) * 128, &tm_w, &full[g % S], h, r);
-        }
-    };
+    // ---- b. exact chains of the candidates, one per thread and round; one CTA barrier
+    // per chunk frees its stage for the refill
     uint32_t g0 = 0;
     bool failed = false;
-    for (int r0 = 0; r0 < nchain; r0 += kCertThreads * kCertChains) {
-        int ctl[kCertChains], cpos[kCertChains];
-        RouterCand cc[kCertChains];
-        float acc[kCertChains];
-        bool on[kCertChains];
-#pragma unroll
-        for (int i = 0; i < kCertChains; ++i) {
-            const int c = r0 + i * kCertThreads + tid;
-            ctl[i] = 0;
-            cpos[i] = 0;
-            acc[i] = 0.0f;
-            on[i] = c < nchain;
-            cc[i] = RouterCand{0, 0, 0.0f, 0.0f};
-            if (on[i]) {
-                int lo = 0, hi = tb;  // largest tl with cb[tl] <= c
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) / 2;
-                    if (cb[mid] <= c) lo = mid;
-                    else hi = mid;
-                }
-                ctl[i] = lo;
-                cpos[i] = c - cb[lo];
-                cc[i] = a.list[(size_t)(t0 + lo) * E + cpos[i]];
+    for (int r0 = 0; r0 < nchain; r0 += NT) {
+        const int c = r0 + tid;
+        const bool on = c < nchain;
+        int ctl = 0, cpos = 0;
+        RouterCand cc{0, 0, 0.0f, 0.0f};
+        float acc = 0.0f;
+        if (on) {
+            int lo = 0, hi = tb;  // largest tl with cb[tl] <= c
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) / 2;
+                if (cb[mid] <= c) lo = mid;
+                else hi = mid;
             }
+            ctl = lo;
+            cpos = clo[lo] + c - cb[lo];
+            cc = a.list[(size_t)(t0 + lo) * E + cpos];
         }
-        if (tid == 0)
+        if (tid == 0 && r0 > 0)
             for (int ch = 0; ch < min(S, nch); ++ch) issue(ch, g0 + ch);
         for (int ch = 0; ch < nch; ++ch) {
             const uint32_t g = g0 + ch;
@@ -325,69 +386,75 @@ __global__ void __launch_bounds__(kCertThreads)
             }
             const uint8_t *st = stage0 + (size_t)(g % S) * a.stage_bytes;
             const int nb = min(a.nbx, (H - ch * hc) / 64);
-            for (int b = 0; b < nb; ++b) {
-                const uint8_t *tile = st + (size_t)b * tile_rows * 128;
-                if (on[0] && on[1]) {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        acc[0] = chain_step8(*sw128_chunk(tile, ctl[0], j), *sw128_chunk(tile, a.xrows + cc[0].e, j),
-                                             acc[0]);
-                        acc[1] = chain_step8(*sw128_chunk(tile, ctl[1], j), *sw128_chunk(tile, a.xrows + cc[1].e, j),
-                                             acc[1]);
-                    }
-                } else if (on[0]) {
+            if (on) {
+                for (int b = 0; b < nb; ++b) {
+                    const uint8_t *tile = st + (size_t)b * tile_rows * 128;
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        acc[0] = chain_step8(*sw128_chunk(tile, ctl[0], j), *sw128_chunk(tile, a.xrows + cc[0].e, j),
-                                             acc[0]);
+                        acc = chain_step8(*sw128_chunk(tile, ctl, j), *sw128_chunk(tile, a.xrows + cc.e - eb0, j),
+                                          acc);
                 }
             }
             __syncthreads();  // stage g % S consumed by every thread
             if (tid == 0 && ch + S < nch) issue(ch + S, g + S);
         }
         g0 += nch;
-#pragma unroll
-        for (int i = 0; i < kCertChains; ++i)
-            if (on[i]) {
-                float v = acc[i];
-                if (a.bias) v = __fadd_rn(v, a.bias[cc[i].e]);
-                a.list[(size_t)(t0 + ctl[i]) * E + cpos[i]].v = v;
-                if (!(fabsf(v - cc[i].v) <= cc[i].d)) atomicCAS(a.status, 0, MOE_ERR_ROUTER_BOUND);
-            }
+        if (on) {
+            float v = acc;
+            if (a.bias) v = __fadd_rn(v, a.bias[cc.e]);
+            a.list[(size_t)(t0 + ctl) * E + cpos].v = v;
+            if (!(fabsf(v - cc.v) <= cc.d)) atomicCAS(a.status, 0, MOE_ERR_ROUTER_BOUND);
+        }
     }
-    __syncthreads();
+    cluster_barrier(C);  // every exact value written
 
-    // ---- c. top-k (larger exact value first, lower index on ties) and softmax
-    for (int tl = warp; tl < tb; tl += kCertWarps) {
+    // ---- c. top-k (larger exact value first, lower index on ties) and softmax; a
+    // token with at most 32 candidates holds one per lane
+    for (int tl = (int)rank + (int)C * warp; tl < tb; tl += (int)C * NW) {
         const int t = t0 + tl;
         const int n = nc[tl];
         const RouterCand *cl = a.list + (size_t)t * E;
-        uint32_t key[MAXV];
-        float val[MAXV];
-        int ce[MAXV];
-#pragma unroll
-        for (int i = 0; i < MAXV; ++i) {
-            const int p = lane + 32 * i;  // candidates are in ascending expert order
-            RouterCand c{0, 0, 0.0f, 0.0f};
-            if (p < n) c = cl[p];
-            ce[i] = c.e;
-            val[i] = c.v;
-            key[i] = p < n ? order_key(c.v) : 0u;
-        }
         int *se = wse + warp * k;
         float *sv = wsv + warp * k;
-        warp_topk<MAXV>(key, val, k, se, sv);
-        // slot -> expert: the slot order is the expert order, so the tie rule holds
-        for (int j = 0; j < k; ++j) {
-            const int p = se[j];
-            int mine = 0;
+        if (n <= 32) {
+            RouterCand c{0, 0, 0.0f, 0.0f};
+            if (lane < n) c = cl[lane];
+            uint32_t key1[1] = {lane < n ? order_key(c.v) : 0u};
+            const float val1[1] = {c.v};
+            warp_topk<1>(key1, val1, k, se, sv);
+            for (int j = 0; j < k; ++j) {
+                const int e = __shfl_sync(0xffffffffu, c.e, se[j] & 31);
+                if (lane == 0) {
+                    a.idx[(size_t)t * k + j] = e;
+                    a.ex[(size_t)t * E + e] = sv[j];
+                }
+            }
+        } else {
+            uint32_t key[MAXV];
+            float val[MAXV];
+            int ce[MAXV];
 #pragma unroll
-            for (int i = 0; i < MAXV; ++i)
-                if (i == (p >> 5)) mine = ce[i];
-            const int e = __shfl_sync(0xffffffffu, mine, p & 31);
-            if (lane == 0) {
-                a.idx[(size_t)t * k + j] = e;
-                a.ex[(size_t)t * E + e] = sv[j];
+            for (int i = 0; i < MAXV; ++i) {
+                const int p = lane + 32 * i;  // candidates are in ascending expert order
+                RouterCand c{0, 0, 0.0f, 0.0f};
+                if (p < n) c = cl[p];
+                ce[i] = c.e;
+                val[i] = c.v;
+                key[i] = p < n ? order_key(c.v) : 0u;
+            }
+            warp_topk<MAXV>(key, val, k, se, sv);
+            // slot -> expert: the slot order is the expert order, so the tie rule holds
+            for (int j = 0; j < k; ++j) {
+                const int p = se[j];
+                int mine = 0;
+#pragma unroll
+                for (int i = 0; i < MAXV; ++i)
+                    if (i == (p >> 5)) mine = ce[i];
+                const int e = __shfl_sync(0xffffffffu, mine, p & 31);
+                if (lane == 0) {
+                    a.idx[(size_t)t * k + j] = e;
+                    a.ex[(size_t)t * E + e] = sv[j];
+                }
             }
         }
         const float m = sv[0];
@@ -400,14 +467,120 @@ __global__ void __launch_bounds__(kCertThreads)
     }
 }
 
+// Launch with C CTAs per cluster (the expert slices of one token block) and
+// programmatic stream serialisation.
 template <int MAXV>
-cudaError_t launch_certify(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const CertifyArgs &a, int grid,
+cudaError_t launch_certify(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const CertifyArgs &a, int grid, int C,
                            cudaStream_t st)
 {
     auto kern = router_certify_kernel<MAXV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kCertSmem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(grid), dim3(kCertThreads), kCertSmem, st, tm_x, tm_w, a);
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)C;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(cert_threads(MAXV));
+    cfg.dynamicSmemBytes = kCertSmem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, a);
+}
+
+// How many clusters of C certify CTAs can be resident at once (0 if none, or if the
+// query fails); C = 1 is one CTA per SM.  Queried once per (kernel, C).
+template <int MAXV>
+int cert_clusters(int C)
+{
+    static std::atomic<int> cached[4] = {-1, -1, -1, -1};
+    const int slot = C == 1 ? 0 : C == 2 ? 1 : C == 4 ? 2 : 3;
+    int v = cached[slot].load();
+    if (v >= 0) return v;
+    if (C == 1) {
+        v = num_sms();
+    } else {
+        auto kern = router_certify_kernel<MAXV>;
+        v = 0;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kCertSmem) == cudaSuccess) {
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)C;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3((unsigned)C);
+            cfg.blockDim = dim3(cert_threads(MAXV));
+            cfg.dynamicSmemBytes = kCertSmem;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess) v = n;
+            else (void)cudaGetLastError();
+        }
+    }
+    cached[slot].store(v);
+    return v;
+}
+
+// The certify launch for T tokens: tokens in blocks of TB, one cluster of C CTAs per
+// block, CTA r of a cluster taking the chains of experts r*EB .. (r+1)*EB - 1.  C is
+// the cluster size (1, 2, 4 or 8 that fit) whose CTAs stage the fewest rows per chunk
+// (the block's x rows plus the slice's router rows): the chain phase is bound by
+// staging, and the per-token phases take T / (resident CTAs) tokens per CTA either way.
+template <int MAXV>
+cudaError_t certify_shape_and_launch(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, CertifyArgs a, int T, int E,
+                                     int k, cudaStream_t st)
+{
+    int bestC = 0, bestTB = 0, bestCost = INT_MAX;
+    for (int C : {1, 2, 4, 8}) {
+        if (C > 1 && E < 16 * C) break;  // slices of fewer than 16 experts stage little less
+        const int clusters = cert_clusters<MAXV>(C);
+        if (clusters < 1) continue;
+        const int TB = (T + clusters - 1) / clusters;
+        if (TB > kCertMaxTB) continue;
+        const int EB = (E + C - 1) / C;
+        const int cost = (TB + 7) / 8 * 8 + (EB <= 256 ? (EB + 7) / 8 * 8 : (EB + 255) / 256 * 256);
+        if (cost < bestCost) {
+            bestCost = cost;
+            bestC = C;
+            bestTB = TB;
+        }
+    }
+    if (bestC == 0) {  // more tokens than the resident CTAs take in blocks of kCertMaxTB
+        bestC = 1;
+        bestTB = kCertMaxTB;
+    }
+    const int C = bestC, TB = bestTB, EB = (E + C - 1) / C;
+    const int xrows = (TB + 7) / 8 * 8;
+    const int erows = EB <= 256 ? (EB + 7) / 8 * 8 : (EB + 255) / 256 * 256;
+    const int ebox = erows < 256 ? erows : 256;
+    const size_t room = (size_t)kCertSmem - 1024 - cert_fixed_bytes(E, k);
+    int nbx = 4, stages = 0;
+    for (; nbx >= 1; nbx /= 2) {  // the widest chunk that still leaves two stages
+        stages = (int)(room / ((size_t)nbx * (xrows + erows) * 128));
+        if (stages >= 2 || nbx == 1) break;
+    }
+    if (stages > kCertMaxStages) stages = kCertMaxStages;
+    if (stages < 1) return cudaErrorInvalidValue;
+    CUtensorMap tm_x, tm_w;
+    if (!encode_sw128_2d_bf16(&tm_x, x, T, a.H, xrows) || !encode_sw128_2d_bf16(&tm_w, wrt, E, a.H, ebox))
+        return cudaErrorInvalidValue;
+    a.TB = TB;
+    a.EB = EB;
+    a.xrows = xrows;
+    a.erows = erows;
+    a.ebox = ebox;
+    a.nbx = nbx;
+    a.stages = stages;
+    a.stage_bytes = nbx * (xrows + erows) * 128;
+    const int grid = (T + TB - 1) / TB * C;
+    return launch_certify<MAXV>(tm_x, tm_w, a, grid, C, st);
 }
 
 }  // namespace
@@ -425,33 +598,15 @@ cudaError_t launch_route_certified(const moe_dims_t &d, const __nv_bfloat16 *x, 
     if ((e = tc_router_logits(x, rs.wrt, T, H, E, logits, hdr, &ks, st)) != cudaSuccess) return e;
     const float u = 5.9604644775390625e-08f;  // 2^-24
     const float eps = ((float)H * u + 256.0f * u + (float)(H / 64 + ks) * u) * 1.01f;
-    int tb = (T + num_sms() - 1) / num_sms();
-    tb = tb < 1 ? 1 : tb > kCertMaxTB ? kCertMaxTB : tb;
-    const int xrows = (tb + 7) / 8 * 8;
-    const int erows = E <= 256 ? (E + 7) / 8 * 8 : (E + 255) / 256 * 256;
-    const int ebox = erows < 256 ? erows : 256;
-    const size_t room = (size_t)kCertSmem - 1024 - cert_fixed_bytes(E, k);
-    int nbx = 4, stages = 0;
-    for (; nbx >= 1; nbx /= 2) {  // the widest chunk that still leaves two stages
-        stages = (int)(room / ((size_t)nbx * (xrows + erows) * 128));
-        if (stages >= 2 || nbx == 1) break;
-    }
-    if (stages > kCertMaxStages) stages = kCertMaxStages;
-    if (stages < 1) return cudaErrorInvalidValue;
-    CUtensorMap tm_x, tm_w;
-    if (!encode_sw128_2d_bf16(&tm_x, x, T, H, xrows) || !encode_sw128_2d_bf16(&tm_w, rs.wrt, E, H, ebox))
-        return cudaErrorInvalidValue;
-    CertifyArgs a{logits, logits, ks, x, rs.wsq, bias, nparts, T, H, E, k, tb, eps, rs.ncand, rs.list,
-                  idx, gate, &hdr->status, rs.audit_v, rs.audit_d, xrows, erows, ebox, nbx, stages,
-                  nbx * (xrows + erows) * 128};
-    const int grid = (T + tb - 1) / tb;
+    CertifyArgs a{logits, logits, ks, x, rs.wsq, bias, nparts, T, H, E, k, 0, 0, eps, rs.ncand, rs.list,
+                  idx, gate, &hdr->status, rs.audit_v, rs.audit_d, 0, 0, 0, 0, 0, 0};
     const int vpl = (E + 31) / 32;
-    if (vpl <= 1) return launch_certify<1>(tm_x, tm_w, a, grid, st);
-    if (vpl <= 2) return launch_certify<2>(tm_x, tm_w, a, grid, st);
-    if (vpl <= 4) return launch_certify<4>(tm_x, tm_w, a, grid, st);
-    if (vpl <= 8) return launch_certify<8>(tm_x, tm_w, a, grid, st);
-    if (vpl <= 16) return launch_certify<16>(tm_x, tm_w, a, grid, st);
-    return launch_certify<32>(tm_x, tm_w, a, grid, st);
+    if (vpl <= 1) return certify_shape_and_launch<1>(x, rs.wrt, a, T, E, k, st);
+    if (vpl <= 2) return certify_shape_and_launch<2>(x, rs.wrt, a, T, E, k, st);
+    if (vpl <= 4) return certify_shape_and_launch<4>(x, rs.wrt, a, T, E, k, st);
+    if (vpl <= 8) return certify_shape_and_launch<8>(x, rs.wrt, a, T, E, k, st);
+    if (vpl <= 16) return certify_shape_and_launch<16>(x, rs.wrt, a, T, E, k, st);
+    return certify_shape_and_launch<32>(x, rs.wrt, a, T, E, k, st);
 }
 
 }  // namespace moe
