@@ -176,6 +176,7 @@ STAGE_SOURCES = {
     "gemm_down": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "fp8.cu", "fp8_common.cuh", "mx.cu", "combine.cuh",
                   "sm100_ptx.cuh", "moe_internal.h"],
     "combine": ["combine.cu", "combine.cuh"],
+    "gemm_layer": ["grouped_gemm.cu", "grouped_gemm_2cta.cu", "combine.cuh", "sm100_ptx.cuh", "moe_internal.h"],
 }
 
 
