@@ -357,9 +357,11 @@ __global__ void __launch_bounds__(NT)
 
     // ---- b. exact chains of the candidates, one per thread and round; one CTA barrier
     // per chunk frees its stage for the refill
+    // (at least one round, so that the chunks issued before the bounds are read even by
+    // a CTA whose expert slice holds no candidate)
     uint32_t g0 = 0;
     bool failed = false;
-    for (int r0 = 0; r0 < nchain; r0 += NT) {
+    for (int r0 = 0; r0 == 0 || r0 < nchain; r0 += NT) {
         const int c = r0 + tid;
         const bool on = c < nchain;
         int ctl = 0, cpos = 0;

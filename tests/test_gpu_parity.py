@@ -82,6 +82,27 @@ def test_one_hot_expert_takes_everything():
     compare_out(out, ref, "hot")
 
 
+def test_router_expert_slice_without_candidates():
+    # The certified router (T > 32) splits the experts of a token block over a
+    # cluster of CTAs; a bias that routes every token to experts 0..3 leaves the upper
+    # slices without a single candidate.  Those CTAs still read and release every
+    # staged chunk, and the routing is the oracle's.
+    cfg = CONFIGS["tiny"].replace(name="slice", T=256, H=256, E=64, I=128, top_k=4, seed=28)
+    g, c = device_inputs(cfg)
+    bias = torch.zeros(cfg.E, dtype=torch.float32)
+    bias[:4] = 1000.0
+    g["bias"], c["bias"] = bias.cuda(), bias
+    idx_ref, gate_ref = oracle.route(c["x"], c["router_w"], bias, cfg.top_k)
+    assert np.all(np.sort(idx_ref, axis=1) == np.arange(4))
+    ws = api.workspace(cfg.T, cfg.H, cfg.I, cfg.E, cfg.top_k, "cuda")
+    out = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k, ws=ws)
+    assert api.moe_get_device_status(ws) == api.MOE_OK
+    ref = oracle.combine_ffn(c["x"], idx_ref, gate_ref, c["w_gate"], c["w_up"], c["w_down"])
+    compare_out(out, ref, "slice")
+    idx, w = api.moe_route(g["x"], g["router_w"], g["bias"], cfg.top_k)
+    compare_routing(idx, w, idx_ref, gate_ref, "slice")
+
+
 def test_group_sizes_at_tile_edges():
     # Groups of exactly 128 rows (one full tile), 129 rows (a full tile plus one row)
     # and 5 rows.  Router rows 0 and 1 give logit(e) = x0*e - x1*e^2, which with
