@@ -31,12 +31,19 @@ namespace moe {
 namespace {
 
 constexpr int HALF = kTileRows;        // rows per CTA of a pair tile
-constexpr int BK2 = 64;
+constexpr int BK2 = 64;                // one TMA box: 64 bf16 = one 128-byte swizzle row
+constexpr int KW2 = 2;                 // 64-column boxes per stage
+constexpr int BKS2 = BK2 * KW2;        // K of a stage: 128
 constexpr int BN2 = 256;               // MMA N (128 B rows per CTA)
-constexpr int ST2 = 6;
+// Three stages of 64 KB rather than six of 32 KB: a stage's loads complete on one
+// barrier, and the SM's TMA throughput from L2 grows with the bytes behind each
+// barrier (about 71 GB/s per SM with two 16 KB boxes per stage, 109 GB/s with four).
+constexpr int ST2 = 3;
 constexpr int RING2 = 4;
-constexpr int A2_BYTES = HALF * BK2 * 2;   // 16 KB
-constexpr int B2_BYTES = 128 * BK2 * 2;    // 16 KB
+constexpr int A2_SUB = HALF * BK2 * 2;     // 16 KB: one box of A rows
+constexpr int B2_SUB = 128 * BK2 * 2;      // 16 KB: one box of B rows
+constexpr int A2_BYTES = A2_SUB * KW2;     // 32 KB
+constexpr int B2_BYTES = B2_SUB * KW2;     // 32 KB
 constexpr int THREADS2 = 192;
 constexpr uint32_t TMEM_COLS2 = 512;
 
@@ -218,8 +225,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_rank();
     const int NP1 = MODE == 3 ? g.N2 : g.N, KP1 = MODE == 3 ? g.K2 : g.K;  // N and K of the down items
-    const int nt0 = (g.N + BNO0 - 1) / BNO0, kb0 = g.K / BK2;
-    const int nt1 = (NP1 + BNO1 - 1) / BNO1, kb1 = KP1 / BK2;
+    const int nt0 = (g.N + BNO0 - 1) / BNO0, kb0 = (g.K + BKS2 - 1) / BKS2;
+    const int nt1 = (NP1 + BNO1 - 1) / BNO1, kb1 = (KP1 + BKS2 - 1) / BKS2;
+    // 64-column boxes of stage kb of a K range of Kd columns (a multiple of 64)
+    auto boxes_of = [](int kb, int Kd) { return min(KW2, (Kd - kb * BKS2) / BK2); };
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < ST2; ++s) {
@@ -343,15 +352,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
             if (g4_lane && !held) load_tokens();
             const uint32_t a_bytes = rows <= 0 ? 0u
                                    : g4        ? (uint32_t)((rows + 3) / 4) * 512u
-                                               : (uint32_t)(a_box_rows(ab) * BK2 * 2);
+                                               : (uint32_t)(a_box_rows(ab) * BK2 * 2);  // per 64-column box
             // B rows of this CTA: gate (CTA 0) or up (CTA 1) rows nt*128.. ; down: output columns
             const int nrow = !p1 ? nt * BNO0 : nt * BNO1 + (int)rank * 128;
             const CUtensorMap *bmap = !p1 ? (rank == 1 ? (tr.s >= 0 ? &sm.b1 : &tmB1) : (tr.s >= 0 ? &sm.b0 : &tmB0))
                                     : MODE == 3 ? (tr.s >= 0 ? &lm.wd_sh : &lm.wd)
                                                 : (tr.s >= 0 ? &sm.b0 : &tmB0);
             const bool b_in = nrow < (p1 ? NP1 : g.N);  // a half entirely past N loads nothing (masked columns)
-            const uint32_t b_bytes = b_in ? (uint32_t)B2_BYTES : 0u;
+            const uint32_t b_bytes = b_in ? (uint32_t)B2_SUB : 0u;  // per 64-column box
             const int num_kb = p1 ? kb1 : kb0;
+            const int Kd = p1 ? KP1 : g.K;
             if (MODE == 3 && p1) {
                 // the h rows of pair tile mt: wait until every gate/up item of mt published
                 // them (4 epilogue warps in each of the 2 CTAs), then order those
@@ -364,41 +374,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
             }
             for (int kb = 0; kb < num_kb; ++kb) {
                 const uint32_t fb = peer_addr(&S->full[stage], 0);
+                const int nbx = boxes_of(kb, Kd);
                 if (lane == 0) {
                     okl = wait2(&S->empty[stage], phase ^ 1, g.wait_ns);
                     if (okl) {
+                        const uint32_t tx = (a_bytes + b_bytes) * (uint32_t)nbx;
                         if (rank == 0)
-                            mbar_arrive_expect_tx(&S->full[stage], a_bytes + b_bytes);
+                            mbar_arrive_expect_tx(&S->full[stage], tx);
                         else
-                            arrive_expect_tx_remote(fb, a_bytes + b_bytes);
-                        if (rows > 0 && !held && !g4)
-                            tma_load_2d_pair(sA + stage * A2_BYTES, amap, fb, kb * BK2, arow0);
-                        if (b_in) {
-                            if (tr.s < 0)
-                                tma_load_3d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, nrow, expert);
-                            else if (!p1)  // shared slice s: rows s*I + nrow.. of the shared gate / up
-                                tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, kb * BK2, tr.s * g.N + nrow);
-                            else  // shared down: columns s*I + kb*BK2..
-                                tma_load_2d_pair(sB + stage * B2_BYTES, bmap, fb, tr.s * KP1 + kb * BK2, nrow);
+                            arrive_expect_tx_remote(fb, tx);
+                        for (int x = 0; x < nbx; ++x) {
+                            const int kx = kb * BKS2 + x * BK2;
+                            if (rows > 0 && !held && !g4)
+                                tma_load_2d_pair(sA + stage * A2_BYTES + x * A2_SUB, amap, fb, kx, arow0);
+                            if (b_in) {
+                                uint8_t *b_dst = sB + stage * B2_BYTES + x * B2_SUB;
+                                if (tr.s < 0)
+                                    tma_load_3d_pair(b_dst, bmap, fb, kx, nrow, expert);
+                                else if (!p1)  // shared slice s: rows s*I + nrow.. of the shared gate / up
+                                    tma_load_2d_pair(b_dst, bmap, fb, kx, tr.s * g.N + nrow);
+                                else  // shared down: columns s*I + kx..
+                                    tma_load_2d_pair(b_dst, bmap, fb, tr.s * KP1 + kx, nrow);
+                            }
                         }
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
                 if (g4_lane && !held)
-                    tma_gather4_pair(sA + stage * A2_BYTES + lane * 512, &sm.xg, fb, kb * BK2, tok[0], tok[1], tok[2],
-                                     tok[3]);
+                    for (int x = 0; x < nbx; ++x)
+                        tma_gather4_pair(sA + stage * A2_BYTES + x * A2_SUB + lane * 512, &sm.xg, fb,
+                                         kb * BKS2 + x * BK2, tok[0], tok[1], tok[2], tok[3]);
                 if (++stage == ST2) { stage = 0; phase ^= 1; }
                 if (held && kb + 1 == min(ST2, num_kb)) {  // first item: stage j holds K block j
                     pdl_wait();
                     held = false;
                     if (g4_lane) load_tokens();
-                    for (int j = 0; j <= kb; ++j) {
-                        if (g4_lane)
-                            tma_gather4_pair(sA + j * A2_BYTES + lane * 512, &sm.xg, peer_addr(&S->full[j], 0),
-                                             j * BK2, tok[0], tok[1], tok[2], tok[3]);
-                        else if (!g4 && lane == 0 && rows > 0)
-                            tma_load_2d_pair(sA + j * A2_BYTES, amap, peer_addr(&S->full[j], 0), j * BK2, arow0);
-                    }
+                    for (int j = 0; j <= kb; ++j)
+                        for (int x = 0; x < boxes_of(j, Kd); ++x) {
+                            const int kx = j * BKS2 + x * BK2;
+                            if (g4_lane)
+                                tma_gather4_pair(sA + j * A2_BYTES + x * A2_SUB + lane * 512, &sm.xg,
+                                                 peer_addr(&S->full[j], 0), kx, tok[0], tok[1], tok[2], tok[3]);
+                            else if (!g4 && lane == 0 && rows > 0)
+                                tma_load_2d_pair(sA + j * A2_BYTES + x * A2_SUB, amap, peer_addr(&S->full[j], 0), kx,
+                                                 arow0);
+                        }
                 }
             }
             if (!ok) break;
@@ -419,7 +439,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                 if (++rs == RING2) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
                 int mt_, nt_;
-                const int num_kb = pos_of(item, mt_, nt_) ? kb1 : kb0;
+                const bool down = pos_of(item, mt_, nt_);
+                const int num_kb = down ? kb1 : kb0, Kd = down ? KP1 : g.K;
                 if (!wait2(&S->acce[acc], aphase ^ 1, g.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + static_cast<uint32_t>(acc * BN2);
@@ -428,10 +449,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sA + stage * A2_BYTES);
                     const uint32_t b0 = smem_u32(sB + stage * B2_BYTES);
+                    const int nbx = boxes_of(kb, Kd);
+                    for (int x = 0; x < nbx; ++x)
 #pragma unroll
-                    for (int k = 0; k < BK2 / 16; ++k)
-                        mma_bf16_pair(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), IDESC,
-                                      (kb | k) != 0);
+                        for (int k = 0; k < BK2 / 16; ++k)
+                            mma_bf16_pair(d, sw128_kmajor_desc(a0 + x * A2_SUB + k * 32),
+                                          sw128_kmajor_desc(b0 + x * B2_SUB + k * 32), IDESC, (kb | x | k) != 0);
                     mma_commit_pair(&S->empty[stage]);
                     if (++stage == ST2) { stage = 0; phase ^= 1; }
                 }
