@@ -282,6 +282,20 @@ bool encode_sw128_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint6
     return encode_2d(m, base, rows, cols, box_rows);
 }
 
+bool encode_sw128_chunked_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                               uint32_t box_chunks)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f || cols % 64) return false;
+    const cuuint64_t dims[3] = {64, rows, cols / 64};
+    const cuuint64_t strides[2] = {cols * 2, 128};  // a row, a 64-column chunk
+    const cuuint32_t box[3] = {64, box_rows, box_chunks};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // A-operand tensor maps with boxes of 16/32/64/128 rows (bf16 64 columns, or 128
 // e4m3 bytes), 128-byte swizzle.
 bool encode_a_maps(AMaps *m, const void *base, uint64_t rows, uint64_t cols, bool u8)

@@ -402,6 +402,11 @@ int num_sms();
 // Tensor map of a row-major bf16 matrix [rows, cols], box_rows x 64 tiles with the
 // 128-byte swizzle (16-byte chunk c of tile row r stored at chunk c ^ (r % 8)).
 bool encode_sw128_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// The same matrix seen as [cols / 64][rows][64]: one box brings box_chunks consecutive
+// 64-column chunks of box_rows rows, stored chunk after chunk (each chunk's rows as the
+// 2-D map's box would store them).
+bool encode_sw128_chunked_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                               uint32_t box_chunks);
 // Tensor map of a row-major bf16 matrix [rows, cols], box_rows x box_cols tiles,
 // no swizzle (box_cols * 2 a multiple of 16).
 bool encode_plain_2d_bf16(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,

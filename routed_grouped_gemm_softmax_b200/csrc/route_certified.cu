@@ -185,24 +185,22 @@ __global__ void __launch_bounds__(NT)
     const uint32_t fixed_end = smem_u32(csm) + (uint32_t)cert_fixed_bytes(E, k);
     uint8_t *stage0 = csm + (((fixed_end + 1023u) & ~1023u) - smem_u32(csm));
 
-    // A chunk is nbx 64-column tiles of h; each tile holds the block's x rows and the
-    // router rows of the CTA's experts (router_w^T), loaded by the TMA engine with the
+    // A chunk is nbx 64-column blocks of h (nbx divides H / 64): the block's x rows of
+    // each, then the router rows of the CTA's experts (router_w^T) of each, stored
+    // [nbx][xrows][128 B] and [erows / ebox][nbx][ebox][128 B], every block with the
     // 128-byte swizzle so that eight lanes reading the same 16-byte column of eight
-    // rows hit eight bank groups when the rows differ mod 8.  Chunk g (a running count
+    // rows hit eight bank groups when the rows differ mod 8.  One TMA box brings all nbx
+    // blocks of the x rows and one each ebox router rows: the SM's TMA throughput
+    // grows with the bytes behind each box and each barrier.  Chunk g (a running count
     // over rounds) lives in stage g % stages and completes on full[g % stages].
-    const int S = a.stages, hc = a.nbx * 64, nch = (H + hc - 1) / hc;
-    const int tile_rows = a.xrows + a.erows;
+    const int S = a.stages, hc = a.nbx * 64, nch = H / hc;
+    const size_t x_bytes = (size_t)a.nbx * a.xrows * 128;
     auto issue = [&](int ch, uint32_t g) {  // thread 0
         uint8_t *st = stage0 + (size_t)(g % S) * a.stage_bytes;
-        const int nb = min(a.nbx, (H - ch * hc) / 64);
-        mbar_arrive_expect_tx(&full[g % S], (uint32_t)(nb * tile_rows * 128));
-        for (int b = 0; b < nb; ++b) {
-            const int h = ch * hc + b * 64;
-            uint8_t *tile = st + (size_t)b * tile_rows * 128;
-            tma_load_2d(tile, &tm_x, &full[g % S], h, t0);
-            for (int r = 0; r < a.erows; r += a.ebox)
-                tma_load_2d(tile + (size_t)(a.xrows + r) * 128, &tm_w, &full[g % S], h, eb0 + r);
-        }
+        mbar_arrive_expect_tx(&full[g % S], (uint32_t)a.stage_bytes);
+        tma_load_3d(st, &tm_x, &full[g % S], 0, t0, ch * a.nbx);
+        for (int r = 0; r < a.erows; r += a.ebox)
+            tma_load_3d(st + x_bytes + (size_t)r * a.nbx * 128, &tm_w, &full[g % S], 0, eb0 + r, ch * a.nbx);
     };
 
     if (tid == 0) {
@@ -387,14 +385,16 @@ __global__ void __launch_bounds__(NT)
                 atomicCAS(a.status, 0, MOE_ERR_TIMEOUT);
             }
             const uint8_t *st = stage0 + (size_t)(g % S) * a.stage_bytes;
-            const int nb = min(a.nbx, (H - ch * hc) / 64);
             if (on) {
-                for (int b = 0; b < nb; ++b) {
-                    const uint8_t *tile = st + (size_t)b * tile_rows * 128;
+                // the chain's router row: block (el / ebox) of the router part, row el % ebox
+                const int el = cc.e - eb0;
+                const uint8_t *wr0 = st + x_bytes + (size_t)(el / a.ebox) * a.nbx * a.ebox * 128;
+                for (int b = 0; b < a.nbx; ++b) {
+                    const uint8_t *xt = st + (size_t)b * a.xrows * 128;
+                    const uint8_t *wt = wr0 + (size_t)b * a.ebox * 128;
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        acc = chain_step8(*sw128_chunk(tile, ctl, j), *sw128_chunk(tile, a.xrows + cc.e - eb0, j),
-                                          acc);
+                        acc = chain_step8(*sw128_chunk(xt, ctl, j), *sw128_chunk(wt, el % a.ebox, j), acc);
                 }
             }
             __syncthreads();  // stage g % S consumed by every thread
@@ -564,14 +564,16 @@ cudaError_t certify_shape_and_launch(const __nv_bfloat16 *x, const __nv_bfloat16
     const int ebox = erows < 256 ? erows : 256;
     const size_t room = (size_t)kCertSmem - 1024 - cert_fixed_bytes(E, k);
     int nbx = 4, stages = 0;
-    for (; nbx >= 1; nbx /= 2) {  // the widest chunk that still leaves two stages
+    for (; nbx >= 1; nbx /= 2) {  // the widest chunk dividing H that still leaves two stages
+        if ((a.H / 64) % nbx) continue;
         stages = (int)(room / ((size_t)nbx * (xrows + erows) * 128));
         if (stages >= 2 || nbx == 1) break;
     }
     if (stages > kCertMaxStages) stages = kCertMaxStages;
     if (stages < 1) return cudaErrorInvalidValue;
     CUtensorMap tm_x, tm_w;
-    if (!encode_sw128_2d_bf16(&tm_x, x, T, a.H, xrows) || !encode_sw128_2d_bf16(&tm_w, wrt, E, a.H, ebox))
+    if (!encode_sw128_chunked_bf16(&tm_x, x, T, a.H, xrows, nbx) ||
+        !encode_sw128_chunked_bf16(&tm_w, wrt, E, a.H, ebox, nbx))
         return cudaErrorInvalidValue;
     a.TB = TB;
     a.EB = EB;
