@@ -50,12 +50,19 @@ namespace moe {
 namespace {
 
 constexpr int BM = kTileRows;  // 128 rows per tile
-constexpr int BK = 64;         // 64 bf16 = one 128-byte swizzle row
-constexpr int BN = 256;        // MMA N
-constexpr int STAGES = 4;
+constexpr int BK = 64;         // a K chunk: 64 bf16 = one 128-byte swizzle row
+constexpr int KC = 2;          // K chunks per stage
+constexpr int BKS = BK * KC;   // K of a stage: 128
+constexpr int BN = 256;        // output columns per item (gate/up: 128 + 128)
+// Two stages of 128 K columns (96 KB) rather than four of 64: each weight box then
+// brings both chunks of its rows, 256 contiguous bytes a row, which DRAM streams about
+// a third faster than 128-byte row pieces, and fewer bytes wait on more barriers.
+constexpr int STAGES = 2;
 constexpr int RING = 4;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int A_SUB = BM * BK * 2;     // 16 KB: one chunk of A rows
+constexpr int B_SUB = BN * BK * 2;     // 32 KB: one chunk of B rows
+constexpr int A_BYTES = A_SUB * KC;    // 32 KB
+constexpr int B_BYTES = B_SUB * KC;    // 64 KB
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;   // two 128 x 256 fp32 accumulators
 
@@ -127,9 +134,12 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     // n-tiles and K blocks of the gate/up items (modes 0, 3) and of the down / dense items
-    const int nt0 = (g.N + BNO0 - 1) / BNO0, kb0 = g.K / BK;
+    const int nt0 = (g.N + BNO0 - 1) / BNO0, kb0 = (g.K + BKS - 1) / BKS;
     const int nt1 = MODE == 3 ? (g.N2 + BNO1 - 1) / BNO1 : (g.N + BNO1 - 1) / BNO1;
-    const int kb1 = MODE == 3 ? g.K2 / BK : g.K / BK;
+    const int K1 = MODE == 3 ? g.K2 : g.K;  // K of the down (or dense) items
+    const int kb1 = (K1 + BKS - 1) / BKS;
+    // K chunks of stage kb of a K range of Kd columns (a multiple of 64)
+    auto chunks_of = [](int kb, int Kd) { return min(KC, (Kd - kb * BKS) / BK); };
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -260,9 +270,12 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                 }
             };
             if (g4_lane && !held) load_tokens();
+            // per K chunk; the weight boxes bring all KC chunks of their rows (a chunk past
+            // the K range reads zeros and is not multiplied)
             const uint32_t a_bytes = g4 ? (uint32_t)((tr.rows + 3) / 4) * 512u : (uint32_t)(a_box_rows(ab) * BK * 2);
             const int n0 = ip.nt * (p1 ? BNO1 : BNO0);
             const int num_kb = p1 ? kb1 : kb0;
+            const int Kd = p1 ? K1 : g.K;
             if (MODE == 3 && p1) {
                 // the down item reads h rows of m-tile mt: wait until every gate/up item of
                 // mt has published them, then order those generic-proxy writes before the
@@ -274,48 +287,54 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                 if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
             }
             for (int kb = 0; kb < num_kb; ++kb) {
+                const int nc = chunks_of(kb, Kd);
                 if (lane == 0) {
                     okl = mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns);
                     if (okl) {
-                        mbar_arrive_expect_tx(&S->full[stage], a_bytes + B_BYTES);
+                        mbar_arrive_expect_tx(&S->full[stage], a_bytes * nc + B_BYTES);
                         armed |= 1u << stage;
                         armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                         uint8_t *b_dst = sB + stage * B_BYTES;
-                        if (!held && !g4) tma_load_2d(sA + stage * A_BYTES, amap, &S->full[stage], kb * BK, arow0);
-                        if (!p1) {  // gate / up rows n0.. of the expert (or of shared slice s)
+                        const int z = kb * KC;  // first K chunk of the stage
+                        if (!held && !g4)
+                            for (int c = 0; c < nc; ++c)
+                                tma_load_2d(sA + stage * A_BYTES + c * A_SUB, amap, &S->full[stage], (z + c) * BK, arow0);
+                        if (!p1) {  // gate / up rows n0.. of the expert (or of shared slice s): [KC][128] each
                             if (tr.s < 0) {
-                                tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * BK, n0, expert);
-                                tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * BK, n0, expert);
+                                tma_load_4d(b_dst, &tmB0, &S->full[stage], 0, n0, z, expert);
+                                tma_load_4d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], 0, n0, z, expert);
                             } else {
-                                tma_load_2d(b_dst, &sm.b0, &S->full[stage], kb * BK, tr.s * g.N + n0);
-                                tma_load_2d(b_dst + B_BYTES / 2, &sm.b1, &S->full[stage], kb * BK, tr.s * g.N + n0);
+                                tma_load_3d(b_dst, &sm.b0, &S->full[stage], 0, tr.s * g.N + n0, z);
+                                tma_load_3d(b_dst + B_BYTES / 2, &sm.b1, &S->full[stage], 0, tr.s * g.N + n0, z);
                             }
-                        } else {  // down (or dense) rows n0..: the expert's, or columns s*I.. of the shared down
+                        } else {  // down rows n0..: the expert's, or chunks of columns s*I.. of the shared down: [KC][256]
                             const CUtensorMap *bm = MODE == 3 ? &lm.wd : &tmB0;
                             const CUtensorMap *bs = MODE == 3 ? &lm.wd_sh : &sm.b0;
                             if (tr.s < 0)
-                                tma_load_3d(b_dst, bm, &S->full[stage], kb * BK, n0, expert);
+                                tma_load_4d(b_dst, bm, &S->full[stage], 0, n0, z, expert);
                             else
-                                tma_load_2d(b_dst, bs, &S->full[stage], tr.s * (MODE == 3 ? g.K2 : g.K) + kb * BK, n0);
+                                tma_load_3d(b_dst, bs, &S->full[stage], 0, n0, tr.s * (K1 / BK) + z);
                         }
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, okl, 0)) { ok = false; break; }
                 if (g4_lane && !held)
-                    tma_gather4(sA + stage * A_BYTES + lane * 512, &sm.xg, &S->full[stage], kb * BK, tok[0], tok[1],
-                                tok[2], tok[3]);
+                    for (int c = 0; c < nc; ++c)
+                        tma_gather4(sA + stage * A_BYTES + c * A_SUB + lane * 512, &sm.xg, &S->full[stage],
+                                    (kb * KC + c) * BK, tok[0], tok[1], tok[2], tok[3]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 if (held && kb + 1 == min(STAGES, num_kb)) {  // first item: stage j holds K block j
                     pdl_wait();
                     held = false;
                     if (g4_lane) load_tokens();
-                    for (int j = 0; j <= kb; ++j) {
-                        if (g4_lane)
-                            tma_gather4(sA + j * A_BYTES + lane * 512, &sm.xg, &S->full[j], j * BK, tok[0], tok[1],
-                                        tok[2], tok[3]);
-                        else if (!g4 && lane == 0)
-                            tma_load_2d(sA + j * A_BYTES, amap, &S->full[j], j * BK, arow0);
-                    }
+                    for (int j = 0; j <= kb; ++j)
+                        for (int c = 0; c < chunks_of(j, Kd); ++c) {
+                            if (g4_lane)
+                                tma_gather4(sA + j * A_BYTES + c * A_SUB + lane * 512, &sm.xg, &S->full[j],
+                                            (j * KC + c) * BK, tok[0], tok[1], tok[2], tok[3]);
+                            else if (!g4 && lane == 0)
+                                tma_load_2d(sA + j * A_BYTES + c * A_SUB, amap, &S->full[j], (j * KC + c) * BK, arow0);
+                        }
                 }
             }
             if (!ok) break;
@@ -337,7 +356,8 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+            constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);           // down: N = 256
+            constexpr uint32_t IDESC_H = idesc_bf16_f32(BM, BN / 2);     // gate, up: N = 128 each
             int stage = 0, rs = 0, acc = 0;
             uint32_t phase = 0, rphase = 0, aphase = 0;
             // timeout test: wait (bounded) on a barrier nothing signals, then unwind
@@ -348,7 +368,8 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                 mbar_arrive(&S->ite[rs]);
                 if (++rs == RING) { rs = 0; rphase ^= 1; }
                 if (item < 0) break;
-                const int num_kb = pos_of(item).p1 ? kb1 : kb0;
+                const bool p1 = pos_of(item).p1;
+                const int num_kb = p1 ? kb1 : kb0, Kd = p1 ? K1 : g.K;
                 if (!mbar_wait(&S->acce[acc], aphase ^ 1, g.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
@@ -357,10 +378,27 @@ grouped_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ C
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
                     const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+                    const int nc = chunks_of(kb, Kd);
+                    for (int c = 0; c < nc; ++c) {
+                        const uint32_t ac = a0 + c * A_SUB;
+                        if (!p1) {
+                            // gate rows [KC][128] then up rows [KC][128]: an N = 128 MMA into
+                            // each half of the accumulator (gate columns 0..127, up 128..255)
+                            const uint32_t bg = b0 + c * (B_SUB / 2), bu = b0 + B_BYTES / 2 + c * (B_SUB / 2);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16(d, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), IDESC,
-                                 (kb | k) != 0);
+                            for (int k = 0; k < BK / 16; ++k) {
+                                const uint64_t ad = sw128_kmajor_desc(ac + k * 32);
+                                mma_bf16(d, ad, sw128_kmajor_desc(bg + k * 32), IDESC_H, (kb | c | k) != 0);
+                                mma_bf16(d + BN / 2, ad, sw128_kmajor_desc(bu + k * 32), IDESC_H, (kb | c | k) != 0);
+                            }
+                        } else {
+                            const uint32_t bc = b0 + c * B_SUB;
+#pragma unroll
+                            for (int k = 0; k < BK / 16; ++k)
+                                mma_bf16(d, sw128_kmajor_desc(ac + k * 32), sw128_kmajor_desc(bc + k * 32), IDESC,
+                                         (kb | c | k) != 0);
+                        }
+                    }
                     mma_commit(&S->empty[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -519,9 +557,9 @@ static bool smem_attr_ready(int mode)
     std::lock_guard<std::mutex> lk(mu);
     if (done[mode] >> dev & 1ull) return true;
     const int a = (int)SMEM_BYTES;
+    if (mode == 2) return false;  // no dense mode: the router's tensor-core logits run in the fp8 kernel
     cudaError_t e = mode == 0   ? cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
                   : mode == 1 ? cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
-                  : mode == 2 ? cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
                               : cudaFuncSetAttribute(grouped_gemm_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, a);
     if (e != cudaSuccess) return false;
     done[mode] |= 1ull << dev;
@@ -532,7 +570,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUten
                                 const CUtensorMap &tmB1, cudaStream_t st, const SharedMaps *sm, const LayerMaps *lm)
 {
     const int grid = g.ctas > 0 ? g.ctas : num_sms();
-    if (g.mode < 0 || g.mode > 3 || !smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
+    if (g.mode < 0 || g.mode > 3 || g.mode == 2 || !smem_attr_ready(g.mode)) return cudaErrorInvalidValue;
     if (g.sh_count && (!sm || g.mode == 2)) return cudaErrorInvalidValue;
     if (g.mode == 3 && (!lm || !g.ready)) return cudaErrorInvalidValue;
     if (g.a_rows && (!sm || g.a_div <= 0 || g.a_tokens <= 0 || (g.mode != 0 && g.mode != 3))) return cudaErrorInvalidValue;
@@ -543,7 +581,6 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, const AMaps &tmA, const CUten
     switch (g.mode) {
     case 0: return launch_pdl(grouped_gemm_kernel<0>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s, l);
     case 1: return launch_pdl(grouped_gemm_kernel<1>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s, l);
-    case 2: return launch_pdl(grouped_gemm_kernel<2>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s, l);
     default: return launch_pdl(grouped_gemm_kernel<3>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, tmA, tmB0, tmB1, g, s, l);
     }
 }

@@ -115,6 +115,15 @@ __device__ __forceinline__ void tma_gather4_pair(void *dst, const CUtensorMap *t
         "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
         : "memory");
 }
+__device__ __forceinline__ void tma_load_4d_pair(void *dst, const CUtensorMap *tm, uint32_t bar, int x, int y, int z,
+                                                 int w)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
 __device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *tm, uint32_t bar, int x, int y, int z)
 {
     asm volatile(
@@ -359,7 +368,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                                     : MODE == 3 ? (tr.s >= 0 ? &lm.wd_sh : &lm.wd)
                                                 : (tr.s >= 0 ? &sm.b0 : &tmB0);
             const bool b_in = nrow < (p1 ? NP1 : g.N);  // a half entirely past N loads nothing (masked columns)
-            const uint32_t b_bytes = b_in ? (uint32_t)B2_SUB : 0u;  // per 64-column box
             const int num_kb = p1 ? kb1 : kb0;
             const int Kd = p1 ? KP1 : g.K;
             if (MODE == 3 && p1) {
@@ -378,24 +386,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS2, 1)
                 if (lane == 0) {
                     okl = wait2(&S->empty[stage], phase ^ 1, g.wait_ns);
                     if (okl) {
-                        const uint32_t tx = (a_bytes + b_bytes) * (uint32_t)nbx;
+                        // the B box brings both chunks of its rows (one past the K range
+                        // reads zeros and is not multiplied)
+                        const uint32_t tx = a_bytes * (uint32_t)nbx + (b_in ? (uint32_t)B2_BYTES : 0u);
                         if (rank == 0)
                             mbar_arrive_expect_tx(&S->full[stage], tx);
                         else
                             arrive_expect_tx_remote(fb, tx);
-                        for (int x = 0; x < nbx; ++x) {
-                            const int kx = kb * BKS2 + x * BK2;
+                        for (int x = 0; x < nbx; ++x)
                             if (rows > 0 && !held && !g4)
-                                tma_load_2d_pair(sA + stage * A2_BYTES + x * A2_SUB, amap, fb, kx, arow0);
-                            if (b_in) {
-                                uint8_t *b_dst = sB + stage * B2_BYTES + x * B2_SUB;
-                                if (tr.s < 0)
-                                    tma_load_3d_pair(b_dst, bmap, fb, kx, nrow, expert);
-                                else if (!p1)  // shared slice s: rows s*I + nrow.. of the shared gate / up
-                                    tma_load_2d_pair(b_dst, bmap, fb, kx, tr.s * g.N + nrow);
-                                else  // shared down: columns s*I + kx..
-                                    tma_load_2d_pair(b_dst, bmap, fb, tr.s * KP1 + kx, nrow);
-                            }
+                                tma_load_2d_pair(sA + stage * A2_BYTES + x * A2_SUB, amap, fb, kb * BKS2 + x * BK2,
+                                                 arow0);
+                        if (b_in) {  // [KW2][128 rows] of B in one box
+                            uint8_t *b_dst = sB + stage * B2_BYTES;
+                            const int z = kb * KW2;
+                            if (tr.s < 0)
+                                tma_load_4d_pair(b_dst, bmap, fb, 0, nrow, z, expert);
+                            else if (!p1)  // shared slice s: rows s*I + nrow.. of the shared gate / up
+                                tma_load_3d_pair(b_dst, bmap, fb, 0, tr.s * g.N + nrow, z);
+                            else  // shared down: chunks of columns s*I..
+                                tma_load_3d_pair(b_dst, bmap, fb, 0, nrow, tr.s * (KP1 / BK2) + z);
                         }
                     }
                 }

@@ -167,6 +167,24 @@ bool encode_3d(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 weights [E, rows, cols] seen as [E][cols / 64][rows][64]: one box brings kc
+// consecutive 64-column chunks of box_rows rows of one expert, chunk after chunk, so
+// each row is read 128 * kc contiguous bytes at a time (DRAM streams such boxes about
+// a third faster than 128-byte row pieces).
+bool encode_4d_chunked(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                       uint32_t kc)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f || cols % 64) return false;
+    const cuuint64_t dims[4] = {64, rows, cols / 64, E};
+    const cuuint64_t strides[3] = {cols * 2, 128, rows * cols * 2};
+    const cuuint32_t box[4] = {64, box_rows, kc, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 moe_status_t check_dims(const moe_dims_t *d)
 {
     if (!d) return MOE_ERR_INVALID_ARG;
@@ -486,18 +504,18 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
     const int plan = bf16_plan(*d);
     const bool pairs = plan & MOE_PLAN_PAIR_TILES;
     if (!moe::encode_a_maps(&tm_xs, xs, A, d->H, false) ||
-        !encode_3d(&tm_wg, w_gate, d->E, d->I, d->H, 128) ||
-        !encode_3d(&tm_wu, w_up, d->E, d->I, d->H, 128) ||
+        !encode_4d_chunked(&tm_wg, w_gate, d->E, d->I, d->H, 128, 2) ||
+        !encode_4d_chunked(&tm_wu, w_up, d->E, d->I, d->H, 128, 2) ||
         !moe::encode_a_maps(&tm_h, h, R, d->I, false) ||
-        !encode_3d(&tm_wd, w_down, d->E, d->H, d->I, pairs ? 128 : 256))
+        !encode_4d_chunked(&tm_wd, w_down, d->E, d->H, d->I, pairs ? 128 : 256, 2))
         return MOE_ERR_CUDA;
-    // the shared expert: x itself as its gate/up A operand, its weights as 2-D maps
+    // the shared expert: x itself as its gate/up A operand, its weights as chunked maps
     // with the boxes of the routed experts' maps
     moe::SharedMaps sm1{}, sm2{};
     if (sh && (!moe::encode_a_maps(&sm1.x, x, d->T, d->H, false) ||
-               !encode_2d(&sm1.b0, shared_gate, shared_I, d->H, 128) ||
-               !encode_2d(&sm1.b1, shared_up, shared_I, d->H, 128) ||
-               !encode_2d(&sm2.b0, shared_down, d->H, shared_I, pairs ? 128 : 256)))
+               !moe::encode_sw128_chunked_bf16(&sm1.b0, shared_gate, shared_I, d->H, 128, 2) ||
+               !moe::encode_sw128_chunked_bf16(&sm1.b1, shared_up, shared_I, d->H, 128, 2) ||
+               !moe::encode_sw128_chunked_bf16(&sm2.b0, shared_down, d->H, shared_I, pairs ? 128 : 256, 2)))
         return MOE_ERR_CUDA;
     // gate/up A rows straight from x: one-row boxes for tile::gather4, the token of
     // sorted row r being sorted_to_flat[r] / k
