@@ -136,6 +136,23 @@ bool encode_3d_fp4(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same e2m1 weights seen as [E][cols / 128][rows][128 codes]: one box brings two
+// consecutive 128-code chunks of box_rows rows (128 contiguous packed bytes a row, where
+// a single chunk reads 64), chunk after chunk.
+bool encode_4d_fp4_pairs(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f || cols % 256) return false;
+    const cuuint64_t dims[4] = {128, rows, cols / 128, E};
+    const cuuint64_t strides[3] = {cols / 2, 64, rows * cols / 2};
+    const cuuint32_t box[4] = {128, box_rows, 2, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Scale codes (bytes) [E, rows, cols], boxes of 16 codes x box_rows, no swizzle: a
 // 3-D map (rank 3, loaded with 3 coordinates) or, with rank 2, a 2-D one over [rows,
 // cols] (E = 1).
@@ -751,12 +768,14 @@ moe_status_t moe_forward_mx(const moe_dims_t *d, const void *x, const void *rout
                      ctas, rev, wait_ns, stall, trace1};
     moe::MxLaunch g2{1, d->I, d->H, tiles, ntiles, &hdr->counter[1], &hdr->status, nullptr, nullptr, y, s2f,
                      ctas, rev, wait_ns, stall, trace2};
-    if (!moe::encode_a_maps(&g1.tmX, xs, A, d->H, true) || !encode_3d_fp4(&g1.tmW0, w_gate_p, d->E, d->I, d->H, 128) ||
-        !encode_3d_fp4(&g1.tmW1, w_up_p, d->E, d->I, d->H, 128) ||
+    if (!moe::encode_a_maps(&g1.tmX, xs, A, d->H, true) ||
+        !encode_4d_fp4_pairs(&g1.tmW0, w_gate_p, d->E, d->I, d->H, 128) ||
+        !encode_4d_fp4_pairs(&g1.tmW1, w_up_p, d->E, d->I, d->H, 128) ||
         !encode_scales_u8(&g1.tmSX, xs_x, 1, A, d->H / 32, 64, 2) ||
         !encode_scales_u8(&g1.tmSW0, w_gate_x, d->E, d->I, d->H / 32, 128, 3) ||
         !encode_scales_u8(&g1.tmSW1, w_up_x, d->E, d->I, d->H / 32, 128, 3) ||
-        !moe::encode_a_maps(&g2.tmX, h, A, d->I, true) || !encode_3d_fp4(&g2.tmW0, w_down_p, d->E, d->H, d->I, 128) ||
+        !moe::encode_a_maps(&g2.tmX, h, A, d->I, true) ||
+        !encode_4d_fp4_pairs(&g2.tmW0, w_down_p, d->E, d->H, d->I, 128) ||
         !encode_scales_u8(&g2.tmSX, h_x, 1, A, d->I / 32, 64, 2) ||
         !encode_scales_u8(&g2.tmSW0, w_down_x, d->E, d->H, d->I / 32, 128, 3))
         return MOE_ERR_CUDA;

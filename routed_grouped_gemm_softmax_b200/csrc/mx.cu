@@ -50,7 +50,7 @@ namespace {
 constexpr int XR = kTileRows / 2;       // token rows per item: the MMA's N at most
 constexpr int FR = 128;                 // weight rows per MMA: the MMA's M
 constexpr int KE = 128;                 // K elements per stage (4 MMAs of K = 32)
-constexpr int MST = 5;                  // stages
+constexpr int MST = 4;                  // stages, filled in pairs (K blocks 2j and 2j+1 on one barrier)
 constexpr int MRING = 4;                // item ring
 constexpr int SG = 4;                   // stages per scale block (16 bytes of e8m0 codes per row)
 constexpr int X_BYTES = XR * KE;        // 8 KB: e4m3 token rows
@@ -186,10 +186,13 @@ grouped_gemm_mx_kernel(const __grid_constant__ AMaps tmX, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     uint8_t *sX = smem_raw + pad;
-    uint8_t *sW = sX + MST * X_BYTES;       // [stage][2][W_BYTES]
+    uint8_t *sW = sX + MST * X_BYTES;       // [stage pair][tile][2 stages][W_BYTES]
     uint8_t *sS = sW + MST * 2 * W_BYTES;   // [2][SBUF]: weight 0, weight 1, token scale blocks
     uint8_t *sC = sS + 2 * SBUF;            // [stage][CP_BYTES]: the stage's scales in the tcgen05.cp layout
     CtrlM *S = reinterpret_cast<CtrlM *>(sC + MST * CP_BYTES);
+    // weight tile t of stage s: a pair of stages shares each tile's box (both K blocks of
+    // its rows, 128 contiguous packed bytes a row)
+    auto w_tile = [&](int s, int t) { return sW + (size_t)(s / 2) * 4 * W_BYTES + t * 2 * W_BYTES + (s & 1) * W_BYTES; };
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int mode = g.mode;
@@ -264,14 +267,19 @@ grouped_gemm_mx_kernel(const __grid_constant__ AMaps tmX, const __grid_constant_
                         tma_load_2d(sb + 2 * SW_BYTES, &tmSX, &S->sgf[gb], kx, it.row0);
                         if (++gb == 2) { gb = 0; gphase ^= 1; }
                     }
-                    if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&S->full[stage], a_box_rows(xb) * KE + 2 * W_TX);
-                    armed |= 1u << stage;
-                    armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-                    uint8_t *w_dst = sW + stage * 2 * W_BYTES;
-                    tma_load_2d(sX + stage * X_BYTES, &tmX.m[xb], &S->full[stage], kb * KE, it.row0);
-                    tma_load_3d(w_dst, &tmW0, &S->full[stage], kb * KE, n0, it.expert);
-                    tma_load_3d(w_dst + W_BYTES, &tmW1, &S->full[stage], kb * KE, n1, it.expert);
+                    if ((kb & 1) == 0) {
+                        // K blocks kb and kb+1 (KB is a multiple of 4, and every item starts on
+                        // an even stage) in stages stage and stage+1, on full[stage]
+                        if (!mbar_wait(&S->empty[stage], phase ^ 1, g.wait_ns) ||
+                            !mbar_wait(&S->empty[stage + 1], phase ^ 1, g.wait_ns)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&S->full[stage], 2 * (a_box_rows(xb) * KE + 2 * W_TX));
+                        armed |= 1u << stage;
+                        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+                        tma_load_2d(sX + stage * X_BYTES, &tmX.m[xb], &S->full[stage], kb * KE, it.row0);
+                        tma_load_2d(sX + (stage + 1) * X_BYTES, &tmX.m[xb], &S->full[stage], (kb + 1) * KE, it.row0);
+                        tma_load_4d(w_tile(stage, 0), &tmW0, &S->full[stage], 0, n0, kb, it.expert);
+                        tma_load_4d(w_tile(stage, 1), &tmW1, &S->full[stage], 0, n1, kb, it.expert);
+                    }
                     if (++stage == MST) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
@@ -311,11 +319,12 @@ grouped_gemm_mx_kernel(const __grid_constant__ AMaps tmX, const __grid_constant_
                 tc_fence_after();
                 const uint32_t d0 = tmem + static_cast<uint32_t>(acc) * ACC_COLS, d1 = d0 + XR;
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&S->full[stage], phase, g.wait_ns)) { ok = false; break; }
+                    // the pair's data lands on the even stage's barrier
+                    if ((kb & 1) == 0 && !mbar_wait(&S->full[stage], phase, g.wait_ns)) { ok = false; break; }
                     if (!mbar_wait(&S->sff[stage], phase, g.wait_ns)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t x0 = smem_u32(sX + stage * X_BYTES);
-                    const uint32_t w0 = smem_u32(sW + stage * 2 * W_BYTES), w1 = w0 + W_BYTES;
+                    const uint32_t w0 = smem_u32(w_tile(stage, 0)), w1 = smem_u32(w_tile(stage, 1));
                     const uint32_t sf = tmem + SF_COL0 + static_cast<uint32_t>(stage) * SF_SLOT;
                     const uint32_t cp0 = smem_u32(sC + stage * CP_BYTES);
                     tmem_cp_32x128b_x4(sf, cp_desc(cp0));             // weight tile 0
