@@ -256,7 +256,7 @@ void moe_set_claim_order(int32_t mode);
 
 /* Pair-of-CTA GEMMs (tcgen05 cta_group::2: a 256 x 256 tile per 2-CTA cluster,
  * each CTA loading half the operands).  0 = automatic (the bf16 forward uses
- * them when the batch is not a small one and averages at least 512 rows per
+ * them when the batch is not a small one and averages at least 768 rows per
  * expert), 1 = whenever the forward can (tests), 2 = never.  Each output is the
  * same K-ordered tensor-core sum either way; the results stay within the layer's
  * tolerance of the oracle.  Process-wide. */

@@ -517,7 +517,7 @@ moe_status_t moe_forward_shared(const moe_dims_t *d, const void *x, const void *
     moe::AMaps tm_xs, tm_h;
     CUtensorMap tm_wg, tm_wu, tm_wd;
     // pair-of-CTA GEMMs for groups large enough to be compute-bound (on average at
-    // least 512 rows per expert), on the queue's claim modes
+    // least 768 rows per expert), on the queue's claim modes
     const int plan = bf16_plan(*d);
     const bool pairs = plan & MOE_PLAN_PAIR_TILES;
     if (!moe::encode_a_maps(&tm_xs, xs, A, d->H, false) ||

@@ -381,7 +381,7 @@ struct TileChoice {
 constexpr TileChoice kTileTable[] = {
     {16, false, true, true, true},
     {64, false, true, true, false},
-    {511, false, true, false, false},
+    {767, false, true, false, false},
     {0x7fffffff, true, true, false, false},
 };
 inline TileChoice tile_choice(long long A, int E)

@@ -155,9 +155,9 @@ def test_forward_plan_follows_the_tile_table(L):
     assert plan(16, 2048, 512, 256, 8) == api.PLAN_SMALL_ROUTER | api.PLAN_FUSED_COMBINE | api.PLAN_LAYER_GEMM
     # 128 rows per expert: 128-row tiles, one GEMM launch, the combine kernel
     assert plan(4096, 2048, 512, 256, 8) == api.PLAN_LAYER_GEMM
-    # 511 rows per expert still 128-row tiles; 512 and up pair tiles
-    assert plan(511 * 64 // 8 + 7, 2048, 1024, 64, 8) & api.PLAN_PAIR_TILES == 0
-    assert plan(512 * 64 // 8, 2048, 1024, 64, 8) & api.PLAN_PAIR_TILES
+    # 767 rows per expert still 128-row tiles; 768 and up pair tiles
+    assert plan(767 * 64 // 8 + 7, 2048, 1024, 64, 8) & api.PLAN_PAIR_TILES == 0
+    assert plan(768 * 64 // 8, 2048, 1024, 64, 8) & api.PLAN_PAIR_TILES
     assert plan(8192, 4096, 1408, 64, 6) == api.PLAN_PAIR_TILES | api.PLAN_LAYER_GEMM   # the Skewed workload
     # the combine inside the down GEMM up to 32 tokens
     assert plan(32, 512, 512, 64, 8) & api.PLAN_FUSED_COMBINE
