@@ -120,25 +120,11 @@ bool encode_3d_u8(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, u
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// e2m1 weights [E, rows, cols] packed two codes per byte, read as 128-code x box_rows
-// tiles that TMA expands to 16 bytes per 16 codes (the MMA's 4-bit operand layout,
-// 128 bytes per tile row), with the 128-byte swizzle.
-bool encode_3d_fp4(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols, uint32_t box_rows)
-{
-    EncodeTiledFn f = encode_fn();
-    if (!f) return false;
-    const cuuint64_t dims[3] = {cols, rows, E};
-    const cuuint64_t strides[2] = {cols / 2, rows * cols / 2};
-    const cuuint32_t box[3] = {128, box_rows, 1};
-    const cuuint32_t es[3] = {1, 1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// The same e2m1 weights seen as [E][cols / 128][rows][128 codes]: one box brings two
-// consecutive 128-code chunks of box_rows rows (128 contiguous packed bytes a row, where
-// a single chunk reads 64), chunk after chunk.
+// e2m1 weights [E, rows, cols], packed two codes per byte, seen as [E][cols / 128][rows]
+// [128 codes]: one box brings two consecutive 128-code chunks of box_rows rows (128
+// contiguous packed bytes a row, where a single chunk reads 64), chunk after chunk. TMA
+// expands every 16 codes to 16 bytes (the MMA's 4-bit operand layout) under the 128-byte
+// swizzle.
 bool encode_4d_fp4_pairs(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, uint64_t cols,
                          uint32_t box_rows)
 {
