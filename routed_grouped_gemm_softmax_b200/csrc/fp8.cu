@@ -61,6 +61,14 @@ struct Ctrl8 {
 };
 
 constexpr size_t SMEM8 = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + sizeof(Ctrl8);
+// Mode 2 adds a transpose buffer per epilogue warp: 32 rows x 16 fp32 logits, rows
+// padded to 80 bytes (five 16-byte slots, so that eight consecutive rows' slots fall
+// in distinct bank groups).
+constexpr int EPI2_ROW = 20;  // floats per buffered row
+constexpr size_t EPI2_BYTES = (size_t)EPI_WARPS * 32 * EPI2_ROW * 4;
+constexpr size_t EPI2_OFF = (sizeof(Ctrl8) + 15) / 16 * 16;  // after the control block, 16-byte aligned
+constexpr size_t smem8_bytes(int mode) { return SMEM8 + (mode == 2 ? 16 + EPI2_BYTES : 0); }
+static_assert(smem8_bytes(2) <= 232448, "mode 2 shared memory");
 
 // ------------------------------------------------------------ quantiser
 
@@ -184,11 +192,12 @@ grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    // The prologue above overlapped the previous kernel.  Modes 0 and 1: warp 0 waits
-    // for it inside the producer, after the first stages' weight loads (mode 2's B
-    // operand is the previous kernel's output).
+    // The prologue above overlapped the previous kernel.  Warp 0 waits for it inside
+    // the producer, after the loads of the first stages that do not depend on it: the
+    // weights in modes 0 and 1 (A is the previous kernel's output), x in mode 2 (B, the
+    // transposed router matrix, is the previous kernel's output).
     constexpr bool kEarlyB = MODE != 2;
-    if (!(kEarlyB && warp == 0)) pdl_wait();
+    if (warp != 0) pdl_wait();
     pdl_trigger();
     if (g.trace && threadIdx.x == 0) g.trace[2 * blockIdx.x] = globaltimer_ns();
 
@@ -200,7 +209,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant
             uint32_t phase = 0, rphase = 0, armed = 0, armed_par = 0;
             bool ok = true;
             int cursor = (int)blockIdx.x * (g.reverse == 2);  // static modes
-            bool held = kEarlyB;  // A loads of the first item's first stages wait for the previous kernel
+            bool held = true;  // the first item's first stages: dependent loads wait for the previous kernel
             for (;;) {
                 const int item = claim_item(g.reverse, g.counter, total, n_tiles * ksplit, dense ? nullptr : g.tiles, cursor);
                 if (!mbar_wait(&S->ite[rs], rphase ^ 1, g.wait_ns)) { ok = false; break; }
@@ -221,15 +230,21 @@ grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant
                     armed |= 1u << stage;
                     armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
                     uint8_t *b_dst = sB + stage * B_BYTES;
-                    if (!held) tma_load_2d(sA + stage * A_BYTES, &tmA.m[ab], &S->full[stage], kb * KEL, row0);
-                    tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * KEL, n0, expert);
-                    if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * KEL, n0, expert);
+                    if (!held || !kEarlyB) tma_load_2d(sA + stage * A_BYTES, &tmA.m[ab], &S->full[stage], kb * KEL, row0);
+                    if (!held || kEarlyB) {
+                        tma_load_3d(b_dst, &tmB0, &S->full[stage], kb * KEL, n0, expert);
+                        if (MODE == 0) tma_load_3d(b_dst + B_BYTES / 2, &tmB1, &S->full[stage], kb * KEL, n0, expert);
+                    }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                     if (held && kb + 1 - kb0 == min(STAGES, kb1 - kb0)) {  // first item: stage j holds its K block kb0 + j
                         pdl_wait();
                         held = false;
-                        for (int j = 0; j <= kb - kb0; ++j)
-                            tma_load_2d(sA + j * A_BYTES, &tmA.m[ab], &S->full[j], (kb0 + j) * KEL, row0);
+                        for (int j = 0; j <= kb - kb0; ++j) {
+                            if (kEarlyB)
+                                tma_load_2d(sA + j * A_BYTES, &tmA.m[ab], &S->full[j], (kb0 + j) * KEL, row0);
+                            else
+                                tma_load_3d(sB + j * B_BYTES, &tmB0, &S->full[j], (kb0 + j) * KEL, n0, expert);
+                        }
                     }
                 }
                 if (!ok) break;
@@ -407,20 +422,39 @@ grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant
                     if (half == 0) g.out_s[(size_t)(row0 + row) * NB + n0 / 128] = sc;
                 }
             } else if (MODE == 2) {
-                // partial logits of K split ks: [ksplit][M][N] fp32
+                // partial logits of K split ks: [ksplit][M][N] fp32.  With N a multiple of
+                // 4 (rows 16-byte aligned), 16 columns at a time go through the warp's
+                // transpose buffer, so that each store covers 64 contiguous bytes of 8 rows
+                // (the thread's own row would be 32 scattered 16-byte pieces per store).
                 const int col = n0 + half * 128;
-                if (row_ok && col < g.N) {
-                    float *dst = g.out_f32 + ((size_t)ks * g.M + row0 + row) * g.N + col;
-                    if (col + 128 <= g.N && (g.N & 3) == 0) {  // rows 16-byte aligned
+                if ((g.N & 3) == 0) {
+                    float *buf = reinterpret_cast<float *>(sB + STAGES * B_BYTES + EPI2_OFF) +
+                                 (warp - 2) * 32 * EPI2_ROW;
+                    const int rr = lane % 8, m = lane / 8;  // read-back: row rr + 8p, 16-byte piece m
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            reinterpret_cast<float4 *>(dst)[i] =
-                                make_float4(accr[4 * i], accr[4 * i + 1], accr[4 * i + 2], accr[4 * i + 3]);
-                    } else {
+                    for (int c = 0; c < 8; ++c) {
+                        if (col + 16 * c >= g.N) break;  // warp-uniform: columns past N
 #pragma unroll
-                        for (int i = 0; i < 128; ++i)
-                            if (col + i < g.N) dst[i] = accr[i];
+                        for (int i = 0; i < 4; ++i)
+                            reinterpret_cast<float4 *>(buf + lane * EPI2_ROW)[i] =
+                                make_float4(accr[16 * c + 4 * i], accr[16 * c + 4 * i + 1], accr[16 * c + 4 * i + 2],
+                                            accr[16 * c + 4 * i + 3]);
+                        __syncwarp();
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) {
+                            const int r = 8 * p + rr;  // row within the warp's 32
+                            const float4 v = reinterpret_cast<const float4 *>(buf + r * EPI2_ROW)[m];
+                            const int cc = col + 16 * c + 4 * m;
+                            if (q * 32 + r < rows && cc < g.N)
+                                *reinterpret_cast<float4 *>(g.out_f32 + ((size_t)ks * g.M + row0 + q * 32 + r) * g.N + cc) = v;
+                        }
+                        __syncwarp();
                     }
+                } else if (row_ok && col < g.N) {
+                    float *dst = g.out_f32 + ((size_t)ks * g.M + row0 + row) * g.N + col;
+#pragma unroll
+                    for (int i = 0; i < 128; ++i)
+                        if (col + i < g.N) dst[i] = accr[i];
                 }
             } else {
                 const int col = n0 + half * 128;
@@ -459,7 +493,7 @@ bool fp8_smem_attr_ready(int v)  // v: 0 gate/up, 1 down, 2 router logits, 3 dow
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     std::lock_guard<std::mutex> lk(mu);
     if (done[v] >> dev & 1ull) return true;
-    const int a = (int)SMEM8;
+    const int a = (int)smem8_bytes(v);
     cudaError_t e = v == 0   ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
                   : v == 1 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
                   : v == 2 ? cudaFuncSetAttribute(grouped_gemm_fp8_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, a)
@@ -503,7 +537,8 @@ cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const AMaps &tmA, cons
     else if (g.mode == 1)
         e = launch_pdl(grouped_gemm_fp8_kernel<1, false>, dim3(grid), dim3(THREADS), SMEM8, st, tmA, tmB0, tmB1, g);
     else
-        e = launch_pdl(grouped_gemm_fp8_kernel<2, true>, dim3(grid), dim3(THREADS), SMEM8, st, tmA, tmB0, tmB1, g);
+        e = launch_pdl(grouped_gemm_fp8_kernel<2, true>, dim3(grid), dim3(THREADS), smem8_bytes(2), st, tmA, tmB0,
+                       tmB1, g);
     return e;
 }
 

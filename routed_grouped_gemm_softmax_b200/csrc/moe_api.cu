@@ -331,7 +331,9 @@ bool encode_a_maps(AMaps *m, const void *base, uint64_t rows, uint64_t cols, boo
 
 // The router's tensor-core logits: the block-promoting GEMM (fp8.cu, mode 2, bf16
 // operands) over plain 128-row blocks of x against the transposed router matrix,
-// K split over enough items to occupy the GPU.  Uses work counter 2.
+// K split over enough items to occupy the GPU.  The items are uniform, so they are
+// dealt out statically (no work counter, and so nothing between the router's prep
+// kernel and this one: x loads overlap the prep kernel's tail).
 cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, int T, int H, int E, float *logits,
                              WsHeader *hdr, int *ksplit_out, cudaStream_t st)
 {
@@ -343,10 +345,8 @@ cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, i
     ks = ks < 1 ? 1 : ks > kRouterKSplitMax ? kRouterKSplitMax : ks;
     if (ks > H / 64) ks = H / 64;
     *ksplit_out = ks;
-    cudaError_t e = cudaMemsetAsync(&hdr->counter[2], 0, sizeof(int32_t), st);
-    if (e != cudaSuccess) return e;
     Fp8GemmArgs g{2, H, E, nullptr, nullptr, &hdr->counter[2], &hdr->status, nullptr, nullptr, nullptr, nullptr,
-                  nullptr, nullptr, nullptr, 0, 0, 2000000000ull, 0, T, ks, logits};
+                  nullptr, nullptr, nullptr, 0, 2, 2000000000ull, 0, T, ks, logits};
     return launch_grouped_gemm_fp8(g, tm_x, tm_w, tm_w, st);
 }
 }  // namespace moe
