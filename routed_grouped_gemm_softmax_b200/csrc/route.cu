@@ -359,25 +359,13 @@ __global__ void __launch_bounds__(TP * 8) route_logits_tma_kernel(const __grid_c
         ok = mbar_wait(&bars[1 + c], 0);
         const uint16_t *wc = reinterpret_cast<const uint16_t *>(wsm + (size_t)c * kLogitsChunk * TE * 2) + ee;
         const uint4 *xc = xv + c * (kLogitsChunk / 8);
-        uint4 xq = xc[0];
-        uint16_t w[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) w[j] = wc[j * TE];
-#pragma unroll 4
         for (int h8 = 0; h8 < kLogitsChunk / 8; ++h8) {
-            uint4 xn = xq;
-            uint16_t wn[8];
-            const int nx = h8 + 1 < kLogitsChunk / 8 ? h8 + 1 : h8;  // the next group (or this one again)
-            xn = xc[nx];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) wn[j] = wc[(nx * 8 + j) * TE];
-            acc = chain_step2(xq.x, w[0], w[1], acc);
-            acc = chain_step2(xq.y, w[2], w[3], acc);
-            acc = chain_step2(xq.z, w[4], w[5], acc);
-            acc = chain_step2(xq.w, w[6], w[7], acc);
-            xq = xn;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) w[j] = wn[j];
+            const uint4 xq = xc[h8];
+            acc = chain_step2(xq.x, wc[(h8 * 8 + 0) * TE], wc[(h8 * 8 + 1) * TE], acc);
+            acc = chain_step2(xq.y, wc[(h8 * 8 + 2) * TE], wc[(h8 * 8 + 3) * TE], acc);
+            acc = chain_step2(xq.z, wc[(h8 * 8 + 4) * TE], wc[(h8 * 8 + 5) * TE], acc);
+            acc = chain_step2(xq.w, wc[(h8 * 8 + 6) * TE], wc[(h8 * 8 + 7) * TE], acc);
         }
     }
     if (!ok) {
@@ -496,10 +484,10 @@ cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *idx, 
 //     and records tbl[c][e], the chunk's count of expert e;
 //  2. a thread per expert turns tbl[.][e] into the exclusive prefix over chunks
 //     (chunks ascending) and its total;
-//  3. warp 0 scans the totals over experts: offsets, the tile list {expert,
-//     row_start, rows} and the number of tiles;
+//  3. a block-wide scan of the totals over experts (a thread per run of experts):
+//     offsets, the tile list {expert, row_start, rows} and the number of tiles;
 //  4. entry f of chunk c on expert e lands at offsets[e] + tbl[c][e] + rank.
-// So equal experts keep flat order (a stable counting sort) with four barriers.
+// So equal experts keep flat order (a stable counting sort) with six barriers.
 struct SmallRouteOut {
     float *logits;
     int32_t *idx;
@@ -571,10 +559,12 @@ __global__ void __launch_bounds__(1024) topk_permute_small_kernel(int T, int E, 
         base[e] = run;
     }
     __syncthreads();
-    // 3. offsets and tile list (warp 0; lane l owns a contiguous run of experts)
-    if (warp == 0) {
-        const int per = (E + 31) / 32;
-        const int lo = min(E, lane * per), hi = min(E, lo + per);
+    // 3. offsets and tile list: thread i takes experts i*per .. i*per + per - 1, and a
+    // block-wide exclusive scan of (rows, tiles) in expert order places them (the
+    // warps' totals in se[], free after the top-k)
+    {
+        const int per = (E + NT - 1) / NT;
+        const int lo = min(E, tid * per), hi = min(E, lo + per);
         int rows = 0, tls = 0;
         for (int e = lo; e < hi; ++e) {
             rows += base[e];
@@ -590,7 +580,31 @@ __global__ void __launch_bounds__(1024) topk_permute_small_kernel(int T, int E, 
                 tinc += q;
             }
         }
-        int off = rinc - rows, toff = tinc - tls;
+        int *wrow = se, *wtil = se + nw;  // 2 nw <= 2 nw k entries
+        if (lane == 31) {
+            wrow[warp] = rinc;
+            wtil[warp] = tinc;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int r = lane < nw ? wrow[lane] : 0, q = lane < nw ? wtil[lane] : 0;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int r2 = __shfl_up_sync(0xffffffffu, r, off);
+                const int q2 = __shfl_up_sync(0xffffffffu, q, off);
+                if (lane >= off) {
+                    r += r2;
+                    q += q2;
+                }
+            }
+            if (lane < nw) {  // inclusive prefix over the warps
+                wrow[lane] = r;
+                wtil[lane] = q;
+            }
+        }
+        __syncthreads();
+        const int rbase = warp > 0 ? wrow[warp - 1] : 0, tbase = warp > 0 ? wtil[warp - 1] : 0;
+        int off = rbase + rinc - rows, toff = tbase + tinc - tls;
         for (int e = lo; e < hi; ++e) {
             const int c = base[e];
             o.offsets[e] = off;
@@ -604,9 +618,9 @@ __global__ void __launch_bounds__(1024) topk_permute_small_kernel(int T, int E, 
             base[e] = off;
             off += c;
         }
-        if (lane == 31) {
-            o.offsets[E] = rinc;
-            *o.ntiles = tinc;
+        if (tid == NT - 1) {
+            o.offsets[E] = wrow[nw - 1];
+            *o.ntiles = wtil[nw - 1];
         }
     }
     __syncthreads();
