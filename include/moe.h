@@ -293,6 +293,16 @@ void moe_set_layer_gemm(int32_t mode);
  * same.  Process-wide; for tests and benchmarks. */
 void moe_set_direct_a(int32_t mode);
 
+/* Staging of the certified router's exact chains (batches of more than 32 tokens):
+ * the block's x rows and router rows pass through shared memory in chunks of
+ * 64 * boxes values of h, several chunks in flight.  max_stages caps the chunks in
+ * flight (1..8), min_stages is the count the widest chunk must still leave (else the
+ * chunk narrows), max_boxes (1, 2, 4 or 8) caps the chunk width; each argument <= 0
+ * keeps its default (3, 2, 8).  Every chunk costs the chain phase a barrier of the
+ * CTA, so the default takes the widest chunk that leaves two stages.  The chains and so the routing are the same either
+ * way.  Process-wide; for tests and benchmarks. */
+void moe_set_cert_staging(int32_t max_stages, int32_t min_stages, int32_t max_boxes);
+
 /* Scheduling trace for benchmarks.  With `trace` a device buffer of 4 * ctas
  * uint64 values (ctas >= the GEMM grid, 148 by default), every later forward
  * records per GEMM CTA the %globaltimer (ns) when it started work and when it

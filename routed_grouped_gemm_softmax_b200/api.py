@@ -25,7 +25,8 @@ EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "m
            "moe_set_stage_events", "moe_forward_noalloc", "moe_set_wait_limit_us",
            "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets", "moe_set_router_audit",
            "moe_forward_shared", "moe_workspace_size_shared", "moe_forward_mx", "moe_quantize_rows_mx",
-           "moe_set_fused_combine", "moe_set_layer_gemm", "moe_forward_plan", "moe_set_direct_a"]
+           "moe_set_fused_combine", "moe_set_layer_gemm", "moe_forward_plan", "moe_set_direct_a",
+           "moe_set_cert_staging"]
 DTYPE_BF16, DTYPE_FP8, DTYPE_MX = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
@@ -97,6 +98,8 @@ def lib():
         L.moe_set_layer_gemm.restype = None
         L.moe_set_direct_a.argtypes = [I32]
         L.moe_set_direct_a.restype = None
+        L.moe_set_cert_staging.argtypes = [I32, I32, I32]
+        L.moe_set_cert_staging.restype = None
         L.moe_set_fused_combine.argtypes = [I32]
         L.moe_set_fused_combine.restype = None
         L.moe_forward_mx.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -418,6 +421,13 @@ def set_direct_a(mode: str):
     """"auto" (default), "always" or "never": bf16 gate/up A rows gathered straight from x
     by the GEMM (never: from a sorted copy of x made by a gather kernel first)."""
     lib().moe_set_direct_a({"auto": 0, "always": 1, "never": 2}[mode])
+
+
+def set_cert_staging(max_stages: int = 0, min_stages: int = 0, max_boxes: int = 0):
+    """The certified router's chain staging: chunks in flight (cap), the count the
+    widest chunk must leave, and the chunk width cap in 64-value boxes (1, 2, 4, 8);
+    0 keeps each default (3, 2, 8).  Routing is the same either way."""
+    lib().moe_set_cert_staging(max_stages, min_stages, max_boxes)
 
 
 def set_fused_combine(mode: str):

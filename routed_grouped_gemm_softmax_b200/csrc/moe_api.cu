@@ -25,6 +25,7 @@ std::atomic<int> g_pair_mode{0};  // 0 auto, 1 pair GEMMs whenever possible, 2 n
 std::atomic<int> g_fp8_swap{0};   // 0 auto, 1 swapped fp8 gate/up GEMM always, 2 never
 std::atomic<int> g_fused_comb{0}; // 0 auto, 1 combine inside the down GEMM always, 2 never
 std::atomic<int> g_layer_gemm{0}; // 0 auto, 1 gate/up and down GEMMs in one launch always, 2 never
+std::atomic<int> g_cert_max_stages{0}, g_cert_min_stages{0}, g_cert_max_boxes{0};  // 0: defaults
 std::atomic<int> g_direct_a{0};   // 0 auto, 1 gate/up A rows gathered straight from x always, 2 never
 std::atomic<int> g_trace_ctas{0};
 std::atomic<unsigned long long> g_wait_ns{0};
@@ -329,6 +330,13 @@ bool encode_a_maps(AMaps *m, const void *base, uint64_t rows, uint64_t cols, boo
     return true;
 }
 
+void cert_staging(int *max_stages, int *min_stages, int *max_boxes)
+{
+    *max_stages = g_cert_max_stages.load();
+    *min_stages = g_cert_min_stages.load();
+    *max_boxes = g_cert_max_boxes.load();
+}
+
 // The router's tensor-core logits: the block-promoting GEMM (fp8.cu, mode 2, bf16
 // operands) over plain 128-row blocks of x against the transposed router matrix,
 // K split over enough items to occupy the GPU.  The items are uniform, so they are
@@ -385,6 +393,13 @@ void moe_set_fused_combine(int32_t mode) { g_fused_comb.store(mode < 0 || mode >
 void moe_set_layer_gemm(int32_t mode) { g_layer_gemm.store(mode < 0 || mode > 2 ? 0 : mode); }
 
 void moe_set_direct_a(int32_t mode) { g_direct_a.store(mode < 0 || mode > 2 ? 0 : mode); }
+
+void moe_set_cert_staging(int32_t max_stages, int32_t min_stages, int32_t max_boxes)
+{
+    g_cert_max_stages.store(max_stages > 0 ? (max_stages > 8 ? 8 : max_stages) : 0);
+    g_cert_min_stages.store(min_stages > 0 ? (min_stages > 8 ? 8 : min_stages) : 0);
+    g_cert_max_boxes.store(max_boxes >= 8 ? 8 : max_boxes >= 4 ? 4 : max_boxes >= 2 ? 2 : max_boxes == 1 ? 1 : 0);
+}
 
 void moe_set_gemm_trace(unsigned long long *trace, int32_t ctas)
 {

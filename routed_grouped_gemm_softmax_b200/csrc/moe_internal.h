@@ -350,6 +350,9 @@ cudaError_t launch_gather_rows_mx(const uint8_t *xq, const uint8_t *xq_x, const 
 // Tensor-core router logits: partial sums over ksplit slices of H,
 // logits [ksplit, T, E] with sum_s logits[s] = x [T,H] . wrt [E,H]^T (fp32 per
 // 64-wide K block, then fp32 sums).  Returns ksplit through *ksplit_out.
+// The certify kernel's staging policy set by moe_set_cert_staging: {max stages, min
+// stages, max boxes per chunk}, each 0 for the default (3, 2, 8).
+void cert_staging(int *max_stages, int *min_stages, int *max_boxes);
 cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, int T, int H, int E, float *logits,
                              WsHeader *hdr, int *ksplit_out, cudaStream_t st);
 

@@ -19,10 +19,11 @@
 //        Lt + d is below tau has k experts strictly above it and cannot be chosen.
 //        The others -- the k chosen plus near-ties -- are the token's candidates;
 //     b. the exact chain of every candidate of the block: the block's x rows and
-//        all of router_w^T stream through shared memory in chunks of h (tensor-map
-//        tiles, up to three stages on mbarriers), each thread running one or two
-//        chains with the mixed-precision chain step; each exact value is checked
-//        against its bound (a miss records MOE_ERR_ROUTER_BOUND);
+//        its slice of router_w^T stream through shared memory in chunks of up to
+//        512 values of h (tensor-map tiles, two or three stages on mbarriers), a
+//        thread running one chain per round with the mixed-precision chain step;
+//        each exact value is checked against its bound (a miss records
+//        MOE_ERR_ROUTER_BOUND);
 //     c. per token (a warp), top-k and softmax on the candidates' exact values.
 // The chosen experts and gates are therefore those of the chain definition.
 #include <atomic>
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const __nv_bfloat16 *_
 // above (the per-lane arrays of 512 or more experts need the registers).
 constexpr int kCertWarps = 32;  // the most warps a CTA has (sizes the per-warp scratch)
 __host__ __device__ constexpr int cert_threads(int maxv) { return maxv <= 8 ? 1024 : 512; }
-constexpr int kCertMaxStages = 3;
+constexpr int kCertMaxStages = 8;  // staging barriers (the policy's cap, 3 by default)
 constexpr int kCertMaxTB = 128;  // tokens per block
 constexpr int kCertSmem = 227 * 1024;
 
@@ -533,8 +534,9 @@ int cert_clusters(int C)
 // The certify launch for T tokens: tokens in blocks of TB, one cluster of C CTAs per
 // block, CTA r of a cluster taking the chains of experts r*EB .. (r+1)*EB - 1.  C is
 // the cluster size (1, 2, 4 or 8 that fit) whose CTAs stage the fewest rows per chunk
-// (the block's x rows plus the slice's router rows): the chain phase is bound by
-// staging, and the per-token phases take T / (resident CTAs) tokens per CTA either way.
+// (the block's x rows plus the slice's router rows): fewer rows leave room for wider
+// chunks, each chunk costs the chain phase a CTA barrier and a pipeline restart, and
+// the per-token phases take T / (resident CTAs) tokens per CTA either way.
 template <int MAXV>
 cudaError_t certify_shape_and_launch(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, CertifyArgs a, int T, int E,
                                      int k, cudaStream_t st)
@@ -563,12 +565,17 @@ cudaError_t certify_shape_and_launch(const __nv_bfloat16 *x, const __nv_bfloat16
     const int erows = EB <= 256 ? (EB + 7) / 8 * 8 : (EB + 255) / 256 * 256;
     const int ebox = erows < 256 ? erows : 256;
     const size_t room = (size_t)kCertSmem - 1024 - cert_fixed_bytes(E, k);
-    int nbx = 4, stages = 0;
-    for (; nbx >= 1; nbx /= 2) {  // the widest chunk dividing H that still leaves two stages
+    int max_st = 0, min_st = 0, max_nbx = 0;  // the staging policy (moe_set_cert_staging)
+    cert_staging(&max_st, &min_st, &max_nbx);
+    max_st = max_st > 0 ? max_st : 3;
+    min_st = min_st > 0 ? min_st : 2;
+    int nbx = max_nbx > 0 ? max_nbx : 8, stages = 0;
+    for (; nbx >= 1; nbx /= 2) {  // the widest chunk dividing H that still leaves min_st stages
         if ((a.H / 64) % nbx) continue;
         stages = (int)(room / ((size_t)nbx * (xrows + erows) * 128));
-        if (stages >= 2 || nbx == 1) break;
+        if (stages >= min_st || nbx == 1) break;
     }
+    if (stages > max_st) stages = max_st;
     if (stages > kCertMaxStages) stages = kCertMaxStages;
     if (stages < 1) return cudaErrorInvalidValue;
     CUtensorMap tm_x, tm_w;

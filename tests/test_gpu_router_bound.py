@@ -75,3 +75,29 @@ def test_router_bound_holds_for_every_pair(name):
     bad = np.argwhere(gap > d)
     assert bad.size == 0, f"{name}: |chain - tensor-core logit| > bound at {bad[:5].tolist()} " \
                           f"(max ratio {ratio.max():.3f})"
+
+
+STAGING = [(8, 2, 4), (8, 4, 4), (8, 2, 2), (1, 1, 1), (2, 2, 1), (3, 2, 8), (2, 2, 8), (1, 1, 8)]
+
+
+@pytest.mark.parametrize("name", ["prefill", "fp8", "ragged_bias"])
+def test_router_staging_policies_route_identically(name):
+    """The exact chains do not depend on how their operands are staged: every staging
+    policy (chunks in flight, chunk width) gives the default's experts and gates bit for
+    bit, and the default matches the oracle."""
+    cfg, x, rw, bias = _inputs(name)
+    T, E, k = cfg.T, cfg.E, cfg.top_k
+    ws = api.workspace(T, cfg.H, cfg.I, E, k, "cuda")
+    idx0, w0 = api.moe_route(x, rw, bias, k, ws=ws)
+    assert api.moe_get_device_status(ws) == api.MOE_OK
+    idx_ref, gate_ref = oracle.get().route(x.cpu(), rw.cpu(), None if bias is None else bias.cpu(), k)[:2]
+    compare_routing(idx0, w0, idx_ref, gate_ref, name)
+    try:
+        for pol in STAGING:
+            api.set_cert_staging(*pol)
+            idx, w = api.moe_route(x, rw, bias, k, ws=ws)
+            assert api.moe_get_device_status(ws) == api.MOE_OK, pol
+            assert torch.equal(idx, idx0), pol
+            assert torch.equal(w, w0), pol
+    finally:
+        api.set_cert_staging()
