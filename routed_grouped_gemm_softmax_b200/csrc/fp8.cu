@@ -427,7 +427,35 @@ grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant
                 // transpose buffer, so that each store covers 64 contiguous bytes of 8 rows
                 // (the thread's own row would be 32 scattered 16-byte pieces per store).
                 const int col = n0 + half * 128;
-                if ((g.N & 3) == 0) {
+                const int total2 = (g.M + BM - 1) / BM * n_tiles * ksplit;
+                if (g.tma_store && g.reverse == 2 && item + (int)gridDim.x >= total2) {
+                    // The CTA's last item (items are dealt out statically): its last
+                    // accumulator wait above means every MMA, and so every read of the
+                    // stages, is done, and no further loads come.  The warp writes its 32
+                    // rows x 128 columns into the idle stages as four 32 x 32 boxes in the
+                    // 128-byte swizzled layout (chunk j of row r at j ^ (r & 7); eight
+                    // consecutive rows hit distinct bank groups) and one lane stores them
+                    // with the TMA, which clips rows past M and columns past N.
+                    uint8_t *box0 = sA + (size_t)(warp - 2) * 4 * 4096;  // 8 warps x 16 KB
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        if (col + 32 * b >= g.N) break;  // warp-uniform
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            *reinterpret_cast<float4 *>(box0 + b * 4096 + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                                make_float4(accr[32 * b + 4 * j], accr[32 * b + 4 * j + 1], accr[32 * b + 4 * j + 2],
+                                            accr[32 * b + 4 * j + 3]);
+                    }
+                    fence_proxy_async_shared_cta();
+                    __syncwarp();
+                    if (lane == 0) {
+                        for (int b = 0; b < 4 && col + 32 * b < g.N; ++b)
+                            tma_store_3d(&tmB1, box0 + b * 4096, col + 32 * b, row0 + q * 32, ks);
+                        bulk_commit_group();
+                        bulk_wait_all();
+                    }
+                    __syncwarp();
+                } else if ((g.N & 3) == 0) {
                     float *buf = reinterpret_cast<float *>(sB + STAGES * B_BYTES + EPI2_OFF) +
                                  (warp - 2) * 32 * EPI2_ROW;
                     const int rr = lane % 8, m = lane / 8;  // read-back: row rr + 8p, 16-byte piece m

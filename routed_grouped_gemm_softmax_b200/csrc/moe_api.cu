@@ -121,6 +121,21 @@ bool encode_3d_u8(CUtensorMap *m, const void *base, uint64_t E, uint64_t rows, u
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 partial logits [ks][M][N] as 32-column x 32-row boxes with the 128-byte swizzle,
+// for tensor-map stores (N a multiple of 4, so that rows are 16-byte aligned).
+bool encode_logits_store(CUtensorMap *m, float *base, uint64_t ks, uint64_t M, uint64_t N)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f || N % 4) return false;
+    const cuuint64_t dims[3] = {N, M, ks};
+    const cuuint64_t strides[2] = {N * 4, M * N * 4};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // e2m1 weights [E, rows, cols], packed two codes per byte, seen as [E][cols / 128][rows]
 // [128 codes]: one box brings two consecutive 128-code chunks of box_rows rows (128
 // contiguous packed bytes a row, where a single chunk reads 64), chunk after chunk. TMA
@@ -339,8 +354,9 @@ void cert_staging(int *max_stages, int *min_stages, int *max_boxes)
 
 // The router's tensor-core logits: the block-promoting GEMM (fp8.cu, mode 2, bf16
 // operands) over plain 128-row blocks of x against the transposed router matrix,
-// K split over enough items to occupy the GPU.  The items are uniform, so they are
-// dealt out statically (no work counter, and so nothing between the router's prep
+// K split over enough items to occupy the GPU, the partial logits stored by tensor
+// map from the stage buffers once a CTA's items are done.  The items are uniform, so
+// they are dealt out statically (no work counter, and so nothing between the router's prep
 // kernel and this one: x loads overlap the prep kernel's tail).
 cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, int T, int H, int E, float *logits,
                              WsHeader *hdr, int *ksplit_out, cudaStream_t st)
@@ -355,7 +371,9 @@ cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, i
     *ksplit_out = ks;
     Fp8GemmArgs g{2, H, E, nullptr, nullptr, &hdr->counter[2], &hdr->status, nullptr, nullptr, nullptr, nullptr,
                   nullptr, nullptr, nullptr, 0, 2, 2000000000ull, 0, T, ks, logits};
-    return launch_grouped_gemm_fp8(g, tm_x, tm_w, tm_w, st);
+    CUtensorMap tm_out;  // the epilogue's tensor-map stores of the partial logits
+    g.tma_store = encode_logits_store(&tm_out, logits, (uint64_t)ks, (uint64_t)T, (uint64_t)E) ? 1 : 0;
+    return launch_grouped_gemm_fp8(g, tm_x, tm_w, g.tma_store ? tm_out : tm_w, st);
 }
 }  // namespace moe
 

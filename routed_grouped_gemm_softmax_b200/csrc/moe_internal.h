@@ -305,6 +305,8 @@ struct Fp8GemmArgs {
     int comb_k;
     int comb_target;
     unsigned long long *trace;  // per CTA {start, end} globaltimer (ns), or null
+    int tma_store;    // mode 2: tmB1 maps out_f32 as [ksplit][M][N] fp32 in 32 x 32 boxes (128-byte
+                      // swizzle); a CTA's last item then stores through it from its idle stages
 };
 cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                     const CUtensorMap &tmB1, cudaStream_t st);
