@@ -49,6 +49,24 @@ constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 
+// Tensor-map store of a box from shared memory (bulk-group completion): the box's
+// elements outside the tensor's extent are not written.  Generic-proxy writes to the
+// box must be made visible to the TMA first (fence_proxy_async_shared_cta).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *tm, const void *src, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until this thread's committed bulk groups have completed (their writes done).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_shared_cta()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 struct Ctrl8 {
     uint64_t full[STAGES], empty[STAGES];
     uint64_t accf[2], acce[2];
@@ -428,7 +446,7 @@ grouped_gemm_fp8_kernel(const __grid_constant__ AMaps tmA, const __grid_constant
                 // (the thread's own row would be 32 scattered 16-byte pieces per store).
                 const int col = n0 + half * 128;
                 const int total2 = (g.M + BM - 1) / BM * n_tiles * ksplit;
-                if (g.tma_store && g.reverse == 2 && item + (int)gridDim.x >= total2) {
+                if ((g.N & 3) == 0 && g.reverse == 2 && item + (int)gridDim.x >= total2) {
                     // The CTA's last item (items are dealt out statically): its last
                     // accumulator wait above means every MMA, and so every read of the
                     // stages, is done, and no further loads come.  The warp writes its 32

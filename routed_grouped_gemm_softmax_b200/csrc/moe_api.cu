@@ -371,9 +371,12 @@ cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, i
     *ksplit_out = ks;
     Fp8GemmArgs g{2, H, E, nullptr, nullptr, &hdr->counter[2], &hdr->status, nullptr, nullptr, nullptr, nullptr,
                   nullptr, nullptr, nullptr, 0, 2, 2000000000ull, 0, T, ks, logits};
-    CUtensorMap tm_out;  // the epilogue's tensor-map stores of the partial logits
-    g.tma_store = encode_logits_store(&tm_out, logits, (uint64_t)ks, (uint64_t)T, (uint64_t)E) ? 1 : 0;
-    return launch_grouped_gemm_fp8(g, tm_x, tm_w, g.tma_store ? tm_out : tm_w, st);
+    // with E a multiple of 4 the epilogue stores the partial logits through this map
+    // (passed as the kernel's third map, which mode 2 does not otherwise use)
+    CUtensorMap tm_out = tm_w;
+    if (E % 4 == 0 && !encode_logits_store(&tm_out, logits, (uint64_t)ks, (uint64_t)T, (uint64_t)E))
+        return cudaErrorInvalidValue;
+    return launch_grouped_gemm_fp8(g, tm_x, tm_w, tm_out, st);
 }
 }  // namespace moe
 

@@ -305,8 +305,6 @@ struct Fp8GemmArgs {
     int comb_k;
     int comb_target;
     unsigned long long *trace;  // per CTA {start, end} globaltimer (ns), or null
-    int tma_store;    // mode 2: tmB1 maps out_f32 as [ksplit][M][N] fp32 in 32 x 32 boxes (128-byte
-                      // swizzle); a CTA's last item then stores through it from its idle stages
 };
 cudaError_t launch_grouped_gemm_fp8(const Fp8GemmArgs &g, const AMaps &tmA, const CUtensorMap &tmB0,
                                     const CUtensorMap &tmB1, cudaStream_t st);
@@ -352,9 +350,6 @@ cudaError_t launch_gather_rows_mx(const uint8_t *xq, const uint8_t *xq_x, const 
 // Tensor-core router logits: partial sums over ksplit slices of H,
 // logits [ksplit, T, E] with sum_s logits[s] = x [T,H] . wrt [E,H]^T (fp32 per
 // 64-wide K block, then fp32 sums).  Returns ksplit through *ksplit_out.
-// The certify kernel's staging policy set by moe_set_cert_staging: {max stages, min
-// stages, max boxes per chunk}, each 0 for the default (3, 2, 8).
-void cert_staging(int *max_stages, int *min_stages, int *max_boxes);
 cudaError_t tc_router_logits(const __nv_bfloat16 *x, const __nv_bfloat16 *wrt, int T, int H, int E, float *logits,
                              WsHeader *hdr, int *ksplit_out, cudaStream_t st);
 

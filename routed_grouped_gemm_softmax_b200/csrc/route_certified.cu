@@ -36,6 +36,11 @@
 #include "sm100_ptx.cuh"
 
 namespace moe {
+
+// The staging policy set by moe_set_cert_staging (moe_api.cu): {max stages, min stages,
+// max boxes per chunk}, each 0 for the default (3, 2, 8).
+void cert_staging(int *max_stages, int *min_stages, int *max_boxes);
+
 namespace {
 
 constexpr int kPrepE = 16;     // experts per CTA of router_prep_kernel

@@ -163,24 +163,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, ui
         : "memory");
 }
 
-// Tensor-map store of a box from shared memory (bulk-group completion): the box's
-// elements outside the tensor's extent are not written.  Generic-proxy writes to the
-// box must be made visible to the TMA first (fence_proxy_async_shared_cta).
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap *tm, const void *src, int x, int y, int z)
-{
-    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(tm)),
-                 "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Waits until this thread's committed bulk groups have completed (their writes done).
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_shared_cta()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *slot_smem, uint32_t ncols)
