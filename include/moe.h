@@ -20,7 +20,8 @@
  * Conventions shared by every call
  *  - Pointers are DEVICE pointers unless stated otherwise; the caller owns all
  *    memory, including the workspace.  The library never allocates or frees
- *    device memory and never synchronises, except moe_get_device_status().
+ *    device memory and never synchronises, except moe_get_device_status() and
+ *    moe_noalloc_get_device_status().
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    All work is enqueued asynchronously on it; calls on one workspace must not
  *    overlap on the GPU.
@@ -357,11 +358,18 @@ void moe_set_stage_events(void *const *events, int32_t n);
  *    array and leaves its contents behind; the parts that must start at zero
  *    are cleared by each call.  Calls whose GPU work overlaps (other streams,
  *    unordered host threads) race on the array: serialise them.
- *  - Device-side status (timeouts) is kept in the array and not reported. */
+ *  - Device-side status (a pipeline timeout) is kept in the array's status word;
+ *    moe_noalloc_get_device_status reads it. */
 #define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
 moe_status_t moe_forward_noalloc(const moe_dims_t *d, const void *x, const void *router_w,
                                  const float *router_bias, const void *w_gate, const void *w_up,
                                  const void *w_down, void *out, void *stream);
+
+/* The device status of moe_forward_noalloc on the current device: synchronises
+ * `stream`, then reads and clears the status word of the fixed scratch, as
+ * moe_get_device_status does for a workspace.  Returns MOE_OK, a device error
+ * (MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX) of the last call, or MOE_ERR_CUDA. */
+moe_status_t moe_noalloc_get_device_status(void *stream);
 
 #ifdef __cplusplus
 }

@@ -26,7 +26,7 @@ EXPORTS = ["moe_workspace_size", "moe_max_tiles", "moe_route", "moe_permute", "m
            "moe_forward_fp8", "moe_quantize_rows_fp8", "moe_workspace_offsets", "moe_set_router_audit",
            "moe_forward_shared", "moe_workspace_size_shared", "moe_forward_mx", "moe_quantize_rows_mx",
            "moe_set_fused_combine", "moe_set_layer_gemm", "moe_forward_plan", "moe_set_direct_a",
-           "moe_set_cert_staging"]
+           "moe_set_cert_staging", "moe_noalloc_get_device_status"]
 DTYPE_BF16, DTYPE_FP8, DTYPE_MX = 0, 1, 2
 NOALLOC_SCRATCH_BYTES = 16 << 20
 STAGES = ["route", "permute", "gemm_gate_up", "gemm_down", "combine"]
@@ -110,6 +110,8 @@ def lib():
         L.moe_set_router_audit.restype = None
         L.moe_forward_noalloc.argtypes = [D, P, P, P, P, P, P, P, P]
         L.moe_forward_noalloc.restype = ctypes.c_int
+        L.moe_noalloc_get_device_status.argtypes = [P]
+        L.moe_noalloc_get_device_status.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -421,6 +423,12 @@ def set_direct_a(mode: str):
     """"auto" (default), "always" or "never": bf16 gate/up A rows gathered straight from x
     by the GEMM (never: from a sorted copy of x made by a gather kernel first)."""
     lib().moe_set_direct_a({"auto": 0, "always": 1, "never": 2}[mode])
+
+
+def noalloc_device_status(stream=None) -> int:
+    """moe_noalloc_get_device_status: synchronises the stream, then reads and clears the
+    device status word of moe_forward_noalloc's scratch on the current device."""
+    return lib().moe_noalloc_get_device_status(_stream(stream, torch.device("cuda", torch.cuda.current_device())))
 
 
 def set_cert_staging(max_stages: int = 0, min_stages: int = 0, max_boxes: int = 0):

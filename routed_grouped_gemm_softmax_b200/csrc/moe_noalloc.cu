@@ -65,3 +65,12 @@ extern "C" moe_status_t moe_forward_noalloc(const moe_dims_t *d, const void *x, 
     return moe_forward(d, x, router_w, router_bias, w_gate, w_up, w_down, out, ws, MOE_NOALLOC_SCRATCH_BYTES,
                        stream);
 }
+
+// The status word sits at the start of the scratch, as at the start of any workspace.
+extern "C" moe_status_t moe_noalloc_get_device_status(void *stream)
+{
+    void *ws = nullptr;
+    const moe_status_t s = scratch_on_current_device(&ws);
+    if (s != MOE_OK) return s;
+    return moe_get_device_status(ws, stream);
+}

@@ -75,3 +75,24 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     assert rc == 7  # MOE_ERR_TOO_LARGE, before any device work
     bad = api.dims(16, 2048, 512, 256, 0)
     assert api.lib().moe_forward_noalloc(ctypes.byref(bad), p, p, None, p, p, p, p, None) == 1
+
+
+def test_noalloc_status_reports_a_pipeline_timeout():
+    # The stall hook: every GEMM CTA's MMA thread first waits, with a 2 ms bound, on a
+    # barrier that nothing signals.  The timeout lands in the status word of the
+    # library's scratch, which moe_noalloc_get_device_status reads (and clears); the next
+    # call with the default settings is correct and reports MOE_OK.
+    cfg = CONFIGS["tiny"]
+    g, c = device_inputs(cfg)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    try:
+        api.set_wait_limit_us(2000, stall_test=True)
+        assert _call_noalloc(g, cfg.top_k, out) == api.MOE_OK
+        assert api.noalloc_device_status() == 5  # MOE_ERR_TIMEOUT
+    finally:
+        api.set_wait_limit_us(0, stall_test=False)
+    assert api.noalloc_device_status() == api.MOE_OK  # cleared by the read
+    ref = api.moe_forward(g["x"], g["router_w"], g["bias"], g["w_gate"], g["w_up"], g["w_down"], cfg.top_k)
+    assert _call_noalloc(g, cfg.top_k, out) == api.MOE_OK
+    assert api.noalloc_device_status() == api.MOE_OK
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
